@@ -1,0 +1,78 @@
+"""The seeded input generator (CPU): determinism, ranges, row-wise regeneration and the decode layout."""
+import numpy as np
+import torch
+
+import dsa_inputs as G
+
+
+def test_hash_is_deterministic_and_stream_separated():
+    c = torch.arange(1000, dtype=torch.int64)
+    a = G.hash64(c, G.stream_key(1, "q"))
+    b = G.hash64(c, G.stream_key(1, "q"))
+    d = G.hash64(c, G.stream_key(1, "c"))
+    e = G.hash64(c, G.stream_key(2, "q"))
+    assert torch.equal(a, b)
+    assert (a != d).float().mean() > 0.99 and (a != e).float().mean() > 0.99
+
+
+def test_integer_mode_ranges_and_balance():
+    cfg = G.PREFILL_CONFIGS["tiny_1k"]
+    x = G.prefill_inputs(cfg, 5)
+    qi = x["q_idx"].float()
+    assert qi.min() == -7 and qi.max() == 7 and torch.equal(qi, qi.round())
+    assert set(x["w"].unique().tolist()) == set(range(-3, 4))
+    counts = torch.bincount((qi.flatten() + 7).long(), minlength=15).float()
+    assert (counts / counts.mean() - 1).abs().max() < 0.05
+    assert x["q_scale"] is None and x["k_scale"] is None
+
+
+def test_normal_inputs_statistics():
+    cfg = G.PREFILL_CONFIGS["tiny_1k"]
+    x = G.prefill_inputs(cfg, 5)
+    for name in ("q", "c"):
+        v = x[name].float()
+        assert abs(v.mean().item()) < 0.01 and abs(v.std().item() - 1) < 0.01
+
+
+def test_rows_regenerate_identically():
+    cfg = G.PREFILL_CONFIGS["prefill_32k"]
+    rows = [0, 17, 4096, 32767]
+    sub = G.prefill_queries(cfg, 9, rows=rows)
+    full_block = G.prefill_queries(cfg, 9, rows=range(4090, 4100))
+    assert torch.equal(sub["q_idx"][2].view(torch.uint8), full_block["q_idx"][6].view(torch.uint8))
+    assert torch.equal(sub["q"][2], full_block["q"][6])
+    assert torch.equal(sub["w"][2], full_block["w"][6])
+    assert torch.equal(sub["q_scale"][2], full_block["q_scale"][6])
+
+
+def test_gaussian_quantisation_recipe():
+    cfg = G.PREFILL_CONFIGS["prefill_32k"]
+    q = G.prefill_queries(cfg, 2, rows=range(8))
+    v = q["q_idx"].float().view(8, -1)
+    assert v.abs().max() <= 448
+    # the per-token scale maps each token's largest magnitude onto the e4m3 maximum
+    assert (v.abs().amax(1) == 448).all()
+    assert (q["q_scale"] > 0).all()
+    assert abs(q["w"].std().item() - cfg.H_I ** -0.5) < 0.03
+
+
+def test_decode_layout_and_append_rows():
+    cfg = G.DecodeConfig("small", B=4, len_lo=100, len_hi=300, steps=5)
+    lens, offs, tot = G.decode_layout(cfg, 3)
+    assert all(100 <= n <= 300 for n in lens)
+    assert offs[0] == 0 and all(offs[i + 1] - offs[i] == lens[i] + 5 for i in range(3))
+    assert tot == offs[-1] + lens[-1] + 5
+    cache = G.decode_fill_cache(cfg, 3)
+    st = G.decode_step_inputs(cfg, 3, 2)
+    for b in range(4):
+        r = G.decode_cache_rows(cfg, 3, b, [lens[b] + 2])
+        assert torch.equal(r["k_idx"].view(torch.uint8)[0], st["k_new"].view(torch.uint8)[b])
+        assert torch.equal(r["c"][0], st["c_new"][b])
+        pre = G.decode_cache_rows(cfg, 3, b, range(lens[b]))
+        assert torch.equal(pre["c"], cache["c_cache"][offs[b]:offs[b] + lens[b]])
+    assert st["q"].shape == (4, cfg.H, cfg.D) and st["q_idx"].shape == (4, cfg.H_I, cfg.d_I)
+
+
+def test_decode_lengths_span():
+    lens = np.array(G.decode_lengths(G.DECODE_CONFIG, 20251202))
+    assert lens.min() >= 4096 and lens.max() <= 131072 and len(lens) == 64

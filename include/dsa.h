@@ -1,0 +1,149 @@
+/*
+ * dsa.h -- C ABI of the B200 (sm_100a) DeepSeek Sparse Attention (DSA) forward library, libdsa.so.
+ *
+ * The method ("DeepSeek-V3.2: Pushing the Frontier of Open Large Language Models", velog.io summary,
+ * DeepSeek Sparse Attention section):
+ *   1. lightning indexer (section 1.1):  I[t,s] = sum_{j<H_I} w[t,j] * ReLU(q_I[t,j] . k_I[s]),  s <= t;
+ *   2. fine-grained token selection (section 1.2): S_t = the k positions s with the largest I[t,s]
+ *      (ties broken by the smaller s; every s <= t when t + 1 <= k);
+ *   3. MLA in MQA mode (section 1.3): u_t[h] = softmax_{s in S_t}(scale * q[t,h] . c_s) . c_s[:D_v], with
+ *      one shared latent entry c_s per token for all query heads.
+ *
+ * Conventions common to every entry point:
+ *   - Pointers are DEVICE pointers owned by the caller, row-major and contiguous.  FP8 tensors are e4m3fn
+ *     bit patterns (uint8_t), bf16 tensors are bf16 bit patterns (uint16_t).  Tensors read by TMA (q_idx,
+ *     k_idx, q, c and the caches) must start on a 16-byte boundary.
+ *   - `stream` is a cudaStream_t passed as void*; every call is asynchronous on it and never synchronises
+ *     the device, except dsa_get_device_status().
+ *   - Arguments are checked on the host before anything is launched; a failed check returns an error code
+ *     and launches nothing.  Errors found while kernels run (an index out of range, a pipeline wait that ran
+ *     out of time) are recorded in a device status word read by dsa_get_device_status().
+ *   - Nothing is allocated inside a call: scratch memory is a caller-provided workspace whose size the
+ *     matching *_workspace_size() function returns.
+ *   - Supported shapes: H_I in {4, 64} with d_I = 64 / 128 respectively, H <= 128 query heads, D = 576 latent
+ *     dims of which the first D_v = 512 are the value, k a multiple of 64 (k in {128, 2048} for the
+ *     prefill and decode drivers).  Other shapes return DSA_ERR_UNSUPPORTED_SHAPE.
+ *   - Results are bitwise deterministic for fixed inputs and launch configuration.
+ */
+#ifndef DSA_H_
+#define DSA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define DSA_API __attribute__((visibility("default")))
+#else
+#define DSA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  DSA_OK = 0,
+  DSA_ERR_INVALID_ARG = 1,        /* null pointer, negative size, ... */
+  DSA_ERR_UNSUPPORTED_SHAPE = 2,  /* shape outside the compiled set */
+  DSA_ERR_ALIGNMENT = 3,          /* a TMA-read tensor is not 16-byte aligned */
+  DSA_ERR_CUDA = 4,               /* a CUDA runtime / driver call failed */
+  DSA_ERR_TIMEOUT = 5,            /* device: a pipeline wait ran out of its clock budget */
+  DSA_ERR_BAD_INDEX = 6,          /* device: a selected index was outside [-1, S) (treated as -1) */
+  DSA_ERR_WORKSPACE = 7           /* workspace missing or smaller than *_workspace_size() */
+} dsa_status_t;
+
+/* Human-readable name of a status code (static storage). */
+DSA_API const char* dsa_status_string(dsa_status_t status);
+
+/* Synchronises `stream`, then reads and clears the device status word of the current device.
+ * *device_status receives DSA_OK or the first device-side error since the last call. */
+DSA_API dsa_status_t dsa_get_device_status(void* stream, int* device_status);
+
+/* Number of SMs the launches of the current device are sized for (148 on a B200). */
+DSA_API int dsa_num_sms(void);
+
+/*
+ * Lightning-indexer scores, materialised for T query rows (velog.io section 1.1).
+ *   q_idx   [T, H_I, d_I] e4m3   indexer queries of rows 0..T-1, whose absolute positions are pos0..pos0+T-1
+ *   q_scale [T] fp32 or NULL     per-token dequantisation scale of q_idx (NULL: 1)
+ *   k_idx   [S, d_I] e4m3        indexer keys of positions 0..S-1
+ *   k_scale [S] fp32 or NULL     per-token dequantisation scale of k_idx (NULL: 1)
+ *   w       [T, H_I] fp32        indexer head weights
+ *   scores  [T, S] fp32 (out)    I[pos0 + r, s] for s <= pos0 + r, -INFINITY for s > pos0 + r
+ * Scores are accumulated in fp32 from exact e4m3 x e4m3 products, so integer-valued inputs with |I| < 2^24
+ * give exact scores.  Needs no workspace.
+ */
+DSA_API dsa_status_t dsa_indexer_scores(const uint8_t* q_idx, const float* q_scale, const uint8_t* k_idx,
+                                const float* k_scale, const float* w, int T, int S, int H_I, int d_I,
+                                int pos0, float* scores, void* stream);
+
+/*
+ * Row-wise top-k selection (velog.io section 1.2) over materialised scores.
+ *   scores  [rows, ld] fp32      row r holds n_r valid scores in columns 0..n_r-1
+ *   row_len [rows] int32 or NULL n_r (device array); NULL means n_r = min(ld, pos0 + r + 1) (causal rows)
+ *   idx     [rows, k] int32 (out) the min(k, n_r) columns with the largest scores, ties to the smaller
+ *                                column, in ascending column order, padded with -1
+ * -0.0 and +0.0 compare equal; NaN ranks below every number.  Needs no workspace.
+ */
+DSA_API dsa_status_t dsa_topk(const float* scores, int rows, int64_t ld, const int32_t* row_len, int pos0, int k,
+                      int32_t* idx, void* stream);
+
+/*
+ * Sparse MLA attention in MQA mode over selected latent entries (velog.io sections 1.2 and 1.3).
+ *   q     [T, H, 576] bf16    queries (H <= 128)
+ *   c     [S, 576] bf16       shared latent entries; the value of an entry is its first 512 dims
+ *   idx   [T, k] int32        selected entries of each row, in [0, S) or -1 (= nothing), any order
+ *   out   [T, H, 512] bf16 (out)  softmax(scale * q . c_s) . c_s[:512] over the selected s
+ *   lse   [T, H] fp32 or NULL (out)  natural-log log-sum-exp of the scaled logits (-INF for an empty row)
+ * A row with no selected entry gets out = 0.  Indices outside [-1, S) are treated as -1 and recorded as
+ * DSA_ERR_BAD_INDEX.  Needs no workspace.
+ */
+DSA_API dsa_status_t dsa_sparse_mla_attn(const uint16_t* q, const uint16_t* c, int S, const int32_t* idx, int T,
+                                 int H, int k, float scale, uint16_t* out, float* lse, void* stream);
+
+/* Workspace bytes of dsa_forward_prefill for these shapes. */
+DSA_API size_t dsa_prefill_workspace_size(int L, int H_I, int d_I, int H, int k);
+
+/*
+ * Whole DSA forward for one causal prefill sequence of L tokens (steps 1-3 above, s <= t).
+ *   q_idx [L, H_I, d_I] e4m3, q_scale [L] or NULL, k_idx [L, d_I] e4m3, k_scale [L] or NULL, w [L, H_I] fp32,
+ *   q [L, H, 576] bf16, c [L, 576] bf16;
+ *   idx_out [L, k] int32 (out, may be NULL): the selected positions of each row (ascending, -1 padded);
+ *   out [L, H, 512] bf16 (out); lse [L, H] fp32 (out, may be NULL).
+ * The L x L score matrix is never stored.
+ */
+DSA_API dsa_status_t dsa_forward_prefill(const uint8_t* q_idx, const float* q_scale, const uint8_t* k_idx,
+                                 const float* k_scale, const float* w, const uint16_t* q, const uint16_t* c,
+                                 int L, int H_I, int d_I, int H, int k, float scale, int32_t* idx_out,
+                                 uint16_t* out, float* lse, void* ws, size_t ws_bytes, void* stream);
+
+/* Workspace bytes of dsa_forward_decode for a batch of B sequences over caches of cache_rows rows. */
+DSA_API size_t dsa_decode_workspace_size(int B, int64_t cache_rows, int H_I, int d_I, int H, int k);
+
+/*
+ * One DSA decode step for a batch of B sequences, each with one new token.
+ * Sequence b owns cache rows [cache_off[b], cache_off[b] + capacity); before the call it holds ctx_len[b]
+ * entries.  The call appends the new token's entries at position ctx_len[b] and then runs steps 1-3 for the
+ * new token (position ctx_len[b]) over positions 0..ctx_len[b].  ctx_len is not modified: the caller
+ * advances it.
+ *   cache_off [B] int64, ctx_len [B] int32                            (device arrays)
+ *   q_idx [B, H_I, d_I] e4m3, q_scale [B] or NULL, w [B, H_I] fp32, q [B, H, 576] bf16   new-token queries
+ *   k_new [B, d_I] e4m3, k_scale_new [B] fp32, c_new [B, 576] bf16                          new-token entries
+ *   k_cache [cache_rows, d_I] e4m3, k_scale_cache [cache_rows] fp32, c_cache [cache_rows, 576] bf16 (in/out)
+ *   idx_out [B, k] int32 (out, may be NULL): selected positions within each sequence (ascending, -1 padded)
+ *   out [B, H, 512] bf16 (out), lse [B, H] fp32 (out, may be NULL)
+ * k_scale_new / k_scale_cache are always stored; pass 1.0 for unscaled (integer-valued) keys, and
+ * q_scale = NULL.
+ */
+DSA_API dsa_status_t dsa_forward_decode(int B, const int64_t* cache_off, const int32_t* ctx_len, const uint8_t* q_idx,
+                                const float* q_scale, const float* w, const uint16_t* q, const uint8_t* k_new,
+                                const float* k_scale_new, const uint16_t* c_new, uint8_t* k_cache,
+                                float* k_scale_cache, uint16_t* c_cache, int64_t cache_rows, int H_I, int d_I,
+                                int H, int k, float scale, int32_t* idx_out, uint16_t* out, float* lse, void* ws,
+                                size_t ws_bytes, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* DSA_H_ */

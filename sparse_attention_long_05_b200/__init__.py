@@ -1,0 +1,17 @@
+"""B200 (sm_100a) DeepSeek Sparse Attention forward: lightning indexer -> top-k selection -> sparse MLA.
+
+The computation lives in libdsa.so (hand-written CUDA, C ABI in include/dsa.h); this package only builds it
+(`build.py`) and binds it (`_lib.py`).  Importing the package loads the library and fails if it is missing.
+"""
+from ._lib import (  # noqa: F401
+    DsaError,
+    dsa_decode_workspace_size,
+    dsa_forward_decode,
+    dsa_forward_prefill,
+    dsa_get_device_status,
+    dsa_indexer_scores,
+    dsa_num_sms,
+    dsa_prefill_workspace_size,
+    dsa_sparse_mla_attn,
+    dsa_topk,
+)

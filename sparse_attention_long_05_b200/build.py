@@ -1,0 +1,59 @@
+"""Build step of the CUDA library: compiles csrc/dsa_api.cu (one translation unit) into libdsa.so, in-tree.
+
+Run as ``python -m sparse_attention_long_05_b200.build`` or through ``__graft_entry__.build()``.  nvcc
+cross-compiles for sm_100a, so this works on a machine without a GPU.
+"""
+from __future__ import annotations
+
+import os
+import shutil
+import subprocess
+import sys
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+ROOT = os.path.dirname(HERE)
+SRC = os.path.join(HERE, "csrc", "dsa_api.cu")
+OUT = os.path.join(HERE, "libdsa.so")
+DEPS = [os.path.join(HERE, "csrc", f) for f in os.listdir(os.path.join(HERE, "csrc"))] + \
+       [os.path.join(ROOT, "include", "dsa.h")]
+
+
+def nvcc() -> str:
+    for cand in (os.environ.get("NVCC"), "/usr/local/cuda/bin/nvcc", shutil.which("nvcc")):
+        if cand and os.path.exists(cand):
+            return cand
+    raise RuntimeError("nvcc not found: the CUDA toolkit is needed to build libdsa.so")
+
+
+def command(out: str = OUT, extra=()):
+    return [nvcc(), "-gencode", "arch=compute_100a,code=sm_100a", "-O3", "-lineinfo", "-std=c++17",
+            "-shared", "-Xcompiler", "-fPIC", "-Xcompiler", "-fvisibility=hidden",
+            "-Xcompiler", "-Wno-unused-function", "-I", os.path.join(ROOT, "include"),
+            *extra, "-o", out, SRC]
+
+
+def up_to_date() -> bool:
+    if not os.path.exists(OUT):
+        return False
+    t = os.path.getmtime(OUT)
+    return all(os.path.getmtime(d) <= t for d in DEPS if os.path.exists(d))
+
+
+def build(force: bool = False, verbose: bool = False, extra=()) -> str:
+    if not force and not extra and up_to_date():
+        return OUT
+    cmd = command(extra=extra)
+    if verbose:
+        print(" ".join(cmd), flush=True)
+    res = subprocess.run(cmd, capture_output=True, text=True)
+    if res.returncode != 0:
+        sys.stderr.write(res.stdout + res.stderr)
+        raise RuntimeError("nvcc failed building libdsa.so")
+    if verbose and (res.stdout or res.stderr):
+        print(res.stdout + res.stderr)
+    return OUT
+
+
+if __name__ == "__main__":
+    build(force="--force" in sys.argv, verbose=True,
+          extra=("-Xptxas", "-v") if "--ptxas-v" in sys.argv else ())

@@ -1,0 +1,334 @@
+// libdsa.so: C ABI of the DSA forward path on B200 (declarations and contracts in include/dsa.h).
+//
+// Host side only: argument checks, TMA tensor-map construction, launch configuration and the order of the
+// kernels of the prefill and decode drivers.  Every step of the computation runs in the kernels included
+// below.
+#include <cmath>
+#include <cstdio>
+#include <mutex>
+
+#include "common.cuh"
+#include "indexer.cuh"
+#include "sparse_mla.cuh"
+#include "topk.cuh"
+
+namespace dsa {
+
+// ------------------------------------------------------------------------------------------ decode append
+// Writes the new token's indexer key (+ scale) and latent entry at position ctx_len[b] of sequence b, and
+// n_b + 1 into len1[b] (the number of keys the new token attends to).
+__global__ void decode_append_kernel(int B, const long long* cache_off, const int* ctx_len, long long cache_rows,
+                                     const uint8_t* k_new, const float* k_scale_new, const uint16_t* c_new,
+                                     uint8_t* k_cache, float* k_scale_cache, uint16_t* c_cache, int d_I,
+                                     int* len1) {
+  const int b = blockIdx.x;
+  if (b >= B) return;
+  const long long row = cache_off[b] + ctx_len[b];
+  if (ctx_len[b] < 0 || row < 0 || row >= cache_rows) {
+    if (threadIdx.x == 0) { raise_status(DSA_ERR_BAD_INDEX); len1[b] = 0; }
+    return;
+  }
+  const uint4* ks = reinterpret_cast<const uint4*>(k_new + static_cast<long long>(b) * d_I);
+  uint4* kd = reinterpret_cast<uint4*>(k_cache + row * d_I);
+  for (int i = threadIdx.x; i < d_I / 16; i += blockDim.x) kd[i] = ks[i];
+  const uint4* cs = reinterpret_cast<const uint4*>(c_new + static_cast<long long>(b) * mla::D);
+  uint4* cd = reinterpret_cast<uint4*>(c_cache + row * mla::D);
+  for (int i = threadIdx.x; i < mla::D * 2 / 16; i += blockDim.x) cd[i] = cs[i];
+  if (threadIdx.x == 0) {
+    k_scale_cache[row] = k_scale_new[b];
+    len1[b] = ctx_len[b] + 1;
+  }
+}
+
+// ------------------------------------------------------------------------------------------ host helpers
+namespace {
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// rank-2/3 tensor map; dims / strides innermost first (strides in bytes, rank-1 entries)
+bool make_map(CUtensorMap* m, CUtensorMapDataType dt, int rank, const void* base, const cuuint64_t* dims,
+              const cuuint64_t* strides, const cuuint32_t* box, CUtensorMapSwizzle sw) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint32_t es[3] = {1, 1, 1};
+  return fn(m, dt, rank, const_cast<void*>(base), dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int num_sms() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) return 148;
+  return n;
+}
+
+template <typename K>
+cudaError_t set_smem(K kernel, int bytes) {
+  return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+}
+
+dsa_status_t last_launch_status() {
+  return cudaGetLastError() == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
+}
+
+size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+// ------------------------------------------------------------------------------------------ launchers
+// One CTA per SM: the indexer allocates all 512 TMEM columns, so at least 120 KB of shared memory is
+// requested to keep a second CTA off the SM.
+constexpr int kMinIndexerSmem = 120 * 1024;
+
+template <int H_I, int D_I, int NT, int NG, int QBUF, int KST, int EPI, int MODE>
+dsa_status_t launch_indexer(const uint8_t* q_idx, int q_rows, const uint8_t* k_idx, long long k_rows,
+                            const IndexerParams& p, int grid, cudaStream_t st) {
+  using C = IndexerCfg<H_I, D_I, NT, NG, QBUF, KST, EPI, MODE>;
+  CUtensorMap tq, tk;
+  const cuuint64_t qd[2] = {static_cast<cuuint64_t>(D_I), static_cast<cuuint64_t>(q_rows) * H_I};
+  const cuuint64_t qs[1] = {static_cast<cuuint64_t>(D_I)};
+  const cuuint32_t qb[2] = {static_cast<cuuint32_t>(D_I), static_cast<cuuint32_t>(C::N)};
+  const cuuint64_t kd[2] = {static_cast<cuuint64_t>(D_I), static_cast<cuuint64_t>(k_rows)};
+  const cuuint32_t kb[2] = {static_cast<cuuint32_t>(D_I), 128u};
+  const CUtensorMapSwizzle sw = (D_I == 128) ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
+  if (!make_map(&tq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, q_idx, qd, qs, qb, sw)) return DSA_ERR_CUDA;
+  if (!make_map(&tk, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, k_idx, kd, qs, kb, sw)) return DSA_ERR_CUDA;
+  auto kern = indexer_kernel<H_I, D_I, NT, NG, QBUF, KST, EPI, MODE>;
+  const int smem = C::SMEM > kMinIndexerSmem ? C::SMEM : kMinIndexerSmem;
+  if (set_smem(kern, smem) != cudaSuccess) return DSA_ERR_CUDA;
+  kern<<<grid, C::NUM_THREADS, smem, st>>>(tq, tk, p);
+  return last_launch_status();
+}
+
+// scores [T, S] of query rows at positions pos0.. against keys 0..S-1 (materialised)
+dsa_status_t run_indexer_scores(const uint8_t* q_idx, const float* q_scale, const uint8_t* k_idx,
+                                const float* k_scale, const float* w, int T, int S, int H_I, int d_I, int pos0,
+                                float* scores, long long ld, cudaStream_t st) {
+  IndexerParams p{};
+  p.w = w;
+  p.q_scale = q_scale;
+  p.k_scale = k_scale;
+  p.scores = scores;
+  p.ld = ld;
+  p.T = T;
+  p.S = S;
+  p.pos0 = pos0;
+  const int tok = (H_I == 64) ? 16 : 256;
+  const int nqb = (T + tok - 1) / tok;
+  const int ntiles = (S + 127) / 128;
+  int nsplit = (2 * num_sms() + nqb - 1) / nqb;
+  nsplit = nsplit < 1 ? 1 : (nsplit > ntiles ? ntiles : nsplit);
+  p.split_tiles = (ntiles + nsplit - 1) / nsplit;
+  p.nsplit = (ntiles + p.split_tiles - 1) / p.split_tiles;
+  p.n_items = nqb * p.nsplit;
+  if (H_I == 64)
+    return launch_indexer<64, 128, 4, 4, 1, 4, 2, kModeScores>(q_idx, T, k_idx, S, p, p.n_items, st);
+  return launch_indexer<4, 64, 64, 4, 1, 4, 2, kModeScores>(q_idx, T, k_idx, S, p, p.n_items, st);
+}
+
+dsa_status_t run_topk(const float* scores, long long ld, const long long* row_off, const int* row_len, int pos0,
+                      int rows, int k, int* idx, long long idx_ld, cudaStream_t st) {
+  if (rows <= 0) return DSA_OK;
+  TopkParams p{scores, ld, row_off, row_len, pos0, rows, k, idx, idx_ld};
+  topk_rows_kernel<<<rows, kTopkThreads, 0, st>>>(p);
+  return last_launch_status();
+}
+
+dsa_status_t run_mla(const uint16_t* q, const uint16_t* c, long long S, const int* idx, const long long* row_off,
+                     int T, int H, int k, float scale, uint16_t* out, float* lse, cudaStream_t st) {
+  if (T <= 0) return DSA_OK;
+  CUtensorMap tq, tc;
+  const cuuint64_t qd[3] = {576, static_cast<cuuint64_t>(H), static_cast<cuuint64_t>(T)};
+  const cuuint64_t qs[2] = {576 * 2, static_cast<cuuint64_t>(H) * 576 * 2};
+  const cuuint32_t qb[3] = {64, 128, 1};
+  const cuuint64_t cd[2] = {576, static_cast<cuuint64_t>(S)};
+  const cuuint64_t cs[1] = {576 * 2};
+  const cuuint32_t cb[2] = {64, 1};
+  if (!make_map(&tq, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, q, qd, qs, qb, CU_TENSOR_MAP_SWIZZLE_128B)) return DSA_ERR_CUDA;
+  if (!make_map(&tc, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, c, cd, cs, cb, CU_TENSOR_MAP_SWIZZLE_128B)) return DSA_ERR_CUDA;
+  MlaParams p{};
+  p.idx = idx;
+  p.row_off = row_off;
+  p.out = out;
+  p.lse = lse;
+  p.T = T;
+  p.H = H;
+  p.k = k;
+  p.S = S;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  if (set_smem(sparse_mla_kernel, mla::SMEM) != cudaSuccess) return DSA_ERR_CUDA;
+  int clusters = num_sms() / 2;
+  if (clusters > T) clusters = T;
+  sparse_mla_kernel<<<2 * clusters, mla::THREADS, mla::SMEM, st>>>(tq, tc, p);
+  return last_launch_status();
+}
+
+bool indexer_shape_ok(int H_I, int d_I) { return (H_I == 64 && d_I == 128) || (H_I == 4 && d_I == 64); }
+
+size_t prefill_chunk_rows(int L) {
+  // rows of scores materialised per chunk: about 1 GiB of fp32 scores, at least 256 rows
+  size_t r = (size_t(1) << 30) / (4 * size_t(L > 0 ? L : 1));
+  if (r < 256) r = 256;
+  if (r > size_t(L)) r = size_t(L);
+  return r;
+}
+
+}  // namespace
+}  // namespace dsa
+
+using namespace dsa;
+
+extern "C" {
+
+const char* dsa_status_string(dsa_status_t s) {
+  switch (s) {
+    case DSA_OK: return "DSA_OK";
+    case DSA_ERR_INVALID_ARG: return "DSA_ERR_INVALID_ARG";
+    case DSA_ERR_UNSUPPORTED_SHAPE: return "DSA_ERR_UNSUPPORTED_SHAPE";
+    case DSA_ERR_ALIGNMENT: return "DSA_ERR_ALIGNMENT";
+    case DSA_ERR_CUDA: return "DSA_ERR_CUDA";
+    case DSA_ERR_TIMEOUT: return "DSA_ERR_TIMEOUT";
+    case DSA_ERR_BAD_INDEX: return "DSA_ERR_BAD_INDEX";
+    case DSA_ERR_WORKSPACE: return "DSA_ERR_WORKSPACE";
+  }
+  return "DSA_UNKNOWN_STATUS";
+}
+
+dsa_status_t dsa_get_device_status(void* stream, int* device_status) {
+  if (!device_status) return DSA_ERR_INVALID_ARG;
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return DSA_ERR_CUDA;
+  int v = 0;
+  if (cudaMemcpyFromSymbol(&v, g_dev_status, sizeof(int)) != cudaSuccess) return DSA_ERR_CUDA;
+  const int zero = 0;
+  if (cudaMemcpyToSymbol(g_dev_status, &zero, sizeof(int)) != cudaSuccess) return DSA_ERR_CUDA;
+  *device_status = v;
+  return DSA_OK;
+}
+
+int dsa_num_sms(void) { return num_sms(); }
+
+dsa_status_t dsa_indexer_scores(const uint8_t* q_idx, const float* q_scale, const uint8_t* k_idx,
+                                const float* k_scale, const float* w, int T, int S, int H_I, int d_I, int pos0,
+                                float* scores, void* stream) {
+  if (T < 0 || S < 0 || pos0 < 0 || (T > 0 && (!q_idx || !w || !scores)) || (S > 0 && !k_idx))
+    return DSA_ERR_INVALID_ARG;
+  if (!indexer_shape_ok(H_I, d_I)) return DSA_ERR_UNSUPPORTED_SHAPE;
+  if (!aligned16(q_idx) || !aligned16(k_idx)) return DSA_ERR_ALIGNMENT;
+  if (T == 0 || S == 0) return DSA_OK;
+  return run_indexer_scores(q_idx, q_scale, k_idx, k_scale, w, T, S, H_I, d_I, pos0, scores, S,
+                            static_cast<cudaStream_t>(stream));
+}
+
+dsa_status_t dsa_topk(const float* scores, int rows, int64_t ld, const int32_t* row_len, int pos0, int k,
+                      int32_t* idx, void* stream) {
+  if (rows < 0 || ld < 0 || k <= 0 || pos0 < 0 || (rows > 0 && (!scores || !idx))) return DSA_ERR_INVALID_ARG;
+  return run_topk(scores, ld, nullptr, row_len, pos0, rows, k, idx, k, static_cast<cudaStream_t>(stream));
+}
+
+dsa_status_t dsa_sparse_mla_attn(const uint16_t* q, const uint16_t* c, int S, const int32_t* idx, int T, int H,
+                                 int k, float scale, uint16_t* out, float* lse, void* stream) {
+  if (T < 0 || S <= 0 || H <= 0 || k <= 0 || (T > 0 && (!q || !c || !idx || !out))) return DSA_ERR_INVALID_ARG;
+  if (H > 128 || k % mla::NK != 0) return DSA_ERR_UNSUPPORTED_SHAPE;
+  if (!aligned16(q) || !aligned16(c) || (reinterpret_cast<uintptr_t>(idx) & 7u) || !aligned16(out))
+    return DSA_ERR_ALIGNMENT;
+  return run_mla(q, c, S, idx, nullptr, T, H, k, scale, out, lse, static_cast<cudaStream_t>(stream));
+}
+
+size_t dsa_prefill_workspace_size(int L, int H_I, int d_I, int H, int k) {
+  (void)H_I; (void)d_I; (void)H;
+  if (L <= 0 || k <= 0) return 0;
+  const size_t rows = prefill_chunk_rows(L);
+  return align_up(rows * size_t(L) * 4, 256) + align_up(size_t(L) * size_t(k) * 4, 256);
+}
+
+dsa_status_t dsa_forward_prefill(const uint8_t* q_idx, const float* q_scale, const uint8_t* k_idx,
+                                 const float* k_scale, const float* w, const uint16_t* q, const uint16_t* c,
+                                 int L, int H_I, int d_I, int H, int k, float scale, int32_t* idx_out,
+                                 uint16_t* out, float* lse, void* ws, size_t ws_bytes, void* stream) {
+  if (L <= 0 || H <= 0 || k <= 0 || !q_idx || !k_idx || !w || !q || !c || !out) return DSA_ERR_INVALID_ARG;
+  if (!indexer_shape_ok(H_I, d_I) || H > 128 || k % mla::NK != 0) return DSA_ERR_UNSUPPORTED_SHAPE;
+  if (!aligned16(q_idx) || !aligned16(k_idx) || !aligned16(q) || !aligned16(c) || !aligned16(out))
+    return DSA_ERR_ALIGNMENT;
+  if (!ws || ws_bytes < dsa_prefill_workspace_size(L, H_I, d_I, H, k)) return DSA_ERR_WORKSPACE;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const size_t R = prefill_chunk_rows(L);
+  float* sc = static_cast<float*>(ws);
+  int32_t* idx = idx_out ? idx_out
+                         : reinterpret_cast<int32_t*>(static_cast<char*>(ws) + align_up(R * size_t(L) * 4, 256));
+  for (int r0 = 0; r0 < L; r0 += static_cast<int>(R)) {
+    const int rows = (L - r0 < static_cast<int>(R)) ? L - r0 : static_cast<int>(R);
+    const int s_eff = r0 + rows;   // keys beyond the chunk's last row are never selected (causal)
+    dsa_status_t e = run_indexer_scores(q_idx + static_cast<size_t>(r0) * H_I * d_I, q_scale ? q_scale + r0 : nullptr,
+                                        k_idx, k_scale, w + static_cast<size_t>(r0) * H_I, rows, s_eff, H_I, d_I,
+                                        r0, sc, s_eff, st);
+    if (e != DSA_OK) return e;
+    e = run_topk(sc, s_eff, nullptr, nullptr, r0, rows, k, idx + static_cast<size_t>(r0) * k, k, st);
+    if (e != DSA_OK) return e;
+  }
+  return run_mla(q, c, L, idx, nullptr, L, H, k, scale, out, lse, st);
+}
+
+size_t dsa_decode_workspace_size(int B, int64_t cache_rows, int H_I, int d_I, int H, int k) {
+  (void)H_I; (void)d_I; (void)H;
+  if (B <= 0 || cache_rows <= 0 || k <= 0) return 0;
+  return align_up(size_t(cache_rows) * 4, 256) + align_up(size_t(B) * 4, 256) + align_up(size_t(B) * k * 4, 256);
+}
+
+dsa_status_t dsa_forward_decode(int B, const int64_t* cache_off, const int32_t* ctx_len, const uint8_t* q_idx,
+                                const float* q_scale, const float* w, const uint16_t* q, const uint8_t* k_new,
+                                const float* k_scale_new, const uint16_t* c_new, uint8_t* k_cache,
+                                float* k_scale_cache, uint16_t* c_cache, int64_t cache_rows, int H_I, int d_I,
+                                int H, int k, float scale, int32_t* idx_out, uint16_t* out, float* lse, void* ws,
+                                size_t ws_bytes, void* stream) {
+  if (B <= 0 || cache_rows <= 0 || H <= 0 || k <= 0 || !cache_off || !ctx_len || !q_idx || !w || !q || !k_new ||
+      !k_scale_new || !c_new || !k_cache || !k_scale_cache || !c_cache || !out)
+    return DSA_ERR_INVALID_ARG;
+  if (H_I != 64 || d_I != 128 || H > 128 || k % mla::NK != 0 || B > kMaxDecodeSeqs) return DSA_ERR_UNSUPPORTED_SHAPE;
+  if (!aligned16(q_idx) || !aligned16(q) || !aligned16(k_new) || !aligned16(c_new) || !aligned16(k_cache) ||
+      !aligned16(c_cache) || !aligned16(out))
+    return DSA_ERR_ALIGNMENT;
+  if (!ws || ws_bytes < dsa_decode_workspace_size(B, cache_rows, H_I, d_I, H, k)) return DSA_ERR_WORKSPACE;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  char* wsb = static_cast<char*>(ws);
+  float* dscores = reinterpret_cast<float*>(wsb);
+  int* len1 = reinterpret_cast<int*>(wsb + align_up(size_t(cache_rows) * 4, 256));
+  int32_t* idx = idx_out ? idx_out
+                         : reinterpret_cast<int32_t*>(wsb + align_up(size_t(cache_rows) * 4, 256) +
+                                                      align_up(size_t(B) * 4, 256));
+  const long long* off = reinterpret_cast<const long long*>(cache_off);
+  decode_append_kernel<<<B, 128, 0, st>>>(B, off, ctx_len, cache_rows, k_new, k_scale_new, c_new, k_cache,
+                                          k_scale_cache, c_cache, d_I, len1);
+  dsa_status_t e = last_launch_status();
+  if (e != DSA_OK) return e;
+  IndexerParams p{};
+  p.w = w;
+  p.q_scale = q_scale;
+  p.k_scale = k_scale_cache;
+  p.scores = dscores;
+  p.T = B;
+  p.cache_off = off;
+  p.ctx_len = ctx_len;
+  p.chunk_tiles = 16;
+  e = launch_indexer<64, 128, 1, 1, 2, 8, 1, kModeDecode>(q_idx, B, k_cache, cache_rows, p, num_sms(), st);
+  if (e != DSA_OK) return e;
+  e = run_topk(dscores, 0, off, len1, 0, B, k, idx, k, st);
+  if (e != DSA_OK) return e;
+  return run_mla(q, c_cache, cache_rows, idx, off, B, H, k, scale, out, lse, st);
+}
+
+}  // extern "C"

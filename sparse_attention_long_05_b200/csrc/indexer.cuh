@@ -1,0 +1,381 @@
+// Lightning-indexer kernel: I[t,s] = sum_j w[t,j] * ReLU(q_I[t,j] . k_I[s])   (velog.io DSA page, §1.1)
+//
+// Data layout on the tensor core.  One tcgen05 MMA computes, for a tile of 128 keys and a group of NT query
+// tokens, D[s, (t, j)] = k_I[s] . q_I[t, j] with FP8 e4m3 operands and fp32 accumulation:
+//   A = 128 keys x d_I   (K-major, TMA-loaded tile of k_I),
+//   B = NT*H_I rows of q_I x d_I (K-major; rows (t, j) are consecutive in q_I's [T, H_I, d_I] layout),
+//   D = 128 TMEM lanes (one per key) x NT*H_I fp32 columns.
+// Because a key owns a TMEM lane, the ReLU and the head-weighted sum over j are thread-local in the
+// epilogue: thread s loads its lane's columns, computes sum_j w[t,j] * max(x, 0) for each of its tokens,
+// multiplies by the key scale (Gaussian mode; the query scale is folded into w), and writes I[t, s].
+//
+// Warp roles (one CTA per SM):
+//   warp 0      TMA producer: q_I block of the work item, then one k_I tile per pipeline stage
+//   warp 1      TMEM allocation + MMA issue (one elected thread)
+//   warps 2..   epilogue warpgroup(s); warp w reads TMEM lanes 32*(w % 4) .. +31
+// Two TMEM accumulators of up to 256 columns let the epilogue of one (tile, group) overlap the MMA of the
+// next.  Tiles lying wholly above the causal diagonal of every token of the item are never loaded.
+//
+// Work items:
+//   kModeScores  item = (block of NG*NT query rows, range of key tiles); writes scores [T, S] (tests,
+//                materialised prefill chunks);
+//   kModeDecode  item = (sequence b, range of its key tiles); one token per sequence; keys are the rows
+//                [cache_off[b], cache_off[b] + ctx_len[b]] of the flat key cache; writes one fp32 score per
+//                cache row (a vector per sequence).
+#pragma once
+#include "common.cuh"
+
+namespace dsa {
+
+enum { kModeScores = 0, kModeDecode = 1 };
+
+struct IndexerParams {
+  const float* w;          // [T, H_I]
+  const float* q_scale;    // [T] or null
+  const float* k_scale;    // per key row, or null
+  float* scores;           // output (see modes)
+  long long ld;            // kModeScores: row stride of scores
+  int T;                   // query rows (kModeScores) / sequences B (kModeDecode)
+  int S;                   // kModeScores: number of keys
+  int pos0;                // kModeScores: absolute position of query row 0
+  int n_items;             // kModeScores: number of work items
+  int nsplit;              // kModeScores: key-range splits per query block
+  int split_tiles;         // kModeScores: key tiles per split
+  const long long* cache_off;  // kModeDecode: [B]
+  const int* ctx_len;          // kModeDecode: [B] entries before the append (the new token sits at ctx_len)
+  int chunk_tiles;             // kModeDecode: key tiles per work item
+};
+
+struct IndexerItem {
+  int q_row0;         // first query row of the item
+  int n_tok;          // valid query rows in the item
+  int pos0;           // absolute position of the item's first query row
+  int tile0, tile1;   // key tile range [tile0, tile1)
+  int n_keys;         // keys s < n_keys exist
+  long long key_row0; // tensor-map row of key 0
+  long long out_base; // output offset of (first row, key 0)
+};
+
+constexpr int kMaxDecodeSeqs = 1024;
+
+template <int H_I, int D_I, int NT, int NG, int QBUF, int KSTAGES, int EPI_WG, int MODE>
+struct IndexerCfg {
+  static constexpr int N = NT * H_I;                 // MMA N
+  static constexpr int TOK = NT * NG;                // query rows per item
+  static constexpr int GBYTES = N * D_I;             // one group of q_I rows
+  static constexpr int KBYTES = 128 * D_I;           // one key tile
+  static constexpr int NUM_EPI_WARPS = 4 * EPI_WG;
+  static constexpr int NUM_THREADS = 64 + 32 * NUM_EPI_WARPS;
+  static constexpr int ALIGN = 1024;
+  // shared memory map (offsets from a 1024-byte aligned base)
+  static constexpr int OFF_BAR = 0;                  // barriers + misc (2 KB)
+  static constexpr int OFF_PREFIX = 2048;            // decode: per-sequence item prefix (4 KB)
+  static constexpr int OFF_W = OFF_PREFIX + (MODE == kModeDecode ? 4 * (kMaxDecodeSeqs + 1) : 0);
+  static constexpr int W_FLOATS = TOK * H_I;
+  static constexpr int OFF_Q = ((OFF_W + QBUF * W_FLOATS * 4 + ALIGN - 1) / ALIGN) * ALIGN;
+  static constexpr int OFF_K = OFF_Q + QBUF * NG * GBYTES;
+  static constexpr int SMEM = OFF_K + KSTAGES * KBYTES + ALIGN;  // + alignment slack
+  static constexpr uint32_t TMEM_COLS = 512;
+  static constexpr uint32_t SW_LAYOUT = (D_I == 128) ? kLayoutSW128 : kLayoutSW64;
+  static constexpr uint32_t SBO = (D_I == 128) ? 1024 : 512;
+  static_assert(N <= 256 && N % 16 == 0, "MMA N");
+  static_assert(D_I == 128 || D_I == 64, "d_I");
+  static_assert((N / EPI_WG) % H_I == 0 || H_I > N / EPI_WG, "epilogue column split");
+};
+
+// barrier slots (8 bytes each) in the barrier area
+template <int QBUF, int KSTAGES>
+struct IndexerBars {
+  static constexpr int Q_FULL = 0;
+  static constexpr int Q_EMPTY = Q_FULL + QBUF;
+  static constexpr int K_FULL = Q_EMPTY + QBUF;
+  static constexpr int K_EMPTY = K_FULL + KSTAGES;
+  static constexpr int ACC_FULL = K_EMPTY + KSTAGES;
+  static constexpr int ACC_EMPTY = ACC_FULL + 2;
+  static constexpr int COUNT = ACC_EMPTY + 2;
+  static constexpr int OFF_TMEM = 8 * COUNT;         // u32: TMEM base address
+  static constexpr int OFF_ABORT = OFF_TMEM + 4;     // int: abort flag
+  static constexpr int OFF_NITEMS = OFF_TMEM + 8;    // int: number of items (decode)
+};
+
+template <int MODE, int TOK>
+__device__ __forceinline__ IndexerItem indexer_item(const IndexerParams& p, int i, const int* prefix) {
+  IndexerItem it;
+  if constexpr (MODE == kModeScores) {
+    const int qb = i / p.nsplit, sp = i % p.nsplit;
+    it.q_row0 = qb * TOK;
+    it.n_tok = min(TOK, p.T - it.q_row0);
+    it.pos0 = p.pos0 + it.q_row0;
+    it.n_keys = p.S;
+    it.key_row0 = 0;
+    const int ntiles = (p.S + 127) / 128;
+    it.tile0 = sp * p.split_tiles;
+    it.tile1 = min(it.tile0 + p.split_tiles, ntiles);
+    it.out_base = static_cast<long long>(it.q_row0) * p.ld;
+  } else {
+    // binary search: prefix[b] <= i < prefix[b + 1]
+    int lo = 0, hi = p.T - 1;
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (prefix[mid] <= i) lo = mid; else hi = mid - 1;
+    }
+    const int b = lo;
+    const int n = p.ctx_len[b] + 1;
+    it.q_row0 = b;
+    it.n_tok = 1;
+    it.pos0 = n - 1;
+    it.n_keys = n;
+    it.key_row0 = p.cache_off[b];
+    it.tile0 = (i - prefix[b]) * p.chunk_tiles;
+    it.tile1 = min(it.tile0 + p.chunk_tiles, (n + 127) / 128);
+    it.out_base = p.cache_off[b];
+  }
+  return it;
+}
+
+// last query position covered by group g of the item (or -1 when the group has no valid row)
+template <int NT>
+__device__ __forceinline__ int group_last_pos(const IndexerItem& it, int g) {
+  if (g * NT >= it.n_tok) return -1;
+  return it.pos0 + min(it.n_tok, (g + 1) * NT) - 1;
+}
+template <int NT>
+__device__ __forceinline__ bool group_active(const IndexerItem& it, int tile, int g) {
+  return tile * 128 < it.n_keys && tile * 128 <= group_last_pos<NT>(it, g);
+}
+__device__ __forceinline__ bool tile_active(const IndexerItem& it, int tile) {
+  return tile * 128 < it.n_keys && tile * 128 <= it.pos0 + it.n_tok - 1;
+}
+
+template <int H_I, int D_I, int NT, int NG, int QBUF, int KSTAGES, int EPI_WG, int MODE>
+__global__ void __launch_bounds__(IndexerCfg<H_I, D_I, NT, NG, QBUF, KSTAGES, EPI_WG, MODE>::NUM_THREADS, 1)
+indexer_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+               const IndexerParams p) {
+  using C = IndexerCfg<H_I, D_I, NT, NG, QBUF, KSTAGES, EPI_WG, MODE>;
+  using Bars = IndexerBars<QBUF, KSTAGES>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + C::ALIGN - 1) &
+                                             ~static_cast<uintptr_t>(C::ALIGN - 1));
+  const uint32_t sbase = smem_u32(smem);
+  auto bar = [&](int slot) -> uint32_t { return sbase + C::OFF_BAR + 8 * slot; };
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Bars::OFF_ABORT);
+  int* prefix = reinterpret_cast<int*>(smem + C::OFF_PREFIX);
+  float* w_s = reinterpret_cast<float*>(smem + C::OFF_W);
+  const uint32_t q_s = sbase + C::OFF_Q;
+  const uint32_t k_s = sbase + C::OFF_K;
+  const int warp = warp_id(), lane = lane_id();
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < QBUF; ++i) { mbar_init(bar(Bars::Q_FULL + i), 1); mbar_init(bar(Bars::Q_EMPTY + i), 1); }
+    for (int i = 0; i < KSTAGES; ++i) { mbar_init(bar(Bars::K_FULL + i), 1); mbar_init(bar(Bars::K_EMPTY + i), 1); }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(bar(Bars::ACC_FULL + i), 1);
+      mbar_init(bar(Bars::ACC_EMPTY + i), C::NUM_EPI_WARPS);
+    }
+    *abort_flag = 0;
+    if constexpr (MODE == kModeDecode) {
+      int tot = 0;
+      for (int b = 0; b < p.T; ++b) {
+        prefix[b] = tot;
+        const int tiles = (p.ctx_len[b] + 1 + 127) / 128;
+        tot += (tiles + p.chunk_tiles - 1) / p.chunk_tiles;
+      }
+      prefix[p.T] = tot;
+      *reinterpret_cast<int*>(smem + Bars::OFF_NITEMS) = tot;
+    }
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) { prefetch_tmap(&tm_q); prefetch_tmap(&tm_k); }
+  if (warp == 1) {
+    tmem_alloc(sbase + Bars::OFF_TMEM, C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *reinterpret_cast<volatile uint32_t*>(smem + Bars::OFF_TMEM);
+  const int n_items = (MODE == kModeDecode) ? *reinterpret_cast<volatile int*>(smem + Bars::OFF_NITEMS)
+                                            : p.n_items;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      Pipe<KSTAGES> kp;
+      int k_issued = 0;                 // k tiles issued so far
+      int q_issued[QBUF] = {};          // per q buffer: loads issued
+      uint32_t q_par[QBUF] = {};        // per q buffer: parity of its last load
+      int qi = 0;
+      bool ok = true;
+      for (int item = blockIdx.x; item < n_items && ok; item += gridDim.x, ++qi) {
+        const IndexerItem it = indexer_item<MODE, C::TOK>(p, item, prefix);
+        const int qb = qi % QBUF;
+        const uint32_t qph = (qi / QBUF) & 1;
+        if (!mbar_wait(bar(Bars::Q_EMPTY + qb), qph ^ 1, abort_flag)) { ok = false; break; }
+        mbar_arrive_expect_tx(bar(Bars::Q_FULL + qb), NG * C::GBYTES);
+        for (int g = 0; g < NG; ++g)
+          tma_load_2d(q_s + (qb * NG + g) * C::GBYTES, &tm_q, bar(Bars::Q_FULL + qb), 0,
+                      (it.q_row0 + g * NT) * H_I);
+        q_issued[qb] += 1;
+        q_par[qb] = qph;
+        for (int tile = it.tile0; tile < it.tile1; ++tile) {
+          if (!tile_active(it, tile)) continue;
+          if (!mbar_wait(bar(Bars::K_EMPTY + kp.stage), kp.phase ^ 1, abort_flag)) { ok = false; break; }
+          mbar_arrive_expect_tx(bar(Bars::K_FULL + kp.stage), C::KBYTES);
+          tma_load_2d(k_s + kp.stage * C::KBYTES, &tm_k, bar(Bars::K_FULL + kp.stage), 0,
+                      static_cast<int>(it.key_row0 + tile * 128));
+          kp.advance();
+          ++k_issued;
+        }
+      }
+      if (*abort_flag) {
+        // leave no TMA write in flight into this CTA's shared memory: wait (bounded) for the last load
+        // issued on every k stage and q buffer
+        for (int st = 0; st < KSTAGES && st < k_issued; ++st)
+          mbar_wait_drain(bar(Bars::K_FULL + st), st < kp.stage ? kp.phase : kp.phase ^ 1);
+        for (int b = 0; b < QBUF; ++b)
+          if (q_issued[b]) mbar_wait_drain(bar(Bars::Q_FULL + b), q_par[b]);
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------------ MMA issue
+    if (lane == 0) {
+      Pipe<KSTAGES> kp;
+      Pipe<2> ap;
+      constexpr uint32_t idesc = idesc_e4m3(128, C::N);
+      int qi = 0;
+      bool ok = true;
+      for (int item = blockIdx.x; item < n_items && ok; item += gridDim.x, ++qi) {
+        const IndexerItem it = indexer_item<MODE, C::TOK>(p, item, prefix);
+        const int qb = qi % QBUF;
+        if (!mbar_wait(bar(Bars::Q_FULL + qb), (qi / QBUF) & 1, abort_flag)) { ok = false; break; }
+        tc_fence_after();
+        for (int tile = it.tile0; tile < it.tile1 && ok; ++tile) {
+          if (!tile_active(it, tile)) continue;
+          if (!mbar_wait(bar(Bars::K_FULL + kp.stage), kp.phase, abort_flag)) { ok = false; break; }
+          tc_fence_after();
+          const uint64_t adesc = smem_desc(k_s + kp.stage * C::KBYTES, 16, C::SBO, C::SW_LAYOUT);
+          for (int g = 0; g < NG; ++g) {
+            if (!group_active<NT>(it, tile, g)) continue;
+            if (!mbar_wait(bar(Bars::ACC_EMPTY + ap.stage), ap.phase ^ 1, abort_flag)) { ok = false; break; }
+            tc_fence_after();
+            const uint64_t bdesc = smem_desc(q_s + (qb * NG + g) * C::GBYTES, 16, C::SBO, C::SW_LAYOUT);
+            const uint32_t d = tmem_base + ap.stage * 256;
+#pragma unroll
+            for (int kk = 0; kk < D_I / 32; ++kk)   // K = 32 e4m3 (32 bytes) per instruction
+              mma_f8_ss(d, adesc + 2 * kk, bdesc + 2 * kk, idesc, kk > 0 ? 1u : 0u);
+            mma_commit(bar(Bars::ACC_FULL + ap.stage));
+            ap.advance();
+          }
+          mma_commit(bar(Bars::K_EMPTY + kp.stage));
+          kp.advance();
+        }
+        mma_commit(bar(Bars::Q_EMPTY + qb));
+      }
+    }
+  } else {
+    // ------------------------------------------------------------------ epilogue
+    constexpr int CPT = C::N / EPI_WG;              // accumulator columns per thread
+    constexpr int TOKS = (CPT >= H_I) ? CPT / H_I : 1;  // query rows per thread
+    constexpr int P = (H_I >= 16) ? 4 : 1;         // partial sums per row (ILP)
+    const int e = warp - 2;
+    const int quad = warp & 3;
+    const int half = e >> 2;
+    const int ethreads = 32 * C::NUM_EPI_WARPS;
+    const int etid = e * 32 + lane;
+    const uint32_t lane_addr = static_cast<uint32_t>(quad * 32) << 16;
+    Pipe<2> ap;
+    int qi = 0;
+    bool ok = true;
+    for (int item = blockIdx.x; item < n_items && ok; item += gridDim.x, ++qi) {
+      const IndexerItem it = indexer_item<MODE, C::TOK>(p, item, prefix);
+      float* wq = w_s + (qi % QBUF) * C::W_FLOATS;
+      named_bar_sync(1, ethreads);
+      for (int i = etid; i < C::W_FLOATS; i += ethreads) {
+        const int r = i / H_I;
+        float v = 0.f;
+        if (r < it.n_tok) {
+          v = p.w[static_cast<long long>(it.q_row0 + r) * H_I + (i % H_I)];
+          if (p.q_scale) v *= p.q_scale[it.q_row0 + r];
+        }
+        wq[i] = v;
+      }
+      named_bar_sync(1, ethreads);
+      for (int tile = it.tile0; tile < it.tile1; ++tile) {
+        const int s = tile * 128 + quad * 32 + lane;      // key of this thread
+        const bool key_ok = s < it.n_keys;
+        float kscale = 1.f;
+        if (p.k_scale && key_ok) kscale = p.k_scale[it.key_row0 + s];
+        for (int g = 0; g < NG; ++g) {
+          if (g * NT >= it.n_tok) break;
+          const int tok0 = g * NT + half * (CPT / H_I > 0 ? CPT / H_I : 0);  // first row of this thread
+          if (!group_active<NT>(it, tile, g)) {
+            if constexpr (MODE == kModeScores) {
+              if (key_ok) {
+#pragma unroll
+                for (int tk = 0; tk < TOKS; ++tk) {
+                  const int r = tok0 + tk;
+                  if (r < it.n_tok) p.scores[it.out_base + static_cast<long long>(r) * p.ld + s] = -INFINITY;
+                }
+              }
+            }
+            continue;
+          }
+          if (!mbar_wait(bar(Bars::ACC_FULL + ap.stage), ap.phase, abort_flag)) { ok = false; break; }
+          tc_fence_after();
+          float acc[TOKS][P];
+#pragma unroll
+          for (int tk = 0; tk < TOKS; ++tk)
+#pragma unroll
+            for (int q = 0; q < P; ++q) acc[tk][q] = 0.f;
+          const uint32_t tcol = tmem_base + ap.stage * 256 + half * CPT;
+#pragma unroll
+          for (int c0 = 0; c0 < CPT; c0 += 64) {
+            uint32_t v0[32], v1[32];
+            tmem_ld32(lane_addr + tcol + c0, v0);
+            if (c0 + 32 < CPT) tmem_ld32(lane_addr + tcol + c0 + 32, v1);
+            tmem_wait_ld();
+#pragma unroll
+            for (int i = 0; i < 64; ++i) {
+              if (c0 + i >= CPT) break;
+              const int col = c0 + i;
+              const int tk = col / H_I, j = col % H_I;
+              const float x = __uint_as_float(i < 32 ? v0[i] : v1[i - 32]);
+              acc[tk][j % P] = fmaf(wq[(tok0 + tk) * H_I + j], fmaxf(x, 0.f), acc[tk][j % P]);
+            }
+          }
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(bar(Bars::ACC_EMPTY + ap.stage));
+          ap.advance();
+          if (key_ok) {
+#pragma unroll
+            for (int tk = 0; tk < TOKS; ++tk) {
+              const int r = tok0 + tk;
+              if (r >= it.n_tok) continue;
+              float sc = 0.f;
+#pragma unroll
+              for (int q = 0; q < P; ++q) sc += acc[tk][q];
+              sc *= kscale;
+              if constexpr (MODE == kModeScores) {
+                p.scores[it.out_base + static_cast<long long>(r) * p.ld + s] = (s <= it.pos0 + r) ? sc : -INFINITY;
+              } else {
+                p.scores[it.out_base + s] = sc;
+              }
+            }
+          }
+        }
+        if (!ok) break;
+      }
+    }
+  }
+
+  // ------------------------------------------------------------------ teardown
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, C::TMEM_COLS);
+  }
+}
+
+}  // namespace dsa

@@ -1,0 +1,70 @@
+"""The C-ABI library (no GPU needed): it builds, loads, exports every declared symbol, and its host-side
+argument checks reject bad calls before launching anything."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared():
+    src = open(os.path.join(ROOT, "include", "dsa.h")).read()
+    return re.findall(r"DSA_API\s+[\w\s\*]*?\b(dsa_\w+)\s*\(", src)
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from sparse_attention_long_05_b200 import build
+    build.build()
+    from sparse_attention_long_05_b200 import _lib
+    return _lib._lib
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = _declared()
+    assert len(names) >= 10
+    from sparse_attention_long_05_b200._lib import SIGNATURES
+    for n in names:
+        assert hasattr(lib, n), n
+        assert n in SIGNATURES, n
+
+
+def test_status_strings(lib):
+    for code, name in [(0, b"DSA_OK"), (2, b"DSA_ERR_UNSUPPORTED_SHAPE"), (5, b"DSA_ERR_TIMEOUT"),
+                       (7, b"DSA_ERR_WORKSPACE"), (99, b"DSA_UNKNOWN_STATUS")]:
+        assert lib.dsa_status_string(code) == name
+
+
+def test_workspace_sizes(lib):
+    assert lib.dsa_prefill_workspace_size(0, 64, 128, 128, 2048) == 0
+    w8 = lib.dsa_prefill_workspace_size(8192, 64, 128, 128, 2048)
+    assert w8 >= 8192 * 2048 * 4 and w8 % 256 == 0
+    w128 = lib.dsa_prefill_workspace_size(131072, 64, 128, 128, 2048)
+    assert w128 <= (1 << 30) + 131072 * 2048 * 4 + 512      # never the L x L score matrix
+    assert lib.dsa_decode_workspace_size(64, 1 << 20, 64, 128, 128, 2048) >= (1 << 20) * 4 + 64 * 2048 * 4
+
+
+def test_host_argument_checks(lib):
+    P = ctypes.c_void_p
+    one = P(16)  # a dummy aligned non-null address: every call below must fail before touching it
+    # unsupported indexer shape
+    assert lib.dsa_indexer_scores(one, None, one, None, one, 4, 4, 32, 128, 0, one, None) == 2
+    # negative sizes / null outputs
+    assert lib.dsa_indexer_scores(one, None, one, None, one, -1, 4, 64, 128, 0, one, None) == 1
+    assert lib.dsa_topk(None, 3, 10, None, 0, 4, one, None) == 1
+    assert lib.dsa_topk(one, 3, 10, None, 0, 0, one, None) == 1
+    # misaligned TMA operand
+    assert lib.dsa_indexer_scores(P(17), None, one, None, one, 4, 4, 64, 128, 0, one, None) == 3
+    # attention: too many heads, k not a multiple of 64
+    assert lib.dsa_sparse_mla_attn(one, one, 10, one, 2, 129, 64, 1.0, one, None, None) == 2
+    assert lib.dsa_sparse_mla_attn(one, one, 10, one, 2, 8, 100, 1.0, one, None, None) == 2
+    # prefill without a big enough workspace
+    assert lib.dsa_forward_prefill(one, None, one, None, one, one, one, 1024, 4, 64, 8, 128, 1.0, None, one, None,
+                                   one, 16, None) == 7
+    # decode: only H_I = 64 / d_I = 128
+    assert lib.dsa_forward_decode(2, one, one, one, None, one, one, one, one, one, one, one, one, 100, 4, 64, 8, 128,
+                                  1.0, None, one, None, one, 1 << 20, None) == 2
+    # empty work is a no-op
+    assert lib.dsa_indexer_scores(one, None, one, None, one, 0, 4, 64, 128, 0, one, None) == 0

@@ -1,0 +1,66 @@
+"""dsa_forward_decode (append -> indexer over the key cache -> top-k -> sparse MLA) against the oracle."""
+import numpy as np
+import pytest
+import torch
+
+import dsa_inputs as G
+import oracle as O
+from gpu_util import MAX_ABS, RECALL, REL_L2, f64, recall, rel_l2
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def dsa():
+    import sparse_attention_long_05_b200 as m
+    return m
+
+
+def _run_steps(dsa, cfg, seed, steps, check_seqs, exact):
+    cache = G.decode_fill_cache(cfg, seed, device="cuda")
+    lens, offs = cache["lens"], cache["offs"]
+    cache_off = torch.tensor(offs, dtype=torch.int64, device="cuda")
+    ctx = torch.tensor(lens, dtype=torch.int32, device="cuda")
+    for step in range(steps):
+        st = G.decode_step_inputs(cfg, seed, step, device="cuda")
+        idx, out, lse = dsa.dsa_forward_decode(cache_off, ctx, st["q_idx"], st["q_scale"], st["w"], st["q"],
+                                               st["k_new"], st["k_scale_new"], st["c_new"], cache["k_cache"],
+                                               cache["k_scale_cache"], cache["c_cache"], cfg.k, cfg.scale)
+        assert dsa.dsa_get_device_status() == 0
+        idx, out = idx.cpu().numpy(), f64(out)
+        step_q = G.decode_step_inputs(cfg, seed, step)
+        recs, refs, gots = [], [], []
+        for b in check_seqs:
+            n = lens[b] + step + 1
+            rows = G.decode_cache_rows(cfg, seed, b, range(n))
+            # the appended entry landed in the cache
+            o = offs[b] + n - 1
+            assert torch.equal(cache["c_cache"][o].cpu(), rows["c"][n - 1])
+            ref = O.decode_row(rows, step_q, b, n, cfg.k, cfg.scale)
+            if exact:
+                assert np.array_equal(idx[b], ref["idx"]), f"seq {b} step {step}"
+            else:
+                recs.append(recall(idx[b], ref["idx"]))
+            refs.append(ref["out"])
+            gots.append(out[b])
+        if recs:
+            assert np.mean(recs) >= RECALL
+        refs, gots = np.stack(refs), np.stack(gots)
+        assert np.abs(gots - refs).max() <= MAX_ABS
+        assert rel_l2(gots, refs) <= REL_L2
+        ctx += 1
+
+
+def test_small_batch_integer_mode_exact(dsa):
+    cfg = G.DecodeConfig("small_int", B=5, len_lo=1000, len_hi=9000, steps=3, mode="int")
+    _run_steps(dsa, cfg, 41, 3, range(5), exact=True)
+
+
+def test_small_batch_gaussian(dsa):
+    cfg = G.DecodeConfig("small_gauss", B=6, len_lo=100, len_hi=6000, steps=2)
+    _run_steps(dsa, cfg, 42, 2, range(6), exact=False)
+
+
+def test_full_batch_sampled_sequences(dsa):
+    cfg = G.DECODE_CONFIG
+    _run_steps(dsa, cfg, 43, 2, [0, 7, 21, 63], exact=False)

@@ -1,0 +1,469 @@
+#!/usr/bin/env python
+"""Throughput of the DSA forward hot path on B200: lightning indexer -> top-k -> sparse MLA.
+
+Default run (N = 1): the 128K-token causal prefill (L = 131072, H_I = 64, d_I = 128 FP8, k = 2048, 128 query
+heads over a 576-dim bf16 latent) is the headline line; the 64-sequence decode batch (contexts 4K..128K, 256
+steps, caches appended every step) is measured in the same run and reported under "decode".
+
+One prefill step = the whole forward of one sequence through the C ABI with inputs resident in HBM:
+dsa_prefill_select (indexer scores of a bounded block of rows + their top-k, block after block) followed by
+dsa_sparse_mla_attn.  Every kernel is bracketed by CUDA events on the launching stream, which gives each
+kernel's share of the step and its roofline fraction.  Inputs (q alone is 19 GB) are far larger than the
+126 MB L2, so no explicit L2 flush is needed between steps.
+
+--impl reference runs the CPU oracle (fp64, test infrastructure) on the host cores on a bounded sample of
+query rows per step and reports the same metric.
+With torchrun (N > 1) every rank runs its own independent sequence (replicas, no collective on the data
+path); the step time is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import dsa_inputs as G  # noqa: E402
+
+METRIC = "DSA forward tokens/s at 1 B200 (128K prefill; 64x128K decode) + % roofline"
+PREFILL = G.PREFILL_CONFIGS["prefill_128k_gauss"]
+DECODE = G.DECODE_CONFIG
+NOMINAL_FP8_PER_BF16 = 2.0   # dense FP8 / BF16 tensor-core rate ratio (4.5 / 2.25 PFLOP/s)
+
+
+# ------------------------------------------------------------------------------------------ environment
+def dist_init():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if ws > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=600),
+                                device_id=torch.device("cuda", local))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(local)
+    return ws, rank, local
+
+
+def barrier(ws):
+    if ws > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x: float, ws: int) -> float:
+    if ws == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        p = json.load(open(path))
+        return {"hbm_gbs": p["hbm_gbs"], "bf16_burst": p["bf16_tflops"],
+                "bf16_sustained": p.get("bf16_tflops_sustained", p["bf16_tflops"]), "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_burst": 1590.0, "bf16_sustained": 1400.0, "source": "fallback"}
+
+
+class ClockSampler:
+    """nvidia-smi samples of this GPU's clocks and throttle reasons while the timed region runs."""
+    FIELDS = ["clocks.sm", "clocks.max.sm", "power.draw", "clocks_event_reasons.hw_slowdown",
+              "clocks_event_reasons.hw_thermal_slowdown", "clocks_event_reasons.sw_thermal_slowdown",
+              "clocks_event_reasons.sw_power_cap"]
+
+    def __init__(self, device_index: int):
+        self.rows = []
+        self.proc = None
+        try:
+            uuid = str(torch.cuda.get_device_properties(device_index).uuid)
+            ident = uuid if uuid.startswith("GPU-") else "GPU-" + uuid
+        except Exception:
+            ident = str(device_index)
+        self.cmd = ["nvidia-smi", "-i", ident, "--query-gpu=" + ",".join(self.FIELDS),
+                    "--format=csv,noheader,nounits", "-lms", "100"]
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(self.cmd, stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except Exception:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) == len(self.FIELDS):
+                self.rows.append(parts)
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self):
+        if not self.rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
+        def num(x):
+            try:
+                return float(x)
+            except ValueError:
+                return None
+        sm = [num(r[0]) for r in self.rows if num(r[0]) is not None]
+        reasons = set()
+        for r in self.rows:
+            for name, v in zip(["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"], r[3:]):
+                if v.lower().startswith("active"):
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": num(self.rows[0][1]),
+                "reasons": sorted(reasons), "samples": len(self.rows),
+                "power_w_max": max((num(r[2]) or 0.0) for r in self.rows)}
+
+
+# ------------------------------------------------------------------------------------------ work counts
+def prefill_work(cfg):
+    """Algorithmic work of one prefill step: indexer FP8 flops, attention bf16 flops, top-k bytes."""
+    L, k = cfg.L, cfg.k
+    pairs = L * (L + 1) // 2                                          # (t, s) with s <= t
+    sel = sum(min(t + 1, k) for t in range(min(L, k))) + max(0, L - k) * k
+    return {"indexer_flops": 2.0 * cfg.H_I * cfg.d_I * pairs,
+            "attention_flops": 2.0 * cfg.H * (cfg.D + cfg.D_v) * sel,
+            "topk_bytes": 4.0 * pairs + 4.0 * L * k}
+
+
+def decode_bytes(cfg, lens, steps):
+    """Algorithmic HBM bytes of `steps` decode steps: key cache (e4m3 + fp32 scale) of every sequence,
+    the selected latent rows, the new-token tensors, selected indices and outputs."""
+    tot = 0.0
+    for s in range(steps):
+        for n in lens:
+            m = n + s + 1
+            tot += m * (cfg.d_I + 4) + min(m, cfg.k) * cfg.D * 2
+        tot += cfg.B * (cfg.H * cfg.D * 2 + cfg.H_I * cfg.d_I + cfg.H_I * 4 + cfg.k * 4 + cfg.H * cfg.D_v * 2
+                        + cfg.d_I + 4 + cfg.D * 2)
+    return tot
+
+
+def prefill_chunk_rows(L):
+    """Rows per score block of dsa_prefill_select (mirrors the library's choice, for reporting)."""
+    return max(256, min(L, (1 << 30) // (4 * L)))
+
+
+# ------------------------------------------------------------------------------------------ GPU arms
+def bench_prefill(dsa, cfg, steps, warmup, ws_n, rank, pk):
+    dev = "cuda"
+    x = G.prefill_keys(cfg, 1000 + rank, device=dev)
+    x.update(G.prefill_queries(cfg, 1000 + rank, None, device=dev))
+    L, k = cfg.L, cfg.k
+    idx = torch.empty((L, k), dtype=torch.int32, device=dev)
+    out = torch.empty((L, cfg.H, cfg.D_v), dtype=torch.bfloat16, device=dev)
+    lse = torch.empty((L, cfg.H), dtype=torch.float32, device=dev)
+    ws = torch.empty((dsa.dsa_prefill_workspace_size(L, cfg.H_I, cfg.d_I, cfg.H, k),), dtype=torch.uint8,
+                     device=dev)
+    evs = []
+
+    def step(record):
+        e = [torch.cuda.Event(enable_timing=True) for _ in range(3)] if record else None
+        if record:
+            e[0].record()
+        dsa.dsa_prefill_select(x["q_idx"], x["q_scale"], x["k_idx"], x["k_scale"], x["w"], k, idx_out=idx, ws=ws)
+        if record:
+            e[1].record()
+        dsa.dsa_sparse_mla_attn(x["q"], x["c"], idx, cfg.scale, out=out, lse=lse)
+        if record:
+            e[2].record()
+            evs.append(e)
+
+    for _ in range(warmup):
+        step(False)
+    torch.cuda.synchronize()
+    assert dsa.dsa_get_device_status() == 0
+    barrier(ws_n)
+    torch.cuda.synchronize()
+    n0 = dsa.dsa_launch_count()
+    with ClockSampler(torch.cuda.current_device()) as clk:
+        t0 = torch.cuda.Event(enable_timing=True)
+        t1 = torch.cuda.Event(enable_timing=True)
+        t0.record()
+        for _ in range(steps):
+            step(True)
+        t1.record()
+        torch.cuda.synchronize()
+    launches = dsa.dsa_launch_count() - n0
+    barrier(ws_n)
+    ms = max_over_ranks(t0.elapsed_time(t1), ws_n) / steps
+    assert dsa.dsa_get_device_status() == 0
+    sel_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in evs)
+    att_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in evs)
+    work = prefill_work(cfg)
+    bf16_peak = pk["bf16_sustained"]
+    att_tflops = work["attention_flops"] / (att_ms * 1e-3) / 1e12
+    sel_tflops = work["indexer_flops"] / (sel_ms * 1e-3) / 1e12
+    kernels = {
+        "sparse_mla_attn": {"ms": att_ms, "share": att_ms / ms, "bound": "tensor", "achieved": att_tflops,
+                            "peak": bf16_peak, "unit": "TFLOP/s", "frac": att_tflops / bf16_peak},
+        "prefill_select": {"ms": sel_ms, "share": sel_ms / ms, "bound": "tensor", "achieved": sel_tflops,
+                           "peak": bf16_peak * NOMINAL_FP8_PER_BF16, "unit": "TFLOP/s",
+                           "frac": sel_tflops / (bf16_peak * NOMINAL_FP8_PER_BF16),
+                           "note": "indexer (FP8 flops) + top-k of materialised blocks of "
+                                   f"{prefill_chunk_rows(L)} rows"},
+    }
+    dom = max(kernels, key=lambda n: kernels[n]["ms"])
+    d = kernels[dom]
+    roof = {"kernel": dom, "bound": d["bound"], "achieved": d["achieved"], "peak": d["peak"], "unit": d["unit"],
+            "frac": d["frac"], "traffic": None,
+            "peak_source": f"{pk['source']} bf16 sustained" + (" x2 (FP8)" if dom == "prefill_select" else "")}
+    del x
+    return {"ms": ms, "tokens_per_s": ws_n * L / (ms * 1e-3), "roofline": roof, "kernels": kernels,
+            "clocks": clk.summary(), "launches": launches}
+
+
+def bench_prefill_e2e(dsa, cfg, steps, rank):
+    """Same metric through dsa_forward_prefill with host buffers: pinned H2D of every input and D2H of
+    every output inside the timed region."""
+    import psutil
+    dev = "cuda"
+    x = G.prefill_keys(cfg, 1000 + rank, device=dev)
+    x.update(G.prefill_queries(cfg, 1000 + rank, None, device=dev))
+    names = ["q_idx", "q_scale", "k_idx", "k_scale", "w", "q", "c"]
+    h2d = sum(x[n].numel() * x[n].element_size() for n in names if x[n] is not None)
+    L, k = cfg.L, cfg.k
+    outs = {"idx": ((L, k), torch.int32), "out": ((L, cfg.H, cfg.D_v), torch.bfloat16),
+            "lse": ((L, cfg.H), torch.float32)}
+    d2h = sum(int(np.prod(s)) * torch.empty((), dtype=dt).element_size() for s, dt in outs.values())
+    if psutil.virtual_memory().available < 1.5 * (h2d + d2h):
+        return {"value": None, "unit": "tokens/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "skipped": "not enough host memory for pinned copies of every input and output"}
+    host = {n: x[n].cpu().pin_memory() for n in names if x[n] is not None}
+    del x
+    dvc = {n: torch.empty_like(host[n], device=dev) for n in host}
+    hout = {n: torch.empty(s, dtype=dt, pin_memory=True) for n, (s, dt) in outs.items()}
+    dout = {n: torch.empty(s, dtype=dt, device=dev) for n, (s, dt) in outs.items()}
+    ws = torch.empty((dsa.dsa_prefill_workspace_size(L, cfg.H_I, cfg.d_I, cfg.H, k),), dtype=torch.uint8,
+                     device=dev)
+
+    def step():
+        for n in host:
+            dvc[n].copy_(host[n], non_blocking=True)
+        dsa.dsa_forward_prefill(dvc["q_idx"], dvc.get("q_scale"), dvc["k_idx"], dvc.get("k_scale"), dvc["w"],
+                                dvc["q"], dvc["c"], k, cfg.scale, idx_out=dout["idx"], out=dout["out"],
+                                lse=dout["lse"], ws=ws)
+        for n in hout:
+            hout[n].copy_(dout[n], non_blocking=True)
+
+    step()
+    torch.cuda.synchronize()
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record()
+    for _ in range(steps):
+        step()
+    t1.record()
+    torch.cuda.synchronize()
+    ms = t0.elapsed_time(t1) / steps
+    return {"value": L / (ms * 1e-3), "unit": "tokens/s", "ms_per_step": ms, "h2d_bytes_per_step": h2d,
+            "d2h_bytes_per_step": d2h, "steps": steps}
+
+
+def bench_decode(dsa, cfg, steps, warmup, ws_n, rank, pk):
+    dev = "cuda"
+    seed = 2000 + rank
+    cache = G.decode_fill_cache(cfg, seed, device=dev)
+    lens, offs = cache["lens"], cache["offs"]
+    cache_off = torch.tensor(offs, dtype=torch.int64, device=dev)
+    ctx = torch.tensor(lens, dtype=torch.int32, device=dev)
+    nsteps = warmup + steps
+    assert nsteps <= cfg.steps, "the caches hold cfg.steps appended entries per sequence"
+    blocks = [G.decode_step_batch(cfg, seed, min(32, nsteps - s0), device=dev, step0=s0)
+              for s0 in range(0, nsteps, 32)]
+    inp = {key: torch.cat([b[key] for b in blocks]) if blocks[0][key] is not None else None for key in blocks[0]}
+    B, k = cfg.B, cfg.k
+    idx = torch.empty((B, k), dtype=torch.int32, device=dev)
+    out = torch.empty((B, cfg.H, cfg.D_v), dtype=torch.bfloat16, device=dev)
+    lse = torch.empty((B, cfg.H), dtype=torch.float32, device=dev)
+    ws = torch.empty((dsa.dsa_decode_workspace_size(B, cache["rows"], cfg.H_I, cfg.d_I, cfg.H, k),),
+                     dtype=torch.uint8, device=dev)
+
+    def step(s):
+        g = lambda key: None if inp[key] is None else inp[key][s]   # noqa: E731
+        dsa.dsa_forward_decode(cache_off, ctx, g("q_idx"), g("q_scale"), g("w"), g("q"), g("k_new"),
+                               g("k_scale_new"), g("c_new"), cache["k_cache"], cache["k_scale_cache"],
+                               cache["c_cache"], k, cfg.scale, idx_out=idx, out=out, lse=lse, ws=ws)
+        ctx.add_(1)
+
+    for s in range(warmup):
+        step(s)
+    torch.cuda.synchronize()
+    assert dsa.dsa_get_device_status() == 0
+    barrier(ws_n)
+    torch.cuda.synchronize()
+    n0 = dsa.dsa_launch_count()
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record()
+    for s in range(warmup, nsteps):
+        step(s)
+    t1.record()
+    torch.cuda.synchronize()
+    launches = dsa.dsa_launch_count() - n0
+    barrier(ws_n)
+    ms = max_over_ranks(t0.elapsed_time(t1), ws_n) / steps
+    assert dsa.dsa_get_device_status() == 0
+    byts = decode_bytes(cfg, lens, nsteps) - decode_bytes(cfg, lens, warmup)
+    gbs = byts / steps / (ms * 1e-3) / 1e9
+    return {"metric": "DSA decode tokens/s (64 sequences, 4K-128K contexts, caches appended every step)",
+            "value": ws_n * B / (ms * 1e-3), "unit": "tokens/s", "ms_per_step": ms, "steps": steps,
+            "warmup": warmup,
+            "roofline": {"kernel": "decode step (append, indexer, top-k, sparse MLA)", "bound": "hbm",
+                         "achieved": gbs, "peak": pk["hbm_gbs"], "unit": "GB/s", "frac": gbs / pk["hbm_gbs"],
+                         "traffic": None, "peak_source": pk["source"] + " copy bandwidth"},
+            "launches": launches}
+
+
+# ------------------------------------------------------------------------------------------ oracle arm
+_KEYS_CACHE = {}
+
+
+def oracle_prefill_rate(cfg, budget_s, seed, max_rows=256, batch=16):
+    """Oracle tokens/s on the host: seeded uniformly random query rows of the workload, in batches until the
+    time budget is used (at least one batch); the mean per-row time (unbiased under uniform sampling)
+    extrapolates to L rows.  Input generation is not timed."""
+    import oracle as O
+    if cfg.name not in _KEYS_CACHE:
+        _KEYS_CACHE[cfg.name] = G.prefill_keys(cfg, 7)
+    keys = _KEYS_CACHE[cfg.name]
+    rng = np.random.default_rng(seed)
+    rows = [int(r) for r in rng.choice(cfg.L, size=max_rows, replace=False)]
+    done, spent = 0, 0.0
+    while done < len(rows) and (done == 0 or spent < budget_s):
+        rs = rows[done:done + batch]
+        qs = G.prefill_queries(cfg, seed, rows=rs)
+        t = time.perf_counter()
+        O.prefill_rows(keys, qs, rs, cfg.k, cfg.scale, D_v=cfg.D_v)
+        spent += time.perf_counter() - t
+        done += len(rs)
+    return done / spent, done, spent
+
+
+def oracle_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        return max(int(i.get("num_threads", 1)) for i in threadpool_info()) or os.cpu_count()
+    except Exception:
+        return os.cpu_count()
+
+
+def run_reference(args, ws_n, rank):
+    if rank != 0:
+        return
+    cfg = PREFILL
+    for w in range(args.warmup):
+        oracle_prefill_rate(cfg, 0.0, 11 + w, max_rows=2, batch=2)
+    vals, rows_tot, spent_tot = [], 0, 0.0
+    for s in range(args.steps):
+        v, n, sp = oracle_prefill_rate(cfg, args.ref_step_seconds, 100 + s)
+        vals.append(v)
+        rows_tot += n
+        spent_tot += sp
+    value = rows_tot / spent_tot
+    cores = oracle_threads()
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": ws_n,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * cfg.L / value,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": cfg.name, "seq_len": cfg.L, "global_batch": 1, "H_I": cfg.H_I,
+                       "d_I": cfg.d_I, "k": cfg.k, "heads": cfg.H, "parallelism": "replicas"},
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                             "sample": f"{rows_tot} seeded random query rows of the L={cfg.L} prefill "
+                                       f"({spent_tot:.1f} s of host time), extrapolated to L rows"},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------------------------------------------------ main
+def main():
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["dsa", "reference"], default="dsa")
+    ap.add_argument("--decode-steps", type=int, default=256 - 3)
+    ap.add_argument("--e2e-steps", type=int, default=2)
+    ap.add_argument("--cpu-seconds", type=float, default=15.0, help="host time budget of the cpu_baseline leg")
+    ap.add_argument("--ref-step-seconds", type=float, default=8.0)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("at least 3 warm-up steps")
+
+    ws_n, rank, local = dist_init()
+    try:
+        if args.impl == "reference":
+            run_reference(args, ws_n, rank)
+        else:
+            run_dsa(args, ws_n, rank)
+    finally:
+        if ws_n > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+def run_dsa(args, ws_n, rank):
+    import sparse_attention_long_05_b200 as dsa
+    pk = peaks()
+    pre = bench_prefill(dsa, PREFILL, args.steps, args.warmup, ws_n, rank, pk)
+    torch.cuda.empty_cache()
+    dec = None
+    if not args.no_decode:
+        dec = bench_decode(dsa, DECODE, args.decode_steps, args.warmup, ws_n, rank, pk)
+        torch.cuda.empty_cache()
+    e2e = None
+    if not args.no_e2e:
+        e2e = bench_prefill_e2e(dsa, PREFILL, args.e2e_steps, rank)
+        torch.cuda.empty_cache()
+    if rank != 0:
+        return
+    cpu = None
+    if not args.no_cpu_baseline and ws_n == 1:
+        v, n, sp = oracle_prefill_rate(PREFILL, args.cpu_seconds, 7)
+        cpu = {"value": v, "unit": "tokens/s", "cores": oracle_threads(), "kind": "oracle",
+               "sample": f"{n} seeded random query rows of the L={PREFILL.L} prefill ({sp:.1f} s of host time), "
+                         "extrapolated to L rows"}
+    line = {
+        "metric": METRIC, "value": pre["tokens_per_s"], "unit": "tokens/s", "n_gpus": ws_n, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": pre["ms"], "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "e4m3+bf16", "data": "synthetic",
+        "config": {"workload": PREFILL.name, "model": "DSA forward (lightning indexer -> top-k -> sparse MLA, MQA)",
+                   "global_batch": ws_n, "seq_len": PREFILL.L, "H_I": PREFILL.H_I, "d_I": PREFILL.d_I,
+                   "k": PREFILL.k, "heads": PREFILL.H, "latent_dim": PREFILL.D, "value_dim": PREFILL.D_v,
+                   "indexer_inputs": "gaussian, fp8 e4m3 with per-token scale", "parallelism": "replicas",
+                   "l2": "inputs larger than L2 (q alone is 19 GB), no flush"},
+        "roofline": pre["roofline"], "kernels": pre["kernels"], "clocks": pre["clocks"],
+        "e2e": e2e, "gpu_launches": pre["launches"], "cpu_baseline": cpu, "decode": dec,
+    }
+    print(json.dumps(line), flush=True)
+
+
+if __name__ == "__main__":
+    main()

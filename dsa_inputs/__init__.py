@@ -36,6 +36,7 @@ __all__ = [
     "PrefillConfig", "DecodeConfig", "PREFILL_CONFIGS", "DECODE_CONFIG",
     "prefill_keys", "prefill_queries", "prefill_inputs",
     "decode_lengths", "decode_layout", "decode_cache_rows", "decode_fill_cache", "decode_step_inputs",
+    "decode_step_batch",
     "hash64", "uniform_int", "normal_index",
 ]
 
@@ -327,3 +328,26 @@ def decode_step_inputs(cfg: DecodeConfig, seed: int, step: int, device="cpu", se
     k_scale_new = torch.cat(kn["k_scale"]) if cfg.mode == "gauss" else torch.ones(len(seqs), device=device)
     return {"q_idx": q8.view(len(seqs), cfg.H_I, cfg.d_I), "q_scale": qs, "w": w, "q": q,
             "k_new": k_new, "k_scale_new": k_scale_new, "c_new": torch.cat(kn["c"])}
+
+
+def decode_step_batch(cfg: DecodeConfig, seed: int, steps: int, device="cpu", step0: int = 0):
+    """New-token tensors of decode steps step0..step0+steps-1 for all B sequences, stacked on a step axis.
+
+    Element for element identical to ``decode_step_inputs(cfg, seed, step)`` for each step.
+    """
+    lens = decode_lengths(cfg, seed)
+    B = cfg.B
+    tok = torch.arange(step0 * B, (step0 + steps) * B, dtype=torch.int64, device=device)   # step * B + b
+    q8, qs = _indexer_rows(stream_key(seed, "dec_q_idx"), tok, cfg.H_I * cfg.d_I, cfg.mode)
+    w = _weights(stream_key(seed, "dec_w"), tok, cfg.H_I, cfg.mode)
+    q = _rows_normal(stream_key(seed, "dec_q"), tok, cfg.H * cfg.D, torch.bfloat16)
+    b = tok % B
+    pos = torch.as_tensor(lens, dtype=torch.int64, device=device)[b] + tok // B
+    gid = b * _DEC_ROW_STRIDE + pos
+    k8, ks = _indexer_rows(stream_key(seed, "k_idx"), gid, cfg.d_I, cfg.mode)
+    c = _rows_normal(stream_key(seed, "c"), gid, cfg.D, torch.bfloat16)
+    if ks is None:
+        ks = torch.ones(steps * B, dtype=torch.float32, device=device)
+    return {"q_idx": q8.view(steps, B, cfg.H_I, cfg.d_I), "q_scale": None if qs is None else qs.view(steps, B),
+            "w": w.view(steps, B, cfg.H_I), "q": q.view(steps, B, cfg.H, cfg.D),
+            "k_new": k8.view(steps, B, cfg.d_I), "k_scale_new": ks.view(steps, B), "c_new": c.view(steps, B, cfg.D)}

@@ -101,8 +101,22 @@ DSA_API dsa_status_t dsa_topk(const float* scores, int rows, int64_t ld, const i
 DSA_API dsa_status_t dsa_sparse_mla_attn(const uint16_t* q, const uint16_t* c, int S, const int32_t* idx, int T,
                                  int H, int k, float scale, uint16_t* out, float* lse, void* stream);
 
-/* Workspace bytes of dsa_forward_prefill for these shapes. */
+/* Number of kernels this library has launched in this process (all devices, all entry points). */
+DSA_API uint64_t dsa_launch_count(void);
+
+/* Workspace bytes of dsa_prefill_select and dsa_forward_prefill for these shapes. */
 DSA_API size_t dsa_prefill_workspace_size(int L, int H_I, int d_I, int H, int k);
+
+/*
+ * Steps 1-2 for one causal prefill sequence of L tokens: the lightning-indexer scores of every row (s <= t)
+ * and their top-k selection (velog.io sections 1.1-1.2).
+ *   q_idx [L, H_I, d_I] e4m3, q_scale [L] or NULL, k_idx [L, d_I] e4m3, k_scale [L] or NULL, w [L, H_I] fp32;
+ *   idx_out [L, k] int32 (out): the selected positions of each row, ascending, padded with -1.
+ * The L x L score matrix is never stored (the workspace holds a bounded block of rows).
+ */
+DSA_API dsa_status_t dsa_prefill_select(const uint8_t* q_idx, const float* q_scale, const uint8_t* k_idx,
+                                        const float* k_scale, const float* w, int L, int H_I, int d_I, int k,
+                                        int32_t* idx_out, void* ws, size_t ws_bytes, void* stream);
 
 /*
  * Whole DSA forward for one causal prefill sequence of L tokens (steps 1-3 above, s <= t).

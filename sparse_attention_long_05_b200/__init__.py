@@ -10,7 +10,9 @@ from ._lib import (  # noqa: F401
     dsa_forward_prefill,
     dsa_get_device_status,
     dsa_indexer_scores,
+    dsa_launch_count,
     dsa_num_sms,
+    dsa_prefill_select,
     dsa_prefill_workspace_size,
     dsa_sparse_mla_attn,
     dsa_topk,

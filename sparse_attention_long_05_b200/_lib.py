@@ -27,7 +27,9 @@ SIGNATURES = {
     "dsa_indexer_scores": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P, _P]),
     "dsa_topk": (_I, [_P, _I, _I64, _P, _I, _I, _P, _P]),
     "dsa_sparse_mla_attn": (_I, [_P, _P, _I, _P, _I, _I, _I, _F, _P, _P, _P]),
+    "dsa_launch_count": (ctypes.c_uint64, []),
     "dsa_prefill_workspace_size": (_SZ, [_I, _I, _I, _I, _I]),
+    "dsa_prefill_select": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _P, _P, _SZ, _P]),
     "dsa_forward_prefill": (_I, [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _P, _P, _P, _P, _SZ, _P]),
     "dsa_decode_workspace_size": (_SZ, [_I, _I64, _I, _I, _I, _I]),
     "dsa_forward_decode": (_I, [_I, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _I64, _I, _I, _I, _I, _F,
@@ -122,6 +124,24 @@ def dsa_sparse_mla_attn(q, c, idx, scale: float, out=None, lse=None, want_lse: b
 
 def dsa_prefill_workspace_size(L: int, H_I: int, d_I: int, H: int, k: int) -> int:
     return int(_lib.dsa_prefill_workspace_size(L, H_I, d_I, H, k))
+
+
+def dsa_launch_count() -> int:
+    return int(_lib.dsa_launch_count())
+
+
+def dsa_prefill_select(q_idx, q_scale, k_idx, k_scale, w, k: int, idx_out=None, ws=None, stream=None):
+    """Indexer scores + top-k of every row of one causal prefill sequence -> idx [L, k] (int32)."""
+    L, H_I, d_I = q_idx.shape
+    dev = q_idx.device
+    if idx_out is None:
+        idx_out = torch.empty((L, k), dtype=torch.int32, device=dev)
+    if ws is None:
+        ws = torch.empty((dsa_prefill_workspace_size(L, H_I, d_I, 1, k),), dtype=torch.uint8, device=dev)
+    _check("dsa_prefill_select", _lib.dsa_prefill_select(
+        _ptr(q_idx), _ptr(q_scale), _ptr(k_idx), _ptr(k_scale), _ptr(w), L, H_I, d_I, k, _ptr(idx_out), _ptr(ws),
+        ws.numel(), _stream(stream)))
+    return idx_out
 
 
 def dsa_forward_prefill(q_idx, q_scale, k_idx, k_scale, w, q, c, k: int, scale: float, idx_out=None, out=None,

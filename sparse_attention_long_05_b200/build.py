@@ -1,7 +1,8 @@
 """Build step of the CUDA library: compiles csrc/dsa_api.cu (one translation unit) into libdsa.so, in-tree.
 
-Run as ``python -m sparse_attention_long_05_b200.build`` or through ``__graft_entry__.build()``.  nvcc
-cross-compiles for sm_100a, so this works on a machine without a GPU.
+Run as ``python sparse_attention_long_05_b200/build.py`` or through ``__graft_entry__.build()`` (both load
+this file by path, so building never imports the package, which loads the library).  nvcc cross-compiles
+for sm_100a, so this works on a machine without a GPU.
 """
 from __future__ import annotations
 
@@ -52,6 +53,11 @@ def build(force: bool = False, verbose: bool = False, extra=()) -> str:
     if verbose and (res.stdout or res.stderr):
         print(res.stdout + res.stderr)
     return OUT
+
+
+def load_module():
+    """This module, loaded by file path (for callers that must not import the package first)."""
+    return sys.modules[__name__]
 
 
 if __name__ == "__main__":

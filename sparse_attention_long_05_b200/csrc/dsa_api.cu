@@ -5,6 +5,7 @@
 // below.
 #include <cmath>
 #include <cstdio>
+#include <atomic>
 #include <mutex>
 
 #include "common.cuh"
@@ -84,7 +85,10 @@ cudaError_t set_smem(K kernel, int bytes) {
   return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
 }
 
+std::atomic<unsigned long long> g_launches{0};
+
 dsa_status_t last_launch_status() {
+  g_launches.fetch_add(1, std::memory_order_relaxed);
   return cudaGetLastError() == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
 }
 
@@ -256,6 +260,29 @@ size_t dsa_prefill_workspace_size(int L, int H_I, int d_I, int H, int k) {
   return align_up(rows * size_t(L) * 4, 256) + align_up(size_t(L) * size_t(k) * 4, 256);
 }
 
+dsa_status_t dsa_prefill_select(const uint8_t* q_idx, const float* q_scale, const uint8_t* k_idx,
+                                const float* k_scale, const float* w, int L, int H_I, int d_I, int k,
+                                int32_t* idx_out, void* ws, size_t ws_bytes, void* stream) {
+  if (L <= 0 || k <= 0 || !q_idx || !k_idx || !w || !idx_out) return DSA_ERR_INVALID_ARG;
+  if (!indexer_shape_ok(H_I, d_I)) return DSA_ERR_UNSUPPORTED_SHAPE;
+  if (!aligned16(q_idx) || !aligned16(k_idx)) return DSA_ERR_ALIGNMENT;
+  if (!ws || ws_bytes < align_up(prefill_chunk_rows(L) * size_t(L) * 4, 256)) return DSA_ERR_WORKSPACE;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const size_t R = prefill_chunk_rows(L);
+  float* sc = static_cast<float*>(ws);
+  for (int r0 = 0; r0 < L; r0 += static_cast<int>(R)) {
+    const int rows = (L - r0 < static_cast<int>(R)) ? L - r0 : static_cast<int>(R);
+    const int s_eff = r0 + rows;   // keys beyond the block's last row are never selected (causal)
+    dsa_status_t e = run_indexer_scores(q_idx + static_cast<size_t>(r0) * H_I * d_I, q_scale ? q_scale + r0 : nullptr,
+                                        k_idx, k_scale, w + static_cast<size_t>(r0) * H_I, rows, s_eff, H_I, d_I,
+                                        r0, sc, s_eff, st);
+    if (e != DSA_OK) return e;
+    e = run_topk(sc, s_eff, nullptr, nullptr, r0, rows, k, idx_out + static_cast<size_t>(r0) * k, k, st);
+    if (e != DSA_OK) return e;
+  }
+  return DSA_OK;
+}
+
 dsa_status_t dsa_forward_prefill(const uint8_t* q_idx, const float* q_scale, const uint8_t* k_idx,
                                  const float* k_scale, const float* w, const uint16_t* q, const uint16_t* c,
                                  int L, int H_I, int d_I, int H, int k, float scale, int32_t* idx_out,
@@ -266,22 +293,15 @@ dsa_status_t dsa_forward_prefill(const uint8_t* q_idx, const float* q_scale, con
     return DSA_ERR_ALIGNMENT;
   if (!ws || ws_bytes < dsa_prefill_workspace_size(L, H_I, d_I, H, k)) return DSA_ERR_WORKSPACE;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  const size_t R = prefill_chunk_rows(L);
-  float* sc = static_cast<float*>(ws);
   int32_t* idx = idx_out ? idx_out
-                         : reinterpret_cast<int32_t*>(static_cast<char*>(ws) + align_up(R * size_t(L) * 4, 256));
-  for (int r0 = 0; r0 < L; r0 += static_cast<int>(R)) {
-    const int rows = (L - r0 < static_cast<int>(R)) ? L - r0 : static_cast<int>(R);
-    const int s_eff = r0 + rows;   // keys beyond the chunk's last row are never selected (causal)
-    dsa_status_t e = run_indexer_scores(q_idx + static_cast<size_t>(r0) * H_I * d_I, q_scale ? q_scale + r0 : nullptr,
-                                        k_idx, k_scale, w + static_cast<size_t>(r0) * H_I, rows, s_eff, H_I, d_I,
-                                        r0, sc, s_eff, st);
-    if (e != DSA_OK) return e;
-    e = run_topk(sc, s_eff, nullptr, nullptr, r0, rows, k, idx + static_cast<size_t>(r0) * k, k, st);
-    if (e != DSA_OK) return e;
-  }
+                         : reinterpret_cast<int32_t*>(static_cast<char*>(ws) +
+                                                      align_up(prefill_chunk_rows(L) * size_t(L) * 4, 256));
+  dsa_status_t e = dsa_prefill_select(q_idx, q_scale, k_idx, k_scale, w, L, H_I, d_I, k, idx, ws, ws_bytes, stream);
+  if (e != DSA_OK) return e;
   return run_mla(q, c, L, idx, nullptr, L, H, k, scale, out, lse, st);
 }
+
+uint64_t dsa_launch_count(void) { return g_launches.load(); }
 
 size_t dsa_decode_workspace_size(int B, int64_t cache_rows, int H_I, int d_I, int H, int k) {
   (void)H_I; (void)d_I; (void)H;

@@ -261,7 +261,9 @@ sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     for (int t = p.T > 0 ? cluster : p.T; t < p.T && ok; t += nclusters) {
       const long long base = p.row_off ? p.row_off[t] : 0;
       const int* irow = p.idx + static_cast<long long>(t) * p.k;
-      float m_ref = -INFINITY, l = 0.f;
+      // l: sum of the bf16-rounded probabilities that enter P . V (normalises O exactly);
+      // le: sum of the unrounded probabilities (for the log-sum-exp output)
+      float m_ref = -INFINITY, l = 0.f, le = 0.f;
       for (int j = 0; j < ntiles; ++j, ++g) {
         const int sb = static_cast<int>(g & 1);
         const int2 e = *reinterpret_cast<const int2*>(irow + j * NK + 2 * lane);
@@ -291,10 +293,11 @@ sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         if (mt > m_ref + RESCALE_LOG2) {
           alpha = (m_ref == -INFINITY) ? 0.f : ex2_approx(m_ref - mt);
           l *= alpha;
+          le *= alpha;
           m_ref = mt;
         }
         uint32_t pk[NK / 2];
-        float ls = 0.f;
+        float ls = 0.f, lx = 0.f;
 #pragma unroll
         for (int i = 0; i < NK / 2; ++i) {
           const float x0 = __uint_as_float(v[2 * i]), x1 = __uint_as_float(v[2 * i + 1]);
@@ -302,9 +305,11 @@ sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
           const float p1 = (x1 == -INFINITY) ? 0.f : ex2_approx(x1 - m_ref);
           const __nv_bfloat162 b = __floats2bfloat162_rn(p0, p1);
           ls += __low2float(b) + __high2float(b);
+          lx += p0 + p1;
           pk[i] = *reinterpret_cast<const uint32_t*>(&b);
         }
         l += ls;
+        le += lx;
         // P buffer sb of the value CTA is free once its PV of tile g - 2 has completed
         if (!(ok = mbar_wait<true>(bar(B_P_EMPTY + sb), ((g >> 1) & 1) ^ 1, abort_flag))) break;
         const uint32_t prow = p_remote + sb * (128 * 128) + h * 128;
@@ -320,7 +325,7 @@ sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
           asm volatile("st.shared::cluster.f32 [%0], %1;" :: "r"(lsum_remote + 4 * h), "f"(l) : "memory");
           if (p.lse && h < p.H)
             p.lse[static_cast<long long>(t) * p.H + h] =
-                (l > 0.f) ? (m_ref + lg2_approx(l)) * 0.69314718055994531f : -INFINITY;
+                (le > 0.f) ? (m_ref + lg2_approx(le)) * 0.69314718055994531f : -INFINITY;
         }
         fence_proxy_async();
         mbar_arrive_remote(pfull_remote + 8 * sb);

@@ -76,3 +76,16 @@ def test_decode_layout_and_append_rows():
 def test_decode_lengths_span():
     lens = np.array(G.decode_lengths(G.DECODE_CONFIG, 20251202))
     assert lens.min() >= 4096 and lens.max() <= 131072 and len(lens) == 64
+
+
+def test_decode_step_batch_matches_single_steps():
+    cfg = G.DecodeConfig("small", B=3, len_lo=100, len_hi=300, steps=4, mode="gauss")
+    batch = G.decode_step_batch(cfg, 5, 4)
+    tail = G.decode_step_batch(cfg, 5, 2, step0=2)
+    assert torch.equal(tail["q"][1], batch["q"][3])
+    for step in (0, 3):
+        one = G.decode_step_inputs(cfg, 5, step)
+        for key in ("q", "w", "q_scale", "k_scale_new", "c_new"):
+            assert torch.equal(batch[key][step], one[key]), key
+        for key in ("q_idx", "k_new"):
+            assert torch.equal(batch[key][step].view(torch.uint8), one[key].view(torch.uint8)), key

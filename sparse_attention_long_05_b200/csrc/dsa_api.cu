@@ -156,18 +156,15 @@ dsa_status_t run_topk(const float* scores, long long ld, const long long* row_of
 dsa_status_t run_mla(const uint16_t* q, const uint16_t* c, long long S, const int* idx, const long long* row_off,
                      int T, int H, int k, float scale, uint16_t* out, float* lse, cudaStream_t st) {
   if (T <= 0) return DSA_OK;
-  CUtensorMap tq, tc;
+  CUtensorMap tq;
   const cuuint64_t qd[3] = {576, static_cast<cuuint64_t>(H), static_cast<cuuint64_t>(T)};
   const cuuint64_t qs[2] = {576 * 2, static_cast<cuuint64_t>(H) * 576 * 2};
   const cuuint32_t qb[3] = {64, 128, 1};
-  const cuuint64_t cd[2] = {576, static_cast<cuuint64_t>(S)};
-  const cuuint64_t cs[1] = {576 * 2};
-  const cuuint32_t cb[2] = {64, 1};
   if (!make_map(&tq, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, q, qd, qs, qb, CU_TENSOR_MAP_SWIZZLE_128B)) return DSA_ERR_CUDA;
-  if (!make_map(&tc, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, c, cd, cs, cb, CU_TENSOR_MAP_SWIZZLE_128B)) return DSA_ERR_CUDA;
   MlaParams p{};
   p.idx = idx;
   p.row_off = row_off;
+  p.c = c;
   p.out = out;
   p.lse = lse;
   p.T = T;
@@ -178,9 +175,11 @@ dsa_status_t run_mla(const uint16_t* q, const uint16_t* c, long long S, const in
   if (set_smem(sparse_mla_kernel, mla::SMEM) != cudaSuccess) return DSA_ERR_CUDA;
   int clusters = num_sms() / 2;
   if (clusters > T) clusters = T;
-  sparse_mla_kernel<<<2 * clusters, mla::THREADS, mla::SMEM, st>>>(tq, tc, p);
+  sparse_mla_kernel<<<2 * clusters, mla::THREADS, mla::SMEM, st>>>(tq, p);
   return last_launch_status();
 }
+
+bool mla_k_ok(int k) { return k > 0 && k % mla::NK == 0 && k <= mla::KMAX; }
 
 bool indexer_shape_ok(int H_I, int d_I) { return (H_I == 64 && d_I == 128) || (H_I == 4 && d_I == 64); }
 
@@ -247,9 +246,8 @@ dsa_status_t dsa_topk(const float* scores, int rows, int64_t ld, const int32_t* 
 dsa_status_t dsa_sparse_mla_attn(const uint16_t* q, const uint16_t* c, int S, const int32_t* idx, int T, int H,
                                  int k, float scale, uint16_t* out, float* lse, void* stream) {
   if (T < 0 || S <= 0 || H <= 0 || k <= 0 || (T > 0 && (!q || !c || !idx || !out))) return DSA_ERR_INVALID_ARG;
-  if (H > 128 || k % mla::NK != 0) return DSA_ERR_UNSUPPORTED_SHAPE;
-  if (!aligned16(q) || !aligned16(c) || (reinterpret_cast<uintptr_t>(idx) & 7u) || !aligned16(out))
-    return DSA_ERR_ALIGNMENT;
+  if (H > 128 || !mla_k_ok(k)) return DSA_ERR_UNSUPPORTED_SHAPE;
+  if (!aligned16(q) || !aligned16(c) || !aligned16(idx) || !aligned16(out)) return DSA_ERR_ALIGNMENT;
   return run_mla(q, c, S, idx, nullptr, T, H, k, scale, out, lse, static_cast<cudaStream_t>(stream));
 }
 
@@ -288,8 +286,9 @@ dsa_status_t dsa_forward_prefill(const uint8_t* q_idx, const float* q_scale, con
                                  int L, int H_I, int d_I, int H, int k, float scale, int32_t* idx_out,
                                  uint16_t* out, float* lse, void* ws, size_t ws_bytes, void* stream) {
   if (L <= 0 || H <= 0 || k <= 0 || !q_idx || !k_idx || !w || !q || !c || !out) return DSA_ERR_INVALID_ARG;
-  if (!indexer_shape_ok(H_I, d_I) || H > 128 || k % mla::NK != 0) return DSA_ERR_UNSUPPORTED_SHAPE;
-  if (!aligned16(q_idx) || !aligned16(k_idx) || !aligned16(q) || !aligned16(c) || !aligned16(out))
+  if (!indexer_shape_ok(H_I, d_I) || H > 128 || !mla_k_ok(k)) return DSA_ERR_UNSUPPORTED_SHAPE;
+  if (!aligned16(q_idx) || !aligned16(k_idx) || !aligned16(q) || !aligned16(c) || !aligned16(out) ||
+      (idx_out && !aligned16(idx_out)))
     return DSA_ERR_ALIGNMENT;
   if (!ws || ws_bytes < dsa_prefill_workspace_size(L, H_I, d_I, H, k)) return DSA_ERR_WORKSPACE;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
@@ -318,9 +317,9 @@ dsa_status_t dsa_forward_decode(int B, const int64_t* cache_off, const int32_t* 
   if (B <= 0 || cache_rows <= 0 || H <= 0 || k <= 0 || !cache_off || !ctx_len || !q_idx || !w || !q || !k_new ||
       !k_scale_new || !c_new || !k_cache || !k_scale_cache || !c_cache || !out)
     return DSA_ERR_INVALID_ARG;
-  if (H_I != 64 || d_I != 128 || H > 128 || k % mla::NK != 0 || B > kMaxDecodeSeqs) return DSA_ERR_UNSUPPORTED_SHAPE;
+  if (H_I != 64 || d_I != 128 || H > 128 || !mla_k_ok(k) || B > kMaxDecodeSeqs) return DSA_ERR_UNSUPPORTED_SHAPE;
   if (!aligned16(q_idx) || !aligned16(q) || !aligned16(k_new) || !aligned16(c_new) || !aligned16(k_cache) ||
-      !aligned16(c_cache) || !aligned16(out))
+      !aligned16(c_cache) || !aligned16(out) || (idx_out && !aligned16(idx_out)))
     return DSA_ERR_ALIGNMENT;
   if (!ws || ws_bytes < dsa_decode_workspace_size(B, cache_rows, H_I, d_I, H, k)) return DSA_ERR_WORKSPACE;
   cudaStream_t st = static_cast<cudaStream_t>(stream);

@@ -21,7 +21,7 @@
  *   - Nothing is allocated inside a call: scratch memory is a caller-provided workspace whose size the
  *     matching *_workspace_size() function returns.
  *   - Supported shapes: H_I in {4, 64} with d_I = 64 / 128 respectively, H <= 128 query heads, D = 576 latent
- *     dims of which the first D_v = 512 are the value, k a multiple of 64 and at most 2048.  Other shapes
+ *     dims of which the first D_v = 512 are the value, k a multiple of 64 from 128 to 2048.  Other shapes
  *     return DSA_ERR_UNSUPPORTED_SHAPE.
  *   - Results are bitwise deterministic for fixed inputs and launch configuration.
  */
@@ -90,7 +90,7 @@ DSA_API dsa_status_t dsa_topk(const float* scores, int rows, int64_t ld, const i
 
 /*
  * Sparse MLA attention in MQA mode over selected latent entries (velog.io sections 1.2 and 1.3).
- * k is a multiple of 64, at most 2048; idx must be 16-byte aligned.
+ * k is a multiple of 64 between 128 and 2048; idx must be 16-byte aligned.
  *   q     [T, H, 576] bf16    queries (H <= 128)
  *   c     [S, 576] bf16       shared latent entries; the value of an entry is its first 512 dims
  *   idx   [T, k] int32        selected entries of each row, in [0, S) or -1 (= nothing), any order

@@ -15,6 +15,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 SRC = os.path.join(HERE, "csrc", "dsa_api.cu")
 OUT = os.path.join(HERE, "libdsa.so")
+OUT_TRACE = os.path.join(HERE, "libdsa_trace.so")   # -DDSA_TRACE: pipeline event stamps, profiling only
 DEPS = [os.path.join(HERE, "csrc", f) for f in os.listdir(os.path.join(HERE, "csrc"))] + \
        [os.path.join(ROOT, "include", "dsa.h")]
 
@@ -60,6 +61,18 @@ def load_module():
     return sys.modules[__name__]
 
 
+def build_traced(verbose: bool = False) -> str:
+    """The same library with the kernels' pipeline tracing compiled in (a separate .so, for profiling)."""
+    res = subprocess.run(command(out=OUT_TRACE, extra=("-DDSA_TRACE",)), capture_output=True, text=True)
+    if res.returncode != 0:
+        sys.stderr.write(res.stdout + res.stderr)
+        raise RuntimeError("nvcc failed building libdsa_trace.so")
+    return OUT_TRACE
+
+
 if __name__ == "__main__":
-    build(force="--force" in sys.argv, verbose=True,
-          extra=("-Xptxas", "-v") if "--ptxas-v" in sys.argv else ())
+    if "--trace" in sys.argv:
+        print(build_traced(verbose=True))
+    else:
+        build(force="--force" in sys.argv, verbose=True,
+              extra=("-Xptxas", "-v") if "--ptxas-v" in sys.argv else ())

@@ -24,6 +24,25 @@ __device__ long long g_wait_limit = (1ll << 31);
 
 __device__ __forceinline__ void raise_status(int code) { atomicCAS(&g_dev_status, 0, code); }
 
+// ------------------------------------------------------------------------------------------ tracing
+// Built with -DDSA_TRACE (the traced library, libdsa_trace.so), kernels record %globaltimer stamps of their
+// pipeline events for the first cluster / CTA into g_trace[event][tile]; read back with dsa_trace_read().
+// In the normal build the hooks compile to nothing.
+#ifdef DSA_TRACE
+constexpr int kTraceEvents = 32, kTraceTiles = 256;
+__device__ unsigned long long g_trace[kTraceEvents][kTraceTiles];
+__device__ __forceinline__ void trace_event(int ev, long long tile) {
+  if (blockIdx.x < 2 && tile >= 0 && tile < kTraceTiles) {
+    unsigned long long t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    g_trace[ev][tile] = t;
+  }
+}
+#define DSA_TRACE_EVENT(ev, tile) ::dsa::trace_event((ev), (tile))
+#else
+#define DSA_TRACE_EVENT(ev, tile) ((void)0)
+#endif
+
 // ------------------------------------------------------------------------------------------ addressing
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -66,13 +85,16 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t byt
 __device__ __forceinline__ void mbar_arrive_remote(uint32_t cluster_addr) {
   asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" :: "r"(cluster_addr) : "memory");
 }
+// Waiting threads are suspended by the hardware (up to kSuspendNs per try) until the phase completes, so a
+// waiting warp does not take issue slots from the warps doing work on the same SM sub-partition.
+constexpr uint32_t kSuspendNs = 20000;
 __device__ __forceinline__ bool mbar_test(uint32_t bar, uint32_t parity) {
   uint32_t ok;
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
       "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(ok) : "r"(bar), "r"(parity) : "memory");
+      : "=r"(ok) : "r"(bar), "r"(parity), "n"(kSuspendNs) : "memory");
   return ok != 0;
 }
 // acquire at cluster scope: for barriers another CTA of the cluster arrives on
@@ -80,9 +102,9 @@ __device__ __forceinline__ bool mbar_test_cluster(uint32_t bar, uint32_t parity)
   uint32_t ok;
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2, %3;\n\t"
       "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(ok) : "r"(bar), "r"(parity) : "memory");
+      : "=r"(ok) : "r"(bar), "r"(parity), "n"(kSuspendNs) : "memory");
   return ok != 0;
 }
 
@@ -170,6 +192,10 @@ __device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" :: "r"(dst), "l"(src) : "memory");
 }
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+// arrive on `bar` (without raising its pending count) once every cp.async this thread issued so far has landed
+__device__ __forceinline__ void cp_async_arrive_noinc(uint32_t bar) {
+  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" :: "r"(bar) : "memory");
+}
 template <int N>
 __device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" :: "n"(N) : "memory"); }
 

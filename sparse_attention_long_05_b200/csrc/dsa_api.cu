@@ -161,10 +161,14 @@ dsa_status_t run_mla(const uint16_t* q, const uint16_t* c, long long S, const in
   const cuuint64_t qs[2] = {576 * 2, static_cast<cuuint64_t>(H) * 576 * 2};
   const cuuint32_t qb[3] = {64, 128, 1};
   if (!make_map(&tq, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, q, qd, qs, qb, CU_TENSOR_MAP_SWIZZLE_128B)) return DSA_ERR_CUDA;
+  CUtensorMap tc;   // rows of c, one 64-column box high 1 row (the form tile::gather4 takes)
+  const cuuint64_t cd[2] = {576, static_cast<cuuint64_t>(S)};
+  const cuuint64_t cs[1] = {576 * 2};
+  const cuuint32_t cb[2] = {64, 1};
+  if (!make_map(&tc, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, c, cd, cs, cb, CU_TENSOR_MAP_SWIZZLE_128B)) return DSA_ERR_CUDA;
   MlaParams p{};
   p.idx = idx;
   p.row_off = row_off;
-  p.c = c;
   p.out = out;
   p.lse = lse;
   p.T = T;
@@ -175,11 +179,11 @@ dsa_status_t run_mla(const uint16_t* q, const uint16_t* c, long long S, const in
   if (set_smem(sparse_mla_kernel, mla::SMEM) != cudaSuccess) return DSA_ERR_CUDA;
   int clusters = num_sms() / 2;
   if (clusters > T) clusters = T;
-  sparse_mla_kernel<<<2 * clusters, mla::THREADS, mla::SMEM, st>>>(tq, p);
+  sparse_mla_kernel<<<2 * clusters, mla::THREADS, mla::SMEM, st>>>(tq, tc, p);
   return last_launch_status();
 }
 
-bool mla_k_ok(int k) { return k > 0 && k % mla::NK == 0 && k <= mla::KMAX; }
+bool mla_k_ok(int k) { return k >= 2 * mla::NK && k % mla::NK == 0 && k <= mla::KMAX; }
 
 bool indexer_shape_ok(int H_I, int d_I) { return (H_I == 64 && d_I == 128) || (H_I == 4 && d_I == 64); }
 
@@ -301,6 +305,15 @@ dsa_status_t dsa_forward_prefill(const uint8_t* q_idx, const float* q_scale, con
 }
 
 uint64_t dsa_launch_count(void) { return g_launches.load(); }
+
+#ifdef DSA_TRACE
+// traced build only: copy the event stamps out and clear them
+__attribute__((visibility("default"))) int dsa_trace_read(unsigned long long* host) {
+  if (cudaMemcpyFromSymbol(host, g_trace, sizeof(g_trace)) != cudaSuccess) return DSA_ERR_CUDA;
+  static unsigned long long zero[kTraceEvents][kTraceTiles];
+  return cudaMemcpyToSymbol(g_trace, zero, sizeof(zero)) == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
+}
+#endif
 
 size_t dsa_decode_workspace_size(int B, int64_t cache_rows, int H_I, int d_I, int H, int k) {
   (void)H_I; (void)d_I; (void)H;

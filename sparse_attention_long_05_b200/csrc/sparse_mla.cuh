@@ -16,18 +16,27 @@
 // logit or probability ever leaves the chip.
 //
 // Data movement.
-//   * Selected rows are gathered with 16-byte cp.async copies by four warps per CTA into 64-key x 64-dim
-//     stages laid out in the 128-byte swizzled K-major form the tensor core reads; a stage is handed to the
-//     MMA warp through an mbarrier after the copies have landed and been fenced into the async proxy.  The
+//   * Selected rows are gathered by TMA tile::gather4 (four rows x one 64-column, 128-byte swizzled box per
+//     instruction) into 64-key x 64-dim stages in the K-major form the tensor core reads.  Eight warps issue
+//     the gathers, each owning every eighth stage, because one warp issues gather4 instructions only about
+//     every 50 ns (gather throughput per SM grows with the number of issuing warps: about 12, 24, 45 and
+//     73 GB/s with 1, 2, 4 and 8); TMA writes are in the async proxy, so the MMA warp consumes a stage as
+//     soon as its
+//     mbarrier transaction count completes, with no proxy fence.  The
 //     same stage bytes serve as the K-major B operand of QK^T (rows = keys) and as the MN-major B operand
 //     of PV (rows = keys = K, 64 dims = N per atom).
 //   * The token's selected-index row is prefetched into shared memory with one bulk copy.
-//   * Q chunks (128 heads x 64 dims) are staged by TMA and copied into tensor memory with tcgen05.cp; the
-//     next token's chunks replace the current ones during the current token's last tile, right after the
-//     MMAs that last read them (tcgen05.mma and tcgen05.cp of one thread execute in issue order).
+//   * Q chunks (128 heads x 64 dims) are staged by TMA (three shared-memory slots) and copied into a ring of
+//     twelve 32-column chunk slots of tensor memory with tcgen05.cp; chunk c of the token with running index
+//     ti lives in slot (9 ti + c) mod 12.  A copy may only overwrite a slot once the MMAs that last read it
+//     have completed, which the MMA thread learns from tcgen05.commit barriers: per token, the next token's
+//     chunks 0-2 are copied at the start of tile 1 (their slots held chunks 6-8 of the token before, retired),
+//     chunks 3-5 during the last tile, three chunks after the MMAs that last read those slots were committed,
+//     and chunks 6-8 during the next token's first tile, just before their first use.  No copy waits on an
+//     MMA issued less than three chunks earlier.
 //
-// Warp roles (10 warps per CTA): w0 loader (index rows, Q chunks), w1 TMEM allocation + MMA issue,
-// w2 w3 w8 w9 gathers, w4..w7 softmax (score CTA) or correction / epilogue (value CTA); warp w owns TMEM
+// Warp roles (14 warps per CTA): w0 loader (index rows, Q chunks), w1 TMEM allocation + MMA issue,
+// w2 w3 w8..w13 gathers, w4..w7 softmax (score CTA) or correction / epilogue (value CTA); warp w owns TMEM
 // lanes (= heads) 32 * (w % 4) .. +31.
 #pragma once
 #include "common.cuh"
@@ -37,7 +46,6 @@ namespace dsa {
 struct MlaParams {
   const int* idx;              // [T, k]
   const long long* row_off;    // [T] row of entry 0 of each token in c, or null (0)
-  const uint16_t* c;           // [S, 576] bf16 (gathered with cp.async)
   uint16_t* out;               // [T, H, 512] bf16
   float* lse;                  // [T, H] or null
   int T, H, k;
@@ -54,18 +62,18 @@ constexpr int CHUNK_BYTES = NK * 128;     // 8 KB: 64 keys x 64 bf16
 constexpr int QCHUNK_BYTES = 128 * 128;   // 16 KB: 128 heads x 64 bf16
 constexpr int KMAX = 2048;                // largest selection handled (index row slot of 8 KB)
 constexpr int QS = 3;                     // Q staging slots (score CTA)
-constexpr int NSB = 3;                    // S buffers in tensor memory (score CTA)
+constexpr int NSB = 2;                    // S buffers in tensor memory (score CTA)
+constexpr int QSLOTS = 12;                // Q chunk slots in tensor memory (score CTA)
 constexpr int NPB = 3;                    // P buffers (value CTA)
 constexpr int NS_S = 15, NS_V = 16;       // gather stages per CTA
-constexpr int GD = 12;                    // gather chunks in flight per thread before signalling
-constexpr int THREADS = 320;
-constexpr int GATHER_THREADS = 128;
+constexpr int THREADS = 448;
+constexpr int GATHER_WARPS = 8;
 constexpr float RESCALE_LOG2 = 8.0f;      // lazy rescale threshold (factor 256)
 constexpr int P_BYTES = 128 * 128;        // 128 heads x 64 keys bf16
 constexpr int XFER = P_BYTES + 512 + 512; // P + alpha[128] + lsum[128]
 constexpr uint32_t TMEM_COLS = 512;
-constexpr uint32_t TQ = 0;                // score CTA: Q in columns 0..287
-constexpr uint32_t TS = 320;              // score CTA: S buffers at 320, 384, 448
+constexpr uint32_t TQ = 0;                // score CTA: Q chunk slots in columns 0..383
+constexpr uint32_t TS = 384;              // score CTA: S buffers at 384, 448
 // barrier slots
 constexpr int B_IDX_FULL = 0, B_IDX_EMPTY = 2;
 constexpr int B_QST_FULL = 4, B_QST_EMPTY = B_QST_FULL + QS;
@@ -74,7 +82,9 @@ constexpr int B_S_FULL = B_RING_EMPTY + 16, B_S_EMPTY = B_S_FULL + NSB, B_P_EMPT
 constexpr int B_P_FULL = B_P_EMPTY + NPB, B_P_READY = B_P_FULL + NPB;
 constexpr int B_O_DONE = B_P_READY + NPB, B_O_FREE = B_O_DONE + 1;
 constexpr int B_SLOT_FREE = B_O_FREE + 1, B_SLOT_WRITTEN = B_SLOT_FREE + 1;   // score CTA softmax handshakes
-constexpr int B_COUNT = B_SLOT_WRITTEN + 1;
+constexpr int B_QRET = B_SLOT_WRITTEN + 1;    // score CTA: last-tile MMAs of chunks 0..2 retired (3 barriers)
+constexpr int B_QTOK = B_QRET + 3;            // score CTA: every MMA of a token retired
+constexpr int B_COUNT = B_QTOK + 1;
 // shared memory map (from a 1024-byte aligned base; both CTAs use the same barrier offsets)
 constexpr int OFF_TMEM = 8 * B_COUNT;
 constexpr int OFF_ABORT = OFF_TMEM + 4;
@@ -91,7 +101,6 @@ static_assert(OFF_TMEM + 8 <= OFF_IDX, "barrier area");
 static_assert(OFF_PST % 1024 == 0 && OFF_QST % 1024 == 0 && OFF_RING_S % 1024 == 0, "1 KB aligned tiles");
 static_assert(OFF_PB % 1024 == 0 && XFER % 1024 == 0 && OFF_RING_V % 1024 == 0, "1 KB aligned tiles");
 static_assert(NS_V % 4 == 0, "value stages come in groups of four 64-dim chunks");
-static_assert(GD < NS_S && GD < NS_V, "gather signalling depth below the ring size");
 static_assert(SMEM <= 232448, "shared memory per CTA");
 }  // namespace mla
 
@@ -104,6 +113,17 @@ __device__ __forceinline__ long long mla_row(int e, long long base, long long S)
 }
 __device__ __forceinline__ bool mla_valid(int e, long long base, long long S) { return e >= 0 && base + e < S; }
 
+// position in a ring of `size` stages (size known at run time): stage index and pass parity, advanced
+// incrementally so that no division runs in the per-chunk loops
+struct RingPos {
+  int stage = 0;
+  uint32_t phase = 0;
+  int size = 1;
+  __device__ __forceinline__ void advance() {
+    if (++stage == size) { stage = 0; phase ^= 1; }
+  }
+};
+
 // every lane waits (bounded); the warp then agrees on the outcome so that it stays converged
 template <bool kCluster = false>
 __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag) {
@@ -112,7 +132,8 @@ __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, volatil
 }
 
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(mla::THREADS, 1)
-sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_q, const MlaParams p) {
+sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_c,
+                  const MlaParams p) {
   using namespace mla;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -131,15 +152,20 @@ sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_q, const MlaParams p) {
   if (threadIdx.x == 0) {
     for (int i = 0; i < 2; ++i) {
       mbar_init(bar(B_IDX_FULL + i), 1);
-      mbar_init(bar(B_IDX_EMPTY + i), rank == 0 ? 8 : 4);
+      mbar_init(bar(B_IDX_EMPTY + i), rank == 0 ? GATHER_WARPS + 4 : GATHER_WARPS);
     }
-    for (int i = 0; i < 16; ++i) { mbar_init(bar(B_RING_FULL + i), 4); mbar_init(bar(B_RING_EMPTY + i), 1); }
+    for (int i = 0; i < 16; ++i) {
+      mbar_init(bar(B_RING_FULL + i), 1);                // the issuing warp's arrive.expect_tx + TMA bytes
+      mbar_init(bar(B_RING_EMPTY + i), 1);
+    }
     if (rank == 0) {
       for (int i = 0; i < QS; ++i) { mbar_init(bar(B_QST_FULL + i), 1); mbar_init(bar(B_QST_EMPTY + i), 1); }
       for (int i = 0; i < NSB; ++i) { mbar_init(bar(B_S_FULL + i), 1); mbar_init(bar(B_S_EMPTY + i), 4); }
       for (int i = 0; i < NPB; ++i) mbar_init(bar(B_P_EMPTY + i), 1);
       mbar_init(bar(B_SLOT_FREE), 1);
       mbar_init(bar(B_SLOT_WRITTEN), 4);
+      for (int i = 0; i < 3; ++i) mbar_init(bar(B_QRET + i), 1);
+      mbar_init(bar(B_QTOK), 1);
     } else {
       for (int i = 0; i < NPB; ++i) { mbar_init(bar(B_P_FULL + i), 1); mbar_init(bar(B_P_READY + i), 4); }
       mbar_init(bar(B_O_DONE), 1);
@@ -148,7 +174,10 @@ sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_q, const MlaParams p) {
     *abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == 0 && lane == 0 && rank == 0) prefetch_tmap(&tm_q);
+  if (warp == 0 && lane == 0) {
+    prefetch_tmap(&tm_c);
+    if (rank == 0) prefetch_tmap(&tm_q);
+  }
   if (warp == 1) {
     tmem_alloc(sbase + OFF_TMEM, TMEM_COLS);
     tmem_relinquish();
@@ -190,15 +219,15 @@ sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_q, const MlaParams p) {
         for (int i = 0; i < QS && i < q_issued; ++i) mbar_wait_drain(bar(B_QST_FULL + i), q_par[i]);
       }
     }
-  } else if (warp == 2 || warp == 3 || warp == 8 || warp == 9) {
-    // ===================================================================== gathers (cp.async)
-    const int gw = (warp == 2) ? 0 : (warp == 3) ? 1 : (warp == 8) ? 2 : 3;
-    const int gi = gw * 32 + lane;
-    const int u = gi & 7, rb = gi >> 3;                   // 16-byte unit within a 128-byte row; first row
-    const uint32_t swz = static_cast<uint32_t>((u ^ (rb & 7)) << 4);
+  } else if (warp == 2 || warp == 3 || warp >= 8) {
+    // ===================================================================== gathers (TMA gather4)
+    // warp gw issues the stages of chunks n with n % 8 == gw; lane L < 16 gathers rows 4L .. 4L+3
+    const int gw = (warp < 8) ? warp - 2 : warp - 6;
     const int nch = (rank == 0) ? QCHUNKS : VCHUNKS;
-    const char* cbytes = reinterpret_cast<const char*>(p.c);
-    long long n = 0;
+    RingPos rp;
+    rp.size = nsr;
+    long long n = 0, n_last = -1;     // n_last: the last chunk this warp issued
+    RingPos last;                      // its ring position
     int ti = 0;
     bool ok = true;
     for (int t = cluster; t < p.T && ok; t += nclusters, ++ti) {
@@ -207,79 +236,116 @@ sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_q, const MlaParams p) {
       const int* ids = idx_s + is * KMAX;
       const long long base = p.row_off ? p.row_off[t] : 0;
       for (int j = 0; j < ntiles && ok; ++j) {
-        const char* src[4];
-#pragma unroll
-        for (int m = 0; m < 4; ++m)
-          src[m] = cbytes + mla_row(ids[j * NK + rb + 16 * m], base, p.S) * (D * 2) + u * 16;
-        for (int c = 0; c < nch; ++c, ++n) {
-          const int st = static_cast<int>(n % nsr);
-          if (!(ok = warp_wait(bar(B_RING_EMPTY + st), static_cast<uint32_t>((n / nsr) & 1) ^ 1, abort_flag)))
-            break;
-          const uint32_t dst = ring + st * CHUNK_BYTES + swz;
-#pragma unroll
-          for (int m = 0; m < 4; ++m) cp_async16(dst + (rb + 16 * m) * 128, src[m] + c * 128);
-          cp_async_commit();
-          if (n >= GD) {
-            cp_async_wait<GD>();
-            fence_proxy_async_smem();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(bar(B_RING_FULL + static_cast<int>((n - GD) % nsr)));
+        int r[4] = {0, 0, 0, 0};
+        if (lane < 16) {
+          const int4 e = reinterpret_cast<const int4*>(ids + j * NK)[lane];
+          r[0] = static_cast<int>(mla_row(e.x, base, p.S));
+          r[1] = static_cast<int>(mla_row(e.y, base, p.S));
+          r[2] = static_cast<int>(mla_row(e.z, base, p.S));
+          r[3] = static_cast<int>(mla_row(e.w, base, p.S));
+        }
+        for (int c = 0; c < nch; ++c, ++n, rp.advance()) {
+          if ((n & (GATHER_WARPS - 1)) != gw) continue;
+          const int st = rp.stage;
+          bool got = true;
+          if (lane == 0) {
+            got = mbar_wait(bar(B_RING_EMPTY + st), rp.phase ^ 1, abort_flag);
+            if (got) mbar_arrive_expect_tx(bar(B_RING_FULL + st), CHUNK_BYTES);
           }
+          if (!(ok = __shfl_sync(0xffffffffu, got, 0))) break;
+          if (lane == 0 && c == 0) DSA_TRACE_EVENT(rank == 0 ? 0 : 16, n / nch);
+          if (lane < 16)
+            tma_gather4(ring + st * CHUNK_BYTES + lane * 512, &tm_c, bar(B_RING_FULL + st), 64 * c, r[0], r[1], r[2],
+                        r[3]);
+          if (lane == 0 && rank == 0) DSA_TRACE_EVENT(8, n);
+          n_last = n;
+          last = rp;
         }
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(bar(B_IDX_EMPTY + is));
     }
-    // the last GD chunks: wait for them, fence, hand them over
-    cp_async_wait<0>();
-    fence_proxy_async_smem();
-    __syncwarp();
-    if (lane == 0 && !*abort_flag)
-      for (long long i = (n > GD ? n - GD : 0); i < n; ++i) mbar_arrive(bar(B_RING_FULL + static_cast<int>(i % nsr)));
+    if (lane == 0 && *abort_flag && n_last >= 0) {
+      // leave no gather in flight into this CTA's shared memory: bounded waits on this warp's loads of the last
+      // pass over the ring (stages below its last stage in that pass' parity, the others one pass earlier)
+      for (int st = 0; st < nsr; ++st)
+        mbar_wait_drain(bar(B_RING_FULL + st), st <= last.stage ? last.phase : last.phase ^ 1);
+    }
   } else if (warp == 1) {
     // ===================================================================== MMA issue
     if (lane == 0) {
       bool ok = true;
-      long long g = 0, n = 0;
+      int g = 0;
+      RingPos rp;
+      rp.size = nsr;
       int ti = 0;
       if (rank == 0) {
         constexpr uint32_t idesc = idesc_bf16(128, NK, false);
-        int qn = 0;
-        // Q chunk c of the next staged token -> tensor memory columns TQ + 32c .. +31
-        auto load_q = [&](int c) -> bool {
+        int qn = 0;          // Q chunks copied into tensor memory so far (= 9 * token index + chunk)
+        // copy the next staged Q chunk (global chunk index qn) into its tensor-memory slot
+        auto copy_q = [&]() -> bool {
           const int qs = qn % QS;
           if (!mbar_wait(bar(B_QST_FULL + qs), (qn / QS) & 1, abort_flag)) return false;
           tc_fence_after();
           const uint32_t src = sbase + OFF_QST + qs * QCHUNK_BYTES;
+          const uint32_t dst = tmem + TQ + 32 * (qn % QSLOTS);
 #pragma unroll
-          for (int s = 0; s < 4; ++s)
-            tmem_cp_128x256b(tmem + TQ + 32 * c + 8 * s, smem_desc(src + 32 * s, 16, 1024, kLayoutSW128));
+          for (int s = 0; s < 4; ++s) tmem_cp_128x256b(dst + 8 * s, smem_desc(src + 32 * s, 16, 1024, kLayoutSW128));
           mma_commit(bar(B_QST_EMPTY + qs));
           ++qn;
           return true;
         };
+        int nret = 0;        // tokens whose last tile committed the QRET barriers
         if (cluster < p.T)
-          for (int c = 0; c < QCHUNKS && ok; ++c) ok = load_q(c);
+          for (int c = 0; c < QCHUNKS && ok; ++c) ok = copy_q();
         for (int t = cluster; t < p.T && ok; t += nclusters, ++ti) {
           const bool has_next = t + nclusters < p.T;
+          const uint32_t prev_tok = static_cast<uint32_t>((ti - 1) & 1);   // parity of the previous token's QTOK
           for (int j = 0; j < ntiles && ok; ++j, ++g) {
-            const int sb = static_cast<int>(g % NSB);
+            const int sb = g % NSB;
+            if (j == 1 && has_next) {
+              // next token's chunks 0..2 go to the slots of the previous token's chunks 6..8
+              if (ti > 0 && !(ok = mbar_wait(bar(B_QTOK), prev_tok, abort_flag))) break;
+              for (int c = 0; c < 3 && ok; ++c) ok = copy_q();
+              if (!ok) break;
+            }
             if (!(ok = mbar_wait(bar(B_S_EMPTY + sb), static_cast<uint32_t>((g / NSB) & 1) ^ 1, abort_flag))) break;
+            DSA_TRACE_EVENT(2, g);
             tc_fence_after();
-            for (int c = 0; c < QCHUNKS; ++c, ++n) {
-              const int st = static_cast<int>(n % nsr);
-              if (!(ok = mbar_wait(bar(B_RING_FULL + st), static_cast<uint32_t>((n / nsr) & 1), abort_flag))) break;
+            const bool last = (j == ntiles - 1) && has_next;
+            for (int c = 0; c < QCHUNKS; ++c, rp.advance()) {
+              if (j == 0 && c >= 6 && ti > 0) {
+                // this token's chunks 6..8 go to the slots of the previous token's chunks 3..5
+                if (c == 6 && !(ok = mbar_wait(bar(B_QTOK), prev_tok, abort_flag))) break;
+                if (!(ok = copy_q())) break;
+              }
+              const int st = rp.stage;
+              DSA_TRACE_EVENT(10, g * QCHUNKS + c);
+              if (!(ok = mbar_wait(bar(B_RING_FULL + st), rp.phase, abort_flag))) break;
+              DSA_TRACE_EVENT(9, g * QCHUNKS + c);
               tc_fence_after();
               const uint64_t bd = smem_desc(ring + st * CHUNK_BYTES, 16, 1024, kLayoutSW128);
+              const uint32_t a = tmem + TQ + 32 * ((9 * ti + c) % QSLOTS);
 #pragma unroll
               for (int s = 0; s < 4; ++s)     // K = 16 bf16 per instruction: 8 TMEM columns of A, 32 bytes of B
-                mma_bf16_ts(tmem + TS + NK * sb, tmem + TQ + 32 * c + 8 * s, bd + 2 * s, idesc, (c | s) ? 1u : 0u);
+                mma_bf16_ts(tmem + TS + NK * sb, a + 8 * s, bd + 2 * s, idesc, (c | s) ? 1u : 0u);
               mma_commit(bar(B_RING_EMPTY + st));
-              if (j == ntiles - 1 && has_next && !(ok = load_q(c))) break;
+              DSA_TRACE_EVENT(11, g * QCHUNKS + c);
+              if (last) {
+                if (c < 3) mma_commit(bar(B_QRET + c));
+                if (c >= 3 && c < 6) {
+                  // next token's chunk c overwrites this token's chunk c - 3, committed three chunks ago
+                  if (!(ok = mbar_wait(bar(B_QRET + c - 3), static_cast<uint32_t>(nret & 1), abort_flag))) break;
+                  if (!(ok = copy_q())) break;
+                }
+              }
             }
             if (!ok) break;
+            if (last) ++nret;
+            DSA_TRACE_EVENT(3, g);
             mma_commit(bar(B_S_FULL + sb));
           }
+          mma_commit(bar(B_QTOK));
         }
       } else {
         constexpr uint32_t idesc = idesc_bf16(128, 256, true);
@@ -288,23 +354,28 @@ sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_q, const MlaParams p) {
             const int pb = static_cast<int>(g % NPB);
             if (j == 0 && !(ok = mbar_wait(bar(B_O_FREE), (ti & 1) ^ 1, abort_flag))) break;
             if (!(ok = mbar_wait(bar(B_P_READY + pb), static_cast<uint32_t>((g / NPB) & 1), abort_flag))) break;
+            DSA_TRACE_EVENT(20, g);
             tc_fence_after();
             const uint64_t ad = smem_desc(sbase + OFF_PB + pb * XFER, 16, 1024, kLayoutSW128);
             for (int hh = 0; hh < 2 && ok; ++hh) {
-              const int st0 = static_cast<int>(n % nsr);
-              for (int q = 0; q < 4 && ok; ++q)
-                ok = mbar_wait(bar(B_RING_FULL + st0 + q), static_cast<uint32_t>(((n + q) / nsr) & 1), abort_flag);
+              const int st0 = rp.stage;          // four consecutive stages (the ring size is a multiple of 4)
+              const uint32_t ph0 = rp.phase;
+              for (int q = 0; q < 4 && ok; ++q) ok = mbar_wait(bar(B_RING_FULL + st0 + q), ph0, abort_flag);
               if (!ok) break;
+              DSA_TRACE_EVENT(21 + hh, g);
               tc_fence_after();
               // MN-major V: 64-dim chunks 8 KB apart (LBO), 8-key row groups 1 KB apart (SBO)
               const uint64_t bd = smem_desc(ring + st0 * CHUNK_BYTES, CHUNK_BYTES, 1024, kLayoutSW128);
 #pragma unroll
               for (int s = 0; s < 4; ++s)     // 16 keys per instruction: two 8-key groups = 2 KB of V
                 mma_bf16_ss(tmem + 256 * hh, ad + 2 * s, bd + ((s * 2048) >> 4), idesc, (j == 0 && s == 0) ? 0u : 1u);
-              for (int q = 0; q < 4; ++q) mma_commit(bar(B_RING_EMPTY + st0 + q));
-              n += 4;
+              for (int q = 0; q < 4; ++q) {
+                mma_commit(bar(B_RING_EMPTY + st0 + q));
+                rp.advance();
+              }
             }
             if (!ok) break;
+            DSA_TRACE_EVENT(23, g);
             mma_commit_mc(bar(B_P_EMPTY + pb), 0x1);   // P buffer pb free again (score CTA waits on it)
             mma_commit(bar(B_O_DONE));
           }
@@ -319,7 +390,7 @@ sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_q, const MlaParams p) {
     const uint32_t lane_addr = static_cast<uint32_t>(quad * 32) << 16;
     const uint32_t pb_remote = map_cluster(sbase + OFF_PB, 1);
     const uint32_t pfull_remote = map_cluster(bar(B_P_FULL), 1);
-    long long g = 0;
+    int g = 0;
     int ti = 0;
     bool ok = true;
     for (int t = cluster; t < p.T && ok; t += nclusters, ++ti) {
@@ -336,6 +407,7 @@ sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_q, const MlaParams p) {
         const uint32_t m_even = __ballot_sync(0xffffffffu, mla_valid(e.x, base, p.S));
         const uint32_t m_odd = __ballot_sync(0xffffffffu, mla_valid(e.y, base, p.S));
         if (!(ok = warp_wait(bar(B_S_FULL + sb), static_cast<uint32_t>((g / NSB) & 1), abort_flag))) break;
+        if (leader) DSA_TRACE_EVENT(4, g);
         tc_fence_after();
         uint32_t v[64];
         {
@@ -348,14 +420,22 @@ sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_q, const MlaParams p) {
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(bar(B_S_EMPTY + sb));
-        float mt = -INFINITY;
+        // running max over the valid keys of the tile (raw logits; the scale is positive), as a 4-way tree
+        const bool full_tile = (m_even & m_odd) == 0xffffffffu;
+        float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+        if (full_tile) {
 #pragma unroll
-        for (int i = 0; i < NK; ++i) {
-          const bool valid = ((i & 1) ? (m_odd >> (i >> 1)) : (m_even >> (i >> 1))) & 1u;
-          const float x = valid ? __uint_as_float(v[i]) * p.scale_log2 : -INFINITY;
-          v[i] = __float_as_uint(x);
-          mt = fmaxf(mt, x);
+          for (int i = 0; i < NK; ++i) mx[i & 3] = fmaxf(mx[i & 3], __uint_as_float(v[i]));
+        } else {
+#pragma unroll
+          for (int i = 0; i < NK; ++i) {
+            const bool valid = ((i & 1) ? (m_odd >> (i >> 1)) : (m_even >> (i >> 1))) & 1u;
+            if (!valid) v[i] = __float_as_uint(-INFINITY);
+            mx[i & 3] = fmaxf(mx[i & 3], __uint_as_float(v[i]));
+          }
         }
+        const float mraw = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
+        const float mt = (mraw == -INFINITY) ? -INFINITY : mraw * p.scale_log2;
         float alpha = 1.f;
         if (mt > m_ref + RESCALE_LOG2) {
           alpha = (m_ref == -INFINITY) ? 0.f : ex2_approx(m_ref - mt);
@@ -363,23 +443,28 @@ sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_q, const MlaParams p) {
           le *= alpha;
           m_ref = mt;
         }
+        // p = 2^(x * scale_log2 - m_ref) as one FMA + ex2; masked keys (-inf) give 0
+        const float neg_m = (m_ref == -INFINITY) ? 0.f : -m_ref;
         uint32_t pk[NK / 2];
-        float ls = 0.f, lx = 0.f;
+        float ls0 = 0.f, ls1 = 0.f, lx0 = 0.f, lx1 = 0.f;
 #pragma unroll
         for (int i = 0; i < NK / 2; ++i) {
-          const float x0 = __uint_as_float(v[2 * i]), x1 = __uint_as_float(v[2 * i + 1]);
-          const float p0 = (x0 == -INFINITY) ? 0.f : ex2_approx(x0 - m_ref);
-          const float p1 = (x1 == -INFINITY) ? 0.f : ex2_approx(x1 - m_ref);
+          const float p0 = ex2_approx(fmaf(__uint_as_float(v[2 * i]), p.scale_log2, neg_m));
+          const float p1 = ex2_approx(fmaf(__uint_as_float(v[2 * i + 1]), p.scale_log2, neg_m));
           const __nv_bfloat162 bb = __floats2bfloat162_rn(p0, p1);
-          ls += __low2float(bb) + __high2float(bb);
-          lx += p0 + p1;
+          ls0 += __low2float(bb);
+          ls1 += __high2float(bb);
+          lx0 += p0;
+          lx1 += p1;
           pk[i] = *reinterpret_cast<const uint32_t*>(&bb);
         }
+        const float ls = ls0 + ls1, lx = lx0 + lx1;
         l += ls;
         le += lx;
         // staging slot b was last read by the bulk copy of tile g - 2: the leader waits for that copy to
         // have read its source, then releases the slot to the four softmax warps
         if (leader) {
+          DSA_TRACE_EVENT(5, g);
           bulk_wait_read<1>();
           mbar_arrive(bar(B_SLOT_FREE));
         }
@@ -406,6 +491,7 @@ sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_q, const MlaParams p) {
           ok = mbar_wait(bar(B_SLOT_WRITTEN), static_cast<uint32_t>(g & 1), abort_flag) &&
                mbar_wait<true>(bar(B_P_EMPTY + pb), static_cast<uint32_t>((g / NPB) & 1) ^ 1, abort_flag);
           if (ok) {
+            DSA_TRACE_EVENT(7, g);
             mbar_arrive_expect_tx_remote(pfull_remote + 8 * pb, XFER);
             bulk_copy_to_peer(pb_remote + pb * XFER, sbase + OFF_PST + b * XFER, XFER, pfull_remote + 8 * pb);
             bulk_commit();
@@ -422,7 +508,7 @@ sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_q, const MlaParams p) {
     const int quad = warp & 3;
     const int h = quad * 32 + lane;
     const uint32_t lane_addr = static_cast<uint32_t>(quad * 32) << 16;
-    long long g = 0;
+    int g = 0;
     int ti = 0;
     bool ok = true;
     for (int t = cluster; t < p.T && ok; t += nclusters, ++ti) {
@@ -430,6 +516,7 @@ sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_q, const MlaParams p) {
       for (int j = 0; j < ntiles; ++j, ++g) {
         const int pb = static_cast<int>(g % NPB);
         if (!(ok = warp_wait<true>(bar(B_P_FULL + pb), static_cast<uint32_t>((g / NPB) & 1), abort_flag))) break;
+        if (warp == 4 && lane == 0) DSA_TRACE_EVENT(18, g);
         const uint8_t* xb = smem + OFF_PB + pb * XFER;
         const float a = reinterpret_cast<const float*>(xb + P_BYTES)[h];
         if (j == ntiles - 1) l = reinterpret_cast<const float*>(xb + P_BYTES + 512)[h];

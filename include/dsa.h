@@ -157,6 +157,31 @@ DSA_API dsa_status_t dsa_forward_decode(int B, const int64_t* cache_off, const i
                                 int H, int k, float scale, int32_t* idx_out, uint16_t* out, float* lse, void* ws,
                                 size_t ws_bytes, void* stream);
 
+/*
+ * dsa_forward_decode without a caller-provided workspace, for callers that cannot allocate device memory
+ * (for example a serving loop that runs under a memory pool it may not grow, or code that only receives
+ * borrowed buffers).  This entry point has no counterpart in the paper: it is the decode step above with its
+ * scratch (per-cache-row scores, per-sequence lengths and, when idx_out is NULL, the selected indices) held
+ * in a fixed device array inside the library, of dsa_decode_noalloc_scratch_bytes() bytes (32 MiB).  Every
+ * GPU that loads the library keeps that array until the process exits.
+ *   - Arguments and results are those of dsa_forward_decode; shapes whose dsa_decode_workspace_size()
+ *     exceeds the array return DSA_ERR_WORKSPACE and launch nothing.
+ *   - The call allocates nothing: no cudaMalloc, no cudaFree, no allocating library routine.
+ *   - The first call on a device looks up the array's device address (cudaGetSymbolAddress) with that device
+ *     current; make that first call before any stream capture on the device.
+ *   - All calls share the one array and it keeps the last call's contents: calls that may overlap on the GPU
+ *     (different streams, or graph replays in flight together) race on it and must be serialised by the
+ *     caller.
+ */
+DSA_API size_t dsa_decode_noalloc_scratch_bytes(void);
+DSA_API dsa_status_t dsa_forward_decode_noalloc(int B, const int64_t* cache_off, const int32_t* ctx_len,
+                                                const uint8_t* q_idx, const float* q_scale, const float* w,
+                                                const uint16_t* q, const uint8_t* k_new, const float* k_scale_new,
+                                                const uint16_t* c_new, uint8_t* k_cache, float* k_scale_cache,
+                                                uint16_t* c_cache, int64_t cache_rows, int H_I, int d_I, int H,
+                                                int k, float scale, int32_t* idx_out, uint16_t* out, float* lse,
+                                                void* stream);
+
 #ifdef __cplusplus
 }
 #endif

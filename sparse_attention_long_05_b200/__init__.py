@@ -5,7 +5,9 @@ The computation lives in libdsa.so (hand-written CUDA, C ABI in include/dsa.h); 
 """
 from ._lib import (  # noqa: F401
     DsaError,
+    dsa_decode_noalloc_scratch_bytes,
     dsa_decode_workspace_size,
+    dsa_forward_decode_noalloc,
     dsa_forward_decode,
     dsa_forward_prefill,
     dsa_get_device_status,

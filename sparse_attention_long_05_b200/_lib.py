@@ -34,6 +34,9 @@ SIGNATURES = {
     "dsa_decode_workspace_size": (_SZ, [_I, _I64, _I, _I, _I, _I]),
     "dsa_forward_decode": (_I, [_I, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _I64, _I, _I, _I, _I, _F,
                                 _P, _P, _P, _P, _SZ, _P]),
+    "dsa_decode_noalloc_scratch_bytes": (_SZ, []),
+    "dsa_forward_decode_noalloc": (_I, [_I, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _I64, _I, _I, _I, _I,
+                                        _F, _P, _P, _P, _P]),
 }
 
 
@@ -189,4 +192,30 @@ def dsa_forward_decode(cache_off, ctx_len, q_idx, q_scale, w, q, k_new, k_scale_
         B, _ptr(cache_off), _ptr(ctx_len), _ptr(q_idx), _ptr(q_scale), _ptr(w), _ptr(q), _ptr(k_new),
         _ptr(k_scale_new), _ptr(c_new), _ptr(k_cache), _ptr(k_scale_cache), _ptr(c_cache), rows, H_I, d_I, H, k,
         float(scale), _ptr(idx_out), _ptr(out), _ptr(lse), _ptr(ws), ws.numel(), _stream(stream)))
+    return idx_out, out, lse
+
+
+def dsa_decode_noalloc_scratch_bytes() -> int:
+    return int(_lib.dsa_decode_noalloc_scratch_bytes())
+
+
+def dsa_forward_decode_noalloc(cache_off, ctx_len, q_idx, q_scale, w, q, k_new, k_scale_new, c_new, k_cache,
+                               k_scale_cache, c_cache, k: int, scale: float, idx_out=None, out=None, lse=None,
+                               stream=None):
+    """dsa_forward_decode with the library's fixed scratch array instead of a workspace (allocates nothing
+    on the device beyond the outputs this wrapper creates when none are passed)."""
+    B, H_I, d_I = q_idx.shape
+    H = q.shape[1]
+    rows = k_cache.shape[0]
+    dev = q.device
+    if idx_out is None:
+        idx_out = torch.empty((B, k), dtype=torch.int32, device=dev)
+    if out is None:
+        out = torch.empty((B, H, 512), dtype=torch.bfloat16, device=dev)
+    if lse is None:
+        lse = torch.empty((B, H), dtype=torch.float32, device=dev)
+    _check("dsa_forward_decode_noalloc", _lib.dsa_forward_decode_noalloc(
+        B, _ptr(cache_off), _ptr(ctx_len), _ptr(q_idx), _ptr(q_scale), _ptr(w), _ptr(q), _ptr(k_new),
+        _ptr(k_scale_new), _ptr(c_new), _ptr(k_cache), _ptr(k_scale_cache), _ptr(c_cache), rows, H_I, d_I, H, k,
+        float(scale), _ptr(idx_out), _ptr(out), _ptr(lse), _stream(stream)))
     return idx_out, out, lse

@@ -363,4 +363,49 @@ dsa_status_t dsa_forward_decode(int B, const int64_t* cache_off, const int32_t* 
   return run_mla(q, c_cache, cache_rows, idx, off, B, H, k, scale, out, lse, st);
 }
 
+// ------------------------------------------------------------------------------------------ no-allocation decode
+// Scratch of dsa_forward_decode_noalloc: a file-scope device array, so the call needs no workspace from the
+// caller.  Every GPU that loads the library holds it until the process exits.
+static constexpr size_t kNoAllocScratchBytes = size_t(32) << 20;
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+namespace {
+// device address of g_noalloc_scratch on each device, looked up once per device with that device current
+// (host code may not use the array's name as a device address)
+constexpr int kMaxDevices = 64;
+void* g_noalloc_ptr[kMaxDevices] = {};
+std::mutex g_noalloc_mutex;
+
+dsa_status_t noalloc_scratch(void** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return DSA_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+  if (!g_noalloc_ptr[dev]) {
+    void* ptr = nullptr;
+    if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess || !ptr) return DSA_ERR_CUDA;
+    g_noalloc_ptr[dev] = ptr;
+  }
+  *out = g_noalloc_ptr[dev];
+  return DSA_OK;
+}
+}  // namespace
+
+size_t dsa_decode_noalloc_scratch_bytes(void) { return kNoAllocScratchBytes; }
+
+dsa_status_t dsa_forward_decode_noalloc(int B, const int64_t* cache_off, const int32_t* ctx_len,
+                                        const uint8_t* q_idx, const float* q_scale, const float* w,
+                                        const uint16_t* q, const uint8_t* k_new, const float* k_scale_new,
+                                        const uint16_t* c_new, uint8_t* k_cache, float* k_scale_cache,
+                                        uint16_t* c_cache, int64_t cache_rows, int H_I, int d_I, int H, int k,
+                                        float scale, int32_t* idx_out, uint16_t* out, float* lse, void* stream) {
+  if (dsa_decode_workspace_size(B, cache_rows, H_I, d_I, H, k) > kNoAllocScratchBytes) return DSA_ERR_WORKSPACE;
+  void* scratch = nullptr;
+  const dsa_status_t e = noalloc_scratch(&scratch);
+  if (e != DSA_OK) return e;
+  // the scratch needs no clearing: every byte a call reads there is written earlier in the same call
+  return dsa_forward_decode(B, cache_off, ctx_len, q_idx, q_scale, w, q, k_new, k_scale_new, c_new, k_cache,
+                            k_scale_cache, c_cache, cache_rows, H_I, d_I, H, k, scale, idx_out, out, lse, scratch,
+                            kNoAllocScratchBytes, stream);
+}
+
 }  // extern "C"

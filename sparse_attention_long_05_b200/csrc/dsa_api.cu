@@ -149,7 +149,8 @@ dsa_status_t run_topk(const float* scores, long long ld, const long long* row_of
                       int rows, int k, int* idx, long long idx_ld, cudaStream_t st) {
   if (rows <= 0) return DSA_OK;
   TopkParams p{scores, ld, row_off, row_len, pos0, rows, k, idx, idx_ld};
-  topk_rows_kernel<<<rows, kTopkThreads, 0, st>>>(p);
+  if (set_smem(topk_rows_kernel, static_cast<int>(sizeof(TopkSmem))) != cudaSuccess) return DSA_ERR_CUDA;
+  topk_rows_kernel<<<rows, kTopkThreads, sizeof(TopkSmem), st>>>(p);
   return last_launch_status();
 }
 

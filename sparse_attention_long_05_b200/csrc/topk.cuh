@@ -1,14 +1,19 @@
 // Row-wise top-k selection (velog.io DSA page, §1.2 Fine-grained Token Selection) over materialised scores.
 //
-// One CTA per row.  Scores are mapped to monotone uint32 order keys (order_key), and the k-th largest key
-// T is found exactly by a 4-pass most-significant-digit radix select (8-bit digits, per-warp shared-memory
-// histograms, one warp scanning the 256 bins).  The selected set is then {key > T} plus the first
-// `need` entries with key == T in ascending column order, which is exactly "score descending, smaller
-// column first on ties".  A final ordered compaction writes the selected columns in ascending order: each
-// warp owns a contiguous segment of the row, a counting pass gives every warp its output offset and its
-// rank among the key == T entries, and a writing pass places the entries with warp ballots.
-// Rows with n <= k select every column.  Nothing but the histograms lives in shared memory, so rows of any
-// length (up to 2^31) are handled; the row is streamed from global memory (L2) six times.
+// One CTA per row.  Scores are mapped to monotone uint32 order keys (order_key); the selected set is
+// {key > T} plus the first `need` entries with key == T in ascending column order, T being the exact key of
+// the k-th largest entry, which is "score descending, smaller column first on ties".  Rows with n <= k select
+// every column.
+//
+// Fast path (two passes over the row): a 2048-bin histogram of the top 11 key bits gives the bin b* that
+// holds the k-th largest key; a second pass appends every entry with bin >= b* (k entries plus the rest of
+// bin b*) to shared memory, each warp owning a contiguous segment of the row and its own region, so the
+// candidates stay in column order.  The exact threshold within bin b* (a 3-pass radix select on the low 21
+// bits over the candidates) and the ordered output then run in shared memory only.
+//
+// Fallback (when a warp's region would overflow, e.g. on massive ties or on rows sorted by score): a 4-pass
+// most-significant-digit radix select over the row (8-bit digits, per-warp histograms) and an ordered
+// compaction with warp ballots, streaming the row six times.  Both paths give identical results.
 #pragma once
 #include "common.cuh"
 
@@ -28,12 +33,77 @@ struct TopkParams {
 
 constexpr int kTopkThreads = 512;
 constexpr int kTopkWarps = kTopkThreads / 32;
+constexpr int kTopkBins = 2048;            // top 11 key bits
+constexpr int kTopkRegion = 384;           // candidates per warp region (fast path)
+
+struct TopkSmem {
+  uint32_t hist[kTopkWarps][256];          // fallback: per-warp histograms
+  uint32_t bins[kTopkBins];                // fast path: top-11-bit histogram
+  uint32_t cand_key[kTopkWarps][kTopkRegion];
+  int cand_idx[kTopkWarps][kTopkRegion];
+  int region_n[kTopkWarps];
+  uint32_t s_need, s_digit, s_bin, s_overflow;
+  int s_gt[kTopkWarps], s_eq[kTopkWarps];
+  int s_out_base[kTopkWarps], s_eq_base[kTopkWarps];
+};
+
+// Radix select on 32-bit keys among the entries of `get(i)`, i < n, that match (key & mask) == prefix:
+// returns the exact k-th largest key and sets `need` to the number of entries equal to it that are taken.
+// hist is a [kTopkWarps][256] shared scratch; every thread of the CTA calls this.
+template <typename Get>
+__device__ __forceinline__ uint32_t radix_select(Get get, int n, uint32_t prefix, uint32_t mask, int first_shift,
+                                                 uint32_t& need, TopkSmem& sm) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  for (int shift = first_shift; shift >= 0; shift -= 8) {
+    for (int i = lane; i < 256; i += 32) sm.hist[warp][i] = 0;
+    __syncthreads();
+    for (int i = tid; i < n; i += kTopkThreads) {
+      const uint32_t key = get(i);
+      if ((key & mask) == prefix) atomicAdd(&sm.hist[warp][(key >> shift) & 255], 1u);
+    }
+    __syncthreads();
+    if (warp == 0) {
+      // lane l owns bins 255-8l .. 248-8l (descending); totals over warps
+      uint32_t cnt[8];
+      uint32_t tot = 0;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const int bin = 255 - 8 * lane - j;
+        uint32_t c = 0;
+        for (int w = 0; w < kTopkWarps; ++w) c += sm.hist[w][bin];
+        cnt[j] = c;
+        tot += c;
+      }
+      uint32_t incl = tot;
+#pragma unroll
+      for (int d = 1; d < 32; d <<= 1) {
+        const uint32_t v = __shfl_up_sync(0xffffffffu, incl, d);
+        if (lane >= d) incl += v;
+      }
+      const uint32_t excl = incl - tot;
+      if (excl < need && need <= incl) {
+        uint32_t run = excl;
+        int j = 0;
+        for (; j < 8; ++j) {
+          if (run + cnt[j] >= need) break;
+          run += cnt[j];
+        }
+        sm.s_digit = static_cast<uint32_t>(255 - 8 * lane - j);
+        sm.s_need = need - run;
+      }
+    }
+    __syncthreads();
+    prefix |= sm.s_digit << shift;
+    mask |= 255u << shift;
+    need = sm.s_need;
+    __syncthreads();
+  }
+  return prefix;
+}
 
 __global__ void __launch_bounds__(kTopkThreads) topk_rows_kernel(const TopkParams p) {
-  __shared__ uint32_t hist[kTopkWarps][256];
-  __shared__ uint32_t s_need, s_digit;
-  __shared__ int s_gt[kTopkWarps], s_eq[kTopkWarps];
-  __shared__ int s_out_base[kTopkWarps], s_eq_base[kTopkWarps];
+  extern __shared__ __align__(16) uint8_t topk_smem_raw[];
+  TopkSmem& sm = *reinterpret_cast<TopkSmem*>(topk_smem_raw);
 
   const int r = blockIdx.x;
   if (r >= p.rows) return;
@@ -50,67 +120,96 @@ __global__ void __launch_bounds__(kTopkThreads) topk_rows_kernel(const TopkParam
     for (int i = tid; i < k; i += kTopkThreads) out[i] = (i < n) ? i : -1;
     return;
   }
-
-  // ---------------------------------------------------------------- radix select of the k-th largest key
-  uint32_t prefix = 0, mask = 0, need = static_cast<uint32_t>(k);
-  for (int pass = 0; pass < 4; ++pass) {
-    const int shift = 24 - 8 * pass;
-    for (int i = lane; i < 256; i += 32) hist[warp][i] = 0;
-    __syncthreads();
-    for (int i = tid; i < n; i += kTopkThreads) {
-      const uint32_t key = order_key(x[i]);
-      if ((key & mask) == prefix) atomicAdd(&hist[warp][(key >> shift) & 255], 1u);
-    }
-    __syncthreads();
-    if (warp == 0) {
-      // lane l owns bins 255-8l .. 248-8l (descending); totals over warps
-      uint32_t cnt[8];
-      uint32_t tot = 0;
-#pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        const int bin = 255 - 8 * lane - j;
-        uint32_t c = 0;
-        for (int w = 0; w < kTopkWarps; ++w) c += hist[w][bin];
-        cnt[j] = c;
-        tot += c;
-      }
-      // inclusive scan of lane totals (descending bin order)
-      uint32_t incl = tot;
-#pragma unroll
-      for (int d = 1; d < 32; d <<= 1) {
-        const uint32_t v = __shfl_up_sync(0xffffffffu, incl, d);
-        if (lane >= d) incl += v;
-      }
-      const uint32_t excl = incl - tot;
-      // the lane whose range holds the need-th largest key
-      const bool mine = excl < need && need <= incl;
-      const uint32_t who = __ballot_sync(0xffffffffu, mine);
-      if (mine) {
-        uint32_t run = excl;
-        int j = 0;
-        for (; j < 8; ++j) {
-          if (run + cnt[j] >= need) break;
-          run += cnt[j];
-        }
-        s_digit = static_cast<uint32_t>(255 - 8 * lane - j);
-        s_need = need - run;
-      }
-      (void)who;
-    }
-    __syncthreads();
-    prefix |= s_digit << shift;
-    mask |= 255u << shift;
-    need = s_need;
-    __syncthreads();
-  }
-  const uint32_t T = prefix;   // exact key of the k-th largest entry; `need` entries equal to T are taken
-
-  // ---------------------------------------------------------------- ordered compaction
   const int seg = (n + kTopkWarps - 1) / kTopkWarps;
   const int seg0 = min(n, warp * seg), seg1 = min(n, seg0 + seg);
+
+  // ---------------------------------------------------------------- fast path, pass 1: top-11-bit histogram
+  for (int i = tid; i < kTopkBins; i += kTopkThreads) sm.bins[i] = 0;
+  if (tid == 0) sm.s_overflow = 0;
+  __syncthreads();
+  for (int i = tid; i < n; i += kTopkThreads) atomicAdd(&sm.bins[order_key(x[i]) >> 21], 1u);
+  __syncthreads();
+  // bin b* holding the k-th largest key: thread t owns bins 2047-4t .. 2044-4t (descending order)
+  {
+    uint32_t c4[4], tot = 0;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) { c4[j] = sm.bins[kTopkBins - 1 - 4 * tid - j]; tot += c4[j]; }
+    uint32_t incl = tot;
+#pragma unroll
+    for (int d = 1; d < 32; d <<= 1) {
+      const uint32_t v = __shfl_up_sync(0xffffffffu, incl, d);
+      if (lane >= d) incl += v;
+    }
+    if (lane == 31) sm.s_gt[warp] = static_cast<int>(incl);
+    __syncthreads();
+    uint32_t wbase = 0;
+    for (int w = 0; w < warp; ++w) wbase += static_cast<uint32_t>(sm.s_gt[w]);
+    const uint32_t excl = wbase + incl - tot;
+    const uint32_t kk = static_cast<uint32_t>(k);
+    if (excl < kk && kk <= excl + tot) {
+      uint32_t run = excl;
+      int j = 0;
+      for (; j < 4; ++j) {
+        if (run + c4[j] >= kk) break;
+        run += c4[j];
+      }
+      sm.s_bin = static_cast<uint32_t>(kTopkBins - 1 - 4 * tid - j);
+      sm.s_need = kk - run;            // entries of bin b* still to take
+    }
+    __syncthreads();
+  }
+  const uint32_t bstar = sm.s_bin;
+  const uint32_t need_bin = sm.s_need;
+  // ---------------------------------------------------------------- pass 2: gather candidates in column order
+  {
+    int cnt = 0;
+    bool over = false;
+    for (int i0 = seg0; i0 < seg1; i0 += 32) {
+      const int i = i0 + lane;
+      const uint32_t key = (i < seg1) ? order_key(x[i]) : 0u;
+      const bool c = i < seg1 && (key >> 21) >= bstar;
+      const uint32_t m = __ballot_sync(0xffffffffu, c);
+      const int pos = cnt + __popc(m & ((1u << lane) - 1));
+      if (c && pos < kTopkRegion) {
+        sm.cand_key[warp][pos] = key;
+        sm.cand_idx[warp][pos] = i;
+      }
+      cnt += __popc(m);
+      if (cnt > kTopkRegion) over = true;
+    }
+    if (lane == 0) {
+      sm.region_n[warp] = min(cnt, kTopkRegion);
+      if (over) atomicOr(&sm.s_overflow, 1u);
+    }
+  }
+  __syncthreads();
+
+  uint32_t T, need;
+  bool from_row;          // fallback: the compaction streams the row instead of the candidates
+  if (!sm.s_overflow) {
+    // exact threshold inside bin b*, over the candidates (shared memory only)
+    need = need_bin;
+    const uint32_t pad = (bstar == kTopkBins - 1) ? 0u : 0xFFFFFFFFu;   // a key outside bin b*
+    auto get = [&](int i) -> uint32_t {
+      const int w = i / kTopkRegion, j = i % kTopkRegion;
+      return (j < sm.region_n[w]) ? sm.cand_key[w][j] : pad;
+    };
+    T = radix_select(get, kTopkWarps * kTopkRegion, bstar << 21, 0xFFE00000u, 16, need, sm);
+    from_row = false;
+  } else {
+    need = static_cast<uint32_t>(k);
+    auto get = [&](int i) -> uint32_t { return order_key(x[i]); };
+    T = radix_select(get, n, 0u, 0u, 24, need, sm);
+    from_row = true;
+  }
+  // ---------------------------------------------------------------- ordered compaction
+  // every warp walks its own span (a contiguous row segment, or its candidate region), in column order
+  const int span = from_row ? seg1 - seg0 : sm.region_n[warp];
+  auto key_at = [&](int j) -> uint32_t { return from_row ? order_key(x[seg0 + j]) : sm.cand_key[warp][j]; };
+  auto col_at = [&](int j) -> int { return from_row ? seg0 + j : sm.cand_idx[warp][j]; };
   int gt = 0, eq = 0;
-  for (int i = seg0 + lane; i < seg1; i += 32) {
-    const uint32_t key = order_key(x[i]);
+  for (int j = lane; j < span; j += 32) {
+    const uint32_t key = key_at(j);
     gt += key > T;
     eq += key == T;
   }
@@ -119,31 +218,31 @@ __global__ void __launch_bounds__(kTopkThreads) topk_rows_kernel(const TopkParam
     gt += __shfl_xor_sync(0xffffffffu, gt, d);
     eq += __shfl_xor_sync(0xffffffffu, eq, d);
   }
-  if (lane == 0) { s_gt[warp] = gt; s_eq[warp] = eq; }
+  if (lane == 0) { sm.s_gt[warp] = gt; sm.s_eq[warp] = eq; }
   __syncthreads();
   if (tid == 0) {
     int base = 0, eqb = 0;
     for (int w = 0; w < kTopkWarps; ++w) {
-      s_out_base[w] = base;
-      s_eq_base[w] = eqb;
-      const int take_eq = max(0, min(s_eq[w], static_cast<int>(need) - eqb));
-      base += s_gt[w] + take_eq;
-      eqb += s_eq[w];
+      sm.s_out_base[w] = base;
+      sm.s_eq_base[w] = eqb;
+      const int take_eq = max(0, min(sm.s_eq[w], static_cast<int>(need) - eqb));
+      base += sm.s_gt[w] + take_eq;
+      eqb += sm.s_eq[w];
     }
   }
   __syncthreads();
-  int pos = s_out_base[warp];
-  int eq_rank = s_eq_base[warp];
-  for (int i0 = seg0; i0 < seg1; i0 += 32) {
-    const int i = i0 + lane;
+  int pos = sm.s_out_base[warp];
+  int eq_rank = sm.s_eq_base[warp];
+  for (int j0 = 0; j0 < span; j0 += 32) {
+    const int j = j0 + lane;
     uint32_t key = 0;
-    if (i < seg1) key = order_key(x[i]);
-    const bool is_eq = i < seg1 && key == T;
+    if (j < span) key = key_at(j);
+    const bool is_eq = j < span && key == T;
     const uint32_t eq_mask = __ballot_sync(0xffffffffu, is_eq);
     const int my_eq_rank = eq_rank + __popc(eq_mask & ((1u << lane) - 1));
-    const bool sel = i < seg1 && (key > T || (is_eq && my_eq_rank < static_cast<int>(need)));
+    const bool sel = j < span && (key > T || (is_eq && my_eq_rank < static_cast<int>(need)));
     const uint32_t sel_mask = __ballot_sync(0xffffffffu, sel);
-    if (sel) out[pos + __popc(sel_mask & ((1u << lane) - 1))] = i;
+    if (sel) out[pos + __popc(sel_mask & ((1u << lane) - 1))] = col_at(j);
     pos += __popc(sel_mask);
     eq_rank += __popc(eq_mask);
   }

@@ -67,3 +67,13 @@ def test_integer_index_scores(dsa):
     w = rng.integers(-3, 4, size=(4, H_I)).astype(np.float64)
     sc = np.stack([O.indexer_scores_row(qi[r], w[r], ki) for r in range(4)])
     _check(dsa, sc, 2048, row_len=[n, n - 1, 5000, 2048])
+
+
+def test_rows_sorted_by_score_take_the_fallback_path(dsa):
+    """Ascending scores put every candidate in the last warps' segments, overflowing their shared-memory
+    regions, so the kernel switches to the multi-pass select; results must not change."""
+    n = 20000
+    asc = np.arange(n, dtype=np.float32)
+    desc = asc[::-1].copy()
+    blocks = np.repeat(np.arange(n // 100, dtype=np.float32), 100)    # 100-long runs of equal scores
+    _check(dsa, np.stack([asc, desc, blocks, -asc]), 2048, row_len=[n, n, n, n])

@@ -340,6 +340,27 @@ def bench_decode(dsa, cfg, steps, warmup, ws_n, rank, pk):
             "launches": launches}
 
 
+# ------------------------------------------------------------------------------------------ profiling cases
+def kernels_small(dsa):
+    """One launch each of the main kernels on small inputs (for ncu captures): sparse MLA over 1184 query
+    tokens of the 128K latent, indexer scores of a 2048-row block against 131072 keys, top-k of those rows."""
+    cfg = PREFILL
+    keys = G.prefill_keys(cfg, 5, device="cuda")
+    rows = range(cfg.L - 2048, cfg.L)
+    qs = G.prefill_queries(cfg, 5, rows=rows, device="cuda")
+    rng = np.random.default_rng(5)
+    T = 1184
+    idx = torch.from_numpy(np.sort(np.stack([rng.choice(cfg.L, cfg.k, replace=False) for _ in range(T)]), axis=1)
+                           .astype(np.int32)).cuda()
+    dsa.dsa_sparse_mla_attn(qs["q"][:T].contiguous(), keys["c"], idx, cfg.scale)
+    sc = dsa.dsa_indexer_scores(qs["q_idx"], qs["q_scale"], keys["k_idx"], keys["k_scale"], qs["w"],
+                                pos0=cfg.L - 2048)
+    dsa.dsa_topk(sc, cfg.k, pos0=cfg.L - 2048)
+    torch.cuda.synchronize()
+    assert dsa.dsa_get_device_status() == 0
+    print(json.dumps({"kernels_small": "ok", "attention_tokens": T, "indexer_rows": 2048, "keys": cfg.L}))
+
+
 # ------------------------------------------------------------------------------------------ oracle arm
 _KEYS_CACHE = {}
 
@@ -413,6 +434,8 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--kernels-small", action="store_true",
+                    help="run one launch of each main kernel on small inputs (profiling) and exit")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("at least 3 warm-up steps")
@@ -431,6 +454,9 @@ def main():
 
 def run_dsa(args, ws_n, rank):
     import sparse_attention_long_05_b200 as dsa
+    if args.kernels_small:
+        kernels_small(dsa)
+        return
     pk = peaks()
     pre = bench_prefill(dsa, PREFILL, args.steps, args.warmup, ws_n, rank, pk)
     torch.cuda.empty_cache()

@@ -328,19 +328,46 @@ indexer_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
 #pragma unroll
             for (int q = 0; q < P; ++q) acc[tk][q] = 0.f;
           const uint32_t tcol = tmem_base + ap.stage * 256 + half * CPT;
+          if constexpr (H_I % 64 == 0 && CPT % 64 == 0) {
+            // heads in pairs: ReLU per element, then one packed FMA per pair (1.5 ALU ops per element)
+            uint64_t acc2[TOKS][2];
 #pragma unroll
-          for (int c0 = 0; c0 < CPT; c0 += 64) {
-            uint32_t v0[32], v1[32];
-            tmem_ld32(lane_addr + tcol + c0, v0);
-            if (c0 + 32 < CPT) tmem_ld32(lane_addr + tcol + c0 + 32, v1);
-            tmem_wait_ld();
+            for (int tk = 0; tk < TOKS; ++tk) acc2[tk][0] = acc2[tk][1] = 0ull;
 #pragma unroll
-            for (int i = 0; i < 64; ++i) {
-              if (c0 + i >= CPT) break;
-              const int col = c0 + i;
-              const int tk = col / H_I, j = col % H_I;
-              const float x = __uint_as_float(i < 32 ? v0[i] : v1[i - 32]);
-              acc[tk][j % P] = fmaf(wq[(tok0 + tk) * H_I + j], fmaxf(x, 0.f), acc[tk][j % P]);
+            for (int c0 = 0; c0 < CPT; c0 += 64) {
+              uint32_t v0[32], v1[32];
+              tmem_ld32(lane_addr + tcol + c0, v0);
+              tmem_ld32(lane_addr + tcol + c0 + 32, v1);
+              tmem_wait_ld();
+              const int tk = c0 / H_I;
+              const uint64_t* w2 = reinterpret_cast<const uint64_t*>(wq + (tok0 + tk) * H_I + (c0 % H_I));
+#pragma unroll
+              for (int i = 0; i < 64; i += 2) {
+                const float a0 = fmaxf(__uint_as_float(i < 32 ? v0[i] : v1[i - 32]), 0.f);
+                const float a1 = fmaxf(__uint_as_float(i < 32 ? v0[i + 1] : v1[i - 31]), 0.f);
+                acc2[tk][(i >> 1) & 1] = fma_f32x2(w2[i >> 1], pack_f32x2(a0, a1), acc2[tk][(i >> 1) & 1]);
+              }
+            }
+#pragma unroll
+            for (int tk = 0; tk < TOKS; ++tk) {
+              unpack_f32x2(acc2[tk][0], acc[tk][0], acc[tk][1]);
+              unpack_f32x2(acc2[tk][1], acc[tk][2], acc[tk][3]);
+            }
+          } else {
+#pragma unroll
+            for (int c0 = 0; c0 < CPT; c0 += 64) {
+              uint32_t v0[32], v1[32];
+              tmem_ld32(lane_addr + tcol + c0, v0);
+              if (c0 + 32 < CPT) tmem_ld32(lane_addr + tcol + c0 + 32, v1);
+              tmem_wait_ld();
+#pragma unroll
+              for (int i = 0; i < 64; ++i) {
+                if (c0 + i >= CPT) break;
+                const int col = c0 + i;
+                const int tk = col / H_I, j = col % H_I;
+                const float x = __uint_as_float(i < 32 ? v0[i] : v1[i - 32]);
+                acc[tk][j % P] = fmaf(wq[(tok0 + tk) * H_I + j], fmaxf(x, 0.f), acc[tk][j % P]);
+              }
             }
           }
           tc_fence_before();

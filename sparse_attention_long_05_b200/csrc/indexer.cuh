@@ -70,7 +70,7 @@ struct IndexerCfg {
   // shared memory map (offsets from a 1024-byte aligned base)
   static constexpr int OFF_BAR = 0;                  // barriers + misc (2 KB)
   static constexpr int OFF_PREFIX = 2048;            // decode: per-sequence item prefix (4 KB)
-  static constexpr int OFF_W = OFF_PREFIX + (MODE == kModeDecode ? 4 * (kMaxDecodeSeqs + 1) : 0);
+  static constexpr int OFF_W = ((OFF_PREFIX + (MODE == kModeDecode ? 4 * (kMaxDecodeSeqs + 1) : 0) + 15) / 16) * 16;
   static constexpr int W_FLOATS = TOK * H_I;
   static constexpr int OFF_Q = ((OFF_W + QBUF * W_FLOATS * 4 + ALIGN - 1) / ALIGN) * ALIGN;
   static constexpr int OFF_K = OFF_Q + QBUF * NG * GBYTES;
@@ -79,6 +79,7 @@ struct IndexerCfg {
   static constexpr uint32_t SW_LAYOUT = (D_I == 128) ? kLayoutSW128 : kLayoutSW64;
   static constexpr uint32_t SBO = (D_I == 128) ? 1024 : 512;
   static_assert(N <= 256 && N % 16 == 0, "MMA N");
+  static_assert(OFF_W % 16 == 0 && (W_FLOATS * 4) % 16 == 0, "head weights are read as 8-byte pairs");
   static_assert(D_I == 128 || D_I == 64, "d_I");
   static_assert((N / EPI_WG) % H_I == 0 || H_I > N / EPI_WG, "epilogue column split");
 };

@@ -72,6 +72,21 @@ def max_over_ranks(x: float, ws: int) -> float:
     return float(t.item())
 
 
+def attention_traffic(tokens):
+    """DRAM bytes of one sparse-MLA launch over `tokens` query tokens, scaled from the committed ncu capture
+    (profiles/traffic.json); None once the kernel source differs from the one that capture measured."""
+    import hashlib
+    try:
+        t = json.load(open(os.path.join(ROOT, "profiles", "traffic.json")))["sparse_mla_attn"]
+        src = b"".join(open(os.path.join(ROOT, "sparse_attention_long_05_b200", "csrc", f), "rb").read()
+                       for f in ("sparse_mla.cuh", "common.cuh"))
+        if hashlib.sha256(src).hexdigest()[:16] != t["source_sha256_16"]:
+            return None
+        return t["dram_bytes_per_query_token"] * tokens
+    except (OSError, KeyError, ValueError):
+        return None
+
+
 def peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(path):
@@ -231,7 +246,7 @@ def bench_prefill(dsa, cfg, steps, warmup, ws_n, rank, pk):
     dom = max(kernels, key=lambda n: kernels[n]["ms"])
     d = kernels[dom]
     roof = {"kernel": dom, "bound": d["bound"], "achieved": d["achieved"], "peak": d["peak"], "unit": d["unit"],
-            "frac": d["frac"], "traffic": None,
+            "frac": d["frac"], "traffic": attention_traffic(L) if dom == "sparse_mla_attn" else None,
             "peak_source": f"{pk['source']} bf16 sustained" + (" x2 (FP8)" if dom == "prefill_select" else "")}
     del x
     return {"ms": ms, "tokens_per_s": ws_n * L / (ms * 1e-3), "roofline": roof, "kernels": kernels,

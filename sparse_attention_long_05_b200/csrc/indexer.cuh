@@ -79,7 +79,7 @@ struct IndexerCfg {
   static constexpr uint32_t SW_LAYOUT = (D_I == 128) ? kLayoutSW128 : kLayoutSW64;
   static constexpr uint32_t SBO = (D_I == 128) ? 1024 : 512;
   static_assert(N <= 256 && N % 16 == 0, "MMA N");
-  static_assert(OFF_W % 16 == 0 && (W_FLOATS * 4) % 16 == 0, "head weights are read as 8-byte pairs");
+  static_assert(OFF_W % 16 == 0 && (W_FLOATS * 4) % 16 == 0, "head weights are read as 16-byte quads");
   static_assert(D_I == 128 || D_I == 64, "d_I");
   static_assert((N / EPI_WG) % H_I == 0 || H_I > N / EPI_WG, "epilogue column split");
 };
@@ -278,6 +278,10 @@ indexer_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     constexpr int CPT = C::N / EPI_WG;              // accumulator columns per thread
     constexpr int TOKS = (CPT >= H_I) ? CPT / H_I : 1;  // query rows per thread
     constexpr int P = (H_I >= 16) ? 4 : 1;         // partial sums per row (ILP)
+    // Packed epilogue (heads in groups of four): w ReLU(x) is formed as w max(x, 0) for even heads (ALU pipe)
+    // and as (w / 2)(x + |x|) for odd heads (FMA pipe, |x| as an operand modifier), so that the two pipes share
+    // the ReLUs; the odd heads' weights are stored halved.  Both forms are exact for integer-valued inputs.
+    constexpr bool kPacked = (H_I % 64 == 0) && (CPT % 64 == 0);
     const int e = warp - 2;
     const int quad = warp & 3;
     const int half = e >> 2;
@@ -297,6 +301,7 @@ indexer_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         if (r < it.n_tok) {
           v = p.w[static_cast<long long>(it.q_row0 + r) * H_I + (i % H_I)];
           if (p.q_scale) v *= p.q_scale[it.q_row0 + r];
+          if (kPacked && (i & 1)) v *= 0.5f;
         }
         wq[i] = v;
       }
@@ -329,8 +334,7 @@ indexer_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
 #pragma unroll
             for (int q = 0; q < P; ++q) acc[tk][q] = 0.f;
           const uint32_t tcol = tmem_base + ap.stage * 256 + half * CPT;
-          if constexpr (H_I % 64 == 0 && CPT % 64 == 0) {
-            // heads in pairs: ReLU per element, then one packed FMA per pair (1.5 ALU ops per element)
+          if constexpr (kPacked) {
             uint64_t acc2[TOKS][2];
 #pragma unroll
             for (int tk = 0; tk < TOKS; ++tk) acc2[tk][0] = acc2[tk][1] = 0ull;
@@ -341,12 +345,18 @@ indexer_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
               tmem_ld32(lane_addr + tcol + c0 + 32, v1);
               tmem_wait_ld();
               const int tk = c0 / H_I;
-              const uint64_t* w2 = reinterpret_cast<const uint64_t*>(wq + (tok0 + tk) * H_I + (c0 % H_I));
+              const float4* w4 = reinterpret_cast<const float4*>(wq + (tok0 + tk) * H_I + (c0 % H_I));
 #pragma unroll
-              for (int i = 0; i < 64; i += 2) {
-                const float a0 = fmaxf(__uint_as_float(i < 32 ? v0[i] : v1[i - 32]), 0.f);
-                const float a1 = fmaxf(__uint_as_float(i < 32 ? v0[i + 1] : v1[i - 31]), 0.f);
-                acc2[tk][(i >> 1) & 1] = fma_f32x2(w2[i >> 1], pack_f32x2(a0, a1), acc2[tk][(i >> 1) & 1]);
+              for (int i = 0; i < 64; i += 4) {
+                const float4 ww = w4[i >> 2];
+                float a[4];
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                  const float x = __uint_as_float(i + u < 32 ? v0[i + u] : v1[i + u - 32]);
+                  a[u] = (u & 1) ? x + fabsf(x) : fmaxf(x, 0.f);
+                }
+                acc2[tk][0] = fma_f32x2(pack_f32x2(ww.x, ww.y), pack_f32x2(a[0], a[1]), acc2[tk][0]);
+                acc2[tk][1] = fma_f32x2(pack_f32x2(ww.z, ww.w), pack_f32x2(a[2], a[3]), acc2[tk][1]);
               }
             }
 #pragma unroll

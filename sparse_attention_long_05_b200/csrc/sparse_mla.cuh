@@ -17,14 +17,16 @@
 //
 // Data movement.
 //   * Selected rows are gathered by TMA tile::gather4 (four rows x one 64-column, 128-byte swizzled box per
-//     instruction) into 64-key x 64-dim stages in the K-major form the tensor core reads.  Eight warps issue
-//     the gathers, each owning every eighth stage, because one warp issues gather4 instructions only about
-//     every 50 ns (gather throughput per SM grows with the number of issuing warps: about 12, 24, 45 and
-//     73 GB/s with 1, 2, 4 and 8); TMA writes are in the async proxy, so the MMA warp consumes a stage as
-//     soon as its
-//     mbarrier transaction count completes, with no proxy fence.  The
-//     same stage bytes serve as the K-major B operand of QK^T (rows = keys) and as the MN-major B operand
-//     of PV (rows = keys = K, 64 dims = N per atom).
+//     instruction) into 64-key x 64-dim chunks in the K-major form the tensor core reads.  A pipeline stage
+//     holds several chunks of one 64-key tile (three in the score CTA, four in the value CTA), because the
+//     issuing thread spends a few hundred cycles per stage on its barrier wait, the tcgen05 issue and the
+//     commit whatever the stage's size: with one 64-dim chunk per stage the QK^T MMA thread, not the tensor
+//     core, set the pace.  Each stage is split over eight gather warps (one warp issues gather4 only about
+//     every 50 ns; gather throughput per SM grows with the issuing warps: about 12, 24, 45 and 73 GB/s
+//     with 1, 2, 4 and 8), each of which arrives on the stage's barrier with its share of the bytes.  TMA
+//     writes are in the async proxy, so the MMA warp consumes a stage as soon as its mbarrier completes,
+//     with no proxy fence.  The same chunk bytes serve as the K-major B operand of QK^T (rows = keys) and
+//     as the MN-major B operand of PV (rows = keys = K, 64 dims = N per atom; four chunks = N 256).
 //   * The token's selected-index row is prefetched into shared memory with one bulk copy.
 //   * Q chunks (128 heads x 64 dims) are staged by TMA (three shared-memory slots) and copied into a ring of
 //     twelve 32-column chunk slots of tensor memory with tcgen05.cp; chunk c of the token with running index
@@ -35,7 +37,8 @@
 //     and chunks 6-8 during the next token's first tile, just before their first use.  No copy waits on an
 //     MMA issued less than three chunks earlier.
 //
-// Warp roles (14 warps per CTA): w0 loader (index rows, Q chunks), w1 TMEM allocation + MMA issue,
+// Warp roles (14 warps per CTA): w0 loader (index rows, Q chunks), w1 TMEM allocation + MMA issue (a
+// warp-uniform loop; one elected lane issues the tcgen05 instructions),
 // w2 w3 w8..w13 gathers, w4..w7 softmax (score CTA) or correction / epilogue (value CTA); warp w owns TMEM
 // lanes (= heads) 32 * (w % 4) .. +31.
 #pragma once
@@ -65,7 +68,10 @@ constexpr int QS = 3;                     // Q staging slots (score CTA)
 constexpr int NSB = 2;                    // S buffers in tensor memory (score CTA)
 constexpr int QSLOTS = 12;                // Q chunk slots in tensor memory (score CTA)
 constexpr int NPB = 3;                    // P buffers (value CTA)
-constexpr int NS_S = 15, NS_V = 16;       // gather stages per CTA
+constexpr int SCH = 3, VCH = 4;           // 64-dim chunks per gather stage (score CTA, value CTA)
+constexpr int S_STAGE = SCH * CHUNK_BYTES, V_STAGE = VCH * CHUNK_BYTES;
+constexpr int SPT_S = QCHUNKS / SCH, SPT_V = VCHUNKS / VCH;   // stages per 64-key tile: 3, 2
+constexpr int NS_S = 5, NS_V = 4;         // gather stages per CTA
 constexpr int THREADS = 448;
 constexpr int GATHER_WARPS = 8;
 constexpr float RESCALE_LOG2 = 8.0f;      // lazy rescale threshold (factor 256)
@@ -80,10 +86,12 @@ constexpr int B_QST_FULL = 4, B_QST_EMPTY = B_QST_FULL + QS;
 constexpr int B_RING_FULL = B_QST_EMPTY + QS, B_RING_EMPTY = B_RING_FULL + 16;
 constexpr int B_S_FULL = B_RING_EMPTY + 16, B_S_EMPTY = B_S_FULL + NSB, B_P_EMPTY = B_S_EMPTY + NSB;
 constexpr int B_P_FULL = B_P_EMPTY + NPB, B_P_READY = B_P_FULL + NPB;
-constexpr int B_O_DONE = B_P_READY + NPB, B_O_FREE = B_O_DONE + 1;
+// O_DONE: one barrier per P buffer (PV of tile g completes O_DONE[g % NPB]); a single barrier would be waited
+// only now and then and could be two phases behind, where a parity test cannot tell the phases apart
+constexpr int B_O_DONE = B_P_READY + NPB, B_O_FREE = B_O_DONE + NPB;
 constexpr int B_SLOT_FREE = B_O_FREE + 1, B_SLOT_WRITTEN = B_SLOT_FREE + 1;   // score CTA softmax handshakes
-constexpr int B_QRET = B_SLOT_WRITTEN + 1;    // score CTA: last-tile MMAs of chunks 0..2 retired (3 barriers)
-constexpr int B_QTOK = B_QRET + 3;            // score CTA: every MMA of a token retired
+constexpr int B_QRET = B_SLOT_WRITTEN + 1;    // score CTA: last-tile MMAs of chunks 0..2 retired
+constexpr int B_QTOK = B_QRET + 1;            // score CTA: every MMA of a token retired
 constexpr int B_COUNT = B_QTOK + 1;
 // shared memory map (from a 1024-byte aligned base; both CTAs use the same barrier offsets)
 constexpr int OFF_TMEM = 8 * B_COUNT;
@@ -94,13 +102,15 @@ constexpr int OFF_QST = OFF_PST + 2 * XFER;                     // score CTA: Q 
 constexpr int OFF_RING_S = OFF_QST + QS * QCHUNK_BYTES;         // score CTA: gather ring
 constexpr int OFF_PB = OFF_IDX + 2 * KMAX * 4;                  // value CTA: P buffers
 constexpr int OFF_RING_V = OFF_PB + NPB * XFER;                 // value CTA: gather ring
-constexpr int SMEM_S = OFF_RING_S + NS_S * CHUNK_BYTES;
-constexpr int SMEM_V = OFF_RING_V + NS_V * CHUNK_BYTES;
+constexpr int SMEM_S = OFF_RING_S + NS_S * S_STAGE;
+constexpr int SMEM_V = OFF_RING_V + NS_V * V_STAGE;
 constexpr int SMEM = (SMEM_S > SMEM_V ? SMEM_S : SMEM_V) + 1024;
 static_assert(OFF_TMEM + 8 <= OFF_IDX, "barrier area");
 static_assert(OFF_PST % 1024 == 0 && OFF_QST % 1024 == 0 && OFF_RING_S % 1024 == 0, "1 KB aligned tiles");
 static_assert(OFF_PB % 1024 == 0 && XFER % 1024 == 0 && OFF_RING_V % 1024 == 0, "1 KB aligned tiles");
-static_assert(NS_V % 4 == 0, "value stages come in groups of four 64-dim chunks");
+static_assert(QCHUNKS % SCH == 0 && VCHUNKS % VCH == 0 && VCH * 64 == 256, "stage split");
+static_assert((SCH * 16) % GATHER_WARPS == 0 && (VCH * 16) % GATHER_WARPS == 0, "gather4 split over warps");
+static_assert(NS_S <= 16 && NS_V <= 16, "ring barrier slots");
 static_assert(SMEM <= 232448, "shared memory per CTA");
 }  // namespace mla
 
@@ -155,7 +165,7 @@ sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
       mbar_init(bar(B_IDX_EMPTY + i), rank == 0 ? GATHER_WARPS + 4 : GATHER_WARPS);
     }
     for (int i = 0; i < 16; ++i) {
-      mbar_init(bar(B_RING_FULL + i), 1);                // the issuing warp's arrive.expect_tx + TMA bytes
+      mbar_init(bar(B_RING_FULL + i), GATHER_WARPS);     // each gather warp's arrive.expect_tx + TMA bytes
       mbar_init(bar(B_RING_EMPTY + i), 1);
     }
     if (rank == 0) {
@@ -164,11 +174,11 @@ sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
       for (int i = 0; i < NPB; ++i) mbar_init(bar(B_P_EMPTY + i), 1);
       mbar_init(bar(B_SLOT_FREE), 1);
       mbar_init(bar(B_SLOT_WRITTEN), 4);
-      for (int i = 0; i < 3; ++i) mbar_init(bar(B_QRET + i), 1);
+      mbar_init(bar(B_QRET), 1);
       mbar_init(bar(B_QTOK), 1);
     } else {
       for (int i = 0; i < NPB; ++i) { mbar_init(bar(B_P_FULL + i), 1); mbar_init(bar(B_P_READY + i), 4); }
-      mbar_init(bar(B_O_DONE), 1);
+      for (int i = 0; i < NPB; ++i) mbar_init(bar(B_O_DONE + i), 1);
       mbar_init(bar(B_O_FREE), 4);
     }
     *abort_flag = 0;
@@ -221,13 +231,21 @@ sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     }
   } else if (warp == 2 || warp == 3 || warp >= 8) {
     // ===================================================================== gathers (TMA gather4)
-    // warp gw issues the stages of chunks n with n % 8 == gw; lane L < 16 gathers rows 4L .. 4L+3
+    // Every stage is split over the eight gather warps: gather4 instruction i of a stage (i = 16 cc + rg)
+    // fetches rows 4 rg .. 4 rg + 3 of the tile into its chunk cc; warp gw issues instructions
+    // gw * per_warp .. + per_warp - 1, one per lane.
     const int gw = (warp < 8) ? warp - 2 : warp - 6;
-    const int nch = (rank == 0) ? QCHUNKS : VCHUNKS;
+    const int cps = (rank == 0) ? SCH : VCH;               // chunks per stage
+    const int spt = (rank == 0) ? SPT_S : SPT_V;           // stages per tile
+    const uint32_t sbytes = cps * CHUNK_BYTES;
+    const int per_warp = cps * 16 / GATHER_WARPS;          // 6 or 8
+    const int gi = gw * per_warp + lane;
+    const int cc = gi >> 4, rg = gi & 15;
+    const bool active = lane < per_warp;
     RingPos rp;
     rp.size = nsr;
-    long long n = 0, n_last = -1;     // n_last: the last chunk this warp issued
-    RingPos last;                      // its ring position
+    bool issued = false;               // this warp issued a load into the ring
+    RingPos last;                      // ring position of its latest stage
     int ti = 0;
     bool ok = true;
     for (int t = cluster; t < p.T && ok; t += nclusters, ++ti) {
@@ -237,148 +255,162 @@ sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
       const long long base = p.row_off ? p.row_off[t] : 0;
       for (int j = 0; j < ntiles && ok; ++j) {
         int r[4] = {0, 0, 0, 0};
-        if (lane < 16) {
-          const int4 e = reinterpret_cast<const int4*>(ids + j * NK)[lane];
+        if (active) {
+          const int4 e = reinterpret_cast<const int4*>(ids + j * NK)[rg];
           r[0] = static_cast<int>(mla_row(e.x, base, p.S));
           r[1] = static_cast<int>(mla_row(e.y, base, p.S));
           r[2] = static_cast<int>(mla_row(e.z, base, p.S));
           r[3] = static_cast<int>(mla_row(e.w, base, p.S));
         }
-        for (int c = 0; c < nch; ++c, ++n, rp.advance()) {
-          if ((n & (GATHER_WARPS - 1)) != gw) continue;
+        for (int s = 0; s < spt; ++s, rp.advance()) {
           const int st = rp.stage;
           bool got = true;
           if (lane == 0) {
             got = mbar_wait(bar(B_RING_EMPTY + st), rp.phase ^ 1, abort_flag);
-            if (got) mbar_arrive_expect_tx(bar(B_RING_FULL + st), CHUNK_BYTES);
+            if (got) mbar_arrive_expect_tx(bar(B_RING_FULL + st), per_warp * 512);
           }
           if (!(ok = __shfl_sync(0xffffffffu, got, 0))) break;
-          if (lane == 0 && c == 0) DSA_TRACE_EVENT(rank == 0 ? 0 : 16, n / nch);
-          if (lane < 16)
-            tma_gather4(ring + st * CHUNK_BYTES + lane * 512, &tm_c, bar(B_RING_FULL + st), 64 * c, r[0], r[1], r[2],
-                        r[3]);
-          if (lane == 0 && rank == 0) DSA_TRACE_EVENT(8, n);
-          n_last = n;
+          if (lane == 0 && gw == 0 && s == 0) DSA_TRACE_EVENT(rank == 0 ? 0 : 16, ti * ntiles + j);
+          if (active)
+            tma_gather4(ring + st * sbytes + cc * CHUNK_BYTES + rg * 512, &tm_c, bar(B_RING_FULL + st),
+                        64 * (s * cps + cc), r[0], r[1], r[2], r[3]);
+          issued = true;
           last = rp;
         }
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(bar(B_IDX_EMPTY + is));
     }
-    if (lane == 0 && *abort_flag && n_last >= 0) {
-      // leave no gather in flight into this CTA's shared memory: bounded waits on this warp's loads of the last
-      // pass over the ring (stages below its last stage in that pass' parity, the others one pass earlier)
+    if (lane == 0 && *abort_flag && issued) {
+      // leave no gather in flight into this CTA's shared memory: bounded waits on the stages of the last pass
+      // over the ring (stages up to this warp's last one in that pass' parity, the others one pass earlier)
       for (int st = 0; st < nsr; ++st)
         mbar_wait_drain(bar(B_RING_FULL + st), st <= last.stage ? last.phase : last.phase ^ 1);
     }
   } else if (warp == 1) {
     // ===================================================================== MMA issue
-    if (lane == 0) {
-      bool ok = true;
-      int g = 0;
-      RingPos rp;
-      rp.size = nsr;
-      int ti = 0;
-      if (rank == 0) {
-        constexpr uint32_t idesc = idesc_bf16(128, NK, false);
-        int qn = 0;          // Q chunks copied into tensor memory so far (= 9 * token index + chunk)
-        // copy the next staged Q chunk (global chunk index qn) into its tensor-memory slot
-        auto copy_q = [&]() -> bool {
-          const int qs = qn % QS;
-          if (!mbar_wait(bar(B_QST_FULL + qs), (qn / QS) & 1, abort_flag)) return false;
-          tc_fence_after();
-          const uint32_t src = sbase + OFF_QST + qs * QCHUNK_BYTES;
-          const uint32_t dst = tmem + TQ + 32 * (qn % QSLOTS);
+    // The whole warp runs the loop (every wait is warp-uniform); one elected lane issues each tcgen05 op.
+    bool ok = true;
+    int g = 0;
+    RingPos rp;
+    rp.size = nsr;
+    int ti = 0;
+    if (rank == 0) {
+      constexpr uint32_t idesc = idesc_bf16(128, NK, false);
+      int qn = 0;          // Q chunks copied into tensor memory so far (= 9 * token index + chunk)
+      // copy the next staged Q chunk (global chunk index qn) into its tensor-memory slot
+      auto copy_q = [&]() -> bool {
+        const int qs = qn % QS;
+        if (!warp_wait(bar(B_QST_FULL + qs), (qn / QS) & 1, abort_flag)) return false;
+        tc_fence_after();
+        const uint32_t src = sbase + OFF_QST + qs * QCHUNK_BYTES;
+        const uint32_t dst = tmem + TQ + 32 * (qn % QSLOTS);
+        if (elect_one()) {
 #pragma unroll
           for (int s = 0; s < 4; ++s) tmem_cp_128x256b(dst + 8 * s, smem_desc(src + 32 * s, 16, 1024, kLayoutSW128));
           mma_commit(bar(B_QST_EMPTY + qs));
-          ++qn;
-          return true;
-        };
-        int nret = 0;        // tokens whose last tile committed the QRET barriers
-        if (cluster < p.T)
-          for (int c = 0; c < QCHUNKS && ok; ++c) ok = copy_q();
-        for (int t = cluster; t < p.T && ok; t += nclusters, ++ti) {
-          const bool has_next = t + nclusters < p.T;
-          const uint32_t prev_tok = static_cast<uint32_t>((ti - 1) & 1);   // parity of the previous token's QTOK
-          for (int j = 0; j < ntiles && ok; ++j, ++g) {
-            const int sb = g % NSB;
-            if (j == 1 && has_next) {
-              // next token's chunks 0..2 go to the slots of the previous token's chunks 6..8
-              if (ti > 0 && !(ok = mbar_wait(bar(B_QTOK), prev_tok, abort_flag))) break;
+        }
+        __syncwarp();
+        ++qn;
+        return true;
+      };
+      int nret = 0;        // tokens whose last tile committed the QRET barriers
+      if (cluster < p.T)
+        for (int c = 0; c < QCHUNKS && ok; ++c) ok = copy_q();
+      for (int t = cluster; t < p.T && ok; t += nclusters, ++ti) {
+        const bool has_next = t + nclusters < p.T;
+        const uint32_t prev_tok = static_cast<uint32_t>((ti - 1) & 1);   // parity of the previous token's QTOK
+        const int q_slot0 = (9 * ti) % QSLOTS;                          // tensor-memory slot of chunk 0
+        for (int j = 0; j < ntiles && ok; ++j, ++g) {
+          const int sb = g % NSB;
+          if (j == 1 && has_next) {
+            // next token's chunks 0..2 go to the slots of the previous token's chunks 6..8
+            if (ti > 0 && !(ok = warp_wait(bar(B_QTOK), prev_tok, abort_flag))) break;
+            for (int c = 0; c < 3 && ok; ++c) ok = copy_q();
+            if (!ok) break;
+          }
+          if (!(ok = warp_wait(bar(B_S_EMPTY + sb), static_cast<uint32_t>((g / NSB) & 1) ^ 1, abort_flag))) break;
+          DSA_TRACE_EVENT(2, g);
+          tc_fence_after();
+          const bool last = (j == ntiles - 1) && has_next;
+          for (int s = 0; s < SPT_S && ok; ++s, rp.advance()) {
+            const int st = rp.stage;
+            if (!(ok = warp_wait(bar(B_RING_FULL + st), rp.phase, abort_flag))) break;
+            DSA_TRACE_EVENT(12 + s, g);
+            tc_fence_after();
+            if (j == 0 && s == SPT_S - 1 && ti > 0) {
+              // this token's chunks 6..8 go to the slots of the previous token's chunks 3..5
+              if (!(ok = warp_wait(bar(B_QTOK), prev_tok, abort_flag))) break;
               for (int c = 0; c < 3 && ok; ++c) ok = copy_q();
               if (!ok) break;
             }
-            if (!(ok = mbar_wait(bar(B_S_EMPTY + sb), static_cast<uint32_t>((g / NSB) & 1) ^ 1, abort_flag))) break;
-            DSA_TRACE_EVENT(2, g);
-            tc_fence_after();
-            const bool last = (j == ntiles - 1) && has_next;
-            for (int c = 0; c < QCHUNKS; ++c, rp.advance()) {
-              if (j == 0 && c >= 6 && ti > 0) {
-                // this token's chunks 6..8 go to the slots of the previous token's chunks 3..5
-                if (c == 6 && !(ok = mbar_wait(bar(B_QTOK), prev_tok, abort_flag))) break;
-                if (!(ok = copy_q())) break;
-              }
-              const int st = rp.stage;
-              DSA_TRACE_EVENT(10, g * QCHUNKS + c);
-              if (!(ok = mbar_wait(bar(B_RING_FULL + st), rp.phase, abort_flag))) break;
-              DSA_TRACE_EVENT(9, g * QCHUNKS + c);
-              tc_fence_after();
-              const uint64_t bd = smem_desc(ring + st * CHUNK_BYTES, 16, 1024, kLayoutSW128);
-              const uint32_t a = tmem + TQ + 32 * ((9 * ti + c) % QSLOTS);
+            // the stage's three chunks: 12 MMAs issued as one block, then one commit
+            const uint64_t bd = smem_desc(ring + st * S_STAGE, 16, 1024, kLayoutSW128);
+            int slot = q_slot0 + s * SCH;
+            if (slot >= QSLOTS) slot -= QSLOTS;
+            if (elect_one()) {
 #pragma unroll
-              for (int s = 0; s < 4; ++s)     // K = 16 bf16 per instruction: 8 TMEM columns of A, 32 bytes of B
-                mma_bf16_ts(tmem + TS + NK * sb, a + 8 * s, bd + 2 * s, idesc, (c | s) ? 1u : 0u);
+              for (int cc = 0; cc < SCH; ++cc) {
+                const uint32_t a = tmem + TQ + 32 * (slot + cc < QSLOTS ? slot + cc : slot + cc - QSLOTS);
+#pragma unroll
+                for (int k = 0; k < 4; ++k)   // K = 16 bf16 per instruction: 8 TMEM columns of A, 32 bytes of B
+                  mma_bf16_ts(tmem + TS + NK * sb, a + 8 * k, bd + ((cc * CHUNK_BYTES) >> 4) + 2 * k, idesc,
+                              (s | cc | k) ? 1u : 0u);
+              }
               mma_commit(bar(B_RING_EMPTY + st));
-              DSA_TRACE_EVENT(11, g * QCHUNKS + c);
-              if (last) {
-                if (c < 3) mma_commit(bar(B_QRET + c));
-                if (c >= 3 && c < 6) {
-                  // next token's chunk c overwrites this token's chunk c - 3, committed three chunks ago
-                  if (!(ok = mbar_wait(bar(B_QRET + c - 3), static_cast<uint32_t>(nret & 1), abort_flag))) break;
-                  if (!(ok = copy_q())) break;
-                }
-              }
+              if (last && s == 0) mma_commit(bar(B_QRET));   // chunks 0..2 of this token retire
             }
-            if (!ok) break;
-            if (last) ++nret;
-            DSA_TRACE_EVENT(3, g);
-            mma_commit(bar(B_S_FULL + sb));
-          }
-          mma_commit(bar(B_QTOK));
-        }
-      } else {
-        constexpr uint32_t idesc = idesc_bf16(128, 256, true);
-        for (int t = cluster; t < p.T && ok; t += nclusters, ++ti) {
-          for (int j = 0; j < ntiles && ok; ++j, ++g) {
-            const int pb = static_cast<int>(g % NPB);
-            if (j == 0 && !(ok = mbar_wait(bar(B_O_FREE), (ti & 1) ^ 1, abort_flag))) break;
-            if (!(ok = mbar_wait(bar(B_P_READY + pb), static_cast<uint32_t>((g / NPB) & 1), abort_flag))) break;
-            DSA_TRACE_EVENT(20, g);
-            tc_fence_after();
-            const uint64_t ad = smem_desc(sbase + OFF_PB + pb * XFER, 16, 1024, kLayoutSW128);
-            for (int hh = 0; hh < 2 && ok; ++hh) {
-              const int st0 = rp.stage;          // four consecutive stages (the ring size is a multiple of 4)
-              const uint32_t ph0 = rp.phase;
-              for (int q = 0; q < 4 && ok; ++q) ok = mbar_wait(bar(B_RING_FULL + st0 + q), ph0, abort_flag);
+            __syncwarp();
+            DSA_TRACE_EVENT(9 + s, g);
+            if (last && s == 1) {
+              // the next token's chunks 3..5 overwrite this token's chunks 0..2
+              if (!(ok = warp_wait(bar(B_QRET), static_cast<uint32_t>(nret & 1), abort_flag))) break;
+              for (int c = 0; c < 3 && ok; ++c) ok = copy_q();
               if (!ok) break;
-              DSA_TRACE_EVENT(21 + hh, g);
-              tc_fence_after();
-              // MN-major V: 64-dim chunks 8 KB apart (LBO), 8-key row groups 1 KB apart (SBO)
-              const uint64_t bd = smem_desc(ring + st0 * CHUNK_BYTES, CHUNK_BYTES, 1024, kLayoutSW128);
-#pragma unroll
-              for (int s = 0; s < 4; ++s)     // 16 keys per instruction: two 8-key groups = 2 KB of V
-                mma_bf16_ss(tmem + 256 * hh, ad + 2 * s, bd + ((s * 2048) >> 4), idesc, (j == 0 && s == 0) ? 0u : 1u);
-              for (int q = 0; q < 4; ++q) {
-                mma_commit(bar(B_RING_EMPTY + st0 + q));
-                rp.advance();
-              }
             }
-            if (!ok) break;
-            DSA_TRACE_EVENT(23, g);
-            mma_commit_mc(bar(B_P_EMPTY + pb), 0x1);   // P buffer pb free again (score CTA waits on it)
-            mma_commit(bar(B_O_DONE));
           }
+          if (!ok) break;
+          if (last) ++nret;
+          DSA_TRACE_EVENT(3, g);
+          if (elect_one()) mma_commit(bar(B_S_FULL + sb));
+          __syncwarp();
+        }
+        if (!ok) break;
+        if (elect_one()) mma_commit(bar(B_QTOK));
+        __syncwarp();
+      }
+    } else {
+      constexpr uint32_t idesc = idesc_bf16(128, 256, true);
+      for (int t = cluster; t < p.T && ok; t += nclusters, ++ti) {
+        for (int j = 0; j < ntiles && ok; ++j, ++g) {
+          const int pb = static_cast<int>(g % NPB);
+          if (j == 0 && !(ok = warp_wait(bar(B_O_FREE), (ti & 1) ^ 1, abort_flag))) break;
+          if (!(ok = warp_wait(bar(B_P_READY + pb), static_cast<uint32_t>((g / NPB) & 1), abort_flag))) break;
+          DSA_TRACE_EVENT(20, g);
+          tc_fence_after();
+          const uint64_t ad = smem_desc(sbase + OFF_PB + pb * XFER, 16, 1024, kLayoutSW128);
+          for (int hh = 0; hh < SPT_V; ++hh, rp.advance()) {
+            const int st = rp.stage;
+            if (!(ok = warp_wait(bar(B_RING_FULL + st), rp.phase, abort_flag))) break;
+            DSA_TRACE_EVENT(21 + hh, g);
+            tc_fence_after();
+            // MN-major V: 64-dim chunks 8 KB apart (LBO), 8-key row groups 1 KB apart (SBO)
+            const uint64_t bd = smem_desc(ring + st * V_STAGE, CHUNK_BYTES, 1024, kLayoutSW128);
+            if (elect_one()) {
+#pragma unroll
+              for (int k = 0; k < 4; ++k)     // 16 keys per instruction: two 8-key groups = 2 KB of V
+                mma_bf16_ss(tmem + 256 * hh, ad + 2 * k, bd + ((k * 2048) >> 4), idesc, (j == 0 && k == 0) ? 0u : 1u);
+              mma_commit(bar(B_RING_EMPTY + st));
+            }
+            __syncwarp();
+          }
+          if (!ok) break;
+          DSA_TRACE_EVENT(23, g);
+          if (elect_one()) {
+            mma_commit_mc(bar(B_P_EMPTY + pb), 0x1);   // P buffer pb free again (score CTA waits on it)
+            mma_commit(bar(B_O_DONE + pb));
+          }
+          __syncwarp();
         }
       }
     }
@@ -420,6 +452,7 @@ sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(bar(B_S_EMPTY + sb));
+        if (leader) DSA_TRACE_EVENT(24, g);
         // running max over the valid keys of the tile (raw logits; the scale is positive), as a 4-way tree
         const bool full_tile = (m_even & m_odd) == 0xffffffffu;
         float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
@@ -466,9 +499,11 @@ sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         if (leader) {
           DSA_TRACE_EVENT(5, g);
           bulk_wait_read<1>();
+          DSA_TRACE_EVENT(26, g);
           mbar_arrive(bar(B_SLOT_FREE));
         }
         if (!(ok = warp_wait(bar(B_SLOT_FREE), static_cast<uint32_t>(g & 1), abort_flag))) break;
+        if (leader) DSA_TRACE_EVENT(27, g);
         uint8_t* st = smem + OFF_PST + b * XFER;
         uint8_t* prow = st + h * 128;
 #pragma unroll
@@ -483,13 +518,15 @@ sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                 (le > 0.f) ? (m_ref + lg2_approx(le)) * 0.69314718055994531f : -INFINITY;
         }
         fence_proxy_async_smem();     // the staging slot is read next by the bulk-copy (async) proxy
+        if (leader) DSA_TRACE_EVENT(28, g);
         __syncwarp();
         if (lane == 0) mbar_arrive(bar(B_SLOT_WRITTEN));
         if (leader) {
           // all four warps wrote the slot; the value CTA's P buffer pb is free once its PV of tile g - NPB
           // has completed
-          ok = mbar_wait(bar(B_SLOT_WRITTEN), static_cast<uint32_t>(g & 1), abort_flag) &&
-               mbar_wait<true>(bar(B_P_EMPTY + pb), static_cast<uint32_t>((g / NPB) & 1) ^ 1, abort_flag);
+          ok = mbar_wait(bar(B_SLOT_WRITTEN), static_cast<uint32_t>(g & 1), abort_flag);
+          DSA_TRACE_EVENT(29, g);
+          ok = ok && mbar_wait<true>(bar(B_P_EMPTY + pb), static_cast<uint32_t>((g / NPB) & 1) ^ 1, abort_flag);
           if (ok) {
             DSA_TRACE_EVENT(7, g);
             mbar_arrive_expect_tx_remote(pfull_remote + 8 * pb, XFER);
@@ -522,7 +559,7 @@ sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         if (j == ntiles - 1) l = reinterpret_cast<const float*>(xb + P_BYTES + 512)[h];
         if (j > 0 && __any_sync(0xffffffffu, a != 1.f)) {
           // wait until every PV up to tile g - 1 has landed in O, then scale the warp's rows of O
-          if (!(ok = warp_wait(bar(B_O_DONE), static_cast<uint32_t>((g - 1) & 1), abort_flag))) break;
+          if (!(ok = warp_wait(bar(B_O_DONE + (g - 1) % NPB), static_cast<uint32_t>(((g - 1) / NPB) & 1), abort_flag))) break;
           tc_fence_after();
           for (int cc = 0; cc < DV / 32; ++cc) {
             uint32_t v[32];
@@ -537,10 +574,11 @@ sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(bar(B_P_READY + pb));
+        if (warp == 4 && lane == 0) DSA_TRACE_EVENT(19, g);
       }
       if (!ok) break;
       // epilogue: O / l -> bf16
-      if (!(ok = warp_wait(bar(B_O_DONE), static_cast<uint32_t>((g - 1) & 1), abort_flag))) break;
+      if (!(ok = warp_wait(bar(B_O_DONE + (g - 1) % NPB), static_cast<uint32_t>(((g - 1) / NPB) & 1), abort_flag))) break;
       tc_fence_after();
       const float inv = (l > 0.f) ? 1.f / l : 0.f;
       uint16_t* orow = p.out + (static_cast<long long>(t) * p.H + h) * DV;

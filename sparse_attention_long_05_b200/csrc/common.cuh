@@ -210,9 +210,11 @@ template <int N>
 __device__ __forceinline__ void bulk_wait_read() {
   asm volatile("cp.async.bulk.wait_group.read %0;" :: "n"(N) : "memory");
 }
-// arrive on a peer CTA's barrier and raise its expected transaction count
+// arrive on a peer CTA's barrier and raise its expected transaction count.  Relaxed: the data this
+// announces arrives by a bulk copy whose transaction completion makes it visible; a release here would make
+// the thread wait for all of its earlier memory operations first (measured: about 1 us per tile)
 __device__ __forceinline__ void mbar_arrive_expect_tx_remote(uint32_t bar_cluster, uint32_t bytes) {
-  asm volatile("mbarrier.arrive.expect_tx.release.cluster.shared::cluster.b64 _, [%0], %1;"
+  asm volatile("mbarrier.arrive.expect_tx.relaxed.cluster.shared::cluster.b64 _, [%0], %1;"
                :: "r"(bar_cluster), "r"(bytes) : "memory");
 }
 // 16-byte global -> shared copy through L2 (LSU path)

@@ -135,14 +135,25 @@ dsa_status_t run_indexer_scores(const uint8_t* q_idx, const float* q_scale, cons
   const int tok = (H_I == 64) ? 16 : 256;
   const int nqb = (T + tok - 1) / tok;
   const int ntiles = (S + 127) / 128;
-  int nsplit = (2 * num_sms() + nqb - 1) / nqb;
-  nsplit = nsplit < 1 ? 1 : (nsplit > ntiles ? ntiles : nsplit);
-  p.split_tiles = (ntiles + nsplit - 1) / nsplit;
+  // Work items (query block x key-tile range) go round-robin to one persistent CTA per SM.  The key range is
+  // split so that the items divide evenly over the SMs: cost = rounds x (tiles per item + ~2 tiles of per-item
+  // setup: query block load, pipeline fill), the fewest splits winning ties.
+  const int sms = num_sms();
+  int best_split = 1;
+  double best_cost = 1e300;
+  for (int ns = 1; ns <= (ntiles < 64 ? ntiles : 64); ++ns) {
+    const int per = (ntiles + ns - 1) / ns;
+    const long long items = static_cast<long long>(nqb) * ((ntiles + per - 1) / per);
+    const double cost = static_cast<double>((items + sms - 1) / sms) * (per + 2.0);
+    if (cost < best_cost - 1e-9) { best_cost = cost; best_split = per; }
+  }
+  p.split_tiles = best_split;
   p.nsplit = (ntiles + p.split_tiles - 1) / p.split_tiles;
   p.n_items = nqb * p.nsplit;
+  const int grid = p.n_items < sms ? p.n_items : sms;
   if (H_I == 64)
-    return launch_indexer<64, 128, 4, 4, 1, 4, 2, kModeScores>(q_idx, T, k_idx, S, p, p.n_items, st);
-  return launch_indexer<4, 64, 64, 4, 1, 4, 2, kModeScores>(q_idx, T, k_idx, S, p, p.n_items, st);
+    return launch_indexer<64, 128, 4, 4, 1, 4, 2, kModeScores>(q_idx, T, k_idx, S, p, grid, st);
+  return launch_indexer<4, 64, 64, 4, 1, 4, 2, kModeScores>(q_idx, T, k_idx, S, p, grid, st);
 }
 
 dsa_status_t run_topk(const float* scores, long long ld, const long long* row_off, const int* row_len, int pos0,

@@ -5,6 +5,8 @@
 // the k-th largest entry, which is "score descending, smaller column first on ties".  Rows with n <= k select
 // every column.
 //
+// Sampled path (rows of 16384+ keys): see below; it reads the row about 1.1 times and falls back to the exact
+// paths when its estimate does not hold.
 // Fast path (two passes over the row): a 2048-bin histogram of the top 11 key bits gives the bin b* that
 // holds the k-th largest key; a second pass appends every entry with bin >= b* (k entries plus the rest of
 // bin b*) to shared memory, each warp owning a contiguous segment of the row and its own region, so the
@@ -35,6 +37,7 @@ constexpr int kTopkThreads = 512;
 constexpr int kTopkWarps = kTopkThreads / 32;
 constexpr int kTopkBins = 2048;            // top 11 key bits
 constexpr int kTopkRegion = 384;           // candidates per warp region (fast path)
+constexpr int kTopkSampleMin = 16384;      // rows at least this long take the sampled path
 
 struct TopkSmem {
   uint32_t hist[kTopkWarps][256];          // fallback: per-warp histograms
@@ -101,6 +104,99 @@ __device__ __forceinline__ uint32_t radix_select(Get get, int n, uint32_t prefix
   return prefix;
 }
 
+// The bin (top 11 key bits) holding the kk-th largest counted key, from the histogram sm.bins: sets sm.s_bin
+// (0xFFFFFFFF when fewer than kk keys were counted) and sm.s_need (keys of that bin still to take).  Thread t
+// owns bins 2047 - 4t .. 2044 - 4t (descending order).  Every thread of the CTA calls this.
+__device__ __forceinline__ void topk_find_bin(uint32_t kk, TopkSmem& sm) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  if (tid == 0) sm.s_bin = 0xFFFFFFFFu;
+  uint32_t c4[4], tot = 0;
+#pragma unroll
+  for (int j = 0; j < 4; ++j) { c4[j] = sm.bins[kTopkBins - 1 - 4 * tid - j]; tot += c4[j]; }
+  uint32_t incl = tot;
+#pragma unroll
+  for (int d = 1; d < 32; d <<= 1) {
+    const uint32_t v = __shfl_up_sync(0xffffffffu, incl, d);
+    if (lane >= d) incl += v;
+  }
+  if (lane == 31) sm.s_gt[warp] = static_cast<int>(incl);
+  __syncthreads();
+  uint32_t wbase = 0;
+  for (int w = 0; w < warp; ++w) wbase += static_cast<uint32_t>(sm.s_gt[w]);
+  const uint32_t excl = wbase + incl - tot;
+  if (excl < kk && kk <= excl + tot) {
+    uint32_t run = excl;
+    int j = 0;
+    for (; j < 4; ++j) {
+      if (run + c4[j] >= kk) break;
+      run += c4[j];
+    }
+    sm.s_bin = static_cast<uint32_t>(kTopkBins - 1 - 4 * tid - j);
+    sm.s_need = kk - run;
+  }
+  __syncthreads();
+}
+
+// Pass over a 16-byte aligned row appending every key of bin >= bmin, in column order, to the per-warp regions
+// (warp w owns columns w * seg .. + seg - 1, seg a multiple of four; lane l reads columns i0 + 4l .. + 3).
+// Sets sm.region_n, sm.s_eq[w] = the warp's uncapped candidate count and sm.s_overflow.
+__device__ __forceinline__ void topk_collect_vec(const float* x, int n, uint32_t bmin, TopkSmem& sm) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int seg = (((n + kTopkWarps - 1) / kTopkWarps) + 3) & ~3;
+  const int seg0 = min(n, warp * seg), seg1 = min(n, seg0 + seg);
+  const uint32_t lt = (1u << lane) - 1;
+  int cnt = 0;
+  constexpr int U = 4;                       // 128-key steps whose loads are in flight together
+  for (int i00 = seg0; i00 < seg1; i00 += U * 128) {
+    float4 vv[U];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int c0 = i00 + 128 * u + 4 * lane;
+      if (c0 + 3 < seg1) {
+        vv[u] = __ldcs(reinterpret_cast<const float4*>(x + c0));   // last read of the row
+      } else {
+        vv[u].x = (c0 + 0 < seg1) ? x[c0 + 0] : 0.f;
+        vv[u].y = (c0 + 1 < seg1) ? x[c0 + 1] : 0.f;
+        vv[u].z = (c0 + 2 < seg1) ? x[c0 + 2] : 0.f;
+        vv[u].w = (c0 + 3 < seg1) ? x[c0 + 3] : 0.f;
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+    const int c0 = i00 + 128 * u + 4 * lane;
+    const float xv[4] = {vv[u].x, vv[u].y, vv[u].z, vv[u].w};
+    uint32_t key[4];
+    bool c[4];
+    int before = 0, total = 0;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      key[j] = order_key(xv[j]);
+      c[j] = c0 + j < seg1 && (key[j] >> 21) >= bmin;
+      const uint32_t m = __ballot_sync(0xffffffffu, c[j]);
+      before += __popc(m & lt);
+      total += __popc(m);
+    }
+    int pos = cnt + before;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      if (c[j]) {
+        if (pos < kTopkRegion) {
+          sm.cand_key[warp][pos] = key[j];
+          sm.cand_idx[warp][pos] = c0 + j;
+        }
+        ++pos;
+      }
+    }
+    cnt += total;
+    }
+  }
+  if (lane == 0) {
+    sm.region_n[warp] = min(cnt, kTopkRegion);
+    sm.s_eq[warp] = cnt;
+    if (cnt > kTopkRegion) atomicOr(&sm.s_overflow, 1u);
+  }
+}
+
 __global__ void __launch_bounds__(kTopkThreads) topk_rows_kernel(const TopkParams p) {
   extern __shared__ __align__(16) uint8_t topk_smem_raw[];
   TopkSmem& sm = *reinterpret_cast<TopkSmem*>(topk_smem_raw);
@@ -122,46 +218,93 @@ __global__ void __launch_bounds__(kTopkThreads) topk_rows_kernel(const TopkParam
   }
   const int seg = (n + kTopkWarps - 1) / kTopkWarps;
   const int seg0 = min(n, warp * seg), seg1 = min(n, seg0 + seg);
+  uint32_t T = 0, need = 0;
+  bool from_row = false;      // the compaction streams the row instead of the candidates
+  bool have_T = false;
 
+  // ---------------------------------------------------------------- sampled path (long 16-byte aligned rows)
+  // A histogram of one eighth of the row (128-key blocks every 1024 keys) picks a bin b_est low enough that,
+  // with a 1.5x margin, at least k keys of the row lie in bins >= b_est; one pass then collects those keys and
+  // counts them exactly.  When they are at least k (and fit), the k-th largest key is among them, and the
+  // exact selection runs on the candidates alone: the row is read about 1.1 times instead of twice, with an
+  // eighth of the histogram atomics.  Otherwise the exact path below runs.
+  if ((reinterpret_cast<uintptr_t>(x) & 15) == 0 && n >= kTopkSampleMin) {
+    for (int i = tid; i < kTopkBins; i += kTopkThreads) sm.bins[i] = 0;
+    if (tid == 0) sm.s_overflow = 0;
+    __syncthreads();
+    const int nblk = n >> 10;
+    for (int b0 = warp; b0 < nblk; b0 += 4 * kTopkWarps) {
+      float4 v[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int b = b0 + u * kTopkWarps;
+        if (b < nblk) v[u] = reinterpret_cast<const float4*>(x + (static_cast<long long>(b) << 10))[lane];
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        if (b0 + u * kTopkWarps >= nblk) break;
+        atomicAdd(&sm.bins[order_key(v[u].x) >> 21], 1u);
+        atomicAdd(&sm.bins[order_key(v[u].y) >> 21], 1u);
+        atomicAdd(&sm.bins[order_key(v[u].z) >> 21], 1u);
+        atomicAdd(&sm.bins[order_key(v[u].w) >> 21], 1u);
+      }
+    }
+    __syncthreads();
+    topk_find_bin((3u * static_cast<uint32_t>(k) + 15u) / 16u + 16u, sm);
+    const uint32_t b_est = sm.s_bin;
+    if (b_est != 0xFFFFFFFFu && b_est >= 1) {
+      topk_collect_vec(x, n, b_est, sm);
+      __syncthreads();
+      int total = 0;
+      for (int w = 0; w < kTopkWarps; ++w) total += sm.s_eq[w];
+      if (!sm.s_overflow && total >= k) {
+        need = static_cast<uint32_t>(k);
+        auto get = [&](int i) -> uint32_t {
+          const int w = i / kTopkRegion, j = i % kTopkRegion;
+          return (j < sm.region_n[w]) ? sm.cand_key[w][j] : 0u;   // padding: the lowest key (all bins >= 1)
+        };
+        T = radix_select(get, kTopkWarps * kTopkRegion, 0u, 0u, 24, need, sm);
+        have_T = true;
+      }
+    }
+    __syncthreads();
+  }
+
+  if (!have_T) {
   // ---------------------------------------------------------------- fast path, pass 1: top-11-bit histogram
   for (int i = tid; i < kTopkBins; i += kTopkThreads) sm.bins[i] = 0;
   if (tid == 0) sm.s_overflow = 0;
   __syncthreads();
-  for (int i = tid; i < n; i += kTopkThreads) atomicAdd(&sm.bins[order_key(x[i]) >> 21], 1u);
-  __syncthreads();
-  // bin b* holding the k-th largest key: thread t owns bins 2047-4t .. 2044-4t (descending order)
-  {
-    uint32_t c4[4], tot = 0;
+  if ((reinterpret_cast<uintptr_t>(x) & 15) == 0) {
+    const float4* x4 = reinterpret_cast<const float4*>(x);
+    const int n4 = n >> 2;
+    for (int i = tid; i < n4; i += 4 * kTopkThreads) {
+      float4 v[4];
 #pragma unroll
-    for (int j = 0; j < 4; ++j) { c4[j] = sm.bins[kTopkBins - 1 - 4 * tid - j]; tot += c4[j]; }
-    uint32_t incl = tot;
+      for (int u = 0; u < 4; ++u)
+        if (i + u * kTopkThreads < n4) v[u] = x4[i + u * kTopkThreads];
 #pragma unroll
-    for (int d = 1; d < 32; d <<= 1) {
-      const uint32_t v = __shfl_up_sync(0xffffffffu, incl, d);
-      if (lane >= d) incl += v;
-    }
-    if (lane == 31) sm.s_gt[warp] = static_cast<int>(incl);
-    __syncthreads();
-    uint32_t wbase = 0;
-    for (int w = 0; w < warp; ++w) wbase += static_cast<uint32_t>(sm.s_gt[w]);
-    const uint32_t excl = wbase + incl - tot;
-    const uint32_t kk = static_cast<uint32_t>(k);
-    if (excl < kk && kk <= excl + tot) {
-      uint32_t run = excl;
-      int j = 0;
-      for (; j < 4; ++j) {
-        if (run + c4[j] >= kk) break;
-        run += c4[j];
+      for (int u = 0; u < 4; ++u) {
+        if (i + u * kTopkThreads >= n4) break;
+        atomicAdd(&sm.bins[order_key(v[u].x) >> 21], 1u);
+        atomicAdd(&sm.bins[order_key(v[u].y) >> 21], 1u);
+        atomicAdd(&sm.bins[order_key(v[u].z) >> 21], 1u);
+        atomicAdd(&sm.bins[order_key(v[u].w) >> 21], 1u);
       }
-      sm.s_bin = static_cast<uint32_t>(kTopkBins - 1 - 4 * tid - j);
-      sm.s_need = kk - run;            // entries of bin b* still to take
     }
-    __syncthreads();
+    for (int i = 4 * n4 + tid; i < n; i += kTopkThreads) atomicAdd(&sm.bins[order_key(x[i]) >> 21], 1u);
+  } else {
+    for (int i = tid; i < n; i += kTopkThreads) atomicAdd(&sm.bins[order_key(x[i]) >> 21], 1u);
   }
+  __syncthreads();
+  // bin b* holding the k-th largest key
+  topk_find_bin(static_cast<uint32_t>(k), sm);
   const uint32_t bstar = sm.s_bin;
   const uint32_t need_bin = sm.s_need;
   // ---------------------------------------------------------------- pass 2: gather candidates in column order
-  {
+  if ((reinterpret_cast<uintptr_t>(x) & 15) == 0) {
+    topk_collect_vec(x, n, bstar, sm);
+  } else {
     int cnt = 0;
     bool over = false;
     for (int i0 = seg0; i0 < seg1; i0 += 32) {
@@ -184,8 +327,6 @@ __global__ void __launch_bounds__(kTopkThreads) topk_rows_kernel(const TopkParam
   }
   __syncthreads();
 
-  uint32_t T, need;
-  bool from_row;          // fallback: the compaction streams the row instead of the candidates
   if (!sm.s_overflow) {
     // exact threshold inside bin b*, over the candidates (shared memory only)
     need = need_bin;
@@ -201,6 +342,7 @@ __global__ void __launch_bounds__(kTopkThreads) topk_rows_kernel(const TopkParam
     auto get = [&](int i) -> uint32_t { return order_key(x[i]); };
     T = radix_select(get, n, 0u, 0u, 24, need, sm);
     from_row = true;
+  }
   }
   // ---------------------------------------------------------------- ordered compaction
   // every warp walks its own span (a contiguous row segment, or its candidate region), in column order

@@ -77,3 +77,20 @@ def test_rows_sorted_by_score_take_the_fallback_path(dsa):
     desc = asc[::-1].copy()
     blocks = np.repeat(np.arange(n // 100, dtype=np.float32), 100)    # 100-long runs of equal scores
     _check(dsa, np.stack([asc, desc, blocks, -asc]), 2048, row_len=[n, n, n, n])
+
+
+def test_long_rows_where_the_sample_misleads(dsa):
+    """Rows of 16384+ keys first estimate a threshold from one eighth of the row (128-key blocks every 1024
+    keys); rows whose sampled blocks are unrepresentative must still select exactly (the kernel falls back)."""
+    rng = np.random.default_rng(4)
+    n = 40000
+    sampled = np.zeros(n, dtype=bool)
+    for b in range(n // 1024):
+        sampled[1024 * b: 1024 * b + 128] = True
+    base = rng.normal(size=(5, n)).astype(np.float32)
+    rows = base.copy()
+    rows[0, sampled] += 10.0          # the sample sees only large scores
+    rows[1, ~sampled] += 10.0         # the sample sees only small scores
+    rows[2, rng.choice(np.flatnonzero(~sampled), 3000, replace=False)] = 50.0   # outliers outside the sample
+    rows[3] = np.round(rows[3])       # heavy ties
+    _check(dsa, rows, 2048, row_len=[n, n, n, n, n - 7])

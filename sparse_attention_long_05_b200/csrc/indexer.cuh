@@ -13,8 +13,9 @@
 //   warp 0      TMA producer: q_I block of the work item, then one k_I tile per pipeline stage
 //   warp 1      TMEM allocation + MMA issue (one elected thread)
 //   warps 2..   epilogue warpgroup(s); warp w reads TMEM lanes 32*(w % 4) .. +31
-// Two TMEM accumulators of up to 256 columns let the epilogue of one (tile, group) overlap the MMA of the
-// next.  Tiles lying wholly above the causal diagonal of every token of the item are never loaded.
+// A ring of TMEM accumulators (as many N-column ones as fit: 2 at N = 256, 8 at N = 64 in decode) lets the
+// epilogue of one (tile, group) overlap the MMAs of the next ones.  Tiles lying wholly above the causal
+// diagonal of every token of the item are never loaded.
 //
 // Work items:
 //   kModeScores  item = (block of NG*NT query rows, range of key tiles); writes scores [T, S] (tests,
@@ -76,6 +77,9 @@ struct IndexerCfg {
   static constexpr int OFF_K = OFF_Q + QBUF * NG * GBYTES;
   static constexpr int SMEM = OFF_K + KSTAGES * KBYTES + ALIGN;  // + alignment slack
   static constexpr uint32_t TMEM_COLS = 512;
+  // accumulator ring: as many N-column accumulators as tensor memory holds (2 at N = 256, 8 at N = 64), so
+  // that the MMAs run that many (token group, key tile) steps ahead of the epilogue
+  static constexpr int NACC = (512 / N) < 8 ? (512 / N) : 8;
   static constexpr uint32_t SW_LAYOUT = (D_I == 128) ? kLayoutSW128 : kLayoutSW64;
   static constexpr uint32_t SBO = (D_I == 128) ? 1024 : 512;
   static_assert(N <= 256 && N % 16 == 0, "MMA N");
@@ -85,15 +89,15 @@ struct IndexerCfg {
 };
 
 // barrier slots (8 bytes each) in the barrier area
-template <int QBUF, int KSTAGES>
+template <int QBUF, int KSTAGES, int NACC>
 struct IndexerBars {
   static constexpr int Q_FULL = 0;
   static constexpr int Q_EMPTY = Q_FULL + QBUF;
   static constexpr int K_FULL = Q_EMPTY + QBUF;
   static constexpr int K_EMPTY = K_FULL + KSTAGES;
   static constexpr int ACC_FULL = K_EMPTY + KSTAGES;
-  static constexpr int ACC_EMPTY = ACC_FULL + 2;
-  static constexpr int COUNT = ACC_EMPTY + 2;
+  static constexpr int ACC_EMPTY = ACC_FULL + NACC;
+  static constexpr int COUNT = ACC_EMPTY + NACC;
   static constexpr int OFF_TMEM = 8 * COUNT;         // u32: TMEM base address
   static constexpr int OFF_ABORT = OFF_TMEM + 4;     // int: abort flag
   static constexpr int OFF_NITEMS = OFF_TMEM + 8;    // int: number of items (decode)
@@ -153,7 +157,7 @@ __global__ void __launch_bounds__(IndexerCfg<H_I, D_I, NT, NG, QBUF, KSTAGES, EP
 indexer_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                const IndexerParams p) {
   using C = IndexerCfg<H_I, D_I, NT, NG, QBUF, KSTAGES, EPI_WG, MODE>;
-  using Bars = IndexerBars<QBUF, KSTAGES>;
+  using Bars = IndexerBars<QBUF, KSTAGES, C::NACC>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + C::ALIGN - 1) &
                                              ~static_cast<uintptr_t>(C::ALIGN - 1));
@@ -169,7 +173,7 @@ indexer_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
   if (threadIdx.x == 0) {
     for (int i = 0; i < QBUF; ++i) { mbar_init(bar(Bars::Q_FULL + i), 1); mbar_init(bar(Bars::Q_EMPTY + i), 1); }
     for (int i = 0; i < KSTAGES; ++i) { mbar_init(bar(Bars::K_FULL + i), 1); mbar_init(bar(Bars::K_EMPTY + i), 1); }
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < C::NACC; ++i) {
       mbar_init(bar(Bars::ACC_FULL + i), 1);
       mbar_init(bar(Bars::ACC_EMPTY + i), C::NUM_EPI_WARPS);
     }
@@ -241,7 +245,7 @@ indexer_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     // ------------------------------------------------------------------ MMA issue
     if (lane == 0) {
       Pipe<KSTAGES> kp;
-      Pipe<2> ap;
+      Pipe<C::NACC> ap;
       constexpr uint32_t idesc = idesc_e4m3(128, C::N);
       int qi = 0;
       bool ok = true;
@@ -260,7 +264,7 @@ indexer_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             if (!mbar_wait(bar(Bars::ACC_EMPTY + ap.stage), ap.phase ^ 1, abort_flag)) { ok = false; break; }
             tc_fence_after();
             const uint64_t bdesc = smem_desc(q_s + (qb * NG + g) * C::GBYTES, 16, C::SBO, C::SW_LAYOUT);
-            const uint32_t d = tmem_base + ap.stage * 256;
+            const uint32_t d = tmem_base + ap.stage * C::N;
 #pragma unroll
             for (int kk = 0; kk < D_I / 32; ++kk)   // K = 32 e4m3 (32 bytes) per instruction
               mma_f8_ss(d, adesc + 2 * kk, bdesc + 2 * kk, idesc, kk > 0 ? 1u : 0u);
@@ -288,7 +292,7 @@ indexer_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     const int ethreads = 32 * C::NUM_EPI_WARPS;
     const int etid = e * 32 + lane;
     const uint32_t lane_addr = static_cast<uint32_t>(quad * 32) << 16;
-    Pipe<2> ap;
+    Pipe<C::NACC> ap;
     int qi = 0;
     bool ok = true;
     for (int item = blockIdx.x; item < n_items && ok; item += gridDim.x, ++qi) {
@@ -333,7 +337,7 @@ indexer_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
           for (int tk = 0; tk < TOKS; ++tk)
 #pragma unroll
             for (int q = 0; q < P; ++q) acc[tk][q] = 0.f;
-          const uint32_t tcol = tmem_base + ap.stage * 256 + half * CPT;
+          const uint32_t tcol = tmem_base + ap.stage * C::N + half * CPT;
           if constexpr (kPacked) {
             uint64_t acc2[TOKS][2];
 #pragma unroll

@@ -36,7 +36,8 @@ struct TopkParams {
 constexpr int kTopkThreads = 512;
 constexpr int kTopkWarps = kTopkThreads / 32;
 constexpr int kTopkBins = 2048;            // top 11 key bits
-constexpr int kTopkRegion = 384;           // candidates per warp region (fast path)
+constexpr int kTopkRegion = 640;           // candidates per warp region (the kernel's 64 registers per thread
+                                           // allow two CTAs per SM; 640 still fits two in shared memory)
 constexpr int kTopkSampleMin = 16384;      // rows at least this long take the sampled path
 
 struct TopkSmem {
@@ -138,57 +139,58 @@ __device__ __forceinline__ void topk_find_bin(uint32_t kk, TopkSmem& sm) {
 }
 
 // Pass over a 16-byte aligned row appending every key of bin >= bmin, in column order, to the per-warp regions
-// (warp w owns columns w * seg .. + seg - 1, seg a multiple of four; lane l reads columns i0 + 4l .. + 3).
-// Sets sm.region_n, sm.s_eq[w] = the warp's uncapped candidate count and sm.s_overflow.
+// (warp w owns columns w * seg .. + seg - 1, seg a multiple of four).  A key is in bin >= bmin exactly when the
+// score is >= the float whose order key is bmin << 21, so the pass compares raw scores and forms order keys
+// for the candidates only.  Lane l takes 16 consecutive columns of each 512-column step (four loads in
+// flight); one warp scan of the lanes' counts places the candidates.  Sets sm.region_n, sm.s_eq[w] = the
+// warp's uncapped candidate count and sm.s_overflow.
 __device__ __forceinline__ void topk_collect_vec(const float* x, int n, uint32_t bmin, TopkSmem& sm) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int seg = (((n + kTopkWarps - 1) / kTopkWarps) + 3) & ~3;
   const int seg0 = min(n, warp * seg), seg1 = min(n, seg0 + seg);
-  const uint32_t lt = (1u << lane) - 1;
+  const uint32_t kk = bmin << 21;
+  uint32_t tb = (kk & 0x80000000u) ? (kk & 0x7FFFFFFFu) : ~kk;
+  if (!(kk & 0x80000000u) && tb > 0xFF800000u) tb = 0xFF800000u;   // no float key lies below that of -inf
+  const float thr = __uint_as_float(tb);
   int cnt = 0;
-  constexpr int U = 4;                       // 128-key steps whose loads are in flight together
-  for (int i00 = seg0; i00 < seg1; i00 += U * 128) {
-    float4 vv[U];
+  for (int i00 = seg0; i00 < seg1; i00 += 512) {
+    const int c0 = i00 + 16 * lane;
+    float xv[16];
 #pragma unroll
-    for (int u = 0; u < U; ++u) {
-      const int c0 = i00 + 128 * u + 4 * lane;
-      if (c0 + 3 < seg1) {
-        vv[u] = __ldcs(reinterpret_cast<const float4*>(x + c0));   // last read of the row
+    for (int u = 0; u < 4; ++u) {
+      const int col = c0 + 4 * u;
+      if (col + 3 < seg1) {
+        const float4 v = __ldcs(reinterpret_cast<const float4*>(x + col));   // last read of the row
+        xv[4 * u] = v.x; xv[4 * u + 1] = v.y; xv[4 * u + 2] = v.z; xv[4 * u + 3] = v.w;
       } else {
-        vv[u].x = (c0 + 0 < seg1) ? x[c0 + 0] : 0.f;
-        vv[u].y = (c0 + 1 < seg1) ? x[c0 + 1] : 0.f;
-        vv[u].z = (c0 + 2 < seg1) ? x[c0 + 2] : 0.f;
-        vv[u].w = (c0 + 3 < seg1) ? x[c0 + 3] : 0.f;
+#pragma unroll
+        for (int e = 0; e < 4; ++e) xv[4 * u + e] = (col + e < seg1) ? x[col + e] : -INFINITY;
       }
     }
+    int c = 0;
 #pragma unroll
-    for (int u = 0; u < U; ++u) {
-    const int c0 = i00 + 128 * u + 4 * lane;
-    const float xv[4] = {vv[u].x, vv[u].y, vv[u].z, vv[u].w};
-    uint32_t key[4];
-    bool c[4];
-    int before = 0, total = 0;
+    for (int e = 0; e < 16; ++e) c += (c0 + e < seg1 && xv[e] >= thr) ? 1 : 0;
+    int incl = c;
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      key[j] = order_key(xv[j]);
-      c[j] = c0 + j < seg1 && (key[j] >> 21) >= bmin;
-      const uint32_t m = __ballot_sync(0xffffffffu, c[j]);
-      before += __popc(m & lt);
-      total += __popc(m);
+    for (int d = 1; d < 32; d <<= 1) {
+      const int v = __shfl_up_sync(0xffffffffu, incl, d);
+      if (lane >= d) incl += v;
     }
-    int pos = cnt + before;
+    const int tot = __shfl_sync(0xffffffffu, incl, 31);
+    if (c) {
+      int pos = cnt + incl - c;
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      if (c[j]) {
-        if (pos < kTopkRegion) {
-          sm.cand_key[warp][pos] = key[j];
-          sm.cand_idx[warp][pos] = c0 + j;
+      for (int e = 0; e < 16; ++e) {
+        if (c0 + e < seg1 && xv[e] >= thr) {
+          if (pos < kTopkRegion) {
+            sm.cand_key[warp][pos] = order_key(xv[e]);
+            sm.cand_idx[warp][pos] = c0 + e;
+          }
+          ++pos;
         }
-        ++pos;
       }
     }
-    cnt += total;
-    }
+    cnt += tot;
   }
   if (lane == 0) {
     sm.region_n[warp] = min(cnt, kTopkRegion);
@@ -224,7 +226,7 @@ __global__ void __launch_bounds__(kTopkThreads) topk_rows_kernel(const TopkParam
 
   // ---------------------------------------------------------------- sampled path (long 16-byte aligned rows)
   // A histogram of one eighth of the row (128-key blocks every 1024 keys) picks a bin b_est low enough that,
-  // with a 1.5x margin, at least k keys of the row lie in bins >= b_est; one pass then collects those keys and
+  // with a 2x margin, at least k keys of the row lie in bins >= b_est; one pass then collects those keys and
   // counts them exactly.  When they are at least k (and fit), the k-th largest key is among them, and the
   // exact selection runs on the candidates alone: the row is read about 1.1 times instead of twice, with an
   // eighth of the histogram atomics.  Otherwise the exact path below runs.
@@ -250,7 +252,7 @@ __global__ void __launch_bounds__(kTopkThreads) topk_rows_kernel(const TopkParam
       }
     }
     __syncthreads();
-    topk_find_bin((3u * static_cast<uint32_t>(k) + 15u) / 16u + 16u, sm);
+    topk_find_bin(static_cast<uint32_t>(k) / 4u + 16u, sm);   // k / 8 sampled keys with a 2x margin
     const uint32_t b_est = sm.s_bin;
     if (b_est != 0xFFFFFFFFu && b_est >= 1) {
       topk_collect_vec(x, n, b_est, sm);

@@ -72,19 +72,34 @@ def max_over_ranks(x: float, ws: int) -> float:
     return float(t.item())
 
 
-def attention_traffic(tokens):
-    """DRAM bytes of one sparse-MLA launch over `tokens` query tokens, scaled from the committed ncu capture
-    (profiles/traffic.json); None once the kernel source differs from the one that capture measured."""
+def _traffic_entry(name, files):
+    """The committed ncu traffic figure of a kernel (profiles/traffic.json), or None once its source differs
+    from the one that capture measured."""
     import hashlib
     try:
-        t = json.load(open(os.path.join(ROOT, "profiles", "traffic.json")))["sparse_mla_attn"]
-        src = b"".join(open(os.path.join(ROOT, "sparse_attention_long_05_b200", "csrc", f), "rb").read()
-                       for f in ("sparse_mla.cuh", "common.cuh"))
+        t = json.load(open(os.path.join(ROOT, "profiles", "traffic.json")))[name]
+        src = b"".join(open(os.path.join(ROOT, "sparse_attention_long_05_b200", "csrc", f), "rb").read() for f in files)
         if hashlib.sha256(src).hexdigest()[:16] != t["source_sha256_16"]:
             return None
-        return t["dram_bytes_per_query_token"] * tokens
+        return t
     except (OSError, KeyError, ValueError):
         return None
+
+
+def attention_traffic(tokens):
+    """DRAM bytes of one sparse-MLA launch over `tokens` query tokens, scaled from the committed capture."""
+    t = _traffic_entry("sparse_mla_attn", ("sparse_mla.cuh", "common.cuh"))
+    return None if t is None else t["dram_bytes_per_query_token"] * tokens
+
+
+def select_traffic(L, rows_per_block):
+    """DRAM bytes of the indexer + top-k of one prefill step (materialised score blocks of rows_per_block rows
+    against the keys up to each block's end), scaled from the committed capture."""
+    t = _traffic_entry("prefill_select", ("indexer.cuh", "topk.cuh", "common.cuh"))
+    if t is None:
+        return None
+    scores = sum(min(rows_per_block, L - r0) * min(L, r0 + rows_per_block) for r0 in range(0, L, rows_per_block))
+    return t["dram_bytes_per_score"] * scores
 
 
 def peaks():
@@ -246,7 +261,8 @@ def bench_prefill(dsa, cfg, steps, warmup, ws_n, rank, pk):
     dom = max(kernels, key=lambda n: kernels[n]["ms"])
     d = kernels[dom]
     roof = {"kernel": dom, "bound": d["bound"], "achieved": d["achieved"], "peak": d["peak"], "unit": d["unit"],
-            "frac": d["frac"], "traffic": attention_traffic(L) if dom == "sparse_mla_attn" else None,
+            "frac": d["frac"],
+            "traffic": attention_traffic(L) if dom == "sparse_mla_attn" else select_traffic(L, prefill_chunk_rows(L)),
             "peak_source": f"{pk['source']} bf16 sustained" + (" x2 (FP8)" if dom == "prefill_select" else "")}
     del x
     return {"ms": ms, "tokens_per_s": ws_n * L / (ms * 1e-3), "roofline": roof, "kernels": kernels,

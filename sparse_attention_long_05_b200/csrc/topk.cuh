@@ -51,20 +51,20 @@ struct TopkSmem {
   int s_out_base[kTopkWarps], s_eq_base[kTopkWarps];
 };
 
-// Radix select on 32-bit keys among the entries of `get(i)`, i < n, that match (key & mask) == prefix:
-// returns the exact k-th largest key and sets `need` to the number of entries equal to it that are taken.
-// hist is a [kTopkWarps][256] shared scratch; every thread of the CTA calls this.
-template <typename Get>
-__device__ __forceinline__ uint32_t radix_select(Get get, int n, uint32_t prefix, uint32_t mask, int first_shift,
+// Radix select on 32-bit keys among the entries that match (key & mask) == prefix: returns the exact k-th
+// largest key and sets `need` to the number of entries equal to it that are taken.  each(visit) calls
+// visit(key) for every entry this thread owns.  hist is a [kTopkWarps][256] shared scratch; every thread of the
+// CTA calls this.
+template <typename Each>
+__device__ __forceinline__ uint32_t radix_select(Each each, uint32_t prefix, uint32_t mask, int first_shift,
                                                  uint32_t& need, TopkSmem& sm) {
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   for (int shift = first_shift; shift >= 0; shift -= 8) {
     for (int i = lane; i < 256; i += 32) sm.hist[warp][i] = 0;
     __syncthreads();
-    for (int i = tid; i < n; i += kTopkThreads) {
-      const uint32_t key = get(i);
+    each([&](uint32_t key) {
       if ((key & mask) == prefix) atomicAdd(&sm.hist[warp][(key >> shift) & 255], 1u);
-    }
+    });
     __syncthreads();
     if (warp == 0) {
       // lane l owns bins 255-8l .. 248-8l (descending); totals over warps
@@ -261,11 +261,11 @@ __global__ void __launch_bounds__(kTopkThreads) topk_rows_kernel(const TopkParam
       for (int w = 0; w < kTopkWarps; ++w) total += sm.s_eq[w];
       if (!sm.s_overflow && total >= k) {
         need = static_cast<uint32_t>(k);
-        auto get = [&](int i) -> uint32_t {
-          const int w = i / kTopkRegion, j = i % kTopkRegion;
-          return (j < sm.region_n[w]) ? sm.cand_key[w][j] : 0u;   // padding: the lowest key (all bins >= 1)
+        // every warp visits its own candidate region
+        auto each = [&](auto visit) {
+          for (int j = lane; j < sm.region_n[warp]; j += 32) visit(sm.cand_key[warp][j]);
         };
-        T = radix_select(get, kTopkWarps * kTopkRegion, 0u, 0u, 24, need, sm);
+        T = radix_select(each, 0u, 0u, 24, need, sm);
         have_T = true;
       }
     }
@@ -332,17 +332,17 @@ __global__ void __launch_bounds__(kTopkThreads) topk_rows_kernel(const TopkParam
   if (!sm.s_overflow) {
     // exact threshold inside bin b*, over the candidates (shared memory only)
     need = need_bin;
-    const uint32_t pad = (bstar == kTopkBins - 1) ? 0u : 0xFFFFFFFFu;   // a key outside bin b*
-    auto get = [&](int i) -> uint32_t {
-      const int w = i / kTopkRegion, j = i % kTopkRegion;
-      return (j < sm.region_n[w]) ? sm.cand_key[w][j] : pad;
+    auto each = [&](auto visit) {
+      for (int j = lane; j < sm.region_n[warp]; j += 32) visit(sm.cand_key[warp][j]);
     };
-    T = radix_select(get, kTopkWarps * kTopkRegion, bstar << 21, 0xFFE00000u, 16, need, sm);
+    T = radix_select(each, bstar << 21, 0xFFE00000u, 16, need, sm);
     from_row = false;
   } else {
     need = static_cast<uint32_t>(k);
-    auto get = [&](int i) -> uint32_t { return order_key(x[i]); };
-    T = radix_select(get, n, 0u, 0u, 24, need, sm);
+    auto each = [&](auto visit) {
+      for (int i = tid; i < n; i += kTopkThreads) visit(order_key(x[i]));
+    };
+    T = radix_select(each, 0u, 0u, 24, need, sm);
     from_row = true;
   }
   }

@@ -70,8 +70,9 @@ struct IndexerCfg {
   static constexpr int ALIGN = 1024;
   // shared memory map (offsets from a 1024-byte aligned base)
   static constexpr int OFF_BAR = 0;                  // barriers + misc (2 KB)
-  static constexpr int OFF_PREFIX = 2048;            // decode: per-sequence item prefix (4 KB)
-  static constexpr int OFF_W = ((OFF_PREFIX + (MODE == kModeDecode ? 4 * (kMaxDecodeSeqs + 1) : 0) + 15) / 16) * 16;
+  static constexpr int OFF_PREFIX = 2048;            // decode: per-sequence item prefix, key counts, cache offsets
+  static constexpr int DEC_BYTES = 4 * (kMaxDecodeSeqs + 1) + 4 * kMaxDecodeSeqs + 8 * kMaxDecodeSeqs + 8;
+  static constexpr int OFF_W = ((OFF_PREFIX + (MODE == kModeDecode ? DEC_BYTES : 0) + 15) / 16) * 16;
   static constexpr int W_FLOATS = TOK * H_I;
   static constexpr int OFF_Q = ((OFF_W + QBUF * W_FLOATS * 4 + ALIGN - 1) / ALIGN) * ALIGN;
   static constexpr int OFF_K = OFF_Q + QBUF * NG * GBYTES;
@@ -125,15 +126,17 @@ __device__ __forceinline__ IndexerItem indexer_item(const IndexerParams& p, int 
       if (prefix[mid] <= i) lo = mid; else hi = mid - 1;
     }
     const int b = lo;
-    const int n = p.ctx_len[b] + 1;
+    const int* n1s = prefix + kMaxDecodeSeqs + 1;
+    const long long* offs = reinterpret_cast<const long long*>(n1s + kMaxDecodeSeqs + 1);   // 8-byte aligned
+    const int n = n1s[b];
     it.q_row0 = b;
     it.n_tok = 1;
     it.pos0 = n - 1;
     it.n_keys = n;
-    it.key_row0 = p.cache_off[b];
+    it.key_row0 = offs[b];
     it.tile0 = (i - prefix[b]) * p.chunk_tiles;
     it.tile1 = min(it.tile0 + p.chunk_tiles, (n + 127) / 128);
-    it.out_base = p.cache_off[b];
+    it.out_base = offs[b];
   }
   return it;
 }
@@ -178,17 +181,43 @@ indexer_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
       mbar_init(bar(Bars::ACC_EMPTY + i), C::NUM_EPI_WARPS);
     }
     *abort_flag = 0;
-    if constexpr (MODE == kModeDecode) {
-      int tot = 0;
-      for (int b = 0; b < p.T; ++b) {
-        prefix[b] = tot;
-        const int tiles = (p.ctx_len[b] + 1 + 127) / 128;
-        tot += (tiles + p.chunk_tiles - 1) / p.chunk_tiles;
-      }
-      prefix[p.T] = tot;
-      *reinterpret_cast<int*>(smem + Bars::OFF_NITEMS) = tot;
-    }
     fence_mbar_init();
+  }
+  if constexpr (MODE == kModeDecode) {
+    // per sequence: keys n_b + 1, cache offset and work items, loaded by all threads in parallel; then an
+    // exclusive scan of the item counts by warp 0 (items of sequence b are prefix[b] .. prefix[b + 1] - 1)
+    int* n1s = prefix + kMaxDecodeSeqs + 1;
+    long long* offs = reinterpret_cast<long long*>(n1s + kMaxDecodeSeqs + 1);
+    int* cnts = prefix + 1;          // counts first, scanned in place below
+    for (int b = threadIdx.x; b < p.T; b += blockDim.x) {
+      const int n1 = p.ctx_len[b] + 1;
+      n1s[b] = n1;
+      offs[b] = p.cache_off[b];
+      const int tiles = (n1 + 127) / 128;
+      cnts[b] = (tiles + p.chunk_tiles - 1) / p.chunk_tiles;
+    }
+    __syncthreads();
+    if (warp == 0) {
+      int carry = 0;
+      for (int b0 = 0; b0 < p.T; b0 += 32) {
+        const int b = b0 + lane;
+        const int c = (b < p.T) ? cnts[b] : 0;
+        int incl = c;
+#pragma unroll
+        for (int d = 1; d < 32; d <<= 1) {
+          const int v = __shfl_up_sync(0xffffffffu, incl, d);
+          if (lane >= d) incl += v;
+        }
+        __syncwarp();
+        if (b < p.T) prefix[b + 1] = carry + incl;    // cnts[b] aliases prefix[b + 1]: read before written
+        carry += __shfl_sync(0xffffffffu, incl, 31);
+        __syncwarp();
+      }
+      if (lane == 0) {
+        prefix[0] = 0;
+        *reinterpret_cast<int*>(smem + Bars::OFF_NITEMS) = carry;
+      }
+    }
   }
   if (warp == 0 && lane == 0) { prefetch_tmap(&tm_q); prefetch_tmap(&tm_k); }
   if (warp == 1) {
@@ -310,11 +339,18 @@ indexer_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         wq[i] = v;
       }
       named_bar_sync(1, ethreads);
+      // key scales are loaded one tile ahead: a load issued at the start of its own tile would expose the
+      // global-memory latency once per tile (the epilogue needs it a few hundred cycles later)
+      auto kscale_of = [&](int tile) -> float {
+        const int s = tile * 128 + quad * 32 + lane;
+        return (p.k_scale && tile < it.tile1 && s < it.n_keys) ? p.k_scale[it.key_row0 + s] : 1.f;
+      };
+      float kscale_next = kscale_of(it.tile0);
       for (int tile = it.tile0; tile < it.tile1; ++tile) {
         const int s = tile * 128 + quad * 32 + lane;      // key of this thread
         const bool key_ok = s < it.n_keys;
-        float kscale = 1.f;
-        if (p.k_scale && key_ok) kscale = p.k_scale[it.key_row0 + s];
+        const float kscale = kscale_next;
+        kscale_next = kscale_of(tile + 1);
         for (int g = 0; g < NG; ++g) {
           if (g * NT >= it.n_tok) break;
           const int tok0 = g * NT + half * (CPT / H_I > 0 ? CPT / H_I : 0);  // first row of this thread

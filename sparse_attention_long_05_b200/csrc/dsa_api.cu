@@ -95,8 +95,8 @@ dsa_status_t last_launch_status() {
 size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 // ------------------------------------------------------------------------------------------ launchers
-// One CTA per SM: the indexer allocates all 512 TMEM columns, so at least 120 KB of shared memory is
-// requested to keep a second CTA off the SM.
+// A configuration that allocates all 512 TMEM columns runs one CTA per SM: at least 120 KB of shared memory is
+// requested to keep a second CTA off the SM (its allocation would wait for the first CTA to finish).
 constexpr int kMinIndexerSmem = 120 * 1024;
 
 template <int H_I, int D_I, int NT, int NG, int QBUF, int KST, int EPI, int MODE>
@@ -113,7 +113,7 @@ dsa_status_t launch_indexer(const uint8_t* q_idx, int q_rows, const uint8_t* k_i
   if (!make_map(&tq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, q_idx, qd, qs, qb, sw)) return DSA_ERR_CUDA;
   if (!make_map(&tk, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, k_idx, kd, qs, kb, sw)) return DSA_ERR_CUDA;
   auto kern = indexer_kernel<H_I, D_I, NT, NG, QBUF, KST, EPI, MODE>;
-  const int smem = C::SMEM > kMinIndexerSmem ? C::SMEM : kMinIndexerSmem;
+  const int smem = (C::TMEM_COLS == 512 && C::SMEM < kMinIndexerSmem) ? kMinIndexerSmem : C::SMEM;
   if (set_smem(kern, smem) != cudaSuccess) return DSA_ERR_CUDA;
   kern<<<grid, C::NUM_THREADS, smem, st>>>(tq, tk, p);
   return last_launch_status();
@@ -368,7 +368,7 @@ dsa_status_t dsa_forward_decode(int B, const int64_t* cache_off, const int32_t* 
   p.cache_off = off;
   p.ctx_len = ctx_len;
   p.chunk_tiles = 16;
-  e = launch_indexer<64, 128, 1, 1, 2, 8, 1, kModeDecode>(q_idx, B, k_cache, cache_rows, p, num_sms(), st);
+  e = launch_indexer<64, 128, 1, 1, 2, 4, 1, kModeDecode>(q_idx, B, k_cache, cache_rows, p, 2 * num_sms(), st);
   if (e != DSA_OK) return e;
   e = run_topk(dscores, 0, off, len1, 0, B, k, idx, k, st);
   if (e != DSA_OK) return e;

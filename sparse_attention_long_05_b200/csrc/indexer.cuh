@@ -13,7 +13,7 @@
 //   warp 0      TMA producer: q_I block of the work item, then one k_I tile per pipeline stage
 //   warp 1      TMEM allocation + MMA issue (one elected thread)
 //   warps 2..   epilogue warpgroup(s); warp w reads TMEM lanes 32*(w % 4) .. +31
-// A ring of TMEM accumulators (as many N-column ones as fit: 2 at N = 256, 8 at N = 64 in decode) lets the
+// A ring of TMEM accumulators (2 of 256 columns; 4 of 64 in decode, two CTAs per SM) lets the
 // epilogue of one (tile, group) overlap the MMAs of the next ones.  Tiles lying wholly above the causal
 // diagonal of every token of the item are never loaded.
 //
@@ -77,10 +77,12 @@ struct IndexerCfg {
   static constexpr int OFF_Q = ((OFF_W + QBUF * W_FLOATS * 4 + ALIGN - 1) / ALIGN) * ALIGN;
   static constexpr int OFF_K = OFF_Q + QBUF * NG * GBYTES;
   static constexpr int SMEM = OFF_K + KSTAGES * KBYTES + ALIGN;  // + alignment slack
-  static constexpr uint32_t TMEM_COLS = 512;
-  // accumulator ring: as many N-column accumulators as tensor memory holds (2 at N = 256, 8 at N = 64), so
-  // that the MMAs run that many (token group, key tile) steps ahead of the epilogue
-  static constexpr int NACC = (512 / N) < 8 ? (512 / N) : 8;
+  // accumulator ring: as many N-column accumulators as tensor memory holds (2 at N = 256), so that the MMAs
+  // run that many (token group, key tile) steps ahead of the epilogue; decode keeps half of tensor memory
+  // (4 x 64 columns) so that two CTAs share an SM
+  static constexpr int NACC = (MODE == kModeDecode) ? 4 : ((512 / N) < 8 ? (512 / N) : 8);
+  static constexpr uint32_t TMEM_COLS = static_cast<uint32_t>(NACC * N);
+  static_assert(TMEM_COLS == 256 || TMEM_COLS == 512, "tensor-memory allocation (power of two)");
   static constexpr uint32_t SW_LAYOUT = (D_I == 128) ? kLayoutSW128 : kLayoutSW64;
   static constexpr uint32_t SBO = (D_I == 128) ? 1024 : 512;
   static_assert(N <= 256 && N % 16 == 0, "MMA N");

@@ -160,8 +160,16 @@ dsa_status_t run_topk(const float* scores, long long ld, const long long* row_of
                       int rows, int k, int* idx, long long idx_ld, cudaStream_t st) {
   if (rows <= 0) return DSA_OK;
   TopkParams p{scores, ld, row_off, row_len, pos0, rows, k, idx, idx_ld};
-  if (set_smem(topk_rows_kernel, static_cast<int>(sizeof(TopkSmem))) != cudaSuccess) return DSA_ERR_CUDA;
-  topk_rows_kernel<<<rows, kTopkThreads, sizeof(TopkSmem), st>>>(p);
+  if (rows < num_sms()) {
+    // fewer rows than SMs (decode): one 1024-thread CTA per row
+    if (set_smem(topk_rows_kernel<kTopkThreadsFew>, static_cast<int>(sizeof(TopkSmem<kTopkThreadsFew>))) != cudaSuccess)
+      return DSA_ERR_CUDA;
+    topk_rows_kernel<kTopkThreadsFew><<<rows, kTopkThreadsFew, sizeof(TopkSmem<kTopkThreadsFew>), st>>>(p);
+  } else {
+    if (set_smem(topk_rows_kernel<kTopkThreads>, static_cast<int>(sizeof(TopkSmem<kTopkThreads>))) != cudaSuccess)
+      return DSA_ERR_CUDA;
+    topk_rows_kernel<kTopkThreads><<<rows, kTopkThreads, sizeof(TopkSmem<kTopkThreads>), st>>>(p);
+  }
   return last_launch_status();
 }
 

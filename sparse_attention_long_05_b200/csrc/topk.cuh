@@ -33,31 +33,35 @@ struct TopkParams {
   long long idx_ld;
 };
 
+// CTA sizes: 512 threads (two CTAs per SM: the 64 registers per thread and ~107 KB of shared memory allow two)
+// when there are many rows, 1024 threads (one CTA per SM) when there are fewer rows than SMs (decode).
 constexpr int kTopkThreads = 512;
-constexpr int kTopkWarps = kTopkThreads / 32;
+constexpr int kTopkThreadsFew = 1024;
 constexpr int kTopkBins = 2048;            // top 11 key bits
-constexpr int kTopkRegion = 640;           // candidates per warp region (the kernel's 64 registers per thread
-                                           // allow two CTAs per SM; 640 still fits two in shared memory)
+constexpr int kTopkCandidates = 10240;     // candidate slots per CTA, split into one region per warp
 constexpr int kTopkSampleMin = 16384;      // rows at least this long take the sampled path
 
+template <int NT>
 struct TopkSmem {
-  uint32_t hist[kTopkWarps][256];          // fallback: per-warp histograms
-  uint32_t bins[kTopkBins];                // fast path: top-11-bit histogram
-  uint32_t cand_key[kTopkWarps][kTopkRegion];
-  int cand_idx[kTopkWarps][kTopkRegion];
-  int region_n[kTopkWarps];
+  static constexpr int W = NT / 32;
+  static constexpr int REGION = kTopkCandidates / W;   // candidates per warp region
+  uint32_t hist[W][256];                   // radix select: per-warp histograms
+  uint32_t bins[kTopkBins];                // top-11-bit histogram
+  uint32_t cand_key[W][REGION];
+  int cand_idx[W][REGION];
+  int region_n[W];
   uint32_t s_need, s_digit, s_bin, s_overflow;
-  int s_gt[kTopkWarps], s_eq[kTopkWarps];
-  int s_out_base[kTopkWarps], s_eq_base[kTopkWarps];
+  int s_gt[W], s_eq[W];
+  int s_out_base[W], s_eq_base[W];
 };
 
 // Radix select on 32-bit keys among the entries that match (key & mask) == prefix: returns the exact k-th
 // largest key and sets `need` to the number of entries equal to it that are taken.  each(visit) calls
-// visit(key) for every entry this thread owns.  hist is a [kTopkWarps][256] shared scratch; every thread of the
+// visit(key) for every entry this thread owns.  hist is a [TopkSmem<NT>::W][256] shared scratch; every thread of the
 // CTA calls this.
-template <typename Each>
+template <int NT, typename Each>
 __device__ __forceinline__ uint32_t radix_select(Each each, uint32_t prefix, uint32_t mask, int first_shift,
-                                                 uint32_t& need, TopkSmem& sm) {
+                                                 uint32_t& need, TopkSmem<NT>& sm) {
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   for (int shift = first_shift; shift >= 0; shift -= 8) {
     for (int i = lane; i < 256; i += 32) sm.hist[warp][i] = 0;
@@ -74,7 +78,7 @@ __device__ __forceinline__ uint32_t radix_select(Each each, uint32_t prefix, uin
       for (int j = 0; j < 8; ++j) {
         const int bin = 255 - 8 * lane - j;
         uint32_t c = 0;
-        for (int w = 0; w < kTopkWarps; ++w) c += sm.hist[w][bin];
+        for (int w = 0; w < TopkSmem<NT>::W; ++w) c += sm.hist[w][bin];
         cnt[j] = c;
         tot += c;
       }
@@ -107,13 +111,15 @@ __device__ __forceinline__ uint32_t radix_select(Each each, uint32_t prefix, uin
 
 // The bin (top 11 key bits) holding the kk-th largest counted key, from the histogram sm.bins: sets sm.s_bin
 // (0xFFFFFFFF when fewer than kk keys were counted) and sm.s_need (keys of that bin still to take).  Thread t
-// owns bins 2047 - 4t .. 2044 - 4t (descending order).  Every thread of the CTA calls this.
-__device__ __forceinline__ void topk_find_bin(uint32_t kk, TopkSmem& sm) {
+// owns bins 2047 - B t .. 2048 - B (t + 1), B = 2048 / threads (descending order).  Every thread of the CTA calls this.
+template <int NT>
+__device__ __forceinline__ void topk_find_bin(uint32_t kk, TopkSmem<NT>& sm) {
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   if (tid == 0) sm.s_bin = 0xFFFFFFFFu;
-  uint32_t c4[4], tot = 0;
+  constexpr int BPT = kTopkBins / NT;       // bins per thread
+  uint32_t c4[BPT], tot = 0;
 #pragma unroll
-  for (int j = 0; j < 4; ++j) { c4[j] = sm.bins[kTopkBins - 1 - 4 * tid - j]; tot += c4[j]; }
+  for (int j = 0; j < BPT; ++j) { c4[j] = sm.bins[kTopkBins - 1 - BPT * tid - j]; tot += c4[j]; }
   uint32_t incl = tot;
 #pragma unroll
   for (int d = 1; d < 32; d <<= 1) {
@@ -128,11 +134,11 @@ __device__ __forceinline__ void topk_find_bin(uint32_t kk, TopkSmem& sm) {
   if (excl < kk && kk <= excl + tot) {
     uint32_t run = excl;
     int j = 0;
-    for (; j < 4; ++j) {
+    for (; j < BPT; ++j) {
       if (run + c4[j] >= kk) break;
       run += c4[j];
     }
-    sm.s_bin = static_cast<uint32_t>(kTopkBins - 1 - 4 * tid - j);
+    sm.s_bin = static_cast<uint32_t>(kTopkBins - 1 - BPT * tid - j);
     sm.s_need = kk - run;
   }
   __syncthreads();
@@ -144,9 +150,10 @@ __device__ __forceinline__ void topk_find_bin(uint32_t kk, TopkSmem& sm) {
 // for the candidates only.  Lane l takes 16 consecutive columns of each 512-column step (four loads in
 // flight); one warp scan of the lanes' counts places the candidates.  Sets sm.region_n, sm.s_eq[w] = the
 // warp's uncapped candidate count and sm.s_overflow.
-__device__ __forceinline__ void topk_collect_vec(const float* x, int n, uint32_t bmin, TopkSmem& sm) {
+template <int NT>
+__device__ __forceinline__ void topk_collect_vec(const float* x, int n, uint32_t bmin, TopkSmem<NT>& sm) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int seg = (((n + kTopkWarps - 1) / kTopkWarps) + 3) & ~3;
+  const int seg = (((n + TopkSmem<NT>::W - 1) / TopkSmem<NT>::W) + 3) & ~3;
   const int seg0 = min(n, warp * seg), seg1 = min(n, seg0 + seg);
   const uint32_t kk = bmin << 21;
   uint32_t tb = (kk & 0x80000000u) ? (kk & 0x7FFFFFFFu) : ~kk;
@@ -182,7 +189,7 @@ __device__ __forceinline__ void topk_collect_vec(const float* x, int n, uint32_t
 #pragma unroll
       for (int e = 0; e < 16; ++e) {
         if (c0 + e < seg1 && xv[e] >= thr) {
-          if (pos < kTopkRegion) {
+          if (pos < TopkSmem<NT>::REGION) {
             sm.cand_key[warp][pos] = order_key(xv[e]);
             sm.cand_idx[warp][pos] = c0 + e;
           }
@@ -193,15 +200,16 @@ __device__ __forceinline__ void topk_collect_vec(const float* x, int n, uint32_t
     cnt += tot;
   }
   if (lane == 0) {
-    sm.region_n[warp] = min(cnt, kTopkRegion);
+    sm.region_n[warp] = min(cnt, TopkSmem<NT>::REGION);
     sm.s_eq[warp] = cnt;
-    if (cnt > kTopkRegion) atomicOr(&sm.s_overflow, 1u);
+    if (cnt > TopkSmem<NT>::REGION) atomicOr(&sm.s_overflow, 1u);
   }
 }
 
-__global__ void __launch_bounds__(kTopkThreads) topk_rows_kernel(const TopkParams p) {
+template <int NT>
+__global__ void __launch_bounds__(NT) topk_rows_kernel(const TopkParams p) {
   extern __shared__ __align__(16) uint8_t topk_smem_raw[];
-  TopkSmem& sm = *reinterpret_cast<TopkSmem*>(topk_smem_raw);
+  TopkSmem<NT>& sm = *reinterpret_cast<TopkSmem<NT>*>(topk_smem_raw);
 
   const int r = blockIdx.x;
   if (r >= p.rows) return;
@@ -215,10 +223,10 @@ __global__ void __launch_bounds__(kTopkThreads) topk_rows_kernel(const TopkParam
   int* out = p.idx + static_cast<long long>(r) * p.idx_ld;
 
   if (n <= k) {
-    for (int i = tid; i < k; i += kTopkThreads) out[i] = (i < n) ? i : -1;
+    for (int i = tid; i < k; i += NT) out[i] = (i < n) ? i : -1;
     return;
   }
-  const int seg = (n + kTopkWarps - 1) / kTopkWarps;
+  const int seg = (n + TopkSmem<NT>::W - 1) / TopkSmem<NT>::W;
   const int seg0 = min(n, warp * seg), seg1 = min(n, seg0 + seg);
   uint32_t T = 0, need = 0;
   bool from_row = false;      // the compaction streams the row instead of the candidates
@@ -231,20 +239,20 @@ __global__ void __launch_bounds__(kTopkThreads) topk_rows_kernel(const TopkParam
   // exact selection runs on the candidates alone: the row is read about 1.1 times instead of twice, with an
   // eighth of the histogram atomics.  Otherwise the exact path below runs.
   if ((reinterpret_cast<uintptr_t>(x) & 15) == 0 && n >= kTopkSampleMin) {
-    for (int i = tid; i < kTopkBins; i += kTopkThreads) sm.bins[i] = 0;
+    for (int i = tid; i < kTopkBins; i += NT) sm.bins[i] = 0;
     if (tid == 0) sm.s_overflow = 0;
     __syncthreads();
     const int nblk = n >> 10;
-    for (int b0 = warp; b0 < nblk; b0 += 4 * kTopkWarps) {
+    for (int b0 = warp; b0 < nblk; b0 += 4 * TopkSmem<NT>::W) {
       float4 v[4];
 #pragma unroll
       for (int u = 0; u < 4; ++u) {
-        const int b = b0 + u * kTopkWarps;
+        const int b = b0 + u * TopkSmem<NT>::W;
         if (b < nblk) v[u] = reinterpret_cast<const float4*>(x + (static_cast<long long>(b) << 10))[lane];
       }
 #pragma unroll
       for (int u = 0; u < 4; ++u) {
-        if (b0 + u * kTopkWarps >= nblk) break;
+        if (b0 + u * TopkSmem<NT>::W >= nblk) break;
         atomicAdd(&sm.bins[order_key(v[u].x) >> 21], 1u);
         atomicAdd(&sm.bins[order_key(v[u].y) >> 21], 1u);
         atomicAdd(&sm.bins[order_key(v[u].z) >> 21], 1u);
@@ -258,7 +266,7 @@ __global__ void __launch_bounds__(kTopkThreads) topk_rows_kernel(const TopkParam
       topk_collect_vec(x, n, b_est, sm);
       __syncthreads();
       int total = 0;
-      for (int w = 0; w < kTopkWarps; ++w) total += sm.s_eq[w];
+      for (int w = 0; w < TopkSmem<NT>::W; ++w) total += sm.s_eq[w];
       if (!sm.s_overflow && total >= k) {
         need = static_cast<uint32_t>(k);
         // every warp visits its own candidate region
@@ -274,29 +282,29 @@ __global__ void __launch_bounds__(kTopkThreads) topk_rows_kernel(const TopkParam
 
   if (!have_T) {
   // ---------------------------------------------------------------- fast path, pass 1: top-11-bit histogram
-  for (int i = tid; i < kTopkBins; i += kTopkThreads) sm.bins[i] = 0;
+  for (int i = tid; i < kTopkBins; i += NT) sm.bins[i] = 0;
   if (tid == 0) sm.s_overflow = 0;
   __syncthreads();
   if ((reinterpret_cast<uintptr_t>(x) & 15) == 0) {
     const float4* x4 = reinterpret_cast<const float4*>(x);
     const int n4 = n >> 2;
-    for (int i = tid; i < n4; i += 4 * kTopkThreads) {
+    for (int i = tid; i < n4; i += 4 * NT) {
       float4 v[4];
 #pragma unroll
       for (int u = 0; u < 4; ++u)
-        if (i + u * kTopkThreads < n4) v[u] = x4[i + u * kTopkThreads];
+        if (i + u * NT < n4) v[u] = x4[i + u * NT];
 #pragma unroll
       for (int u = 0; u < 4; ++u) {
-        if (i + u * kTopkThreads >= n4) break;
+        if (i + u * NT >= n4) break;
         atomicAdd(&sm.bins[order_key(v[u].x) >> 21], 1u);
         atomicAdd(&sm.bins[order_key(v[u].y) >> 21], 1u);
         atomicAdd(&sm.bins[order_key(v[u].z) >> 21], 1u);
         atomicAdd(&sm.bins[order_key(v[u].w) >> 21], 1u);
       }
     }
-    for (int i = 4 * n4 + tid; i < n; i += kTopkThreads) atomicAdd(&sm.bins[order_key(x[i]) >> 21], 1u);
+    for (int i = 4 * n4 + tid; i < n; i += NT) atomicAdd(&sm.bins[order_key(x[i]) >> 21], 1u);
   } else {
-    for (int i = tid; i < n; i += kTopkThreads) atomicAdd(&sm.bins[order_key(x[i]) >> 21], 1u);
+    for (int i = tid; i < n; i += NT) atomicAdd(&sm.bins[order_key(x[i]) >> 21], 1u);
   }
   __syncthreads();
   // bin b* holding the k-th largest key
@@ -315,15 +323,15 @@ __global__ void __launch_bounds__(kTopkThreads) topk_rows_kernel(const TopkParam
       const bool c = i < seg1 && (key >> 21) >= bstar;
       const uint32_t m = __ballot_sync(0xffffffffu, c);
       const int pos = cnt + __popc(m & ((1u << lane) - 1));
-      if (c && pos < kTopkRegion) {
+      if (c && pos < TopkSmem<NT>::REGION) {
         sm.cand_key[warp][pos] = key;
         sm.cand_idx[warp][pos] = i;
       }
       cnt += __popc(m);
-      if (cnt > kTopkRegion) over = true;
+      if (cnt > TopkSmem<NT>::REGION) over = true;
     }
     if (lane == 0) {
-      sm.region_n[warp] = min(cnt, kTopkRegion);
+      sm.region_n[warp] = min(cnt, TopkSmem<NT>::REGION);
       if (over) atomicOr(&sm.s_overflow, 1u);
     }
   }
@@ -340,7 +348,7 @@ __global__ void __launch_bounds__(kTopkThreads) topk_rows_kernel(const TopkParam
   } else {
     need = static_cast<uint32_t>(k);
     auto each = [&](auto visit) {
-      for (int i = tid; i < n; i += kTopkThreads) visit(order_key(x[i]));
+      for (int i = tid; i < n; i += NT) visit(order_key(x[i]));
     };
     T = radix_select(each, 0u, 0u, 24, need, sm);
     from_row = true;
@@ -366,7 +374,7 @@ __global__ void __launch_bounds__(kTopkThreads) topk_rows_kernel(const TopkParam
   __syncthreads();
   if (tid == 0) {
     int base = 0, eqb = 0;
-    for (int w = 0; w < kTopkWarps; ++w) {
+    for (int w = 0; w < TopkSmem<NT>::W; ++w) {
       sm.s_out_base[w] = base;
       sm.s_eq_base[w] = eqb;
       const int take_eq = max(0, min(sm.s_eq[w], static_cast<int>(need) - eqb));

@@ -43,15 +43,19 @@ NOMINAL_FP8_PER_BF16 = 2.0   # dense FP8 / BF16 tensor-core rate ratio (4.5 / 2.
 
 # ------------------------------------------------------------------------------------------ environment
 def dist_init():
+    """One process per GPU under torchrun: NCCL over the GPUs; gloo where no GPU is visible (host-side tests)."""
     ws = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
     if ws > 1:
         import datetime
         import torch.distributed as dist
-        torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=600),
-                                device_id=torch.device("cuda", local))
+        if torch.cuda.is_available():
+            torch.cuda.set_device(local)
+            dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=600),
+                                    device_id=torch.device("cuda", local))
+        else:
+            dist.init_process_group("gloo", timeout=datetime.timedelta(seconds=60))
     elif torch.cuda.is_available():
         torch.cuda.set_device(local)
     return ws, rank, local
@@ -64,12 +68,24 @@ def barrier(ws):
 
 
 def max_over_ranks(x: float, ws: int) -> float:
+    """The largest of every rank's x (every rank calls this, in the same order)."""
     if ws == 1:
         return x
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def replica_seed(base: int, rank: int) -> int:
+    """Each rank draws its own independent sequence (replicas, no exchange on the data path)."""
+    return base + rank
+
+
+def job_rate(units_per_rank: float, ws: int, ms_max: float) -> float:
+    """Whole-job throughput: the units all ranks processed over the slowest rank's time."""
+    return ws * units_per_rank / (ms_max * 1e-3)
 
 
 def _traffic_entry(name, files):
@@ -202,8 +218,8 @@ def prefill_chunk_rows(L):
 # ------------------------------------------------------------------------------------------ GPU arms
 def bench_prefill(dsa, cfg, steps, warmup, ws_n, rank, pk):
     dev = "cuda"
-    x = G.prefill_keys(cfg, 1000 + rank, device=dev)
-    x.update(G.prefill_queries(cfg, 1000 + rank, None, device=dev))
+    x = G.prefill_keys(cfg, replica_seed(1000, rank), device=dev)
+    x.update(G.prefill_queries(cfg, replica_seed(1000, rank), None, device=dev))
     L, k = cfg.L, cfg.k
     idx = torch.empty((L, k), dtype=torch.int32, device=dev)
     out = torch.empty((L, cfg.H, cfg.D_v), dtype=torch.bfloat16, device=dev)
@@ -265,7 +281,7 @@ def bench_prefill(dsa, cfg, steps, warmup, ws_n, rank, pk):
             "traffic": attention_traffic(L) if dom == "sparse_mla_attn" else select_traffic(L, prefill_chunk_rows(L)),
             "peak_source": f"{pk['source']} bf16 sustained" + (" x2 (FP8)" if dom == "prefill_select" else "")}
     del x
-    return {"ms": ms, "tokens_per_s": ws_n * L / (ms * 1e-3), "roofline": roof, "kernels": kernels,
+    return {"ms": ms, "tokens_per_s": job_rate(L, ws_n, ms), "roofline": roof, "kernels": kernels,
             "clocks": clk.summary(), "launches": launches}
 
 
@@ -274,8 +290,8 @@ def bench_prefill_e2e(dsa, cfg, steps, rank):
     every output inside the timed region."""
     import psutil
     dev = "cuda"
-    x = G.prefill_keys(cfg, 1000 + rank, device=dev)
-    x.update(G.prefill_queries(cfg, 1000 + rank, None, device=dev))
+    x = G.prefill_keys(cfg, replica_seed(1000, rank), device=dev)
+    x.update(G.prefill_queries(cfg, replica_seed(1000, rank), None, device=dev))
     names = ["q_idx", "q_scale", "k_idx", "k_scale", "w", "q", "c"]
     h2d = sum(x[n].numel() * x[n].element_size() for n in names if x[n] is not None)
     L, k = cfg.L, cfg.k
@@ -318,7 +334,7 @@ def bench_prefill_e2e(dsa, cfg, steps, rank):
 
 def bench_decode(dsa, cfg, steps, warmup, ws_n, rank, pk):
     dev = "cuda"
-    seed = 2000 + rank
+    seed = replica_seed(2000, rank)
     cache = G.decode_fill_cache(cfg, seed, device=dev)
     lens, offs = cache["lens"], cache["offs"]
     cache_off = torch.tensor(offs, dtype=torch.int64, device=dev)
@@ -363,7 +379,7 @@ def bench_decode(dsa, cfg, steps, warmup, ws_n, rank, pk):
     byts = decode_bytes(cfg, lens, nsteps) - decode_bytes(cfg, lens, warmup)
     gbs = byts / steps / (ms * 1e-3) / 1e9
     return {"metric": "DSA decode tokens/s (64 sequences, 4K-128K contexts, caches appended every step)",
-            "value": ws_n * B / (ms * 1e-3), "unit": "tokens/s", "ms_per_step": ms, "steps": steps,
+            "value": job_rate(B, ws_n, ms), "unit": "tokens/s", "ms_per_step": ms, "steps": steps,
             "warmup": warmup,
             "roofline": {"kernel": "decode step (append, indexer, top-k, sparse MLA)", "bound": "hbm",
                          "achieved": gbs, "peak": pk["hbm_gbs"], "unit": "GB/s", "frac": gbs / pk["hbm_gbs"],

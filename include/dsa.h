@@ -59,6 +59,17 @@ DSA_API const char* dsa_status_string(dsa_status_t status);
  * *device_status receives DSA_OK or the first device-side error since the last call. */
 DSA_API dsa_status_t dsa_get_device_status(void* stream, int* device_status);
 
+/* Self-check of failure detection: launches one small kernel whose two warps run the library's bounded
+ * pipeline wait on barriers that nothing arrives on.  Warp 0 runs out of its clock budget (about a second),
+ * which records DSA_ERR_TIMEOUT in the device status word and raises the block's abort flag; warp 1 starts
+ * waiting half a budget later and must leave on that flag.  The kernel then returns normally and the context
+ * stays usable.  result: caller-owned device array of 4 int32 (16-byte aligned), written as
+ * [warp 0 succeeded (0/1), warp 0's wait in 2^20 cycles, warp 1 succeeded, warp 1's wait in 2^20 cycles].
+ * Asynchronous on `stream`; read the status with dsa_get_device_status afterwards.  Returns
+ * DSA_ERR_INVALID_ARG for a null result, DSA_ERR_ALIGNMENT for a misaligned one, DSA_ERR_CUDA if the launch
+ * fails.  This entry point has no counterpart in the paper. */
+DSA_API dsa_status_t dsa_check_bounded_wait(int32_t* result, void* stream);
+
 /* Number of SMs the launches of the current device are sized for (148 on a B200). */
 DSA_API int dsa_num_sms(void);
 
@@ -149,6 +160,10 @@ DSA_API size_t dsa_decode_workspace_size(int B, int64_t cache_rows, int H_I, int
  *   out [B, H, 512] bf16 (out), lse [B, H] fp32 (out, may be NULL)
  * k_scale_new / k_scale_cache are always stored; pass 1.0 for unscaled (integer-valued) keys, and
  * q_scale = NULL.
+ * Sequences must own disjoint cache ranges.  A sequence with cache_off[b] < 0, ctx_len[b] < 0 or
+ * cache_off[b] + ctx_len[b] >= cache_rows sets the device status to DSA_ERR_BAD_INDEX (read it with
+ * dsa_get_device_status); nothing of its cache is read or written, its idx_out row is all -1, and the other
+ * sequences of the batch are computed as usual.
  */
 DSA_API dsa_status_t dsa_forward_decode(int B, const int64_t* cache_off, const int32_t* ctx_len, const uint8_t* q_idx,
                                 const float* q_scale, const float* w, const uint16_t* q, const uint8_t* k_new,
@@ -161,9 +176,9 @@ DSA_API dsa_status_t dsa_forward_decode(int B, const int64_t* cache_off, const i
  * dsa_forward_decode without a caller-provided workspace, for callers that cannot allocate device memory
  * (for example a serving loop that runs under a memory pool it may not grow, or code that only receives
  * borrowed buffers).  This entry point has no counterpart in the paper: it is the decode step above with its
- * scratch (per-cache-row scores, per-sequence lengths and, when idx_out is NULL, the selected indices) held
- * in a fixed device array inside the library, of dsa_decode_noalloc_scratch_bytes() bytes (32 MiB).  Every
- * GPU that loads the library keeps that array until the process exits.
+ * scratch (the packed score rows, per-sequence lengths and offsets and, when idx_out is NULL, the selected
+ * indices) held in a fixed device array inside the library, of dsa_decode_noalloc_scratch_bytes() bytes
+ * (32 MiB).  Every GPU that loads the library keeps that array until the process exits.
  *   - Arguments and results are those of dsa_forward_decode; shapes whose dsa_decode_workspace_size()
  *     exceeds the array return DSA_ERR_WORKSPACE and launch nothing.
  *   - The call allocates nothing: no cudaMalloc, no cudaFree, no allocating library routine.

@@ -5,6 +5,7 @@ The computation lives in libdsa.so (hand-written CUDA, C ABI in include/dsa.h); 
 """
 from ._lib import (  # noqa: F401
     DsaError,
+    dsa_check_bounded_wait,
     dsa_decode_noalloc_scratch_bytes,
     dsa_decode_workspace_size,
     dsa_forward_decode_noalloc,

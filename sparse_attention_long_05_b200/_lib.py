@@ -23,6 +23,7 @@ _P, _I, _I64, _F, _SZ = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_
 SIGNATURES = {
     "dsa_status_string": (ctypes.c_char_p, [_I]),
     "dsa_get_device_status": (_I, [_P, ctypes.POINTER(ctypes.c_int)]),
+    "dsa_check_bounded_wait": (_I, [_P, _P]),
     "dsa_num_sms": (_I, []),
     "dsa_indexer_scores": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P, _P]),
     "dsa_topk": (_I, [_P, _I, _I64, _P, _I, _I, _P, _P]),
@@ -88,6 +89,14 @@ def dsa_get_device_status(stream=None) -> int:
     v = ctypes.c_int(0)
     _check("dsa_get_device_status", _lib.dsa_get_device_status(_stream(stream), ctypes.byref(v)))
     return v.value
+
+
+def dsa_check_bounded_wait(stream=None):
+    """Run the bounded-wait self-check kernel (about a second) and return (result [4] int32 on the device,
+    device status).  result = [warp 0 succeeded, its wait in 2^20 cycles, warp 1 succeeded, its wait]."""
+    res = torch.full((4,), -1, dtype=torch.int32, device="cuda")
+    _check("dsa_check_bounded_wait", _lib.dsa_check_bounded_wait(_ptr(res), _stream(stream)))
+    return res, dsa_get_device_status(stream)
 
 
 def dsa_indexer_scores(q_idx, q_scale, k_idx, k_scale, w, pos0: int = 0, scores=None, stream=None):

@@ -16,19 +16,52 @@
 namespace dsa {
 
 // ------------------------------------------------------------------------------------------ decode append
-// Writes the new token's indexer key (+ scale) and latent entry at position ctx_len[b] of sequence b, and
-// n_b + 1 into len1[b] (the number of keys the new token attends to).
-__global__ void decode_append_kernel(int B, const long long* cache_off, const int* ctx_len, long long cache_rows,
-                                     const uint8_t* k_new, const float* k_scale_new, const uint16_t* c_new,
-                                     uint8_t* k_cache, float* k_scale_cache, uint16_t* c_cache, int d_I,
-                                     int* len1) {
+// Writes the new token's indexer key (+ scale) and latent entry at position ctx_len[b] of sequence b, n_b + 1
+// into len1[b] (the number of keys the new token attends to) and the start of the sequence's score row into
+// score_off[b].  Score rows are packed in sequence order, each padded to a multiple of 4 floats, so that every
+// row starts on a 16-byte boundary (the top-k reads rows with 16-byte loads); they do not follow the cache
+// layout.  A sequence whose cache range is invalid (cache_off < 0, ctx_len < 0, or the new row outside the
+// cache) or whose score row would not fit in score_cap floats raises DSA_ERR_BAD_INDEX and gets len1 = 0: no
+// kernel after this one reads or writes anything of it.
+
+__device__ __forceinline__ bool decode_seq_valid(const long long* cache_off, const int* ctx_len,
+                                                 long long cache_rows, int b) {
+  const long long off = cache_off[b];
+  const int n = ctx_len[b];
+  return off >= 0 && n >= 0 && off + n < cache_rows;
+}
+
+__device__ __forceinline__ long long padded4(long long n) { return (n + 3) & ~3ll; }
+
+constexpr int kAppendThreads = 128;
+
+__global__ void __launch_bounds__(kAppendThreads)
+    decode_append_kernel(int B, const long long* cache_off, const int* ctx_len, long long cache_rows,
+                         const uint8_t* k_new, const float* k_scale_new, const uint16_t* c_new, uint8_t* k_cache,
+                         float* k_scale_cache, uint16_t* c_cache, int d_I, int* len1, long long* score_off,
+                         long long score_cap) {
   const int b = blockIdx.x;
   if (b >= B) return;
-  const long long row = cache_off[b] + ctx_len[b];
-  if (ctx_len[b] < 0 || row < 0 || row >= cache_rows) {
-    if (threadIdx.x == 0) { raise_status(DSA_ERR_BAD_INDEX); len1[b] = 0; }
+  // start of this sequence's score row: the padded lengths of the valid sequences before it
+  __shared__ long long part[kAppendThreads / 32];
+  long long acc = 0;
+  for (int j = threadIdx.x; j < b; j += blockDim.x)
+    if (decode_seq_valid(cache_off, ctx_len, cache_rows, j))
+      acc += padded4(static_cast<long long>(ctx_len[j]) + 1);
+#pragma unroll
+  for (int d = 16; d > 0; d >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, d);
+  if ((threadIdx.x & 31) == 0) part[threadIdx.x >> 5] = acc;
+  __syncthreads();
+  long long s0 = 0;
+#pragma unroll
+  for (int w = 0; w < kAppendThreads / 32; ++w) s0 += part[w];
+  const bool valid = decode_seq_valid(cache_off, ctx_len, cache_rows, b) &&
+                     s0 + padded4(static_cast<long long>(ctx_len[b]) + 1) <= score_cap;
+  if (!valid) {
+    if (threadIdx.x == 0) { raise_status(DSA_ERR_BAD_INDEX); len1[b] = 0; score_off[b] = 0; }
     return;
   }
+  const long long row = cache_off[b] + ctx_len[b];
   const uint4* ks = reinterpret_cast<const uint4*>(k_new + static_cast<long long>(b) * d_I);
   uint4* kd = reinterpret_cast<uint4*>(k_cache + row * d_I);
   for (int i = threadIdx.x; i < d_I / 16; i += blockDim.x) kd[i] = ks[i];
@@ -38,7 +71,37 @@ __global__ void decode_append_kernel(int B, const long long* cache_off, const in
   if (threadIdx.x == 0) {
     k_scale_cache[row] = k_scale_new[b];
     len1[b] = ctx_len[b] + 1;
+    score_off[b] = s0;
   }
+}
+
+// ------------------------------------------------------------------------------------------ bounded-wait self-check
+// One CTA of two warps exercises the bounded mbarrier wait every pipeline of the library uses, on barriers
+// that nothing arrives on.  Warp 0 waits from the start and runs out of budget (g_wait_limit cycles, about a
+// second): it records DSA_ERR_TIMEOUT and raises the CTA's abort flag.  Warp 1 starts its wait half a budget
+// later and must leave on the abort flag, well before its own budget ends.  result[2w] = 1 if warp w's wait
+// succeeded, result[2w + 1] = its wait in units of 2^20 cycles.
+__global__ void __launch_bounds__(64) wait_selfcheck_kernel(int* result) {
+  __shared__ __align__(8) uint64_t bars[2];
+  __shared__ int abort_flag;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    mbar_init(smem_u32(&bars[0]), 1);
+    mbar_init(smem_u32(&bars[1]), 1);
+    abort_flag = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+  if (lane != 0) return;
+  if (warp == 1) {
+    const long long t0 = clock64();
+    while (clock64() - t0 < (g_wait_limit >> 1)) {
+    }
+  }
+  const long long t0 = clock64();
+  const bool ok = mbar_wait(smem_u32(&bars[warp]), 0, &abort_flag);
+  result[2 * warp] = ok ? 1 : 0;
+  result[2 * warp + 1] = static_cast<int>((clock64() - t0) >> 20);
 }
 
 // ------------------------------------------------------------------------------------------ host helpers
@@ -93,6 +156,10 @@ dsa_status_t last_launch_status() {
 }
 
 size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+// floats of the decode score rows: every valid sequence's n_b + 1 keys, padded to a multiple of 4; sequences
+// own disjoint cache ranges, so the rows need at most cache_rows + 3 B floats
+size_t decode_score_cap(int B, int64_t cache_rows) { return size_t(cache_rows) + 4 * size_t(B); }
 
 // ------------------------------------------------------------------------------------------ launchers
 // A configuration that allocates all 512 TMEM columns runs one CTA per SM: at least 120 KB of shared memory is
@@ -326,6 +393,13 @@ dsa_status_t dsa_forward_prefill(const uint8_t* q_idx, const float* q_scale, con
 
 uint64_t dsa_launch_count(void) { return g_launches.load(); }
 
+dsa_status_t dsa_check_bounded_wait(int32_t* result, void* stream) {
+  if (!result) return DSA_ERR_INVALID_ARG;
+  if (!aligned16(result)) return DSA_ERR_ALIGNMENT;
+  wait_selfcheck_kernel<<<1, 64, 0, static_cast<cudaStream_t>(stream)>>>(result);
+  return last_launch_status();
+}
+
 #ifdef DSA_TRACE
 // traced build only: copy the event stamps out and clear them
 __attribute__((visibility("default"))) int dsa_trace_read(unsigned long long* host) {
@@ -338,7 +412,8 @@ __attribute__((visibility("default"))) int dsa_trace_read(unsigned long long* ho
 size_t dsa_decode_workspace_size(int B, int64_t cache_rows, int H_I, int d_I, int H, int k) {
   (void)H_I; (void)d_I; (void)H;
   if (B <= 0 || cache_rows <= 0 || k <= 0) return 0;
-  return align_up(size_t(cache_rows) * 4, 256) + align_up(size_t(B) * 4, 256) + align_up(size_t(B) * k * 4, 256);
+  return align_up(decode_score_cap(B, cache_rows) * 4, 256) + align_up(size_t(B) * 4, 256) +
+         align_up(size_t(B) * 8, 256) + align_up(size_t(B) * k * 4, 256);
 }
 
 dsa_status_t dsa_forward_decode(int B, const int64_t* cache_off, const int32_t* ctx_len, const uint8_t* q_idx,
@@ -357,14 +432,19 @@ dsa_status_t dsa_forward_decode(int B, const int64_t* cache_off, const int32_t* 
   if (!ws || ws_bytes < dsa_decode_workspace_size(B, cache_rows, H_I, d_I, H, k)) return DSA_ERR_WORKSPACE;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   char* wsb = static_cast<char*>(ws);
+  // workspace: score rows (packed, 16-byte aligned), len1 [B], score_off [B], selected indices [B, k]
+  const size_t score_cap = decode_score_cap(B, cache_rows);
   float* dscores = reinterpret_cast<float*>(wsb);
-  int* len1 = reinterpret_cast<int*>(wsb + align_up(size_t(cache_rows) * 4, 256));
-  int32_t* idx = idx_out ? idx_out
-                         : reinterpret_cast<int32_t*>(wsb + align_up(size_t(cache_rows) * 4, 256) +
-                                                      align_up(size_t(B) * 4, 256));
+  size_t at = align_up(score_cap * 4, 256);
+  int* len1 = reinterpret_cast<int*>(wsb + at);
+  at += align_up(size_t(B) * 4, 256);
+  long long* soff = reinterpret_cast<long long*>(wsb + at);
+  at += align_up(size_t(B) * 8, 256);
+  int32_t* idx = idx_out ? idx_out : reinterpret_cast<int32_t*>(wsb + at);
   const long long* off = reinterpret_cast<const long long*>(cache_off);
-  decode_append_kernel<<<B, 128, 0, st>>>(B, off, ctx_len, cache_rows, k_new, k_scale_new, c_new, k_cache,
-                                          k_scale_cache, c_cache, d_I, len1);
+  decode_append_kernel<<<B, kAppendThreads, 0, st>>>(B, off, ctx_len, cache_rows, k_new, k_scale_new, c_new,
+                                                     k_cache, k_scale_cache, c_cache, d_I, len1, soff,
+                                                     static_cast<long long>(score_cap));
   dsa_status_t e = last_launch_status();
   if (e != DSA_OK) return e;
   IndexerParams p{};
@@ -374,11 +454,13 @@ dsa_status_t dsa_forward_decode(int B, const int64_t* cache_off, const int32_t* 
   p.scores = dscores;
   p.T = B;
   p.cache_off = off;
-  p.ctx_len = ctx_len;
+  p.len1 = len1;
+  p.score_off = soff;
   p.chunk_tiles = 16;
-  e = launch_indexer<64, 128, 1, 1, 2, 4, 1, kModeDecode>(q_idx, B, k_cache, cache_rows, p, 2 * num_sms(), st);
+  e = launch_indexer<64, 128, 1, 1, 2, 4, 1, kModeDecode>(
+      q_idx, B, k_cache, cache_rows, p, IndexerCfg<64, 128, 1, 1, 2, 4, 1, kModeDecode>::CTAS_PER_SM * num_sms(), st);
   if (e != DSA_OK) return e;
-  e = run_topk(dscores, 0, off, len1, 0, B, k, idx, k, st);
+  e = run_topk(dscores, 0, soff, len1, 0, B, k, idx, k, st);
   if (e != DSA_OK) return e;
   return run_mla(q, c_cache, cache_rows, idx, off, B, H, k, scale, out, lse, st);
 }

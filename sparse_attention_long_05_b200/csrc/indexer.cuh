@@ -21,8 +21,8 @@
 //   kModeScores  item = (block of NG*NT query rows, range of key tiles); writes scores [T, S] (tests,
 //                materialised prefill chunks);
 //   kModeDecode  item = (sequence b, range of its key tiles); one token per sequence; keys are the rows
-//                [cache_off[b], cache_off[b] + ctx_len[b]] of the flat key cache; writes one fp32 score per
-//                cache row (a vector per sequence).
+//                [cache_off[b], cache_off[b] + len1[b]) of the flat key cache; writes the sequence's len1[b]
+//                fp32 scores from score_off[b] on (one packed row per sequence).
 #pragma once
 #include "common.cuh"
 
@@ -42,8 +42,9 @@ struct IndexerParams {
   int n_items;             // kModeScores: number of work items
   int nsplit;              // kModeScores: key-range splits per query block
   int split_tiles;         // kModeScores: key tiles per split
-  const long long* cache_off;  // kModeDecode: [B]
-  const int* ctx_len;          // kModeDecode: [B] entries before the append (the new token sits at ctx_len)
+  const long long* cache_off;  // kModeDecode: [B] first cache row of each sequence
+  const int* len1;             // kModeDecode: [B] keys of each sequence after the append (0: skip it)
+  const long long* score_off;  // kModeDecode: [B] start of each sequence's score row
   int chunk_tiles;             // kModeDecode: key tiles per work item
 };
 
@@ -67,6 +68,8 @@ struct IndexerCfg {
   static constexpr int KBYTES = 128 * D_I;           // one key tile
   static constexpr int NUM_EPI_WARPS = 4 * EPI_WG;
   static constexpr int NUM_THREADS = 64 + 32 * NUM_EPI_WARPS;
+  // CTAs per SM the launch relies on (decode: two, so that two sequences' chunks share an SM)
+  static constexpr int CTAS_PER_SM = (MODE == kModeDecode) ? 2 : 1;
   static constexpr int ALIGN = 1024;
   // shared memory map (offsets from a 1024-byte aligned base)
   static constexpr int OFF_BAR = 0;                  // barriers + misc (2 KB)
@@ -138,7 +141,7 @@ __device__ __forceinline__ IndexerItem indexer_item(const IndexerParams& p, int 
     it.key_row0 = offs[b];
     it.tile0 = (i - prefix[b]) * p.chunk_tiles;
     it.tile1 = min(it.tile0 + p.chunk_tiles, (n + 127) / 128);
-    it.out_base = offs[b];
+    it.out_base = p.score_off[b];
   }
   return it;
 }
@@ -158,7 +161,8 @@ __device__ __forceinline__ bool tile_active(const IndexerItem& it, int tile) {
 }
 
 template <int H_I, int D_I, int NT, int NG, int QBUF, int KSTAGES, int EPI_WG, int MODE>
-__global__ void __launch_bounds__(IndexerCfg<H_I, D_I, NT, NG, QBUF, KSTAGES, EPI_WG, MODE>::NUM_THREADS, 1)
+__global__ void __launch_bounds__(IndexerCfg<H_I, D_I, NT, NG, QBUF, KSTAGES, EPI_WG, MODE>::NUM_THREADS,
+                                  IndexerCfg<H_I, D_I, NT, NG, QBUF, KSTAGES, EPI_WG, MODE>::CTAS_PER_SM)
 indexer_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                const IndexerParams p) {
   using C = IndexerCfg<H_I, D_I, NT, NG, QBUF, KSTAGES, EPI_WG, MODE>;
@@ -192,7 +196,7 @@ indexer_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     long long* offs = reinterpret_cast<long long*>(n1s + kMaxDecodeSeqs + 1);
     int* cnts = prefix + 1;          // counts first, scanned in place below
     for (int b = threadIdx.x; b < p.T; b += blockDim.x) {
-      const int n1 = p.ctx_len[b] + 1;
+      const int n1 = p.len1[b];
       n1s[b] = n1;
       offs[b] = p.cache_off[b];
       const int tiles = (n1 + 127) / 128;

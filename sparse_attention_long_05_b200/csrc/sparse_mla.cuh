@@ -117,11 +117,13 @@ static_assert(SMEM <= 232448, "shared memory per CTA");
 // row of c gathered for selection entry e of a token whose entries start at row `base`
 __device__ __forceinline__ long long mla_row(int e, long long base, long long S) {
   const long long r = base + e;
-  const bool valid = (e >= 0) && (r < S);
+  const bool valid = (e >= 0) && (r >= 0) && (r < S);
   if (!valid && e != -1) raise_status(DSA_ERR_BAD_INDEX);
-  return valid ? r : (base < S ? base : 0);
+  return valid ? r : ((base >= 0 && base < S) ? base : 0);
 }
-__device__ __forceinline__ bool mla_valid(int e, long long base, long long S) { return e >= 0 && base + e < S; }
+__device__ __forceinline__ bool mla_valid(int e, long long base, long long S) {
+  return e >= 0 && base + e >= 0 && base + e < S;
+}
 
 // position in a ring of `size` stages (size known at run time): stage index and pass parity, advanced
 // incrementally so that no division runs in the per-chunk loops

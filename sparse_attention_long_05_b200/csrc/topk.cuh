@@ -38,13 +38,18 @@ struct TopkParams {
 constexpr int kTopkThreads = 512;
 constexpr int kTopkThreadsFew = 1024;
 constexpr int kTopkBins = 2048;            // top 11 key bits
-constexpr int kTopkCandidates = 10240;     // candidate slots per CTA, split into one region per warp
 constexpr int kTopkSampleMin = 16384;      // rows at least this long take the sampled path
+
+// Candidate slots per CTA, split into one region per warp.  The sampled path's threshold bin spans about 19 %
+// in score, so on 128K-key rows it can collect 11K+ candidates; the one-CTA-per-SM variant (fewer rows than
+// SMs) spends its larger shared memory on twice the slots, which keeps such rows off the exact path.
+template <int NT>
+constexpr int topk_candidates() { return NT >= 1024 ? 20480 : 10240; }
 
 template <int NT>
 struct TopkSmem {
   static constexpr int W = NT / 32;
-  static constexpr int REGION = kTopkCandidates / W;   // candidates per warp region
+  static constexpr int REGION = topk_candidates<NT>() / W;   // candidates per warp region
   uint32_t hist[W][256];                   // radix select: per-warp histograms
   uint32_t bins[kTopkBins];                // top-11-bit histogram
   uint32_t cand_key[W][REGION];
@@ -54,6 +59,8 @@ struct TopkSmem {
   int s_gt[W], s_eq[W];
   int s_out_base[W], s_eq_base[W];
 };
+static_assert(sizeof(TopkSmem<1024>) <= 227 * 1024 && 2 * sizeof(TopkSmem<512>) <= 228 * 1024 - 2048,
+              "top-k shared memory: one 1024-thread CTA or two 512-thread CTAs per SM");
 
 // Radix select on 32-bit keys among the entries that match (key & mask) == prefix: returns the exact k-th
 // largest key and sets `need` to the number of entries equal to it that are taken.  each(visit) calls

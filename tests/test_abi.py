@@ -70,5 +70,8 @@ def test_host_argument_checks(lib):
     # decode: only H_I = 64 / d_I = 128
     assert lib.dsa_forward_decode(2, one, one, one, None, one, one, one, one, one, one, one, one, 100, 4, 64, 8, 128,
                                   1.0, None, one, None, one, 1 << 20, None) == 2
+    # bounded-wait self-check: null or misaligned result array
+    assert lib.dsa_check_bounded_wait(None, None) == 1
+    assert lib.dsa_check_bounded_wait(P(20), None) == 3
     # empty work is a no-op
     assert lib.dsa_indexer_scores(one, None, one, None, one, 0, 4, 64, 128, 0, one, None) == 0

@@ -69,3 +69,41 @@ def test_small_batch_gaussian(dsa):
 def test_full_batch_sampled_sequences(dsa):
     cfg = G.DECODE_CONFIG
     _run_steps(dsa, cfg, 43, 2, [0, 7, 21, 63], exact=False)
+
+
+def test_long_rows_integer_mode_exact(dsa):
+    # Score rows of 16K-40K keys take the top-k's sampled path; integer mode has many tied scores, which it
+    # must still break exactly as the oracle does.  The rows' cache offsets are not multiples of 4.
+    cfg = G.DecodeConfig("long_int", B=4, len_lo=16384, len_hi=40000, steps=2, mode="int")
+    assert any(o % 4 for o in G.decode_layout(cfg, 45)[1])
+    _run_steps(dsa, cfg, 45, 2, range(4), exact=True)
+
+
+def test_invalid_sequence_is_reported_and_skipped(dsa):
+    # Sequence 1 points past the end of the cache: the call reports DSA_ERR_BAD_INDEX, touches none of its
+    # rows, selects nothing for it, and the other sequences (whose score rows move up) are unaffected.
+    cfg = G.DecodeConfig("bad_seq", B=3, len_lo=17000, len_hi=30000, steps=1, mode="int")
+    seed = 46
+    cache = G.decode_fill_cache(cfg, seed, device="cuda")
+    lens, offs = cache["lens"], list(cache["offs"])
+    offs[1] = cache["rows"]
+    cache_off = torch.tensor(offs, dtype=torch.int64, device="cuda")
+    ctx = torch.tensor(lens, dtype=torch.int32, device="cuda")
+    before = cache["c_cache"].clone()
+    st = G.decode_step_inputs(cfg, seed, 0, device="cuda")
+    idx, out, _ = dsa.dsa_forward_decode(cache_off, ctx, st["q_idx"], st["q_scale"], st["w"], st["q"],
+                                         st["k_new"], st["k_scale_new"], st["c_new"], cache["k_cache"],
+                                         cache["k_scale_cache"], cache["c_cache"], cfg.k, cfg.scale)
+    assert dsa.dsa_get_device_status() == 6
+    idx, out = idx.cpu().numpy(), f64(out)
+    assert (idx[1] == -1).all()
+    step_q = G.decode_step_inputs(cfg, seed, 0)
+    changed = (cache["c_cache"] != before).any(dim=1).nonzero().flatten().tolist()
+    assert changed == [cache["offs"][0] + lens[0], cache["offs"][2] + lens[2]]
+    for b in (0, 2):
+        n = lens[b] + 1
+        rows = G.decode_cache_rows(cfg, seed, b, range(n))
+        ref = O.decode_row(rows, step_q, b, n, cfg.k, cfg.scale)
+        assert np.array_equal(idx[b], ref["idx"])
+        assert np.abs(out[b] - ref["out"]).max() <= MAX_ABS
+        assert rel_l2(out[b], ref["out"]) <= REL_L2

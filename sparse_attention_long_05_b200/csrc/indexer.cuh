@@ -384,25 +384,36 @@ indexer_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             uint64_t acc2[TOKS][2];
 #pragma unroll
             for (int tk = 0; tk < TOKS; ++tk) acc2[tk][0] = acc2[tk][1] = 0ull;
+            // tensor-memory loads run two 32-column chunks ahead of the arithmetic (a ring of three register
+            // buffers): only the first wait of a stage is exposed
+            constexpr int NCH = CPT / 32;
+            constexpr int RD = 3;
+            uint32_t v[RD][32];
 #pragma unroll
-            for (int c0 = 0; c0 < CPT; c0 += 64) {
-              uint32_t v0[32], v1[32];
-              tmem_ld32(lane_addr + tcol + c0, v0);
-              tmem_ld32(lane_addr + tcol + c0 + 32, v1);
-              tmem_wait_ld();
-              const int tk = c0 / H_I;
-              const float4* w4 = reinterpret_cast<const float4*>(wq + (tok0 + tk) * H_I + (c0 % H_I));
+            for (int c = 0; c < RD - 1 && c < NCH; ++c) tmem_ld32(lane_addr + tcol + 32 * c, v[c]);
+            tmem_wait_ld();
 #pragma unroll
-              for (int i = 0; i < 64; i += 4) {
+            for (int c = 0; c < RD - 1 && c < NCH; ++c) tmem_regs_after_wait(v[c]);
+#pragma unroll
+            for (int c = 0; c < NCH; ++c) {
+              if (c + RD - 1 < NCH) tmem_ld32(lane_addr + tcol + 32 * (c + RD - 1), v[(c + RD - 1) % RD]);
+              const int tk = (32 * c) / H_I;
+              const float4* w4 = reinterpret_cast<const float4*>(wq + (tok0 + tk) * H_I + ((32 * c) % H_I));
+#pragma unroll
+              for (int i = 0; i < 32; i += 4) {
                 const float4 ww = w4[i >> 2];
                 float a[4];
 #pragma unroll
                 for (int u = 0; u < 4; ++u) {
-                  const float x = __uint_as_float(i + u < 32 ? v0[i + u] : v1[i + u - 32]);
+                  const float x = __uint_as_float(v[c % RD][i + u]);
                   a[u] = (u & 1) ? x + fabsf(x) : fmaxf(x, 0.f);
                 }
                 acc2[tk][0] = fma_f32x2(pack_f32x2(ww.x, ww.y), pack_f32x2(a[0], a[1]), acc2[tk][0]);
                 acc2[tk][1] = fma_f32x2(pack_f32x2(ww.z, ww.w), pack_f32x2(a[2], a[3]), acc2[tk][1]);
+              }
+              if (c + RD - 1 < NCH) {
+                tmem_wait_ld();
+                tmem_regs_after_wait(v[(c + RD - 1) % RD]);
               }
             }
 #pragma unroll

@@ -7,8 +7,10 @@ steps, caches appended every step) is measured in the same run and reported unde
 
 One prefill step = the whole forward of one sequence through the C ABI with inputs resident in HBM:
 dsa_prefill_select (indexer scores of a bounded block of rows + their top-k, block after block) followed by
-dsa_sparse_mla_attn.  Every kernel is bracketed by CUDA events on the launching stream, which gives each
-kernel's share of the step and its roofline fraction.  Inputs (q alone is 19 GB) are far larger than the
+dsa_sparse_mla_attn.  Both calls are bracketed by CUDA events on the launching stream.  After the timed region
+the step's select blocks are re-run one by one through dsa_indexer_scores and dsa_topk (the same kernels and
+arguments), with events around every launch; that gives the indexer's and the top-k's own share of the step.
+The roofline line reports the kernel with the largest per-step time among attention, indexer and top-k.  Inputs (q alone is 19 GB) are far larger than the
 126 MB L2, so no explicit L2 flush is needed between steps.
 
 --impl reference runs the CPU oracle (fp64, test infrastructure) on the host cores on a bounded sample of
@@ -108,14 +110,16 @@ def attention_traffic(tokens):
     return None if t is None else t["dram_bytes_per_query_token"] * tokens
 
 
-def select_traffic(L, rows_per_block):
-    """DRAM bytes of the indexer + top-k of one prefill step (materialised score blocks of rows_per_block rows
-    against the keys up to each block's end), scaled from the committed capture."""
-    t = _traffic_entry("prefill_select", ("indexer.cuh", "topk.cuh", "common.cuh"))
-    if t is None:
-        return None
-    scores = sum(min(rows_per_block, L - r0) * min(L, r0 + rows_per_block) for r0 in range(0, L, rows_per_block))
-    return t["dram_bytes_per_score"] * scores
+def materialised_scores(L, rows_per_block):
+    """Scores one prefill step materialises: blocks of rows_per_block rows against the keys up to each block's end."""
+    return sum(min(rows_per_block, L - r0) * min(L, r0 + rows_per_block) for r0 in range(0, L, rows_per_block))
+
+
+def select_traffic(L, rows_per_block, name="prefill_select", files=("indexer.cuh", "topk.cuh", "common.cuh")):
+    """DRAM bytes of one prefill step's indexer + top-k (or of one of them, by `name`), scaled from the committed
+    capture's bytes per materialised score."""
+    t = _traffic_entry(name, files)
+    return None if t is None else t["dram_bytes_per_score"] * materialised_scores(L, rows_per_block)
 
 
 def peaks():
@@ -216,6 +220,30 @@ def prefill_chunk_rows(L):
 
 
 # ------------------------------------------------------------------------------------------ GPU arms
+def select_split(dsa, x, cfg, ws, idx):
+    """Per-kernel time of one step's select: its score blocks re-run one by one through dsa_indexer_scores and
+    dsa_topk (the kernels and arguments dsa_prefill_select launches block after block), each launch bracketed by
+    CUDA events on the launching stream.  Returns (indexer ms, top-k ms, blocks)."""
+    L, k = cfg.L, cfg.k
+    R = prefill_chunk_rows(L)
+    evs = []
+    for r0 in range(0, L, R):
+        rows, S = min(R, L - r0), min(L, r0 + R)
+        sc = ws[:rows * S * 4].view(torch.float32).view(rows, S)
+        qs = None if x["q_scale"] is None else x["q_scale"][r0:r0 + rows]
+        ks = None if x["k_scale"] is None else x["k_scale"][:S]
+        e = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+        e[0].record()
+        dsa.dsa_indexer_scores(x["q_idx"][r0:r0 + rows], qs, x["k_idx"][:S], ks, x["w"][r0:r0 + rows], pos0=r0,
+                               scores=sc)
+        e[1].record()
+        dsa.dsa_topk(sc, k, pos0=r0, idx=idx[r0:r0 + rows])
+        e[2].record()
+        evs.append(e)
+    torch.cuda.synchronize()
+    return (sum(e[0].elapsed_time(e[1]) for e in evs), sum(e[1].elapsed_time(e[2]) for e in evs), len(evs))
+
+
 def bench_prefill(dsa, cfg, steps, warmup, ws_n, rank, pk):
     dev = "cuda"
     x = G.prefill_keys(cfg, replica_seed(1000, rank), device=dev)
@@ -274,12 +302,30 @@ def bench_prefill(dsa, cfg, steps, warmup, ws_n, rank, pk):
                            "note": "indexer (FP8 flops) + top-k of materialised blocks of "
                                    f"{prefill_chunk_rows(L)} rows"},
     }
-    dom = max(kernels, key=lambda n: kernels[n]["ms"])
+    # the select call's two kernels, timed one by one after the timed region (same kernels, inputs and blocks)
+    ind_ms, tk_ms, nblk = select_split(dsa, x, cfg, ws, idx)
+    assert dsa.dsa_get_device_status() == 0
+    ind_tflops = work["indexer_flops"] / (ind_ms * 1e-3) / 1e12
+    tk_gbs = work["topk_bytes"] / (tk_ms * 1e-3) / 1e9
+    split_note = ("the step's score blocks re-run one by one after the timed region through dsa_indexer_scores / "
+                  "dsa_topk, CUDA events around every launch")
+    kernels["indexer"] = {"ms": ind_ms, "launches": nblk, "share": ind_ms / ms, "bound": "tensor",
+                          "achieved": ind_tflops, "peak": bf16_peak * NOMINAL_FP8_PER_BF16, "unit": "TFLOP/s",
+                          "frac": ind_tflops / (bf16_peak * NOMINAL_FP8_PER_BF16), "timed": split_note}
+    kernels["topk"] = {"ms": tk_ms, "launches": nblk, "share": tk_ms / ms, "bound": "hbm", "achieved": tk_gbs,
+                       "peak": pk["hbm_gbs"], "unit": "GB/s", "frac": tk_gbs / pk["hbm_gbs"], "timed": split_note}
+    # dominant kernel: the largest per-step time among the three kernels (the select call is two of them)
+    dom = max(("sparse_mla_attn", "indexer", "topk"), key=lambda n: kernels[n]["ms"])
     d = kernels[dom]
+    R = prefill_chunk_rows(L)
+    traffic = {"sparse_mla_attn": lambda: attention_traffic(L),
+               "indexer": lambda: select_traffic(L, R, "indexer", ("indexer.cuh", "common.cuh")),
+               "topk": lambda: select_traffic(L, R, "topk", ("topk.cuh", "common.cuh"))}[dom]()
+    peak_src = {"sparse_mla_attn": f"{pk['source']} bf16 sustained",
+                "indexer": f"{pk['source']} bf16 sustained x2 (FP8)",
+                "topk": f"{pk['source']} copy bandwidth"}[dom]
     roof = {"kernel": dom, "bound": d["bound"], "achieved": d["achieved"], "peak": d["peak"], "unit": d["unit"],
-            "frac": d["frac"],
-            "traffic": attention_traffic(L) if dom == "sparse_mla_attn" else select_traffic(L, prefill_chunk_rows(L)),
-            "peak_source": f"{pk['source']} bf16 sustained" + (" x2 (FP8)" if dom == "prefill_select" else "")}
+            "frac": d["frac"], "traffic": traffic, "peak_source": peak_src}
     del x
     return {"ms": ms, "tokens_per_s": job_rate(L, ws_n, ms), "roofline": roof, "kernels": kernels,
             "clocks": clk.summary(), "launches": launches}

@@ -303,8 +303,11 @@ def bench_prefill(dsa, cfg, steps, warmup, ws_n, rank, pk):
                                    f"{prefill_chunk_rows(L)} rows"},
     }
     # the select call's two kernels, timed one by one after the timed region (same kernels, inputs and blocks)
+    idx_step = idx.clone()
     ind_ms, tk_ms, nblk = select_split(dsa, x, cfg, ws, idx)
     assert dsa.dsa_get_device_status() == 0
+    assert torch.equal(idx, idx_step), "the launch-by-launch re-run must reproduce the step's selection"
+    del idx_step
     ind_tflops = work["indexer_flops"] / (ind_ms * 1e-3) / 1e12
     tk_gbs = work["topk_bytes"] / (tk_ms * 1e-3) / 1e9
     split_note = ("the step's score blocks re-run one by one after the timed region through dsa_indexer_scores / "

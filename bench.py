@@ -2,16 +2,17 @@
 """Throughput of the DSA forward hot path on B200: lightning indexer -> top-k -> sparse MLA.
 
 Default run (N = 1): the 128K-token causal prefill (L = 131072, H_I = 64, d_I = 128 FP8, k = 2048, 128 query
-heads over a 576-dim bf16 latent) is the headline line; the 64-sequence decode batch (contexts 4K..128K, 256
-steps, caches appended every step) is measured in the same run and reported under "decode".
+heads over a 576-dim bf16 latent) is the headline line.  The same run also measures two other workloads:
+- the 64-sequence decode batch (contexts 4K..128K, 256 steps, caches appended every step), under "decode";
+- a packed batch of 32 independent 4K-token sequences through the varlen entry point, under "varlen".
 
 One prefill step = the whole forward of one sequence through the C ABI with inputs resident in HBM:
 dsa_prefill_select (indexer scores of a bounded block of rows + their top-k, block after block) followed by
 dsa_sparse_mla_attn.  Both calls are bracketed by CUDA events on the launching stream.  After the timed region
 the step's select blocks are re-run one by one through dsa_indexer_scores and dsa_topk (the same kernels and
 arguments), with events around every launch; that gives the indexer's and the top-k's own share of the step.
-The roofline line reports the kernel with the largest per-step time among attention, indexer and top-k.  Inputs (q alone is 19 GB) are far larger than the
-126 MB L2, so no explicit L2 flush is needed between steps.
+The roofline line reports the kernel with the largest per-step time among attention, indexer and top-k.
+Inputs (q alone is 19 GB) are far larger than the 126 MB L2, so no explicit L2 flush is needed between steps.
 
 --impl reference runs the CPU oracle (fp64, test infrastructure) on the host cores on a bounded sample of
 query rows per step and reports the same metric.
@@ -194,7 +195,8 @@ class ClockSampler:
 def prefill_work(cfg):
     """Algorithmic work of one prefill step: indexer FP8 flops, attention bf16 flops, top-k bytes."""
     L, k = cfg.L, cfg.k
-    pairs = L * (L + 1) // 2                                          # (t, s) with s <= t
+    # (t, s) with s <= t over the rows whose selection needs scores (t + 1 > k; earlier rows take all of 0..t)
+    pairs = L * (L + 1) // 2 - min(L, k) * (min(L, k) + 1) // 2
     sel = sum(min(t + 1, k) for t in range(min(L, k))) + max(0, L - k) * k
     return {"indexer_flops": 2.0 * cfg.H_I * cfg.d_I * pairs,
             "attention_flops": 2.0 * cfg.H * (cfg.D + cfg.D_v) * sel,
@@ -223,7 +225,7 @@ def prefill_chunk_rows(L):
 def select_split(dsa, x, cfg, ws, idx):
     """Per-kernel time of one step's select: its score blocks re-run one by one through dsa_indexer_scores and
     dsa_topk (the kernels and arguments dsa_prefill_select launches block after block), each launch bracketed by
-    CUDA events on the launching stream.  Returns (indexer ms, top-k ms, blocks)."""
+    CUDA events on the launching stream.  Returns (indexer ms, top-k ms, indexer launches, top-k launches)."""
     L, k = cfg.L, cfg.k
     R = prefill_chunk_rows(L)
     evs = []
@@ -234,14 +236,16 @@ def select_split(dsa, x, cfg, ws, idx):
         ks = None if x["k_scale"] is None else x["k_scale"][:S]
         e = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
         e[0].record()
-        dsa.dsa_indexer_scores(x["q_idx"][r0:r0 + rows], qs, x["k_idx"][:S], ks, x["w"][r0:r0 + rows], pos0=r0,
-                               scores=sc)
+        if S > k:    # as in the select: a block of rows t < k has its selection implied, without scores
+            dsa.dsa_indexer_scores(x["q_idx"][r0:r0 + rows], qs, x["k_idx"][:S], ks, x["w"][r0:r0 + rows],
+                                   pos0=r0, scores=sc)
         e[1].record()
         dsa.dsa_topk(sc, k, pos0=r0, idx=idx[r0:r0 + rows])
         e[2].record()
         evs.append(e)
     torch.cuda.synchronize()
-    return (sum(e[0].elapsed_time(e[1]) for e in evs), sum(e[1].elapsed_time(e[2]) for e in evs), len(evs))
+    return (sum(e[0].elapsed_time(e[1]) for e in evs), sum(e[1].elapsed_time(e[2]) for e in evs),
+            sum(1 for r0 in range(0, L, R) if min(L, r0 + R) > k), len(evs))
 
 
 def bench_prefill(dsa, cfg, steps, warmup, ws_n, rank, pk):
@@ -304,7 +308,7 @@ def bench_prefill(dsa, cfg, steps, warmup, ws_n, rank, pk):
     }
     # the select call's two kernels, timed one by one after the timed region (same kernels, inputs and blocks)
     idx_step = idx.clone()
-    ind_ms, tk_ms, nblk = select_split(dsa, x, cfg, ws, idx)
+    ind_ms, tk_ms, n_ind, n_tk = select_split(dsa, x, cfg, ws, idx)
     assert dsa.dsa_get_device_status() == 0
     assert torch.equal(idx, idx_step), "the launch-by-launch re-run must reproduce the step's selection"
     del idx_step
@@ -312,10 +316,10 @@ def bench_prefill(dsa, cfg, steps, warmup, ws_n, rank, pk):
     tk_gbs = work["topk_bytes"] / (tk_ms * 1e-3) / 1e9
     split_note = ("the step's score blocks re-run one by one after the timed region through dsa_indexer_scores / "
                   "dsa_topk, CUDA events around every launch")
-    kernels["indexer"] = {"ms": ind_ms, "launches": nblk, "share": ind_ms / ms, "bound": "tensor",
+    kernels["indexer"] = {"ms": ind_ms, "launches": n_ind, "share": ind_ms / ms, "bound": "tensor",
                           "achieved": ind_tflops, "peak": bf16_peak * NOMINAL_FP8_PER_BF16, "unit": "TFLOP/s",
                           "frac": ind_tflops / (bf16_peak * NOMINAL_FP8_PER_BF16), "timed": split_note}
-    kernels["topk"] = {"ms": tk_ms, "launches": nblk, "share": tk_ms / ms, "bound": "hbm", "achieved": tk_gbs,
+    kernels["topk"] = {"ms": tk_ms, "launches": n_tk, "share": tk_ms / ms, "bound": "hbm", "achieved": tk_gbs,
                        "peak": pk["hbm_gbs"], "unit": "GB/s", "frac": tk_gbs / pk["hbm_gbs"], "timed": split_note}
     # dominant kernel: the largest per-step time among the three kernels (the select call is two of them)
     dom = max(("sparse_mla_attn", "indexer", "topk"), key=lambda n: kernels[n]["ms"])
@@ -379,6 +383,60 @@ def bench_prefill_e2e(dsa, cfg, steps, rank):
     ms = t0.elapsed_time(t1) / steps
     return {"value": L / (ms * 1e-3), "unit": "tokens/s", "ms_per_step": ms, "h2d_bytes_per_step": h2d,
             "d2h_bytes_per_step": d2h, "steps": steps}
+
+
+def bench_varlen(dsa, cfg, nseq, steps, warmup, ws_n, rank, pk):
+    """A packed batch of nseq independent causal sequences of cfg.L / nseq tokens each (the same token count and
+    shapes as the single-sequence prefill), one dsa_forward_prefill_varlen call per step, CUDA events around the
+    timed steps."""
+    import dataclasses
+    dev = "cuda"
+    n = cfg.L // nseq
+    scfg = dataclasses.replace(cfg, name=f"{cfg.name}_varlen", L=n)
+    parts = []
+    for b in range(nseq):
+        x = G.prefill_keys(scfg, replica_seed(3000, rank) + 7 * b, device=dev)
+        x.update(G.prefill_queries(scfg, replica_seed(3000, rank) + 7 * b, None, device=dev))
+        parts.append(x)
+    keys = ("q_idx", "q_scale", "k_idx", "k_scale", "w", "q", "c")
+    cat = {key: torch.cat([x[key] for x in parts]) if parts[0][key] is not None else None for key in keys}
+    del parts
+    cu = [b * n for b in range(nseq + 1)]
+    total = cu[-1]
+    idx = torch.empty((total, cfg.k), dtype=torch.int32, device=dev)
+    out = torch.empty((total, cfg.H, cfg.D_v), dtype=torch.bfloat16, device=dev)
+    lse = torch.empty((total, cfg.H), dtype=torch.float32, device=dev)
+    ws = torch.empty((dsa.dsa_prefill_varlen_workspace_size(nseq, total, n, cfg.H_I, cfg.d_I, cfg.H, cfg.k),),
+                     dtype=torch.uint8, device=dev)
+
+    def step():
+        dsa.dsa_forward_prefill_varlen(cu, cat["q_idx"], cat["q_scale"], cat["k_idx"], cat["k_scale"], cat["w"],
+                                       cat["q"], cat["c"], cfg.k, cfg.scale, idx_out=idx, out=out, lse=lse, ws=ws)
+
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize()
+    barrier(ws_n)
+    n0 = dsa.dsa_launch_count()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record()
+    for _ in range(steps):
+        step()
+    t1.record()
+    torch.cuda.synchronize()
+    launches = dsa.dsa_launch_count() - n0
+    barrier(ws_n)
+    ms = max_over_ranks(t0.elapsed_time(t1), ws_n) / steps
+    assert dsa.dsa_get_device_status() == 0
+    work = prefill_work(scfg)
+    flops = nseq * (work["indexer_flops"] / NOMINAL_FP8_PER_BF16 + work["attention_flops"])
+    del cat
+    return {"metric": f"DSA forward tokens/s, {nseq} packed causal sequences of {n} tokens (varlen)",
+            "value": job_rate(total, ws_n, ms), "unit": "tokens/s", "ms_per_step": ms, "steps": steps,
+            "warmup": warmup, "launches_per_step": launches / steps,
+            "bf16_equivalent_tflops": flops / (ms * 1e-3) / 1e12,
+            "note": "indexer FP8 flops counted at half weight (the nominal FP8/bf16 rate ratio) plus attention "
+                    "bf16 flops, over the whole call"}
 
 
 def bench_decode(dsa, cfg, steps, warmup, ws_n, rank, pk):
@@ -529,6 +587,7 @@ def main():
     ap.add_argument("--ref-step-seconds", type=float, default=8.0)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-varlen", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--kernels-small", action="store_true",
                     help="run one launch of each main kernel on small inputs (profiling) and exit")
@@ -560,6 +619,10 @@ def run_dsa(args, ws_n, rank):
     if not args.no_decode:
         dec = bench_decode(dsa, DECODE, args.decode_steps, args.warmup, ws_n, rank, pk)
         torch.cuda.empty_cache()
+    var = None
+    if not args.no_varlen:
+        var = bench_varlen(dsa, PREFILL, 32, max(3, args.steps // 2), args.warmup, ws_n, rank, pk)
+        torch.cuda.empty_cache()
     e2e = None
     if not args.no_e2e:
         e2e = bench_prefill_e2e(dsa, PREFILL, args.e2e_steps, rank)
@@ -582,7 +645,7 @@ def run_dsa(args, ws_n, rank):
                    "indexer_inputs": "gaussian, fp8 e4m3 with per-token scale", "parallelism": "replicas",
                    "l2": "inputs larger than L2 (q alone is 19 GB), no flush"},
         "roofline": pre["roofline"], "kernels": pre["kernels"], "clocks": pre["clocks"],
-        "e2e": e2e, "gpu_launches": pre["launches"], "cpu_baseline": cpu, "decode": dec,
+        "e2e": e2e, "gpu_launches": pre["launches"], "cpu_baseline": cpu, "decode": dec, "varlen": var,
     }
     print(json.dumps(line), flush=True)
 

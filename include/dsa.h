@@ -124,7 +124,9 @@ DSA_API size_t dsa_prefill_workspace_size(int L, int H_I, int d_I, int H, int k)
  * and their top-k selection (velog.io sections 1.1-1.2).
  *   q_idx [L, H_I, d_I] e4m3, q_scale [L] or NULL, k_idx [L, d_I] e4m3, k_scale [L] or NULL, w [L, H_I] fp32;
  *   idx_out [L, k] int32 (out): the selected positions of each row, ascending, padded with -1.
- * The L x L score matrix is never stored (the workspace holds a bounded block of rows).
+ * The L x L score matrix is never stored (the workspace holds a bounded block of rows).  A block whose rows all
+ * have t + 1 <= k (every prefill with L <= k) needs no scores: each of its rows selects all of 0..t, and the
+ * indexer is not launched for it.
  */
 DSA_API dsa_status_t dsa_prefill_select(const uint8_t* q_idx, const float* q_scale, const uint8_t* k_idx,
                                         const float* k_scale, const float* w, int L, int H_I, int d_I, int k,
@@ -142,6 +144,33 @@ DSA_API dsa_status_t dsa_forward_prefill(const uint8_t* q_idx, const float* q_sc
                                  const float* k_scale, const float* w, const uint16_t* q, const uint16_t* c,
                                  int L, int H_I, int d_I, int H, int k, float scale, int32_t* idx_out,
                                  uint16_t* out, float* lse, void* ws, size_t ws_bytes, void* stream);
+
+/* Workspace bytes of dsa_forward_prefill_varlen: nseq sequences of `total` rows in all, the longest max_len. */
+DSA_API size_t dsa_prefill_varlen_workspace_size(int nseq, int64_t total, int max_len, int H_I, int d_I, int H,
+                                                 int k);
+
+/*
+ * Steps 1-3 for a batch of independent causal prefill sequences packed one after another ("varlen").  The
+ * pages describe one sequence; this is that computation for each sequence of the batch.
+ * Sequence b holds rows [cu_seqlens[b], cu_seqlens[b + 1]) of every per-row array.  Its positions and its
+ * selected indices count from its first row, and it attends only to its own rows.
+ *   cu_seqlens: HOST array of nseq + 1 int64; cu_seqlens[0] = 0, non-decreasing (empty sequences allowed),
+ *     total = cu_seqlens[nseq] rows in all, at most INT32_MAX.
+ *   q_idx [total, H_I, d_I] e4m3, q_scale [total] or NULL, k_idx [total, d_I] e4m3, k_scale [total] or NULL,
+ *     w [total, H_I] fp32, q [total, H, 576] bf16, c [total, 576] bf16 (device arrays);
+ *   idx_out [total, k] int32 (out, may be NULL): each row's selection within its own sequence;
+ *   out [total, H, 512] bf16 (out), lse [total, H] fp32 (out, may be NULL).
+ * Steps 1-2 run per sequence, as dsa_prefill_select.  Step 3 runs once for every row of the batch: each row
+ * reads c from its own sequence's first row.  cu_seqlens is read on the host during the call and copied into
+ * the workspace, so the caller may reuse it when the call returns.
+ * Returns DSA_ERR_INVALID_ARG for a malformed cu_seqlens and the errors of dsa_forward_prefill otherwise.
+ */
+DSA_API dsa_status_t dsa_forward_prefill_varlen(int nseq, const int64_t* cu_seqlens, const uint8_t* q_idx,
+                                                const float* q_scale, const uint8_t* k_idx, const float* k_scale,
+                                                const float* w, const uint16_t* q, const uint16_t* c, int H_I,
+                                                int d_I, int H, int k, float scale, int32_t* idx_out,
+                                                uint16_t* out, float* lse, void* ws, size_t ws_bytes,
+                                                void* stream);
 
 /* Workspace bytes of dsa_forward_decode for a batch of B sequences over caches of cache_rows rows. */
 DSA_API size_t dsa_decode_workspace_size(int B, int64_t cache_rows, int H_I, int d_I, int H, int k);

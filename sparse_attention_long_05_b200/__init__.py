@@ -11,11 +11,13 @@ from ._lib import (  # noqa: F401
     dsa_forward_decode_noalloc,
     dsa_forward_decode,
     dsa_forward_prefill,
+    dsa_forward_prefill_varlen,
     dsa_get_device_status,
     dsa_indexer_scores,
     dsa_launch_count,
     dsa_num_sms,
     dsa_prefill_select,
+    dsa_prefill_varlen_workspace_size,
     dsa_prefill_workspace_size,
     dsa_sparse_mla_attn,
     dsa_topk,

@@ -32,6 +32,9 @@ SIGNATURES = {
     "dsa_prefill_workspace_size": (_SZ, [_I, _I, _I, _I, _I]),
     "dsa_prefill_select": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _P, _P, _SZ, _P]),
     "dsa_forward_prefill": (_I, [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _P, _P, _P, _P, _SZ, _P]),
+    "dsa_prefill_varlen_workspace_size": (_SZ, [_I, _I64, _I, _I, _I, _I, _I]),
+    "dsa_forward_prefill_varlen": (_I, [_I, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _F, _P, _P, _P, _P, _SZ,
+                                        _P]),
     "dsa_decode_workspace_size": (_SZ, [_I, _I64, _I, _I, _I, _I]),
     "dsa_forward_decode": (_I, [_I, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _I64, _I, _I, _I, _I, _F,
                                 _P, _P, _P, _P, _SZ, _P]),
@@ -174,6 +177,38 @@ def dsa_forward_prefill(q_idx, q_scale, k_idx, k_scale, w, q, c, k: int, scale: 
     _check("dsa_forward_prefill", _lib.dsa_forward_prefill(
         _ptr(q_idx), _ptr(q_scale), _ptr(k_idx), _ptr(k_scale), _ptr(w), _ptr(q), _ptr(c), L, H_I, d_I, H, k,
         float(scale), _ptr(idx_out), _ptr(out), _ptr(lse), _ptr(ws), ws.numel(), _stream(stream)))
+    return idx_out, out, lse
+
+
+def dsa_prefill_varlen_workspace_size(nseq: int, total: int, max_len: int, H_I: int, d_I: int, H: int,
+                                      k: int) -> int:
+    return int(_lib.dsa_prefill_varlen_workspace_size(nseq, total, max_len, H_I, d_I, H, k))
+
+
+def dsa_forward_prefill_varlen(cu_seqlens, q_idx, q_scale, k_idx, k_scale, w, q, c, k: int, scale: float,
+                               idx_out=None, out=None, lse=None, ws=None, stream=None):
+    """DSA forward of a packed batch of causal sequences (sequence b = rows cu_seqlens[b]..cu_seqlens[b+1]-1)
+    -> (idx [total, k] within each sequence, out [total, H, 512], lse [total, H])."""
+    cu = [int(v) for v in cu_seqlens]
+    nseq = len(cu) - 1
+    total, H_I, d_I = q_idx.shape
+    H = q.shape[1]
+    dev = q.device
+    max_len = max((cu[b + 1] - cu[b] for b in range(nseq)), default=0)
+    if idx_out is None:
+        idx_out = torch.empty((total, k), dtype=torch.int32, device=dev)
+    if out is None:
+        out = torch.empty((total, H, 512), dtype=torch.bfloat16, device=dev)
+    if lse is None:
+        lse = torch.empty((total, H), dtype=torch.float32, device=dev)
+    if ws is None:
+        need = dsa_prefill_varlen_workspace_size(nseq, total, max(max_len, 1), H_I, d_I, H, k)
+        ws = torch.empty((max(need, 1),), dtype=torch.uint8, device=dev)
+    cu_arr = (ctypes.c_int64 * len(cu))(*cu)
+    _check("dsa_forward_prefill_varlen", _lib.dsa_forward_prefill_varlen(
+        nseq, ctypes.cast(cu_arr, ctypes.c_void_p), _ptr(q_idx), _ptr(q_scale), _ptr(k_idx), _ptr(k_scale),
+        _ptr(w), _ptr(q), _ptr(c), H_I, d_I, H, k, float(scale), _ptr(idx_out), _ptr(out), _ptr(lse), _ptr(ws),
+        ws.numel(), _stream(stream)))
     return idx_out, out, lse
 
 

@@ -4,6 +4,7 @@
 // kernels of the prefill and decode drivers.  Every step of the computation runs in the kernels included
 // below.
 #include <cmath>
+#include <cstdint>
 #include <cstdio>
 #include <atomic>
 #include <mutex>
@@ -73,6 +74,20 @@ __global__ void __launch_bounds__(kAppendThreads)
     len1[b] = ctx_len[b] + 1;
     score_off[b] = s0;
   }
+}
+
+// ------------------------------------------------------------------------------------------ varlen prefill
+// Row offset of every token of a packed batch of sequences: the first row of its own sequence (the largest b
+// with cu[b] <= t, so an empty sequence never owns a token).
+__global__ void varlen_row_off_kernel(const long long* cu, int nseq, long long total, long long* row_off) {
+  const long long t = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (t >= total) return;
+  int lo = 0, hi = nseq - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (cu[mid] <= t) lo = mid; else hi = mid - 1;
+  }
+  row_off[t] = cu[lo];
 }
 
 // ------------------------------------------------------------------------------------------ bounded-wait self-check
@@ -362,10 +377,14 @@ dsa_status_t dsa_prefill_select(const uint8_t* q_idx, const float* q_scale, cons
   for (int r0 = 0; r0 < L; r0 += static_cast<int>(R)) {
     const int rows = (L - r0 < static_cast<int>(R)) ? L - r0 : static_cast<int>(R);
     const int s_eff = r0 + rows;   // keys beyond the block's last row are never selected (causal)
-    dsa_status_t e = run_indexer_scores(q_idx + static_cast<size_t>(r0) * H_I * d_I, q_scale ? q_scale + r0 : nullptr,
-                                        k_idx, k_scale, w + static_cast<size_t>(r0) * H_I, rows, s_eff, H_I, d_I,
-                                        r0, sc, s_eff, st);
-    if (e != DSA_OK) return e;
+    // a block whose every row t has t + 1 <= k selects all of 0..t whatever the scores: no indexer launch (the
+    // top-k kernel writes 0..t and the -1 padding of such rows without reading them)
+    dsa_status_t e = DSA_OK;
+    if (s_eff > k) {
+      e = run_indexer_scores(q_idx + static_cast<size_t>(r0) * H_I * d_I, q_scale ? q_scale + r0 : nullptr, k_idx,
+                             k_scale, w + static_cast<size_t>(r0) * H_I, rows, s_eff, H_I, d_I, r0, sc, s_eff, st);
+      if (e != DSA_OK) return e;
+    }
     e = run_topk(sc, s_eff, nullptr, nullptr, r0, rows, k, idx_out + static_cast<size_t>(r0) * k, k, st);
     if (e != DSA_OK) return e;
   }
@@ -389,6 +408,63 @@ dsa_status_t dsa_forward_prefill(const uint8_t* q_idx, const float* q_scale, con
   dsa_status_t e = dsa_prefill_select(q_idx, q_scale, k_idx, k_scale, w, L, H_I, d_I, k, idx, ws, ws_bytes, stream);
   if (e != DSA_OK) return e;
   return run_mla(q, c, L, idx, nullptr, L, H, k, scale, out, lse, st);
+}
+
+size_t dsa_prefill_varlen_workspace_size(int nseq, int64_t total, int max_len, int H_I, int d_I, int H, int k) {
+  (void)H_I; (void)d_I; (void)H;
+  if (nseq <= 0 || total <= 0 || max_len <= 0 || k <= 0) return 0;
+  return align_up(prefill_chunk_rows(max_len) * size_t(max_len) * 4, 256) + align_up(size_t(total) * 8, 256) +
+         align_up(size_t(nseq + 1) * 8, 256) + align_up(size_t(total) * size_t(k) * 4, 256);
+}
+
+dsa_status_t dsa_forward_prefill_varlen(int nseq, const int64_t* cu_seqlens, const uint8_t* q_idx,
+                                        const float* q_scale, const uint8_t* k_idx, const float* k_scale,
+                                        const float* w, const uint16_t* q, const uint16_t* c, int H_I, int d_I,
+                                        int H, int k, float scale, int32_t* idx_out, uint16_t* out, float* lse,
+                                        void* ws, size_t ws_bytes, void* stream) {
+  if (nseq <= 0 || !cu_seqlens || H <= 0 || k <= 0 || !q_idx || !k_idx || !w || !q || !c || !out)
+    return DSA_ERR_INVALID_ARG;
+  if (cu_seqlens[0] != 0) return DSA_ERR_INVALID_ARG;
+  int max_len = 0;
+  for (int b = 0; b < nseq; ++b) {
+    const int64_t len = cu_seqlens[b + 1] - cu_seqlens[b];
+    if (len < 0 || cu_seqlens[b + 1] > INT32_MAX) return DSA_ERR_INVALID_ARG;
+    if (len > max_len) max_len = static_cast<int>(len);
+  }
+  const int64_t total = cu_seqlens[nseq];
+  if (total <= 0) return DSA_ERR_INVALID_ARG;
+  if (!indexer_shape_ok(H_I, d_I) || H > 128 || !mla_k_ok(k)) return DSA_ERR_UNSUPPORTED_SHAPE;
+  if (!aligned16(q_idx) || !aligned16(k_idx) || !aligned16(q) || !aligned16(c) || !aligned16(out) ||
+      (idx_out && !aligned16(idx_out)))
+    return DSA_ERR_ALIGNMENT;
+  if (!ws || ws_bytes < dsa_prefill_varlen_workspace_size(nseq, total, max_len, H_I, d_I, H, k))
+    return DSA_ERR_WORKSPACE;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  // workspace: one sequence's score block (sized for the longest), per-token row offsets, cu_seqlens, indices
+  char* wsb = static_cast<char*>(ws);
+  const size_t score_bytes = align_up(prefill_chunk_rows(max_len) * size_t(max_len) * 4, 256);
+  size_t at = score_bytes;
+  long long* row_off = reinterpret_cast<long long*>(wsb + at);
+  at += align_up(size_t(total) * 8, 256);
+  long long* cu_dev = reinterpret_cast<long long*>(wsb + at);
+  at += align_up(size_t(nseq + 1) * 8, 256);
+  int32_t* idx = idx_out ? idx_out : reinterpret_cast<int32_t*>(wsb + at);
+  if (cudaMemcpyAsync(cu_dev, cu_seqlens, size_t(nseq + 1) * 8, cudaMemcpyHostToDevice, st) != cudaSuccess)
+    return DSA_ERR_CUDA;
+  varlen_row_off_kernel<<<static_cast<unsigned>((total + 255) / 256), 256, 0, st>>>(cu_dev, nseq, total, row_off);
+  dsa_status_t e = last_launch_status();
+  if (e != DSA_OK) return e;
+  // steps 1-2 per sequence (its own causal positions 0..len-1), then step 3 for every token in one launch
+  for (int b = 0; b < nseq; ++b) {
+    const int64_t r = cu_seqlens[b];
+    const int len = static_cast<int>(cu_seqlens[b + 1] - r);
+    if (len == 0) continue;
+    e = dsa_prefill_select(q_idx + r * H_I * d_I, q_scale ? q_scale + r : nullptr, k_idx + r * d_I,
+                           k_scale ? k_scale + r : nullptr, w + r * H_I, len, H_I, d_I, k, idx + r * k, ws,
+                           score_bytes, stream);
+    if (e != DSA_OK) return e;
+  }
+  return run_mla(q, c, static_cast<int>(total), idx, row_off, static_cast<int>(total), H, k, scale, out, lse, st);
 }
 
 uint64_t dsa_launch_count(void) { return g_launches.load(); }

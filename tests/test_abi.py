@@ -70,6 +70,23 @@ def test_host_argument_checks(lib):
     # decode: only H_I = 64 / d_I = 128
     assert lib.dsa_forward_decode(2, one, one, one, None, one, one, one, one, one, one, one, one, 100, 4, 64, 8, 128,
                                   1.0, None, one, None, one, 1 << 20, None) == 2
+    # varlen prefill: malformed cu_seqlens (first entry not 0, decreasing, empty batch)
+    cu = (ctypes.c_int64 * 3)(0, 100, 50)
+    assert lib.dsa_forward_prefill_varlen(2, ctypes.cast(cu, P), one, None, one, None, one, one, one, 64, 128, 128,
+                                          2048, 1.0, None, one, None, one, 1 << 30, None) == 1
+    cu = (ctypes.c_int64 * 2)(5, 100)
+    assert lib.dsa_forward_prefill_varlen(1, ctypes.cast(cu, P), one, None, one, None, one, one, one, 64, 128, 128,
+                                          2048, 1.0, None, one, None, one, 1 << 30, None) == 1
+    cu = (ctypes.c_int64 * 2)(0, 0)
+    assert lib.dsa_forward_prefill_varlen(1, ctypes.cast(cu, P), one, None, one, None, one, one, one, 64, 128, 128,
+                                          2048, 1.0, None, one, None, one, 1 << 30, None) == 1
+    # ... an unsupported shape, and a workspace below dsa_prefill_varlen_workspace_size
+    cu = (ctypes.c_int64 * 3)(0, 100, 300)
+    assert lib.dsa_forward_prefill_varlen(2, ctypes.cast(cu, P), one, None, one, None, one, one, one, 4, 128, 128,
+                                          2048, 1.0, None, one, None, one, 1 << 30, None) == 2
+    assert lib.dsa_forward_prefill_varlen(2, ctypes.cast(cu, P), one, None, one, None, one, one, one, 64, 128, 128,
+                                          2048, 1.0, None, one, None, one, 16, None) == 7
+    assert lib.dsa_prefill_varlen_workspace_size(2, 300, 200, 64, 128, 128, 2048) >= 300 * 2048 * 4 + 300 * 8
     # bounded-wait self-check: null or misaligned result array
     assert lib.dsa_check_bounded_wait(None, None) == 1
     assert lib.dsa_check_bounded_wait(P(20), None) == 3

@@ -1,4 +1,5 @@
 """dsa_forward_prefill (indexer -> top-k -> sparse MLA) end to end against the fp64 oracle."""
+import dataclasses
 import os
 
 import numpy as np
@@ -90,3 +91,52 @@ def test_128k_sampled_rows(dsa, name):
     n = int(os.environ.get("DSA_ORACLE_ROWS_128K", "64"))
     rows = sample_rows(cfg.L, cfg.k, n, 34)
     _check_rows(cfg, 34, rows, idx, out, exact_idx=(cfg.mode == "int"))
+
+
+def test_short_prefill_takes_the_implied_selection(dsa):
+    # With L <= k every row t selects all of 0..t, whatever the scores: the select writes that selection without
+    # launching the indexer (one top-k and one attention launch in all), and the outputs match the oracle.
+    cfg = G.PrefillConfig("short_1500", L=1500, H_I=64, d_I=128, k=2048, H=128)
+    n0 = dsa.dsa_launch_count()
+    idx, out, _ = _forward(dsa, cfg, 35)
+    assert dsa.dsa_launch_count() - n0 == 2
+    for t in (0, 1, 777, cfg.L - 1):
+        assert np.array_equal(idx[t], np.r_[np.arange(t + 1), -np.ones(cfg.k - t - 1, dtype=np.int64)])
+    _check_rows(cfg, 35, sample_rows(cfg.L, cfg.k, 16, 35), idx, out, exact_idx=True)
+
+
+def test_varlen_batch_matches_each_sequence_alone(dsa):
+    # Three causal sequences packed one after another, with an empty one among them: each row's selection,
+    # output and LSE equal those of its sequence run alone through dsa_forward_prefill (bit for bit), and the
+    # longest sequence matches the oracle on sampled rows.
+    base = G.PREFILL_CONFIGS["prefill_8k"]       # integer mode, H_I = 64, d_I = 128, k = 2048, H = 128
+    lens, seeds = [700, 0, 2500, 1300], [36, 0, 37, 38]
+    cfgs = [dataclasses.replace(base, name=f"varlen_{n}", L=n) for n in lens]
+    parts = [prefill_device(cfg, sd) for cfg, sd, n in zip(cfgs, seeds, lens) if n]
+    cat = {key: torch.cat([x[key] for x in parts]) for key in ("q_idx", "k_idx", "w", "q", "c")}
+    cu = np.concatenate([[0], np.cumsum(lens)]).tolist()
+    n0 = dsa.dsa_launch_count()
+    idx, out, lse = dsa.dsa_forward_prefill_varlen(cu, cat["q_idx"], None, cat["k_idx"], None, cat["w"], cat["q"],
+                                                   cat["c"], base.k, base.scale)
+    assert dsa.dsa_get_device_status() == 0
+    # the row offsets; a top-k per non-empty sequence and an indexer only for the one longer than k; one attention
+    assert dsa.dsa_launch_count() - n0 == 1 + 3 + 1 + 1
+    for b, (cfg, sd, n) in enumerate(zip(cfgs, seeds, lens)):
+        if not n:
+            continue
+        r0, r1 = cu[b], cu[b + 1]
+        i1, o1, l1 = _forward_full(dsa, cfg, sd)
+        assert torch.equal(idx[r0:r1], i1), f"sequence {b}: selection"
+        assert torch.equal(out[r0:r1], o1), f"sequence {b}: output"
+        assert torch.equal(lse[r0:r1], l1), f"sequence {b}: lse"
+    cfg, sd = cfgs[2], seeds[2]
+    _check_rows(cfg, sd, sample_rows(cfg.L, cfg.k, 12, sd), idx[cu[2]:cu[3]].cpu().numpy(), out[cu[2]:cu[3]],
+                exact_idx=True)
+
+
+def _forward_full(dsa, cfg, seed):
+    x = prefill_device(cfg, seed)
+    idx, out, lse = dsa.dsa_forward_prefill(x["q_idx"], x["q_scale"], x["k_idx"], x["k_scale"], x["w"], x["q"],
+                                            x["c"], cfg.k, cfg.scale)
+    assert dsa.dsa_get_device_status() == 0
+    return idx, out, lse

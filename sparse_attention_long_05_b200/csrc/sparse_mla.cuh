@@ -114,12 +114,15 @@ static_assert(NS_S <= 16 && NS_V <= 16, "ring barrier slots");
 static_assert(SMEM <= 232448, "shared memory per CTA");
 }  // namespace mla
 
-// row of c gathered for selection entry e of a token whose entries start at row `base`
-__device__ __forceinline__ long long mla_row(int e, long long base, long long S) {
+// row of c gathered for selection entry e (in slot `slot` of its token's k entries) of a token whose entries
+// start at row `base`.  An empty or invalid entry is masked out of the softmax but its stage still holds a row:
+// it reads row `slot` (any row in [0, S) would do), so that the padding of short rows spreads over many L2 lines
+// instead of hammering one
+__device__ __forceinline__ long long mla_row(int e, long long base, long long S, int slot) {
   const long long r = base + e;
   const bool valid = (e >= 0) && (r >= 0) && (r < S);
   if (!valid && e != -1) raise_status(DSA_ERR_BAD_INDEX);
-  return valid ? r : ((base >= 0 && base < S) ? base : 0);
+  return valid ? r : (slot < S ? slot : 0);
 }
 __device__ __forceinline__ bool mla_valid(int e, long long base, long long S) {
   return e >= 0 && base + e >= 0 && base + e < S;
@@ -259,10 +262,11 @@ sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         int r[4] = {0, 0, 0, 0};
         if (active) {
           const int4 e = reinterpret_cast<const int4*>(ids + j * NK)[rg];
-          r[0] = static_cast<int>(mla_row(e.x, base, p.S));
-          r[1] = static_cast<int>(mla_row(e.y, base, p.S));
-          r[2] = static_cast<int>(mla_row(e.z, base, p.S));
-          r[3] = static_cast<int>(mla_row(e.w, base, p.S));
+          const int slot = j * NK + 4 * rg;
+          r[0] = static_cast<int>(mla_row(e.x, base, p.S, slot));
+          r[1] = static_cast<int>(mla_row(e.y, base, p.S, slot + 1));
+          r[2] = static_cast<int>(mla_row(e.z, base, p.S, slot + 2));
+          r[3] = static_cast<int>(mla_row(e.w, base, p.S, slot + 3));
         }
         for (int s = 0; s < spt; ++s, rp.advance()) {
           const int st = rp.stage;

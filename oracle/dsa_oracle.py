@@ -15,7 +15,7 @@ on the velog.io page (DeepSeek Sparse Attention, §1.1-§1.3) and the yuuk.io no
 * §1.3 MLA in MQA mode: every latent entry c_s (one vector per token) is shared by all query heads, so
   u_t[h] = softmax_s(scale * q[t,h] . c_s) . c_s[:D_v] over the selected s.
 
-Readings where the pages are silent (each one is listed in the design doc with its reason):
+Readings where the pages are silent:
 * causal includes s = t; when t + 1 <= k every s <= t is selected; the output index list is in ascending s
   and padded with -1;
 * ties in the top-k are broken by the smaller s (a total order on (score desc, s asc) makes the set unique);

@@ -111,16 +111,17 @@ def attention_traffic(tokens):
     return None if t is None else t["dram_bytes_per_query_token"] * tokens
 
 
-def materialised_scores(L, rows_per_block):
-    """Scores one prefill step materialises: blocks of rows_per_block rows against the keys up to each block's end."""
-    return sum(min(rows_per_block, L - r0) * min(L, r0 + rows_per_block) for r0 in range(0, L, rows_per_block))
+def materialised_scores(blocks, k):
+    """Scores one prefill step materialises: each score block's rows against the keys up to the block's end (a
+    block whose rows all have t < k needs none)."""
+    return sum(n * (r0 + n) for r0, n in blocks if r0 + n > k)
 
 
-def select_traffic(L, rows_per_block, name="prefill_select", files=("indexer.cuh", "topk.cuh", "common.cuh")):
+def select_traffic(blocks, k, name="prefill_select", files=("indexer.cuh", "topk.cuh", "common.cuh")):
     """DRAM bytes of one prefill step's indexer + top-k (or of one of them, by `name`), scaled from the committed
     capture's bytes per materialised score."""
     t = _traffic_entry(name, files)
-    return None if t is None else t["dram_bytes_per_score"] * materialised_scores(L, rows_per_block)
+    return None if t is None else t["dram_bytes_per_score"] * materialised_scores(blocks, k)
 
 
 def peaks():
@@ -216,21 +217,16 @@ def decode_bytes(cfg, lens, steps):
     return tot
 
 
-def prefill_chunk_rows(L):
-    """Rows per score block of dsa_prefill_select (mirrors the library's choice, for reporting)."""
-    return max(256, min(L, (1 << 30) // (4 * L)))
-
-
 # ------------------------------------------------------------------------------------------ GPU arms
 def select_split(dsa, x, cfg, ws, idx):
     """Per-kernel time of one step's select: its score blocks re-run one by one through dsa_indexer_scores and
     dsa_topk (the kernels and arguments dsa_prefill_select launches block after block), each launch bracketed by
     CUDA events on the launching stream.  Returns (indexer ms, top-k ms, indexer launches, top-k launches)."""
     L, k = cfg.L, cfg.k
-    R = prefill_chunk_rows(L)
+    blocks = dsa.prefill_blocks(L, k)      # the library's own block schedule
     evs = []
-    for r0 in range(0, L, R):
-        rows, S = min(R, L - r0), min(L, r0 + R)
+    for r0, rows in blocks:
+        S = r0 + rows
         sc = ws[:rows * S * 4].view(torch.float32).view(rows, S)
         qs = None if x["q_scale"] is None else x["q_scale"][r0:r0 + rows]
         ks = None if x["k_scale"] is None else x["k_scale"][:S]
@@ -245,7 +241,7 @@ def select_split(dsa, x, cfg, ws, idx):
         evs.append(e)
     torch.cuda.synchronize()
     return (sum(e[0].elapsed_time(e[1]) for e in evs), sum(e[1].elapsed_time(e[2]) for e in evs),
-            sum(1 for r0 in range(0, L, R) if min(L, r0 + R) > k), len(evs))
+            sum(1 for r0, rows in blocks if r0 + rows > k), len(evs))
 
 
 def bench_prefill(dsa, cfg, steps, warmup, ws_n, rank, pk):
@@ -303,8 +299,8 @@ def bench_prefill(dsa, cfg, steps, warmup, ws_n, rank, pk):
         "prefill_select": {"ms": sel_ms, "share": sel_ms / ms, "bound": "tensor", "achieved": sel_tflops,
                            "peak": bf16_peak * NOMINAL_FP8_PER_BF16, "unit": "TFLOP/s",
                            "frac": sel_tflops / (bf16_peak * NOMINAL_FP8_PER_BF16),
-                           "note": "indexer (FP8 flops) + top-k of materialised blocks of "
-                                   f"{prefill_chunk_rows(L)} rows"},
+                           "note": "indexer (FP8 flops) + top-k of materialised score blocks: "
+                                   f"{len(dsa.prefill_blocks(L, k))} blocks (the first k rows, then blocks of 1 GiB of scores)"},
     }
     # the select call's two kernels, timed one by one after the timed region (same kernels, inputs and blocks)
     idx_step = idx.clone()
@@ -324,10 +320,10 @@ def bench_prefill(dsa, cfg, steps, warmup, ws_n, rank, pk):
     # dominant kernel: the largest per-step time among the three kernels (the select call is two of them)
     dom = max(("sparse_mla_attn", "indexer", "topk"), key=lambda n: kernels[n]["ms"])
     d = kernels[dom]
-    R = prefill_chunk_rows(L)
+    blocks = dsa.prefill_blocks(L, k)
     traffic = {"sparse_mla_attn": lambda: attention_traffic(L),
-               "indexer": lambda: select_traffic(L, R, "indexer", ("indexer.cuh", "common.cuh")),
-               "topk": lambda: select_traffic(L, R, "topk", ("topk.cuh", "common.cuh"))}[dom]()
+               "indexer": lambda: select_traffic(blocks, k, "indexer", ("indexer.cuh", "common.cuh")),
+               "topk": lambda: select_traffic(blocks, k, "topk", ("topk.cuh", "common.cuh"))}[dom]()
     peak_src = {"sparse_mla_attn": f"{pk['source']} bf16 sustained",
                 "indexer": f"{pk['source']} bf16 sustained x2 (FP8)",
                 "topk": f"{pk['source']} copy bandwidth"}[dom]

@@ -116,6 +116,12 @@ DSA_API dsa_status_t dsa_sparse_mla_attn(const uint16_t* q, const uint16_t* c, i
 /* Number of kernels this library has launched in this process (all devices, all entry points). */
 DSA_API uint64_t dsa_launch_count(void);
 
+/* Rows of the score block that dsa_prefill_select (and dsa_forward_prefill) processes next, starting at row r0
+ * of an L-row prefill with selection size k: rows r0 < k form one block (their selection needs no scores);
+ * later blocks hold the workspace's row count (about 1 GiB of fp32 scores at L keys, at least 256 rows).
+ * 0 when r0 is outside [0, L) or L, k <= 0.  Host function, no GPU. */
+DSA_API int dsa_prefill_block_rows(int L, int k, int r0);
+
 /* Workspace bytes of dsa_prefill_select and dsa_forward_prefill for these shapes. */
 DSA_API size_t dsa_prefill_workspace_size(int L, int H_I, int d_I, int H, int k);
 

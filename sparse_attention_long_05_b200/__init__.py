@@ -16,9 +16,11 @@ from ._lib import (  # noqa: F401
     dsa_indexer_scores,
     dsa_launch_count,
     dsa_num_sms,
+    dsa_prefill_block_rows,
     dsa_prefill_select,
     dsa_prefill_varlen_workspace_size,
     dsa_prefill_workspace_size,
     dsa_sparse_mla_attn,
     dsa_topk,
+    prefill_blocks,
 )

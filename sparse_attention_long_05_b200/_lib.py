@@ -29,6 +29,7 @@ SIGNATURES = {
     "dsa_topk": (_I, [_P, _I, _I64, _P, _I, _I, _P, _P]),
     "dsa_sparse_mla_attn": (_I, [_P, _P, _I, _P, _I, _I, _I, _F, _P, _P, _P]),
     "dsa_launch_count": (ctypes.c_uint64, []),
+    "dsa_prefill_block_rows": (_I, [_I, _I, _I]),
     "dsa_prefill_workspace_size": (_SZ, [_I, _I, _I, _I, _I]),
     "dsa_prefill_select": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _P, _P, _SZ, _P]),
     "dsa_forward_prefill": (_I, [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _P, _P, _P, _P, _SZ, _P]),
@@ -139,6 +140,20 @@ def dsa_sparse_mla_attn(q, c, idx, scale: float, out=None, lse=None, want_lse: b
 
 def dsa_prefill_workspace_size(L: int, H_I: int, d_I: int, H: int, k: int) -> int:
     return int(_lib.dsa_prefill_workspace_size(L, H_I, d_I, H, k))
+
+
+def dsa_prefill_block_rows(L: int, k: int, r0: int) -> int:
+    return int(_lib.dsa_prefill_block_rows(L, k, r0))
+
+
+def prefill_blocks(L: int, k: int):
+    """(first row, rows) of every score block of an L-row prefill, in the order the select processes them."""
+    out, r0 = [], 0
+    while r0 < L:
+        n = dsa_prefill_block_rows(L, k, r0)
+        out.append((r0, n))
+        r0 += n
+    return out
 
 
 def dsa_launch_count() -> int:

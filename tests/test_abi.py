@@ -92,3 +92,24 @@ def test_host_argument_checks(lib):
     assert lib.dsa_check_bounded_wait(P(20), None) == 3
     # empty work is a no-op
     assert lib.dsa_indexer_scores(one, None, one, None, one, 0, 4, 64, 128, 0, one, None) == 0
+
+
+def test_prefill_block_schedule(lib):
+    # dsa_prefill_block_rows (host only): the blocks tile [0, L) in order; rows t < k form the first block; every
+    # later block's scores (rows x keys up to its end) fit the workspace's prefill_chunk_rows(L) x L scores, and
+    # blocks get no longer as their key ranges grow
+    for L, k in ((1024, 128), (1500, 2048), (8192, 2048), (32768, 2048), (131072, 2048), (300000, 2048)):
+        cap = (lib.dsa_prefill_workspace_size(L, 64, 128, 128, k) - (((L * k * 4) + 255) // 256) * 256) // 4
+        r0, blocks = 0, []
+        while r0 < L:
+            n = lib.dsa_prefill_block_rows(L, k, r0)
+            assert n >= 1
+            blocks.append((r0, n))
+            r0 += n
+        assert r0 == L
+        assert blocks[0] == (0, min(k, L))
+        for (a, n), (b, m) in zip(blocks[1:], blocks[2:]):
+            assert b == a + n and m <= n
+        for a, n in blocks[1:]:
+            assert n * (a + n) <= cap
+    assert lib.dsa_prefill_block_rows(100, 10, 100) == 0 and lib.dsa_prefill_block_rows(0, 10, 0) == 0

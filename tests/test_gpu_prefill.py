@@ -119,8 +119,11 @@ def test_varlen_batch_matches_each_sequence_alone(dsa):
     idx, out, lse = dsa.dsa_forward_prefill_varlen(cu, cat["q_idx"], None, cat["k_idx"], None, cat["w"], cat["q"],
                                                    cat["c"], base.k, base.scale)
     assert dsa.dsa_get_device_status() == 0
-    # the row offsets; a top-k per non-empty sequence and an indexer only for the one longer than k; one attention
-    assert dsa.dsa_launch_count() - n0 == 1 + 3 + 1 + 1
+    # the row offsets; per non-empty sequence a top-k for its rows t < k, and for the one longer than k an indexer
+    # and a top-k for the rest; one attention launch
+    blocks = [dsa.prefill_blocks(n, base.k) for n in lens if n]
+    assert [len(b) for b in blocks] == [1, 2, 1]
+    assert dsa.dsa_launch_count() - n0 == 1 + (1 + 3 + 1) + 1
     for b, (cfg, sd, n) in enumerate(zip(cfgs, seeds, lens)):
         if not n:
             continue

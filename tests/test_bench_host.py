@@ -1,0 +1,74 @@
+"""bench.py's host arithmetic, on the CPU: the algorithmic work each roofline figure divides by, the scores a
+prefill step materialises, the decode step's HBM bytes and the clock-sample summary.  Every expected value is
+counted here by brute force, independently of the closed forms bench.py uses."""
+import dataclasses
+
+import pytest
+
+import bench
+import dsa_inputs as G
+
+
+def _count_prefill(cfg):
+    """(indexer flops, attention flops, top-k bytes) counted row by row."""
+    ind = att = tk = 0
+    for t in range(cfg.L):
+        n = t + 1
+        if n > cfg.k:                      # only rows with more than k candidates need scores
+            ind += 2 * cfg.H_I * cfg.d_I * n
+            tk += 4 * n
+        att += 2 * cfg.H * (cfg.D + cfg.D_v) * min(n, cfg.k)
+        tk += 4 * cfg.k
+    return ind, att, tk
+
+
+@pytest.mark.parametrize("L,k", [(1024, 128), (3000, 2048), (2048, 2048), (700, 2048)])
+def test_prefill_work_counts(L, k):
+    cfg = dataclasses.replace(G.PREFILL_CONFIGS["prefill_8k"], L=L, k=k)
+    w = bench.prefill_work(cfg)
+    ind, att, tk = _count_prefill(cfg)
+    assert w["indexer_flops"] == ind
+    assert w["attention_flops"] == att
+    assert w["topk_bytes"] == tk
+
+
+def test_materialised_scores():
+    # blocks of rows t < k materialise nothing; later blocks their rows times the keys up to their end
+    blocks = [(0, 2048), (2048, 2048), (4096, 1000)]
+    assert bench.materialised_scores(blocks, 2048) == 2048 * 4096 + 1000 * 5096
+    assert bench.materialised_scores([(0, 500)], 2048) == 0
+    assert bench.materialised_scores([(0, 128), (128, 896)], 128) == 896 * 1024
+
+
+def test_decode_bytes_counted_per_sequence():
+    cfg = G.DecodeConfig("tiny", B=3, len_lo=10, len_hi=3000, steps=4)
+    lens = [10, 2047, 2900]
+    got = bench.decode_bytes(cfg, lens, 2)
+    want = 0
+    for s in range(2):
+        for n in lens:
+            keys = n + s + 1                                 # the new token attends to its own entry too
+            want += keys * (cfg.d_I + 4)                     # e4m3 key row + fp32 scale, every key
+            want += min(keys, cfg.k) * cfg.D * 2             # the selected bf16 latent rows
+        per_seq = (cfg.H * cfg.D * 2                         # q
+                   + cfg.H_I * cfg.d_I + cfg.H_I * 4         # q_I and w
+                   + cfg.k * 4                               # selected indices
+                   + cfg.H * cfg.D_v * 2                     # output
+                   + cfg.d_I + 4 + cfg.D * 2)                # the appended key, scale and latent row
+        want += cfg.B * per_seq
+    assert got == want
+
+
+def test_clock_summary_reasons_and_median():
+    cs = bench.ClockSampler.__new__(bench.ClockSampler)
+    cs.rows = [["1965", "1965", "700.5", "Not Active", "Not Active", "Not Active", "Not Active"],
+               ["1800", "1965", "990.1", "Not Active", "Not Active", "Not Active", "Active"],
+               ["1900", "1965", "980.0", "Not Active", "Not Active", "Not Active", "Active"]]
+    sm = cs.summary()
+    assert sm["sm_mhz"] == 1900 and sm["sm_max_mhz"] == 1965
+    assert sm["reasons"] == ["sw_power_cap"] and sm["samples"] == 3 and sm["power_w_max"] == 990.1
+    cs.rows = [["1000", "1965", "[N/A]", "Active", "Not Active", "Active", "Not Active"]]
+    sm = cs.summary()
+    assert sm["reasons"] == ["hw_slowdown", "sw_thermal_slowdown"] and sm["power_w_max"] == 0.0
+    cs.rows = []
+    assert cs.summary()["reasons"] == ["unsampled"]

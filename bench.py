@@ -22,6 +22,7 @@ path); the step time is the max over ranks.
 from __future__ import annotations
 
 import argparse
+import dataclasses
 import json
 import os
 import statistics
@@ -435,15 +436,22 @@ def bench_varlen(dsa, cfg, nseq, steps, warmup, ws_n, rank, pk):
                     "bf16 flops, over the whole call"}
 
 
+def decode_plan(cfg, warmup, steps):
+    """The decode workload of a run of `warmup` untimed and `steps` timed steps: the same sequences (lengths and
+    cache contents depend only on the seed), with caches that hold every entry the run appends.  Returns the
+    workload and the total number of steps."""
+    nsteps = warmup + steps
+    return dataclasses.replace(cfg, steps=max(cfg.steps, nsteps)), nsteps
+
+
 def bench_decode(dsa, cfg, steps, warmup, ws_n, rank, pk):
     dev = "cuda"
     seed = replica_seed(2000, rank)
+    cfg, nsteps = decode_plan(cfg, warmup, steps)
     cache = G.decode_fill_cache(cfg, seed, device=dev)
     lens, offs = cache["lens"], cache["offs"]
     cache_off = torch.tensor(offs, dtype=torch.int64, device=dev)
     ctx = torch.tensor(lens, dtype=torch.int32, device=dev)
-    nsteps = warmup + steps
-    assert nsteps <= cfg.steps, "the caches hold cfg.steps appended entries per sequence"
     blocks = [G.decode_step_batch(cfg, seed, min(32, nsteps - s0), device=dev, step0=s0)
               for s0 in range(0, nsteps, 32)]
     inp = {key: torch.cat([b[key] for b in blocks]) if blocks[0][key] is not None else None for key in blocks[0]}
@@ -545,52 +553,67 @@ def oracle_threads():
 
 
 def run_reference(args, ws_n, rank):
+    """The oracle arm: each step is a bounded sample of seeded random query rows of the headline prefill, timed
+    on the host cores.  ms_per_step is the measured host time of a step (the sample's oracle time); the rate
+    extrapolates the mean per-row time to whole sequences of L rows."""
     if rank != 0:
         return
     cfg = PREFILL
     for w in range(args.warmup):
         oracle_prefill_rate(cfg, 0.0, 11 + w, max_rows=2, batch=2)
-    vals, rows_tot, spent_tot = [], 0, 0.0
+    rows_tot, spent_tot, wall_tot = 0, 0.0, 0.0
     for s in range(args.steps):
+        t0 = time.perf_counter()
         v, n, sp = oracle_prefill_rate(cfg, args.ref_step_seconds, 100 + s)
-        vals.append(v)
+        wall_tot += time.perf_counter() - t0
         rows_tot += n
         spent_tot += sp
     value = rows_tot / spent_tot
     cores = oracle_threads()
+    sample = (f"{rows_tot} seeded random query rows of the L={cfg.L} prefill over {args.steps} steps "
+              f"({spent_tot:.1f} s of host time), extrapolated to L rows")
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": ws_n,
-            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * cfg.L / value,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * spent_tot / args.steps,
+            "host_wall_ms_per_step": 1e3 * wall_tot / args.steps,
+            "extrapolated_ms_per_sequence": 1e3 * cfg.L / value,
+            "step": "one bounded sample of query rows (the oracle's time, input generation excluded)",
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": {"workload": cfg.name, "seq_len": cfg.L, "global_batch": 1, "H_I": cfg.H_I,
                        "d_I": cfg.d_I, "k": cfg.k, "heads": cfg.H, "parallelism": "replicas"},
-            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
-                             "sample": f"{rows_tot} seeded random query rows of the L={cfg.L} prefill "
-                                       f"({spent_tot:.1f} s of host time), extrapolated to L rows"},
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle", "sample": sample},
             "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 
 
 # ------------------------------------------------------------------------------------------ main
-def main():
+def parse_args(argv=None):
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=10)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["dsa", "reference"], default="dsa")
-    ap.add_argument("--decode-steps", type=int, default=256 - 3)
+    ap.add_argument("--decode-steps", type=int, default=DECODE.steps,
+                    help="timed decode steps (the caches are sized for these plus the warm-up steps)")
     ap.add_argument("--e2e-steps", type=int, default=2)
     ap.add_argument("--cpu-seconds", type=float, default=15.0, help="host time budget of the cpu_baseline leg")
     ap.add_argument("--ref-step-seconds", type=float, default=8.0)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-varlen", action="store_true")
+    ap.add_argument("--no-configs", action="store_true", help="skip the 8K and 32K prefill lines")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--kernels-small", action="store_true",
                     help="run one launch of each main kernel on small inputs (profiling) and exit")
-    args = ap.parse_args()
+    args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("at least 3 warm-up steps")
+    if args.steps < 1 or args.decode_steps < 1:
+        ap.error("at least one timed step")
+    return args
 
+
+def main(argv=None):
+    args = parse_args(argv)
     ws_n, rank, local = dist_init()
     try:
         if args.impl == "reference":
@@ -601,6 +624,19 @@ def main():
         if ws_n > 1:
             import torch.distributed as dist
             dist.destroy_process_group()
+
+
+# the other prefill configurations of the workload, each measured like the headline (parity cases otherwise)
+SIDE_CONFIGS = ("prefill_8k", "prefill_32k")
+
+
+def side_line(pre, cfg):
+    """Summary of one side configuration's prefill measurement."""
+    return {"workload": cfg.name, "seq_len": cfg.L, "indexer_inputs": "integer-valued fp8" if cfg.mode == "int"
+            else "gaussian fp8 with per-token scale", "value": pre["tokens_per_s"], "unit": "tokens/s",
+            "ms_per_step": pre["ms"], "roofline": pre["roofline"],
+            "kernels": {n: {key: v[key] for key in ("ms", "frac", "achieved", "unit")}
+                        for n, v in pre["kernels"].items()}}
 
 
 def run_dsa(args, ws_n, rank):
@@ -619,6 +655,13 @@ def run_dsa(args, ws_n, rank):
     if not args.no_varlen:
         var = bench_varlen(dsa, PREFILL, 32, max(3, args.steps // 2), args.warmup, ws_n, rank, pk)
         torch.cuda.empty_cache()
+    side = None
+    if not args.no_configs:
+        side = {}
+        for name in SIDE_CONFIGS:
+            cfg = G.PREFILL_CONFIGS[name]
+            side[name] = side_line(bench_prefill(dsa, cfg, args.steps, args.warmup, ws_n, rank, pk), cfg)
+            torch.cuda.empty_cache()
     e2e = None
     if not args.no_e2e:
         e2e = bench_prefill_e2e(dsa, PREFILL, args.e2e_steps, rank)
@@ -642,6 +685,7 @@ def run_dsa(args, ws_n, rank):
                    "l2": "inputs larger than L2 (q alone is 19 GB), no flush"},
         "roofline": pre["roofline"], "kernels": pre["kernels"], "clocks": pre["clocks"],
         "e2e": e2e, "gpu_launches": pre["launches"], "cpu_baseline": cpu, "decode": dec, "varlen": var,
+        "configs": side,
     }
     print(json.dumps(line), flush=True)
 

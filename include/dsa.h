@@ -19,7 +19,8 @@
  *     and launches nothing.  Errors found while kernels run (an index out of range, a pipeline wait that ran
  *     out of time) are recorded in a device status word read by dsa_get_device_status().
  *   - Nothing is allocated inside a call: scratch memory is a caller-provided workspace whose size the
- *     matching *_workspace_size() function returns.
+ *     matching *_workspace_size() function returns.  The one exception is dsa_forward_decode_noalloc, whose
+ *     scratch is a fixed array inside the library (no workspace argument, and still no allocation).
  *   - Supported shapes: H_I in {4, 64} with d_I = 64 / 128 respectively, H <= 128 query heads, D = 576 latent
  *     dims of which the first D_v = 512 are the value, k a multiple of 64 from 128 to 2048.  Other shapes
  *     return DSA_ERR_UNSUPPORTED_SHAPE.
@@ -217,8 +218,12 @@ DSA_API dsa_status_t dsa_forward_decode(int B, const int64_t* cache_off, const i
  *   - Arguments and results are those of dsa_forward_decode; shapes whose dsa_decode_workspace_size()
  *     exceeds the array return DSA_ERR_WORKSPACE and launch nothing.
  *   - The call allocates nothing: no cudaMalloc, no cudaFree, no allocating library routine.
+ *   - Argument and shape checks are those of dsa_forward_decode and come first, with its error codes; the
+ *     size check against the array comes after them.
  *   - The first call on a device looks up the array's device address (cudaGetSymbolAddress) with that device
- *     current; make that first call before any stream capture on the device.
+ *     current; make that first call before any stream capture on the device.  The address is kept with the
+ *     context it was looked up in and looked up again when the device's current context changes (after a
+ *     cudaDeviceReset, for instance); a first call in a new context must also come before any capture.
  *   - All calls share the one array and it keeps the last call's contents: calls that may overlap on the GPU
  *     (different streams, or graph replays in flight together) race on it and must be serialised by the
  *     caller.

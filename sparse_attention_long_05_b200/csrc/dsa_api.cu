@@ -308,6 +308,22 @@ int prefill_block_rows(int L, int k, int r0) {
   return static_cast<int>(std::min<size_t>(prefill_chunk_rows(L), static_cast<size_t>(L - r0)));
 }
 
+// Host checks of a decode step's arguments, shared by both decode entry points (everything but the scratch).
+dsa_status_t decode_args_status(int B, const int64_t* cache_off, const int32_t* ctx_len, const uint8_t* q_idx,
+                                const float* w, const uint16_t* q, const uint8_t* k_new, const float* k_scale_new,
+                                const uint16_t* c_new, const uint8_t* k_cache, const float* k_scale_cache,
+                                const uint16_t* c_cache, int64_t cache_rows, int H_I, int d_I, int H, int k,
+                                const int32_t* idx_out, const uint16_t* out) {
+  if (B <= 0 || cache_rows <= 0 || H <= 0 || k <= 0 || !cache_off || !ctx_len || !q_idx || !w || !q || !k_new ||
+      !k_scale_new || !c_new || !k_cache || !k_scale_cache || !c_cache || !out)
+    return DSA_ERR_INVALID_ARG;
+  if (H_I != 64 || d_I != 128 || H > 128 || !mla_k_ok(k) || B > kMaxDecodeSeqs) return DSA_ERR_UNSUPPORTED_SHAPE;
+  if (!aligned16(q_idx) || !aligned16(q) || !aligned16(k_new) || !aligned16(c_new) || !aligned16(k_cache) ||
+      !aligned16(c_cache) || !aligned16(out) || (idx_out && !aligned16(idx_out)))
+    return DSA_ERR_ALIGNMENT;
+  return DSA_OK;
+}
+
 }  // namespace
 }  // namespace dsa
 
@@ -513,13 +529,9 @@ dsa_status_t dsa_forward_decode(int B, const int64_t* cache_off, const int32_t* 
                                 float* k_scale_cache, uint16_t* c_cache, int64_t cache_rows, int H_I, int d_I,
                                 int H, int k, float scale, int32_t* idx_out, uint16_t* out, float* lse, void* ws,
                                 size_t ws_bytes, void* stream) {
-  if (B <= 0 || cache_rows <= 0 || H <= 0 || k <= 0 || !cache_off || !ctx_len || !q_idx || !w || !q || !k_new ||
-      !k_scale_new || !c_new || !k_cache || !k_scale_cache || !c_cache || !out)
-    return DSA_ERR_INVALID_ARG;
-  if (H_I != 64 || d_I != 128 || H > 128 || !mla_k_ok(k) || B > kMaxDecodeSeqs) return DSA_ERR_UNSUPPORTED_SHAPE;
-  if (!aligned16(q_idx) || !aligned16(q) || !aligned16(k_new) || !aligned16(c_new) || !aligned16(k_cache) ||
-      !aligned16(c_cache) || !aligned16(out) || (idx_out && !aligned16(idx_out)))
-    return DSA_ERR_ALIGNMENT;
+  const dsa_status_t chk = decode_args_status(B, cache_off, ctx_len, q_idx, w, q, k_new, k_scale_new, c_new, k_cache,
+                                              k_scale_cache, c_cache, cache_rows, H_I, d_I, H, k, idx_out, out);
+  if (chk != DSA_OK) return chk;
   if (!ws || ws_bytes < dsa_decode_workspace_size(B, cache_rows, H_I, d_I, H, k)) return DSA_ERR_WORKSPACE;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   char* wsb = static_cast<char*>(ws);
@@ -563,22 +575,49 @@ static constexpr size_t kNoAllocScratchBytes = size_t(32) << 20;
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
 
 namespace {
-// device address of g_noalloc_scratch on each device, looked up once per device with that device current
-// (host code may not use the array's name as a device address)
+// Device address of g_noalloc_scratch on each device, looked up with that device current (host code may not use
+// the array's name as a device address).  The address belongs to the context that loaded the module: it is kept
+// together with that context and looked up again when the device's current context is another one (after a
+// cudaDeviceReset, for instance).
 constexpr int kMaxDevices = 64;
-void* g_noalloc_ptr[kMaxDevices] = {};
+struct ScratchAddr {
+  void* ctx = nullptr;
+  void* ptr = nullptr;
+};
+ScratchAddr g_noalloc[kMaxDevices];
 std::mutex g_noalloc_mutex;
+
+using CtxGetCurrentFn = CUresult (*)(CUcontext*);
+CtxGetCurrentFn ctx_get_current_fn() {
+  static CtxGetCurrentFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<CtxGetCurrentFn>(p);
+  });
+  return fn;
+}
 
 dsa_status_t noalloc_scratch(void** out) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return DSA_ERR_CUDA;
+  CtxGetCurrentFn get_ctx = ctx_get_current_fn();
+  CUcontext ctx = nullptr;   // null while this thread has no current context yet
+  if (!get_ctx || get_ctx(&ctx) != CUDA_SUCCESS) return DSA_ERR_CUDA;
   std::lock_guard<std::mutex> lock(g_noalloc_mutex);
-  if (!g_noalloc_ptr[dev]) {
+  ScratchAddr& a = g_noalloc[dev];
+  if (!a.ptr || !ctx || a.ctx != static_cast<void*>(ctx)) {
     void* ptr = nullptr;
+    // the lookup makes the device's primary context current when it is not yet
     if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess || !ptr) return DSA_ERR_CUDA;
-    g_noalloc_ptr[dev] = ptr;
+    if (get_ctx(&ctx) != CUDA_SUCCESS || !ctx) return DSA_ERR_CUDA;
+    a.ctx = ctx;
+    a.ptr = ptr;
   }
-  *out = g_noalloc_ptr[dev];
+  *out = a.ptr;
   return DSA_OK;
 }
 }  // namespace
@@ -591,6 +630,9 @@ dsa_status_t dsa_forward_decode_noalloc(int B, const int64_t* cache_off, const i
                                         const uint16_t* c_new, uint8_t* k_cache, float* k_scale_cache,
                                         uint16_t* c_cache, int64_t cache_rows, int H_I, int d_I, int H, int k,
                                         float scale, int32_t* idx_out, uint16_t* out, float* lse, void* stream) {
+  const dsa_status_t chk = decode_args_status(B, cache_off, ctx_len, q_idx, w, q, k_new, k_scale_new, c_new, k_cache,
+                                              k_scale_cache, c_cache, cache_rows, H_I, d_I, H, k, idx_out, out);
+  if (chk != DSA_OK) return chk;
   if (dsa_decode_workspace_size(B, cache_rows, H_I, d_I, H, k) > kNoAllocScratchBytes) return DSA_ERR_WORKSPACE;
   void* scratch = nullptr;
   const dsa_status_t e = noalloc_scratch(&scratch);

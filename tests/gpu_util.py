@@ -11,6 +11,16 @@ REL_L2 = 5e-3
 RECALL = 0.995
 
 
+def e2e_bound(mean_recall: float) -> float:
+    """Bound on the end-to-end relative-L2 error of Gaussian-mode outputs against the oracle's own selection,
+    given the measured recall.  The attention weight of a key is independent of its index score, so a swapped
+    key (a fraction f = 1 - recall of the k selected) is a random draw from the same weight distribution as the
+    key it replaced.  With logits x ~ N(0, 1), sum_i p_i^2 = e / k per output dimension, so swapping m = f k
+    keys moves the output by sqrt(2 m e) / k against an output of sqrt(e / k): a relative-L2 of sqrt(2 f).
+    The bound allows 1.5 times that (the swap count and the weights fluctuate) plus the attention tolerance."""
+    return 1.5 * float(np.sqrt(2.0 * max(0.0, 1.0 - mean_recall))) + REL_L2
+
+
 def rel_l2(got, ref) -> float:
     got, ref = np.asarray(got, dtype=np.float64), np.asarray(ref, dtype=np.float64)
     return float(np.linalg.norm(got - ref) / max(np.linalg.norm(ref), 1e-300))

@@ -4,6 +4,7 @@ counted here by brute force, independently of the closed forms bench.py uses."""
 import dataclasses
 
 import pytest
+import torch
 
 import bench
 import dsa_inputs as G
@@ -72,3 +73,46 @@ def test_clock_summary_reasons_and_median():
     assert sm["reasons"] == ["hw_slowdown", "sw_thermal_slowdown"] and sm["power_w_max"] == 0.0
     cs.rows = []
     assert cs.summary()["reasons"] == ["unsampled"]
+
+
+@pytest.mark.parametrize("argv", [["--gpus", "1", "--steps", "20", "--warmup", "5"], [],
+                                  ["--steps", "3", "--warmup", "40", "--decode-steps", "300"]])
+def test_decode_caches_hold_every_step_the_run_appends(argv):
+    # The run appends one entry per sequence at every warm-up and timed step; the caches bench.py allocates must
+    # hold all of them, whatever the warm-up count, and the timed part is the 256 steps of the decode workload
+    # unless asked otherwise.
+    args = bench.parse_args(argv)
+    cfg, nsteps = bench.decode_plan(bench.DECODE, args.warmup, args.decode_steps)
+    assert nsteps == args.warmup + args.decode_steps
+    if "--decode-steps" not in argv:
+        assert args.decode_steps == 256
+    seed = bench.replica_seed(2000, 0)
+    lens, offs, tot = G.decode_layout(cfg, seed)
+    assert lens == G.decode_lengths(bench.DECODE, seed)          # the same sequences as the workload
+    ends = offs[1:] + [tot]
+    for b, (n, o) in enumerate(zip(lens, offs)):
+        assert o + n + nsteps <= ends[b], f"sequence {b}: the last appended entry falls outside its range"
+
+
+def test_decode_plan_keeps_the_cache_contents():
+    # A larger capacity moves the sequences' cache offsets but not their contents: the entry appended at step s
+    # is the cache row at position n_b + s under either layout.
+    small = G.DecodeConfig("tiny", B=3, len_lo=20, len_hi=60, steps=4, mode="int")
+    big, nsteps = bench.decode_plan(small, 5, 6)
+    assert big.steps == 11 and nsteps == 11
+    seed = 9
+    assert G.decode_layout(big, seed)[1] != G.decode_layout(small, seed)[1]
+    lens = G.decode_lengths(small, seed)
+    batch = G.decode_step_batch(big, seed, 2, step0=nsteps - 2)
+    for i, s in enumerate((nsteps - 2, nsteps - 1)):
+        for b in range(small.B):
+            row = G.decode_cache_rows(small, seed, b, [lens[b] + s])
+            assert torch.equal(batch["k_new"][i, b].view(torch.uint8), row["k_idx"][0].view(torch.uint8))
+            assert torch.equal(batch["c_new"][i, b], row["c"][0])
+
+
+def test_argument_checks():
+    with pytest.raises(SystemExit):
+        bench.parse_args(["--warmup", "2"])
+    with pytest.raises(SystemExit):
+        bench.parse_args(["--decode-steps", "0"])

@@ -125,7 +125,9 @@ def _rows_uniform(key: int, rows: torch.Tensor, row_len: int, a: int) -> torch.T
 def quantise_e4m3_per_row(x: torch.Tensor):
     """fp32 rows -> (e4m3 rows, fp32 scale per row) with scale = amax / 448 (input recipe, not the method)."""
     amax = x.abs().amax(dim=1).clamp_min(1e-30)
-    s = amax / E4M3_MAX
+    # tensor / tensor: a correctly rounded division on every device (a CUDA division by a Python scalar multiplies
+    # by its reciprocal, which can differ in the last bit from the CPU's result)
+    s = amax / torch.full_like(amax, E4M3_MAX)
     q = (x / s[:, None]).clamp(-E4M3_MAX, E4M3_MAX).to(torch.float8_e4m3fn)
     return q, s
 

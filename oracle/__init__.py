@@ -12,6 +12,9 @@ Parity status of each function (what pins it is in ``tests/test_oracle.py``):
   attention_row                pinned: golden example, torch scaled_dot_product_attention (fp64) on dense
                                causal rows, q = 0 closed form, k = 1, permutation invariance, logsumexp
   prefill_rows, decode_row     pinned: pure-Python brute force on micro sequences, t < k dense invariant
+  indexer_kl_row               pinned: hand-worked closed form (two heads, three keys), zero divergence when
+                               I = log p + const, invariance to a constant shift of I, non-negativity,
+                               pure-Python brute force
 """
 from .dsa_oracle import *  # noqa: F401,F403
 from .dsa_oracle import __all__  # noqa: F401

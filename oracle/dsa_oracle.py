@@ -14,6 +14,8 @@ on the velog.io page (DeepSeek Sparse Attention, §1.1-§1.3) and the yuuk.io no
   u_t = Attn(h_t, {c_s : s selected}).  k = 2048 (velog.io Stage 2; aisparkup.com; macaron.im).
 * §1.3 MLA in MQA mode: every latent entry c_s (one vector per token) is shared by all query heads, so
   u_t[h] = softmax_s(scale * q[t,h] . c_s) . c_s[:D_v] over the selected s.
+* Stage 1 (dense warm-up) training objective of the indexer: the target p_{t,:} is the main attention's
+  probabilities summed over the heads and L1-normalised, and L_I = sum_t KL(p_{t,:} || Softmax(I_{t,:})).
 
 Readings where the pages are silent:
 * causal includes s = t; when t + 1 <= k every s <= t is selected; the output index list is in ascending s
@@ -35,7 +37,7 @@ import numpy as np
 
 __all__ = [
     "e4m3_table", "e4m3_to_f64", "bf16_to_f64", "f32_to_f64",
-    "indexer_scores_row", "topk_row", "attention_row", "prefill_rows", "decode_row",
+    "indexer_scores_row", "topk_row", "attention_row", "prefill_rows", "decode_row", "indexer_kl_row",
 ]
 
 
@@ -113,6 +115,30 @@ def attention_row(q_t: np.ndarray, c_sel: np.ndarray, scale: float, D_v: int):
     u = (p @ c_sel[:, :D_v]) / l
     lse = (mx + np.log(l))[:, 0]
     return u, lse
+
+
+def indexer_kl_row(I_keys: np.ndarray, q_t: np.ndarray, c_keys: np.ndarray, scale: float) -> float:
+    """KL(p_t || Softmax(I_t)) of one query token over a set of keys (velog.io page, Stage 1 Dense Warm-up: the
+    target is the main attention heads' scores summed and L1-normalised; the loss is the KL divergence of the
+    indexer's output distribution from it).
+
+    I_keys: [m] index scores I[t, s] of the keys; q_t: [H, D] queries of token t; c_keys: [m, D] the keys' shared
+    latent entries (all D dims enter the logits, as in attention_row).  The keys are all s <= t in the dense
+    warm-up; over a selected set S_t both distributions are taken over S_t.  Returns the divergence in nats (0 for
+    an empty set).
+    """
+    m = I_keys.shape[0]
+    if m == 0:
+        return 0.0
+    logits = scale * (q_t @ c_keys.T)                 # [H, m]
+    P = np.exp(logits - logits.max(axis=1, keepdims=True))
+    P = P / P.sum(axis=1, keepdims=True)              # each head's attention distribution over the keys
+    a = P.sum(axis=0)                                 # summed over the heads ...
+    p = a / a.sum()                                   # ... and L1-normalised: the target p_{t,:}
+    mI = I_keys.max()
+    log_q = I_keys - (mI + np.log(np.exp(I_keys - mI).sum()))   # log Softmax(I_{t,:})
+    nz = p > 0                                        # 0 log 0 = 0
+    return float((p[nz] * (np.log(p[nz]) - log_q[nz])).sum())
 
 
 def _dequant(bits, scale=None):

@@ -293,3 +293,50 @@ def test_decode_row_equals_prefill_row():
     dec = O.decode_row(keys, step_q, 0, t + 1, k, 0.5, D_v=D_v)
     assert np.array_equal(dec["idx"], pre["idx"][0])
     np.testing.assert_allclose(dec["out"], pre["out"][0], rtol=1e-14)
+
+
+# ------------------------------------------------------------------------------------------ indexer KL objective
+def test_indexer_kl_hand_worked():
+    # velog.io page, Stage 1 Dense Warm-up: target p = the heads' attention summed and L1-normalised, loss
+    # KL(p || Softmax(I)).  Two heads, three keys, scale 1.  Head 0 has logits (0, ln 2, ln 4): probabilities
+    # (1, 2, 4) / 7; head 1 has logits 0: probabilities 1/3 each.  Summed: (10, 13, 19) / 21, L1-normalised:
+    # p = (10, 13, 19) / 42.  I = (0, 0, ln 2): Softmax(I) = (1, 1, 2) / 4.
+    q = np.array([[math.log(2.0), math.log(4.0)], [0.0, 0.0]])
+    c = np.array([[0.0, 0.0], [1.0, 0.0], [0.0, 1.0]])
+    I = np.array([0.0, 0.0, math.log(2.0)])
+    want = (10 / 42) * math.log((10 / 42) / 0.25) + (13 / 42) * math.log((13 / 42) / 0.25) + \
+        (19 / 42) * math.log((19 / 42) / 0.5)
+    assert O.indexer_kl_row(I, q, c, 1.0) == pytest.approx(want, abs=1e-14)
+
+
+def test_indexer_kl_zero_when_the_indexer_matches_the_target():
+    rng = np.random.default_rng(11)
+    q, c = rng.standard_normal((4, 16)), rng.standard_normal((30, 16))
+    logits = 0.25 * q @ c.T
+    P = np.exp(logits) / np.exp(logits).sum(axis=1, keepdims=True)
+    p = P.sum(axis=0) / 4
+    assert O.indexer_kl_row(np.log(p) + 7.5, q, c, 0.25) == pytest.approx(0.0, abs=1e-12)
+    # any other I: strictly positive, and unchanged by a constant shift
+    I = rng.standard_normal(30) * 3
+    kl = O.indexer_kl_row(I, q, c, 0.25)
+    assert kl > 1e-3
+    assert O.indexer_kl_row(I - 40.0, q, c, 0.25) == pytest.approx(kl, rel=1e-12)
+    assert O.indexer_kl_row(np.zeros(0), q, c[:0], 0.25) == 0.0
+
+
+def test_indexer_kl_brute_force_loops():
+    rng = np.random.default_rng(12)
+    H, m, D = 3, 7, 5
+    q, c, I = rng.standard_normal((H, D)), rng.standard_normal((m, D)), rng.standard_normal(m) * 2
+    # pure-Python: each head's softmax, the sum over heads, its L1 normalisation, then the divergence
+    p = [0.0] * m
+    for h in range(H):
+        lg = [0.4 * sum(q[h][d] * c[s][d] for d in range(D)) for s in range(m)]
+        z = sum(math.exp(v) for v in lg)
+        for s in range(m):
+            p[s] += math.exp(lg[s]) / z
+    tot = sum(p)
+    p = [v / tot for v in p]
+    zq = sum(math.exp(v) for v in I)
+    want = sum(p[s] * math.log(p[s] / (math.exp(I[s]) / zq)) for s in range(m))
+    assert O.indexer_kl_row(I, q, c, 0.4) == pytest.approx(want, rel=1e-12)

@@ -335,6 +335,40 @@ def bench_prefill(dsa, cfg, steps, warmup, ws_n, rank, pk):
             "clocks": clk.summary(), "launches": launches}
 
 
+def bench_prefill_sharded(dsa, cfg, steps, warmup, ws_n, rank):
+    """One sequence's prefill with its query rows split zig-zag over the ranks (sparse_attention_long_05_b200.shard):
+    each rank generates the tensors of its own rows, and every step all-gathers the key-side tensors (NCCL) and
+    runs dsa_forward_prefill_rows on the rank's two blocks.  Strong scaling: the job's work is one sequence."""
+    from sparse_attention_long_05_b200 import shard
+    dev = "cuda"
+    L, k = cfg.L, cfg.k
+    rows = shard.rank_rows(L, ws_n, rank)
+    keys = G.prefill_keys(cfg, 1000, device=dev)
+    local_keys = {n: (None if t is None else t[rows].contiguous()) for n, t in keys.items()}
+    del keys
+    local_q = G.prefill_queries(cfg, 1000, rows=rows, device=dev)
+
+    def step():
+        return shard.sharded_prefill(local_q, local_keys, L, k, cfg.scale)
+
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize()
+    barrier(ws_n)
+    torch.cuda.synchronize()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record()
+    for _ in range(steps):
+        res = step()
+    t1.record()
+    torch.cuda.synchronize()
+    barrier(ws_n)
+    ms = max_over_ranks(t0.elapsed_time(t1), ws_n) / steps
+    assert dsa.dsa_get_device_status() == 0
+    del res
+    return {"ms": ms, "tokens_per_s": L / (ms * 1e-3), "rows_per_rank": len(rows)}
+
+
 def bench_prefill_e2e(dsa, cfg, steps, rank):
     """Same metric through dsa_forward_prefill with host buffers: pinned H2D of every input and D2H of
     every output inside the timed region."""
@@ -601,6 +635,9 @@ def parse_args(argv=None):
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-varlen", action="store_true")
     ap.add_argument("--no-configs", action="store_true", help="skip the 8K and 32K prefill lines")
+    ap.add_argument("--prefill-shard", action="store_true",
+                    help="with N > 1: one 128K sequence row-sharded over the N ranks (an all-gather of the key-side "
+                         "tensors per step, strong scaling) instead of one independent sequence per rank")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--kernels-small", action="store_true",
                     help="run one launch of each main kernel on small inputs (profiling) and exit")
@@ -645,6 +682,17 @@ def run_dsa(args, ws_n, rank):
         kernels_small(dsa)
         return
     pk = peaks()
+    if args.prefill_shard and ws_n > 1:
+        sh = bench_prefill_sharded(dsa, PREFILL, args.steps, args.warmup, ws_n, rank)
+        if rank == 0:
+            print(json.dumps({
+                "metric": METRIC, "value": sh["tokens_per_s"], "unit": "tokens/s", "n_gpus": ws_n,
+                "steps": args.steps, "warmup": args.warmup, "ms_per_step": sh["ms"], "higher_is_better": True,
+                "scaling": "strong", "vs_baseline": None, "dtype": "e4m3+bf16", "data": "synthetic",
+                "config": {"workload": PREFILL.name, "seq_len": PREFILL.L, "global_batch": 1,
+                           "parallelism": f"rows{ws_n} (zig-zag query-row blocks, all-gather of k_I, scales and c)",
+                           "rows_per_rank": sh["rows_per_rank"]}}), flush=True)
+        return
     pre = bench_prefill(dsa, PREFILL, args.steps, args.warmup, ws_n, rank, pk)
     torch.cuda.empty_cache()
     dec = None

@@ -114,6 +114,37 @@ DSA_API dsa_status_t dsa_topk(const float* scores, int rows, int64_t ld, const i
 DSA_API dsa_status_t dsa_sparse_mla_attn(const uint16_t* q, const uint16_t* c, int S, const int32_t* idx, int T,
                                  int H, int k, float scale, uint16_t* out, float* lse, void* stream);
 
+/*
+ * The indexer's training objective (velog.io page, Stage 1 Dense Warm-up): for each query token t,
+ *   kl[t] = KL(p_t || Softmax(I_t)),  p_t = the heads' attention probabilities summed and L1-normalised,
+ * both distributions taken over the token's selected entries (all s <= t in the dense warm-up, where the selection
+ * is every earlier token; the selected set S_t in sparse training, a reading of the page, which does not say it).
+ *   q [T, H, 576] bf16, c [S, 576] bf16, idx [T, k] int32: as in dsa_sparse_mla_attn;
+ *   sel_scores [T, k] fp32: the index score I[t, idx[t][i]] of each selected entry (ignored where idx is -1);
+ *   lse [T, H] fp32: the attention's natural-log log-sum-exp per head over the same entries (dsa_sparse_mla_attn's
+ *     lse output), from which the probabilities are formed;
+ *   kl [T] fp32 (out): the divergence in nats (0 for a token without entries).
+ * The logits are recomputed on the tensor cores as in the attention.  Needs no workspace.
+ */
+DSA_API dsa_status_t dsa_indexer_kl(const uint16_t* q, const uint16_t* c, int S, const int32_t* idx,
+                                    const float* sel_scores, const float* lse, int T, int H, int k, float scale,
+                                    float* kl, void* stream);
+
+/* Workspace bytes of dsa_forward_prefill_kl. */
+DSA_API size_t dsa_prefill_kl_workspace_size(int L, int H_I, int d_I, int H, int k);
+
+/*
+ * dsa_forward_prefill plus the indexer objective of every row: the selection also scores the rows t < k (the
+ * objective needs their index scores), the attention writes out and lse, and kl [L] fp32 (out) receives
+ * KL(p_t || Softmax(I_t)) over each row's selected entries, as dsa_indexer_kl.  L_I is the sum of kl over the
+ * rows.  Other arguments as in dsa_forward_prefill (lse may be NULL: the workspace then holds it).
+ */
+DSA_API dsa_status_t dsa_forward_prefill_kl(const uint8_t* q_idx, const float* q_scale, const uint8_t* k_idx,
+                                            const float* k_scale, const float* w, const uint16_t* q,
+                                            const uint16_t* c, int L, int H_I, int d_I, int H, int k, float scale,
+                                            int32_t* idx_out, uint16_t* out, float* lse, float* kl, void* ws,
+                                            size_t ws_bytes, void* stream);
+
 /* Number of kernels this library has launched in this process (all devices, all entry points). */
 DSA_API uint64_t dsa_launch_count(void);
 
@@ -151,6 +182,28 @@ DSA_API dsa_status_t dsa_forward_prefill(const uint8_t* q_idx, const float* q_sc
                                  const float* k_scale, const float* w, const uint16_t* q, const uint16_t* c,
                                  int L, int H_I, int d_I, int H, int k, float scale, int32_t* idx_out,
                                  uint16_t* out, float* lse, void* ws, size_t ws_bytes, void* stream);
+
+/* Workspace bytes of dsa_forward_prefill_rows for the rows [row0, row0 + nrows) of a sequence. */
+DSA_API size_t dsa_prefill_rows_workspace_size(int row0, int nrows, int H_I, int d_I, int H, int k);
+
+/*
+ * Steps 1-3 for the rows [row0, row0 + nrows) of one causal sequence: a block of query rows that attends to all of
+ * the sequence's keys up to its own positions.  With the sequence's rows split over several GPUs (each GPU
+ * computes the query-side tensors of its own rows and receives every key-side tensor), each GPU calls this for
+ * each of its blocks.  The pages describe the computation of one sequence; this is that computation for a
+ * subset of its rows.  Results are bitwise identical to the same rows of dsa_forward_prefill.
+ *   q_idx [nrows, H_I, d_I] e4m3, q_scale [nrows] or NULL, w [nrows, H_I] fp32, q [nrows, H, 576] bf16: the
+ *     block's query-side tensors (row i is position row0 + i);
+ *   k_idx [>= row0 + nrows, d_I] e4m3, k_scale [>= row0 + nrows] or NULL, c [>= row0 + nrows, 576] bf16: the
+ *     sequence's key-side tensors from position 0 (rows past row0 + nrows - 1 are not read);
+ *   idx_out [nrows, k] int32 (out, may be NULL), out [nrows, H, 512] bf16 (out), lse [nrows, H] fp32 (out, may be
+ *     NULL), as in dsa_forward_prefill.
+ */
+DSA_API dsa_status_t dsa_forward_prefill_rows(const uint8_t* q_idx, const float* q_scale, const uint8_t* k_idx,
+                                              const float* k_scale, const float* w, const uint16_t* q,
+                                              const uint16_t* c, int row0, int nrows, int H_I, int d_I, int H, int k,
+                                              float scale, int32_t* idx_out, uint16_t* out, float* lse, void* ws,
+                                              size_t ws_bytes, void* stream);
 
 /* Workspace bytes of dsa_forward_prefill_varlen: nseq sequences of `total` rows in all, the longest max_len. */
 DSA_API size_t dsa_prefill_varlen_workspace_size(int nseq, int64_t total, int max_len, int H_I, int d_I, int H,
@@ -207,6 +260,37 @@ DSA_API dsa_status_t dsa_forward_decode(int B, const int64_t* cache_off, const i
                                 float* k_scale_cache, uint16_t* c_cache, int64_t cache_rows, int H_I, int d_I,
                                 int H, int k, float scale, int32_t* idx_out, uint16_t* out, float* lse, void* ws,
                                 size_t ws_bytes, void* stream);
+
+/* Workspace bytes of dsa_forward_decode_paged for a batch of B sequences whose page tables hold max_pages
+ * entries of page_rows positions. */
+DSA_API size_t dsa_decode_paged_workspace_size(int B, int max_pages, int page_rows, int H_I, int d_I, int H, int k);
+
+/*
+ * dsa_forward_decode over paged caches.  The pages describe one cache per sequence; a serving system keeps the
+ * caches of many sequences in pools of fixed-size pages (macaron.im page, decode cost at 128K: the decode reads
+ * the indexer keys and the selected latent entries of every sequence of the batch), and this is the same decode
+ * step with the positions of each sequence mapped through a page table.
+ *   page_table [B, max_pages] int32 (device): position p of sequence b is row
+ *     page_table[b][p / page_rows] * page_rows + p % page_rows of the pools;
+ *   page_rows: positions per page, a positive multiple of 128 (a 128-key indexer tile lies in one page);
+ *   k_cache [num_pages * page_rows, d_I] e4m3, k_scale_cache [num_pages * page_rows] fp32,
+ *   c_cache [num_pages * page_rows, 576] bf16: the page pools (in/out), at most INT32_MAX rows;
+ *   every other argument as in dsa_forward_decode (ctx_len[b] positions before the call; the new entries go to
+ *   position ctx_len[b]).
+ * Pages may be shared between sequences (a common prefix) except the page that receives the new entry.  A
+ * sequence whose new position falls outside its table (ctx_len[b] / page_rows >= max_pages) or whose table names
+ * a page outside [0, num_pages) among the pages 0 .. ctx_len[b] / page_rows sets DSA_ERR_BAD_INDEX, and nothing
+ * of it is read or written, as in dsa_forward_decode.  Results are bitwise identical to dsa_forward_decode's over
+ * flat caches holding the same entries.  Returns DSA_ERR_UNSUPPORTED_SHAPE for a page_rows that is not a
+ * multiple of 128 and the errors of dsa_forward_decode otherwise.
+ */
+DSA_API dsa_status_t dsa_forward_decode_paged(int B, const int32_t* page_table, int max_pages, int page_rows,
+                                              const int32_t* ctx_len, const uint8_t* q_idx, const float* q_scale,
+                                              const float* w, const uint16_t* q, const uint8_t* k_new,
+                                              const float* k_scale_new, const uint16_t* c_new, uint8_t* k_cache,
+                                              float* k_scale_cache, uint16_t* c_cache, int num_pages, int H_I,
+                                              int d_I, int H, int k, float scale, int32_t* idx_out, uint16_t* out,
+                                              float* lse, void* ws, size_t ws_bytes, void* stream);
 
 /*
  * dsa_forward_decode without a caller-provided workspace, for callers that cannot allocate device memory

@@ -28,17 +28,27 @@ SIGNATURES = {
     "dsa_indexer_scores": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P, _P]),
     "dsa_topk": (_I, [_P, _I, _I64, _P, _I, _I, _P, _P]),
     "dsa_sparse_mla_attn": (_I, [_P, _P, _I, _P, _I, _I, _I, _F, _P, _P, _P]),
+    "dsa_indexer_kl": (_I, [_P, _P, _I, _P, _P, _P, _I, _I, _I, _F, _P, _P]),
+    "dsa_prefill_kl_workspace_size": (_SZ, [_I, _I, _I, _I, _I]),
+    "dsa_forward_prefill_kl": (_I, [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _P, _P, _P, _P, _P, _SZ,
+                                    _P]),
     "dsa_launch_count": (ctypes.c_uint64, []),
     "dsa_prefill_block_rows": (_I, [_I, _I, _I]),
     "dsa_prefill_workspace_size": (_SZ, [_I, _I, _I, _I, _I]),
     "dsa_prefill_select": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _P, _P, _SZ, _P]),
     "dsa_forward_prefill": (_I, [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _P, _P, _P, _P, _SZ, _P]),
+    "dsa_prefill_rows_workspace_size": (_SZ, [_I, _I, _I, _I, _I, _I]),
+    "dsa_forward_prefill_rows": (_I, [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _P, _P, _P, _P, _SZ,
+                                      _P]),
     "dsa_prefill_varlen_workspace_size": (_SZ, [_I, _I64, _I, _I, _I, _I, _I]),
     "dsa_forward_prefill_varlen": (_I, [_I, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _F, _P, _P, _P, _P, _SZ,
                                         _P]),
     "dsa_decode_workspace_size": (_SZ, [_I, _I64, _I, _I, _I, _I]),
     "dsa_forward_decode": (_I, [_I, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _I64, _I, _I, _I, _I, _F,
                                 _P, _P, _P, _P, _SZ, _P]),
+    "dsa_decode_paged_workspace_size": (_SZ, [_I, _I, _I, _I, _I, _I, _I]),
+    "dsa_forward_decode_paged": (_I, [_I, _P, _I, _I, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I,
+                                      _F, _P, _P, _P, _P, _SZ, _P]),
     "dsa_decode_noalloc_scratch_bytes": (_SZ, []),
     "dsa_forward_decode_noalloc": (_I, [_I, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _I64, _I, _I, _I, _I,
                                         _F, _P, _P, _P, _P]),
@@ -138,6 +148,46 @@ def dsa_sparse_mla_attn(q, c, idx, scale: float, out=None, lse=None, want_lse: b
     return out, lse
 
 
+def dsa_indexer_kl(q, c, idx, sel_scores, lse, scale: float, kl=None, stream=None):
+    """KL(p_t || Softmax(I_t)) [T] of each token over its selected entries, from the attention's lse [T, H] and the
+    selected entries' index scores sel_scores [T, k]."""
+    T, H, _ = q.shape
+    S = c.shape[0]
+    k = idx.shape[1]
+    if kl is None:
+        kl = torch.empty((T,), dtype=torch.float32, device=q.device)
+    _check("dsa_indexer_kl", _lib.dsa_indexer_kl(
+        _ptr(q), _ptr(c), S, _ptr(idx), _ptr(sel_scores), _ptr(lse), T, H, k, float(scale), _ptr(kl),
+        _stream(stream)))
+    return kl
+
+
+def dsa_prefill_kl_workspace_size(L: int, H_I: int, d_I: int, H: int, k: int) -> int:
+    return int(_lib.dsa_prefill_kl_workspace_size(L, H_I, d_I, H, k))
+
+
+def dsa_forward_prefill_kl(q_idx, q_scale, k_idx, k_scale, w, q, c, k: int, scale: float, idx_out=None, out=None,
+                           lse=None, kl=None, ws=None, stream=None):
+    """DSA forward of one causal prefill sequence plus the indexer objective per row -> (idx, out, lse, kl [L])."""
+    L, H_I, d_I = q_idx.shape
+    H = q.shape[1]
+    dev = q.device
+    if idx_out is None:
+        idx_out = torch.empty((L, k), dtype=torch.int32, device=dev)
+    if out is None:
+        out = torch.empty((L, H, 512), dtype=torch.bfloat16, device=dev)
+    if lse is None:
+        lse = torch.empty((L, H), dtype=torch.float32, device=dev)
+    if kl is None:
+        kl = torch.empty((L,), dtype=torch.float32, device=dev)
+    if ws is None:
+        ws = torch.empty((dsa_prefill_kl_workspace_size(L, H_I, d_I, H, k),), dtype=torch.uint8, device=dev)
+    _check("dsa_forward_prefill_kl", _lib.dsa_forward_prefill_kl(
+        _ptr(q_idx), _ptr(q_scale), _ptr(k_idx), _ptr(k_scale), _ptr(w), _ptr(q), _ptr(c), L, H_I, d_I, H, k,
+        float(scale), _ptr(idx_out), _ptr(out), _ptr(lse), _ptr(kl), _ptr(ws), ws.numel(), _stream(stream)))
+    return idx_out, out, lse, kl
+
+
 def dsa_prefill_workspace_size(L: int, H_I: int, d_I: int, H: int, k: int) -> int:
     return int(_lib.dsa_prefill_workspace_size(L, H_I, d_I, H, k))
 
@@ -192,6 +242,32 @@ def dsa_forward_prefill(q_idx, q_scale, k_idx, k_scale, w, q, c, k: int, scale: 
     _check("dsa_forward_prefill", _lib.dsa_forward_prefill(
         _ptr(q_idx), _ptr(q_scale), _ptr(k_idx), _ptr(k_scale), _ptr(w), _ptr(q), _ptr(c), L, H_I, d_I, H, k,
         float(scale), _ptr(idx_out), _ptr(out), _ptr(lse), _ptr(ws), ws.numel(), _stream(stream)))
+    return idx_out, out, lse
+
+
+def dsa_prefill_rows_workspace_size(row0: int, nrows: int, H_I: int, d_I: int, H: int, k: int) -> int:
+    return int(_lib.dsa_prefill_rows_workspace_size(row0, nrows, H_I, d_I, H, k))
+
+
+def dsa_forward_prefill_rows(row0: int, q_idx, q_scale, k_idx, k_scale, w, q, c, k: int, scale: float, idx_out=None,
+                             out=None, lse=None, ws=None, stream=None):
+    """Steps 1-3 for the rows row0 .. row0 + nrows - 1 of one causal sequence (query-side tensors of those rows,
+    key-side tensors of the sequence from position 0) -> (idx [nrows, k], out [nrows, H, 512], lse [nrows, H])."""
+    nrows, H_I, d_I = q_idx.shape
+    H = q.shape[1]
+    dev = q.device
+    if idx_out is None:
+        idx_out = torch.empty((nrows, k), dtype=torch.int32, device=dev)
+    if out is None:
+        out = torch.empty((nrows, H, 512), dtype=torch.bfloat16, device=dev)
+    if lse is None:
+        lse = torch.empty((nrows, H), dtype=torch.float32, device=dev)
+    if ws is None:
+        ws = torch.empty((dsa_prefill_rows_workspace_size(row0, nrows, H_I, d_I, H, k),), dtype=torch.uint8,
+                         device=dev)
+    _check("dsa_forward_prefill_rows", _lib.dsa_forward_prefill_rows(
+        _ptr(q_idx), _ptr(q_scale), _ptr(k_idx), _ptr(k_scale), _ptr(w), _ptr(q), _ptr(c), row0, nrows, H_I, d_I, H,
+        k, float(scale), _ptr(idx_out), _ptr(out), _ptr(lse), _ptr(ws), ws.numel(), _stream(stream)))
     return idx_out, out, lse
 
 
@@ -251,6 +327,37 @@ def dsa_forward_decode(cache_off, ctx_len, q_idx, q_scale, w, q, k_new, k_scale_
         B, _ptr(cache_off), _ptr(ctx_len), _ptr(q_idx), _ptr(q_scale), _ptr(w), _ptr(q), _ptr(k_new),
         _ptr(k_scale_new), _ptr(c_new), _ptr(k_cache), _ptr(k_scale_cache), _ptr(c_cache), rows, H_I, d_I, H, k,
         float(scale), _ptr(idx_out), _ptr(out), _ptr(lse), _ptr(ws), ws.numel(), _stream(stream)))
+    return idx_out, out, lse
+
+
+def dsa_decode_paged_workspace_size(B: int, max_pages: int, page_rows: int, H_I: int, d_I: int, H: int,
+                                    k: int) -> int:
+    return int(_lib.dsa_decode_paged_workspace_size(B, max_pages, page_rows, H_I, d_I, H, k))
+
+
+def dsa_forward_decode_paged(page_table, page_rows: int, ctx_len, q_idx, q_scale, w, q, k_new, k_scale_new, c_new,
+                             k_cache, k_scale_cache, c_cache, k: int, scale: float, idx_out=None, out=None, lse=None,
+                             ws=None, stream=None):
+    """One decode step over paged caches (page_table [B, max_pages] int32; pools of page_rows-row pages)
+    -> (idx, out, lse)."""
+    B, H_I, d_I = q_idx.shape
+    H = q.shape[1]
+    max_pages = page_table.shape[1]
+    num_pages = k_cache.shape[0] // page_rows
+    dev = q.device
+    if idx_out is None:
+        idx_out = torch.empty((B, k), dtype=torch.int32, device=dev)
+    if out is None:
+        out = torch.empty((B, H, 512), dtype=torch.bfloat16, device=dev)
+    if lse is None:
+        lse = torch.empty((B, H), dtype=torch.float32, device=dev)
+    if ws is None:
+        ws = torch.empty((dsa_decode_paged_workspace_size(B, max_pages, page_rows, H_I, d_I, H, k),),
+                         dtype=torch.uint8, device=dev)
+    _check("dsa_forward_decode_paged", _lib.dsa_forward_decode_paged(
+        B, _ptr(page_table), max_pages, page_rows, _ptr(ctx_len), _ptr(q_idx), _ptr(q_scale), _ptr(w), _ptr(q),
+        _ptr(k_new), _ptr(k_scale_new), _ptr(c_new), _ptr(k_cache), _ptr(k_scale_cache), _ptr(c_cache), num_pages,
+        H_I, d_I, H, k, float(scale), _ptr(idx_out), _ptr(out), _ptr(lse), _ptr(ws), ws.numel(), _stream(stream)))
     return idx_out, out, lse
 
 

@@ -14,6 +14,7 @@
 #include "indexer.cuh"
 #include "sparse_mla.cuh"
 #include "topk.cuh"
+#include "topk_cluster.cuh"
 
 namespace dsa {
 
@@ -33,23 +34,54 @@ __device__ __forceinline__ bool decode_seq_valid(const long long* cache_off, con
   return off >= 0 && n >= 0 && off + n < cache_rows;
 }
 
+// Paged caches: the caches are pools of pages of page_rows rows; row (page_table[b][pos / page_rows] * page_rows +
+// pos % page_rows) holds position pos of sequence b.  A sequence is valid when its new position ctx_len[b] falls
+// inside its table and every page up to it is in [0, num_pages).  Every thread of the CTA calls this.
+__device__ __forceinline__ bool decode_seq_valid_paged(const int* page_table, int max_pages, int page_rows,
+                                                       long long num_pages, const int* ctx_len, int b) {
+  __shared__ int bad;
+  const int n = ctx_len[b];
+  if (threadIdx.x == 0) bad = (n < 0 || n / page_rows >= max_pages) ? 1 : 0;
+  __syncthreads();
+  if (!bad) {
+    const int* row = page_table + static_cast<long long>(b) * max_pages;
+    for (int j = threadIdx.x; j <= n / page_rows; j += blockDim.x)
+      if (row[j] < 0 || row[j] >= num_pages) bad = 1;
+  }
+  __syncthreads();
+  return bad == 0;
+}
+
 __device__ __forceinline__ long long padded4(long long n) { return (n + 3) & ~3ll; }
 
 constexpr int kAppendThreads = 128;
 
+// Cache layout of a decode step: flat (sequence b owns rows cache_off[b] ..) or paged (page_table non-null).
+struct DecodeLayout {
+  const long long* cache_off;   // flat: [B]
+  long long cache_rows;         // flat: rows of the caches
+  const int* page_table;        // paged: [B, max_pages], or null
+  int max_pages, page_rows;
+  long long num_pages;
+};
+
 __global__ void __launch_bounds__(kAppendThreads)
-    decode_append_kernel(int B, const long long* cache_off, const int* ctx_len, long long cache_rows,
-                         const uint8_t* k_new, const float* k_scale_new, const uint16_t* c_new, uint8_t* k_cache,
-                         float* k_scale_cache, uint16_t* c_cache, int d_I, int* len1, long long* score_off,
-                         long long score_cap) {
+    decode_append_kernel(int B, DecodeLayout lay, const int* ctx_len, const uint8_t* k_new,
+                         const float* k_scale_new, const uint16_t* c_new, uint8_t* k_cache, float* k_scale_cache,
+                         uint16_t* c_cache, int d_I, int* len1, long long* score_off, long long score_cap) {
   const int b = blockIdx.x;
   if (b >= B) return;
-  // start of this sequence's score row: the padded lengths of the valid sequences before it
+  // start of this sequence's score row: the padded lengths of the sequences before it that pass the cheap part
+  // of their check (paged: the page-table entries of another sequence are not read here; a sequence that fails
+  // only on those keeps its reserved row unused)
   __shared__ long long part[kAppendThreads / 32];
   long long acc = 0;
-  for (int j = threadIdx.x; j < b; j += blockDim.x)
-    if (decode_seq_valid(cache_off, ctx_len, cache_rows, j))
-      acc += padded4(static_cast<long long>(ctx_len[j]) + 1);
+  for (int j = threadIdx.x; j < b; j += blockDim.x) {
+    const int nj = ctx_len[j];
+    if (lay.page_table ? (nj >= 0 && nj / lay.page_rows < lay.max_pages)
+                       : decode_seq_valid(lay.cache_off, ctx_len, lay.cache_rows, j))
+      acc += padded4(static_cast<long long>(nj) + 1);
+  }
 #pragma unroll
   for (int d = 16; d > 0; d >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, d);
   if ((threadIdx.x & 31) == 0) part[threadIdx.x >> 5] = acc;
@@ -57,13 +89,19 @@ __global__ void __launch_bounds__(kAppendThreads)
   long long s0 = 0;
 #pragma unroll
   for (int w = 0; w < kAppendThreads / 32; ++w) s0 += part[w];
-  const bool valid = decode_seq_valid(cache_off, ctx_len, cache_rows, b) &&
-                     s0 + padded4(static_cast<long long>(ctx_len[b]) + 1) <= score_cap;
+  const bool fits = s0 + padded4(static_cast<long long>(ctx_len[b]) + 1) <= score_cap;
+  const bool valid = (lay.page_table ? decode_seq_valid_paged(lay.page_table, lay.max_pages, lay.page_rows,
+                                                              lay.num_pages, ctx_len, b)
+                                     : decode_seq_valid(lay.cache_off, ctx_len, lay.cache_rows, b)) && fits;
   if (!valid) {
     if (threadIdx.x == 0) { raise_status(DSA_ERR_BAD_INDEX); len1[b] = 0; score_off[b] = 0; }
     return;
   }
-  const long long row = cache_off[b] + ctx_len[b];
+  const int n = ctx_len[b];
+  const long long row = lay.page_table
+      ? static_cast<long long>(lay.page_table[static_cast<long long>(b) * lay.max_pages + n / lay.page_rows]) *
+            lay.page_rows + n % lay.page_rows
+      : lay.cache_off[b] + n;
   const uint4* ks = reinterpret_cast<const uint4*>(k_new + static_cast<long long>(b) * d_I);
   uint4* kd = reinterpret_cast<uint4*>(k_cache + row * d_I);
   for (int i = threadIdx.x; i < d_I / 16; i += blockDim.x) kd[i] = ks[i];
@@ -240,14 +278,13 @@ dsa_status_t run_indexer_scores(const uint8_t* q_idx, const float* q_scale, cons
 }
 
 dsa_status_t run_topk(const float* scores, long long ld, const long long* row_off, const int* row_len, int pos0,
-                      int rows, int k, int* idx, long long idx_ld, cudaStream_t st) {
+                      int rows, int k, int* idx, long long idx_ld, cudaStream_t st, float* sel_scores = nullptr) {
   if (rows <= 0) return DSA_OK;
-  TopkParams p{scores, ld, row_off, row_len, pos0, rows, k, idx, idx_ld};
+  TopkParams p{scores, ld, row_off, row_len, pos0, rows, k, idx, idx_ld, sel_scores};
   if (rows < num_sms()) {
-    // fewer rows than SMs (decode): one 1024-thread CTA per row
-    if (set_smem(topk_rows_kernel<kTopkThreadsFew>, static_cast<int>(sizeof(TopkSmem<kTopkThreadsFew>))) != cudaSuccess)
-      return DSA_ERR_CUDA;
-    topk_rows_kernel<kTopkThreadsFew><<<rows, kTopkThreadsFew, sizeof(TopkSmem<kTopkThreadsFew>), st>>>(p);
+    // fewer rows than SMs (decode): one cluster of kTkcCluster CTAs per row
+    if (set_smem(topk_cluster_kernel, static_cast<int>(sizeof(TkcSmem))) != cudaSuccess) return DSA_ERR_CUDA;
+    topk_cluster_kernel<<<rows * kTkcCluster, kTkcThreads, sizeof(TkcSmem), st>>>(p);
   } else {
     if (set_smem(topk_rows_kernel<kTopkThreads>, static_cast<int>(sizeof(TopkSmem<kTopkThreads>))) != cudaSuccess)
       return DSA_ERR_CUDA;
@@ -256,8 +293,14 @@ dsa_status_t run_topk(const float* scores, long long ld, const long long* row_of
   return last_launch_status();
 }
 
+// Attention launch.  dense: kMlaSparse (every token gathers its index row), kMlaCausal (token t has the
+// t - row_off[t] + 1 keys of its sequence) or kMlaCounts (token t has n_keys[t] keys); in the dense modes a
+// token with at most k keys attends to all of them, read as contiguous tiles.
 dsa_status_t run_mla(const uint16_t* q, const uint16_t* c, long long S, const int* idx, const long long* row_off,
-                     int T, int H, int k, float scale, uint16_t* out, float* lse, cudaStream_t st) {
+                     int T, int H, int k, float scale, uint16_t* out, float* lse, cudaStream_t st,
+                     int dense = kMlaSparse, const int* n_keys = nullptr, const int* page_table = nullptr,
+                     int pt_stride = 0, int page_rows = 0, int pos0 = 0, const float* kl_lse = nullptr,
+                     const float* kl_scores = nullptr, float* kl_out = nullptr) {
   if (T <= 0) return DSA_OK;
   CUtensorMap tq;
   const cuuint64_t qd[3] = {576, static_cast<cuuint64_t>(H), static_cast<cuuint64_t>(T)};
@@ -269,7 +312,20 @@ dsa_status_t run_mla(const uint16_t* q, const uint16_t* c, long long S, const in
   const cuuint64_t cs[1] = {576 * 2};
   const cuuint32_t cb[2] = {64, 1};
   if (!make_map(&tc, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, c, cd, cs, cb, CU_TENSOR_MAP_SWIZZLE_128B)) return DSA_ERR_CUDA;
+  CUtensorMap tcd;  // contiguous tiles of c: one 64-column box 64 rows high (dense tokens)
+  const cuuint32_t cbd[2] = {64, 64};
+  if (!make_map(&tcd, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, c, cd, cs, cbd, CU_TENSOR_MAP_SWIZZLE_128B))
+    return DSA_ERR_CUDA;
   MlaParams p{};
+  p.dense = dense;
+  p.pos0 = pos0;
+  p.n_keys = n_keys;
+  p.page_table = page_table;
+  p.pt_stride = pt_stride;
+  p.page_rows = page_rows;
+  p.kl_lse = kl_lse;
+  p.kl_scores = kl_scores;
+  p.kl_out = kl_out;
   p.idx = idx;
   p.row_off = row_off;
   p.out = out;
@@ -280,9 +336,11 @@ dsa_status_t run_mla(const uint16_t* q, const uint16_t* c, long long S, const in
   p.S = S;
   p.scale_log2 = scale * 1.4426950408889634f;
   if (set_smem(sparse_mla_kernel, mla::SMEM) != cudaSuccess) return DSA_ERR_CUDA;
+  // KL mode: every CTA takes tokens of its own (the grid still comes in pairs, the kernel's cluster shape)
+  const int per_cluster = kl_out ? 2 : 1;
   int clusters = num_sms() / 2;
-  if (clusters > T) clusters = T;
-  sparse_mla_kernel<<<2 * clusters, mla::THREADS, mla::SMEM, st>>>(tq, tc, p);
+  if (clusters > (T + per_cluster - 1) / per_cluster) clusters = (T + per_cluster - 1) / per_cluster;
+  sparse_mla_kernel<<<2 * clusters, mla::THREADS, mla::SMEM, st>>>(tq, tc, tcd, p);
   return last_launch_status();
 }
 
@@ -296,6 +354,33 @@ size_t prefill_chunk_rows(int L) {
   if (r < 256) r = 256;
   if (r > size_t(L)) r = size_t(L);
   return r;
+}
+
+// Steps 1-2 for rows [pos_begin, pos_end) of one causal sequence (row r attends to keys 0..r): q_idx, q_scale, w and
+// idx_out point at row pos_begin; k_idx, k_scale hold keys 0..pos_end-1.  Rows t < k form one block whose
+// selection needs no scores; later rows go in blocks of chunk_rows, each an indexer launch into `sc` (room for
+// chunk_rows x pos_end scores) and a top-k launch.  With sel_scores (pointing at row pos_begin), the index score of
+// every selected position is written too, and the indexer then also scores the rows t < k.
+dsa_status_t select_rows(const uint8_t* q_idx, const float* q_scale, const uint8_t* k_idx, const float* k_scale,
+                         const float* w, int H_I, int d_I, int k, int pos_begin, int pos_end, int32_t* idx_out,
+                         float* sc, size_t chunk_rows, cudaStream_t st, float* sel_scores = nullptr) {
+  for (int r0 = pos_begin, rows = 0; r0 < pos_end; r0 += rows) {
+    rows = (r0 < k) ? std::min(k, pos_end) - r0 : static_cast<int>(std::min<size_t>(chunk_rows, pos_end - r0));
+    const int s_eff = r0 + rows;   // keys beyond the block's last row are never selected (causal)
+    const size_t i = static_cast<size_t>(r0 - pos_begin);
+    // a block whose every row t has t + 1 <= k selects all of 0..t whatever the scores: no indexer launch (the
+    // top-k kernel writes 0..t and the -1 padding of such rows without reading them)
+    dsa_status_t e = DSA_OK;
+    if (s_eff > k || sel_scores) {
+      e = run_indexer_scores(q_idx + i * H_I * d_I, q_scale ? q_scale + i : nullptr, k_idx, k_scale, w + i * H_I,
+                             rows, s_eff, H_I, d_I, r0, sc, s_eff, st);
+      if (e != DSA_OK) return e;
+    }
+    e = run_topk(sc, s_eff, nullptr, nullptr, r0, rows, k, idx_out + i * k, k, st,
+                 sel_scores ? sel_scores + i * k : nullptr);
+    if (e != DSA_OK) return e;
+  }
+  return DSA_OK;
 }
 
 // Rows of the score block of an L-row prefill that starts at row r0: rows t < k form a block of their own, whose
@@ -322,6 +407,55 @@ dsa_status_t decode_args_status(int B, const int64_t* cache_off, const int32_t* 
       !aligned16(c_cache) || !aligned16(out) || (idx_out && !aligned16(idx_out)))
     return DSA_ERR_ALIGNMENT;
   return DSA_OK;
+}
+
+size_t decode_ws_bytes(int B, size_t score_cap, int k) {
+  return align_up(score_cap * 4, 256) + align_up(size_t(B) * 4, 256) + align_up(size_t(B) * 8, 256) +
+         align_up(size_t(B) * k * 4, 256);
+}
+
+// One decode step once the arguments are checked: append -> indexer over each sequence's keys -> top-k -> sparse
+// MLA.  Workspace: score rows (packed, 16-byte aligned, score_cap floats), len1 [B], score_off [B], selected
+// indices [B, k] (when idx_out is null).
+dsa_status_t run_decode(int B, const DecodeLayout& lay, const int32_t* ctx_len, const uint8_t* q_idx,
+                        const float* q_scale, const float* w, const uint16_t* q, const uint8_t* k_new,
+                        const float* k_scale_new, const uint16_t* c_new, uint8_t* k_cache, float* k_scale_cache,
+                        uint16_t* c_cache, size_t score_cap, int H, int k, float scale, int32_t* idx_out,
+                        uint16_t* out, float* lse, void* ws, cudaStream_t st) {
+  constexpr int H_I = 64, d_I = 128;
+  char* wsb = static_cast<char*>(ws);
+  float* dscores = reinterpret_cast<float*>(wsb);
+  size_t at = align_up(score_cap * 4, 256);
+  int* len1 = reinterpret_cast<int*>(wsb + at);
+  at += align_up(size_t(B) * 4, 256);
+  long long* soff = reinterpret_cast<long long*>(wsb + at);
+  at += align_up(size_t(B) * 8, 256);
+  int32_t* idx = idx_out ? idx_out : reinterpret_cast<int32_t*>(wsb + at);
+  decode_append_kernel<<<B, kAppendThreads, 0, st>>>(B, lay, ctx_len, k_new, k_scale_new, c_new, k_cache,
+                                                     k_scale_cache, c_cache, d_I, len1, soff,
+                                                     static_cast<long long>(score_cap));
+  dsa_status_t e = last_launch_status();
+  if (e != DSA_OK) return e;
+  IndexerParams p{};
+  p.w = w;
+  p.q_scale = q_scale;
+  p.k_scale = k_scale_cache;
+  p.scores = dscores;
+  p.T = B;
+  p.cache_off = lay.cache_off;
+  p.len1 = len1;
+  p.score_off = soff;
+  p.page_table = lay.page_table;
+  p.max_pages = lay.max_pages;
+  p.page_rows = lay.page_rows;
+  using DecCfg = IndexerCfg<H_I, d_I, 1, 1, 2, 4, 1, kModeDecode>;
+  e = launch_indexer<H_I, d_I, 1, 1, 2, 4, 1, kModeDecode>(q_idx, B, k_cache, lay.cache_rows, p,
+                                                         DecCfg::CTAS_PER_SM * num_sms(), st);
+  if (e != DSA_OK) return e;
+  e = run_topk(dscores, 0, soff, len1, 0, B, k, idx, k, st);
+  if (e != DSA_OK) return e;
+  return run_mla(q, c_cache, lay.cache_rows, idx, lay.cache_off, B, H, k, scale, out, lse, st, kMlaCounts, len1,
+                 lay.page_table, lay.max_pages, lay.page_rows);
 }
 
 }  // namespace
@@ -376,6 +510,50 @@ dsa_status_t dsa_topk(const float* scores, int rows, int64_t ld, const int32_t* 
   return run_topk(scores, ld, nullptr, row_len, pos0, rows, k, idx, k, static_cast<cudaStream_t>(stream));
 }
 
+dsa_status_t dsa_indexer_kl(const uint16_t* q, const uint16_t* c, int S, const int32_t* idx, const float* sel_scores,
+                            const float* lse, int T, int H, int k, float scale, float* kl, void* stream) {
+  if (T < 0 || S <= 0 || H <= 0 || k <= 0 || (T > 0 && (!q || !c || !idx || !sel_scores || !lse || !kl)))
+    return DSA_ERR_INVALID_ARG;
+  if (H > 128 || !mla_k_ok(k)) return DSA_ERR_UNSUPPORTED_SHAPE;
+  if (!aligned16(q) || !aligned16(c) || !aligned16(idx)) return DSA_ERR_ALIGNMENT;
+  return run_mla(q, c, S, idx, nullptr, T, H, k, scale, nullptr, nullptr, static_cast<cudaStream_t>(stream),
+                 kMlaSparse, nullptr, nullptr, 0, 0, 0, lse, sel_scores, kl);
+}
+
+size_t dsa_prefill_kl_workspace_size(int L, int H_I, int d_I, int H, int k) {
+  if (L <= 0 || k <= 0 || H <= 0) return 0;
+  return dsa_prefill_workspace_size(L, H_I, d_I, H, k) + align_up(size_t(L) * size_t(k) * 4, 256) +
+         align_up(size_t(L) * size_t(H) * 4, 256);
+}
+
+dsa_status_t dsa_forward_prefill_kl(const uint8_t* q_idx, const float* q_scale, const uint8_t* k_idx,
+                                    const float* k_scale, const float* w, const uint16_t* q, const uint16_t* c,
+                                    int L, int H_I, int d_I, int H, int k, float scale, int32_t* idx_out,
+                                    uint16_t* out, float* lse, float* kl, void* ws, size_t ws_bytes, void* stream) {
+  if (L <= 0 || H <= 0 || k <= 0 || !q_idx || !k_idx || !w || !q || !c || !out || !kl) return DSA_ERR_INVALID_ARG;
+  if (!indexer_shape_ok(H_I, d_I) || H > 128 || !mla_k_ok(k)) return DSA_ERR_UNSUPPORTED_SHAPE;
+  if (!aligned16(q_idx) || !aligned16(k_idx) || !aligned16(q) || !aligned16(c) || !aligned16(out) ||
+      (idx_out && !aligned16(idx_out)))
+    return DSA_ERR_ALIGNMENT;
+  if (!ws || ws_bytes < dsa_prefill_kl_workspace_size(L, H_I, d_I, H, k)) return DSA_ERR_WORKSPACE;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  // workspace: the prefill's (score block, selected indices), then the selected index scores [L, k] and lse [L, H]
+  char* wsb = static_cast<char*>(ws);
+  const size_t score_bytes = align_up(prefill_chunk_rows(L) * size_t(L) * 4, 256);
+  int32_t* idx = idx_out ? idx_out : reinterpret_cast<int32_t*>(wsb + score_bytes);
+  size_t at = dsa_prefill_workspace_size(L, H_I, d_I, H, k);
+  float* sel = reinterpret_cast<float*>(wsb + at);
+  at += align_up(size_t(L) * size_t(k) * 4, 256);
+  float* lse_buf = lse ? lse : reinterpret_cast<float*>(wsb + at);
+  dsa_status_t e = select_rows(q_idx, q_scale, k_idx, k_scale, w, H_I, d_I, k, 0, L, idx, reinterpret_cast<float*>(wsb),
+                               prefill_chunk_rows(L), st, sel);
+  if (e != DSA_OK) return e;
+  e = run_mla(q, c, L, idx, nullptr, L, H, k, scale, out, lse_buf, st, kMlaCausal);
+  if (e != DSA_OK) return e;
+  return run_mla(q, c, L, idx, nullptr, L, H, k, scale, nullptr, nullptr, st, kMlaCausal, nullptr, nullptr, 0, 0, 0,
+                 lse_buf, sel, kl);
+}
+
 dsa_status_t dsa_sparse_mla_attn(const uint16_t* q, const uint16_t* c, int S, const int32_t* idx, int T, int H,
                                  int k, float scale, uint16_t* out, float* lse, void* stream) {
   if (T < 0 || S <= 0 || H <= 0 || k <= 0 || (T > 0 && (!q || !c || !idx || !out))) return DSA_ERR_INVALID_ARG;
@@ -398,23 +576,38 @@ dsa_status_t dsa_prefill_select(const uint8_t* q_idx, const float* q_scale, cons
   if (!indexer_shape_ok(H_I, d_I)) return DSA_ERR_UNSUPPORTED_SHAPE;
   if (!aligned16(q_idx) || !aligned16(k_idx)) return DSA_ERR_ALIGNMENT;
   if (!ws || ws_bytes < align_up(prefill_chunk_rows(L) * size_t(L) * 4, 256)) return DSA_ERR_WORKSPACE;
+  return select_rows(q_idx, q_scale, k_idx, k_scale, w, H_I, d_I, k, 0, L, idx_out, static_cast<float*>(ws),
+                     prefill_chunk_rows(L), static_cast<cudaStream_t>(stream));
+}
+
+size_t dsa_prefill_rows_workspace_size(int row0, int nrows, int H_I, int d_I, int H, int k) {
+  (void)H_I; (void)d_I; (void)H;
+  if (row0 < 0 || nrows <= 0 || k <= 0) return 0;
+  const int S = row0 + nrows;
+  return align_up(prefill_chunk_rows(S) * size_t(S) * 4, 256) + align_up(size_t(nrows) * size_t(k) * 4, 256);
+}
+
+dsa_status_t dsa_forward_prefill_rows(const uint8_t* q_idx, const float* q_scale, const uint8_t* k_idx,
+                                      const float* k_scale, const float* w, const uint16_t* q, const uint16_t* c,
+                                      int row0, int nrows, int H_I, int d_I, int H, int k, float scale,
+                                      int32_t* idx_out, uint16_t* out, float* lse, void* ws, size_t ws_bytes,
+                                      void* stream) {
+  if (row0 < 0 || nrows <= 0 || H <= 0 || k <= 0 || !q_idx || !k_idx || !w || !q || !c || !out)
+    return DSA_ERR_INVALID_ARG;
+  if (static_cast<long long>(row0) + nrows > INT32_MAX) return DSA_ERR_INVALID_ARG;
+  if (!indexer_shape_ok(H_I, d_I) || H > 128 || !mla_k_ok(k)) return DSA_ERR_UNSUPPORTED_SHAPE;
+  if (!aligned16(q_idx) || !aligned16(k_idx) || !aligned16(q) || !aligned16(c) || !aligned16(out) ||
+      (idx_out && !aligned16(idx_out)))
+    return DSA_ERR_ALIGNMENT;
+  if (!ws || ws_bytes < dsa_prefill_rows_workspace_size(row0, nrows, H_I, d_I, H, k)) return DSA_ERR_WORKSPACE;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  float* sc = static_cast<float*>(ws);
-  for (int r0 = 0, rows = 0; r0 < L; r0 += rows) {
-    rows = prefill_block_rows(L, k, r0);
-    const int s_eff = r0 + rows;   // keys beyond the block's last row are never selected (causal)
-    // a block whose every row t has t + 1 <= k selects all of 0..t whatever the scores: no indexer launch (the
-    // top-k kernel writes 0..t and the -1 padding of such rows without reading them)
-    dsa_status_t e = DSA_OK;
-    if (s_eff > k) {
-      e = run_indexer_scores(q_idx + static_cast<size_t>(r0) * H_I * d_I, q_scale ? q_scale + r0 : nullptr, k_idx,
-                             k_scale, w + static_cast<size_t>(r0) * H_I, rows, s_eff, H_I, d_I, r0, sc, s_eff, st);
-      if (e != DSA_OK) return e;
-    }
-    e = run_topk(sc, s_eff, nullptr, nullptr, r0, rows, k, idx_out + static_cast<size_t>(r0) * k, k, st);
-    if (e != DSA_OK) return e;
-  }
-  return DSA_OK;
+  const int S = row0 + nrows;
+  const size_t score_bytes = align_up(prefill_chunk_rows(S) * size_t(S) * 4, 256);
+  int32_t* idx = idx_out ? idx_out : reinterpret_cast<int32_t*>(static_cast<char*>(ws) + score_bytes);
+  dsa_status_t e = select_rows(q_idx, q_scale, k_idx, k_scale, w, H_I, d_I, k, row0, S, idx, static_cast<float*>(ws),
+                               prefill_chunk_rows(S), st);
+  if (e != DSA_OK) return e;
+  return run_mla(q, c, S, idx, nullptr, nrows, H, k, scale, out, lse, st, kMlaCausal, nullptr, nullptr, 0, 0, row0);
 }
 
 dsa_status_t dsa_forward_prefill(const uint8_t* q_idx, const float* q_scale, const uint8_t* k_idx,
@@ -433,7 +626,7 @@ dsa_status_t dsa_forward_prefill(const uint8_t* q_idx, const float* q_scale, con
                                                       align_up(prefill_chunk_rows(L) * size_t(L) * 4, 256));
   dsa_status_t e = dsa_prefill_select(q_idx, q_scale, k_idx, k_scale, w, L, H_I, d_I, k, idx, ws, ws_bytes, stream);
   if (e != DSA_OK) return e;
-  return run_mla(q, c, L, idx, nullptr, L, H, k, scale, out, lse, st);
+  return run_mla(q, c, L, idx, nullptr, L, H, k, scale, out, lse, st, kMlaCausal);
 }
 
 size_t dsa_prefill_varlen_workspace_size(int nseq, int64_t total, int max_len, int H_I, int d_I, int H, int k) {
@@ -490,7 +683,8 @@ dsa_status_t dsa_forward_prefill_varlen(int nseq, const int64_t* cu_seqlens, con
                            score_bytes, stream);
     if (e != DSA_OK) return e;
   }
-  return run_mla(q, c, static_cast<int>(total), idx, row_off, static_cast<int>(total), H, k, scale, out, lse, st);
+  return run_mla(q, c, static_cast<int>(total), idx, row_off, static_cast<int>(total), H, k, scale, out, lse, st,
+                 kMlaCausal);
 }
 
 uint64_t dsa_launch_count(void) { return g_launches.load(); }
@@ -519,8 +713,7 @@ __attribute__((visibility("default"))) int dsa_trace_read(unsigned long long* ho
 size_t dsa_decode_workspace_size(int B, int64_t cache_rows, int H_I, int d_I, int H, int k) {
   (void)H_I; (void)d_I; (void)H;
   if (B <= 0 || cache_rows <= 0 || k <= 0) return 0;
-  return align_up(decode_score_cap(B, cache_rows) * 4, 256) + align_up(size_t(B) * 4, 256) +
-         align_up(size_t(B) * 8, 256) + align_up(size_t(B) * k * 4, 256);
+  return decode_ws_bytes(B, decode_score_cap(B, cache_rows), k);
 }
 
 dsa_status_t dsa_forward_decode(int B, const int64_t* cache_off, const int32_t* ctx_len, const uint8_t* q_idx,
@@ -533,39 +726,47 @@ dsa_status_t dsa_forward_decode(int B, const int64_t* cache_off, const int32_t* 
                                               k_scale_cache, c_cache, cache_rows, H_I, d_I, H, k, idx_out, out);
   if (chk != DSA_OK) return chk;
   if (!ws || ws_bytes < dsa_decode_workspace_size(B, cache_rows, H_I, d_I, H, k)) return DSA_ERR_WORKSPACE;
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
-  char* wsb = static_cast<char*>(ws);
-  // workspace: score rows (packed, 16-byte aligned), len1 [B], score_off [B], selected indices [B, k]
-  const size_t score_cap = decode_score_cap(B, cache_rows);
-  float* dscores = reinterpret_cast<float*>(wsb);
-  size_t at = align_up(score_cap * 4, 256);
-  int* len1 = reinterpret_cast<int*>(wsb + at);
-  at += align_up(size_t(B) * 4, 256);
-  long long* soff = reinterpret_cast<long long*>(wsb + at);
-  at += align_up(size_t(B) * 8, 256);
-  int32_t* idx = idx_out ? idx_out : reinterpret_cast<int32_t*>(wsb + at);
-  const long long* off = reinterpret_cast<const long long*>(cache_off);
-  decode_append_kernel<<<B, kAppendThreads, 0, st>>>(B, off, ctx_len, cache_rows, k_new, k_scale_new, c_new,
-                                                     k_cache, k_scale_cache, c_cache, d_I, len1, soff,
-                                                     static_cast<long long>(score_cap));
-  dsa_status_t e = last_launch_status();
-  if (e != DSA_OK) return e;
-  IndexerParams p{};
-  p.w = w;
-  p.q_scale = q_scale;
-  p.k_scale = k_scale_cache;
-  p.scores = dscores;
-  p.T = B;
-  p.cache_off = off;
-  p.len1 = len1;
-  p.score_off = soff;
-  p.chunk_tiles = 16;
-  e = launch_indexer<64, 128, 1, 1, 2, 4, 1, kModeDecode>(
-      q_idx, B, k_cache, cache_rows, p, IndexerCfg<64, 128, 1, 1, 2, 4, 1, kModeDecode>::CTAS_PER_SM * num_sms(), st);
-  if (e != DSA_OK) return e;
-  e = run_topk(dscores, 0, soff, len1, 0, B, k, idx, k, st);
-  if (e != DSA_OK) return e;
-  return run_mla(q, c_cache, cache_rows, idx, off, B, H, k, scale, out, lse, st);
+  DecodeLayout lay{};
+  lay.cache_off = reinterpret_cast<const long long*>(cache_off);
+  lay.cache_rows = cache_rows;
+  return run_decode(B, lay, ctx_len, q_idx, q_scale, w, q, k_new, k_scale_new, c_new, k_cache, k_scale_cache,
+                    c_cache, decode_score_cap(B, cache_rows), H, k, scale, idx_out, out, lse, ws,
+                    static_cast<cudaStream_t>(stream));
+}
+
+size_t dsa_decode_paged_workspace_size(int B, int max_pages, int page_rows, int H_I, int d_I, int H, int k) {
+  (void)H_I; (void)d_I; (void)H;
+  if (B <= 0 || max_pages <= 0 || page_rows <= 0 || k <= 0) return 0;
+  return decode_ws_bytes(B, decode_score_cap(B, static_cast<int64_t>(B) * max_pages * page_rows), k);
+}
+
+dsa_status_t dsa_forward_decode_paged(int B, const int32_t* page_table, int max_pages, int page_rows,
+                                      const int32_t* ctx_len, const uint8_t* q_idx, const float* q_scale,
+                                      const float* w, const uint16_t* q, const uint8_t* k_new,
+                                      const float* k_scale_new, const uint16_t* c_new, uint8_t* k_cache,
+                                      float* k_scale_cache, uint16_t* c_cache, int num_pages, int H_I, int d_I,
+                                      int H, int k, float scale, int32_t* idx_out, uint16_t* out, float* lse,
+                                      void* ws, size_t ws_bytes, void* stream) {
+  if (!page_table || max_pages <= 0 || num_pages <= 0) return DSA_ERR_INVALID_ARG;
+  if (page_rows <= 0 || page_rows % 128 != 0) return DSA_ERR_UNSUPPORTED_SHAPE;
+  const int64_t pool_rows = static_cast<int64_t>(num_pages) * page_rows;
+  if (pool_rows > INT32_MAX) return DSA_ERR_UNSUPPORTED_SHAPE;   // tensor-map row coordinates are 32-bit
+  // every check of the flat call applies, with the page pools as the caches (any non-null cache_off passes)
+  const dsa_status_t chk = decode_args_status(B, reinterpret_cast<const int64_t*>(page_table), ctx_len, q_idx, w, q,
+                                              k_new, k_scale_new, c_new, k_cache, k_scale_cache, c_cache, pool_rows,
+                                              H_I, d_I, H, k, idx_out, out);
+  if (chk != DSA_OK) return chk;
+  if (!ws || ws_bytes < dsa_decode_paged_workspace_size(B, max_pages, page_rows, H_I, d_I, H, k))
+    return DSA_ERR_WORKSPACE;
+  DecodeLayout lay{};
+  lay.cache_rows = pool_rows;
+  lay.page_table = page_table;
+  lay.max_pages = max_pages;
+  lay.page_rows = page_rows;
+  lay.num_pages = num_pages;
+  return run_decode(B, lay, ctx_len, q_idx, q_scale, w, q, k_new, k_scale_new, c_new, k_cache, k_scale_cache,
+                    c_cache, decode_score_cap(B, static_cast<int64_t>(B) * max_pages * page_rows), H, k, scale,
+                    idx_out, out, lse, ws, static_cast<cudaStream_t>(stream));
 }
 
 // ------------------------------------------------------------------------------------------ no-allocation decode

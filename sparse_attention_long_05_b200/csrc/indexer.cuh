@@ -22,7 +22,9 @@
 //                materialised prefill chunks);
 //   kModeDecode  item = (sequence b, range of its key tiles); one token per sequence; keys are the rows
 //                [cache_off[b], cache_off[b] + len1[b]) of the flat key cache; writes the sequence's len1[b]
-//                fp32 scores from score_off[b] on (one packed row per sequence).
+//                fp32 scores from score_off[b] on (one packed row per sequence).  The key tiles of all sequences,
+//                laid end to end, are cut into gridDim.x equal ranges, one per CTA; a CTA's items are the pieces
+//                of the sequences its range covers, so every CTA streams the same number of key tiles.
 #pragma once
 #include "common.cuh"
 
@@ -45,7 +47,8 @@ struct IndexerParams {
   const long long* cache_off;  // kModeDecode: [B] first cache row of each sequence
   const int* len1;             // kModeDecode: [B] keys of each sequence after the append (0: skip it)
   const long long* score_off;  // kModeDecode: [B] start of each sequence's score row
-  int chunk_tiles;             // kModeDecode: key tiles per work item
+  const int* page_table;       // kModeDecode, paged caches: [B, max_pages] page of each 'page_rows' positions
+  int max_pages, page_rows;    // (page_rows a multiple of 128, so that a key tile lies in one page)
 };
 
 struct IndexerItem {
@@ -54,9 +57,18 @@ struct IndexerItem {
   int pos0;           // absolute position of the item's first query row
   int tile0, tile1;   // key tile range [tile0, tile1)
   int n_keys;         // keys s < n_keys exist
-  long long key_row0; // tensor-map row of key 0
+  long long key_row0; // tensor-map row of key 0 (flat layouts)
+  const int* pages;   // paged decode caches: the sequence's page-table row, else null
+  int page_rows;
   long long out_base; // output offset of (first row, key 0)
 };
+
+// tensor-map row of key tile*128 + i of an item (i < 128)
+__device__ __forceinline__ long long key_row(const IndexerItem& it, int tile, int i) {
+  if (!it.pages) return it.key_row0 + static_cast<long long>(tile) * 128 + i;
+  const int pos = tile * 128;
+  return static_cast<long long>(it.pages[pos / it.page_rows]) * it.page_rows + pos % it.page_rows + i;
+}
 
 constexpr int kMaxDecodeSeqs = 1024;
 
@@ -106,11 +118,17 @@ struct IndexerBars {
   static constexpr int COUNT = ACC_EMPTY + NACC;
   static constexpr int OFF_TMEM = 8 * COUNT;         // u32: TMEM base address
   static constexpr int OFF_ABORT = OFF_TMEM + 4;     // int: abort flag
-  static constexpr int OFF_NITEMS = OFF_TMEM + 8;    // int: number of items (decode)
+  static constexpr int OFF_NITEMS = OFF_TMEM + 8;    // int: key tiles of all sequences (decode)
+};
+
+// decode: the key-tile range [lo, hi) of this CTA over the tiles of all sequences laid end to end
+struct TileRange {
+  int lo, hi;
 };
 
 template <int MODE, int TOK>
-__device__ __forceinline__ IndexerItem indexer_item(const IndexerParams& p, int i, const int* prefix) {
+__device__ __forceinline__ IndexerItem indexer_item(const IndexerParams& p, int i, const int* prefix,
+                                                    TileRange tr) {
   IndexerItem it;
   if constexpr (MODE == kModeScores) {
     const int qb = i / p.nsplit, sp = i % p.nsplit;
@@ -119,18 +137,15 @@ __device__ __forceinline__ IndexerItem indexer_item(const IndexerParams& p, int 
     it.pos0 = p.pos0 + it.q_row0;
     it.n_keys = p.S;
     it.key_row0 = 0;
+    it.pages = nullptr;
+    it.page_rows = 0;
     const int ntiles = (p.S + 127) / 128;
     it.tile0 = sp * p.split_tiles;
     it.tile1 = min(it.tile0 + p.split_tiles, ntiles);
     it.out_base = static_cast<long long>(it.q_row0) * p.ld;
   } else {
-    // binary search: prefix[b] <= i < prefix[b + 1]
-    int lo = 0, hi = p.T - 1;
-    while (lo < hi) {
-      const int mid = (lo + hi + 1) >> 1;
-      if (prefix[mid] <= i) lo = mid; else hi = mid - 1;
-    }
-    const int b = lo;
+    // item i is sequence b = i, clipped to the CTA's tile range (prefix[b] = its first tile in the joint order)
+    const int b = i;
     const int* n1s = prefix + kMaxDecodeSeqs + 1;
     const long long* offs = reinterpret_cast<const long long*>(n1s + kMaxDecodeSeqs + 1);   // 8-byte aligned
     const int n = n1s[b];
@@ -139,8 +154,10 @@ __device__ __forceinline__ IndexerItem indexer_item(const IndexerParams& p, int 
     it.pos0 = n - 1;
     it.n_keys = n;
     it.key_row0 = offs[b];
-    it.tile0 = (i - prefix[b]) * p.chunk_tiles;
-    it.tile1 = min(it.tile0 + p.chunk_tiles, (n + 127) / 128);
+    it.pages = p.page_table ? p.page_table + static_cast<long long>(b) * p.max_pages : nullptr;
+    it.page_rows = p.page_rows;
+    it.tile0 = max(tr.lo, prefix[b]) - prefix[b];
+    it.tile1 = min(tr.hi, prefix[b + 1]) - prefix[b];
     it.out_base = p.score_off[b];
   }
   return it;
@@ -190,17 +207,17 @@ indexer_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     fence_mbar_init();
   }
   if constexpr (MODE == kModeDecode) {
-    // per sequence: keys n_b + 1, cache offset and work items, loaded by all threads in parallel; then an
-    // exclusive scan of the item counts by warp 0 (items of sequence b are prefix[b] .. prefix[b + 1] - 1)
+    // per sequence: keys n_b + 1, cache offset and key tiles, loaded by all threads in parallel; then an
+    // exclusive scan of the tile counts by warp 0 (tiles of sequence b are prefix[b] .. prefix[b + 1] - 1 in the
+    // joint order)
     int* n1s = prefix + kMaxDecodeSeqs + 1;
     long long* offs = reinterpret_cast<long long*>(n1s + kMaxDecodeSeqs + 1);
     int* cnts = prefix + 1;          // counts first, scanned in place below
     for (int b = threadIdx.x; b < p.T; b += blockDim.x) {
       const int n1 = p.len1[b];
       n1s[b] = n1;
-      offs[b] = p.cache_off[b];
-      const int tiles = (n1 + 127) / 128;
-      cnts[b] = (tiles + p.chunk_tiles - 1) / p.chunk_tiles;
+      offs[b] = p.cache_off ? p.cache_off[b] : 0;     // paged caches: rows come from the page table
+      cnts[b] = (n1 + 127) / 128;
     }
     __syncthreads();
     if (warp == 0) {
@@ -234,8 +251,41 @@ indexer_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *reinterpret_cast<volatile uint32_t*>(smem + Bars::OFF_TMEM);
-  const int n_items = (MODE == kModeDecode) ? *reinterpret_cast<volatile int*>(smem + Bars::OFF_NITEMS)
-                                            : p.n_items;
+  // The CTA's items.  kModeScores: items blockIdx.x, + gridDim.x, ... below p.n_items.  kModeDecode: the
+  // sequences whose tiles meet the CTA's range [lo, hi), skipping those without keys (every role walks the same
+  // list, which must hold no empty item: each item loads its queries once).
+  TileRange tr{0, 0};
+  if constexpr (MODE == kModeDecode) {
+    const long long tot = *reinterpret_cast<volatile int*>(smem + Bars::OFF_NITEMS);
+    tr.lo = static_cast<int>(tot * blockIdx.x / gridDim.x);
+    tr.hi = static_cast<int>(tot * (blockIdx.x + 1) / gridDim.x);
+  }
+  auto first_item = [&]() -> int {
+    if constexpr (MODE == kModeDecode) {
+      // the last sequence starting at or before lo: it holds tile lo (when lo < hi)
+      int lo = 0, hi = p.T - 1;
+      while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (prefix[mid] <= tr.lo) lo = mid; else hi = mid - 1;
+      }
+      return lo;
+    } else {
+      return static_cast<int>(blockIdx.x);
+    }
+  };
+  auto has_item = [&](int i) -> bool {
+    if constexpr (MODE == kModeDecode) return i < p.T && prefix[i] < tr.hi;
+    else return i < p.n_items;
+  };
+  auto next_item = [&](int i) -> int {
+    if constexpr (MODE == kModeDecode) {
+      ++i;
+      while (i < p.T && prefix[i + 1] == prefix[i]) ++i;     // sequences without keys
+      return i;
+    } else {
+      return i + static_cast<int>(gridDim.x);
+    }
+  };
 
   if (warp == 0) {
     // ------------------------------------------------------------------ TMA producer
@@ -246,8 +296,8 @@ indexer_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
       uint32_t q_par[QBUF] = {};        // per q buffer: parity of its last load
       int qi = 0;
       bool ok = true;
-      for (int item = blockIdx.x; item < n_items && ok; item += gridDim.x, ++qi) {
-        const IndexerItem it = indexer_item<MODE, C::TOK>(p, item, prefix);
+      for (int item = first_item(); has_item(item) && ok; item = next_item(item), ++qi) {
+        const IndexerItem it = indexer_item<MODE, C::TOK>(p, item, prefix, tr);
         const int qb = qi % QBUF;
         const uint32_t qph = (qi / QBUF) & 1;
         if (!mbar_wait(bar(Bars::Q_EMPTY + qb), qph ^ 1, abort_flag)) { ok = false; break; }
@@ -262,7 +312,7 @@ indexer_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
           if (!mbar_wait(bar(Bars::K_EMPTY + kp.stage), kp.phase ^ 1, abort_flag)) { ok = false; break; }
           mbar_arrive_expect_tx(bar(Bars::K_FULL + kp.stage), C::KBYTES);
           tma_load_2d(k_s + kp.stage * C::KBYTES, &tm_k, bar(Bars::K_FULL + kp.stage), 0,
-                      static_cast<int>(it.key_row0 + tile * 128));
+                      static_cast<int>(key_row(it, tile, 0)));
           kp.advance();
           ++k_issued;
         }
@@ -284,8 +334,8 @@ indexer_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
       constexpr uint32_t idesc = idesc_e4m3(128, C::N);
       int qi = 0;
       bool ok = true;
-      for (int item = blockIdx.x; item < n_items && ok; item += gridDim.x, ++qi) {
-        const IndexerItem it = indexer_item<MODE, C::TOK>(p, item, prefix);
+      for (int item = first_item(); has_item(item) && ok; item = next_item(item), ++qi) {
+        const IndexerItem it = indexer_item<MODE, C::TOK>(p, item, prefix, tr);
         const int qb = qi % QBUF;
         if (!mbar_wait(bar(Bars::Q_FULL + qb), (qi / QBUF) & 1, abort_flag)) { ok = false; break; }
         tc_fence_after();
@@ -330,8 +380,8 @@ indexer_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     Pipe<C::NACC> ap;
     int qi = 0;
     bool ok = true;
-    for (int item = blockIdx.x; item < n_items && ok; item += gridDim.x, ++qi) {
-      const IndexerItem it = indexer_item<MODE, C::TOK>(p, item, prefix);
+    for (int item = first_item(); has_item(item) && ok; item = next_item(item), ++qi) {
+      const IndexerItem it = indexer_item<MODE, C::TOK>(p, item, prefix, tr);
       float* wq = w_s + (qi % QBUF) * C::W_FLOATS;
       named_bar_sync(1, ethreads);
       for (int i = etid; i < C::W_FLOATS; i += ethreads) {
@@ -349,7 +399,7 @@ indexer_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
       // global-memory latency once per tile (the epilogue needs it a few hundred cycles later)
       auto kscale_of = [&](int tile) -> float {
         const int s = tile * 128 + quad * 32 + lane;
-        return (p.k_scale && tile < it.tile1 && s < it.n_keys) ? p.k_scale[it.key_row0 + s] : 1.f;
+        return (p.k_scale && tile < it.tile1 && s < it.n_keys) ? p.k_scale[key_row(it, tile, quad * 32 + lane)] : 1.f;
       };
       float kscale_next = kscale_of(it.tile0);
       for (int tile = it.tile0; tile < it.tile1; ++tile) {

@@ -46,12 +46,32 @@
 
 namespace dsa {
 
+// How a token's keys are found.  kMlaSparse: the k entries of its index row are gathered.  The dense modes
+// give each token the number n_t of keys its sequence shows it (positions 0..n_t-1, rows base..base+n_t-1 of
+// c); a token with n_t <= k then selects all of them, whatever its index row says, and its keys are read as
+// contiguous 64-row tiles, ceil(n_t / 64) of them, instead of k / 64 gathered tiles.  kMlaCausal: n_t = pos0 + t
+// - base + 1 (prefill rows at their positions, the launch's first row at position pos0); kMlaCounts: n_t =
+// n_keys[t] (decode tokens after the append).
+enum { kMlaSparse = 0, kMlaCausal = 1, kMlaCounts = 2 };
+
 struct MlaParams {
   const int* idx;              // [T, k]
   const long long* row_off;    // [T] row of entry 0 of each token in c, or null (0)
+  const int* n_keys;           // [T] keys of each token (kMlaCounts), else null
   uint16_t* out;               // [T, H, 512] bf16
   float* lse;                  // [T, H] or null
   int T, H, k;
+  int dense;                   // kMlaSparse / kMlaCausal / kMlaCounts
+  int pos0;                    // kMlaCausal: position of the launch's token 0 in its sequence
+  // KL mode (kl_out non-null): no attention output; every CTA runs the score role on its own tokens and writes
+  // kl_out[t] = KL(p_t || Softmax(I_t)) over the token's keys, p_t the heads' attention probabilities (from the
+  // logits and the attention's lse [T, H]) summed and L1-normalised, I_t = kl_scores [T, k] (the index score of
+  // each selected entry)
+  const float* kl_lse;
+  const float* kl_scores;
+  float* kl_out;
+  const int* page_table;       // paged c: [T, pt_stride] page of each page_rows positions of token t's keys, or null
+  int pt_stride, page_rows;    // (page_rows a multiple of 64: a 64-key tile lies in one page)
   long long S;                 // rows of c
   float scale_log2;            // softmax scale * log2(e)
 };
@@ -92,7 +112,9 @@ constexpr int B_O_DONE = B_P_READY + NPB, B_O_FREE = B_O_DONE + NPB;
 constexpr int B_SLOT_FREE = B_O_FREE + 1, B_SLOT_WRITTEN = B_SLOT_FREE + 1;   // score CTA softmax handshakes
 constexpr int B_QRET = B_SLOT_WRITTEN + 1;    // score CTA: last-tile MMAs of chunks 0..2 retired
 constexpr int B_QTOK = B_QRET + 1;            // score CTA: every MMA of a token retired
-constexpr int B_COUNT = B_QTOK + 1;
+constexpr int B_RED_FULL = B_QTOK + 1;        // KL mode: the four warps' head sums of a tile written (2 buffers)
+constexpr int B_RED_FREE = B_RED_FULL + 2;    // KL mode: the head sums of a tile read (2 buffers)
+constexpr int B_COUNT = B_RED_FREE + 2;
 // shared memory map (from a 1024-byte aligned base; both CTAs use the same barrier offsets)
 constexpr int OFF_TMEM = 8 * B_COUNT;
 constexpr int OFF_ABORT = OFF_TMEM + 4;
@@ -114,18 +136,40 @@ static_assert(NS_S <= 16 && NS_V <= 16, "ring barrier slots");
 static_assert(SMEM <= 232448, "shared memory per CTA");
 }  // namespace mla
 
-// row of c gathered for selection entry e (in slot `slot` of its token's k entries) of a token whose entries
-// start at row `base`.  An empty or invalid entry is masked out of the softmax but its stage still holds a row:
-// it reads row `slot` (any row in [0, S) would do), so that the padding of short rows spreads over many L2 lines
-// instead of hammering one
-__device__ __forceinline__ long long mla_row(int e, long long base, long long S, int slot) {
-  const long long r = base + e;
-  const bool valid = (e >= 0) && (r >= 0) && (r < S);
-  if (!valid && e != -1) raise_status(DSA_ERR_BAD_INDEX);
-  return valid ? r : (slot < S ? slot : 0);
+// Row of c holding position `pos` (>= 0) of token t's keys: base + pos, or through the token's page-table row.
+__device__ __forceinline__ long long mla_pos_row(const MlaParams& p, int t, long long base, long long pos) {
+  if (!p.page_table) return base + pos;
+  const int* pr = p.page_table + static_cast<long long>(t) * p.pt_stride;
+  return static_cast<long long>(pr[pos / p.page_rows]) * p.page_rows + pos % p.page_rows;
 }
-__device__ __forceinline__ bool mla_valid(int e, long long base, long long S) {
-  return e >= 0 && base + e >= 0 && base + e < S;
+// Whether selection entry e of token t names a row of c (an entry of -1 is padding; anything else outside the
+// token's keys is an error).
+__device__ __forceinline__ bool mla_valid(const MlaParams& p, int t, int e, long long base) {
+  if (e < 0) return false;
+  if (p.page_table && e >= static_cast<long long>(p.pt_stride) * p.page_rows) return false;
+  const long long r = mla_pos_row(p, t, base, e);
+  return r >= 0 && r < p.S;
+}
+// Row of c gathered for selection entry e (in slot `slot` of its token's k entries).  An empty or invalid entry is
+// masked out of the softmax but its stage still holds a row: it reads row `slot` (any row in [0, S) would do), so
+// that the padding of short rows spreads over many L2 lines instead of hammering one.
+__device__ __forceinline__ long long mla_row(const MlaParams& p, int t, int e, long long base, int slot) {
+  const bool valid = mla_valid(p, t, e, base);
+  if (!valid && e != -1) raise_status(DSA_ERR_BAD_INDEX);
+  return valid ? mla_pos_row(p, t, base, e) : (slot < p.S ? slot : 0);
+}
+
+// Number of keys n_t of token t when it takes the dense path (n_t <= k), -1 when its index row is gathered.
+__device__ __forceinline__ int mla_dense_keys(const MlaParams& p, int t, long long base) {
+  if (p.dense == kMlaSparse) return -1;
+  const long long n = (p.dense == kMlaCausal) ? static_cast<long long>(p.pos0) + t - base + 1 : p.n_keys[t];
+  if (n > p.k) return -1;
+  return n > 0 ? static_cast<int>(n) : 0;
+}
+// 64-key tiles of a token: k / 64 gathered tiles, or the tiles holding its n_t dense keys (at least two: the
+// score CTA's schedule of Q-chunk copies needs a second tile; a tile past n_t is wholly masked)
+__device__ __forceinline__ int mla_tiles(const MlaParams& p, int nd) {
+  return nd < 0 ? p.k / mla::NK : max(2, (nd + mla::NK - 1) / mla::NK);
 }
 
 // position in a ring of `size` stages (size known at run time): stage index and pass parity, advanced
@@ -148,7 +192,7 @@ __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, volatil
 
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(mla::THREADS, 1)
 sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_c,
-                  const MlaParams p) {
+                  const __grid_constant__ CUtensorMap tm_cd, const MlaParams p) {
   using namespace mla;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -157,9 +201,11 @@ sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
   auto bar = [&](int slot) -> uint32_t { return sbase + 8 * slot; };
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + OFF_ABORT);
   const int warp = warp_id(), lane = lane_id();
-  const uint32_t rank = cluster_rank();            // 0 = score CTA, 1 = value CTA
-  const int cluster = blockIdx.x >> 1, nclusters = gridDim.x >> 1;
-  const int ntiles = p.k / NK;
+  // 0 = score CTA, 1 = value CTA; in KL mode every CTA takes the score role on tokens of its own
+  const bool kl_mode = p.kl_out != nullptr;
+  const uint32_t rank = kl_mode ? 0u : cluster_rank();
+  const int cluster = kl_mode ? static_cast<int>(blockIdx.x) : static_cast<int>(blockIdx.x >> 1);
+  const int nclusters = kl_mode ? static_cast<int>(gridDim.x) : static_cast<int>(gridDim.x >> 1);
   const int nsr = (rank == 0) ? NS_S : NS_V;
   const uint32_t ring = sbase + ((rank == 0) ? OFF_RING_S : OFF_RING_V);
   const int* idx_s = reinterpret_cast<const int*>(smem + OFF_IDX);
@@ -181,6 +227,7 @@ sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
       mbar_init(bar(B_SLOT_WRITTEN), 4);
       mbar_init(bar(B_QRET), 1);
       mbar_init(bar(B_QTOK), 1);
+      for (int i = 0; i < 2; ++i) { mbar_init(bar(B_RED_FULL + i), 4); mbar_init(bar(B_RED_FREE + i), 1); }
     } else {
       for (int i = 0; i < NPB; ++i) { mbar_init(bar(B_P_FULL + i), 1); mbar_init(bar(B_P_READY + i), 4); }
       for (int i = 0; i < NPB; ++i) mbar_init(bar(B_O_DONE + i), 1);
@@ -191,6 +238,7 @@ sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
   }
   if (warp == 0 && lane == 0) {
     prefetch_tmap(&tm_c);
+    if (p.dense != kMlaSparse) prefetch_tmap(&tm_cd);
     if (rank == 0) prefetch_tmap(&tm_q);
   }
   if (warp == 1) {
@@ -238,7 +286,11 @@ sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     // ===================================================================== gathers (TMA gather4)
     // Every stage is split over the eight gather warps: gather4 instruction i of a stage (i = 16 cc + rg)
     // fetches rows 4 rg .. 4 rg + 3 of the tile into its chunk cc; warp gw issues instructions
-    // gw * per_warp .. + per_warp - 1, one per lane.
+    // gw * per_warp .. + per_warp - 1, one per lane.  A dense token's full tiles are 64 contiguous rows: lane c
+    // of gather warp 0 loads its chunk c as one 64 x 64 box, and the other warps arrive with no bytes.  Its
+    // last, partial tile is gathered, its masked slots reading rows of the token's own keys: the rows after
+    // the sequence's last key may be memory the caller never wrote, and a NaN there would survive the zero
+    // probability in P . V.
     const int gw = (warp < 8) ? warp - 2 : warp - 6;
     const int cps = (rank == 0) ? SCH : VCH;               // chunks per stage
     const int spt = (rank == 0) ? SPT_S : SPT_V;           // stages per tile
@@ -258,28 +310,49 @@ sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
       if (!(ok = warp_wait(bar(B_IDX_FULL + is), (ti >> 1) & 1, abort_flag))) break;
       const int* ids = idx_s + is * KMAX;
       const long long base = p.row_off ? p.row_off[t] : 0;
+      const int nd = mla_dense_keys(p, t, base);
+      const int ntiles = mla_tiles(p, nd);
       for (int j = 0; j < ntiles && ok; ++j) {
+        const bool full_dense = nd >= 0 && (j + 1) * NK <= nd;    // 64 contiguous rows of keys
+        const uint32_t tx = full_dense ? (gw == 0 ? sbytes : 0) : per_warp * 512;
         int r[4] = {0, 0, 0, 0};
-        if (active) {
-          const int4 e = reinterpret_cast<const int4*>(ids + j * NK)[rg];
+        if (active && !full_dense) {
           const int slot = j * NK + 4 * rg;
-          r[0] = static_cast<int>(mla_row(e.x, base, p.S, slot));
-          r[1] = static_cast<int>(mla_row(e.y, base, p.S, slot + 1));
-          r[2] = static_cast<int>(mla_row(e.z, base, p.S, slot + 2));
-          r[3] = static_cast<int>(mla_row(e.w, base, p.S, slot + 3));
+          if (nd < 0) {
+            const int4 e = reinterpret_cast<const int4*>(ids + j * NK)[rg];
+            r[0] = static_cast<int>(mla_row(p, t, e.x, base, slot));
+            r[1] = static_cast<int>(mla_row(p, t, e.y, base, slot + 1));
+            r[2] = static_cast<int>(mla_row(p, t, e.z, base, slot + 2));
+            r[3] = static_cast<int>(mla_row(p, t, e.w, base, slot + 3));
+          } else {
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+              const int pos = slot + u;
+              r[u] = static_cast<int>(nd > 0 ? mla_pos_row(p, t, base, pos < nd ? pos : pos % nd)
+                                             : (pos < p.S ? pos : 0));
+            }
+          }
         }
         for (int s = 0; s < spt; ++s, rp.advance()) {
           const int st = rp.stage;
           bool got = true;
           if (lane == 0) {
             got = mbar_wait(bar(B_RING_EMPTY + st), rp.phase ^ 1, abort_flag);
-            if (got) mbar_arrive_expect_tx(bar(B_RING_FULL + st), per_warp * 512);
+            if (got) {
+              if (tx) mbar_arrive_expect_tx(bar(B_RING_FULL + st), tx);
+              else mbar_arrive(bar(B_RING_FULL + st));
+            }
           }
           if (!(ok = __shfl_sync(0xffffffffu, got, 0))) break;
           if (lane == 0 && gw == 0 && s == 0) DSA_TRACE_EVENT(rank == 0 ? 0 : 16, ti * ntiles + j);
-          if (active)
-            tma_gather4(ring + st * sbytes + cc * CHUNK_BYTES + rg * 512, &tm_c, bar(B_RING_FULL + st),
-                        64 * (s * cps + cc), r[0], r[1], r[2], r[3]);
+          if (!full_dense) {
+            if (active)
+              tma_gather4(ring + st * sbytes + cc * CHUNK_BYTES + rg * 512, &tm_c, bar(B_RING_FULL + st),
+                          64 * (s * cps + cc), r[0], r[1], r[2], r[3]);
+          } else if (gw == 0 && lane < cps) {
+            tma_load_2d(ring + st * sbytes + lane * CHUNK_BYTES, &tm_cd, bar(B_RING_FULL + st),
+                        64 * (s * cps + lane), static_cast<int>(mla_pos_row(p, t, base, j * NK)));
+          }
           issued = true;
           last = rp;
         }
@@ -327,6 +400,7 @@ sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         const bool has_next = t + nclusters < p.T;
         const uint32_t prev_tok = static_cast<uint32_t>((ti - 1) & 1);   // parity of the previous token's QTOK
         const int q_slot0 = (9 * ti) % QSLOTS;                          // tensor-memory slot of chunk 0
+        const int ntiles = mla_tiles(p, mla_dense_keys(p, t, p.row_off ? p.row_off[t] : 0));
         for (int j = 0; j < ntiles && ok; ++j, ++g) {
           const int sb = g % NSB;
           if (j == 1 && has_next) {
@@ -388,6 +462,7 @@ sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     } else {
       constexpr uint32_t idesc = idesc_bf16(128, 256, true);
       for (int t = cluster; t < p.T && ok; t += nclusters, ++ti) {
+        const int ntiles = mla_tiles(p, mla_dense_keys(p, t, p.row_off ? p.row_off[t] : 0));
         for (int j = 0; j < ntiles && ok; ++j, ++g) {
           const int pb = static_cast<int>(g % NPB);
           if (j == 0 && !(ok = warp_wait(bar(B_O_FREE), (ti & 1) ^ 1, abort_flag))) break;
@@ -420,6 +495,135 @@ sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         }
       }
     }
+  } else if (kl_mode) {
+    // ===================================================================== KL objective (warps 4..7)
+    // Per tile: each thread (one head) forms its head's probabilities of the tile's 64 keys from the logits and the
+    // head's lse; a halving exchange sums them over the warp's 32 heads (lane l ends with keys 2 l, 2 l + 1), and
+    // warp 4 adds the four warps' sums (handed over through double-buffered shared memory under mbarriers) and
+    // accumulates the token's sums of a log a, a I, a and the log-sum-exp of I over the valid keys.
+    const int quad = warp & 3;
+    const int h = quad * 32 + lane;
+    const uint32_t lane_addr = static_cast<uint32_t>(quad * 32) << 16;
+    float* red = reinterpret_cast<float*>(smem + OFF_PST);     // [2 buffers][4 warps][64 keys]
+    constexpr float kLog2e = 1.4426950408889634f, kLn2 = 0.69314718055994531f;
+    int g = 0;
+    int ti = 0;
+    bool ok = true;
+    for (int t = cluster; t < p.T && ok; t += nclusters, ++ti) {
+      const int is = ti & 1;
+      if (!(ok = warp_wait(bar(B_IDX_FULL + is), (ti >> 1) & 1, abort_flag))) break;
+      const int* ids = idx_s + is * KMAX;
+      const long long base = p.row_off ? p.row_off[t] : 0;
+      const int nd = mla_dense_keys(p, t, base);
+      const int ntiles = mla_tiles(p, nd);
+      const bool head_on = h < p.H;
+      const float lse2 = head_on ? p.kl_lse[static_cast<long long>(t) * p.H + h] * kLog2e : 0.f;
+      const float inv_h = 1.f / static_cast<float>(p.H);
+      float s_alog = 0.f, s_ai = 0.f, s_a = 0.f, m_i = -INFINITY, z_i = 0.f;   // warp 4, per lane
+      for (int j = 0; j < ntiles && ok; ++j, ++g) {
+        const int sb = static_cast<int>(g % NSB), b = static_cast<int>(g & 1);
+        const uint32_t use = static_cast<uint32_t>((g >> 1) & 1);
+        bool v_even, v_odd;
+        if (nd < 0) {
+          const int2 e = reinterpret_cast<const int2*>(ids + j * NK)[lane];
+          v_even = mla_valid(p, t, e.x, base);
+          v_odd = mla_valid(p, t, e.y, base);
+        } else {
+          v_even = j * NK + 2 * lane < nd;
+          v_odd = j * NK + 2 * lane + 1 < nd;
+        }
+        const uint32_t m_even = __ballot_sync(0xffffffffu, v_even);
+        const uint32_t m_odd = __ballot_sync(0xffffffffu, v_odd);
+        if (!(ok = warp_wait(bar(B_S_FULL + sb), static_cast<uint32_t>((g / NSB) & 1), abort_flag))) break;
+        tc_fence_after();
+        uint32_t v[64];
+        {
+          uint32_t (&v0)[32] = *reinterpret_cast<uint32_t(*)[32]>(&v[0]);
+          uint32_t (&v1)[32] = *reinterpret_cast<uint32_t(*)[32]>(&v[32]);
+          tmem_ld32(lane_addr + tmem + TS + NK * sb, v0);
+          tmem_ld32(lane_addr + tmem + TS + NK * sb + 32, v1);
+        }
+        tmem_wait_ld();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(B_S_EMPTY + sb));
+        float x[64];
+#pragma unroll
+        for (int i = 0; i < NK; ++i) {
+          const bool valid = ((i & 1) ? (m_odd >> (i >> 1)) : (m_even >> (i >> 1))) & 1u;
+          x[i] = (valid && head_on) ? ex2_approx(fmaf(__uint_as_float(v[i]), p.scale_log2, -lse2)) : 0.f;
+        }
+        // sum over the warp's heads: five halving steps, each lane keeping the half its lane bit selects
+#define DSA_KL_HALVE(O, N)                                                              \
+  {                                                                                     \
+    const bool up = (lane & (O)) != 0;                                                  \
+    _Pragma("unroll") for (int i = 0; i < (N); ++i) {                                   \
+      const float keep = up ? x[(N) + i] : x[i];                                        \
+      const float send = up ? x[i] : x[(N) + i];                                        \
+      x[i] = keep + __shfl_xor_sync(0xffffffffu, send, (O));                            \
+    }                                                                                   \
+  }
+        DSA_KL_HALVE(16, 32)
+        DSA_KL_HALVE(8, 16)
+        DSA_KL_HALVE(4, 8)
+        DSA_KL_HALVE(2, 4)
+        DSA_KL_HALVE(1, 2)
+#undef DSA_KL_HALVE
+        if (!(ok = warp_wait(bar(B_RED_FREE + b), use ^ 1u, abort_flag))) break;
+        float* rb = red + b * 4 * NK;
+        rb[quad * NK + 2 * lane] = x[0];
+        rb[quad * NK + 2 * lane + 1] = x[1];
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(B_RED_FULL + b));
+        if (warp == 4) {
+          if (!(ok = warp_wait(bar(B_RED_FULL + b), use, abort_flag))) break;
+#pragma unroll
+          for (int u = 0; u < 2; ++u) {
+            const int key = 2 * lane + u;
+            const bool valid = ((u ? m_odd : m_even) >> lane) & 1u;
+            const float a = (rb[key] + rb[NK + key] + rb[2 * NK + key] + rb[3 * NK + key]) * inv_h;
+            if (valid) {
+              const float iv = p.kl_scores[static_cast<long long>(t) * p.k + j * NK + key];
+              if (a > 0.f) s_alog += a * lg2_approx(a) * kLn2;
+              s_ai += a * iv;
+              s_a += a;
+              if (iv > m_i) {
+                z_i = (m_i == -INFINITY ? 0.f : z_i * ex2_approx((m_i - iv) * kLog2e)) + 1.f;
+                m_i = iv;
+              } else {
+                z_i += ex2_approx((iv - m_i) * kLog2e);
+              }
+            }
+          }
+          __syncwarp();
+          if (lane == 0) mbar_arrive(bar(B_RED_FREE + b));
+        }
+      }
+      if (ok && warp == 4) {
+        // the token's divergence: p = a / sum(a) (L1-normalised), log Softmax(I) = I - lse(I)
+        float mm = m_i;
+#pragma unroll
+        for (int d = 16; d > 0; d >>= 1) mm = fmaxf(mm, __shfl_xor_sync(0xffffffffu, mm, d));
+        float z = (m_i == -INFINITY) ? 0.f : z_i * ex2_approx((m_i - mm) * kLog2e);
+#pragma unroll
+        for (int d = 16; d > 0; d >>= 1) {
+          z += __shfl_xor_sync(0xffffffffu, z, d);
+          s_alog += __shfl_xor_sync(0xffffffffu, s_alog, d);
+          s_ai += __shfl_xor_sync(0xffffffffu, s_ai, d);
+          s_a += __shfl_xor_sync(0xffffffffu, s_a, d);
+        }
+        if (lane == 0) {
+          float kl = 0.f;
+          if (s_a > 0.f && z > 0.f) {
+            const float lse_i = mm + lg2_approx(z) * kLn2;
+            kl = (s_alog - s_a * lg2_approx(s_a) * kLn2 - s_ai) / s_a + lse_i;
+          }
+          p.kl_out[t] = kl;
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(B_IDX_EMPTY + is));
+    }
   } else if (rank == 0) {
     // ===================================================================== softmax (score CTA, warps 4..7)
     const int quad = warp & 3;
@@ -436,14 +640,25 @@ sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
       if (!(ok = warp_wait(bar(B_IDX_FULL + is), (ti >> 1) & 1, abort_flag))) break;
       const int* ids = idx_s + is * KMAX;
       const long long base = p.row_off ? p.row_off[t] : 0;
+      const int nd = mla_dense_keys(p, t, base);
+      const int ntiles = mla_tiles(p, nd);
       // l: sum of the bf16-rounded probabilities that enter P . V (normalises O exactly);
       // le: sum of the unrounded probabilities (for the log-sum-exp output)
       float m_ref = -INFINITY, l = 0.f, le = 0.f;
       for (int j = 0; j < ntiles && ok; ++j, ++g) {
         const int sb = static_cast<int>(g % NSB), pb = static_cast<int>(g % NPB), b = static_cast<int>(g & 1);
-        const int2 e = reinterpret_cast<const int2*>(ids + j * NK)[lane];
-        const uint32_t m_even = __ballot_sync(0xffffffffu, mla_valid(e.x, base, p.S));
-        const uint32_t m_odd = __ballot_sync(0xffffffffu, mla_valid(e.y, base, p.S));
+        // keys of the tile that enter the softmax: valid index entries, or dense positions below n_t
+        bool v_even, v_odd;
+        if (nd < 0) {
+          const int2 e = reinterpret_cast<const int2*>(ids + j * NK)[lane];
+          v_even = mla_valid(p, t, e.x, base);
+          v_odd = mla_valid(p, t, e.y, base);
+        } else {
+          v_even = j * NK + 2 * lane < nd;
+          v_odd = j * NK + 2 * lane + 1 < nd;
+        }
+        const uint32_t m_even = __ballot_sync(0xffffffffu, v_even);
+        const uint32_t m_odd = __ballot_sync(0xffffffffu, v_odd);
         if (!(ok = warp_wait(bar(B_S_FULL + sb), static_cast<uint32_t>((g / NSB) & 1), abort_flag))) break;
         if (leader) DSA_TRACE_EVENT(4, g);
         tc_fence_after();
@@ -555,6 +770,7 @@ sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     int ti = 0;
     bool ok = true;
     for (int t = cluster; t < p.T && ok; t += nclusters, ++ti) {
+      const int ntiles = mla_tiles(p, mla_dense_keys(p, t, p.row_off ? p.row_off[t] : 0));
       float l = 0.f;
       for (int j = 0; j < ntiles; ++j, ++g) {
         const int pb = static_cast<int>(g % NPB);

@@ -31,20 +31,24 @@ struct TopkParams {
   int k;
   int* idx;                     // [rows, k]
   long long idx_ld;
+  float* sel_scores;            // [rows, k] score of each selected column (-inf for padding), or null
 };
 
-// CTA sizes: 512 threads (two CTAs per SM: the 64 registers per thread and ~107 KB of shared memory allow two)
-// when there are many rows, 1024 threads (one CTA per SM) when there are fewer rows than SMs (decode).
+// Inverse of order_key on the keys it produces (+0.0 for a folded -0.0; NaN stays NaN)
+__device__ __forceinline__ float key_score(uint32_t key) {
+  return __uint_as_float((key & 0x80000000u) ? (key & 0x7FFFFFFFu) : ~key);
+}
+
+// CTA size: 512 threads (two CTAs per SM: the 64 registers per thread and ~107 KB of shared memory allow two).
+// Fewer rows than SMs (a decode step) take topk_cluster_kernel, one cluster of CTAs per row.
 constexpr int kTopkThreads = 512;
-constexpr int kTopkThreadsFew = 1024;
 constexpr int kTopkBins = 2048;            // top 11 key bits
 constexpr int kTopkSampleMin = 16384;      // rows at least this long take the sampled path
 
 // Candidate slots per CTA, split into one region per warp.  The sampled path's threshold bin spans about 19 %
-// in score, so on 128K-key rows it can collect 11K+ candidates; the one-CTA-per-SM variant (fewer rows than
-// SMs) spends its larger shared memory on twice the slots, which keeps such rows off the exact path.
+// in score, so on 128K-key rows it collects 4K+ candidates on average.
 template <int NT>
-constexpr int topk_candidates() { return NT >= 1024 ? 20480 : 10240; }
+constexpr int topk_candidates() { return 10240; }
 
 template <int NT>
 struct TopkSmem {
@@ -59,8 +63,7 @@ struct TopkSmem {
   int s_gt[W], s_eq[W];
   int s_out_base[W], s_eq_base[W];
 };
-static_assert(sizeof(TopkSmem<1024>) <= 227 * 1024 && 2 * sizeof(TopkSmem<512>) <= 228 * 1024 - 2048,
-              "top-k shared memory: one 1024-thread CTA or two 512-thread CTAs per SM");
+static_assert(2 * sizeof(TopkSmem<kTopkThreads>) <= 228 * 1024 - 2048, "top-k shared memory: two CTAs per SM");
 
 // Radix select on 32-bit keys among the entries that match (key & mask) == prefix: returns the exact k-th
 // largest key and sets `need` to the number of entries equal to it that are taken.  each(visit) calls
@@ -166,6 +169,7 @@ __device__ __forceinline__ void topk_collect_vec(const float* x, int n, uint32_t
   uint32_t tb = (kk & 0x80000000u) ? (kk & 0x7FFFFFFFu) : ~kk;
   if (!(kk & 0x80000000u) && tb > 0xFF800000u) tb = 0xFF800000u;   // no float key lies below that of -inf
   const float thr = __uint_as_float(tb);
+  const bool low = bmin == 0;    // bin 0 holds NaN (order key 0), which compares false: take every key
   int cnt = 0;
   for (int i00 = seg0; i00 < seg1; i00 += 512) {
     const int c0 = i00 + 16 * lane;
@@ -183,7 +187,7 @@ __device__ __forceinline__ void topk_collect_vec(const float* x, int n, uint32_t
     }
     int c = 0;
 #pragma unroll
-    for (int e = 0; e < 16; ++e) c += (c0 + e < seg1 && xv[e] >= thr) ? 1 : 0;
+    for (int e = 0; e < 16; ++e) c += (c0 + e < seg1 && (low || xv[e] >= thr)) ? 1 : 0;
     int incl = c;
 #pragma unroll
     for (int d = 1; d < 32; d <<= 1) {
@@ -195,7 +199,7 @@ __device__ __forceinline__ void topk_collect_vec(const float* x, int n, uint32_t
       int pos = cnt + incl - c;
 #pragma unroll
       for (int e = 0; e < 16; ++e) {
-        if (c0 + e < seg1 && xv[e] >= thr) {
+        if (c0 + e < seg1 && (low || xv[e] >= thr)) {
           if (pos < TopkSmem<NT>::REGION) {
             sm.cand_key[warp][pos] = order_key(xv[e]);
             sm.cand_idx[warp][pos] = c0 + e;
@@ -228,9 +232,13 @@ __global__ void __launch_bounds__(NT) topk_rows_kernel(const TopkParams p) {
   const int n = static_cast<int>(nl < 0 ? 0 : nl);
   const int k = p.k;
   int* out = p.idx + static_cast<long long>(r) * p.idx_ld;
+  float* sel_out = p.sel_scores ? p.sel_scores + static_cast<long long>(r) * p.idx_ld : nullptr;
 
   if (n <= k) {
-    for (int i = tid; i < k; i += NT) out[i] = (i < n) ? i : -1;
+    for (int i = tid; i < k; i += NT) {
+      out[i] = (i < n) ? i : -1;
+      if (sel_out) sel_out[i] = (i < n) ? x[i] : -INFINITY;
+    }
     return;
   }
   const int seg = (n + TopkSmem<NT>::W - 1) / TopkSmem<NT>::W;
@@ -401,7 +409,11 @@ __global__ void __launch_bounds__(NT) topk_rows_kernel(const TopkParams p) {
     const int my_eq_rank = eq_rank + __popc(eq_mask & ((1u << lane) - 1));
     const bool sel = j < span && (key > T || (is_eq && my_eq_rank < static_cast<int>(need)));
     const uint32_t sel_mask = __ballot_sync(0xffffffffu, sel);
-    if (sel) out[pos + __popc(sel_mask & ((1u << lane) - 1))] = col_at(j);
+    if (sel) {
+      const int dst = pos + __popc(sel_mask & ((1u << lane) - 1));
+      out[dst] = col_at(j);
+      if (sel_out) sel_out[dst] = key_score(key);
+    }
     pos += __popc(sel_mask);
     eq_rank += __popc(eq_mask);
   }

@@ -1,0 +1,371 @@
+// Top-k selection of a few long rows (velog.io DSA page, §1.2 Fine-grained Token Selection), one cluster of
+// kTkcCluster CTAs per row.
+//
+// With fewer rows than SMs (a decode step: one row per sequence, up to 131K keys) one CTA per row leaves most of
+// the GPU idle and serialises the row's passes on one SM.  Here the row is cut into kTkcCluster contiguous
+// segments, one per CTA of a cluster, and the CTAs combine their counts through distributed shared memory:
+//   1. every CTA builds the histogram of the top 11 order-key bits of its segment; the cluster's histogram (the
+//      sum of the CTAs', read from each peer) gives the bin b* holding the k-th largest key, the same in every CTA;
+//   2. every CTA collects the keys of bin >= b* of its segment into per-warp regions in column order;
+//   3. a radix select over those candidates finds the exact k-th largest key T and the number `need` of keys
+//      equal to T to take: each pass sums the CTAs' digit histograms (double-buffered, so one cluster barrier per
+//      pass suffices), and every CTA picks the same digit;
+//   4. the CTAs exchange their counts of keys > T and == T; each then writes its selected columns, in column order,
+//      at its offset in the output row.
+// The selection is "score descending, smaller column first on ties", identical to topk_rows_kernel's.  When a
+// warp's candidate region would overflow (massive ties), the whole cluster takes a 4-pass radix select over the
+// row segments instead, and the output walks the segments.
+#pragma once
+#include "topk.cuh"
+
+namespace dsa {
+
+constexpr int kTkcCluster = 8;          // CTAs per row (portable cluster size)
+constexpr int kTkcThreads = 256;
+constexpr int kTkcRegion = 384;         // candidate slots per warp (3072 per CTA)
+
+struct TkcSmem {
+  static constexpr int W = kTkcThreads / 32;
+  uint32_t bins[kTopkBins];             // this CTA's top-11-bit histogram of its segment (peers read it)
+  uint32_t merged[kTopkBins];           // the cluster's histogram (radix passes use its first 256 entries)
+  uint32_t hist[W][256];                // radix pass: per-warp digit histograms
+  uint32_t hist_cta[2][256];            // radix pass: this CTA's digit histogram, double-buffered (peers read it)
+  uint32_t cand_key[W][kTkcRegion];
+  int cand_idx[W][kTkcRegion];
+  int region_n[W];
+  int w_gt[W], w_eq[W], w_base[W], w_eqb[W];
+  int cta_gt, cta_eq;                   // peers read them for the output offsets
+  uint32_t cta_over;                    // peers read it: a warp region of this CTA overflowed
+  uint32_t s_bin, s_need, s_digit;
+};
+static_assert(4 * (sizeof(TkcSmem) + 1024) <= 228 * 1024, "four cluster top-k CTAs per SM");
+
+__device__ __forceinline__ uint32_t ld_cluster_u32(uint32_t cluster_addr) {
+  uint32_t v;
+  asm volatile("ld.shared::cluster.u32 %0, [%1];" : "=r"(v) : "r"(cluster_addr) : "memory");
+  return v;
+}
+__device__ __forceinline__ int ld_cluster_s32(uint32_t cluster_addr) {
+  return static_cast<int>(ld_cluster_u32(cluster_addr));
+}
+// sum over the cluster's CTAs of the u32 at the same shared-memory offset as `local`
+__device__ __forceinline__ uint32_t cluster_sum_u32(const void* local) {
+  const uint32_t a = smem_u32(local);
+  uint32_t s = 0;
+#pragma unroll
+  for (int q = 0; q < kTkcCluster; ++q) s += ld_cluster_u32(map_cluster(a, q));
+  return s;
+}
+
+// Digit of a descending scan: the largest digit d with (count of digits > d) < need <= (count of digits >= d), over
+// the 256 counts in sm.merged[0..255]; sets sm.s_digit and sm.s_need (entries of digit d still to take).  Run by
+// warp 0; lane l owns digits 255 - 8 l .. 248 - 8 l.
+__device__ __forceinline__ void tkc_pick_digit(uint32_t need, TkcSmem& sm) {
+  const int lane = threadIdx.x & 31;
+  uint32_t cnt[8], tot = 0;
+#pragma unroll
+  for (int j = 0; j < 8; ++j) { cnt[j] = sm.merged[255 - 8 * lane - j]; tot += cnt[j]; }
+  uint32_t incl = tot;
+#pragma unroll
+  for (int d = 1; d < 32; d <<= 1) {
+    const uint32_t v = __shfl_up_sync(0xffffffffu, incl, d);
+    if (lane >= d) incl += v;
+  }
+  const uint32_t excl = incl - tot;
+  if (excl < need && need <= incl) {
+    uint32_t run = excl;
+    int j = 0;
+    for (; j < 8; ++j) {
+      if (run + cnt[j] >= need) break;
+      run += cnt[j];
+    }
+    sm.s_digit = static_cast<uint32_t>(255 - 8 * lane - j);
+    sm.s_need = need - run;
+  }
+}
+
+// Cluster-wide radix select on 32-bit keys among the entries with (key & mask) == prefix: returns the exact
+// need-th largest key and sets `need` to the number of entries equal to it that are taken.  each(visit) visits
+// every key this thread owns.  Every thread of every CTA of the cluster calls this with the same arguments.
+template <typename Each>
+__device__ __forceinline__ uint32_t tkc_radix_select(Each each, uint32_t prefix, uint32_t mask, int first_shift,
+                                                     uint32_t& need, TkcSmem& sm) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  int buf = 0;
+  for (int shift = first_shift; shift >= 0; shift -= 8, buf ^= 1) {
+    for (int i = lane; i < 256; i += 32) sm.hist[warp][i] = 0;
+    __syncthreads();
+    each([&](uint32_t key) {
+      if ((key & mask) == prefix) atomicAdd(&sm.hist[warp][(key >> shift) & 255], 1u);
+    });
+    __syncthreads();
+    for (int b = tid; b < 256; b += kTkcThreads) {
+      uint32_t s = 0;
+#pragma unroll
+      for (int w = 0; w < TkcSmem::W; ++w) s += sm.hist[w][b];
+      sm.hist_cta[buf][b] = s;
+    }
+    // every CTA's histogram of this pass is complete; the buffer of the previous pass is no longer read by any
+    // peer (each read it before arriving here), so the next pass may overwrite it
+    cluster_sync();
+    for (int b = tid; b < 256; b += kTkcThreads) sm.merged[b] = cluster_sum_u32(&sm.hist_cta[buf][b]);
+    __syncthreads();
+    if (warp == 0) tkc_pick_digit(need, sm);
+    __syncthreads();
+    prefix |= sm.s_digit << shift;
+    mask |= 255u << shift;
+    need = sm.s_need;
+  }
+  return prefix;
+}
+
+__global__ void __cluster_dims__(kTkcCluster, 1, 1) __launch_bounds__(kTkcThreads, 4)
+    topk_cluster_kernel(const TopkParams p) {
+  extern __shared__ __align__(16) uint8_t tkc_smem_raw[];
+  TkcSmem& sm = *reinterpret_cast<TkcSmem*>(tkc_smem_raw);
+  constexpr int W = TkcSmem::W;
+  const int r = blockIdx.x / kTkcCluster;
+  const int rank = static_cast<int>(cluster_rank());
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  if (r >= p.rows) return;                       // whole clusters only: the grid is rows x kTkcCluster
+  const long long off = p.row_off ? p.row_off[r] : static_cast<long long>(r) * p.ld;
+  const float* x = p.scores + off;
+  long long nl = p.row_len ? p.row_len[r] : static_cast<long long>(p.pos0) + r + 1;
+  if (!p.row_off && nl > p.ld) nl = p.ld;
+  const int n = static_cast<int>(nl < 0 ? 0 : nl);
+  const int k = p.k;
+  int* out = p.idx + static_cast<long long>(r) * p.idx_ld;
+  float* sel_out = p.sel_scores ? p.sel_scores + static_cast<long long>(r) * p.idx_ld : nullptr;
+  if (n <= k) {                                  // the same for every CTA of the cluster: no barrier is skipped
+    if (rank == 0)
+      for (int i = tid; i < k; i += kTkcThreads) {
+        out[i] = (i < n) ? i : -1;
+        if (sel_out) sel_out[i] = (i < n) ? x[i] : -INFINITY;
+      }
+    return;
+  }
+  const bool vec = (reinterpret_cast<uintptr_t>(x) & 15) == 0;
+  // this CTA's segment (a multiple of four columns, so that it starts 16-byte aligned when the row does) and its
+  // warps' sub-segments, all in column order
+  const int cseg = (((n + kTkcCluster - 1) / kTkcCluster) + 3) & ~3;
+  const int c0 = min(n, rank * cseg), c1 = min(n, c0 + cseg);
+  const int wseg = (((c1 - c0 + W - 1) / W) + 3) & ~3;
+  const int w0 = min(c1, c0 + warp * wseg), w1 = min(c1, w0 + wseg);
+
+  // ---------------------------------------------------------------- 1. histograms, the cluster's bin b*
+  for (int i = tid; i < kTopkBins; i += kTkcThreads) sm.bins[i] = 0;
+  if (tid == 0) sm.s_bin = 0xFFFFFFFFu;
+  __syncthreads();
+  if (vec) {
+    for (int i0 = c0 + 4 * tid; i0 < c1; i0 += 16 * kTkcThreads) {
+      float4 v[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int i = i0 + 4 * u * kTkcThreads;
+        if (i + 3 < c1) {
+          v[u] = *reinterpret_cast<const float4*>(x + i);
+        } else {
+          v[u].x = (i < c1) ? x[i] : NAN;
+          v[u].y = (i + 1 < c1) ? x[i + 1] : NAN;
+          v[u].z = (i + 2 < c1) ? x[i + 2] : NAN;
+          v[u].w = NAN;
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int i = i0 + 4 * u * kTkcThreads;
+        if (i < c1) atomicAdd(&sm.bins[order_key(v[u].x) >> 21], 1u);
+        if (i + 1 < c1) atomicAdd(&sm.bins[order_key(v[u].y) >> 21], 1u);
+        if (i + 2 < c1) atomicAdd(&sm.bins[order_key(v[u].z) >> 21], 1u);
+        if (i + 3 < c1) atomicAdd(&sm.bins[order_key(v[u].w) >> 21], 1u);
+      }
+    }
+  } else {
+    for (int i = c0 + tid; i < c1; i += kTkcThreads) atomicAdd(&sm.bins[order_key(x[i]) >> 21], 1u);
+  }
+  cluster_sync();                                // every CTA's histogram is complete
+  for (int b = tid; b < kTopkBins; b += kTkcThreads) sm.merged[b] = cluster_sum_u32(&sm.bins[b]);
+  __syncthreads();
+  {
+    // bin holding the k-th largest key of the row: thread t owns bins 2047 - 8 t .. 2040 - 8 t (descending)
+    constexpr int BPT = kTopkBins / kTkcThreads;
+    uint32_t c8[BPT], tot = 0;
+#pragma unroll
+    for (int j = 0; j < BPT; ++j) { c8[j] = sm.merged[kTopkBins - 1 - BPT * tid - j]; tot += c8[j]; }
+    uint32_t incl = tot;
+#pragma unroll
+    for (int d = 1; d < 32; d <<= 1) {
+      const uint32_t v = __shfl_up_sync(0xffffffffu, incl, d);
+      if (lane >= d) incl += v;
+    }
+    if (lane == 31) sm.w_gt[warp] = static_cast<int>(incl);
+    __syncthreads();
+    uint32_t wbase = 0;
+    for (int w = 0; w < warp; ++w) wbase += static_cast<uint32_t>(sm.w_gt[w]);
+    const uint32_t excl = wbase + incl - tot;
+    const uint32_t kk = static_cast<uint32_t>(k);
+    if (excl < kk && kk <= excl + tot) {
+      uint32_t run = excl;
+      int j = 0;
+      for (; j < BPT; ++j) {
+        if (run + c8[j] >= kk) break;
+        run += c8[j];
+      }
+      sm.s_bin = static_cast<uint32_t>(kTopkBins - 1 - BPT * tid - j);
+      sm.s_need = kk - run;
+    }
+    __syncthreads();
+  }
+  const uint32_t bstar = sm.s_bin;               // n > k keys were counted, so the bin exists
+  const uint32_t need_bin = sm.s_need;
+
+  // ---------------------------------------------------------------- 2. candidates of bin >= b*, in column order
+  // A key is in bin >= b* exactly when the score is >= the float whose order key is b* << 21, so the pass compares
+  // raw scores.  Lane l takes 16 consecutive columns of each 512-column step of its warp's sub-segment (four
+  // 16-byte loads in flight when the row is aligned); one warp scan of the lanes' counts places the candidates.
+  {
+    const uint32_t kb = bstar << 21;
+    uint32_t tb = (kb & 0x80000000u) ? (kb & 0x7FFFFFFFu) : ~kb;
+    if (!(kb & 0x80000000u) && tb > 0xFF800000u) tb = 0xFF800000u;   // no float key lies below that of -inf
+    const float thr = __uint_as_float(tb);
+    const bool low = bstar == 0;               // bin 0 holds NaN too, which compares false: take every key
+    int cnt = 0;
+    for (int i00 = w0; i00 < w1; i00 += 512) {
+      const int c0l = i00 + 16 * lane;
+      float xv[16];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int col = c0l + 4 * u;
+        if (vec && col + 3 < w1) {
+          const float4 v = *reinterpret_cast<const float4*>(x + col);
+          xv[4 * u] = v.x; xv[4 * u + 1] = v.y; xv[4 * u + 2] = v.z; xv[4 * u + 3] = v.w;
+        } else {
+#pragma unroll
+          for (int e = 0; e < 4; ++e) xv[4 * u + e] = (col + e < w1) ? x[col + e] : -INFINITY;
+        }
+      }
+      int c = 0;
+#pragma unroll
+      for (int e = 0; e < 16; ++e) c += (c0l + e < w1 && (low || xv[e] >= thr)) ? 1 : 0;
+      int incl = c;
+#pragma unroll
+      for (int d = 1; d < 32; d <<= 1) {
+        const int v = __shfl_up_sync(0xffffffffu, incl, d);
+        if (lane >= d) incl += v;
+      }
+      const int tot = __shfl_sync(0xffffffffu, incl, 31);
+      if (c) {
+        int pos = cnt + incl - c;
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          if (c0l + e < w1 && (low || xv[e] >= thr)) {
+            if (pos < kTkcRegion) {
+              sm.cand_key[warp][pos] = order_key(xv[e]);
+              sm.cand_idx[warp][pos] = c0l + e;
+            }
+            ++pos;
+          }
+        }
+      }
+      cnt += tot;
+    }
+    if (lane == 0) {
+      sm.region_n[warp] = min(cnt, kTkcRegion);
+      sm.w_eq[warp] = cnt > kTkcRegion ? 1 : 0;
+    }
+  }
+  __syncthreads();
+  if (tid == 0) {
+    uint32_t over = 0;
+    for (int w = 0; w < W; ++w) over |= static_cast<uint32_t>(sm.w_eq[w]);
+    sm.cta_over = over;
+  }
+  cluster_sync();                                // every CTA's overflow flag is set
+  bool from_row = false;
+  {
+    uint32_t over = 0;
+#pragma unroll
+    for (int q = 0; q < kTkcCluster; ++q) over |= ld_cluster_u32(map_cluster(smem_u32(&sm.cta_over), q));
+    from_row = over != 0;                        // the same decision in every CTA
+  }
+
+  // ---------------------------------------------------------------- 3. the exact threshold
+  uint32_t need, T;
+  if (!from_row) {
+    need = need_bin;
+    auto each = [&](auto visit) {
+      for (int j = lane; j < sm.region_n[warp]; j += 32) visit(sm.cand_key[warp][j]);
+    };
+    T = tkc_radix_select(each, bstar << 21, 0xFFE00000u, 16, need, sm);
+  } else {
+    need = static_cast<uint32_t>(k);
+    auto each = [&](auto visit) {
+      for (int i = w0 + lane; i < w1; i += 32) visit(order_key(x[i]));
+    };
+    T = tkc_radix_select(each, 0u, 0u, 24, need, sm);
+  }
+
+  // ---------------------------------------------------------------- 4. ordered output
+  const int span = from_row ? w1 - w0 : sm.region_n[warp];
+  auto key_at = [&](int j) -> uint32_t { return from_row ? order_key(x[w0 + j]) : sm.cand_key[warp][j]; };
+  auto col_at = [&](int j) -> int { return from_row ? w0 + j : sm.cand_idx[warp][j]; };
+  int gt = 0, eq = 0;
+  for (int j = lane; j < span; j += 32) {
+    const uint32_t key = key_at(j);
+    gt += key > T;
+    eq += key == T;
+  }
+#pragma unroll
+  for (int d = 16; d > 0; d >>= 1) {
+    gt += __shfl_xor_sync(0xffffffffu, gt, d);
+    eq += __shfl_xor_sync(0xffffffffu, eq, d);
+  }
+  if (lane == 0) { sm.w_gt[warp] = gt; sm.w_eq[warp] = eq; }
+  __syncthreads();
+  if (tid == 0) {
+    int g = 0, e = 0;
+    for (int w = 0; w < W; ++w) { g += sm.w_gt[w]; e += sm.w_eq[w]; }
+    sm.cta_gt = g;
+    sm.cta_eq = e;
+  }
+  cluster_sync();                                // every CTA's counts are set
+  if (tid == 0) {
+    // this CTA's place in the row: the entries the CTAs before it take
+    int base = 0, eqb = 0;
+    for (int q = 0; q < rank; ++q) {
+      const int gq = ld_cluster_s32(map_cluster(smem_u32(&sm.cta_gt), q));
+      const int eqq = ld_cluster_s32(map_cluster(smem_u32(&sm.cta_eq), q));
+      base += gq + max(0, min(eqq, static_cast<int>(need) - eqb));
+      eqb += eqq;
+    }
+    for (int w = 0; w < W; ++w) {
+      sm.w_base[w] = base;
+      sm.w_eqb[w] = eqb;
+      base += sm.w_gt[w] + max(0, min(sm.w_eq[w], static_cast<int>(need) - eqb));
+      eqb += sm.w_eq[w];
+    }
+  }
+  __syncthreads();
+  int pos = sm.w_base[warp];
+  int eq_rank = sm.w_eqb[warp];
+  for (int j0 = 0; j0 < span; j0 += 32) {
+    const int j = j0 + lane;
+    uint32_t key = 0;
+    if (j < span) key = key_at(j);
+    const bool is_eq = j < span && key == T;
+    const uint32_t eq_mask = __ballot_sync(0xffffffffu, is_eq);
+    const int my_eq_rank = eq_rank + __popc(eq_mask & ((1u << lane) - 1));
+    const bool sel = j < span && (key > T || (is_eq && my_eq_rank < static_cast<int>(need)));
+    const uint32_t sel_mask = __ballot_sync(0xffffffffu, sel);
+    const int dst = pos + __popc(sel_mask & ((1u << lane) - 1));
+    if (sel && dst < k) {                        // dst < k always; the bound keeps a fault out of other rows
+      out[dst] = col_at(j);
+      if (sel_out) sel_out[dst] = key_score(key);
+    }
+    pos += __popc(sel_mask);
+    eq_rank += __popc(eq_mask);
+  }
+  cluster_sync();                                // no CTA leaves while a peer may still read its shared memory
+}
+
+}  // namespace dsa

@@ -166,3 +166,87 @@ def test_full_batch_256_steps_checked_at_first_and_last(dsa):
         assert np.mean(recs) >= RECALL, f"step {step}: mean recall {np.mean(recs)}"
         assert np.abs(gots - att).max() <= MAX_ABS and rel_l2(gots, att) <= REL_L2, f"step {step}"
         assert rel_l2(gots, e2e_ref) <= e2e_bound(np.mean(recs)), f"step {step}"
+
+
+def _paged_copy(cache, lens, offs, steps, page_rows, seed, spare=5):
+    """The flat caches' sequences moved into shuffled pages of page pools (with spare pages full of NaN), and
+    the page table [B, max_pages] that maps them."""
+    B = len(lens)
+    need = [-(-(n + steps) // page_rows) for n in lens]
+    max_pages = max(need) + 1
+    num_pages = sum(need) + spare
+    perm = np.random.default_rng(seed).permutation(num_pages)
+    table = np.full((B, max_pages), -1, dtype=np.int32)
+    kc = torch.zeros((num_pages * page_rows, cache["k_cache"].shape[1]), dtype=torch.uint8, device="cuda")
+    ks = torch.full((num_pages * page_rows,), float("nan"), dtype=torch.float32, device="cuda")
+    nan_bf16 = torch.tensor([0x7FC0], dtype=torch.int16).view(torch.bfloat16).item()
+    cc = torch.full((num_pages * page_rows, cache["c_cache"].shape[1]), nan_bf16, dtype=torch.bfloat16, device="cuda")
+    at = 0
+    for b in range(B):
+        for j in range(need[b]):
+            pg = int(perm[at])
+            at += 1
+            table[b, j] = pg
+            r0, r1 = offs[b] + j * page_rows, min(offs[b] + lens[b] + steps, offs[b] + (j + 1) * page_rows)
+            d0 = pg * page_rows
+            kc[d0:d0 + r1 - r0] = cache["k_cache"][r0:r1].view(torch.uint8)
+            ks[d0:d0 + r1 - r0] = cache["k_scale_cache"][r0:r1]
+            cc[d0:d0 + r1 - r0] = cache["c_cache"][r0:r1]
+    return torch.from_numpy(table).cuda(), kc.view(torch.float8_e4m3fn), ks, cc
+
+
+@pytest.mark.parametrize("page_rows", [128, 256])
+def test_paged_cache_identical_to_flat(dsa, page_rows):
+    # The same sequences in flat caches and in shuffled pages of page pools (spare pages hold NaN): every step's
+    # selection, output and LSE are bit-identical, and the appended entries land in the right pages.
+    cfg = G.DecodeConfig("paged", B=6, len_lo=100, len_hi=20000, steps=3)
+    seed = 47
+    cache = G.decode_fill_cache(cfg, seed, device="cuda")
+    lens, offs = cache["lens"], cache["offs"]
+    table, kc, ks, cc = _paged_copy(cache, lens, offs, cfg.steps, page_rows, seed)
+    cache_off = torch.tensor(offs, dtype=torch.int64, device="cuda")
+    ctx = torch.tensor(lens, dtype=torch.int32, device="cuda")
+    for step in range(cfg.steps):
+        st = G.decode_step_inputs(cfg, seed, step, device="cuda")
+        args = (st["q_idx"], st["q_scale"], st["w"], st["q"], st["k_new"], st["k_scale_new"], st["c_new"])
+        i1, o1, l1 = dsa.dsa_forward_decode(cache_off, ctx, *args, cache["k_cache"], cache["k_scale_cache"],
+                                            cache["c_cache"], cfg.k, cfg.scale)
+        i2, o2, l2 = dsa.dsa_forward_decode_paged(table, page_rows, ctx, *args, kc, ks, cc, cfg.k, cfg.scale)
+        assert dsa.dsa_get_device_status() == 0
+        assert torch.equal(i1, i2), f"step {step}: selection"
+        assert torch.equal(o1, o2), f"step {step}: output"
+        assert torch.equal(l1, l2), f"step {step}: lse"
+        ctx += 1
+    tab = table.cpu().numpy()
+    for b in range(cfg.B):
+        for s in range(cfg.steps):
+            pos = lens[b] + s
+            row = int(tab[b, pos // page_rows]) * page_rows + pos % page_rows
+            assert torch.equal(cc[row], cache["c_cache"][offs[b] + pos])
+            assert torch.equal(kc[row].view(torch.uint8), cache["k_cache"][offs[b] + pos].view(torch.uint8))
+
+
+def test_paged_bad_page_is_reported_and_skipped(dsa):
+    cfg = G.DecodeConfig("paged_bad", B=3, len_lo=3000, len_hi=9000, steps=1, mode="int")
+    seed = 48
+    cache = G.decode_fill_cache(cfg, seed, device="cuda")
+    lens, offs = cache["lens"], cache["offs"]
+    table, kc, ks, cc = _paged_copy(cache, lens, offs, cfg.steps, 128, seed)
+    table[1, 0] = kc.shape[0] // 128          # one past the last page of the pools
+    before = cc.clone()
+    ctx = torch.tensor(lens, dtype=torch.int32, device="cuda")
+    st = G.decode_step_inputs(cfg, seed, 0, device="cuda")
+    idx, out, _ = dsa.dsa_forward_decode_paged(table, 128, ctx, st["q_idx"], st["q_scale"], st["w"], st["q"],
+                                               st["k_new"], st["k_scale_new"], st["c_new"], kc, ks, cc, cfg.k,
+                                               cfg.scale)
+    assert dsa.dsa_get_device_status() == 6
+    idx = idx.cpu().numpy()
+    assert (idx[1] == -1).all()
+    changed = (cc.view(torch.int16) != before.view(torch.int16)).any(dim=1).nonzero().flatten().tolist()
+    tab = table.cpu().numpy()
+    assert changed == sorted(int(tab[b, lens[b] // 128]) * 128 + lens[b] % 128 for b in (0, 2))
+    step_q = G.decode_step_inputs(cfg, seed, 0)
+    for b in (0, 2):
+        n = lens[b] + 1
+        ref = O.decode_row(G.decode_cache_rows(cfg, seed, b, range(n)), step_q, b, n, cfg.k, cfg.scale)
+        assert np.array_equal(idx[b], ref["idx"])

@@ -535,7 +535,8 @@ def bench_decode(dsa, cfg, steps, warmup, ws_n, rank, pk):
 # ------------------------------------------------------------------------------------------ profiling cases
 def kernels_small(dsa):
     """One launch each of the main kernels on small inputs (for ncu captures): sparse MLA over 1184 query
-    tokens of the 128K latent, indexer scores of a 2048-row block against 131072 keys, top-k of those rows."""
+    tokens of the 128K latent, indexer scores of a 2048-row block against 131072 keys, top-k of those rows, and one
+    decode step of 16 sequences with contexts of 4K-128K."""
     cfg = PREFILL
     keys = G.prefill_keys(cfg, 5, device="cuda")
     rows = range(cfg.L - 2048, cfg.L)
@@ -550,7 +551,19 @@ def kernels_small(dsa):
     dsa.dsa_topk(sc, cfg.k, pos0=cfg.L - 2048)
     torch.cuda.synchronize()
     assert dsa.dsa_get_device_status() == 0
-    print(json.dumps({"kernels_small": "ok", "attention_tokens": T, "indexer_rows": 2048, "keys": cfg.L}))
+    del sc, qs, idx
+    # one decode step of 16 sequences with contexts of 4K-128K (append, indexer, cluster top-k, attention)
+    dcfg = G.DecodeConfig("decode_16", B=16, len_lo=4096, len_hi=131072, steps=4)
+    cache = G.decode_fill_cache(dcfg, 5, device="cuda")
+    st = G.decode_step_inputs(dcfg, 5, 0, device="cuda")
+    dsa.dsa_forward_decode(torch.tensor(cache["offs"], dtype=torch.int64, device="cuda"),
+                           torch.tensor(cache["lens"], dtype=torch.int32, device="cuda"), st["q_idx"], st["q_scale"],
+                           st["w"], st["q"], st["k_new"], st["k_scale_new"], st["c_new"], cache["k_cache"],
+                           cache["k_scale_cache"], cache["c_cache"], dcfg.k, dcfg.scale)
+    torch.cuda.synchronize()
+    assert dsa.dsa_get_device_status() == 0
+    print(json.dumps({"kernels_small": "ok", "attention_tokens": T, "indexer_rows": 2048, "keys": cfg.L,
+                      "decode_sequences": dcfg.B, "decode_keys": sum(n + 1 for n in cache["lens"])}))
 
 
 # ------------------------------------------------------------------------------------------ oracle arm

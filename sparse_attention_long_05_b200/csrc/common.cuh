@@ -43,6 +43,14 @@ __device__ __forceinline__ void trace_event(int ev, long long tile) {
 #define DSA_TRACE_EVENT(ev, tile) ((void)0)
 #endif
 
+// ------------------------------------------------------------------------------------------ launch order
+// Programmatic dependent launch: the library launches its kernels so that a kernel may be scheduled before its
+// predecessor on the stream has finished.  Each kernel lets its successor be scheduled early (pdl_allow_next) and
+// waits for its predecessor to complete, with its writes visible (pdl_wait), before it reads or writes any memory
+// the predecessor may touch.  Launched without the attribute, both are no-ops.
+__device__ __forceinline__ void pdl_allow_next() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 // ------------------------------------------------------------------------------------------ addressing
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));

@@ -9,6 +9,7 @@
 #include <algorithm>
 #include <atomic>
 #include <mutex>
+#include <vector>
 
 #include "common.cuh"
 #include "indexer.cuh"
@@ -69,6 +70,8 @@ __global__ void __launch_bounds__(kAppendThreads)
     decode_append_kernel(int B, DecodeLayout lay, const int* ctx_len, const uint8_t* k_new,
                          const float* k_scale_new, const uint16_t* c_new, uint8_t* k_cache, float* k_scale_cache,
                          uint16_t* c_cache, int d_I, int* len1, long long* score_off, long long score_cap) {
+  pdl_allow_next();
+  pdl_wait();
   const int b = blockIdx.x;
   if (b >= B) return;
   // start of this sequence's score row: the padded lengths of the sequences before it that pass the cheap part
@@ -127,6 +130,25 @@ __global__ void varlen_row_off_kernel(const long long* cu, int nseq, long long t
     if (cu[mid] <= t) lo = mid; else hi = mid - 1;
   }
   row_off[t] = cu[lo];
+}
+
+// Score-row offset and length of every row of a group of packed sequences for the top-k: row r of sequence b at
+// position t reads the t + 1 scores at seq_off[b] + (t - k) * seq_ld[b] (rows t < k read nothing: every earlier key
+// is selected).  cu: the group's sequence starts relative to its first row, nseq + 1 entries.
+__global__ void varlen_score_rows_kernel(const long long* cu, int nseq, const long long* seq_off, const int* seq_ld,
+                                         int k, long long* row_off, int* row_len) {
+  pdl_allow_next();
+  pdl_wait();
+  const long long r = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (r >= cu[nseq]) return;
+  int lo = 0, hi = nseq - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (cu[mid] <= r) lo = mid; else hi = mid - 1;
+  }
+  const long long t = r - cu[lo];
+  row_len[r] = static_cast<int>(t + 1);
+  row_off[r] = (t >= k) ? seq_off[lo] + (t - k) * seq_ld[lo] : 0;
 }
 
 // ------------------------------------------------------------------------------------------ bounded-wait self-check
@@ -204,6 +226,24 @@ cudaError_t set_smem(K kernel, int bytes) {
 
 std::atomic<unsigned long long> g_launches{0};
 
+// Launch with programmatic stream serialisation (see pdl_wait): the kernel may be scheduled while its predecessor
+// on the stream finishes, and waits for it on the device.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                       Args... args) {
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
+}
+
 dsa_status_t last_launch_status() {
   g_launches.fetch_add(1, std::memory_order_relaxed);
   return cudaGetLastError() == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
@@ -236,7 +276,7 @@ dsa_status_t launch_indexer(const uint8_t* q_idx, int q_rows, const uint8_t* k_i
   auto kern = indexer_kernel<H_I, D_I, NT, NG, QBUF, KST, EPI, MODE>;
   const int smem = (C::TMEM_COLS == 512 && C::SMEM < kMinIndexerSmem) ? kMinIndexerSmem : C::SMEM;
   if (set_smem(kern, smem) != cudaSuccess) return DSA_ERR_CUDA;
-  kern<<<grid, C::NUM_THREADS, smem, st>>>(tq, tk, p);
+  if (launch_pdl(kern, dim3(grid), dim3(C::NUM_THREADS), smem, st, tq, tk, p) != cudaSuccess) return DSA_ERR_CUDA;
   return last_launch_status();
 }
 
@@ -277,6 +317,56 @@ dsa_status_t run_indexer_scores(const uint8_t* q_idx, const float* q_scale, cons
   return launch_indexer<4, 64, 64, 4, 1, 4, 2, kModeScores>(q_idx, T, k_idx, S, p, grid, st);
 }
 
+// Indexer scores of the runs of query rows in segs_host (one launch; segs_dev: a device copy of the table, written
+// by the caller), into `scores`.  Chooses the key split and fills each run's nsplit and item0 in segs_host before
+// the caller copies it.  Returns the number of items through *n_items.
+void plan_segments(IndexerSeg* segs, int n_segs, int tok, int* split_tiles, int* n_items) {
+  const int sms = num_sms();
+  int best = 1;
+  double best_cost = 1e300;
+  for (int split = 1; split <= 64; ++split) {
+    long long items = 0;
+    for (int i = 0; i < n_segs; ++i) {
+      const int nqb = (segs[i].n_rows + tok - 1) / tok, ntiles = (segs[i].S + 127) / 128;
+      items += static_cast<long long>(nqb) * ((ntiles + split - 1) / split);
+    }
+    const double cost = static_cast<double>((items + sms - 1) / sms) * (split + 2.0);
+    if (cost < best_cost - 1e-9) { best_cost = cost; best = split; }
+  }
+  int item = 0;
+  for (int i = 0; i < n_segs; ++i) {
+    const int nqb = (segs[i].n_rows + tok - 1) / tok, ntiles = (segs[i].S + 127) / 128;
+    segs[i].nsplit = (ntiles + best - 1) / best;
+    segs[i].item0 = item;
+    item += nqb * segs[i].nsplit;
+  }
+  *split_tiles = best;
+  *n_items = item;
+}
+
+dsa_status_t run_indexer_segments(const uint8_t* q_idx, long long q_rows, const float* q_scale, const uint8_t* k_idx,
+                                  long long k_rows, const float* k_scale, const float* w, int H_I, int d_I,
+                                  const IndexerSeg* segs_dev, int n_segs, int split_tiles, int n_items,
+                                  float* scores, cudaStream_t st) {
+  if (n_items <= 0) return DSA_OK;
+  IndexerParams p{};
+  p.w = w;
+  p.q_scale = q_scale;
+  p.k_scale = k_scale;
+  p.scores = scores;
+  p.segs = segs_dev;
+  p.n_segs = n_segs;
+  p.split_tiles = split_tiles;
+  p.n_items = n_items;
+  const int sms = num_sms();
+  const int grid = n_items < sms ? n_items : sms;
+  if (H_I == 64)
+    return launch_indexer<64, 128, 4, 4, 1, 4, 2, kModeSegments>(q_idx, static_cast<int>(q_rows), k_idx, k_rows, p,
+                                                                 grid, st);
+  return launch_indexer<4, 64, 64, 4, 1, 4, 2, kModeSegments>(q_idx, static_cast<int>(q_rows), k_idx, k_rows, p, grid,
+                                                             st);
+}
+
 dsa_status_t run_topk(const float* scores, long long ld, const long long* row_off, const int* row_len, int pos0,
                       int rows, int k, int* idx, long long idx_ld, cudaStream_t st, float* sel_scores = nullptr) {
   if (rows <= 0) return DSA_OK;
@@ -284,11 +374,15 @@ dsa_status_t run_topk(const float* scores, long long ld, const long long* row_of
   if (rows < num_sms()) {
     // fewer rows than SMs (decode): one cluster of kTkcCluster CTAs per row
     if (set_smem(topk_cluster_kernel, static_cast<int>(sizeof(TkcSmem))) != cudaSuccess) return DSA_ERR_CUDA;
-    topk_cluster_kernel<<<rows * kTkcCluster, kTkcThreads, sizeof(TkcSmem), st>>>(p);
+    if (launch_pdl(topk_cluster_kernel, dim3(rows * kTkcCluster), dim3(kTkcThreads), sizeof(TkcSmem), st, p) !=
+        cudaSuccess)
+      return DSA_ERR_CUDA;
   } else {
     if (set_smem(topk_rows_kernel<kTopkThreads>, static_cast<int>(sizeof(TopkSmem<kTopkThreads>))) != cudaSuccess)
       return DSA_ERR_CUDA;
-    topk_rows_kernel<kTopkThreads><<<rows, kTopkThreads, sizeof(TopkSmem<kTopkThreads>), st>>>(p);
+    if (launch_pdl(topk_rows_kernel<kTopkThreads>, dim3(rows), dim3(kTopkThreads), sizeof(TopkSmem<kTopkThreads>), st,
+                   p) != cudaSuccess)
+      return DSA_ERR_CUDA;
   }
   return last_launch_status();
 }
@@ -340,7 +434,9 @@ dsa_status_t run_mla(const uint16_t* q, const uint16_t* c, long long S, const in
   const int per_cluster = kl_out ? 2 : 1;
   int clusters = num_sms() / 2;
   if (clusters > (T + per_cluster - 1) / per_cluster) clusters = (T + per_cluster - 1) / per_cluster;
-  sparse_mla_kernel<<<2 * clusters, mla::THREADS, mla::SMEM, st>>>(tq, tc, tcd, p);
+  if (launch_pdl(sparse_mla_kernel, dim3(2 * clusters), dim3(mla::THREADS), mla::SMEM, st, tq, tc, tcd, p) !=
+      cudaSuccess)
+    return DSA_ERR_CUDA;
   return last_launch_status();
 }
 
@@ -354,6 +450,22 @@ size_t prefill_chunk_rows(int L) {
   if (r < 256) r = 256;
   if (r > size_t(L)) r = size_t(L);
   return r;
+}
+
+int round4(int n) { return (n + 3) & ~3; }
+
+// Scores the varlen select holds at once: at least one sequence's blocked select (the longest), and up to 1 GiB
+// for groups of sequences scored together.
+size_t varlen_score_floats(int64_t total, int max_len) {
+  const size_t one = prefill_chunk_rows(max_len) * size_t(max_len);
+  const size_t all = size_t(total) * size_t(round4(max_len));
+  const size_t cap = size_t(1) << 28;
+  return std::max(one, std::min(all, cap));
+}
+
+// Group metadata of the varlen select: runs of query rows, relative sequence starts, score offsets and strides.
+size_t varlen_meta_bytes(int nseq) {
+  return align_up(size_t(nseq) * sizeof(IndexerSeg), 256) + align_up(size_t(nseq + 1) * 8 + size_t(nseq) * 12, 256);
 }
 
 // Steps 1-2 for rows [pos_begin, pos_end) of one causal sequence (row r attends to keys 0..r): q_idx, q_scale, w and
@@ -431,9 +543,10 @@ dsa_status_t run_decode(int B, const DecodeLayout& lay, const int32_t* ctx_len, 
   long long* soff = reinterpret_cast<long long*>(wsb + at);
   at += align_up(size_t(B) * 8, 256);
   int32_t* idx = idx_out ? idx_out : reinterpret_cast<int32_t*>(wsb + at);
-  decode_append_kernel<<<B, kAppendThreads, 0, st>>>(B, lay, ctx_len, k_new, k_scale_new, c_new, k_cache,
-                                                     k_scale_cache, c_cache, d_I, len1, soff,
-                                                     static_cast<long long>(score_cap));
+  if (launch_pdl(decode_append_kernel, dim3(B), dim3(kAppendThreads), 0, st, B, lay, ctx_len, k_new, k_scale_new,
+                 c_new, k_cache, k_scale_cache, c_cache, d_I, len1, soff, static_cast<long long>(score_cap)) !=
+      cudaSuccess)
+    return DSA_ERR_CUDA;
   dsa_status_t e = last_launch_status();
   if (e != DSA_OK) return e;
   IndexerParams p{};
@@ -632,8 +745,9 @@ dsa_status_t dsa_forward_prefill(const uint8_t* q_idx, const float* q_scale, con
 size_t dsa_prefill_varlen_workspace_size(int nseq, int64_t total, int max_len, int H_I, int d_I, int H, int k) {
   (void)H_I; (void)d_I; (void)H;
   if (nseq <= 0 || total <= 0 || max_len <= 0 || k <= 0) return 0;
-  return align_up(prefill_chunk_rows(max_len) * size_t(max_len) * 4, 256) + align_up(size_t(total) * 8, 256) +
-         align_up(size_t(nseq + 1) * 8, 256) + align_up(size_t(total) * size_t(k) * 4, 256);
+  return align_up(varlen_score_floats(total, max_len) * 4, 256) + align_up(size_t(total) * 8, 256) +
+         align_up(size_t(nseq + 1) * 8, 256) + align_up(size_t(total) * size_t(k) * 4, 256) +
+         align_up(size_t(total) * 8, 256) + align_up(size_t(total) * 4, 256) + varlen_meta_bytes(nseq);
 }
 
 dsa_status_t dsa_forward_prefill_varlen(int nseq, const int64_t* cu_seqlens, const uint8_t* q_idx,
@@ -659,29 +773,106 @@ dsa_status_t dsa_forward_prefill_varlen(int nseq, const int64_t* cu_seqlens, con
   if (!ws || ws_bytes < dsa_prefill_varlen_workspace_size(nseq, total, max_len, H_I, d_I, H, k))
     return DSA_ERR_WORKSPACE;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  // workspace: one sequence's score block (sized for the longest), per-token row offsets, cu_seqlens, indices
+  // workspace: scores, per-token row offsets (attention), cu_seqlens, indices, per-row score offsets and lengths
+  // (top-k), then the metadata of a group of sequences (runs of query rows, relative starts, score offsets, strides)
   char* wsb = static_cast<char*>(ws);
-  const size_t score_bytes = align_up(prefill_chunk_rows(max_len) * size_t(max_len) * 4, 256);
-  size_t at = score_bytes;
+  const size_t budget = varlen_score_floats(total, max_len);
+  float* sc = reinterpret_cast<float*>(wsb);
+  size_t at = align_up(budget * 4, 256);
   long long* row_off = reinterpret_cast<long long*>(wsb + at);
   at += align_up(size_t(total) * 8, 256);
   long long* cu_dev = reinterpret_cast<long long*>(wsb + at);
   at += align_up(size_t(nseq + 1) * 8, 256);
   int32_t* idx = idx_out ? idx_out : reinterpret_cast<int32_t*>(wsb + at);
+  at += align_up(size_t(total) * size_t(k) * 4, 256);
+  long long* tk_off = reinterpret_cast<long long*>(wsb + at);
+  at += align_up(size_t(total) * 8, 256);
+  int* tk_len = reinterpret_cast<int*>(wsb + at);
+  at += align_up(size_t(total) * 4, 256);
+  char* meta = wsb + at;
+  IndexerSeg* segs_dev = reinterpret_cast<IndexerSeg*>(meta);
+  long long* gcu_dev = reinterpret_cast<long long*>(meta + align_up(size_t(nseq) * sizeof(IndexerSeg), 256));
+  long long* soff_dev = gcu_dev + (nseq + 1);
+  int* sld_dev = reinterpret_cast<int*>(soff_dev + nseq);
   if (cudaMemcpyAsync(cu_dev, cu_seqlens, size_t(nseq + 1) * 8, cudaMemcpyHostToDevice, st) != cudaSuccess)
     return DSA_ERR_CUDA;
   varlen_row_off_kernel<<<static_cast<unsigned>((total + 255) / 256), 256, 0, st>>>(cu_dev, nseq, total, row_off);
   dsa_status_t e = last_launch_status();
   if (e != DSA_OK) return e;
-  // steps 1-2 per sequence (its own causal positions 0..len-1), then step 3 for every token in one launch
-  for (int b = 0; b < nseq; ++b) {
-    const int64_t r = cu_seqlens[b];
-    const int len = static_cast<int>(cu_seqlens[b + 1] - r);
-    if (len == 0) continue;
-    e = dsa_prefill_select(q_idx + r * H_I * d_I, q_scale ? q_scale + r : nullptr, k_idx + r * d_I,
-                           k_scale ? k_scale + r : nullptr, w + r * H_I, len, H_I, d_I, k, idx + r * k, ws,
-                           score_bytes, stream);
-    if (e != DSA_OK) return e;
+  // Steps 1-2.  Consecutive sequences are grouped while their scored rows (t >= k) fit the score buffer; a group
+  // is one indexer launch over all of its sequences' scored rows and one top-k launch over all of its rows.  A
+  // sequence whose scores alone exceed the buffer takes the blocked select of dsa_prefill_select.
+  std::vector<IndexerSeg> segs;
+  std::vector<long long> gcu, soff;
+  std::vector<int> sld;
+  const int tok = (H_I == 64) ? 16 : 256;
+  for (int b = 0; b < nseq;) {
+    const int64_t r0 = cu_seqlens[b];
+    const int len = static_cast<int>(cu_seqlens[b + 1] - r0);
+    const size_t need = (len > k) ? size_t(len - k) * size_t(round4(len)) : 0;
+    if (need > budget) {
+      e = select_rows(q_idx + r0 * H_I * d_I, q_scale ? q_scale + r0 : nullptr, k_idx + r0 * d_I,
+                      k_scale ? k_scale + r0 : nullptr, w + r0 * H_I, H_I, d_I, k, 0, len, idx + r0 * k, sc,
+                      prefill_chunk_rows(len), st);
+      if (e != DSA_OK) return e;
+      ++b;
+      continue;
+    }
+    const int b0 = b;
+    size_t used = 0;
+    segs.clear();
+    gcu.assign(1, 0);
+    soff.clear();
+    sld.clear();
+    while (b < nseq && segs.size() < static_cast<size_t>(kMaxDecodeSeqs)) {
+      const int64_t rb = cu_seqlens[b];
+      const int lb = static_cast<int>(cu_seqlens[b + 1] - rb);
+      const size_t nb = (lb > k) ? size_t(lb - k) * size_t(round4(lb)) : 0;
+      if (used + nb > budget) break;
+      if (nb) {
+        IndexerSeg sg{};
+        sg.q_row0 = rb + k;
+        sg.key_row0 = rb;
+        sg.out_base = static_cast<long long>(used);
+        sg.pos0 = k;
+        sg.n_rows = lb - k;
+        sg.S = lb;
+        sg.ld = round4(lb);
+        segs.push_back(sg);
+      }
+      soff.push_back(static_cast<long long>(used));
+      sld.push_back(round4(lb));
+      used += nb;
+      gcu.push_back(cu_seqlens[b + 1] - cu_seqlens[b0]);
+      ++b;
+    }
+    const int ng = b - b0;
+    int split = 1, n_items = 0;
+    if (!segs.empty()) {
+      plan_segments(segs.data(), static_cast<int>(segs.size()), tok, &split, &n_items);
+      if (cudaMemcpyAsync(segs_dev, segs.data(), segs.size() * sizeof(IndexerSeg), cudaMemcpyHostToDevice, st) !=
+          cudaSuccess)
+        return DSA_ERR_CUDA;
+      e = run_indexer_segments(q_idx, total, q_scale, k_idx, total, k_scale, w, H_I, d_I, segs_dev,
+                               static_cast<int>(segs.size()), split, n_items, sc, st);
+      if (e != DSA_OK) return e;
+    }
+    if (cudaMemcpyAsync(gcu_dev, gcu.data(), size_t(ng + 1) * 8, cudaMemcpyHostToDevice, st) != cudaSuccess ||
+        cudaMemcpyAsync(soff_dev, soff.data(), size_t(ng) * 8, cudaMemcpyHostToDevice, st) != cudaSuccess ||
+        cudaMemcpyAsync(sld_dev, sld.data(), size_t(ng) * 4, cudaMemcpyHostToDevice, st) != cudaSuccess)
+      return DSA_ERR_CUDA;
+    const long long grows = gcu[ng];
+    if (grows > 0) {
+      const long long rbase = cu_seqlens[b0];
+      if (launch_pdl(varlen_score_rows_kernel, dim3(static_cast<unsigned>((grows + 255) / 256)), dim3(256), 0, st,
+                     static_cast<const long long*>(gcu_dev), ng, static_cast<const long long*>(soff_dev),
+                     static_cast<const int*>(sld_dev), k, tk_off + rbase, tk_len + rbase) != cudaSuccess)
+        return DSA_ERR_CUDA;
+      e = last_launch_status();
+      if (e != DSA_OK) return e;
+      e = run_topk(sc, 0, tk_off + rbase, tk_len + rbase, 0, static_cast<int>(grows), k, idx + rbase * k, k, st);
+      if (e != DSA_OK) return e;
+    }
   }
   return run_mla(q, c, static_cast<int>(total), idx, row_off, static_cast<int>(total), H, k, scale, out, lse, st,
                  kMlaCausal);

@@ -25,12 +25,28 @@
 //                fp32 scores from score_off[b] on (one packed row per sequence).  The key tiles of all sequences,
 //                laid end to end, are cut into gridDim.x equal ranges, one per CTA; a CTA's items are the pieces
 //                of the sequences its range covers, so every CTA streams the same number of key tiles.
+//   kModeSegments item = (segment, block of NG*NT query rows, range of key tiles); a segment is a run of query rows
+//                of one sequence of a packed batch (its own query rows, key rows, positions and score rows), so
+//                that one launch scores the rows of many sequences.
 #pragma once
 #include "common.cuh"
 
 namespace dsa {
 
-enum { kModeScores = 0, kModeDecode = 1 };
+enum { kModeScores = 0, kModeDecode = 1, kModeSegments = 2 };
+
+// kModeSegments: one run of consecutive query rows of one sequence
+struct IndexerSeg {
+  long long q_row0;     // row of q_I / w / q_scale holding the run's first query row
+  long long key_row0;   // row of k_I / k_scale holding key 0 of the sequence
+  long long out_base;   // score offset of (first query row, key 0)
+  int pos0;             // position of the first query row in its sequence
+  int n_rows;           // query rows of the run
+  int S;                // keys the run sees (pos0 + n_rows)
+  int ld;               // row stride of the run's scores
+  int nsplit;           // key-range splits per query block
+  int item0;            // first work item of the run
+};
 
 struct IndexerParams {
   const float* w;          // [T, H_I]
@@ -47,6 +63,8 @@ struct IndexerParams {
   const long long* cache_off;  // kModeDecode: [B] first cache row of each sequence
   const int* len1;             // kModeDecode: [B] keys of each sequence after the append (0: skip it)
   const long long* score_off;  // kModeDecode: [B] start of each sequence's score row
+  const IndexerSeg* segs;      // kModeSegments: [n_segs]
+  int n_segs;
   const int* page_table;       // kModeDecode, paged caches: [B, max_pages] page of each 'page_rows' positions
   int max_pages, page_rows;    // (page_rows a multiple of 128, so that a key tile lies in one page)
 };
@@ -61,6 +79,7 @@ struct IndexerItem {
   const int* pages;   // paged decode caches: the sequence's page-table row, else null
   int page_rows;
   long long out_base; // output offset of (first row, key 0)
+  long long ld;       // row stride of the scores (kModeScores, kModeSegments)
 };
 
 // tensor-map row of key tile*128 + i of an item (i < 128)
@@ -87,7 +106,7 @@ struct IndexerCfg {
   static constexpr int OFF_BAR = 0;                  // barriers + misc (2 KB)
   static constexpr int OFF_PREFIX = 2048;            // decode: per-sequence item prefix, key counts, cache offsets
   static constexpr int DEC_BYTES = 4 * (kMaxDecodeSeqs + 1) + 4 * kMaxDecodeSeqs + 8 * kMaxDecodeSeqs + 8;
-  static constexpr int OFF_W = ((OFF_PREFIX + (MODE == kModeDecode ? DEC_BYTES : 0) + 15) / 16) * 16;
+  static constexpr int OFF_W = ((OFF_PREFIX + (MODE != kModeScores ? DEC_BYTES : 0) + 15) / 16) * 16;
   static constexpr int W_FLOATS = TOK * H_I;
   static constexpr int OFF_Q = ((OFF_W + QBUF * W_FLOATS * 4 + ALIGN - 1) / ALIGN) * ALIGN;
   static constexpr int OFF_K = OFF_Q + QBUF * NG * GBYTES;
@@ -143,6 +162,29 @@ __device__ __forceinline__ IndexerItem indexer_item(const IndexerParams& p, int 
     it.tile0 = sp * p.split_tiles;
     it.tile1 = min(it.tile0 + p.split_tiles, ntiles);
     it.out_base = static_cast<long long>(it.q_row0) * p.ld;
+    it.ld = p.ld;
+  } else if constexpr (MODE == kModeSegments) {
+    // binary search: prefix[sg] <= i < prefix[sg + 1] (prefix[sg] = the segment's first item)
+    int lo = 0, hi = p.n_segs - 1;
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (prefix[mid] <= i) lo = mid; else hi = mid - 1;
+    }
+    const IndexerSeg sg = p.segs[lo];
+    const int li = i - prefix[lo];
+    const int qb = li / sg.nsplit, sp = li % sg.nsplit;
+    it.q_row0 = static_cast<int>(sg.q_row0) + qb * TOK;
+    it.n_tok = min(TOK, sg.n_rows - qb * TOK);
+    it.pos0 = sg.pos0 + qb * TOK;
+    it.n_keys = sg.S;
+    it.key_row0 = sg.key_row0;
+    it.pages = nullptr;
+    it.page_rows = 0;
+    const int ntiles = (sg.S + 127) / 128;
+    it.tile0 = sp * p.split_tiles;
+    it.tile1 = min(it.tile0 + p.split_tiles, ntiles);
+    it.out_base = sg.out_base + static_cast<long long>(qb * TOK) * sg.ld;
+    it.ld = sg.ld;
   } else {
     // item i is sequence b = i, clipped to the CTA's tile range (prefix[b] = its first tile in the joint order)
     const int b = i;
@@ -159,6 +201,7 @@ __device__ __forceinline__ IndexerItem indexer_item(const IndexerParams& p, int 
     it.tile0 = max(tr.lo, prefix[b]) - prefix[b];
     it.tile1 = min(tr.hi, prefix[b + 1]) - prefix[b];
     it.out_base = p.score_off[b];
+    it.ld = 0;
   }
   return it;
 }
@@ -206,6 +249,8 @@ indexer_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     *abort_flag = 0;
     fence_mbar_init();
   }
+  pdl_allow_next();
+  pdl_wait();
   if constexpr (MODE == kModeDecode) {
     // per sequence: keys n_b + 1, cache offset and key tiles, loaded by all threads in parallel; then an
     // exclusive scan of the tile counts by warp 0 (tiles of sequence b are prefix[b] .. prefix[b + 1] - 1 in the
@@ -241,6 +286,9 @@ indexer_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         *reinterpret_cast<int*>(smem + Bars::OFF_NITEMS) = carry;
       }
     }
+  }
+  if constexpr (MODE == kModeSegments) {
+    for (int sgi = threadIdx.x; sgi < p.n_segs; sgi += blockDim.x) prefix[sgi] = p.segs[sgi].item0;
   }
   if (warp == 0 && lane == 0) { prefetch_tmap(&tm_q); prefetch_tmap(&tm_k); }
   if (warp == 1) {
@@ -411,12 +459,12 @@ indexer_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
           if (g * NT >= it.n_tok) break;
           const int tok0 = g * NT + half * (CPT / H_I > 0 ? CPT / H_I : 0);  // first row of this thread
           if (!group_active<NT>(it, tile, g)) {
-            if constexpr (MODE == kModeScores) {
+            if constexpr (MODE != kModeDecode) {
               if (key_ok) {
 #pragma unroll
                 for (int tk = 0; tk < TOKS; ++tk) {
                   const int r = tok0 + tk;
-                  if (r < it.n_tok) p.scores[it.out_base + static_cast<long long>(r) * p.ld + s] = -INFINITY;
+                  if (r < it.n_tok) p.scores[it.out_base + static_cast<long long>(r) * it.ld + s] = -INFINITY;
                 }
               }
             }
@@ -501,8 +549,8 @@ indexer_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
 #pragma unroll
               for (int q = 0; q < P; ++q) sc += acc[tk][q];
               sc *= kscale;
-              if constexpr (MODE == kModeScores) {
-                p.scores[it.out_base + static_cast<long long>(r) * p.ld + s] = (s <= it.pos0 + r) ? sc : -INFINITY;
+              if constexpr (MODE != kModeDecode) {
+                p.scores[it.out_base + static_cast<long long>(r) * it.ld + s] = (s <= it.pos0 + r) ? sc : -INFINITY;
               } else {
                 p.scores[it.out_base + s] = sc;
               }

@@ -250,6 +250,9 @@ sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
   cluster_sync();        // both CTAs' barriers are initialised before any remote arrive
   tc_fence_after();
   const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(smem + OFF_TMEM);
+  // the set-up above touches no global memory; from here on the predecessor's results are read
+  pdl_allow_next();
+  pdl_wait();
 
   if (warp == 0) {
     // ===================================================================== loader

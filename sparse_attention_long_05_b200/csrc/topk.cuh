@@ -222,6 +222,8 @@ __global__ void __launch_bounds__(NT) topk_rows_kernel(const TopkParams p) {
   extern __shared__ __align__(16) uint8_t topk_smem_raw[];
   TopkSmem<NT>& sm = *reinterpret_cast<TopkSmem<NT>*>(topk_smem_raw);
 
+  pdl_allow_next();
+  pdl_wait();
   const int r = blockIdx.x;
   if (r >= p.rows) return;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;

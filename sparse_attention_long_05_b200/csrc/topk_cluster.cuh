@@ -124,6 +124,8 @@ __global__ void __cluster_dims__(kTkcCluster, 1, 1) __launch_bounds__(kTkcThread
   extern __shared__ __align__(16) uint8_t tkc_smem_raw[];
   TkcSmem& sm = *reinterpret_cast<TkcSmem*>(tkc_smem_raw);
   constexpr int W = TkcSmem::W;
+  pdl_allow_next();
+  pdl_wait();
   const int r = blockIdx.x / kTkcCluster;
   const int rank = static_cast<int>(cluster_rank());
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;

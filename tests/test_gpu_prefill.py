@@ -123,11 +123,9 @@ def test_varlen_batch_matches_each_sequence_alone(dsa):
     idx, out, lse = dsa.dsa_forward_prefill_varlen(cu, cat["q_idx"], None, cat["k_idx"], None, cat["w"], cat["q"],
                                                    cat["c"], base.k, base.scale)
     assert dsa.dsa_get_device_status() == 0
-    # the row offsets; per non-empty sequence a top-k for its rows t < k, and for the one longer than k an indexer
-    # and a top-k for the rest; one attention launch
-    blocks = [dsa.prefill_blocks(n, base.k) for n in lens if n]
-    assert [len(b) for b in blocks] == [1, 2, 1]
-    assert dsa.dsa_launch_count() - n0 == 1 + (1 + 3 + 1) + 1
+    # the batch is one group: the attention's row offsets, one indexer launch over the scored rows (t >= k) of every
+    # sequence, the top-k's row offsets and lengths, one top-k launch over every row, one attention launch
+    assert dsa.dsa_launch_count() - n0 == 5
     for b, (cfg, sd, n) in enumerate(zip(cfgs, seeds, lens)):
         if not n:
             continue
@@ -147,3 +145,30 @@ def _forward_full(dsa, cfg, seed):
                                             x["c"], cfg.k, cfg.scale)
     assert dsa.dsa_get_device_status() == 0
     return idx, out, lse
+
+
+def test_varlen_many_sequences_one_select(dsa):
+    # 24 sequences of 100..3000 tokens (integer mode, k = 2048): every sequence's rows match its own prefill bit for
+    # bit, while the select of the whole batch is one indexer launch and one top-k launch
+    base = G.PREFILL_CONFIGS["prefill_8k"]
+    rng = np.random.default_rng(39)
+    lens = [int(x) for x in rng.integers(100, 3001, size=24)]
+    lens[5] = 0
+    seeds = [100 + b for b in range(len(lens))]
+    cfgs = [dataclasses.replace(base, name=f"varlen_{n}", L=max(n, 1)) for n in lens]
+    parts = [prefill_device(cfg, sd) for cfg, sd, n in zip(cfgs, seeds, lens) if n]
+    cat = {key: torch.cat([x[key] for x in parts]) for key in ("q_idx", "k_idx", "w", "q", "c")}
+    cu = np.concatenate([[0], np.cumsum(lens)]).tolist()
+    n0 = dsa.dsa_launch_count()
+    idx, out, lse = dsa.dsa_forward_prefill_varlen(cu, cat["q_idx"], None, cat["k_idx"], None, cat["w"], cat["q"],
+                                                   cat["c"], base.k, base.scale)
+    assert dsa.dsa_get_device_status() == 0
+    assert dsa.dsa_launch_count() - n0 == 5
+    for b, (cfg, sd, n) in enumerate(zip(cfgs, seeds, lens)):
+        if not n:
+            continue
+        i1, o1, l1 = _forward_full(dsa, cfg, sd)
+        r0, r1 = cu[b], cu[b + 1]
+        assert torch.equal(idx[r0:r1], i1), f"sequence {b}: selection"
+        assert torch.equal(out[r0:r1], o1), f"sequence {b}: output"
+        assert torch.equal(lse[r0:r1], l1), f"sequence {b}: lse"

@@ -183,6 +183,29 @@ DSA_API dsa_status_t dsa_forward_prefill(const uint8_t* q_idx, const float* q_sc
                                  int L, int H_I, int d_I, int H, int k, float scale, int32_t* idx_out,
                                  uint16_t* out, float* lse, void* ws, size_t ws_bytes, void* stream);
 
+/* Device workspace bytes of dsa_forward_prefill_host: the prefill's workspace plus device copies of every input and
+ * output. */
+DSA_API size_t dsa_prefill_host_workspace_size(int L, int H_I, int d_I, int H, int k);
+
+/*
+ * dsa_forward_prefill with every input and output in HOST memory (steps 1-3 for one causal sequence, as
+ * dsa_forward_prefill; same arguments, HOST pointers; lse and idx_out may be NULL).  The call moves the data
+ * itself and overlaps the transfers with the kernels: the indexer's inputs are copied first; then, in
+ * 8 chunks of rows, each chunk's selection runs while later queries are still arriving, each chunk's attention
+ * starts once its queries have landed, and its results go back while the next chunk computes.  Host-to-device
+ * and device-to-host copies run on two copy streams of the library's own (created once per device on first
+ * use), so both directions of the host link are busy at once.  For the copies to be asynchronous the host
+ * buffers must be page-locked (cudaHostAlloc / cudaHostRegister); pageable buffers work but serialise.
+ *   ws: DEVICE workspace of dsa_prefill_host_workspace_size() bytes (it holds the device copies).
+ * Everything is enqueued on `stream`: when `stream` reaches the end of the call's work, the host outputs hold the
+ * results.  The host inputs must stay unchanged and the host outputs unread until then.
+ */
+DSA_API dsa_status_t dsa_forward_prefill_host(const uint8_t* q_idx, const float* q_scale, const uint8_t* k_idx,
+                                              const float* k_scale, const float* w, const uint16_t* q,
+                                              const uint16_t* c, int L, int H_I, int d_I, int H, int k, float scale,
+                                              int32_t* idx_out, uint16_t* out, float* lse, void* ws, size_t ws_bytes,
+                                              void* stream);
+
 /* Workspace bytes of dsa_forward_prefill_rows for the rows [row0, row0 + nrows) of a sequence. */
 DSA_API size_t dsa_prefill_rows_workspace_size(int row0, int nrows, int H_I, int d_I, int H, int k);
 

@@ -13,6 +13,7 @@ from ._lib import (  # noqa: F401
     dsa_forward_decode,
     dsa_forward_decode_paged,
     dsa_forward_prefill,
+    dsa_forward_prefill_host,
     dsa_forward_prefill_kl,
     dsa_forward_prefill_rows,
     dsa_forward_prefill_varlen,
@@ -22,6 +23,7 @@ from ._lib import (  # noqa: F401
     dsa_launch_count,
     dsa_num_sms,
     dsa_prefill_block_rows,
+    dsa_prefill_host_workspace_size,
     dsa_prefill_kl_workspace_size,
     dsa_prefill_rows_workspace_size,
     dsa_prefill_select,

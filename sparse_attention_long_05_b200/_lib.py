@@ -37,6 +37,9 @@ SIGNATURES = {
     "dsa_prefill_workspace_size": (_SZ, [_I, _I, _I, _I, _I]),
     "dsa_prefill_select": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _P, _P, _SZ, _P]),
     "dsa_forward_prefill": (_I, [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _P, _P, _P, _P, _SZ, _P]),
+    "dsa_prefill_host_workspace_size": (_SZ, [_I, _I, _I, _I, _I]),
+    "dsa_forward_prefill_host": (_I, [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _P, _P, _P, _P, _SZ,
+                                      _P]),
     "dsa_prefill_rows_workspace_size": (_SZ, [_I, _I, _I, _I, _I, _I]),
     "dsa_forward_prefill_rows": (_I, [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _P, _P, _P, _P, _SZ,
                                       _P]),
@@ -242,6 +245,32 @@ def dsa_forward_prefill(q_idx, q_scale, k_idx, k_scale, w, q, c, k: int, scale: 
     _check("dsa_forward_prefill", _lib.dsa_forward_prefill(
         _ptr(q_idx), _ptr(q_scale), _ptr(k_idx), _ptr(k_scale), _ptr(w), _ptr(q), _ptr(c), L, H_I, d_I, H, k,
         float(scale), _ptr(idx_out), _ptr(out), _ptr(lse), _ptr(ws), ws.numel(), _stream(stream)))
+    return idx_out, out, lse
+
+
+def _hptr(t):
+    if t is None:
+        return None
+    if t.is_cuda:
+        raise ValueError("dsa_forward_prefill_host takes host tensors")
+    if not t.is_contiguous():
+        raise ValueError("libdsa takes contiguous tensors")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def dsa_prefill_host_workspace_size(L: int, H_I: int, d_I: int, H: int, k: int) -> int:
+    return int(_lib.dsa_prefill_host_workspace_size(L, H_I, d_I, H, k))
+
+
+def dsa_forward_prefill_host(q_idx, q_scale, k_idx, k_scale, w, q, c, k: int, scale: float, idx_out, out, lse, ws,
+                             stream=None):
+    """dsa_forward_prefill over HOST tensors (page-locked for overlapped copies): fills idx_out, out and lse (host
+    tensors, the latter two may be None); ws is a device workspace of dsa_prefill_host_workspace_size bytes."""
+    L, H_I, d_I = q_idx.shape
+    H = q.shape[1]
+    _check("dsa_forward_prefill_host", _lib.dsa_forward_prefill_host(
+        _hptr(q_idx), _hptr(q_scale), _hptr(k_idx), _hptr(k_scale), _hptr(w), _hptr(q), _hptr(c), L, H_I, d_I, H, k,
+        float(scale), _hptr(idx_out), _hptr(out), _hptr(lse), _ptr(ws), ws.numel(), _stream(stream)))
     return idx_out, out, lse
 
 

@@ -742,6 +742,148 @@ dsa_status_t dsa_forward_prefill(const uint8_t* q_idx, const float* q_scale, con
   return run_mla(q, c, L, idx, nullptr, L, H, k, scale, out, lse, st, kMlaCausal);
 }
 
+// ------------------------------------------------------------------------------------------ host-buffer prefill
+namespace {
+constexpr int kHostChunks = 8;          // token chunks of the host-buffer prefill's pipeline
+
+// The host-buffer prefill's device copies, laid out after the prefill workspace.
+struct HostPrefillLayout {
+  size_t ws, q_idx, q_scale, k_idx, k_scale, w, q, c, out, lse, total;
+};
+HostPrefillLayout host_prefill_layout(int L, int H_I, int d_I, int H, int k) {
+  HostPrefillLayout lo{};
+  size_t at = dsa_prefill_workspace_size(L, H_I, d_I, H, k);
+  auto take = [&](size_t bytes) { const size_t o = at; at += align_up(bytes, 256); return o; };
+  lo.ws = 0;
+  lo.q_idx = take(size_t(L) * H_I * d_I);
+  lo.q_scale = take(size_t(L) * 4);
+  lo.k_idx = take(size_t(L) * d_I);
+  lo.k_scale = take(size_t(L) * 4);
+  lo.w = take(size_t(L) * H_I * 4);
+  lo.q = take(size_t(L) * H * 576 * 2);
+  lo.c = take(size_t(L) * 576 * 2);
+  lo.out = take(size_t(L) * H * 512 * 2);
+  lo.lse = take(size_t(L) * H * 4);
+  lo.total = at;
+  return lo;
+}
+
+// One copy stream per direction and device, created on first use (the call allocates no memory).
+struct CopyStreams {
+  cudaStream_t h2d = nullptr, d2h = nullptr;
+};
+CopyStreams g_copy_streams[64];
+std::mutex g_copy_mutex;
+
+dsa_status_t copy_streams(CopyStreams* out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return DSA_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_copy_mutex);
+  CopyStreams& cs = g_copy_streams[dev];
+  if (!cs.h2d && cudaStreamCreateWithFlags(&cs.h2d, cudaStreamNonBlocking) != cudaSuccess) return DSA_ERR_CUDA;
+  if (!cs.d2h && cudaStreamCreateWithFlags(&cs.d2h, cudaStreamNonBlocking) != cudaSuccess) return DSA_ERR_CUDA;
+  *out = cs;
+  return DSA_OK;
+}
+}  // namespace
+
+size_t dsa_prefill_host_workspace_size(int L, int H_I, int d_I, int H, int k) {
+  if (L <= 0 || k <= 0 || H <= 0 || !indexer_shape_ok(H_I, d_I)) return 0;
+  return host_prefill_layout(L, H_I, d_I, H, k).total;
+}
+
+dsa_status_t dsa_forward_prefill_host(const uint8_t* q_idx, const float* q_scale, const uint8_t* k_idx,
+                                      const float* k_scale, const float* w, const uint16_t* q, const uint16_t* c,
+                                      int L, int H_I, int d_I, int H, int k, float scale, int32_t* idx_out,
+                                      uint16_t* out, float* lse, void* ws, size_t ws_bytes, void* stream) {
+  if (L <= 0 || H <= 0 || k <= 0 || !q_idx || !k_idx || !w || !q || !c || !out) return DSA_ERR_INVALID_ARG;
+  if (!indexer_shape_ok(H_I, d_I) || H > 128 || !mla_k_ok(k)) return DSA_ERR_UNSUPPORTED_SHAPE;
+  if (!ws || ws_bytes < dsa_prefill_host_workspace_size(L, H_I, d_I, H, k)) return DSA_ERR_WORKSPACE;
+  CopyStreams cs;
+  dsa_status_t e = copy_streams(&cs);
+  if (e != DSA_OK) return e;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const HostPrefillLayout lo = host_prefill_layout(L, H_I, d_I, H, k);
+  char* d = static_cast<char*>(ws);
+  uint8_t* dq_idx = reinterpret_cast<uint8_t*>(d + lo.q_idx);
+  float* dq_scale = q_scale ? reinterpret_cast<float*>(d + lo.q_scale) : nullptr;
+  uint8_t* dk_idx = reinterpret_cast<uint8_t*>(d + lo.k_idx);
+  float* dk_scale = k_scale ? reinterpret_cast<float*>(d + lo.k_scale) : nullptr;
+  float* dw = reinterpret_cast<float*>(d + lo.w);
+  uint16_t* dq = reinterpret_cast<uint16_t*>(d + lo.q);
+  uint16_t* dc = reinterpret_cast<uint16_t*>(d + lo.c);
+  uint16_t* dout = reinterpret_cast<uint16_t*>(d + lo.out);
+  float* dlse = reinterpret_cast<float*>(d + lo.lse);
+  float* sc = reinterpret_cast<float*>(d);
+  int32_t* didx = reinterpret_cast<int32_t*>(d + align_up(prefill_chunk_rows(L) * size_t(L) * 4, 256));
+  // events: start, indexer inputs landed, per chunk its queries landed and its attention done, all copies back
+  constexpr int NE = 2 + 2 * kHostChunks + 1;
+  cudaEvent_t ev[NE] = {};
+  for (int i = 0; i < NE; ++i)
+    if (cudaEventCreateWithFlags(&ev[i], cudaEventDisableTiming) != cudaSuccess) {
+      for (int j = 0; j < i; ++j) cudaEventDestroy(ev[j]);
+      return DSA_ERR_CUDA;
+    }
+  cudaEvent_t& ev_start = ev[0];
+  cudaEvent_t& ev_inputs = ev[1];
+  cudaEvent_t* ev_q = ev + 2;
+  cudaEvent_t* ev_att = ev + 2 + kHostChunks;
+  cudaEvent_t& ev_done = ev[NE - 1];
+  auto h2d = [&](void* dst, const void* src, size_t bytes) {
+    return !src || cudaMemcpyAsync(dst, src, bytes, cudaMemcpyHostToDevice, cs.h2d) == cudaSuccess;
+  };
+  auto d2h = [&](void* dst, const void* src, size_t bytes) {
+    return !dst || cudaMemcpyAsync(dst, src, bytes, cudaMemcpyDeviceToHost, cs.d2h) == cudaSuccess;
+  };
+  const size_t qrow = size_t(H) * 576 * 2, orow = size_t(H) * 512 * 2;
+  bool ok = cudaEventRecord(ev_start, st) == cudaSuccess && cudaStreamWaitEvent(cs.h2d, ev_start, 0) == cudaSuccess &&
+            cudaStreamWaitEvent(cs.d2h, ev_start, 0) == cudaSuccess;
+  // host -> device: the indexer's inputs first, then c and the queries chunk by chunk
+  ok = ok && h2d(dk_idx, k_idx, size_t(L) * d_I) && h2d(dk_scale, k_scale, size_t(L) * 4) &&
+       h2d(dq_idx, q_idx, size_t(L) * H_I * d_I) && h2d(dq_scale, q_scale, size_t(L) * 4) &&
+       h2d(dw, w, size_t(L) * H_I * 4) && cudaEventRecord(ev_inputs, cs.h2d) == cudaSuccess &&
+       h2d(dc, c, size_t(L) * 576 * 2);
+  int t0[kHostChunks + 1];
+  for (int j = 0; j <= kHostChunks; ++j) t0[j] = static_cast<int>((static_cast<long long>(L) * j) / kHostChunks);
+  for (int j = 0; j < kHostChunks && ok; ++j) {
+    ok = h2d(reinterpret_cast<char*>(dq) + t0[j] * qrow, reinterpret_cast<const char*>(q) + t0[j] * qrow,
+             size_t(t0[j + 1] - t0[j]) * qrow) &&
+         cudaEventRecord(ev_q[j], cs.h2d) == cudaSuccess;
+  }
+  // compute, chunk by chunk: the chunk's rows' selection, then (once its queries landed) its attention
+  ok = ok && cudaStreamWaitEvent(st, ev_inputs, 0) == cudaSuccess;
+  for (int j = 0; j < kHostChunks && ok && e == DSA_OK; ++j) {
+    const int n = t0[j + 1] - t0[j];
+    if (n == 0) {
+      ok = cudaEventRecord(ev_att[j], st) == cudaSuccess;
+      continue;
+    }
+    e = select_rows(dq_idx + size_t(t0[j]) * H_I * d_I, dq_scale ? dq_scale + t0[j] : nullptr, dk_idx, dk_scale,
+                    dw + size_t(t0[j]) * H_I, H_I, d_I, k, t0[j], t0[j + 1], didx + size_t(t0[j]) * k, sc,
+                    prefill_chunk_rows(L), st);
+    if (e != DSA_OK) break;
+    ok = cudaStreamWaitEvent(st, ev_q[j], 0) == cudaSuccess;
+    if (!ok) break;
+    e = run_mla(reinterpret_cast<const uint16_t*>(reinterpret_cast<const char*>(dq) + t0[j] * qrow), dc, L,
+                didx + size_t(t0[j]) * k, nullptr, n, H, k, scale,
+                reinterpret_cast<uint16_t*>(reinterpret_cast<char*>(dout) + t0[j] * orow), dlse + size_t(t0[j]) * H,
+                st, kMlaCausal, nullptr, nullptr, 0, 0, t0[j]);
+    if (e != DSA_OK) break;
+    ok = cudaEventRecord(ev_att[j], st) == cudaSuccess;
+    // device -> host of the chunk's results, on the other copy stream
+    ok = ok && cudaStreamWaitEvent(cs.d2h, ev_att[j], 0) == cudaSuccess &&
+         d2h(reinterpret_cast<char*>(out) + t0[j] * orow, reinterpret_cast<char*>(dout) + t0[j] * orow,
+             size_t(n) * orow) &&
+         d2h(lse ? lse + size_t(t0[j]) * H : nullptr, dlse + size_t(t0[j]) * H, size_t(n) * H * 4) &&
+         d2h(idx_out ? idx_out + size_t(t0[j]) * k : nullptr, didx + size_t(t0[j]) * k, size_t(n) * k * 4);
+  }
+  // the caller's stream ends when every copy back has landed
+  ok = ok && cudaEventRecord(ev_done, cs.d2h) == cudaSuccess && cudaStreamWaitEvent(st, ev_done, 0) == cudaSuccess;
+  for (int i = 0; i < NE; ++i) cudaEventDestroy(ev[i]);     // released once the work that uses them completes
+  if (e != DSA_OK) return e;
+  return ok ? DSA_OK : DSA_ERR_CUDA;
+}
+
 size_t dsa_prefill_varlen_workspace_size(int nseq, int64_t total, int max_len, int H_I, int d_I, int H, int k) {
   (void)H_I; (void)d_I; (void)H;
   if (nseq <= 0 || total <= 0 || max_len <= 0 || k <= 0) return 0;

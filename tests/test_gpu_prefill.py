@@ -172,3 +172,26 @@ def test_varlen_many_sequences_one_select(dsa):
         assert torch.equal(idx[r0:r1], i1), f"sequence {b}: selection"
         assert torch.equal(out[r0:r1], o1), f"sequence {b}: output"
         assert torch.equal(lse[r0:r1], l1), f"sequence {b}: lse"
+
+
+@pytest.mark.parametrize("name,L", [("prefill_8k", 8192), ("prefill_32k", 5000), ("tiny_1k", 1024)])
+def test_host_buffer_prefill_identical(dsa, name, L):
+    # dsa_forward_prefill_host: inputs in page-locked host memory, results copied back by the call, the transfers
+    # overlapped with the kernels chunk by chunk; every result equals dsa_forward_prefill's bit for bit
+    cfg = dataclasses.replace(G.PREFILL_CONFIGS[name], L=L)
+    x = prefill_device(cfg, 81)
+    idx, out, lse = dsa.dsa_forward_prefill(x["q_idx"], x["q_scale"], x["k_idx"], x["k_scale"], x["w"], x["q"],
+                                            x["c"], cfg.k, cfg.scale)
+    host = {n: (None if t is None else t.cpu().pin_memory()) for n, t in x.items()}
+    h_idx = torch.empty((L, cfg.k), dtype=torch.int32, pin_memory=True)
+    h_out = torch.empty((L, cfg.H, 512), dtype=torch.bfloat16, pin_memory=True)
+    h_lse = torch.empty((L, cfg.H), dtype=torch.float32, pin_memory=True)
+    ws = torch.empty((dsa.dsa_prefill_host_workspace_size(L, cfg.H_I, cfg.d_I, cfg.H, cfg.k),), dtype=torch.uint8,
+                     device="cuda")
+    dsa.dsa_forward_prefill_host(host["q_idx"], host["q_scale"], host["k_idx"], host["k_scale"], host["w"], host["q"],
+                                 host["c"], cfg.k, cfg.scale, h_idx, h_out, h_lse, ws)
+    torch.cuda.current_stream().synchronize()
+    assert dsa.dsa_get_device_status() == 0
+    assert torch.equal(h_idx, idx.cpu())
+    assert torch.equal(h_out, out.cpu())
+    assert torch.equal(h_lse, lse.cpu())

@@ -43,7 +43,7 @@ def test_decode_dense_tokens_identical_to_gathered(dsa):
     # Short contexts (n_b + 1 <= k) take the dense path in decode too; each sequence's output equals the gathered
     # path over its own cache rows.  The cache rows after each sequence's entries are filled with NaN: the dense
     # path never lets them into a tile.
-    cfg = G.DecodeConfig("dense_dec", B=6, len_lo=30, len_hi=2100, steps=2)
+    cfg = G.DecodeConfig("dense_dec", B=6, len_lo=30, len_hi=4000, steps=2)   # 3 of the 6 contexts are below k
     seed = 52
     cache = G.decode_fill_cache(cfg, seed, device="cuda")
     lens, offs = cache["lens"], cache["offs"]

@@ -80,17 +80,23 @@ __device__ __forceinline__ uint32_t radix_select(Each each, uint32_t prefix, uin
       if ((key & mask) == prefix) atomicAdd(&sm.hist[warp][(key >> shift) & 255], 1u);
     });
     __syncthreads();
+    // totals over the warps, one bin per thread (the top-11-bit histogram is no longer needed: its first 256 entries
+    // hold the totals)
+    for (int b = tid; b < 256; b += NT) {
+      uint32_t c = 0;
+#pragma unroll
+      for (int w = 0; w < TopkSmem<NT>::W; ++w) c += sm.hist[w][b];
+      sm.bins[b] = c;
+    }
+    __syncthreads();
     if (warp == 0) {
-      // lane l owns bins 255-8l .. 248-8l (descending); totals over warps
+      // lane l owns bins 255-8l .. 248-8l (descending)
       uint32_t cnt[8];
       uint32_t tot = 0;
 #pragma unroll
       for (int j = 0; j < 8; ++j) {
-        const int bin = 255 - 8 * lane - j;
-        uint32_t c = 0;
-        for (int w = 0; w < TopkSmem<NT>::W; ++w) c += sm.hist[w][bin];
-        cnt[j] = c;
-        tot += c;
+        cnt[j] = sm.bins[255 - 8 * lane - j];
+        tot += cnt[j];
       }
       uint32_t incl = tot;
 #pragma unroll
@@ -218,7 +224,7 @@ __device__ __forceinline__ void topk_collect_vec(const float* x, int n, uint32_t
 }
 
 template <int NT>
-__global__ void __launch_bounds__(NT) topk_rows_kernel(const TopkParams p) {
+__global__ void __launch_bounds__(NT, 2) topk_rows_kernel(const TopkParams p) {
   extern __shared__ __align__(16) uint8_t topk_smem_raw[];
   TopkSmem<NT>& sm = *reinterpret_cast<TopkSmem<NT>*>(topk_smem_raw);
 

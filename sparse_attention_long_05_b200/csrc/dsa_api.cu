@@ -429,13 +429,13 @@ dsa_status_t run_mla(const uint16_t* q, const uint16_t* c, long long S, const in
   p.k = k;
   p.S = S;
   p.scale_log2 = scale * 1.4426950408889634f;
-  if (set_smem(sparse_mla_kernel, mla::SMEM) != cudaSuccess) return DSA_ERR_CUDA;
+  auto kern = kl_out ? sparse_mla_kernel<true> : sparse_mla_kernel<false>;
+  if (set_smem(kern, mla::SMEM) != cudaSuccess) return DSA_ERR_CUDA;
   // KL mode: every CTA takes tokens of its own (the grid still comes in pairs, the kernel's cluster shape)
   const int per_cluster = kl_out ? 2 : 1;
   int clusters = num_sms() / 2;
   if (clusters > (T + per_cluster - 1) / per_cluster) clusters = (T + per_cluster - 1) / per_cluster;
-  if (launch_pdl(sparse_mla_kernel, dim3(2 * clusters), dim3(mla::THREADS), mla::SMEM, st, tq, tc, tcd, p) !=
-      cudaSuccess)
+  if (launch_pdl(kern, dim3(2 * clusters), dim3(mla::THREADS), mla::SMEM, st, tq, tc, tcd, p) != cudaSuccess)
     return DSA_ERR_CUDA;
   return last_launch_status();
 }

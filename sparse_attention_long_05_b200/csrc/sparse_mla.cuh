@@ -190,6 +190,9 @@ __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, volatil
   return __all_sync(0xffffffffu, ok);
 }
 
+// KL selects the indexer-objective instantiation (p.kl_out set): a separate kernel, so that the attention's code
+// carries none of the objective's unrolled loops (the warps of the attention run from the instruction cache).
+template <bool KL>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(mla::THREADS, 1)
 sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_c,
                   const __grid_constant__ CUtensorMap tm_cd, const MlaParams p) {
@@ -202,7 +205,7 @@ sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + OFF_ABORT);
   const int warp = warp_id(), lane = lane_id();
   // 0 = score CTA, 1 = value CTA; in KL mode every CTA takes the score role on tokens of its own
-  const bool kl_mode = p.kl_out != nullptr;
+  constexpr bool kl_mode = KL;
   const uint32_t rank = kl_mode ? 0u : cluster_rank();
   const int cluster = kl_mode ? static_cast<int>(blockIdx.x) : static_cast<int>(blockIdx.x >> 1);
   const int nclusters = kl_mode ? static_cast<int>(gridDim.x) : static_cast<int>(gridDim.x >> 1);
@@ -291,8 +294,8 @@ sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     // fetches rows 4 rg .. 4 rg + 3 of the tile into its chunk cc; warp gw issues instructions
     // gw * per_warp .. + per_warp - 1, one per lane.  A dense token's full tiles are 64 contiguous rows: lane c
     // of gather warp 0 loads its chunk c as one 64 x 64 box, and the other warps arrive with no bytes.  Its
-    // last, partial tile is gathered, its masked slots reading rows of the token's own keys: the rows after
-    // the sequence's last key may be memory the caller never wrote, and a NaN there would survive the zero
+    // last, partial tile is gathered, its masked slots reading the token's last key row: the rows after the
+    // sequence's last key may be memory the caller never wrote, and a NaN there would survive the zero
     // probability in P . V.
     const int gw = (warp < 8) ? warp - 2 : warp - 6;
     const int cps = (rank == 0) ? SCH : VCH;               // chunks per stage
@@ -331,7 +334,7 @@ sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
 #pragma unroll
             for (int u = 0; u < 4; ++u) {
               const int pos = slot + u;
-              r[u] = static_cast<int>(nd > 0 ? mla_pos_row(p, t, base, pos < nd ? pos : pos % nd)
+              r[u] = static_cast<int>(nd > 0 ? mla_pos_row(p, t, base, pos < nd ? pos : nd - 1)
                                              : (pos < p.S ? pos : 0));
             }
           }
@@ -498,7 +501,7 @@ sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         }
       }
     }
-  } else if (kl_mode) {
+  } else if constexpr (KL) {
     // ===================================================================== KL objective (warps 4..7)
     // Per tile: each thread (one head) forms its head's probabilities of the tile's 64 keys from the logits and the
     // head's lse; a halving exchange sums them over the warp's 32 heads (lane l ends with keys 2 l, 2 l + 1), and

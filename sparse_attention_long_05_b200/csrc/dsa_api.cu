@@ -429,7 +429,13 @@ dsa_status_t run_mla(const uint16_t* q, const uint16_t* c, long long S, const in
   p.k = k;
   p.S = S;
   p.scale_log2 = scale * 1.4426950408889634f;
-  auto kern = kl_out ? sparse_mla_kernel<true> : sparse_mla_kernel<false>;
+  // the instantiation with exactly the features this launch uses
+  const bool dn = dense != kMlaSparse, pg = page_table != nullptr;
+  auto kern = kl_out ? (dn ? sparse_mla_kernel<true, true, false> : sparse_mla_kernel<true, false, false>)
+            : pg     ? sparse_mla_kernel<false, true, true>
+            : dn     ? sparse_mla_kernel<false, true, false>
+                     : sparse_mla_kernel<false, false, false>;
+  if (pg && !dn) return DSA_ERR_INVALID_ARG;      // paged caches only come with per-token key counts
   if (set_smem(kern, mla::SMEM) != cudaSuccess) return DSA_ERR_CUDA;
   // KL mode: every CTA takes tokens of its own (the grid still comes in pairs, the kernel's cluster shape)
   const int per_cluster = kl_out ? 2 : 1;
@@ -438,6 +444,25 @@ dsa_status_t run_mla(const uint16_t* q, const uint16_t* c, long long S, const in
   if (launch_pdl(kern, dim3(2 * clusters), dim3(mla::THREADS), mla::SMEM, st, tq, tc, tcd, p) != cudaSuccess)
     return DSA_ERR_CUDA;
   return last_launch_status();
+}
+
+// Causal rows [pos0, pos0 + T) of one sequence (row r at position pos0 + r, its keys from row 0 of c): the rows at
+// positions below k (every earlier key selected) run on the dense instantiation, the others on the gathered one.
+dsa_status_t run_mla_causal(const uint16_t* q, const uint16_t* c, long long S, const int* idx, int T, int H, int k,
+                            float scale, uint16_t* out, float* lse, cudaStream_t st, int pos0,
+                            const float* kl_lse = nullptr, const float* kl_scores = nullptr,
+                            float* kl_out = nullptr) {
+  const int nd = std::max(0, std::min(T, k - pos0));
+  dsa_status_t e = DSA_OK;
+  if (nd > 0)
+    e = run_mla(q, c, S, idx, nullptr, nd, H, k, scale, out, lse, st, kMlaCausal, nullptr, nullptr, 0, 0, pos0,
+                kl_lse, kl_scores, kl_out);
+  if (e != DSA_OK || nd == T) return e;
+  const size_t n = static_cast<size_t>(nd);
+  return run_mla(q + n * H * 576, c, S, idx + n * k, nullptr, T - nd, H, k, scale, out ? out + n * H * 512 : nullptr,
+                 lse ? lse + n * H : nullptr, st, kMlaSparse, nullptr, nullptr, 0, 0, 0,
+                 kl_lse ? kl_lse + n * H : nullptr, kl_scores ? kl_scores + n * k : nullptr,
+                 kl_out ? kl_out + n : nullptr);
 }
 
 bool mla_k_ok(int k) { return k >= 2 * mla::NK && k % mla::NK == 0 && k <= mla::KMAX; }
@@ -661,10 +686,9 @@ dsa_status_t dsa_forward_prefill_kl(const uint8_t* q_idx, const float* q_scale, 
   dsa_status_t e = select_rows(q_idx, q_scale, k_idx, k_scale, w, H_I, d_I, k, 0, L, idx, reinterpret_cast<float*>(wsb),
                                prefill_chunk_rows(L), st, sel);
   if (e != DSA_OK) return e;
-  e = run_mla(q, c, L, idx, nullptr, L, H, k, scale, out, lse_buf, st, kMlaCausal);
+  e = run_mla_causal(q, c, L, idx, L, H, k, scale, out, lse_buf, st, 0);
   if (e != DSA_OK) return e;
-  return run_mla(q, c, L, idx, nullptr, L, H, k, scale, nullptr, nullptr, st, kMlaCausal, nullptr, nullptr, 0, 0, 0,
-                 lse_buf, sel, kl);
+  return run_mla_causal(q, c, L, idx, L, H, k, scale, nullptr, nullptr, st, 0, lse_buf, sel, kl);
 }
 
 dsa_status_t dsa_sparse_mla_attn(const uint16_t* q, const uint16_t* c, int S, const int32_t* idx, int T, int H,
@@ -720,7 +744,7 @@ dsa_status_t dsa_forward_prefill_rows(const uint8_t* q_idx, const float* q_scale
   dsa_status_t e = select_rows(q_idx, q_scale, k_idx, k_scale, w, H_I, d_I, k, row0, S, idx, static_cast<float*>(ws),
                                prefill_chunk_rows(S), st);
   if (e != DSA_OK) return e;
-  return run_mla(q, c, S, idx, nullptr, nrows, H, k, scale, out, lse, st, kMlaCausal, nullptr, nullptr, 0, 0, row0);
+  return run_mla_causal(q, c, S, idx, nrows, H, k, scale, out, lse, st, row0);
 }
 
 dsa_status_t dsa_forward_prefill(const uint8_t* q_idx, const float* q_scale, const uint8_t* k_idx,
@@ -739,7 +763,7 @@ dsa_status_t dsa_forward_prefill(const uint8_t* q_idx, const float* q_scale, con
                                                       align_up(prefill_chunk_rows(L) * size_t(L) * 4, 256));
   dsa_status_t e = dsa_prefill_select(q_idx, q_scale, k_idx, k_scale, w, L, H_I, d_I, k, idx, ws, ws_bytes, stream);
   if (e != DSA_OK) return e;
-  return run_mla(q, c, L, idx, nullptr, L, H, k, scale, out, lse, st, kMlaCausal);
+  return run_mla_causal(q, c, L, idx, L, H, k, scale, out, lse, st, 0);
 }
 
 // ------------------------------------------------------------------------------------------ host-buffer prefill
@@ -864,10 +888,10 @@ dsa_status_t dsa_forward_prefill_host(const uint8_t* q_idx, const float* q_scale
     if (e != DSA_OK) break;
     ok = cudaStreamWaitEvent(st, ev_q[j], 0) == cudaSuccess;
     if (!ok) break;
-    e = run_mla(reinterpret_cast<const uint16_t*>(reinterpret_cast<const char*>(dq) + t0[j] * qrow), dc, L,
-                didx + size_t(t0[j]) * k, nullptr, n, H, k, scale,
-                reinterpret_cast<uint16_t*>(reinterpret_cast<char*>(dout) + t0[j] * orow), dlse + size_t(t0[j]) * H,
-                st, kMlaCausal, nullptr, nullptr, 0, 0, t0[j]);
+    e = run_mla_causal(reinterpret_cast<const uint16_t*>(reinterpret_cast<const char*>(dq) + t0[j] * qrow), dc, L,
+                       didx + size_t(t0[j]) * k, n, H, k, scale,
+                       reinterpret_cast<uint16_t*>(reinterpret_cast<char*>(dout) + t0[j] * orow),
+                       dlse + size_t(t0[j]) * H, st, t0[j]);
     if (e != DSA_OK) break;
     ok = cudaEventRecord(ev_att[j], st) == cudaSuccess;
     // device -> host of the chunk's results, on the other copy stream

@@ -136,35 +136,50 @@ static_assert(NS_S <= 16 && NS_V <= 16, "ring barrier slots");
 static_assert(SMEM <= 232448, "shared memory per CTA");
 }  // namespace mla
 
+// The kernel is instantiated per feature set (DENSE: the dense modes; PAGED: a page table; KL: the objective), so that
+// each launch runs code with none of the branches of the features it does not use: the attention's warps run from
+// the instruction cache, and code for an unused feature in their loops showed up as instruction-fetch stalls.
+
 // Row of c holding position `pos` (>= 0) of token t's keys: base + pos, or through the token's page-table row.
+template <bool PAGED>
 __device__ __forceinline__ long long mla_pos_row(const MlaParams& p, int t, long long base, long long pos) {
-  if (!p.page_table) return base + pos;
-  const int* pr = p.page_table + static_cast<long long>(t) * p.pt_stride;
-  return static_cast<long long>(pr[pos / p.page_rows]) * p.page_rows + pos % p.page_rows;
+  if constexpr (!PAGED) {
+    return base + pos;
+  } else {
+    const int* pr = p.page_table + static_cast<long long>(t) * p.pt_stride;
+    return static_cast<long long>(pr[pos / p.page_rows]) * p.page_rows + pos % p.page_rows;
+  }
 }
 // Whether selection entry e of token t names a row of c (an entry of -1 is padding; anything else outside the
 // token's keys is an error).
+template <bool PAGED>
 __device__ __forceinline__ bool mla_valid(const MlaParams& p, int t, int e, long long base) {
   if (e < 0) return false;
-  if (p.page_table && e >= static_cast<long long>(p.pt_stride) * p.page_rows) return false;
-  const long long r = mla_pos_row(p, t, base, e);
+  if (PAGED && e >= static_cast<long long>(p.pt_stride) * p.page_rows) return false;
+  const long long r = mla_pos_row<PAGED>(p, t, base, e);
   return r >= 0 && r < p.S;
 }
 // Row of c gathered for selection entry e (in slot `slot` of its token's k entries).  An empty or invalid entry is
 // masked out of the softmax but its stage still holds a row: it reads row `slot` (any row in [0, S) would do), so
 // that the padding of short rows spreads over many L2 lines instead of hammering one.
+template <bool PAGED>
 __device__ __forceinline__ long long mla_row(const MlaParams& p, int t, int e, long long base, int slot) {
-  const bool valid = mla_valid(p, t, e, base);
+  const bool valid = mla_valid<PAGED>(p, t, e, base);
   if (!valid && e != -1) raise_status(DSA_ERR_BAD_INDEX);
-  return valid ? mla_pos_row(p, t, base, e) : (slot < p.S ? slot : 0);
+  return valid ? mla_pos_row<PAGED>(p, t, base, e) : (slot < p.S ? slot : 0);
 }
 
 // Number of keys n_t of token t when it takes the dense path (n_t <= k), -1 when its index row is gathered.
+template <bool DENSE>
 __device__ __forceinline__ int mla_dense_keys(const MlaParams& p, int t, long long base) {
-  if (p.dense == kMlaSparse) return -1;
-  const long long n = (p.dense == kMlaCausal) ? static_cast<long long>(p.pos0) + t - base + 1 : p.n_keys[t];
-  if (n > p.k) return -1;
-  return n > 0 ? static_cast<int>(n) : 0;
+  if constexpr (!DENSE) {
+    return -1;
+  } else {
+    if (p.dense == kMlaSparse) return -1;
+    const long long n = (p.dense == kMlaCausal) ? static_cast<long long>(p.pos0) + t - base + 1 : p.n_keys[t];
+    if (n > p.k) return -1;
+    return n > 0 ? static_cast<int>(n) : 0;
+  }
 }
 // 64-key tiles of a token: k / 64 gathered tiles, or the tiles holding its n_t dense keys (at least two: the
 // score CTA's schedule of Q-chunk copies needs a second tile; a tile past n_t is wholly masked)
@@ -192,7 +207,7 @@ __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, volatil
 
 // KL selects the indexer-objective instantiation (p.kl_out set): a separate kernel, so that the attention's code
 // carries none of the objective's unrolled loops (the warps of the attention run from the instruction cache).
-template <bool KL>
+template <bool KL, bool DENSE, bool PAGED>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(mla::THREADS, 1)
 sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_c,
                   const __grid_constant__ CUtensorMap tm_cd, const MlaParams p) {
@@ -241,7 +256,7 @@ sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
   }
   if (warp == 0 && lane == 0) {
     prefetch_tmap(&tm_c);
-    if (p.dense != kMlaSparse) prefetch_tmap(&tm_cd);
+    if (DENSE && p.dense != kMlaSparse) prefetch_tmap(&tm_cd);
     if (rank == 0) prefetch_tmap(&tm_q);
   }
   if (warp == 1) {
@@ -316,7 +331,7 @@ sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
       if (!(ok = warp_wait(bar(B_IDX_FULL + is), (ti >> 1) & 1, abort_flag))) break;
       const int* ids = idx_s + is * KMAX;
       const long long base = p.row_off ? p.row_off[t] : 0;
-      const int nd = mla_dense_keys(p, t, base);
+      const int nd = mla_dense_keys<DENSE>(p, t, base);
       const int ntiles = mla_tiles(p, nd);
       for (int j = 0; j < ntiles && ok; ++j) {
         const bool full_dense = nd >= 0 && (j + 1) * NK <= nd;    // 64 contiguous rows of keys
@@ -326,15 +341,15 @@ sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
           const int slot = j * NK + 4 * rg;
           if (nd < 0) {
             const int4 e = reinterpret_cast<const int4*>(ids + j * NK)[rg];
-            r[0] = static_cast<int>(mla_row(p, t, e.x, base, slot));
-            r[1] = static_cast<int>(mla_row(p, t, e.y, base, slot + 1));
-            r[2] = static_cast<int>(mla_row(p, t, e.z, base, slot + 2));
-            r[3] = static_cast<int>(mla_row(p, t, e.w, base, slot + 3));
+            r[0] = static_cast<int>(mla_row<PAGED>(p, t, e.x, base, slot));
+            r[1] = static_cast<int>(mla_row<PAGED>(p, t, e.y, base, slot + 1));
+            r[2] = static_cast<int>(mla_row<PAGED>(p, t, e.z, base, slot + 2));
+            r[3] = static_cast<int>(mla_row<PAGED>(p, t, e.w, base, slot + 3));
           } else {
 #pragma unroll
             for (int u = 0; u < 4; ++u) {
               const int pos = slot + u;
-              r[u] = static_cast<int>(nd > 0 ? mla_pos_row(p, t, base, pos < nd ? pos : nd - 1)
+              r[u] = static_cast<int>(nd > 0 ? mla_pos_row<PAGED>(p, t, base, pos < nd ? pos : nd - 1)
                                              : (pos < p.S ? pos : 0));
             }
           }
@@ -357,7 +372,7 @@ sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                           64 * (s * cps + cc), r[0], r[1], r[2], r[3]);
           } else if (gw == 0 && lane < cps) {
             tma_load_2d(ring + st * sbytes + lane * CHUNK_BYTES, &tm_cd, bar(B_RING_FULL + st),
-                        64 * (s * cps + lane), static_cast<int>(mla_pos_row(p, t, base, j * NK)));
+                        64 * (s * cps + lane), static_cast<int>(mla_pos_row<PAGED>(p, t, base, j * NK)));
           }
           issued = true;
           last = rp;
@@ -406,7 +421,7 @@ sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         const bool has_next = t + nclusters < p.T;
         const uint32_t prev_tok = static_cast<uint32_t>((ti - 1) & 1);   // parity of the previous token's QTOK
         const int q_slot0 = (9 * ti) % QSLOTS;                          // tensor-memory slot of chunk 0
-        const int ntiles = mla_tiles(p, mla_dense_keys(p, t, p.row_off ? p.row_off[t] : 0));
+        const int ntiles = mla_tiles(p, mla_dense_keys<DENSE>(p, t, p.row_off ? p.row_off[t] : 0));
         for (int j = 0; j < ntiles && ok; ++j, ++g) {
           const int sb = g % NSB;
           if (j == 1 && has_next) {
@@ -468,7 +483,7 @@ sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     } else {
       constexpr uint32_t idesc = idesc_bf16(128, 256, true);
       for (int t = cluster; t < p.T && ok; t += nclusters, ++ti) {
-        const int ntiles = mla_tiles(p, mla_dense_keys(p, t, p.row_off ? p.row_off[t] : 0));
+        const int ntiles = mla_tiles(p, mla_dense_keys<DENSE>(p, t, p.row_off ? p.row_off[t] : 0));
         for (int j = 0; j < ntiles && ok; ++j, ++g) {
           const int pb = static_cast<int>(g % NPB);
           if (j == 0 && !(ok = warp_wait(bar(B_O_FREE), (ti & 1) ^ 1, abort_flag))) break;
@@ -520,7 +535,7 @@ sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
       if (!(ok = warp_wait(bar(B_IDX_FULL + is), (ti >> 1) & 1, abort_flag))) break;
       const int* ids = idx_s + is * KMAX;
       const long long base = p.row_off ? p.row_off[t] : 0;
-      const int nd = mla_dense_keys(p, t, base);
+      const int nd = mla_dense_keys<DENSE>(p, t, base);
       const int ntiles = mla_tiles(p, nd);
       const bool head_on = h < p.H;
       const float lse2 = head_on ? p.kl_lse[static_cast<long long>(t) * p.H + h] * kLog2e : 0.f;
@@ -532,8 +547,8 @@ sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         bool v_even, v_odd;
         if (nd < 0) {
           const int2 e = reinterpret_cast<const int2*>(ids + j * NK)[lane];
-          v_even = mla_valid(p, t, e.x, base);
-          v_odd = mla_valid(p, t, e.y, base);
+          v_even = mla_valid<PAGED>(p, t, e.x, base);
+          v_odd = mla_valid<PAGED>(p, t, e.y, base);
         } else {
           v_even = j * NK + 2 * lane < nd;
           v_odd = j * NK + 2 * lane + 1 < nd;
@@ -646,7 +661,7 @@ sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
       if (!(ok = warp_wait(bar(B_IDX_FULL + is), (ti >> 1) & 1, abort_flag))) break;
       const int* ids = idx_s + is * KMAX;
       const long long base = p.row_off ? p.row_off[t] : 0;
-      const int nd = mla_dense_keys(p, t, base);
+      const int nd = mla_dense_keys<DENSE>(p, t, base);
       const int ntiles = mla_tiles(p, nd);
       // l: sum of the bf16-rounded probabilities that enter P . V (normalises O exactly);
       // le: sum of the unrounded probabilities (for the log-sum-exp output)
@@ -657,8 +672,8 @@ sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         bool v_even, v_odd;
         if (nd < 0) {
           const int2 e = reinterpret_cast<const int2*>(ids + j * NK)[lane];
-          v_even = mla_valid(p, t, e.x, base);
-          v_odd = mla_valid(p, t, e.y, base);
+          v_even = mla_valid<PAGED>(p, t, e.x, base);
+          v_odd = mla_valid<PAGED>(p, t, e.y, base);
         } else {
           v_even = j * NK + 2 * lane < nd;
           v_odd = j * NK + 2 * lane + 1 < nd;
@@ -776,7 +791,7 @@ sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     int ti = 0;
     bool ok = true;
     for (int t = cluster; t < p.T && ok; t += nclusters, ++ti) {
-      const int ntiles = mla_tiles(p, mla_dense_keys(p, t, p.row_off ? p.row_off[t] : 0));
+      const int ntiles = mla_tiles(p, mla_dense_keys<DENSE>(p, t, p.row_off ? p.row_off[t] : 0));
       float l = 0.f;
       for (int j = 0; j < ntiles; ++j, ++g) {
         const int pb = static_cast<int>(g % NPB);

@@ -40,20 +40,28 @@ struct TkcSmem {
 };
 static_assert(4 * (sizeof(TkcSmem) + 1024) <= 228 * 1024, "four cluster top-k CTAs per SM");
 
-__device__ __forceinline__ uint32_t ld_cluster_u32(uint32_t cluster_addr) {
-  uint32_t v;
-  asm volatile("ld.shared::cluster.u32 %0, [%1];" : "=r"(v) : "r"(cluster_addr) : "memory");
-  return v;
-}
-__device__ __forceinline__ int ld_cluster_s32(uint32_t cluster_addr) {
-  return static_cast<int>(ld_cluster_u32(cluster_addr));
+// The u32 at the same shared-memory offset as `local` in each of the cluster's eight CTAs, loaded by one block of
+// eight loads, so that their latencies overlap.
+__device__ __forceinline__ void cluster_load8(const void* local, uint32_t (&v)[kTkcCluster]) {
+  static_assert(kTkcCluster == 8, "eight loads");
+  const uint32_t a = smem_u32(local);
+  asm volatile(
+      "ld.shared::cluster.u32 %0, [%8];\n\tld.shared::cluster.u32 %1, [%9];\n\t"
+      "ld.shared::cluster.u32 %2, [%10];\n\tld.shared::cluster.u32 %3, [%11];\n\t"
+      "ld.shared::cluster.u32 %4, [%12];\n\tld.shared::cluster.u32 %5, [%13];\n\t"
+      "ld.shared::cluster.u32 %6, [%14];\n\tld.shared::cluster.u32 %7, [%15];"
+      : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7])
+      : "r"(map_cluster(a, 0)), "r"(map_cluster(a, 1)), "r"(map_cluster(a, 2)), "r"(map_cluster(a, 3)),
+        "r"(map_cluster(a, 4)), "r"(map_cluster(a, 5)), "r"(map_cluster(a, 6)), "r"(map_cluster(a, 7))
+      : "memory");
 }
 // sum over the cluster's CTAs of the u32 at the same shared-memory offset as `local`
 __device__ __forceinline__ uint32_t cluster_sum_u32(const void* local) {
-  const uint32_t a = smem_u32(local);
+  uint32_t v[kTkcCluster];
+  cluster_load8(local, v);
   uint32_t s = 0;
 #pragma unroll
-  for (int q = 0; q < kTkcCluster; ++q) s += ld_cluster_u32(map_cluster(a, q));
+  for (int q = 0; q < kTkcCluster; ++q) s += v[q];
   return s;
 }
 
@@ -186,7 +194,20 @@ __global__ void __cluster_dims__(kTkcCluster, 1, 1) __launch_bounds__(kTkcThread
     for (int i = c0 + tid; i < c1; i += kTkcThreads) atomicAdd(&sm.bins[order_key(x[i]) >> 21], 1u);
   }
   cluster_sync();                                // every CTA's histogram is complete
-  for (int b = tid; b < kTopkBins; b += kTkcThreads) sm.merged[b] = cluster_sum_u32(&sm.bins[b]);
+  {
+    // the eight bins of this thread from every CTA: 64 loads issued before any is summed
+    constexpr int BPT = kTopkBins / kTkcThreads;
+    uint32_t v[BPT][kTkcCluster];
+#pragma unroll
+    for (int j = 0; j < BPT; ++j) cluster_load8(&sm.bins[tid + j * kTkcThreads], v[j]);
+#pragma unroll
+    for (int j = 0; j < BPT; ++j) {
+      uint32_t s = 0;
+#pragma unroll
+      for (int q = 0; q < kTkcCluster; ++q) s += v[j][q];
+      sm.merged[tid + j * kTkcThreads] = s;
+    }
+  }
   __syncthreads();
   {
     // bin holding the k-th largest key of the row: thread t owns bins 2047 - 8 t .. 2040 - 8 t (descending)
@@ -285,9 +306,11 @@ __global__ void __cluster_dims__(kTkcCluster, 1, 1) __launch_bounds__(kTkcThread
   cluster_sync();                                // every CTA's overflow flag is set
   bool from_row = false;
   {
+    uint32_t v[kTkcCluster];
+    cluster_load8(&sm.cta_over, v);
     uint32_t over = 0;
 #pragma unroll
-    for (int q = 0; q < kTkcCluster; ++q) over |= ld_cluster_u32(map_cluster(smem_u32(&sm.cta_over), q));
+    for (int q = 0; q < kTkcCluster; ++q) over |= v[q];
     from_row = over != 0;                        // the same decision in every CTA
   }
 
@@ -331,20 +354,26 @@ __global__ void __cluster_dims__(kTkcCluster, 1, 1) __launch_bounds__(kTkcThread
     sm.cta_eq = e;
   }
   cluster_sync();                                // every CTA's counts are set
-  if (tid == 0) {
-    // this CTA's place in the row: the entries the CTAs before it take
+  if (warp == 0) {
+    // this CTA's place in the row: the entries the CTAs before it take (all eight CTAs' counts, loaded at once)
+    uint32_t gv[kTkcCluster], ev[kTkcCluster];
+    cluster_load8(&sm.cta_gt, gv);
+    cluster_load8(&sm.cta_eq, ev);
     int base = 0, eqb = 0;
-    for (int q = 0; q < rank; ++q) {
-      const int gq = ld_cluster_s32(map_cluster(smem_u32(&sm.cta_gt), q));
-      const int eqq = ld_cluster_s32(map_cluster(smem_u32(&sm.cta_eq), q));
-      base += gq + max(0, min(eqq, static_cast<int>(need) - eqb));
-      eqb += eqq;
+#pragma unroll
+    for (int q = 0; q < kTkcCluster; ++q) {
+      if (q < rank) {
+        base += static_cast<int>(gv[q]) + max(0, min(static_cast<int>(ev[q]), static_cast<int>(need) - eqb));
+        eqb += static_cast<int>(ev[q]);
+      }
     }
-    for (int w = 0; w < W; ++w) {
-      sm.w_base[w] = base;
-      sm.w_eqb[w] = eqb;
-      base += sm.w_gt[w] + max(0, min(sm.w_eq[w], static_cast<int>(need) - eqb));
-      eqb += sm.w_eq[w];
+    if (lane == 0) {
+      for (int w = 0; w < W; ++w) {
+        sm.w_base[w] = base;
+        sm.w_eqb[w] = eqb;
+        base += sm.w_gt[w] + max(0, min(sm.w_eq[w], static_cast<int>(need) - eqb));
+        eqb += sm.w_eq[w];
+      }
     }
   }
   __syncthreads();

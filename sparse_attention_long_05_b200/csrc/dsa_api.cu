@@ -574,18 +574,14 @@ dsa_status_t select_rows(const uint8_t* q_idx, const float* q_scale, const uint8
   return DSA_OK;
 }
 
-// The digit rows of T query rows in the workspace area `at` (digit_bytes(T) long), computed on the stream for rows
-// from..T-1 only (the rows the indexer will score); nothing for configurations without digits.
+// The digit rows of T query rows in the workspace area `at` (digit_bytes(T) long), computed on the stream; nothing
+// for configurations without digits.
 dsa_status_t prepare_digits(const uint8_t* q_idx, const float* q_scale, const float* w, int T, int H_I, int d_I,
-                            void* at, DigitBufs* dig, cudaStream_t st, int from = 0) {
+                            void* at, DigitBufs* dig, cudaStream_t st) {
   *dig = DigitBufs();
   if (!uses_digits(H_I, d_I) || T <= 0) return DSA_OK;
   *dig = digit_bufs(at, T);
-  from = std::max(0, from);
-  if (from >= T) return DSA_OK;
-  const size_t f = static_cast<size_t>(from);
-  return run_digits(q_idx + f * H_I * d_I, q_scale ? q_scale + f : nullptr, w + f * H_I, T - from,
-                    dig->digits + f * kDigitRows * 128, dig->dscale + f * kDigitStride, st);
+  return run_digits(q_idx, q_scale, w, T, dig->digits, dig->dscale, st);
 }
 
 // Rows of the score block of an L-row prefill that starts at row r0: rows t < k form a block of their own, whose
@@ -798,7 +794,7 @@ dsa_status_t dsa_prefill_select(const uint8_t* q_idx, const float* q_scale, cons
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   DigitBufs dig;
   dsa_status_t e = prepare_digits(q_idx, q_scale, w, L, H_I, d_I, static_cast<char*>(ws) + prefill_digits_offset(L, k),
-                                  &dig, st, k);
+                                  &dig, st);
   if (e != DSA_OK) return e;
   return select_rows(q_idx, q_scale, k_idx, k_scale, w, H_I, d_I, k, 0, L, idx_out, static_cast<float*>(ws),
                      prefill_chunk_rows(L), st, dig);
@@ -832,7 +828,7 @@ dsa_status_t dsa_forward_prefill_rows(const uint8_t* q_idx, const float* q_scale
   DigitBufs dig;
   dsa_status_t e = prepare_digits(q_idx, q_scale, w, nrows, H_I, d_I,
                                   static_cast<char*>(ws) + score_bytes + align_up(size_t(nrows) * size_t(k) * 4, 256),
-                                  &dig, st, k - row0);
+                                  &dig, st);
   if (e != DSA_OK) return e;
   e = select_rows(q_idx, q_scale, k_idx, k_scale, w, H_I, d_I, k, row0, S, idx, static_cast<float*>(ws),
                   prefill_chunk_rows(S), st, dig);
@@ -981,13 +977,9 @@ dsa_status_t dsa_forward_prefill_host(const uint8_t* q_idx, const float* q_scale
       const DigitBufs all = digit_bufs(d + prefill_digits_offset(L, k), L);
       dig.digits = all.digits + size_t(t0[j]) * kDigitRows * 128;
       dig.dscale = all.dscale + size_t(t0[j]) * kDigitStride;
-      const int from = std::max(t0[j], std::min(k, t0[j + 1]));      // the chunk's rows the indexer scores
-      if (from < t0[j + 1]) {
-        const size_t f = static_cast<size_t>(from);
-        e = run_digits(dq_idx + f * H_I * d_I, dq_scale ? dq_scale + from : nullptr, dw + f * H_I, t0[j + 1] - from,
-                       all.digits + f * kDigitRows * 128, all.dscale + f * kDigitStride, st);
-        if (e != DSA_OK) break;
-      }
+      e = run_digits(dq_idx + size_t(t0[j]) * H_I * d_I, dq_scale ? dq_scale + t0[j] : nullptr, dw + size_t(t0[j]) * H_I,
+                     n, dig.digits, dig.dscale, st);
+      if (e != DSA_OK) break;
     }
     e = select_rows(dq_idx + size_t(t0[j]) * H_I * d_I, dq_scale ? dq_scale + t0[j] : nullptr, dk_idx, dk_scale,
                     dw + size_t(t0[j]) * H_I, H_I, d_I, k, t0[j], t0[j + 1], didx + size_t(t0[j]) * k, sc,

@@ -225,8 +225,6 @@ def select_split(dsa, x, cfg, ws, idx):
     CUDA events on the launching stream.  Returns (indexer ms, top-k ms, indexer launches, top-k launches)."""
     L, k = cfg.L, cfg.k
     blocks = dsa.prefill_blocks(L, k)      # the library's own block schedule
-    iws = torch.empty((max(1, dsa.dsa_indexer_scores_workspace_size(max(n for _, n in blocks), cfg.H_I, cfg.d_I)),),
-                      dtype=torch.uint8, device=ws.device)
     evs = []
     for r0, rows in blocks:
         S = r0 + rows
@@ -237,7 +235,7 @@ def select_split(dsa, x, cfg, ws, idx):
         e[0].record()
         if S > k:    # as in the select: a block of rows t < k has its selection implied, without scores
             dsa.dsa_indexer_scores(x["q_idx"][r0:r0 + rows], qs, x["k_idx"][:S], ks, x["w"][r0:r0 + rows],
-                                   pos0=r0, scores=sc, ws=iws)
+                                   pos0=r0, scores=sc)
         e[1].record()
         dsa.dsa_topk(sc, k, pos0=r0, idx=idx[r0:r0 + rows])
         e[2].record()

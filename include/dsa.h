@@ -83,15 +83,11 @@ DSA_API int dsa_num_sms(void);
  *   w       [T, H_I] fp32        indexer head weights
  *   scores  [T, S] fp32 (out)    I[pos0 + r, s] for s <= pos0 + r, -INFINITY for s > pos0 + r
  * Scores are accumulated in fp32 from exact e4m3 x e4m3 products, so integer-valued inputs with |I| < 2^24
- * give exact scores.  With H_I = 64, d_I = 128 the linear half of the sum, sum_j w[t,j] (q_I[t,j] . k_I[s]), is
- * formed on the tensor core from digit vectors of sum_j w[t,j] q_I[t,j] that the call writes into the
- * workspace (exact for integer-valued inputs; about 2^-20 relative otherwise).
- *   ws: device workspace of dsa_indexer_scores_workspace_size(T, H_I, d_I) bytes (0 for H_I = 4: may be NULL).
+ * give exact scores.  Needs no workspace.
  */
-DSA_API size_t dsa_indexer_scores_workspace_size(int T, int H_I, int d_I);
 DSA_API dsa_status_t dsa_indexer_scores(const uint8_t* q_idx, const float* q_scale, const uint8_t* k_idx,
                                 const float* k_scale, const float* w, int T, int S, int H_I, int d_I,
-                                int pos0, float* scores, void* ws, size_t ws_bytes, void* stream);
+                                int pos0, float* scores, void* stream);
 
 /*
  * Row-wise top-k selection (velog.io section 1.2) over materialised scores.

@@ -20,7 +20,6 @@ from ._lib import (  # noqa: F401
     dsa_get_device_status,
     dsa_indexer_kl,
     dsa_indexer_scores,
-    dsa_indexer_scores_workspace_size,
     dsa_launch_count,
     dsa_num_sms,
     dsa_prefill_block_rows,

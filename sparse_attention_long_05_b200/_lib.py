@@ -25,8 +25,7 @@ SIGNATURES = {
     "dsa_get_device_status": (_I, [_P, ctypes.POINTER(ctypes.c_int)]),
     "dsa_check_bounded_wait": (_I, [_P, _P]),
     "dsa_num_sms": (_I, []),
-    "dsa_indexer_scores_workspace_size": (_SZ, [_I, _I, _I]),
-    "dsa_indexer_scores": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P, _P, _SZ, _P]),
+    "dsa_indexer_scores": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P, _P]),
     "dsa_topk": (_I, [_P, _I, _I64, _P, _I, _I, _P, _P]),
     "dsa_sparse_mla_attn": (_I, [_P, _P, _I, _P, _I, _I, _I, _F, _P, _P, _P]),
     "dsa_indexer_kl": (_I, [_P, _P, _I, _P, _P, _P, _I, _I, _I, _F, _P, _P]),
@@ -117,22 +116,15 @@ def dsa_check_bounded_wait(stream=None):
     return res, dsa_get_device_status(stream)
 
 
-def dsa_indexer_scores_workspace_size(T: int, H_I: int, d_I: int) -> int:
-    return int(_lib.dsa_indexer_scores_workspace_size(T, H_I, d_I))
-
-
-def dsa_indexer_scores(q_idx, q_scale, k_idx, k_scale, w, pos0: int = 0, scores=None, ws=None, stream=None):
+def dsa_indexer_scores(q_idx, q_scale, k_idx, k_scale, w, pos0: int = 0, scores=None, stream=None):
     """Index scores [T, S] (fp32) of query rows at positions pos0.. against keys 0..S-1."""
     T, H_I, d_I = q_idx.shape
     S = k_idx.shape[0]
     if scores is None:
         scores = torch.empty((T, S), dtype=torch.float32, device=q_idx.device)
-    need = dsa_indexer_scores_workspace_size(T, H_I, d_I)
-    if ws is None and need:
-        ws = torch.empty((need,), dtype=torch.uint8, device=q_idx.device)
     _check("dsa_indexer_scores", _lib.dsa_indexer_scores(
         _ptr(q_idx), _ptr(q_scale), _ptr(k_idx), _ptr(k_scale), _ptr(w), T, S, H_I, d_I, pos0, _ptr(scores),
-        _ptr(ws), 0 if ws is None else ws.numel(), _stream(stream)))
+        _stream(stream)))
     return scores
 
 

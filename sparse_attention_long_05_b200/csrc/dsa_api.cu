@@ -260,84 +260,40 @@ size_t decode_score_cap(int B, int64_t cache_rows) { return size_t(cache_rows) +
 // requested to keep a second CTA off the SM (its allocation would wait for the first CTA to finish).
 constexpr int kMinIndexerSmem = 120 * 1024;
 
-template <int H_I, int D_I, int NT, int NG, int QBUF, int KST, int EPI, int MODE, int DIG = 0>
+template <int H_I, int D_I, int NT, int NG, int QBUF, int KST, int EPI, int MODE>
 dsa_status_t launch_indexer(const uint8_t* q_idx, int q_rows, const uint8_t* k_idx, long long k_rows,
-                            const IndexerParams& p, int grid, cudaStream_t st, const uint8_t* digits = nullptr) {
-  using C = IndexerCfg<H_I, D_I, NT, NG, QBUF, KST, EPI, MODE, DIG>;
-  CUtensorMap tq, tk, td;
+                            const IndexerParams& p, int grid, cudaStream_t st) {
+  using C = IndexerCfg<H_I, D_I, NT, NG, QBUF, KST, EPI, MODE>;
+  CUtensorMap tq, tk;
   const cuuint64_t qd[2] = {static_cast<cuuint64_t>(D_I), static_cast<cuuint64_t>(q_rows) * H_I};
   const cuuint64_t qs[1] = {static_cast<cuuint64_t>(D_I)};
-  const cuuint32_t qb[2] = {static_cast<cuuint32_t>(D_I), static_cast<cuuint32_t>(C::NQ)};
+  const cuuint32_t qb[2] = {static_cast<cuuint32_t>(D_I), static_cast<cuuint32_t>(C::N)};
   const cuuint64_t kd[2] = {static_cast<cuuint64_t>(D_I), static_cast<cuuint64_t>(k_rows)};
   const cuuint32_t kb[2] = {static_cast<cuuint32_t>(D_I), 128u};
   const CUtensorMapSwizzle sw = (D_I == 128) ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
   if (!make_map(&tq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, q_idx, qd, qs, qb, sw)) return DSA_ERR_CUDA;
   if (!make_map(&tk, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, k_idx, kd, qs, kb, sw)) return DSA_ERR_CUDA;
-  td = tq;   // configurations without digit rows never read this map
-  if (DIG) {
-    // the digit rows of the query rows: [q_rows * kDigitRows, D_I], DIG rows per group
-    if (!digits || !aligned16(digits)) return DSA_ERR_INVALID_ARG;
-    const cuuint64_t dd[2] = {static_cast<cuuint64_t>(D_I), static_cast<cuuint64_t>(q_rows) * kDigitRows};
-    const cuuint32_t db[2] = {static_cast<cuuint32_t>(D_I), static_cast<cuuint32_t>(DIG)};
-    if (!make_map(&td, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, digits, dd, qs, db, sw)) return DSA_ERR_CUDA;
-  }
-  auto kern = indexer_kernel<H_I, D_I, NT, NG, QBUF, KST, EPI, MODE, DIG>;
+  auto kern = indexer_kernel<H_I, D_I, NT, NG, QBUF, KST, EPI, MODE>;
   const int smem = (C::TMEM_COLS == 512 && C::SMEM < kMinIndexerSmem) ? kMinIndexerSmem : C::SMEM;
   if (set_smem(kern, smem) != cudaSuccess) return DSA_ERR_CUDA;
-  if (launch_pdl(kern, dim3(grid), dim3(C::NUM_THREADS), smem, st, tq, tk, td, p) != cudaSuccess) return DSA_ERR_CUDA;
+  if (launch_pdl(kern, dim3(grid), dim3(C::NUM_THREADS), smem, st, tq, tk, p) != cudaSuccess) return DSA_ERR_CUDA;
   return last_launch_status();
 }
 
-// The prefill indexer with 64 heads of 128 dims runs the digit configuration (see indexer.cuh): three query rows per
-// MMA group, their digit rows after their q_I rows, one token per epilogue warpgroup.
-constexpr int kDigitTok = 12;   // query rows per item of the digit configuration (3 per group, 4 groups)
-bool uses_digits(int H_I, int d_I) { return H_I == 64 && d_I == 128; }
-
-// digit rows and scales of T query rows (indexer_digits_kernel), into digits [T, kDigitRows, 128] and
-// dscale [T, kDigitStride]
-dsa_status_t run_digits(const uint8_t* q_idx, const float* q_scale, const float* w, int T, uint8_t* digits,
-                        float* dscale, cudaStream_t st) {
-  if (T <= 0) return DSA_OK;
-  const unsigned blocks = static_cast<unsigned>((static_cast<long long>(T) * 32 + 255) / 256);
-  if (launch_pdl(indexer_digits_kernel, dim3(blocks), dim3(256), 0, st, q_idx, q_scale, w, T, digits, dscale) !=
-      cudaSuccess)
-    return DSA_ERR_CUDA;
-  return last_launch_status();
-}
-
-// bytes of the digit rows and scales of T query rows (zero when the configuration uses none)
-size_t digit_bytes(long long T, int H_I, int d_I) {
-  if (!uses_digits(H_I, d_I) || T <= 0) return 0;
-  return align_up(size_t(T) * kDigitRows * 128, 256) + align_up(size_t(T) * kDigitStride * 4, 256);
-}
-struct DigitBufs {
-  uint8_t* digits = nullptr;
-  float* dscale = nullptr;
-};
-DigitBufs digit_bufs(void* at, long long T) {
-  DigitBufs d;
-  d.digits = static_cast<uint8_t*>(at);
-  d.dscale = reinterpret_cast<float*>(static_cast<char*>(at) + align_up(size_t(T) * kDigitRows * 128, 256));
-  return d;
-}
-
-// scores [T, S] of query rows at positions pos0.. against keys 0..S-1 (materialised); the digit configuration reads
-// the rows' digits (digits / dscale point at row 0 of this launch)
+// scores [T, S] of query rows at positions pos0.. against keys 0..S-1 (materialised)
 dsa_status_t run_indexer_scores(const uint8_t* q_idx, const float* q_scale, const uint8_t* k_idx,
                                 const float* k_scale, const float* w, int T, int S, int H_I, int d_I, int pos0,
-                                float* scores, long long ld, cudaStream_t st, const uint8_t* digits = nullptr,
-                                const float* dscale = nullptr) {
+                                float* scores, long long ld, cudaStream_t st) {
   IndexerParams p{};
   p.w = w;
   p.q_scale = q_scale;
-  p.dscale = dscale;
   p.k_scale = k_scale;
   p.scores = scores;
   p.ld = ld;
   p.T = T;
   p.S = S;
   p.pos0 = pos0;
-  const int tok = uses_digits(H_I, d_I) ? kDigitTok : 256;
+  const int tok = (H_I == 64) ? 16 : 256;
   const int nqb = (T + tok - 1) / tok;
   const int ntiles = (S + 127) / 128;
   // Work items (query block x key-tile range) go round-robin to one persistent CTA per SM.  The key range is
@@ -356,8 +312,8 @@ dsa_status_t run_indexer_scores(const uint8_t* q_idx, const float* q_scale, cons
   p.nsplit = (ntiles + p.split_tiles - 1) / p.split_tiles;
   p.n_items = nqb * p.nsplit;
   const int grid = p.n_items < sms ? p.n_items : sms;
-  if (uses_digits(H_I, d_I))
-    return launch_indexer<64, 128, 3, 4, 1, 4, 3, kModeScores, 16>(q_idx, T, k_idx, S, p, grid, st, digits);
+  if (H_I == 64)
+    return launch_indexer<64, 128, 4, 4, 1, 4, 2, kModeScores>(q_idx, T, k_idx, S, p, grid, st);
   return launch_indexer<4, 64, 64, 4, 1, 4, 2, kModeScores>(q_idx, T, k_idx, S, p, grid, st);
 }
 
@@ -391,12 +347,11 @@ void plan_segments(IndexerSeg* segs, int n_segs, int tok, int* split_tiles, int*
 dsa_status_t run_indexer_segments(const uint8_t* q_idx, long long q_rows, const float* q_scale, const uint8_t* k_idx,
                                   long long k_rows, const float* k_scale, const float* w, int H_I, int d_I,
                                   const IndexerSeg* segs_dev, int n_segs, int split_tiles, int n_items,
-                                  float* scores, cudaStream_t st, const uint8_t* digits, const float* dscale) {
+                                  float* scores, cudaStream_t st) {
   if (n_items <= 0) return DSA_OK;
   IndexerParams p{};
   p.w = w;
   p.q_scale = q_scale;
-  p.dscale = dscale;
   p.k_scale = k_scale;
   p.scores = scores;
   p.segs = segs_dev;
@@ -405,9 +360,9 @@ dsa_status_t run_indexer_segments(const uint8_t* q_idx, long long q_rows, const 
   p.n_items = n_items;
   const int sms = num_sms();
   const int grid = n_items < sms ? n_items : sms;
-  if (uses_digits(H_I, d_I))
-    return launch_indexer<64, 128, 3, 4, 1, 4, 3, kModeSegments, 16>(q_idx, static_cast<int>(q_rows), k_idx, k_rows,
-                                                                     p, grid, st, digits);
+  if (H_I == 64)
+    return launch_indexer<64, 128, 4, 4, 1, 4, 2, kModeSegments>(q_idx, static_cast<int>(q_rows), k_idx, k_rows, p,
+                                                                 grid, st);
   return launch_indexer<4, 64, 64, 4, 1, 4, 2, kModeSegments>(q_idx, static_cast<int>(q_rows), k_idx, k_rows, p, grid,
                                                              st);
 }
@@ -524,11 +479,6 @@ size_t prefill_chunk_rows(int L) {
 
 int round4(int n) { return (n + 3) & ~3; }
 
-// offset of the digit rows in a prefill workspace: after the score block and the selected indices
-size_t prefill_digits_offset(int L, int k) {
-  return align_up(prefill_chunk_rows(L) * size_t(L) * 4, 256) + align_up(size_t(L) * size_t(k) * 4, 256);
-}
-
 // Scores the varlen select holds at once: at least one sequence's blocked select (the longest), and up to 1 GiB
 // for groups of sequences scored together.
 size_t varlen_score_floats(int64_t total, int max_len) {
@@ -547,12 +497,10 @@ size_t varlen_meta_bytes(int nseq) {
 // idx_out point at row pos_begin; k_idx, k_scale hold keys 0..pos_end-1.  Rows t < k form one block whose
 // selection needs no scores; later rows go in blocks of chunk_rows, each an indexer launch into `sc` (room for
 // chunk_rows x pos_end scores) and a top-k launch.  With sel_scores (pointing at row pos_begin), the index score of
-// every selected position is written too, and the indexer then also scores the rows t < k.  dig: the digit rows of
-// row pos_begin onwards (written by run_digits), for the configurations that read them.
+// every selected position is written too, and the indexer then also scores the rows t < k.
 dsa_status_t select_rows(const uint8_t* q_idx, const float* q_scale, const uint8_t* k_idx, const float* k_scale,
                          const float* w, int H_I, int d_I, int k, int pos_begin, int pos_end, int32_t* idx_out,
-                         float* sc, size_t chunk_rows, cudaStream_t st, DigitBufs dig,
-                         float* sel_scores = nullptr) {
+                         float* sc, size_t chunk_rows, cudaStream_t st, float* sel_scores = nullptr) {
   for (int r0 = pos_begin, rows = 0; r0 < pos_end; r0 += rows) {
     rows = (r0 < k) ? std::min(k, pos_end) - r0 : static_cast<int>(std::min<size_t>(chunk_rows, pos_end - r0));
     const int s_eff = r0 + rows;   // keys beyond the block's last row are never selected (causal)
@@ -562,9 +510,7 @@ dsa_status_t select_rows(const uint8_t* q_idx, const float* q_scale, const uint8
     dsa_status_t e = DSA_OK;
     if (s_eff > k || sel_scores) {
       e = run_indexer_scores(q_idx + i * H_I * d_I, q_scale ? q_scale + i : nullptr, k_idx, k_scale, w + i * H_I,
-                             rows, s_eff, H_I, d_I, r0, sc, s_eff, st,
-                             dig.digits ? dig.digits + i * kDigitRows * 128 : nullptr,
-                             dig.dscale ? dig.dscale + i * kDigitStride : nullptr);
+                             rows, s_eff, H_I, d_I, r0, sc, s_eff, st);
       if (e != DSA_OK) return e;
     }
     e = run_topk(sc, s_eff, nullptr, nullptr, r0, rows, k, idx_out + i * k, k, st,
@@ -572,16 +518,6 @@ dsa_status_t select_rows(const uint8_t* q_idx, const float* q_scale, const uint8
     if (e != DSA_OK) return e;
   }
   return DSA_OK;
-}
-
-// The digit rows of T query rows in the workspace area `at` (digit_bytes(T) long), computed on the stream; nothing
-// for configurations without digits.
-dsa_status_t prepare_digits(const uint8_t* q_idx, const float* q_scale, const float* w, int T, int H_I, int d_I,
-                            void* at, DigitBufs* dig, cudaStream_t st) {
-  *dig = DigitBufs();
-  if (!uses_digits(H_I, d_I) || T <= 0) return DSA_OK;
-  *dig = digit_bufs(at, T);
-  return run_digits(q_idx, q_scale, w, T, dig->digits, dig->dscale, st);
 }
 
 // Rows of the score block of an L-row prefill that starts at row r0: rows t < k form a block of their own, whose
@@ -694,27 +630,16 @@ dsa_status_t dsa_get_device_status(void* stream, int* device_status) {
 
 int dsa_num_sms(void) { return num_sms(); }
 
-size_t dsa_indexer_scores_workspace_size(int T, int H_I, int d_I) {
-  if (T <= 0 || !indexer_shape_ok(H_I, d_I)) return 0;
-  return digit_bytes(T, H_I, d_I);
-}
-
 dsa_status_t dsa_indexer_scores(const uint8_t* q_idx, const float* q_scale, const uint8_t* k_idx,
                                 const float* k_scale, const float* w, int T, int S, int H_I, int d_I, int pos0,
-                                float* scores, void* ws, size_t ws_bytes, void* stream) {
+                                float* scores, void* stream) {
   if (T < 0 || S < 0 || pos0 < 0 || (T > 0 && (!q_idx || !w || !scores)) || (S > 0 && !k_idx))
     return DSA_ERR_INVALID_ARG;
   if (!indexer_shape_ok(H_I, d_I)) return DSA_ERR_UNSUPPORTED_SHAPE;
   if (!aligned16(q_idx) || !aligned16(k_idx)) return DSA_ERR_ALIGNMENT;
   if (T == 0 || S == 0) return DSA_OK;
-  const size_t need = dsa_indexer_scores_workspace_size(T, H_I, d_I);
-  if (need && (!ws || ws_bytes < need)) return DSA_ERR_WORKSPACE;
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
-  DigitBufs dig;
-  const dsa_status_t e = prepare_digits(q_idx, q_scale, w, T, H_I, d_I, ws, &dig, st);
-  if (e != DSA_OK) return e;
-  return run_indexer_scores(q_idx, q_scale, k_idx, k_scale, w, T, S, H_I, d_I, pos0, scores, S, st, dig.digits,
-                            dig.dscale);
+  return run_indexer_scores(q_idx, q_scale, k_idx, k_scale, w, T, S, H_I, d_I, pos0, scores, S,
+                            static_cast<cudaStream_t>(stream));
 }
 
 dsa_status_t dsa_topk(const float* scores, int rows, int64_t ld, const int32_t* row_len, int pos0, int k,
@@ -750,8 +675,7 @@ dsa_status_t dsa_forward_prefill_kl(const uint8_t* q_idx, const float* q_scale, 
     return DSA_ERR_ALIGNMENT;
   if (!ws || ws_bytes < dsa_prefill_kl_workspace_size(L, H_I, d_I, H, k)) return DSA_ERR_WORKSPACE;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  // workspace: the prefill's (score block, selected indices, digit rows), then the selected index scores [L, k] and
-  // lse [L, H]
+  // workspace: the prefill's (score block, selected indices), then the selected index scores [L, k] and lse [L, H]
   char* wsb = static_cast<char*>(ws);
   const size_t score_bytes = align_up(prefill_chunk_rows(L) * size_t(L) * 4, 256);
   int32_t* idx = idx_out ? idx_out : reinterpret_cast<int32_t*>(wsb + score_bytes);
@@ -759,11 +683,8 @@ dsa_status_t dsa_forward_prefill_kl(const uint8_t* q_idx, const float* q_scale, 
   float* sel = reinterpret_cast<float*>(wsb + at);
   at += align_up(size_t(L) * size_t(k) * 4, 256);
   float* lse_buf = lse ? lse : reinterpret_cast<float*>(wsb + at);
-  DigitBufs dig;
-  dsa_status_t e = prepare_digits(q_idx, q_scale, w, L, H_I, d_I, wsb + prefill_digits_offset(L, k), &dig, st);
-  if (e != DSA_OK) return e;
-  e = select_rows(q_idx, q_scale, k_idx, k_scale, w, H_I, d_I, k, 0, L, idx, reinterpret_cast<float*>(wsb),
-                  prefill_chunk_rows(L), st, dig, sel);
+  dsa_status_t e = select_rows(q_idx, q_scale, k_idx, k_scale, w, H_I, d_I, k, 0, L, idx, reinterpret_cast<float*>(wsb),
+                               prefill_chunk_rows(L), st, sel);
   if (e != DSA_OK) return e;
   e = run_mla_causal(q, c, L, idx, L, H, k, scale, out, lse_buf, st, 0);
   if (e != DSA_OK) return e;
@@ -779,9 +700,10 @@ dsa_status_t dsa_sparse_mla_attn(const uint16_t* q, const uint16_t* c, int S, co
 }
 
 size_t dsa_prefill_workspace_size(int L, int H_I, int d_I, int H, int k) {
-  (void)H;
+  (void)H_I; (void)d_I; (void)H;
   if (L <= 0 || k <= 0) return 0;
-  return prefill_digits_offset(L, k) + digit_bytes(L, H_I, d_I);
+  const size_t rows = prefill_chunk_rows(L);
+  return align_up(rows * size_t(L) * 4, 256) + align_up(size_t(L) * size_t(k) * 4, 256);
 }
 
 dsa_status_t dsa_prefill_select(const uint8_t* q_idx, const float* q_scale, const uint8_t* k_idx,
@@ -790,22 +712,16 @@ dsa_status_t dsa_prefill_select(const uint8_t* q_idx, const float* q_scale, cons
   if (L <= 0 || k <= 0 || !q_idx || !k_idx || !w || !idx_out) return DSA_ERR_INVALID_ARG;
   if (!indexer_shape_ok(H_I, d_I)) return DSA_ERR_UNSUPPORTED_SHAPE;
   if (!aligned16(q_idx) || !aligned16(k_idx)) return DSA_ERR_ALIGNMENT;
-  if (!ws || ws_bytes < dsa_prefill_workspace_size(L, H_I, d_I, 1, k)) return DSA_ERR_WORKSPACE;
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
-  DigitBufs dig;
-  dsa_status_t e = prepare_digits(q_idx, q_scale, w, L, H_I, d_I, static_cast<char*>(ws) + prefill_digits_offset(L, k),
-                                  &dig, st);
-  if (e != DSA_OK) return e;
+  if (!ws || ws_bytes < align_up(prefill_chunk_rows(L) * size_t(L) * 4, 256)) return DSA_ERR_WORKSPACE;
   return select_rows(q_idx, q_scale, k_idx, k_scale, w, H_I, d_I, k, 0, L, idx_out, static_cast<float*>(ws),
-                     prefill_chunk_rows(L), st, dig);
+                     prefill_chunk_rows(L), static_cast<cudaStream_t>(stream));
 }
 
 size_t dsa_prefill_rows_workspace_size(int row0, int nrows, int H_I, int d_I, int H, int k) {
-  (void)H;
+  (void)H_I; (void)d_I; (void)H;
   if (row0 < 0 || nrows <= 0 || k <= 0) return 0;
   const int S = row0 + nrows;
-  return align_up(prefill_chunk_rows(S) * size_t(S) * 4, 256) + align_up(size_t(nrows) * size_t(k) * 4, 256) +
-         digit_bytes(nrows, H_I, d_I);
+  return align_up(prefill_chunk_rows(S) * size_t(S) * 4, 256) + align_up(size_t(nrows) * size_t(k) * 4, 256);
 }
 
 dsa_status_t dsa_forward_prefill_rows(const uint8_t* q_idx, const float* q_scale, const uint8_t* k_idx,
@@ -825,13 +741,8 @@ dsa_status_t dsa_forward_prefill_rows(const uint8_t* q_idx, const float* q_scale
   const int S = row0 + nrows;
   const size_t score_bytes = align_up(prefill_chunk_rows(S) * size_t(S) * 4, 256);
   int32_t* idx = idx_out ? idx_out : reinterpret_cast<int32_t*>(static_cast<char*>(ws) + score_bytes);
-  DigitBufs dig;
-  dsa_status_t e = prepare_digits(q_idx, q_scale, w, nrows, H_I, d_I,
-                                  static_cast<char*>(ws) + score_bytes + align_up(size_t(nrows) * size_t(k) * 4, 256),
-                                  &dig, st);
-  if (e != DSA_OK) return e;
-  e = select_rows(q_idx, q_scale, k_idx, k_scale, w, H_I, d_I, k, row0, S, idx, static_cast<float*>(ws),
-                  prefill_chunk_rows(S), st, dig);
+  dsa_status_t e = select_rows(q_idx, q_scale, k_idx, k_scale, w, H_I, d_I, k, row0, S, idx, static_cast<float*>(ws),
+                               prefill_chunk_rows(S), st);
   if (e != DSA_OK) return e;
   return run_mla_causal(q, c, S, idx, nrows, H, k, scale, out, lse, st, row0);
 }
@@ -971,19 +882,9 @@ dsa_status_t dsa_forward_prefill_host(const uint8_t* q_idx, const float* q_scale
       ok = cudaEventRecord(ev_att[j], st) == cudaSuccess;
       continue;
     }
-    // the chunk's digit rows (in the prefill workspace's digit area, at the chunk's rows), then its selection
-    DigitBufs dig;
-    if (uses_digits(H_I, d_I)) {
-      const DigitBufs all = digit_bufs(d + prefill_digits_offset(L, k), L);
-      dig.digits = all.digits + size_t(t0[j]) * kDigitRows * 128;
-      dig.dscale = all.dscale + size_t(t0[j]) * kDigitStride;
-      e = run_digits(dq_idx + size_t(t0[j]) * H_I * d_I, dq_scale ? dq_scale + t0[j] : nullptr, dw + size_t(t0[j]) * H_I,
-                     n, dig.digits, dig.dscale, st);
-      if (e != DSA_OK) break;
-    }
     e = select_rows(dq_idx + size_t(t0[j]) * H_I * d_I, dq_scale ? dq_scale + t0[j] : nullptr, dk_idx, dk_scale,
                     dw + size_t(t0[j]) * H_I, H_I, d_I, k, t0[j], t0[j + 1], didx + size_t(t0[j]) * k, sc,
-                    prefill_chunk_rows(L), st, dig);
+                    prefill_chunk_rows(L), st);
     if (e != DSA_OK) break;
     ok = cudaStreamWaitEvent(st, ev_q[j], 0) == cudaSuccess;
     if (!ok) break;
@@ -1008,12 +909,11 @@ dsa_status_t dsa_forward_prefill_host(const uint8_t* q_idx, const float* q_scale
 }
 
 size_t dsa_prefill_varlen_workspace_size(int nseq, int64_t total, int max_len, int H_I, int d_I, int H, int k) {
-  (void)H;
+  (void)H_I; (void)d_I; (void)H;
   if (nseq <= 0 || total <= 0 || max_len <= 0 || k <= 0) return 0;
   return align_up(varlen_score_floats(total, max_len) * 4, 256) + align_up(size_t(total) * 8, 256) +
          align_up(size_t(nseq + 1) * 8, 256) + align_up(size_t(total) * size_t(k) * 4, 256) +
-         align_up(size_t(total) * 8, 256) + align_up(size_t(total) * 4, 256) + varlen_meta_bytes(nseq) +
-         digit_bytes(total, H_I, d_I);
+         align_up(size_t(total) * 8, 256) + align_up(size_t(total) * 4, 256) + varlen_meta_bytes(nseq);
 }
 
 dsa_status_t dsa_forward_prefill_varlen(int nseq, const int64_t* cu_seqlens, const uint8_t* q_idx,
@@ -1056,11 +956,6 @@ dsa_status_t dsa_forward_prefill_varlen(int nseq, const int64_t* cu_seqlens, con
   int* tk_len = reinterpret_cast<int*>(wsb + at);
   at += align_up(size_t(total) * 4, 256);
   char* meta = wsb + at;
-  at += varlen_meta_bytes(nseq);
-  // the digit rows of every row of the batch (rows are packed, so a sequence's rows are a slice of them)
-  DigitBufs dig_all;
-  dsa_status_t e0 = prepare_digits(q_idx, q_scale, w, static_cast<int>(total), H_I, d_I, wsb + at, &dig_all, st);
-  if (e0 != DSA_OK) return e0;
   IndexerSeg* segs_dev = reinterpret_cast<IndexerSeg*>(meta);
   long long* gcu_dev = reinterpret_cast<long long*>(meta + align_up(size_t(nseq) * sizeof(IndexerSeg), 256));
   long long* soff_dev = gcu_dev + (nseq + 1);
@@ -1076,20 +971,15 @@ dsa_status_t dsa_forward_prefill_varlen(int nseq, const int64_t* cu_seqlens, con
   std::vector<IndexerSeg> segs;
   std::vector<long long> gcu, soff;
   std::vector<int> sld;
-  const int tok = uses_digits(H_I, d_I) ? kDigitTok : 256;
+  const int tok = (H_I == 64) ? 16 : 256;
   for (int b = 0; b < nseq;) {
     const int64_t r0 = cu_seqlens[b];
     const int len = static_cast<int>(cu_seqlens[b + 1] - r0);
     const size_t need = (len > k) ? size_t(len - k) * size_t(round4(len)) : 0;
     if (need > budget) {
-      DigitBufs dig;
-      if (dig_all.digits) {
-        dig.digits = dig_all.digits + r0 * kDigitRows * 128;
-        dig.dscale = dig_all.dscale + r0 * kDigitStride;
-      }
       e = select_rows(q_idx + r0 * H_I * d_I, q_scale ? q_scale + r0 : nullptr, k_idx + r0 * d_I,
                       k_scale ? k_scale + r0 : nullptr, w + r0 * H_I, H_I, d_I, k, 0, len, idx + r0 * k, sc,
-                      prefill_chunk_rows(len), st, dig);
+                      prefill_chunk_rows(len), st);
       if (e != DSA_OK) return e;
       ++b;
       continue;
@@ -1130,8 +1020,7 @@ dsa_status_t dsa_forward_prefill_varlen(int nseq, const int64_t* cu_seqlens, con
           cudaSuccess)
         return DSA_ERR_CUDA;
       e = run_indexer_segments(q_idx, total, q_scale, k_idx, total, k_scale, w, H_I, d_I, segs_dev,
-                               static_cast<int>(segs.size()), split, n_items, sc, st, dig_all.digits,
-                               dig_all.dscale);
+                               static_cast<int>(segs.size()), split, n_items, sc, st);
       if (e != DSA_OK) return e;
     }
     if (cudaMemcpyAsync(gcu_dev, gcu.data(), size_t(ng + 1) * 8, cudaMemcpyHostToDevice, st) != cudaSuccess ||

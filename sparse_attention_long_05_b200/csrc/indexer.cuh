@@ -17,15 +17,6 @@
 // epilogue of one (tile, group) overlap the MMAs of the next ones.  Tiles lying wholly above the causal
 // diagonal of every token of the item are never loaded.
 //
-// Linear half on the tensor core (prefill configuration, DIG > 0).  w ReLU(x) = (w x + w |x|) / 2, and the linear
-// half summed over the heads is one dot product: sum_j w[t,j] x_j = k_I[s] . q'[t] with q'[t] = sum_j w[t,j] q_I[t,j].
-// indexer_digits_kernel writes q'[t] (scaled by s_q) as kDigitRows e4m3 "digit" vectors d_i and fp32 scales
-// sigma_i, q' = sum_i sigma_i d_i (integer inputs: balanced base-16 digits with sigma = 1, 16, 256, exact; otherwise
-// a greedy refinement, each digit carrying the residual of the ones before, about 2^-20 relative after five).  The
-// digit rows of a group's tokens ride in the MMA's B operand after its q_I rows, so the accumulator holds
-// k_I[s] . d_i beside the per-head products, and the epilogue needs one FMA per (key, token, head) element:
-// I = s_k (sum_j (w_j s_q / 2) |x_j| + sum_i (sigma_i / 2) (k_I . d_i)).
-//
 // Work items:
 //   kModeScores  item = (block of NG*NT query rows, range of key tiles); writes scores [T, S] (tests,
 //                materialised prefill chunks);
@@ -60,7 +51,6 @@ struct IndexerSeg {
 struct IndexerParams {
   const float* w;          // [T, H_I]
   const float* q_scale;    // [T] or null
-  const float* dscale;     // digit configuration: [T, kDigitStride] digit scales of each query row
   const float* k_scale;    // per key row, or null
   float* scores;           // output (see modes)
   long long ld;            // kModeScores: row stride of scores
@@ -100,80 +90,10 @@ __device__ __forceinline__ long long key_row(const IndexerItem& it, int tile, in
 }
 
 constexpr int kMaxDecodeSeqs = 1024;
-constexpr int kDigitRows = 5;      // e4m3 digit vectors of q' per query row (prefill configuration)
-constexpr int kDigitStride = 8;    // floats per query row in the digit-scale array
 
-// q'[t] = s_q[t] sum_j w[t,j] q_I[t,j] of each query row (H_I = 64 heads of d_I = 128) as kDigitRows e4m3 digit
-// vectors digits[t][i][128] and scales dscale[t][i] (kDigitStride per row), q' = sum_i dscale * digit.  One warp per
-// row; lane l owns dims 4 l .. 4 l + 3.  Integer-valued q' with |q'| <= 2184 (the integer input mode) takes
-// balanced base-16 digits, exactly; anything else a greedy refinement: sigma_i = max|r| / 448, d_i = e4m3(r /
-// sigma_i), r -= sigma_i d_i.
-__global__ void __launch_bounds__(256) indexer_digits_kernel(const uint8_t* q_idx, const float* q_scale,
-                                                            const float* w, int T, uint8_t* digits,
-                                                            float* dscale) {
-  pdl_allow_next();
-  pdl_wait();
-  const int row = static_cast<int>((static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5);
-  const int lane = threadIdx.x & 31;
-  if (row >= T) return;
-  const uint8_t* qr = q_idx + static_cast<long long>(row) * 64 * 128;
-  const float* wr = w + static_cast<long long>(row) * 64;
-  float r[4] = {0.f, 0.f, 0.f, 0.f};
-  for (int j = 0; j < 64; ++j) {
-    const uint32_t bits = *reinterpret_cast<const uint32_t*>(qr + j * 128 + 4 * lane);
-    const float wj = wr[j];
-#pragma unroll
-    for (int d = 0; d < 4; ++d) {
-      __nv_fp8_e4m3 v;
-      v.__x = static_cast<__nv_fp8_storage_t>((bits >> (8 * d)) & 0xFFu);
-      r[d] = fmaf(wj, static_cast<float>(v), r[d]);
-    }
-  }
-  const float sq = q_scale ? q_scale[row] : 1.f;
-#pragma unroll
-  for (int d = 0; d < 4; ++d) r[d] *= sq;
-  bool integral = true;
-#pragma unroll
-  for (int d = 0; d < 4; ++d) integral = integral && r[d] == rintf(r[d]) && fabsf(r[d]) <= 2184.f;
-  integral = __all_sync(0xffffffffu, integral);
-  uint8_t* out = digits + static_cast<long long>(row) * kDigitRows * 128 + 4 * lane;
-  float* sc = dscale + static_cast<long long>(row) * kDigitStride;
-  for (int i = 0; i < kDigitRows; ++i) {
-    float sigma;
-    if (integral) {
-      sigma = (i < 3) ? static_cast<float>(1 << (4 * i)) : 0.f;
-    } else {
-      float m = fmaxf(fmaxf(fabsf(r[0]), fabsf(r[1])), fmaxf(fabsf(r[2]), fabsf(r[3])));
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-      sigma = m / 448.f;
-    }
-    uint32_t packed = 0;
-#pragma unroll
-    for (int d = 0; d < 4; ++d) {
-      float dv = 0.f;
-      if (sigma > 0.f) {
-        if (integral) {
-          // balanced base-16 digit of the remaining integer r / sigma
-          const float q = r[d] / sigma;
-          dv = (i < 2) ? q - 16.f * rintf(q * 0.0625f) : q;
-        } else {
-          dv = static_cast<float>(__nv_fp8_e4m3(r[d] / sigma));
-        }
-      }
-      const __nv_fp8_e4m3 e(dv);
-      packed |= static_cast<uint32_t>(e.__x) << (8 * d);
-      r[d] -= sigma * static_cast<float>(e);
-    }
-    *reinterpret_cast<uint32_t*>(out + i * 128) = packed;
-    if (lane == 0) sc[i] = sigma;
-  }
-}
-
-template <int H_I, int D_I, int NT, int NG, int QBUF, int KSTAGES, int EPI_WG, int MODE, int DIG = 0>
+template <int H_I, int D_I, int NT, int NG, int QBUF, int KSTAGES, int EPI_WG, int MODE>
 struct IndexerCfg {
-  static constexpr int NQ = NT * H_I;                // q_I rows of a group
-  static constexpr int N = NQ + DIG;                 // MMA N: the q_I rows, then DIG digit rows
+  static constexpr int N = NT * H_I;                 // MMA N
   static constexpr int TOK = NT * NG;                // query rows per item
   static constexpr int GBYTES = N * D_I;             // one group of q_I rows
   static constexpr int KBYTES = 128 * D_I;           // one key tile
@@ -188,26 +108,21 @@ struct IndexerCfg {
   static constexpr int DEC_BYTES = 4 * (kMaxDecodeSeqs + 1) + 4 * kMaxDecodeSeqs + 8 * kMaxDecodeSeqs + 8;
   static constexpr int OFF_W = ((OFF_PREFIX + (MODE != kModeScores ? DEC_BYTES : 0) + 15) / 16) * 16;
   static constexpr int W_FLOATS = TOK * H_I;
-  static constexpr int DS_FLOATS = DIG ? TOK * kDigitStride : 0;     // digit scales of the item's rows
-  static constexpr int OFF_DS = OFF_W + QBUF * W_FLOATS * 4;
-  static constexpr int OFF_Q = ((OFF_DS + QBUF * DS_FLOATS * 4 + ALIGN - 1) / ALIGN) * ALIGN;
+  static constexpr int OFF_Q = ((OFF_W + QBUF * W_FLOATS * 4 + ALIGN - 1) / ALIGN) * ALIGN;
   static constexpr int OFF_K = OFF_Q + QBUF * NG * GBYTES;
   static constexpr int SMEM = OFF_K + KSTAGES * KBYTES + ALIGN;  // + alignment slack
   // accumulator ring: as many N-column accumulators as tensor memory holds (2 at N = 256), so that the MMAs
   // run that many (token group, key tile) steps ahead of the epilogue; decode keeps half of tensor memory
   // (4 x 64 columns) so that two CTAs share an SM
   static constexpr int NACC = (MODE == kModeDecode) ? 4 : ((512 / N) < 8 ? (512 / N) : 8);
-  static constexpr uint32_t TMEM_USED = static_cast<uint32_t>(NACC * N);
-  static constexpr uint32_t TMEM_COLS = TMEM_USED <= 256 ? 256u : 512u;   // allocations are powers of two
-  static_assert(TMEM_USED <= 512, "tensor memory");
+  static constexpr uint32_t TMEM_COLS = static_cast<uint32_t>(NACC * N);
+  static_assert(TMEM_COLS == 256 || TMEM_COLS == 512, "tensor-memory allocation (power of two)");
   static constexpr uint32_t SW_LAYOUT = (D_I == 128) ? kLayoutSW128 : kLayoutSW64;
   static constexpr uint32_t SBO = (D_I == 128) ? 1024 : 512;
   static_assert(N <= 256 && N % 16 == 0, "MMA N");
   static_assert(OFF_W % 16 == 0 && (W_FLOATS * 4) % 16 == 0, "head weights are read as 16-byte quads");
   static_assert(D_I == 128 || D_I == 64, "d_I");
-  static_assert((NQ / EPI_WG) % H_I == 0 || H_I > NQ / EPI_WG, "epilogue column split");
-  static_assert(DIG == 0 || (NT * kDigitRows <= DIG && DIG % 16 == 0 && NQ / EPI_WG == H_I && H_I == 64),
-                "digit configuration: one token of 64 heads per epilogue warpgroup");
+  static_assert((N / EPI_WG) % H_I == 0 || H_I > N / EPI_WG, "epilogue column split");
 };
 
 // barrier slots (8 bytes each) in the barrier area
@@ -305,12 +220,12 @@ __device__ __forceinline__ bool tile_active(const IndexerItem& it, int tile) {
   return tile * 128 < it.n_keys && tile * 128 <= it.pos0 + it.n_tok - 1;
 }
 
-template <int H_I, int D_I, int NT, int NG, int QBUF, int KSTAGES, int EPI_WG, int MODE, int DIG = 0>
-__global__ void __launch_bounds__(IndexerCfg<H_I, D_I, NT, NG, QBUF, KSTAGES, EPI_WG, MODE, DIG>::NUM_THREADS,
-                                  IndexerCfg<H_I, D_I, NT, NG, QBUF, KSTAGES, EPI_WG, MODE, DIG>::CTAS_PER_SM)
+template <int H_I, int D_I, int NT, int NG, int QBUF, int KSTAGES, int EPI_WG, int MODE>
+__global__ void __launch_bounds__(IndexerCfg<H_I, D_I, NT, NG, QBUF, KSTAGES, EPI_WG, MODE>::NUM_THREADS,
+                                  IndexerCfg<H_I, D_I, NT, NG, QBUF, KSTAGES, EPI_WG, MODE>::CTAS_PER_SM)
 indexer_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-               const __grid_constant__ CUtensorMap tm_d, const IndexerParams p) {
-  using C = IndexerCfg<H_I, D_I, NT, NG, QBUF, KSTAGES, EPI_WG, MODE, DIG>;
+               const IndexerParams p) {
+  using C = IndexerCfg<H_I, D_I, NT, NG, QBUF, KSTAGES, EPI_WG, MODE>;
   using Bars = IndexerBars<QBUF, KSTAGES, C::NACC>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + C::ALIGN - 1) &
@@ -320,7 +235,6 @@ indexer_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Bars::OFF_ABORT);
   int* prefix = reinterpret_cast<int*>(smem + C::OFF_PREFIX);
   float* w_s = reinterpret_cast<float*>(smem + C::OFF_W);
-  float* ds_s = reinterpret_cast<float*>(smem + C::OFF_DS);
   const uint32_t q_s = sbase + C::OFF_Q;
   const uint32_t k_s = sbase + C::OFF_K;
   const int warp = warp_id(), lane = lane_id();
@@ -376,11 +290,7 @@ indexer_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
   if constexpr (MODE == kModeSegments) {
     for (int sgi = threadIdx.x; sgi < p.n_segs; sgi += blockDim.x) prefix[sgi] = p.segs[sgi].item0;
   }
-  if (warp == 0 && lane == 0) {
-    prefetch_tmap(&tm_q);
-    prefetch_tmap(&tm_k);
-    if (DIG) prefetch_tmap(&tm_d);
-  }
+  if (warp == 0 && lane == 0) { prefetch_tmap(&tm_q); prefetch_tmap(&tm_k); }
   if (warp == 1) {
     tmem_alloc(sbase + Bars::OFF_TMEM, C::TMEM_COLS);
     tmem_relinquish();
@@ -440,13 +350,9 @@ indexer_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         const uint32_t qph = (qi / QBUF) & 1;
         if (!mbar_wait(bar(Bars::Q_EMPTY + qb), qph ^ 1, abort_flag)) { ok = false; break; }
         mbar_arrive_expect_tx(bar(Bars::Q_FULL + qb), NG * C::GBYTES);
-        for (int g = 0; g < NG; ++g) {
+        for (int g = 0; g < NG; ++g)
           tma_load_2d(q_s + (qb * NG + g) * C::GBYTES, &tm_q, bar(Bars::Q_FULL + qb), 0,
                       (it.q_row0 + g * NT) * H_I);
-          if (DIG)   // the group's digit rows after its q_I rows (rows past the last token are not read)
-            tma_load_2d(q_s + (qb * NG + g) * C::GBYTES + C::NQ * D_I, &tm_d, bar(Bars::Q_FULL + qb), 0,
-                        (it.q_row0 + g * NT) * kDigitRows);
-        }
         q_issued[qb] += 1;
         q_par[qb] = qph;
         for (int tile = it.tile0; tile < it.tile1; ++tile) {
@@ -506,16 +412,13 @@ indexer_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     }
   } else {
     // ------------------------------------------------------------------ epilogue
-    constexpr int CPT = C::NQ / EPI_WG;             // accumulator columns (heads of its tokens) per thread
+    constexpr int CPT = C::N / EPI_WG;              // accumulator columns per thread
     constexpr int TOKS = (CPT >= H_I) ? CPT / H_I : 1;  // query rows per thread
     constexpr int P = (H_I >= 16) ? 4 : 1;         // partial sums per row (ILP)
     // Packed epilogue (heads in groups of four): w ReLU(x) is formed as w max(x, 0) for even heads (ALU pipe)
     // and as (w / 2)(x + |x|) for odd heads (FMA pipe, |x| as an operand modifier), so that the two pipes share
     // the ReLUs; the odd heads' weights are stored halved.  Both forms are exact for integer-valued inputs.
-    constexpr bool kPacked = DIG == 0 && (H_I % 64 == 0) && (CPT % 64 == 0);
-    // Digit epilogue (DIG > 0): one token per thread; w |x| with halved weights (one FMA, |x| as an operand
-    // modifier) plus the linear half from the digit columns.
-    constexpr bool kDigits = DIG > 0;
+    constexpr bool kPacked = (H_I % 64 == 0) && (CPT % 64 == 0);
     const int e = warp - 2;
     const int quad = warp & 3;
     const int half = e >> 2;
@@ -528,7 +431,6 @@ indexer_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     for (int item = first_item(); has_item(item) && ok; item = next_item(item), ++qi) {
       const IndexerItem it = indexer_item<MODE, C::TOK>(p, item, prefix, tr);
       float* wq = w_s + (qi % QBUF) * C::W_FLOATS;
-      float* dsq = ds_s + (qi % QBUF) * C::DS_FLOATS;
       named_bar_sync(1, ethreads);
       for (int i = etid; i < C::W_FLOATS; i += ethreads) {
         const int r = i / H_I;
@@ -536,16 +438,9 @@ indexer_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         if (r < it.n_tok) {
           v = p.w[static_cast<long long>(it.q_row0 + r) * H_I + (i % H_I)];
           if (p.q_scale) v *= p.q_scale[it.q_row0 + r];
-          if ((kPacked && (i & 1)) || kDigits) v *= 0.5f;
+          if (kPacked && (i & 1)) v *= 0.5f;
         }
         wq[i] = v;
-      }
-      if constexpr (kDigits) {
-        for (int i = etid; i < C::DS_FLOATS; i += ethreads) {
-          const int r = i / kDigitStride, d = i % kDigitStride;
-          dsq[i] = (r < it.n_tok && d < kDigitRows)
-                       ? 0.5f * p.dscale[static_cast<long long>(it.q_row0 + r) * kDigitStride + d] : 0.f;
-        }
       }
       named_bar_sync(1, ethreads);
       // key scales are loaded one tile ahead: a load issued at the start of its own tile would expose the
@@ -583,36 +478,7 @@ indexer_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
 #pragma unroll
             for (int q = 0; q < P; ++q) acc[tk][q] = 0.f;
           const uint32_t tcol = tmem_base + ap.stage * C::N + half * CPT;
-          if constexpr (kDigits) {
-            // this thread's token (row tok0): 64 head columns, then the group's digit columns
-            uint32_t v0[32], v1[32], dg[16];
-            tmem_ld32(lane_addr + tcol, v0);
-            tmem_ld32(lane_addr + tcol + 32, v1);
-            tmem_ld16(lane_addr + tmem_base + ap.stage * C::N + C::NQ, dg);
-            tmem_wait_ld();
-            tmem_regs_after_wait(v0);
-            tmem_regs_after_wait(v1);
-            tmem_regs_after_wait(dg);
-            const float4* w4 = reinterpret_cast<const float4*>(wq + tok0 * H_I);
-#pragma unroll
-            for (int i = 0; i < 64; i += 4) {
-              const float4 ww = w4[i >> 2];
-              const uint32_t* xs = (i < 32) ? &v0[i] : &v1[i - 32];
-              acc[0][0] = fmaf(ww.x, fabsf(__uint_as_float(xs[0])), acc[0][0]);
-              acc[0][1] = fmaf(ww.y, fabsf(__uint_as_float(xs[1])), acc[0][1]);
-              acc[0][2] = fmaf(ww.z, fabsf(__uint_as_float(xs[2])), acc[0][2]);
-              acc[0][3] = fmaf(ww.w, fabsf(__uint_as_float(xs[3])), acc[0][3]);
-            }
-            // linear half: the digit columns of this token (group slot `half`, compile-time register indices)
-            const float* dsr = dsq + tok0 * kDigitStride;
-            float lin = 0.f;
-#pragma unroll
-            for (int i = 0; i < kDigitRows; ++i) {
-              const uint32_t y = (half == 0) ? dg[i] : (half == 1) ? dg[kDigitRows + i] : dg[2 * kDigitRows + i];
-              lin = fmaf(dsr[i], __uint_as_float(y), lin);
-            }
-            acc[0][0] += lin;
-          } else if constexpr (kPacked) {
+          if constexpr (kPacked) {
             uint64_t acc2[TOKS][2];
 #pragma unroll
             for (int tk = 0; tk < TOKS; ++tk) acc2[tk][0] = acc2[tk][1] = 0ull;

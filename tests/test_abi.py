@@ -54,16 +54,13 @@ def test_host_argument_checks(lib):
     P = ctypes.c_void_p
     one = P(16)  # a dummy aligned non-null address: every call below must fail before touching it
     # unsupported indexer shape
-    assert lib.dsa_indexer_scores(one, None, one, None, one, 4, 4, 32, 128, 0, one, None, 0, None) == 2
+    assert lib.dsa_indexer_scores(one, None, one, None, one, 4, 4, 32, 128, 0, one, None) == 2
     # negative sizes / null outputs
-    assert lib.dsa_indexer_scores(one, None, one, None, one, -1, 4, 64, 128, 0, one, None, 0, None) == 1
+    assert lib.dsa_indexer_scores(one, None, one, None, one, -1, 4, 64, 128, 0, one, None) == 1
     assert lib.dsa_topk(None, 3, 10, None, 0, 4, one, None) == 1
     assert lib.dsa_topk(one, 3, 10, None, 0, 0, one, None) == 1
     # misaligned TMA operand
-    assert lib.dsa_indexer_scores(P(17), None, one, None, one, 4, 4, 64, 128, 0, one, None, 0, None) == 3
-    # the 64-head configuration needs its digit workspace
-    assert lib.dsa_indexer_scores_workspace_size(4, 64, 128) > 0 and lib.dsa_indexer_scores_workspace_size(4, 4, 64) == 0
-    assert lib.dsa_indexer_scores(one, None, one, None, one, 4, 4, 64, 128, 0, one, None, 0, None) == 7
+    assert lib.dsa_indexer_scores(P(17), None, one, None, one, 4, 4, 64, 128, 0, one, None) == 3
     # attention: too many heads, k not a multiple of 64
     assert lib.dsa_sparse_mla_attn(one, one, 10, one, 2, 129, 64, 1.0, one, None, None) == 2
     assert lib.dsa_sparse_mla_attn(one, one, 10, one, 2, 8, 100, 1.0, one, None, None) == 2
@@ -94,7 +91,7 @@ def test_host_argument_checks(lib):
     assert lib.dsa_check_bounded_wait(None, None) == 1
     assert lib.dsa_check_bounded_wait(P(20), None) == 3
     # empty work is a no-op
-    assert lib.dsa_indexer_scores(one, None, one, None, one, 0, 4, 64, 128, 0, one, None, 0, None) == 0
+    assert lib.dsa_indexer_scores(one, None, one, None, one, 0, 4, 64, 128, 0, one, None) == 0
 
 
 def test_prefill_block_schedule(lib):

@@ -201,21 +201,18 @@ __device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_
   asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
                :: "r"(dst), "l"(src), "r"(bytes), "r"(bar) : "memory");
 }
-// 1-D bulk copy from this CTA's shared memory to another CTA's shared memory in the cluster, completing
-// `bytes` of transaction count on the destination CTA's mbarrier (both given as shared::cluster addresses)
-__device__ __forceinline__ void bulk_copy_to_peer(uint32_t dst_cluster, uint32_t src_local, uint32_t bytes,
-                                                  uint32_t bar_cluster) {
-  asm volatile("cp.async.bulk.shared::cluster.shared::cta.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
-               :: "r"(dst_cluster), "r"(src_local), "r"(bytes), "r"(bar_cluster) : "memory");
+// store 16 (4) bytes into a peer CTA's shared memory; the store counts its bytes as a completed transaction on the
+// peer's barrier bar_cluster when it lands (no fence is needed before the peer reads them after that barrier)
+__device__ __forceinline__ void st_async_v4(uint32_t dst_cluster, uint4 v, uint32_t bar_cluster) {
+  asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.b32 [%0], {%1, %2, %3, %4}, [%5];"
+               :: "r"(dst_cluster), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w), "r"(bar_cluster) : "memory");
 }
-__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
-// the bulk copies of all but the newest N committed groups have finished reading their sources
-template <int N>
-__device__ __forceinline__ void bulk_wait_read() {
-  asm volatile("cp.async.bulk.wait_group.read %0;" :: "n"(N) : "memory");
+__device__ __forceinline__ void st_async_b32(uint32_t dst_cluster, uint32_t v, uint32_t bar_cluster) {
+  asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.b32 [%0], %1, [%2];"
+               :: "r"(dst_cluster), "r"(v), "r"(bar_cluster) : "memory");
 }
 // arrive on a peer CTA's barrier and raise its expected transaction count.  Relaxed: the data this
-// announces arrives by a bulk copy whose transaction completion makes it visible; a release here would make
+// announces arrives by st.async stores whose transaction completion makes it visible; a release here would make
 // the thread wait for all of its earlier memory operations first (measured: about 1 us per tile)
 __device__ __forceinline__ void mbar_arrive_expect_tx_remote(uint32_t bar_cluster, uint32_t bytes) {
   asm volatile("mbarrier.arrive.expect_tx.relaxed.cluster.shared::cluster.b64 _, [%0], %1;"

@@ -406,8 +406,8 @@ dsa_status_t run_mla(const uint16_t* q, const uint16_t* c, long long S, const in
   const cuuint64_t cs[1] = {576 * 2};
   const cuuint32_t cb[2] = {64, 1};
   if (!make_map(&tc, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, c, cd, cs, cb, CU_TENSOR_MAP_SWIZZLE_128B)) return DSA_ERR_CUDA;
-  CUtensorMap tcd;  // contiguous tiles of c: one 64-column box 64 rows high (dense tokens)
-  const cuuint32_t cbd[2] = {64, 64};
+  CUtensorMap tcd;  // contiguous tiles of c: one 64-column box one key tile high (dense tokens)
+  const cuuint32_t cbd[2] = {64, static_cast<cuuint32_t>(mla::NK)};
   if (!make_map(&tcd, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, c, cd, cs, cbd, CU_TENSOR_MAP_SWIZZLE_128B))
     return DSA_ERR_CUDA;
   MlaParams p{};
@@ -465,7 +465,8 @@ dsa_status_t run_mla_causal(const uint16_t* q, const uint16_t* c, long long S, c
                  kl_out ? kl_out + n : nullptr);
 }
 
-bool mla_k_ok(int k) { return k >= 2 * mla::NK && k % mla::NK == 0 && k <= mla::KMAX; }
+// k: at least 128 and a multiple of 64 (slots of a last, half-filled 128-key tile are masked), at most KMAX
+bool mla_k_ok(int k) { return k >= 128 && k % 64 == 0 && k <= mla::KMAX; }
 
 bool indexer_shape_ok(int H_I, int d_I) { return (H_I == 64 && d_I == 128) || (H_I == 4 && d_I == 64); }
 

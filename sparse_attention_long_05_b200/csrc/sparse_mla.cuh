@@ -5,10 +5,9 @@
 // the M = 128 dimension of the MMAs and every gathered entry is reused by all heads.  The output of one token
 // (128 heads x 512 fp32) fills all 512 columns of one SM's tensor memory, leaving no room for the logits.
 // The work is therefore split by role across the two CTAs of a cluster, each on its own SM:
-//   score CTA (rank 0): keeps the token's queries in tensor memory, gathers the 576-dim selected rows,
-//     computes S = Q . C^T on tcgen05 (A from tensor memory, bf16 -> fp32), runs the online softmax (fp32,
-//     exp2 domain) and ships P (bf16) plus per-head rescale factors and row sums to the value CTA with one
-//     shared-to-shared bulk copy per 64-key tile;
+//   score CTA (rank 0): keeps the token's queries on chip, gathers the 576-dim selected rows, computes
+//     S = Q . C^T on tcgen05 (bf16 -> fp32), runs the online softmax (fp32, exp2 domain) and stores P (bf16)
+//     plus per-head rescale factors and row sums straight into the value CTA's shared memory;
 //   value CTA (rank 1): gathers the first 512 dims of the same rows, accumulates O += P . V on tcgen05 into
 //     its tensor memory (two N = 256 halves), rescales O rows when a head's running maximum jumps (lazy:
 //     only when the max grows by more than 2^8), and writes out = O / l in bf16.
@@ -16,26 +15,30 @@
 // logit or probability ever leaves the chip.
 //
 // Data movement.
+//   * Keys are processed in tiles of 128: the QK^T MMAs then have N = 128 (the tensor core ran the N = 64 ones
+//     of 64-key tiles at about 40 % of its rate).  The score CTA's tensor memory holds Q chunks 0..7 (128 heads
+//     x 64 dims each, 32 columns) in columns 0..255 and two 128-column S buffers, so the QK^T of tile g + 1
+//     runs while the softmax reads tile g's logits.  Q chunk 8 (the 64 position dims) is the A operand of its
+//     MMAs from shared memory (two buffers, one per token in flight).
 //   * Selected rows are gathered by TMA tile::gather4 (four rows x one 64-column, 128-byte swizzled box per
-//     instruction) into 64-key x 64-dim chunks in the K-major form the tensor core reads.  A pipeline stage
-//     holds several chunks of one 64-key tile (three in the score CTA, four in the value CTA), because the
+//     instruction) into 128-key x 64-dim chunks in the K-major form the tensor core reads.  A pipeline stage
+//     holds several chunks of one tile (three in the score CTA, four in the value CTA), because the
 //     issuing thread spends a few hundred cycles per stage on its barrier wait, the tcgen05 issue and the
-//     commit whatever the stage's size: with one 64-dim chunk per stage the QK^T MMA thread, not the tensor
-//     core, set the pace.  Each stage is split over eight gather warps (one warp issues gather4 only about
-//     every 50 ns; gather throughput per SM grows with the issuing warps: about 12, 24, 45 and 73 GB/s
-//     with 1, 2, 4 and 8), each of which arrives on the stage's barrier with its share of the bytes.  TMA
+//     commit whatever the stage's size.  Each stage is split over eight gather warps (one warp issues gather4
+//     only about every 50 ns; gather throughput per SM grows with the issuing warps: about 12, 24, 45 and 73
+//     GB/s with 1, 2, 4 and 8), each of which arrives on the stage's barrier with its share of the bytes.  TMA
 //     writes are in the async proxy, so the MMA warp consumes a stage as soon as its mbarrier completes,
 //     with no proxy fence.  The same chunk bytes serve as the K-major B operand of QK^T (rows = keys) and
 //     as the MN-major B operand of PV (rows = keys = K, 64 dims = N per atom; four chunks = N 256).
+//   * P goes to the value CTA by st.async stores from the softmax threads, each completing its bytes on the
+//     value CTA's P_FULL barrier: no staging buffer, and no bulk copy queued behind the gathers in the score
+//     SM's TMA unit (such a copy took about 1.2 us per tile there).
 //   * The token's selected-index row is prefetched into shared memory with one bulk copy.
-//   * Q chunks (128 heads x 64 dims) are staged by TMA (three shared-memory slots) and copied into a ring of
-//     twelve 32-column chunk slots of tensor memory with tcgen05.cp; chunk c of the token with running index
-//     ti lives in slot (9 ti + c) mod 12.  A copy may only overwrite a slot once the MMAs that last read it
-//     have completed, which the MMA thread learns from tcgen05.commit barriers: per token, the next token's
-//     chunks 0-2 are copied at the start of tile 1 (their slots held chunks 6-8 of the token before, retired),
-//     chunks 3-5 during the last tile, three chunks after the MMAs that last read those slots were committed,
-//     and chunks 6-8 during the next token's first tile, just before their first use.  No copy waits on an
-//     MMA issued less than three chunks earlier.
+//   * Q chunks 0..7 are staged by TMA (three shared-memory slots) and copied into tensor memory with
+//     tcgen05.cp.  A copy may only overwrite a slot once the MMAs that last read it have completed, which the
+//     MMA thread learns from tcgen05.commit barriers on the stages of a token's last tile: the next token's
+//     chunks 0-2 are copied during that tile, chunks 3-5 and 6-7 in the next token's first tile, just
+//     before the stages that read them.
 //
 // Warp roles (14 warps per CTA): w0 loader (index rows, Q chunks), w1 TMEM allocation + MMA issue (a
 // warp-uniform loop; one elected lane issues the tcgen05 instructions),
@@ -49,9 +52,9 @@ namespace dsa {
 // How a token's keys are found.  kMlaSparse: the k entries of its index row are gathered.  The dense modes
 // give each token the number n_t of keys its sequence shows it (positions 0..n_t-1, rows base..base+n_t-1 of
 // c); a token with n_t <= k then selects all of them, whatever its index row says, and its keys are read as
-// contiguous 64-row tiles, ceil(n_t / 64) of them, instead of k / 64 gathered tiles.  kMlaCausal: n_t = pos0 + t
-// - base + 1 (prefill rows at their positions, the launch's first row at position pos0); kMlaCounts: n_t =
-// n_keys[t] (decode tokens after the append).
+// contiguous 128-row tiles, ceil(n_t / 128) of them (at least one), instead of ceil(k / 128) gathered tiles.
+// kMlaCausal: n_t = pos0 + t - base + 1 (prefill rows at their positions, the launch's first row at position
+// pos0); kMlaCounts: n_t = n_keys[t] (decode tokens after the append).
 enum { kMlaSparse = 0, kMlaCausal = 1, kMlaCounts = 2 };
 
 struct MlaParams {
@@ -71,67 +74,77 @@ struct MlaParams {
   const float* kl_scores;
   float* kl_out;
   const int* page_table;       // paged c: [T, pt_stride] page of each page_rows positions of token t's keys, or null
-  int pt_stride, page_rows;    // (page_rows a multiple of 64: a 64-key tile lies in one page)
+  int pt_stride, page_rows;    // (page_rows a multiple of 128: a 128-key tile lies in one page)
   long long S;                 // rows of c
   float scale_log2;            // softmax scale * log2(e)
 };
 
 namespace mla {
-constexpr int NK = 64;                    // keys per tile
+// 128-key tiles: the QK^T MMAs have N = 128 (the tensor core ran N = 64 MMAs at about 40 % of its rate, N = 256
+// ones near the full rate).  Two 128-column S buffers fit in tensor memory beside eight of the nine Q chunks; the
+// ninth (the 64 position dims) is the A operand of its MMAs from shared memory.
+constexpr int NK = 128;                   // keys per tile
 constexpr int D = 576, DV = 512;
 constexpr int QCHUNKS = D / 64;           // 9
+constexpr int QTM = 8;                    // Q chunks in tensor memory (chunk 8 from shared memory)
 constexpr int VCHUNKS = DV / 64;          // 8
-constexpr int CHUNK_BYTES = NK * 128;     // 8 KB: 64 keys x 64 bf16
+constexpr int CHUNK_BYTES = NK * 128;     // 16 KB: 128 keys x 64 bf16
 constexpr int QCHUNK_BYTES = 128 * 128;   // 16 KB: 128 heads x 64 bf16
 constexpr int KMAX = 2048;                // largest selection handled (index row slot of 8 KB)
 constexpr int QS = 3;                     // Q staging slots (score CTA)
-constexpr int NSB = 2;                    // S buffers in tensor memory (score CTA)
-constexpr int QSLOTS = 12;                // Q chunk slots in tensor memory (score CTA)
-constexpr int NPB = 3;                    // P buffers (value CTA)
+constexpr int NPB = 2;                    // P buffers (value CTA)
 constexpr int SCH = 3, VCH = 4;           // 64-dim chunks per gather stage (score CTA, value CTA)
 constexpr int S_STAGE = SCH * CHUNK_BYTES, V_STAGE = VCH * CHUNK_BYTES;
-constexpr int SPT_S = QCHUNKS / SCH, SPT_V = VCHUNKS / VCH;   // stages per 64-key tile: 3, 2
-constexpr int NS_S = 5, NS_V = 4;         // gather stages per CTA
+constexpr int SPT_S = QCHUNKS / SCH, SPT_V = VCHUNKS / VCH;   // stages per 128-key tile: 3, 2
+constexpr int NS_S = 2, NS_V = 2;         // gather stages per CTA
 constexpr int THREADS = 448;
 constexpr int GATHER_WARPS = 8;
+constexpr int G4_PER_CHUNK = NK / 4;      // gather4 instructions per chunk (four rows each)
 constexpr float RESCALE_LOG2 = 8.0f;      // lazy rescale threshold (factor 256)
-constexpr int P_BYTES = 128 * 128;        // 128 heads x 64 keys bf16
-constexpr int XFER = P_BYTES + 512 + 512; // P + alpha[128] + lsum[128]
+constexpr int P_CHUNK = 128 * 128;        // one 64-key K chunk of P: 128 heads x 64 keys bf16
+constexpr int P_BYTES = 2 * P_CHUNK;      // 128 heads x 128 keys bf16
+constexpr int XFER = P_BYTES + 512 + 512; // P + alpha[128] + lsum[128]: the bytes of one tile to the value CTA
 constexpr uint32_t TMEM_COLS = 512;
-constexpr uint32_t TQ = 0;                // score CTA: Q chunk slots in columns 0..383
-constexpr uint32_t TS = 384;              // score CTA: S buffers at 384, 448
+constexpr uint32_t TQ = 0;                // score CTA: Q chunks 0..7 in columns 0..255
+constexpr uint32_t TS = 256;              // score CTA: S buffers in columns 256..383 and 384..511
 // barrier slots
 constexpr int B_IDX_FULL = 0, B_IDX_EMPTY = 2;
 constexpr int B_QST_FULL = 4, B_QST_EMPTY = B_QST_FULL + QS;
 constexpr int B_RING_FULL = B_QST_EMPTY + QS, B_RING_EMPTY = B_RING_FULL + 16;
-constexpr int B_S_FULL = B_RING_EMPTY + 16, B_S_EMPTY = B_S_FULL + NSB, B_P_EMPTY = B_S_EMPTY + NSB;
+constexpr int B_S_FULL = B_RING_EMPTY + 16, B_S_EMPTY = B_S_FULL + 2, B_P_EMPTY = B_S_EMPTY + 2;
 constexpr int B_P_FULL = B_P_EMPTY + NPB, B_P_READY = B_P_FULL + NPB;
 // O_DONE: one barrier per P buffer (PV of tile g completes O_DONE[g % NPB]); a single barrier would be waited
 // only now and then and could be two phases behind, where a parity test cannot tell the phases apart
 constexpr int B_O_DONE = B_P_READY + NPB, B_O_FREE = B_O_DONE + NPB;
-constexpr int B_SLOT_FREE = B_O_FREE + 1, B_SLOT_WRITTEN = B_SLOT_FREE + 1;   // score CTA softmax handshakes
-constexpr int B_QRET = B_SLOT_WRITTEN + 1;    // score CTA: last-tile MMAs of chunks 0..2 retired
-constexpr int B_QTOK = B_QRET + 1;            // score CTA: every MMA of a token retired
-constexpr int B_RED_FULL = B_QTOK + 1;        // KL mode: the four warps' head sums of a tile written (2 buffers)
+constexpr int B_QRET = B_O_FREE + 1;          // score CTA: stage s of a token's last tile retired (3 barriers)
+constexpr int B_ROPE_FULL = B_QRET + SPT_S;   // score CTA: Q chunk 8 of a token staged (2 buffers)
+constexpr int B_ROPE_EMPTY = B_ROPE_FULL + 2; // score CTA: every MMA reading a Q chunk 8 buffer retired
+constexpr int B_RED_FULL = B_ROPE_EMPTY + 2;  // KL mode: the four warps' head sums of a tile written (2 buffers)
 constexpr int B_RED_FREE = B_RED_FULL + 2;    // KL mode: the head sums of a tile read (2 buffers)
 constexpr int B_COUNT = B_RED_FREE + 2;
 // shared memory map (from a 1024-byte aligned base; both CTAs use the same barrier offsets)
 constexpr int OFF_TMEM = 8 * B_COUNT;
 constexpr int OFF_ABORT = OFF_TMEM + 4;
-constexpr int OFF_IDX = 2048;                                   // both: 2 x 8 KB index rows
-constexpr int OFF_PST = OFF_IDX + 2 * KMAX * 4;                 // score CTA: 2 P staging slots
-constexpr int OFF_QST = OFF_PST + 2 * XFER;                     // score CTA: Q staging
-constexpr int OFF_RING_S = OFF_QST + QS * QCHUNK_BYTES;         // score CTA: gather ring
+constexpr int OFF_IDX = 1024;                                   // both: 2 x 8 KB index rows
+constexpr int OFF_RED = OFF_IDX + 2 * KMAX * 4;                 // score CTA, KL mode: head sums [2][4][NK]
+constexpr int OFF_QST = OFF_RED + 2 * 4 * NK * 4;               // score CTA: Q staging
+constexpr int OFF_ROPE = OFF_QST + QS * QCHUNK_BYTES;           // score CTA: Q chunk 8, two buffers
+constexpr int OFF_RING_S = OFF_ROPE + 2 * QCHUNK_BYTES;         // score CTA: gather ring
 constexpr int OFF_PB = OFF_IDX + 2 * KMAX * 4;                  // value CTA: P buffers
 constexpr int OFF_RING_V = OFF_PB + NPB * XFER;                 // value CTA: gather ring
 constexpr int SMEM_S = OFF_RING_S + NS_S * S_STAGE;
 constexpr int SMEM_V = OFF_RING_V + NS_V * V_STAGE;
 constexpr int SMEM = (SMEM_S > SMEM_V ? SMEM_S : SMEM_V) + 1024;
-static_assert(OFF_TMEM + 8 <= OFF_IDX, "barrier area");
-static_assert(OFF_PST % 1024 == 0 && OFF_QST % 1024 == 0 && OFF_RING_S % 1024 == 0, "1 KB aligned tiles");
+static_assert(OFF_ABORT + 4 <= OFF_IDX, "barrier area");
+static_assert(OFF_QST % 1024 == 0 && OFF_ROPE % 1024 == 0 && OFF_RING_S % 1024 == 0, "1 KB aligned tiles");
 static_assert(OFF_PB % 1024 == 0 && XFER % 1024 == 0 && OFF_RING_V % 1024 == 0, "1 KB aligned tiles");
 static_assert(QCHUNKS % SCH == 0 && VCHUNKS % VCH == 0 && VCH * 64 == 256, "stage split");
-static_assert((SCH * 16) % GATHER_WARPS == 0 && (VCH * 16) % GATHER_WARPS == 0, "gather4 split over warps");
+static_assert(QTM == QCHUNKS - 1 && SPT_S == 3, "Q chunk 8 in the last score stage");
+static_assert(TQ + 32 * QTM <= TS && TS + 2 * NK <= TMEM_COLS, "tensor memory columns");
+static_assert((SCH * G4_PER_CHUNK) % GATHER_WARPS == 0 && (VCH * G4_PER_CHUNK) % GATHER_WARPS == 0,
+              "gather4 split over warps");
+static_assert((SCH * G4_PER_CHUNK) / GATHER_WARPS <= 32 && (VCH * G4_PER_CHUNK) / GATHER_WARPS <= 32,
+              "one gather4 per lane");
 static_assert(NS_S <= 16 && NS_V <= 16, "ring barrier slots");
 static_assert(SMEM <= 232448, "shared memory per CTA");
 }  // namespace mla
@@ -181,10 +194,31 @@ __device__ __forceinline__ int mla_dense_keys(const MlaParams& p, int t, long lo
     return n > 0 ? static_cast<int>(n) : 0;
   }
 }
-// 64-key tiles of a token: k / 64 gathered tiles, or the tiles holding its n_t dense keys (at least two: the
-// score CTA's schedule of Q-chunk copies needs a second tile; a tile past n_t is wholly masked)
+// Which of the 128 keys of tile j of token t enter the softmax, as four warp-uniform ballots: lane l tests the keys
+// in slots j NK + 4 l .. + 3, and key i of the tile is valid iff bit i / 4 of msk[i % 4] is set.  A gathered token's
+// key is valid when its slot is below k and its entry names a row of c; a dense token's when its position is below n_t.
+template <bool DENSE, bool PAGED>
+__device__ __forceinline__ void mla_tile_masks(const MlaParams& p, int t, const int* ids, long long base, int nd, int j,
+                                               int lane, uint32_t (&msk)[4]) {
+  const int slot = j * mla::NK + 4 * lane;
+  bool v[4];
+  if (nd < 0) {
+    const int4 e = (slot < p.k) ? *reinterpret_cast<const int4*>(ids + slot) : make_int4(-1, -1, -1, -1);
+    v[0] = mla_valid<PAGED>(p, t, e.x, base);
+    v[1] = mla_valid<PAGED>(p, t, e.y, base);
+    v[2] = mla_valid<PAGED>(p, t, e.z, base);
+    v[3] = mla_valid<PAGED>(p, t, e.w, base);
+  } else {
+#pragma unroll
+    for (int u = 0; u < 4; ++u) v[u] = slot + u < nd;
+  }
+#pragma unroll
+  for (int u = 0; u < 4; ++u) msk[u] = __ballot_sync(0xffffffffu, v[u]);
+}
+// 128-key tiles of a token: the tiles holding its k selection slots, or its n_t dense keys (at least one; slots past
+// k or keys past n_t are masked)
 __device__ __forceinline__ int mla_tiles(const MlaParams& p, int nd) {
-  return nd < 0 ? p.k / mla::NK : max(2, (nd + mla::NK - 1) / mla::NK);
+  return max(1, ((nd < 0 ? p.k : nd) + mla::NK - 1) / mla::NK);
 }
 
 // position in a ring of `size` stages (size known at run time): stage index and pass parity, advanced
@@ -239,12 +273,10 @@ sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     }
     if (rank == 0) {
       for (int i = 0; i < QS; ++i) { mbar_init(bar(B_QST_FULL + i), 1); mbar_init(bar(B_QST_EMPTY + i), 1); }
-      for (int i = 0; i < NSB; ++i) { mbar_init(bar(B_S_FULL + i), 1); mbar_init(bar(B_S_EMPTY + i), 4); }
+      for (int i = 0; i < 2; ++i) { mbar_init(bar(B_S_FULL + i), 1); mbar_init(bar(B_S_EMPTY + i), 4); }
       for (int i = 0; i < NPB; ++i) mbar_init(bar(B_P_EMPTY + i), 1);
-      mbar_init(bar(B_SLOT_FREE), 1);
-      mbar_init(bar(B_SLOT_WRITTEN), 4);
-      mbar_init(bar(B_QRET), 1);
-      mbar_init(bar(B_QTOK), 1);
+      for (int i = 0; i < SPT_S; ++i) mbar_init(bar(B_QRET + i), 1);
+      for (int i = 0; i < 2; ++i) { mbar_init(bar(B_ROPE_FULL + i), 1); mbar_init(bar(B_ROPE_EMPTY + i), 1); }
       for (int i = 0; i < 2; ++i) { mbar_init(bar(B_RED_FULL + i), 4); mbar_init(bar(B_RED_FREE + i), 1); }
     } else {
       for (int i = 0; i < NPB; ++i) { mbar_init(bar(B_P_FULL + i), 1); mbar_init(bar(B_P_READY + i), 4); }
@@ -277,8 +309,8 @@ sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     if (lane == 0) {
       int qn = 0, ti = 0;
       bool ok = true;
-      int idx_issued = 0, q_issued = 0;
-      uint32_t idx_par[2] = {0, 0}, q_par[QS] = {};
+      int idx_issued = 0, q_issued = 0, rope_issued = 0;
+      uint32_t idx_par[2] = {0, 0}, q_par[QS] = {}, rope_par[2] = {0, 0};
       for (int t = cluster; t < p.T && ok; t += nclusters, ++ti) {
         const int is = ti & 1;
         if (!(ok = mbar_wait(bar(B_IDX_EMPTY + is), ((ti >> 1) & 1) ^ 1, abort_flag))) break;
@@ -288,7 +320,15 @@ sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         idx_par[is] = (ti >> 1) & 1;
         ++idx_issued;
         if (rank == 0) {
-          for (int c = 0; c < QCHUNKS; ++c, ++qn) {
+          // chunk 8 (the position dims) into its own buffer, read by the MMAs from shared memory
+          const int rb = ti & 1;
+          if (!(ok = mbar_wait(bar(B_ROPE_EMPTY + rb), ((ti >> 1) & 1) ^ 1, abort_flag))) break;
+          mbar_arrive_expect_tx(bar(B_ROPE_FULL + rb), QCHUNK_BYTES);
+          tma_load_3d(sbase + OFF_ROPE + rb * QCHUNK_BYTES, &tm_q, bar(B_ROPE_FULL + rb), 64 * QTM, 0, t);
+          rope_par[rb] = (ti >> 1) & 1;
+          ++rope_issued;
+          // chunks 0..7 through the staging slots, copied into tensor memory by the MMA warp
+          for (int c = 0; c < QTM; ++c, ++qn) {
             const int qs = qn % QS;
             if (!(ok = mbar_wait(bar(B_QST_EMPTY + qs), ((qn / QS) & 1) ^ 1, abort_flag))) break;
             mbar_arrive_expect_tx(bar(B_QST_FULL + qs), QCHUNK_BYTES);
@@ -301,14 +341,15 @@ sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
       if (*abort_flag) {
         for (int i = 0; i < 2 && i < idx_issued; ++i) mbar_wait_drain(bar(B_IDX_FULL + i), idx_par[i]);
         for (int i = 0; i < QS && i < q_issued; ++i) mbar_wait_drain(bar(B_QST_FULL + i), q_par[i]);
+        for (int i = 0; i < 2 && i < rope_issued; ++i) mbar_wait_drain(bar(B_ROPE_FULL + i), rope_par[i]);
       }
     }
   } else if (warp == 2 || warp == 3 || warp >= 8) {
     // ===================================================================== gathers (TMA gather4)
-    // Every stage is split over the eight gather warps: gather4 instruction i of a stage (i = 16 cc + rg)
+    // Every stage is split over the eight gather warps: gather4 instruction i of a stage (i = 32 cc + rg)
     // fetches rows 4 rg .. 4 rg + 3 of the tile into its chunk cc; warp gw issues instructions
-    // gw * per_warp .. + per_warp - 1, one per lane.  A dense token's full tiles are 64 contiguous rows: lane c
-    // of gather warp 0 loads its chunk c as one 64 x 64 box, and the other warps arrive with no bytes.  Its
+    // gw * per_warp .. + per_warp - 1, one per lane.  A dense token's full tiles are 128 contiguous rows: lane c
+    // of gather warp 0 loads its chunk c as one 64 x 128 box, and the other warps arrive with no bytes.  Its
     // last, partial tile is gathered, its masked slots reading the token's last key row: the rows after the
     // sequence's last key may be memory the caller never wrote, and a NaN there would survive the zero
     // probability in P . V.
@@ -316,9 +357,9 @@ sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     const int cps = (rank == 0) ? SCH : VCH;               // chunks per stage
     const int spt = (rank == 0) ? SPT_S : SPT_V;           // stages per tile
     const uint32_t sbytes = cps * CHUNK_BYTES;
-    const int per_warp = cps * 16 / GATHER_WARPS;          // 6 or 8
+    const int per_warp = cps * G4_PER_CHUNK / GATHER_WARPS; // 12 or 16
     const int gi = gw * per_warp + lane;
-    const int cc = gi >> 4, rg = gi & 15;
+    const int cc = gi / G4_PER_CHUNK, rg = gi % G4_PER_CHUNK;
     const bool active = lane < per_warp;
     RingPos rp;
     rp.size = nsr;
@@ -334,13 +375,14 @@ sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
       const int nd = mla_dense_keys<DENSE>(p, t, base);
       const int ntiles = mla_tiles(p, nd);
       for (int j = 0; j < ntiles && ok; ++j) {
-        const bool full_dense = nd >= 0 && (j + 1) * NK <= nd;    // 64 contiguous rows of keys
+        const bool full_dense = nd >= 0 && (j + 1) * NK <= nd;    // 128 contiguous rows of keys
         const uint32_t tx = full_dense ? (gw == 0 ? sbytes : 0) : per_warp * 512;
         int r[4] = {0, 0, 0, 0};
         if (active && !full_dense) {
           const int slot = j * NK + 4 * rg;
           if (nd < 0) {
-            const int4 e = reinterpret_cast<const int4*>(ids + j * NK)[rg];
+            // slots past the token's k entries (a k that is not a multiple of the tile) are padding
+            const int4 e = (slot < p.k) ? *reinterpret_cast<const int4*>(ids + slot) : make_int4(-1, -1, -1, -1);
             r[0] = static_cast<int>(mla_row<PAGED>(p, t, e.x, base, slot));
             r[1] = static_cast<int>(mla_row<PAGED>(p, t, e.y, base, slot + 1));
             r[2] = static_cast<int>(mla_row<PAGED>(p, t, e.z, base, slot + 2));
@@ -396,89 +438,88 @@ sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     rp.size = nsr;
     int ti = 0;
     if (rank == 0) {
+      // Q chunks 0..7 of a token live in tensor-memory slots 0..7, chunk 8 in its shared-memory buffer (ti % 2).
+      // A copy overwrites a slot only after the MMAs that last read it have completed (tcgen05.commit barriers
+      // QRET[s], stage s of a token's last tile): the next token's chunks 0..2 are copied during the last tile,
+      // after the stage that follows stage 0 (stage 2 for a one-tile token, so that chunks leave the staging
+      // slots in order), chunks 3..5 and 6..7 in its own first tile, just before stages 1 and 2 read them.
       constexpr uint32_t idesc = idesc_bf16(128, NK, false);
-      int qn = 0;          // Q chunks copied into tensor memory so far (= 9 * token index + chunk)
-      // copy the next staged Q chunk (global chunk index qn) into its tensor-memory slot
-      auto copy_q = [&]() -> bool {
-        const int qs = qn % QS;
-        if (!warp_wait(bar(B_QST_FULL + qs), (qn / QS) & 1, abort_flag)) return false;
-        tc_fence_after();
-        const uint32_t src = sbase + OFF_QST + qs * QCHUNK_BYTES;
-        const uint32_t dst = tmem + TQ + 32 * (qn % QSLOTS);
-        if (elect_one()) {
+      int qn = 0;          // Q chunks copied into tensor memory so far (= 8 * token index + chunk)
+      // copy the next `n` staged Q chunks (global chunk index qn ...) into their tensor-memory slots
+      auto copy_q = [&](int n) -> bool {
+        for (int i = 0; i < n; ++i, ++qn) {
+          const int qs = qn % QS;
+          if (!warp_wait(bar(B_QST_FULL + qs), (qn / QS) & 1, abort_flag)) return false;
+          tc_fence_after();
+          const uint32_t src = sbase + OFF_QST + qs * QCHUNK_BYTES;
+          const uint32_t dst = tmem + TQ + 32 * (qn % QTM);
+          if (elect_one()) {
 #pragma unroll
-          for (int s = 0; s < 4; ++s) tmem_cp_128x256b(dst + 8 * s, smem_desc(src + 32 * s, 16, 1024, kLayoutSW128));
-          mma_commit(bar(B_QST_EMPTY + qs));
+            for (int s = 0; s < 4; ++s) tmem_cp_128x256b(dst + 8 * s, smem_desc(src + 32 * s, 16, 1024, kLayoutSW128));
+            mma_commit(bar(B_QST_EMPTY + qs));
+          }
+          __syncwarp();
         }
-        __syncwarp();
-        ++qn;
         return true;
       };
       int nret = 0;        // tokens whose last tile committed the QRET barriers
-      if (cluster < p.T)
-        for (int c = 0; c < QCHUNKS && ok; ++c) ok = copy_q();
+      if (cluster < p.T) ok = copy_q(QTM);
       for (int t = cluster; t < p.T && ok; t += nclusters, ++ti) {
         const bool has_next = t + nclusters < p.T;
-        const uint32_t prev_tok = static_cast<uint32_t>((ti - 1) & 1);   // parity of the previous token's QTOK
-        const int q_slot0 = (9 * ti) % QSLOTS;                          // tensor-memory slot of chunk 0
+        const int rb = ti & 1;
         const int ntiles = mla_tiles(p, mla_dense_keys<DENSE>(p, t, p.row_off ? p.row_off[t] : 0));
         for (int j = 0; j < ntiles && ok; ++j, ++g) {
-          const int sb = g % NSB;
-          if (j == 1 && has_next) {
-            // next token's chunks 0..2 go to the slots of the previous token's chunks 6..8
-            if (ti > 0 && !(ok = warp_wait(bar(B_QTOK), prev_tok, abort_flag))) break;
-            for (int c = 0; c < 3 && ok; ++c) ok = copy_q();
-            if (!ok) break;
-          }
-          if (!(ok = warp_wait(bar(B_S_EMPTY + sb), static_cast<uint32_t>((g / NSB) & 1) ^ 1, abort_flag))) break;
+          const int sb = static_cast<int>(g & 1);
+          const bool last = (j == ntiles - 1);
+          if (!(ok = warp_wait(bar(B_S_EMPTY + sb), static_cast<uint32_t>((g >> 1) & 1) ^ 1, abort_flag))) break;
           DSA_TRACE_EVENT(2, g);
           tc_fence_after();
-          const bool last = (j == ntiles - 1) && has_next;
           for (int s = 0; s < SPT_S && ok; ++s, rp.advance()) {
             const int st = rp.stage;
+            if (j == 0 && s > 0 && ti > 0) {
+              // this token's chunks 3s .. 3s + 2 (6, 7) replace the previous token's, read last by its stage s
+              if (!(ok = warp_wait(bar(B_QRET + s), static_cast<uint32_t>((nret - 1) & 1), abort_flag))) break;
+              if (!(ok = copy_q(s == 1 ? 3 : 2))) break;
+            }
+            if (j == 0 && s == SPT_S - 1 &&
+                !(ok = warp_wait(bar(B_ROPE_FULL + rb), static_cast<uint32_t>((ti >> 1) & 1), abort_flag)))
+              break;
             if (!(ok = warp_wait(bar(B_RING_FULL + st), rp.phase, abort_flag))) break;
             DSA_TRACE_EVENT(12 + s, g);
             tc_fence_after();
-            if (j == 0 && s == SPT_S - 1 && ti > 0) {
-              // this token's chunks 6..8 go to the slots of the previous token's chunks 3..5
-              if (!(ok = warp_wait(bar(B_QTOK), prev_tok, abort_flag))) break;
-              for (int c = 0; c < 3 && ok; ++c) ok = copy_q();
-              if (!ok) break;
-            }
             // the stage's three chunks: 12 MMAs issued as one block, then one commit
             const uint64_t bd = smem_desc(ring + st * S_STAGE, 16, 1024, kLayoutSW128);
-            int slot = q_slot0 + s * SCH;
-            if (slot >= QSLOTS) slot -= QSLOTS;
+            const uint64_t rd = smem_desc(sbase + OFF_ROPE + rb * QCHUNK_BYTES, 16, 1024, kLayoutSW128);
             if (elect_one()) {
 #pragma unroll
               for (int cc = 0; cc < SCH; ++cc) {
-                const uint32_t a = tmem + TQ + 32 * (slot + cc < QSLOTS ? slot + cc : slot + cc - QSLOTS);
+                const int qc = s * SCH + cc;
+                const uint64_t b = bd + ((cc * CHUNK_BYTES) >> 4);
 #pragma unroll
-                for (int k = 0; k < 4; ++k)   // K = 16 bf16 per instruction: 8 TMEM columns of A, 32 bytes of B
-                  mma_bf16_ts(tmem + TS + NK * sb, a + 8 * k, bd + ((cc * CHUNK_BYTES) >> 4) + 2 * k, idesc,
-                              (s | cc | k) ? 1u : 0u);
+                for (int k = 0; k < 4; ++k) {  // K = 16 bf16 per instruction: 8 TMEM columns / 32 bytes of A, 32 bytes of B
+                  const uint32_t acc = (s | cc | k) ? 1u : 0u;
+                  if (qc < QTM) mma_bf16_ts(tmem + TS + NK * sb, tmem + TQ + 32 * qc + 8 * k, b + 2 * k, idesc, acc);
+                  else mma_bf16_ss(tmem + TS + NK * sb, rd + 2 * k, b + 2 * k, idesc, acc);
+                }
               }
               mma_commit(bar(B_RING_EMPTY + st));
-              if (last && s == 0) mma_commit(bar(B_QRET));   // chunks 0..2 of this token retire
+              if (last && has_next) mma_commit(bar(B_QRET + s));
+              if (last && s == SPT_S - 1) mma_commit(bar(B_ROPE_EMPTY + rb));
             }
             __syncwarp();
             DSA_TRACE_EVENT(9 + s, g);
-            if (last && s == 1) {
-              // the next token's chunks 3..5 overwrite this token's chunks 0..2
+            if (last && has_next && s == (j == 0 ? SPT_S - 1 : 1)) {
+              // the next token's chunks 0..2 overwrite this token's, read last by this tile's stage 0
               if (!(ok = warp_wait(bar(B_QRET), static_cast<uint32_t>(nret & 1), abort_flag))) break;
-              for (int c = 0; c < 3 && ok; ++c) ok = copy_q();
-              if (!ok) break;
+              if (!(ok = copy_q(3))) break;
             }
           }
           if (!ok) break;
-          if (last) ++nret;
+          if (last && has_next) ++nret;
           DSA_TRACE_EVENT(3, g);
           if (elect_one()) mma_commit(bar(B_S_FULL + sb));
           __syncwarp();
         }
-        if (!ok) break;
-        if (elect_one()) mma_commit(bar(B_QTOK));
-        __syncwarp();
       }
     } else {
       constexpr uint32_t idesc = idesc_bf16(128, 256, true);
@@ -490,18 +531,20 @@ sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
           if (!(ok = warp_wait(bar(B_P_READY + pb), static_cast<uint32_t>((g / NPB) & 1), abort_flag))) break;
           DSA_TRACE_EVENT(20, g);
           tc_fence_after();
+          // P: two K-major chunks of 64 keys (128 heads x 128 bytes each, P_CHUNK apart)
           const uint64_t ad = smem_desc(sbase + OFF_PB + pb * XFER, 16, 1024, kLayoutSW128);
           for (int hh = 0; hh < SPT_V; ++hh, rp.advance()) {
             const int st = rp.stage;
             if (!(ok = warp_wait(bar(B_RING_FULL + st), rp.phase, abort_flag))) break;
             DSA_TRACE_EVENT(21 + hh, g);
             tc_fence_after();
-            // MN-major V: 64-dim chunks 8 KB apart (LBO), 8-key row groups 1 KB apart (SBO)
+            // MN-major V: 64-dim chunks 16 KB apart (LBO), 8-key row groups 1 KB apart (SBO)
             const uint64_t bd = smem_desc(ring + st * V_STAGE, CHUNK_BYTES, 1024, kLayoutSW128);
             if (elect_one()) {
 #pragma unroll
-              for (int k = 0; k < 4; ++k)     // 16 keys per instruction: two 8-key groups = 2 KB of V
-                mma_bf16_ss(tmem + 256 * hh, ad + 2 * k, bd + ((k * 2048) >> 4), idesc, (j == 0 && k == 0) ? 0u : 1u);
+              for (int k = 0; k < NK / 16; ++k)   // 16 keys per instruction: two 8-key groups = 2 KB of V
+                mma_bf16_ss(tmem + 256 * hh, ad + (((k >> 2) * P_CHUNK) >> 4) + 2 * (k & 3), bd + ((k * 2048) >> 4),
+                            idesc, (j == 0 && k == 0) ? 0u : 1u);
               mma_commit(bar(B_RING_EMPTY + st));
             }
             __syncwarp();
@@ -518,14 +561,15 @@ sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     }
   } else if constexpr (KL) {
     // ===================================================================== KL objective (warps 4..7)
-    // Per tile: each thread (one head) forms its head's probabilities of the tile's 64 keys from the logits and the
-    // head's lse; a halving exchange sums them over the warp's 32 heads (lane l ends with keys 2 l, 2 l + 1), and
-    // warp 4 adds the four warps' sums (handed over through double-buffered shared memory under mbarriers) and
-    // accumulates the token's sums of a log a, a I, a and the log-sum-exp of I over the valid keys.
+    // Per tile, in two halves of 64 keys: each thread (one head) forms its head's probabilities of the half's keys
+    // from the logits and the head's lse; a halving exchange sums them over the warp's 32 heads (lane l ends with
+    // keys 2 l, 2 l + 1 of the half), and warp 4 adds the four warps' sums (handed over through double-buffered
+    // shared memory under mbarriers) and accumulates the token's sums of a log a, a I, a and the log-sum-exp of I
+    // over the valid keys.
     const int quad = warp & 3;
     const int h = quad * 32 + lane;
     const uint32_t lane_addr = static_cast<uint32_t>(quad * 32) << 16;
-    float* red = reinterpret_cast<float*>(smem + OFF_PST);     // [2 buffers][4 warps][64 keys]
+    float* red = reinterpret_cast<float*>(smem + OFF_RED);     // [2 buffers][4 warps][NK keys]
     constexpr float kLog2e = 1.4426950408889634f, kLn2 = 0.69314718055994531f;
     int g = 0;
     int ti = 0;
@@ -542,39 +586,37 @@ sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
       const float inv_h = 1.f / static_cast<float>(p.H);
       float s_alog = 0.f, s_ai = 0.f, s_a = 0.f, m_i = -INFINITY, z_i = 0.f;   // warp 4, per lane
       for (int j = 0; j < ntiles && ok; ++j, ++g) {
-        const int sb = static_cast<int>(g % NSB), b = static_cast<int>(g & 1);
+        const int b = static_cast<int>(g & 1);     // S buffer and head-sum buffer of the tile
         const uint32_t use = static_cast<uint32_t>((g >> 1) & 1);
-        bool v_even, v_odd;
-        if (nd < 0) {
-          const int2 e = reinterpret_cast<const int2*>(ids + j * NK)[lane];
-          v_even = mla_valid<PAGED>(p, t, e.x, base);
-          v_odd = mla_valid<PAGED>(p, t, e.y, base);
-        } else {
-          v_even = j * NK + 2 * lane < nd;
-          v_odd = j * NK + 2 * lane + 1 < nd;
-        }
-        const uint32_t m_even = __ballot_sync(0xffffffffu, v_even);
-        const uint32_t m_odd = __ballot_sync(0xffffffffu, v_odd);
-        if (!(ok = warp_wait(bar(B_S_FULL + sb), static_cast<uint32_t>((g / NSB) & 1), abort_flag))) break;
+        uint32_t msk[4];   // key i of the tile enters the sums iff bit i / 4 of msk[i % 4] is set
+        mla_tile_masks<DENSE, PAGED>(p, t, ids, base, nd, j, lane, msk);
+        if (!(ok = warp_wait(bar(B_S_FULL + b), use, abort_flag))) break;
         tc_fence_after();
-        uint32_t v[64];
-        {
-          uint32_t (&v0)[32] = *reinterpret_cast<uint32_t(*)[32]>(&v[0]);
-          uint32_t (&v1)[32] = *reinterpret_cast<uint32_t(*)[32]>(&v[32]);
-          tmem_ld32(lane_addr + tmem + TS + NK * sb, v0);
-          tmem_ld32(lane_addr + tmem + TS + NK * sb + 32, v1);
-        }
-        tmem_wait_ld();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(bar(B_S_EMPTY + sb));
-        float x[64];
+        if (!(ok = warp_wait(bar(B_RED_FREE + b), use ^ 1u, abort_flag))) break;
+        float* rb = red + b * 4 * NK;
 #pragma unroll
-        for (int i = 0; i < NK; ++i) {
-          const bool valid = ((i & 1) ? (m_odd >> (i >> 1)) : (m_even >> (i >> 1))) & 1u;
-          x[i] = (valid && head_on) ? ex2_approx(fmaf(__uint_as_float(v[i]), p.scale_log2, -lse2)) : 0.f;
-        }
-        // sum over the warp's heads: five halving steps, each lane keeping the half its lane bit selects
+        for (int hq = 0; hq < 2; ++hq) {
+          uint32_t v[64];
+          {
+            uint32_t (&v0)[32] = *reinterpret_cast<uint32_t(*)[32]>(&v[0]);
+            uint32_t (&v1)[32] = *reinterpret_cast<uint32_t(*)[32]>(&v[32]);
+            tmem_ld32(lane_addr + tmem + TS + NK * b + 64 * hq, v0);
+            tmem_ld32(lane_addr + tmem + TS + NK * b + 64 * hq + 32, v1);
+          }
+          tmem_wait_ld();
+          if (hq == 1) {
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar(B_S_EMPTY + b));
+          }
+          float x[64];
+#pragma unroll
+          for (int i = 0; i < 64; ++i) {
+            const int key = 64 * hq + i;
+            const bool valid = (msk[key & 3] >> (key >> 2)) & 1u;
+            x[i] = (valid && head_on) ? ex2_approx(fmaf(__uint_as_float(v[i]), p.scale_log2, -lse2)) : 0.f;
+          }
+          // sum over the warp's heads: five halving steps, each lane keeping the half its lane bit selects
 #define DSA_KL_HALVE(O, N)                                                              \
   {                                                                                     \
     const bool up = (lane & (O)) != 0;                                                  \
@@ -584,24 +626,26 @@ sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
       x[i] = keep + __shfl_xor_sync(0xffffffffu, send, (O));                            \
     }                                                                                   \
   }
-        DSA_KL_HALVE(16, 32)
-        DSA_KL_HALVE(8, 16)
-        DSA_KL_HALVE(4, 8)
-        DSA_KL_HALVE(2, 4)
-        DSA_KL_HALVE(1, 2)
+          DSA_KL_HALVE(16, 32)
+          DSA_KL_HALVE(8, 16)
+          DSA_KL_HALVE(4, 8)
+          DSA_KL_HALVE(2, 4)
+          DSA_KL_HALVE(1, 2)
 #undef DSA_KL_HALVE
-        if (!(ok = warp_wait(bar(B_RED_FREE + b), use ^ 1u, abort_flag))) break;
-        float* rb = red + b * 4 * NK;
-        rb[quad * NK + 2 * lane] = x[0];
-        rb[quad * NK + 2 * lane + 1] = x[1];
+          rb[quad * NK + 64 * hq + 2 * lane] = x[0];
+          rb[quad * NK + 64 * hq + 2 * lane + 1] = x[1];
+        }
         __syncwarp();
         if (lane == 0) mbar_arrive(bar(B_RED_FULL + b));
         if (warp == 4) {
           if (!(ok = warp_wait(bar(B_RED_FULL + b), use, abort_flag))) break;
 #pragma unroll
-          for (int u = 0; u < 2; ++u) {
-            const int key = 2 * lane + u;
-            const bool valid = ((u ? m_odd : m_even) >> lane) & 1u;
+          for (int u = 0; u < 4; ++u) {
+            // key 64 hq + 2 lane + e of the tile (u = 2 hq + e): its bit is lane / 2 + 16 hq of msk[2 (lane % 2) + e]
+            const int hq = u >> 1, e = u & 1;
+            const int key = 64 * hq + 2 * lane + e;
+            const uint32_t mw = (lane & 1) ? msk[2 + e] : msk[e];
+            const bool valid = (mw >> (16 * hq + (lane >> 1))) & 1u;
             const float a = (rb[key] + rb[NK + key] + rb[2 * NK + key] + rb[3 * NK + key]) * inv_h;
             if (valid) {
               const float iv = p.kl_scores[static_cast<long long>(t) * p.k + j * NK + key];
@@ -647,6 +691,11 @@ sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     }
   } else if (rank == 0) {
     // ===================================================================== softmax (score CTA, warps 4..7)
+    // Per tile: pass 1 reads the 128 logits of each head from tensor memory in two halves and takes the tile's
+    // maximum; pass 2 forms the probabilities of the second half from the registers still holding it, reads the
+    // first half again (after which the S buffer is released to the QK^T two tiles on), and stores P as bf16
+    // straight into the value CTA's P buffer with st.async, each store completing its bytes on that CTA's P_FULL
+    // barrier (no staging copy, and nothing queued behind the gathers in this SM's TMA unit).
     const int quad = warp & 3;
     const int h = quad * 32 + lane;
     const bool leader = (warp == 4 && lane == 0);
@@ -667,48 +716,37 @@ sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
       // le: sum of the unrounded probabilities (for the log-sum-exp output)
       float m_ref = -INFINITY, l = 0.f, le = 0.f;
       for (int j = 0; j < ntiles && ok; ++j, ++g) {
-        const int sb = static_cast<int>(g % NSB), pb = static_cast<int>(g % NPB), b = static_cast<int>(g & 1);
-        // keys of the tile that enter the softmax: valid index entries, or dense positions below n_t
-        bool v_even, v_odd;
-        if (nd < 0) {
-          const int2 e = reinterpret_cast<const int2*>(ids + j * NK)[lane];
-          v_even = mla_valid<PAGED>(p, t, e.x, base);
-          v_odd = mla_valid<PAGED>(p, t, e.y, base);
-        } else {
-          v_even = j * NK + 2 * lane < nd;
-          v_odd = j * NK + 2 * lane + 1 < nd;
-        }
-        const uint32_t m_even = __ballot_sync(0xffffffffu, v_even);
-        const uint32_t m_odd = __ballot_sync(0xffffffffu, v_odd);
-        if (!(ok = warp_wait(bar(B_S_FULL + sb), static_cast<uint32_t>((g / NSB) & 1), abort_flag))) break;
+        const int sb = static_cast<int>(g & 1), pb = static_cast<int>(g % NPB);
+        const uint32_t s_tmem = lane_addr + tmem + TS + NK * sb;
+        uint32_t msk[4];   // key i of the tile is valid iff bit i / 4 of msk[i % 4] is set
+        mla_tile_masks<DENSE, PAGED>(p, t, ids, base, nd, j, lane, msk);
+        const bool full_tile = (msk[0] & msk[1] & msk[2] & msk[3]) == 0xffffffffu;
+        if (!(ok = warp_wait(bar(B_S_FULL + sb), static_cast<uint32_t>((g >> 1) & 1), abort_flag))) break;
         if (leader) DSA_TRACE_EVENT(4, g);
         tc_fence_after();
         uint32_t v[64];
-        {
-          uint32_t (&v0)[32] = *reinterpret_cast<uint32_t(*)[32]>(&v[0]);
-          uint32_t (&v1)[32] = *reinterpret_cast<uint32_t(*)[32]>(&v[32]);
-          tmem_ld32(lane_addr + tmem + TS + NK * sb, v0);
-          tmem_ld32(lane_addr + tmem + TS + NK * sb + 32, v1);
-        }
-        tmem_wait_ld();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(bar(B_S_EMPTY + sb));
-        if (leader) DSA_TRACE_EVENT(24, g);
-        // running max over the valid keys of the tile (raw logits; the scale is positive), as a 4-way tree
-        const bool full_tile = (m_even & m_odd) == 0xffffffffu;
-        float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-        if (full_tile) {
+        uint32_t (&v0)[32] = *reinterpret_cast<uint32_t(*)[32]>(&v[0]);
+        uint32_t (&v1)[32] = *reinterpret_cast<uint32_t(*)[32]>(&v[32]);
+        // masked keys become -inf (their probability is then 0)
+        auto mask_half = [&](int hq) {
 #pragma unroll
-          for (int i = 0; i < NK; ++i) mx[i & 3] = fmaxf(mx[i & 3], __uint_as_float(v[i]));
-        } else {
-#pragma unroll
-          for (int i = 0; i < NK; ++i) {
-            const bool valid = ((i & 1) ? (m_odd >> (i >> 1)) : (m_even >> (i >> 1))) & 1u;
-            if (!valid) v[i] = __float_as_uint(-INFINITY);
-            mx[i & 3] = fmaxf(mx[i & 3], __uint_as_float(v[i]));
+          for (int i = 0; i < 64; ++i) {
+            const int key = 64 * hq + i;
+            if (!((msk[key & 3] >> (key >> 2)) & 1u)) v[i] = __float_as_uint(-INFINITY);
           }
+        };
+        // pass 1: running max over the valid keys (raw logits; the scale is positive), as a 4-way tree
+        float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+        for (int hq = 0; hq < 2; ++hq) {
+          tmem_ld32(s_tmem + 64 * hq, v0);
+          tmem_ld32(s_tmem + 64 * hq + 32, v1);
+          tmem_wait_ld();
+          if (!full_tile) mask_half(hq);
+#pragma unroll
+          for (int i = 0; i < 64; ++i) mx[i & 3] = fmaxf(mx[i & 3], __uint_as_float(v[i]));
         }
+        if (leader) DSA_TRACE_EVENT(24, g);
         const float mraw = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
         const float mt = (mraw == -INFINITY) ? -INFINITY : mraw * p.scale_log2;
         float alpha = 1.f;
@@ -718,70 +756,59 @@ sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
           le *= alpha;
           m_ref = mt;
         }
-        // p = 2^(x * scale_log2 - m_ref) as one FMA + ex2; masked keys (-inf) give 0
+        // the value CTA's P buffer pb is free once its PV of tile g - NPB has completed
+        if (!(ok = warp_wait<true>(bar(B_P_EMPTY + pb), static_cast<uint32_t>((g / NPB) & 1) ^ 1, abort_flag))) break;
+        if (leader) {
+          DSA_TRACE_EVENT(7, g);
+          mbar_arrive_expect_tx_remote(pfull_remote + 8 * pb, XFER);
+        }
+        const uint32_t dst = pb_remote + pb * XFER, fb = pfull_remote + 8 * pb;
+        // p = 2^(x * scale_log2 - m_ref) as one FMA + ex2, stored as one 64-key K chunk of P (128-byte swizzled
+        // rows: 16-byte unit c of head h at unit c ^ (h % 8))
         const float neg_m = (m_ref == -INFINITY) ? 0.f : -m_ref;
-        uint32_t pk[NK / 2];
         float ls0 = 0.f, ls1 = 0.f, lx0 = 0.f, lx1 = 0.f;
+        auto emit_half = [&](int hq) {
+          const uint32_t prow = dst + hq * P_CHUNK + h * 128;
 #pragma unroll
-        for (int i = 0; i < NK / 2; ++i) {
-          const float p0 = ex2_approx(fmaf(__uint_as_float(v[2 * i]), p.scale_log2, neg_m));
-          const float p1 = ex2_approx(fmaf(__uint_as_float(v[2 * i + 1]), p.scale_log2, neg_m));
-          const __nv_bfloat162 bb = __floats2bfloat162_rn(p0, p1);
-          ls0 += __low2float(bb);
-          ls1 += __high2float(bb);
-          lx0 += p0;
-          lx1 += p1;
-          pk[i] = *reinterpret_cast<const uint32_t*>(&bb);
-        }
-        const float ls = ls0 + ls1, lx = lx0 + lx1;
-        l += ls;
-        le += lx;
-        // staging slot b was last read by the bulk copy of tile g - 2: the leader waits for that copy to
-        // have read its source, then releases the slot to the four softmax warps
-        if (leader) {
-          DSA_TRACE_EVENT(5, g);
-          bulk_wait_read<1>();
-          DSA_TRACE_EVENT(26, g);
-          mbar_arrive(bar(B_SLOT_FREE));
-        }
-        if (!(ok = warp_wait(bar(B_SLOT_FREE), static_cast<uint32_t>(g & 1), abort_flag))) break;
-        if (leader) DSA_TRACE_EVENT(27, g);
-        uint8_t* st = smem + OFF_PST + b * XFER;
-        uint8_t* prow = st + h * 128;
+          for (int c = 0; c < 8; ++c) {
+            uint32_t pk[4];
 #pragma unroll
-        for (int c = 0; c < 8; ++c)
-          *reinterpret_cast<uint4*>(prow + ((c ^ (h & 7)) << 4)) =
-              make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
-        reinterpret_cast<float*>(st + P_BYTES)[h] = alpha;
-        if (j == ntiles - 1) {
-          reinterpret_cast<float*>(st + P_BYTES + 512)[h] = l;
-          if (p.lse && h < p.H)
-            p.lse[static_cast<long long>(t) * p.H + h] =
-                (le > 0.f) ? (m_ref + lg2_approx(le)) * 0.69314718055994531f : -INFINITY;
-        }
-        fence_proxy_async_smem();     // the staging slot is read next by the bulk-copy (async) proxy
-        if (leader) DSA_TRACE_EVENT(28, g);
-        __syncwarp();
-        if (lane == 0) mbar_arrive(bar(B_SLOT_WRITTEN));
-        if (leader) {
-          // all four warps wrote the slot; the value CTA's P buffer pb is free once its PV of tile g - NPB
-          // has completed
-          ok = mbar_wait(bar(B_SLOT_WRITTEN), static_cast<uint32_t>(g & 1), abort_flag);
-          DSA_TRACE_EVENT(29, g);
-          ok = ok && mbar_wait<true>(bar(B_P_EMPTY + pb), static_cast<uint32_t>((g / NPB) & 1) ^ 1, abort_flag);
-          if (ok) {
-            DSA_TRACE_EVENT(7, g);
-            mbar_arrive_expect_tx_remote(pfull_remote + 8 * pb, XFER);
-            bulk_copy_to_peer(pb_remote + pb * XFER, sbase + OFF_PST + b * XFER, XFER, pfull_remote + 8 * pb);
-            bulk_commit();
+            for (int i = 0; i < 4; ++i) {
+              const float p0 = ex2_approx(fmaf(__uint_as_float(v[8 * c + 2 * i]), p.scale_log2, neg_m));
+              const float p1 = ex2_approx(fmaf(__uint_as_float(v[8 * c + 2 * i + 1]), p.scale_log2, neg_m));
+              const __nv_bfloat162 bb = __floats2bfloat162_rn(p0, p1);
+              ls0 += __low2float(bb);
+              ls1 += __high2float(bb);
+              lx0 += p0;
+              lx1 += p1;
+              pk[i] = *reinterpret_cast<const uint32_t*>(&bb);
+            }
+            st_async_v4(prow + ((c ^ (h & 7)) << 4), make_uint4(pk[0], pk[1], pk[2], pk[3]), fb);
           }
-        }
-        ok = __shfl_sync(0xffffffffu, ok, 0) && !*abort_flag;
+        };
+        emit_half(1);    // keys 64..127: still in v from pass 1
+        tmem_ld32(s_tmem, v0);
+        tmem_ld32(s_tmem + 32, v1);
+        tmem_wait_ld();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(B_S_EMPTY + sb));
+        if (!full_tile) mask_half(0);
+        emit_half(0);
+        l += ls0 + ls1;
+        le += lx0 + lx1;
+        // per-head rescale factor and running row sum (the value CTA reads the sum of the token's last tile)
+        st_async_b32(dst + P_BYTES + 4 * h, __float_as_uint(alpha), fb);
+        st_async_b32(dst + P_BYTES + 512 + 4 * h, __float_as_uint(l), fb);
+        if (leader) DSA_TRACE_EVENT(28, g);
+        if (j == ntiles - 1 && p.lse && h < p.H)
+          p.lse[static_cast<long long>(t) * p.H + h] =
+              (le > 0.f) ? (m_ref + lg2_approx(le)) * 0.69314718055994531f : -INFINITY;
+        ok = __shfl_sync(0xffffffffu, *abort_flag == 0, 0);
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(bar(B_IDX_EMPTY + is));
     }
-    if (leader) bulk_wait_read<0>();
   } else {
     // ===================================================================== correction + epilogue (value CTA)
     const int quad = warp & 3;
@@ -797,6 +824,8 @@ sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         const int pb = static_cast<int>(g % NPB);
         if (!(ok = warp_wait<true>(bar(B_P_FULL + pb), static_cast<uint32_t>((g / NPB) & 1), abort_flag))) break;
         if (warp == 4 && lane == 0) DSA_TRACE_EVENT(18, g);
+        // P arrived by st.async; the PV MMA reads it through the async proxy
+        fence_proxy_async_smem();
         const uint8_t* xb = smem + OFF_PB + pb * XFER;
         const float a = reinterpret_cast<const float*>(xb + P_BYTES)[h];
         if (j == ntiles - 1) l = reinterpret_cast<const float*>(xb + P_BYTES + 512)[h];

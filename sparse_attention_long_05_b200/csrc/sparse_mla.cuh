@@ -19,14 +19,20 @@
 //     of 64-key tiles at about 40 % of its rate).  The score CTA's tensor memory holds Q chunks 0..7 (128 heads
 //     x 64 dims each, 32 columns) in columns 0..255 and two 128-column S buffers, so the QK^T of tile g + 1
 //     runs while the softmax reads tile g's logits.  Q chunk 8 (the 64 position dims) is the A operand of its
-//     MMAs from shared memory (two buffers, one per token in flight).
+//     MMAs from shared memory, loaded for the next token as soon as the current token's last MMAs reading it
+//     have retired.
 //   * Selected rows are gathered by TMA tile::gather4 (four rows x one 64-column, 128-byte swizzled box per
 //     instruction) into 128-key x 64-dim chunks in the K-major form the tensor core reads.  A pipeline stage
-//     holds several chunks of one tile (three in the score CTA, four in the value CTA), because the
-//     issuing thread spends a few hundred cycles per stage on its barrier wait, the tcgen05 issue and the
-//     commit whatever the stage's size.  Each stage is split over eight gather warps (one warp issues gather4
-//     only about every 50 ns; gather throughput per SM grows with the issuing warps: about 12, 24, 45 and 73
-//     GB/s with 1, 2, 4 and 8), each of which arrives on the stage's barrier with its share of the bytes.  TMA
+//     holds several chunks of one tile (three in the score CTA, four in the value CTA): each gather warp spends
+//     about 300 ns per stage on its barrier handshake whatever the stage's size, so a stage gives each warp a
+//     dozen or more gather4 to issue.  The ring is as deep as shared memory allows (three stages, 144 KB, in
+//     the score CTA; two, 128 KB, in the value CTA): a gather takes about 1.5 us to land under load, so the
+//     bytes in flight set the rate.  With every SM gathering random rows of a 151 MB latent and each stage
+//     freed as soon as it landed, one SM's gathers ran at about 44 GB/s with two 48 KB stages, 66 with four,
+//     and 73 with three 64 KB stages (near the TMA unit's limit of about 75).  Each stage is split over eight
+//     gather warps (one warp issues gather4 only about every 50 ns; gather throughput per SM grows with the
+//     issuing warps: about 12, 24, 45 and 73 GB/s with 1, 2, 4 and 8), each of which arrives on the stage's
+//     barrier with its share of the bytes.  TMA
 //     writes are in the async proxy, so the MMA warp consumes a stage as soon as its mbarrier completes,
 //     with no proxy fence.  The same chunk bytes serve as the K-major B operand of QK^T (rows = keys) and
 //     as the MN-major B operand of PV (rows = keys = K, 64 dims = N per atom; four chunks = N 256).
@@ -96,7 +102,7 @@ constexpr int NPB = 2;                    // P buffers (value CTA)
 constexpr int SCH = 3, VCH = 4;           // 64-dim chunks per gather stage (score CTA, value CTA)
 constexpr int S_STAGE = SCH * CHUNK_BYTES, V_STAGE = VCH * CHUNK_BYTES;
 constexpr int SPT_S = QCHUNKS / SCH, SPT_V = VCHUNKS / VCH;   // stages per 128-key tile: 3, 2
-constexpr int NS_S = 2, NS_V = 2;         // gather stages per CTA
+constexpr int NS_S = 3, NS_V = 2;         // gather stages per CTA (KL mode: NS_S - 1, its head sums in the last)
 constexpr int THREADS = 448;
 constexpr int GATHER_WARPS = 8;
 constexpr int G4_PER_CHUNK = NK / 4;      // gather4 instructions per chunk (four rows each)
@@ -117,19 +123,19 @@ constexpr int B_P_FULL = B_P_EMPTY + NPB, B_P_READY = B_P_FULL + NPB;
 // only now and then and could be two phases behind, where a parity test cannot tell the phases apart
 constexpr int B_O_DONE = B_P_READY + NPB, B_O_FREE = B_O_DONE + NPB;
 constexpr int B_QRET = B_O_FREE + 1;          // score CTA: stage s of a token's last tile retired (3 barriers)
-constexpr int B_ROPE_FULL = B_QRET + SPT_S;   // score CTA: Q chunk 8 of a token staged (2 buffers)
-constexpr int B_ROPE_EMPTY = B_ROPE_FULL + 2; // score CTA: every MMA reading a Q chunk 8 buffer retired
-constexpr int B_RED_FULL = B_ROPE_EMPTY + 2;  // KL mode: the four warps' head sums of a tile written (2 buffers)
+constexpr int B_ROPE_FULL = B_QRET + SPT_S;   // score CTA: Q chunk 8 of a token staged
+constexpr int B_ROPE_EMPTY = B_ROPE_FULL + 1; // score CTA: every MMA reading Q chunk 8 of a token retired
+constexpr int B_RED_FULL = B_ROPE_EMPTY + 1;  // KL mode: the four warps' head sums of a tile written (2 buffers)
 constexpr int B_RED_FREE = B_RED_FULL + 2;    // KL mode: the head sums of a tile read (2 buffers)
 constexpr int B_COUNT = B_RED_FREE + 2;
 // shared memory map (from a 1024-byte aligned base; both CTAs use the same barrier offsets)
 constexpr int OFF_TMEM = 8 * B_COUNT;
 constexpr int OFF_ABORT = OFF_TMEM + 4;
 constexpr int OFF_IDX = 1024;                                   // both: 2 x 8 KB index rows
-constexpr int OFF_RED = OFF_IDX + 2 * KMAX * 4;                 // score CTA, KL mode: head sums [2][4][NK]
-constexpr int OFF_QST = OFF_RED + 2 * 4 * NK * 4;               // score CTA: Q staging
-constexpr int OFF_ROPE = OFF_QST + QS * QCHUNK_BYTES;           // score CTA: Q chunk 8, two buffers
-constexpr int OFF_RING_S = OFF_ROPE + 2 * QCHUNK_BYTES;         // score CTA: gather ring
+constexpr int OFF_QST = OFF_IDX + 2 * KMAX * 4;                 // score CTA: Q staging
+constexpr int OFF_ROPE = OFF_QST + QS * QCHUNK_BYTES;           // score CTA: Q chunk 8 of the current token
+constexpr int OFF_RING_S = OFF_ROPE + QCHUNK_BYTES;             // score CTA: gather ring
+constexpr int OFF_RED = OFF_RING_S + (NS_S - 1) * S_STAGE;      // score CTA, KL mode: head sums [2][4][NK]
 constexpr int OFF_PB = OFF_IDX + 2 * KMAX * 4;                  // value CTA: P buffers
 constexpr int OFF_RING_V = OFF_PB + NPB * XFER;                 // value CTA: gather ring
 constexpr int SMEM_S = OFF_RING_S + NS_S * S_STAGE;
@@ -137,6 +143,7 @@ constexpr int SMEM_V = OFF_RING_V + NS_V * V_STAGE;
 constexpr int SMEM = (SMEM_S > SMEM_V ? SMEM_S : SMEM_V) + 1024;
 static_assert(OFF_ABORT + 4 <= OFF_IDX, "barrier area");
 static_assert(OFF_QST % 1024 == 0 && OFF_ROPE % 1024 == 0 && OFF_RING_S % 1024 == 0, "1 KB aligned tiles");
+static_assert(2 * 4 * NK * 4 <= S_STAGE, "KL mode: head sums in the ring's last stage");
 static_assert(OFF_PB % 1024 == 0 && XFER % 1024 == 0 && OFF_RING_V % 1024 == 0, "1 KB aligned tiles");
 static_assert(QCHUNKS % SCH == 0 && VCHUNKS % VCH == 0 && VCH * 64 == 256, "stage split");
 static_assert(QTM == QCHUNKS - 1 && SPT_S == 3, "Q chunk 8 in the last score stage");
@@ -258,7 +265,7 @@ sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
   const uint32_t rank = kl_mode ? 0u : cluster_rank();
   const int cluster = kl_mode ? static_cast<int>(blockIdx.x) : static_cast<int>(blockIdx.x >> 1);
   const int nclusters = kl_mode ? static_cast<int>(gridDim.x) : static_cast<int>(gridDim.x >> 1);
-  const int nsr = (rank == 0) ? NS_S : NS_V;
+  const int nsr = (rank == 0) ? (KL ? NS_S - 1 : NS_S) : NS_V;
   const uint32_t ring = sbase + ((rank == 0) ? OFF_RING_S : OFF_RING_V);
   const int* idx_s = reinterpret_cast<const int*>(smem + OFF_IDX);
 
@@ -276,7 +283,8 @@ sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
       for (int i = 0; i < 2; ++i) { mbar_init(bar(B_S_FULL + i), 1); mbar_init(bar(B_S_EMPTY + i), 4); }
       for (int i = 0; i < NPB; ++i) mbar_init(bar(B_P_EMPTY + i), 1);
       for (int i = 0; i < SPT_S; ++i) mbar_init(bar(B_QRET + i), 1);
-      for (int i = 0; i < 2; ++i) { mbar_init(bar(B_ROPE_FULL + i), 1); mbar_init(bar(B_ROPE_EMPTY + i), 1); }
+      mbar_init(bar(B_ROPE_FULL), 1);
+      mbar_init(bar(B_ROPE_EMPTY), 1);
       for (int i = 0; i < 2; ++i) { mbar_init(bar(B_RED_FULL + i), 4); mbar_init(bar(B_RED_FREE + i), 1); }
     } else {
       for (int i = 0; i < NPB; ++i) { mbar_init(bar(B_P_FULL + i), 1); mbar_init(bar(B_P_READY + i), 4); }
@@ -309,8 +317,8 @@ sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     if (lane == 0) {
       int qn = 0, ti = 0;
       bool ok = true;
-      int idx_issued = 0, q_issued = 0, rope_issued = 0;
-      uint32_t idx_par[2] = {0, 0}, q_par[QS] = {}, rope_par[2] = {0, 0};
+      int idx_issued = 0, q_issued = 0;
+      uint32_t idx_par[2] = {0, 0}, q_par[QS] = {};
       for (int t = cluster; t < p.T && ok; t += nclusters, ++ti) {
         const int is = ti & 1;
         if (!(ok = mbar_wait(bar(B_IDX_EMPTY + is), ((ti >> 1) & 1) ^ 1, abort_flag))) break;
@@ -320,13 +328,6 @@ sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         idx_par[is] = (ti >> 1) & 1;
         ++idx_issued;
         if (rank == 0) {
-          // chunk 8 (the position dims) into its own buffer, read by the MMAs from shared memory
-          const int rb = ti & 1;
-          if (!(ok = mbar_wait(bar(B_ROPE_EMPTY + rb), ((ti >> 1) & 1) ^ 1, abort_flag))) break;
-          mbar_arrive_expect_tx(bar(B_ROPE_FULL + rb), QCHUNK_BYTES);
-          tma_load_3d(sbase + OFF_ROPE + rb * QCHUNK_BYTES, &tm_q, bar(B_ROPE_FULL + rb), 64 * QTM, 0, t);
-          rope_par[rb] = (ti >> 1) & 1;
-          ++rope_issued;
           // chunks 0..7 through the staging slots, copied into tensor memory by the MMA warp
           for (int c = 0; c < QTM; ++c, ++qn) {
             const int qs = qn % QS;
@@ -341,8 +342,20 @@ sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
       if (*abort_flag) {
         for (int i = 0; i < 2 && i < idx_issued; ++i) mbar_wait_drain(bar(B_IDX_FULL + i), idx_par[i]);
         for (int i = 0; i < QS && i < q_issued; ++i) mbar_wait_drain(bar(B_QST_FULL + i), q_par[i]);
-        for (int i = 0; i < 2 && i < rope_issued; ++i) mbar_wait_drain(bar(B_ROPE_FULL + i), rope_par[i]);
       }
+    } else if (lane == 1 && rank == 0) {
+      // chunk 8 (the position dims) of each token into its buffer, read by the MMAs from shared memory: loaded as
+      // soon as the previous token's last MMAs reading it have retired, on a lane of its own so that the Q chunk
+      // staging above never waits for it
+      int ti = 0, issued = 0;
+      bool ok = true;
+      for (int t = cluster; t < p.T && ok; t += nclusters, ++ti) {
+        if (!(ok = mbar_wait(bar(B_ROPE_EMPTY), (ti & 1) ^ 1, abort_flag))) break;
+        mbar_arrive_expect_tx(bar(B_ROPE_FULL), QCHUNK_BYTES);
+        tma_load_3d(sbase + OFF_ROPE, &tm_q, bar(B_ROPE_FULL), 64 * QTM, 0, t);
+        ++issued;
+      }
+      if (*abort_flag && issued) mbar_wait_drain(bar(B_ROPE_FULL), (issued - 1) & 1);
     }
   } else if (warp == 2 || warp == 3 || warp >= 8) {
     // ===================================================================== gathers (TMA gather4)
@@ -438,7 +451,7 @@ sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     rp.size = nsr;
     int ti = 0;
     if (rank == 0) {
-      // Q chunks 0..7 of a token live in tensor-memory slots 0..7, chunk 8 in its shared-memory buffer (ti % 2).
+      // Q chunks 0..7 of a token live in tensor-memory slots 0..7, chunk 8 in its shared-memory buffer.
       // A copy overwrites a slot only after the MMAs that last read it have completed (tcgen05.commit barriers
       // QRET[s], stage s of a token's last tile): the next token's chunks 0..2 are copied during the last tile,
       // after the stage that follows stage 0 (stage 2 for a one-tile token, so that chunks leave the staging
@@ -466,7 +479,6 @@ sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
       if (cluster < p.T) ok = copy_q(QTM);
       for (int t = cluster; t < p.T && ok; t += nclusters, ++ti) {
         const bool has_next = t + nclusters < p.T;
-        const int rb = ti & 1;
         const int ntiles = mla_tiles(p, mla_dense_keys<DENSE>(p, t, p.row_off ? p.row_off[t] : 0));
         for (int j = 0; j < ntiles && ok; ++j, ++g) {
           const int sb = static_cast<int>(g & 1);
@@ -482,14 +494,14 @@ sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
               if (!(ok = copy_q(s == 1 ? 3 : 2))) break;
             }
             if (j == 0 && s == SPT_S - 1 &&
-                !(ok = warp_wait(bar(B_ROPE_FULL + rb), static_cast<uint32_t>((ti >> 1) & 1), abort_flag)))
+                !(ok = warp_wait(bar(B_ROPE_FULL), static_cast<uint32_t>(ti & 1), abort_flag)))
               break;
             if (!(ok = warp_wait(bar(B_RING_FULL + st), rp.phase, abort_flag))) break;
             DSA_TRACE_EVENT(12 + s, g);
             tc_fence_after();
             // the stage's three chunks: 12 MMAs issued as one block, then one commit
             const uint64_t bd = smem_desc(ring + st * S_STAGE, 16, 1024, kLayoutSW128);
-            const uint64_t rd = smem_desc(sbase + OFF_ROPE + rb * QCHUNK_BYTES, 16, 1024, kLayoutSW128);
+            const uint64_t rd = smem_desc(sbase + OFF_ROPE, 16, 1024, kLayoutSW128);
             if (elect_one()) {
 #pragma unroll
               for (int cc = 0; cc < SCH; ++cc) {
@@ -504,7 +516,7 @@ sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
               }
               mma_commit(bar(B_RING_EMPTY + st));
               if (last && has_next) mma_commit(bar(B_QRET + s));
-              if (last && s == SPT_S - 1) mma_commit(bar(B_ROPE_EMPTY + rb));
+              if (last && s == SPT_S - 1) mma_commit(bar(B_ROPE_EMPTY));
             }
             __syncwarp();
             DSA_TRACE_EVENT(9 + s, g);

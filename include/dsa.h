@@ -191,7 +191,7 @@ DSA_API size_t dsa_prefill_host_workspace_size(int L, int H_I, int d_I, int H, i
  * dsa_forward_prefill with every input and output in HOST memory (steps 1-3 for one causal sequence, as
  * dsa_forward_prefill; same arguments, HOST pointers; lse and idx_out may be NULL).  The call moves the data
  * itself and overlaps the transfers with the kernels: the indexer's inputs are copied first; then, in
- * 8 chunks of rows, each chunk's selection runs while later queries are still arriving, each chunk's attention
+ * 16 chunks of rows, each chunk's selection runs while later queries are still arriving, each chunk's attention
  * starts once its queries have landed, and its results go back while the next chunk computes.  Host-to-device
  * and device-to-host copies run on two copy streams of the library's own (created once per device on first
  * use), so both directions of the host link are busy at once.  For the copies to be asynchronous the host

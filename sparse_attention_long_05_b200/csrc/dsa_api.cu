@@ -769,7 +769,7 @@ dsa_status_t dsa_forward_prefill(const uint8_t* q_idx, const float* q_scale, con
 
 // ------------------------------------------------------------------------------------------ host-buffer prefill
 namespace {
-constexpr int kHostChunks = 8;          // token chunks of the host-buffer prefill's pipeline
+constexpr int kHostChunks = 16;         // token chunks of the host-buffer prefill's pipeline
 
 // The host-buffer prefill's device copies, laid out after the prefill workspace.
 struct HostPrefillLayout {

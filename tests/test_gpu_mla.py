@@ -80,6 +80,20 @@ def test_selection_order_and_padding_do_not_matter(dsa):
     assert np.abs(a[:2] - b[:2]).max() <= 2 * MAX_ABS
 
 
+@pytest.mark.parametrize("k", [192, 320, 640])
+def test_k_ending_in_half_a_tile(dsa, k):
+    # k a multiple of 64 but not of 128: a token's last 128-key tile holds 64 selection slots and 64 masked ones.
+    # The rows straddle k, so tokens below it carry -1 padding as well; 160 tokens put two or three on every
+    # cluster (token transitions in the score CTA's Q-chunk schedule).
+    cfg = G.PREFILL_CONFIGS["prefill_8k"]
+    keys = G.prefill_keys(cfg, 25, device="cuda")
+    rows = list(range(k - 80, k + 80))
+    qs = G.prefill_queries(cfg, 25, rows=rows, device="cuda")
+    rng = np.random.default_rng(25 + k)
+    idx = np.concatenate([_random_selection(rng, 1, cfg.L, k, t) for t in rows])
+    _compare(dsa, qs["q"], keys["c"], idx, cfg.scale)
+
+
 def test_bad_index_is_reported_and_skipped(dsa):
     cfg = G.PREFILL_CONFIGS["tiny_1k"]
     x = G.prefill_inputs(cfg, 24, device="cuda")

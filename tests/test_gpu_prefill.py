@@ -70,6 +70,15 @@ def test_tiny_all_rows(dsa):
     _check_rows(cfg, 31, rows, idx, out, exact_idx=True)
 
 
+def test_k_ending_in_half_a_tile_end_to_end(dsa):
+    # k = 320: dense rows t + 1 <= 320 run ceil((t + 1) / 128) tiles, gathered rows three tiles, the last half
+    # masked; integer mode, so the selections are exact
+    cfg = dataclasses.replace(G.PREFILL_CONFIGS["prefill_8k"], L=1500, k=320)
+    idx, out, _ = _forward(dsa, cfg, 35)
+    rows = sorted(set(list(range(0, 1500, 23)) + [127, 128, 255, 256, 318, 319, 320, 321, 383, 384, 1499]))
+    _check_rows(cfg, 35, rows, idx, out, exact_idx=True)
+
+
 def test_8k_integer_mode(dsa):
     cfg = G.PREFILL_CONFIGS["prefill_8k"]
     idx, out, _ = _forward(dsa, cfg, 32)

@@ -92,6 +92,7 @@ def test_host_argument_checks(lib):
     assert lib.dsa_check_bounded_wait(P(20), None) == 3
     # empty work is a no-op
     assert lib.dsa_indexer_scores(one, None, one, None, one, 0, 4, 64, 128, 0, one, None) == 0
+    assert lib.dsa_sparse_mla_attn(None, None, 10, None, 0, 8, 128, 1.0, None, None, None) == 0
 
 
 def test_prefill_block_schedule(lib):

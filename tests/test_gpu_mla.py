@@ -94,6 +94,19 @@ def test_k_ending_in_half_a_tile(dsa, k):
     _compare(dsa, qs["q"], keys["c"], idx, cfg.scale)
 
 
+def test_rows_with_nothing_selected(dsa):
+    # rows whose k entries are all padding attend to nothing: output 0 and lse -inf (the oracle's empty selection),
+    # next to ordinary rows in the same launch; one row selects a single entry
+    cfg = G.PREFILL_CONFIGS["tiny_1k"]
+    x = G.prefill_inputs(cfg, 26, device="cuda")
+    idx = _random_selection(np.random.default_rng(26), 6, cfg.L, cfg.k, 700)
+    idx[1] = -1
+    idx[4] = -1
+    idx[5, 1:] = -1
+    out = _compare(dsa, x["q"][700:706].contiguous(), x["c"], idx, cfg.scale)
+    assert not np.abs(out[1]).any() and not np.abs(out[4]).any()
+
+
 def test_bad_index_is_reported_and_skipped(dsa):
     cfg = G.PREFILL_CONFIGS["tiny_1k"]
     x = G.prefill_inputs(cfg, 24, device="cuda")

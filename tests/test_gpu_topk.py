@@ -94,3 +94,6 @@ def test_long_rows_where_the_sample_misleads(dsa):
     rows[2, rng.choice(np.flatnonzero(~sampled), 3000, replace=False)] = 50.0   # outliers outside the sample
     rows[3] = np.round(rows[3])       # heavy ties
     _check(dsa, rows, 2048, row_len=[n, n, n, n, n - 7])
+    # the same rows, 150 of them: at least as many rows as SMs take the one-CTA-per-row kernel and its sampled path
+    many = np.tile(rows, (30, 1))
+    _check(dsa, many, 2048, row_len=[n, n, n, n, n - 7] * 30)

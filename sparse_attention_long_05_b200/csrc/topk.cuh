@@ -257,7 +257,7 @@ __global__ void __launch_bounds__(NT, 2) topk_rows_kernel(const TopkParams p) {
 
   // ---------------------------------------------------------------- sampled path (long 16-byte aligned rows)
   // A histogram of one eighth of the row (128-key blocks every 1024 keys) picks a bin b_est low enough that,
-  // with a 1.5x margin, at least k keys of the row lie in bins >= b_est; one pass then collects those keys and
+  // with a 1.25x margin, at least k keys of the row lie in bins >= b_est; one pass then collects those keys and
   // counts them exactly.  When they are at least k (and fit), the k-th largest key is among them, and the
   // exact selection runs on the candidates alone: the row is read about 1.1 times instead of twice, with an
   // eighth of the histogram atomics.  Otherwise the exact path below runs.
@@ -283,7 +283,7 @@ __global__ void __launch_bounds__(NT, 2) topk_rows_kernel(const TopkParams p) {
       }
     }
     __syncthreads();
-    topk_find_bin(3u * static_cast<uint32_t>(k) / 16u + 16u, sm);   // k / 8 sampled keys with a 1.5x margin
+    topk_find_bin(5u * static_cast<uint32_t>(k) / 32u + 16u, sm);   // k / 8 sampled keys with a 1.25x margin
     const uint32_t b_est = sm.s_bin;
     if (b_est != 0xFFFFFFFFu && b_est >= 1) {
       topk_collect_vec(x, n, b_est, sm);

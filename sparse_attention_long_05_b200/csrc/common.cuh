@@ -286,6 +286,16 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&v)[32]) {
       : DSA_R8(0), DSA_R8(8), DSA_R8(16), DSA_R8(24)
       : "r"(taddr));
 }
+// 16 lanes x 256 bits, 8 repetitions along the columns (64 columns): thread i receives, for repetition m,
+// v[4m], v[4m+1] = lane (i / 4), columns 8m + 2(i % 4) + {0, 1}, and v[4m+2], v[4m+3] = lane (i / 4 + 8), the
+// same columns (lanes counted from the lane field of taddr)
+__device__ __forceinline__ void tmem_ld16x256_x8(uint32_t taddr, uint32_t (&v)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.16x256b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+      : DSA_R8(0), DSA_R8(8), DSA_R8(16), DSA_R8(24)
+      : "r"(taddr));
+}
 __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&v)[32]) {
   asm volatile(
       "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
@@ -294,6 +304,11 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&v)[32
       : "memory");
 }
 __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+// The same wait, ordered after the arithmetic that produced a, b and x: without the tie the compiler may sink
+// register-only arithmetic below the wait, and the loads it was meant to hide stay exposed.
+__device__ __forceinline__ void tmem_wait_ld_after(uint64_t& a, uint64_t& b, float& x) {
+  asm volatile("tcgen05.wait::ld.sync.aligned;" : "+l"(a), "+l"(b), "+f"(x) :: "memory");
+}
 // Placed after tmem_wait_ld: ties the registers of an earlier tcgen05.ld to a point after the wait, so that no
 // use of them is scheduled before the loads complete.
 __device__ __forceinline__ void tmem_regs_after_wait(uint32_t (&v)[32]) {

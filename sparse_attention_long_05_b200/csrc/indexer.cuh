@@ -5,17 +5,19 @@
 //   A = 128 keys x d_I   (K-major, TMA-loaded tile of k_I),
 //   B = NT*H_I rows of q_I x d_I (K-major; rows (t, j) are consecutive in q_I's [T, H_I, d_I] layout),
 //   D = 128 TMEM lanes (one per key) x NT*H_I fp32 columns.
-// Because a key owns a TMEM lane, the ReLU and the head-weighted sum over j are thread-local in the
-// epilogue: thread s loads its lane's columns, computes sum_j w[t,j] * max(x, 0) for each of its tokens,
-// multiplies by the key scale (Gaussian mode; the query scale is folded into w), and writes I[t, s].
+// Because a key owns a TMEM lane, the ReLU and the head-weighted sum over j stay within a warp: the epilogue
+// reads its lanes' columns, forms sum_j w[t,j] * max(x, 0) for each token of the stage (sixteen heads per thread,
+// then a two-step shuffle over the four threads sharing a key), multiplies by the key scale (Gaussian mode; the
+// query scale is folded into w), and writes I[t, s].
 //
 // Warp roles (one CTA per SM):
 //   warp 0      TMA producer: q_I block of the work item, then one k_I tile per pipeline stage
 //   warp 1      TMEM allocation + MMA issue (one elected thread)
 //   warps 2..   epilogue warpgroup(s); warp w reads TMEM lanes 32*(w % 4) .. +31
 // A ring of TMEM accumulators (2 of 256 columns; 4 of 64 in decode, two CTAs per SM) lets the
-// epilogue of one (tile, group) overlap the MMAs of the next ones.  Tiles lying wholly above the causal
-// diagonal of every token of the item are never loaded.
+// epilogue of one (tile, group) overlap the MMAs of the next ones; with two epilogue warpgroups, each takes
+// every other accumulator stage.  Tiles lying wholly above the causal diagonal of every token of the item are
+// never loaded.
 //
 // Work items:
 //   kModeScores  item = (block of NG*NT query rows, range of key tiles); writes scores [T, S] (tests,
@@ -98,7 +100,6 @@ struct IndexerCfg {
   static constexpr int GBYTES = N * D_I;             // one group of q_I rows
   static constexpr int KBYTES = 128 * D_I;           // one key tile
   static constexpr int NUM_EPI_WARPS = 4 * EPI_WG;
-  static constexpr int NUM_THREADS = 64 + 32 * NUM_EPI_WARPS;
   // CTAs per SM the launch relies on (decode: two, so that two sequences' chunks share an SM)
   static constexpr int CTAS_PER_SM = (MODE == kModeDecode) ? 2 : 1;
   static constexpr int ALIGN = 1024;
@@ -116,6 +117,13 @@ struct IndexerCfg {
   // (4 x 64 columns) so that two CTAs share an SM
   static constexpr int NACC = (MODE == kModeDecode) ? 4 : ((512 / N) < 8 ? (512 / N) : 8);
   static constexpr uint32_t TMEM_COLS = static_cast<uint32_t>(NACC * N);
+  // two epilogue warpgroups on alternate accumulator stages (H_I = 64 with two accumulators), each reading all N
+  // columns of its stages; otherwise each warpgroup reads a column half of every stage
+  static constexpr bool ALT_STAGES = (H_I == 64) && (EPI_WG == 2) && (NACC % 2 == 0) && ((N / EPI_WG) % 64 == 0);
+  static constexpr int ACC_READERS = ALT_STAGES ? NUM_EPI_WARPS / 2 : NUM_EPI_WARPS;   // arrivals per stage
+  // warps: 0 TMA producer, 1 MMA issue, EPI_WARP0.. the epilogue
+  static constexpr int EPI_WARP0 = 2;
+  static constexpr int NUM_THREADS = 32 * (EPI_WARP0 + NUM_EPI_WARPS);
   static_assert(TMEM_COLS == 256 || TMEM_COLS == 512, "tensor-memory allocation (power of two)");
   static constexpr uint32_t SW_LAYOUT = (D_I == 128) ? kLayoutSW128 : kLayoutSW64;
   static constexpr uint32_t SBO = (D_I == 128) ? 1024 : 512;
@@ -244,7 +252,7 @@ indexer_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     for (int i = 0; i < KSTAGES; ++i) { mbar_init(bar(Bars::K_FULL + i), 1); mbar_init(bar(Bars::K_EMPTY + i), 1); }
     for (int i = 0; i < C::NACC; ++i) {
       mbar_init(bar(Bars::ACC_FULL + i), 1);
-      mbar_init(bar(Bars::ACC_EMPTY + i), C::NUM_EPI_WARPS);
+      mbar_init(bar(Bars::ACC_EMPTY + i), C::ACC_READERS);
     }
     *abort_flag = 0;
     fence_mbar_init();
@@ -335,96 +343,112 @@ indexer_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     }
   };
 
-  if (warp == 0) {
-    // ------------------------------------------------------------------ TMA producer
-    if (lane == 0) {
-      Pipe<KSTAGES> kp;
-      int k_issued = 0;                 // k tiles issued so far
-      int q_issued[QBUF] = {};          // per q buffer: loads issued
-      uint32_t q_par[QBUF] = {};        // per q buffer: parity of its last load
-      int qi = 0;
-      bool ok = true;
-      for (int item = first_item(); has_item(item) && ok; item = next_item(item), ++qi) {
-        const IndexerItem it = indexer_item<MODE, C::TOK>(p, item, prefix, tr);
-        const int qb = qi % QBUF;
-        const uint32_t qph = (qi / QBUF) & 1;
-        if (!mbar_wait(bar(Bars::Q_EMPTY + qb), qph ^ 1, abort_flag)) { ok = false; break; }
-        mbar_arrive_expect_tx(bar(Bars::Q_FULL + qb), NG * C::GBYTES);
-        for (int g = 0; g < NG; ++g)
-          tma_load_2d(q_s + (qb * NG + g) * C::GBYTES, &tm_q, bar(Bars::Q_FULL + qb), 0,
-                      (it.q_row0 + g * NT) * H_I);
-        q_issued[qb] += 1;
-        q_par[qb] = qph;
-        for (int tile = it.tile0; tile < it.tile1; ++tile) {
-          if (!tile_active(it, tile)) continue;
-          if (!mbar_wait(bar(Bars::K_EMPTY + kp.stage), kp.phase ^ 1, abort_flag)) { ok = false; break; }
-          mbar_arrive_expect_tx(bar(Bars::K_FULL + kp.stage), C::KBYTES);
-          tma_load_2d(k_s + kp.stage * C::KBYTES, &tm_k, bar(Bars::K_FULL + kp.stage), 0,
-                      static_cast<int>(key_row(it, tile, 0)));
-          kp.advance();
-          ++k_issued;
-        }
-      }
-      if (*abort_flag) {
-        // leave no TMA write in flight into this CTA's shared memory: wait (bounded) for the last load
-        // issued on every k stage and q buffer
-        for (int st = 0; st < KSTAGES && st < k_issued; ++st)
-          mbar_wait_drain(bar(Bars::K_FULL + st), st < kp.stage ? kp.phase : kp.phase ^ 1);
-        for (int b = 0; b < QBUF; ++b)
-          if (q_issued[b]) mbar_wait_drain(bar(Bars::Q_FULL + b), q_par[b]);
-      }
-    }
-  } else if (warp == 1) {
-    // ------------------------------------------------------------------ MMA issue
-    if (lane == 0) {
-      Pipe<KSTAGES> kp;
-      Pipe<C::NACC> ap;
-      constexpr uint32_t idesc = idesc_e4m3(128, C::N);
-      int qi = 0;
-      bool ok = true;
-      for (int item = first_item(); has_item(item) && ok; item = next_item(item), ++qi) {
-        const IndexerItem it = indexer_item<MODE, C::TOK>(p, item, prefix, tr);
-        const int qb = qi % QBUF;
-        if (!mbar_wait(bar(Bars::Q_FULL + qb), (qi / QBUF) & 1, abort_flag)) { ok = false; break; }
-        tc_fence_after();
-        for (int tile = it.tile0; tile < it.tile1 && ok; ++tile) {
-          if (!tile_active(it, tile)) continue;
-          if (!mbar_wait(bar(Bars::K_FULL + kp.stage), kp.phase, abort_flag)) { ok = false; break; }
-          tc_fence_after();
-          const uint64_t adesc = smem_desc(k_s + kp.stage * C::KBYTES, 16, C::SBO, C::SW_LAYOUT);
-          for (int g = 0; g < NG; ++g) {
-            if (!group_active<NT>(it, tile, g)) continue;
-            if (!mbar_wait(bar(Bars::ACC_EMPTY + ap.stage), ap.phase ^ 1, abort_flag)) { ok = false; break; }
-            tc_fence_after();
-            const uint64_t bdesc = smem_desc(q_s + (qb * NG + g) * C::GBYTES, 16, C::SBO, C::SW_LAYOUT);
-            const uint32_t d = tmem_base + ap.stage * C::N;
-#pragma unroll
-            for (int kk = 0; kk < D_I / 32; ++kk)   // K = 32 e4m3 (32 bytes) per instruction
-              mma_f8_ss(d, adesc + 2 * kk, bdesc + 2 * kk, idesc, kk > 0 ? 1u : 0u);
-            mma_commit(bar(Bars::ACC_FULL + ap.stage));
-            ap.advance();
+  if (warp < C::EPI_WARP0) {
+    if (warp == 0) {
+      // ------------------------------------------------------------------ TMA producer
+      if (lane == 0) {
+        Pipe<KSTAGES> kp;
+        int k_issued = 0;                 // k tiles issued so far
+        int q_issued[QBUF] = {};          // per q buffer: loads issued
+        uint32_t q_par[QBUF] = {};        // per q buffer: parity of its last load
+        int qi = 0;
+        bool ok = true;
+        for (int item = first_item(); has_item(item) && ok; item = next_item(item), ++qi) {
+          const IndexerItem it = indexer_item<MODE, C::TOK>(p, item, prefix, tr);
+          const int qb = qi % QBUF;
+          const uint32_t qph = (qi / QBUF) & 1;
+          if (!mbar_wait(bar(Bars::Q_EMPTY + qb), qph ^ 1, abort_flag)) { ok = false; break; }
+          mbar_arrive_expect_tx(bar(Bars::Q_FULL + qb), NG * C::GBYTES);
+          for (int g = 0; g < NG; ++g)
+            tma_load_2d(q_s + (qb * NG + g) * C::GBYTES, &tm_q, bar(Bars::Q_FULL + qb), 0,
+                        (it.q_row0 + g * NT) * H_I);
+          q_issued[qb] += 1;
+          q_par[qb] = qph;
+          for (int tile = it.tile0; tile < it.tile1; ++tile) {
+            if (!tile_active(it, tile)) continue;
+            if (!mbar_wait(bar(Bars::K_EMPTY + kp.stage), kp.phase ^ 1, abort_flag)) { ok = false; break; }
+            mbar_arrive_expect_tx(bar(Bars::K_FULL + kp.stage), C::KBYTES);
+            tma_load_2d(k_s + kp.stage * C::KBYTES, &tm_k, bar(Bars::K_FULL + kp.stage), 0,
+                        static_cast<int>(key_row(it, tile, 0)));
+            kp.advance();
+            ++k_issued;
           }
-          mma_commit(bar(Bars::K_EMPTY + kp.stage));
-          kp.advance();
         }
-        mma_commit(bar(Bars::Q_EMPTY + qb));
+        if (*abort_flag) {
+          // leave no TMA write in flight into this CTA's shared memory: wait (bounded) for the last load
+          // issued on every k stage and q buffer
+          for (int st = 0; st < KSTAGES && st < k_issued; ++st)
+            mbar_wait_drain(bar(Bars::K_FULL + st), st < kp.stage ? kp.phase : kp.phase ^ 1);
+          for (int b = 0; b < QBUF; ++b)
+            if (q_issued[b]) mbar_wait_drain(bar(Bars::Q_FULL + b), q_par[b]);
+        }
+      }
+    } else if (warp == 1) {
+      // ------------------------------------------------------------------ MMA issue
+      if (lane == 0) {
+        Pipe<KSTAGES> kp;
+        Pipe<C::NACC> ap;
+        constexpr uint32_t idesc = idesc_e4m3(128, C::N);
+        int qi = 0;
+        bool ok = true;
+        for (int item = first_item(); has_item(item) && ok; item = next_item(item), ++qi) {
+          const IndexerItem it = indexer_item<MODE, C::TOK>(p, item, prefix, tr);
+          const int qb = qi % QBUF;
+          if (!mbar_wait(bar(Bars::Q_FULL + qb), (qi / QBUF) & 1, abort_flag)) { ok = false; break; }
+          tc_fence_after();
+          for (int tile = it.tile0; tile < it.tile1 && ok; ++tile) {
+            if (!tile_active(it, tile)) continue;
+            if (!mbar_wait(bar(Bars::K_FULL + kp.stage), kp.phase, abort_flag)) { ok = false; break; }
+            tc_fence_after();
+            const uint64_t adesc = smem_desc(k_s + kp.stage * C::KBYTES, 16, C::SBO, C::SW_LAYOUT);
+            for (int g = 0; g < NG; ++g) {
+              if (!group_active<NT>(it, tile, g)) continue;
+              if (!mbar_wait(bar(Bars::ACC_EMPTY + ap.stage), ap.phase ^ 1, abort_flag)) { ok = false; break; }
+              tc_fence_after();
+              const uint64_t bdesc = smem_desc(q_s + (qb * NG + g) * C::GBYTES, 16, C::SBO, C::SW_LAYOUT);
+              const uint32_t d = tmem_base + ap.stage * C::N;
+  #pragma unroll
+              for (int kk = 0; kk < D_I / 32; ++kk)   // K = 32 e4m3 (32 bytes) per instruction
+                mma_f8_ss(d, adesc + 2 * kk, bdesc + 2 * kk, idesc, kk > 0 ? 1u : 0u);
+              mma_commit(bar(Bars::ACC_FULL + ap.stage));
+              ap.advance();
+            }
+            mma_commit(bar(Bars::K_EMPTY + kp.stage));
+            kp.advance();
+          }
+          mma_commit(bar(Bars::Q_EMPTY + qb));
+        }
       }
     }
   } else {
     // ------------------------------------------------------------------ epilogue
-    constexpr int CPT = C::N / EPI_WG;              // accumulator columns per thread
+    // Alternate stages (C::ALT_STAGES): warpgroup h reads the accumulator stages of parity h, all N columns.  The
+    // two warps sharing a sub-partition then work on different stages, and one computes while the other waits
+    // for its tensor-memory loads; with a column half each, both waited at the same moments and left the
+    // sub-partition idle.
+    constexpr int CPT = C::ALT_STAGES ? C::N : C::N / EPI_WG;   // accumulator columns per thread and stage
     constexpr int TOKS = (CPT >= H_I) ? CPT / H_I : 1;  // query rows per thread
-    constexpr int P = (H_I >= 16) ? 4 : 1;         // partial sums per row (ILP)
-    // Packed epilogue (heads in groups of four): w ReLU(x) is formed as w max(x, 0) for even heads (ALU pipe)
+    constexpr int INF_TOKS = (NT / EPI_WG > 0) ? NT / EPI_WG : 1;   // rows of a skipped group per thread
+    // Packed epilogue (heads in pairs): w ReLU(x) is formed as w max(x, 0) for even heads (ALU pipe)
     // and as (w / 2)(x + |x|) for odd heads (FMA pipe, |x| as an operand modifier), so that the two pipes share
     // the ReLUs; the odd heads' weights are stored halved.  Both forms are exact for integer-valued inputs.
-    constexpr bool kPacked = (H_I % 64 == 0) && (CPT % 64 == 0);
-    const int e = warp - 2;
+    constexpr bool kPacked = (H_I == 64) && ((C::N / EPI_WG) % 64 == 0);
+    constexpr int P = kPacked ? 1 : ((H_I >= 16) ? 4 : 1);   // partial sums per row (ILP)
+    // Fragment reads (kPacked): the accumulator is read in 16-lane x 256-bit fragments, so that a thread holds
+    // four keys (lanes g, g + 8, g + 16, g + 24 of its warp's 32, g = lane / 4) and, of every eight columns, the
+    // two columns 2c, 2c + 1 (c = lane % 4).  One 8-byte load of a head-weight pair then serves four keys, where
+    // per-key reads (one key per thread) broadcast every weight to the whole warp, and a warp-uniform 16-byte
+    // shared load takes four wavefronts.  Each thread sums its sixteen heads of a token, and two shuffle rounds
+    // (lane ^ 1, lane ^ 2) add the four partial sums of a key, leaving thread (g, c) with key
+    // g + 8 (c >> 1) + 16 (c & 1).
+    const int e = warp - C::EPI_WARP0;
     const int quad = warp & 3;
     const int half = e >> 2;
     const int ethreads = 32 * C::NUM_EPI_WARPS;
     const int etid = e * 32 + lane;
     const uint32_t lane_addr = static_cast<uint32_t>(quad * 32) << 16;
+    const int fc = lane & 3, fg = lane >> 2;        // fragment column pair and row (kPacked)
+    const int key_lane = kPacked ? fg + 8 * (fc >> 1) + 16 * (fc & 1) : lane;   // this thread's key in the warp
     Pipe<C::NACC> ap;
     int qi = 0;
     bool ok = true;
@@ -446,30 +470,36 @@ indexer_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
       // key scales are loaded one tile ahead: a load issued at the start of its own tile would expose the
       // global-memory latency once per tile (the epilogue needs it a few hundred cycles later)
       auto kscale_of = [&](int tile) -> float {
-        const int s = tile * 128 + quad * 32 + lane;
-        return (p.k_scale && tile < it.tile1 && s < it.n_keys) ? p.k_scale[key_row(it, tile, quad * 32 + lane)] : 1.f;
+        const int s = tile * 128 + quad * 32 + key_lane;
+        return (p.k_scale && tile < it.tile1 && s < it.n_keys) ? p.k_scale[key_row(it, tile, quad * 32 + key_lane)]
+                                                                : 1.f;
       };
       float kscale_next = kscale_of(it.tile0);
       for (int tile = it.tile0; tile < it.tile1; ++tile) {
-        const int s = tile * 128 + quad * 32 + lane;      // key of this thread
+        const int s = tile * 128 + quad * 32 + key_lane;      // key of this thread
         const bool key_ok = s < it.n_keys;
         const float kscale = kscale_next;
         kscale_next = kscale_of(tile + 1);
         for (int g = 0; g < NG; ++g) {
           if (g * NT >= it.n_tok) break;
-          const int tok0 = g * NT + half * (CPT / H_I > 0 ? CPT / H_I : 0);  // first row of this thread
           if (!group_active<NT>(it, tile, g)) {
             if constexpr (MODE != kModeDecode) {
               if (key_ok) {
 #pragma unroll
-                for (int tk = 0; tk < TOKS; ++tk) {
-                  const int r = tok0 + tk;
+                for (int tk = 0; tk < INF_TOKS; ++tk) {
+                  const int r = g * NT + half * INF_TOKS + tk;
                   if (r < it.n_tok) p.scores[it.out_base + static_cast<long long>(r) * it.ld + s] = -INFINITY;
                 }
               }
             }
             continue;
           }
+          if (C::ALT_STAGES && (ap.stage & 1) != half) {   // the other warpgroup's stage
+            ap.advance();
+            continue;
+          }
+          // first row of this thread
+          const int tok0 = g * NT + (C::ALT_STAGES ? 0 : half * (CPT / H_I > 0 ? CPT / H_I : 0));
           if (!mbar_wait(bar(Bars::ACC_FULL + ap.stage), ap.phase, abort_flag)) { ok = false; break; }
           tc_fence_after();
           float acc[TOKS][P];
@@ -477,47 +507,75 @@ indexer_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
           for (int tk = 0; tk < TOKS; ++tk)
 #pragma unroll
             for (int q = 0; q < P; ++q) acc[tk][q] = 0.f;
-          const uint32_t tcol = tmem_base + ap.stage * C::N + half * CPT;
+          const uint32_t tcol = tmem_base + ap.stage * C::N + (C::ALT_STAGES ? 0 : half * CPT);
           if constexpr (kPacked) {
-            uint64_t acc2[TOKS][2];
-#pragma unroll
-            for (int tk = 0; tk < TOKS; ++tk) acc2[tk][0] = acc2[tk][1] = 0ull;
-            // tensor-memory loads run two 32-column chunks ahead of the arithmetic (a ring of three register
-            // buffers): only the first wait of a stage is exposed
-            constexpr int NCH = CPT / 32;
-            constexpr int RD = 3;
+            // Chunks of 64 columns (one token) x 16 lanes: c = 2 * token + lane half.  A tcgen05.wait::ld waits for
+            // every load in flight, so a load is hidden only behind the arithmetic done between its issue and the
+            // next wait.  One chunk is loaded per chunk computed, LEAD chunks ahead, and the warp waits once per
+            // SPAN chunks (a ring of LEAD + SPAN register buffers).  Two loads issued back to back, with no
+            // arithmetic between them, ran far slower.
+            constexpr int NCH = 2 * TOKS;
+            constexpr int SPAN = C::ALT_STAGES ? 2 : 1;
+            constexpr int LEAD = 2;
+            constexpr int RD = LEAD + SPAN;
+            uint64_t acc2[4];           // the current token: [key slot 2 * half + (row g: 0, row g + 8: 1)]
+            auto chunk_addr = [&](int c) -> uint32_t {
+              return lane_addr + (static_cast<uint32_t>(16 * (c & 1)) << 16) + tcol + 64 * (c >> 1);
+            };
             uint32_t v[RD][32];
 #pragma unroll
-            for (int c = 0; c < RD - 1 && c < NCH; ++c) tmem_ld32(lane_addr + tcol + 32 * c, v[c]);
+            for (int c = 0; c < LEAD && c < NCH; ++c) tmem_ld16x256_x8(chunk_addr(c), v[c]);
             tmem_wait_ld();
 #pragma unroll
-            for (int c = 0; c < RD - 1 && c < NCH; ++c) tmem_regs_after_wait(v[c]);
+            for (int c = 0; c < LEAD && c < NCH; ++c) tmem_regs_after_wait(v[c]);
+            uint64_t ww[8];             // (w[8m + 2c], w[8m + 2c + 1] / 2) of the current token
+            const bool odd1 = (fc & 1) != 0, odd2 = (fc & 2) != 0;
 #pragma unroll
             for (int c = 0; c < NCH; ++c) {
-              if (c + RD - 1 < NCH) tmem_ld32(lane_addr + tcol + 32 * (c + RD - 1), v[(c + RD - 1) % RD]);
-              const int tk = (32 * c) / H_I;
-              const float4* w4 = reinterpret_cast<const float4*>(wq + (tok0 + tk) * H_I + ((32 * c) % H_I));
+              if (c + LEAD < NCH) tmem_ld16x256_x8(chunk_addr(c + LEAD), v[(c + LEAD) % RD]);
+              const int tk = c >> 1, hl = c & 1;
+              if (hl == 0) {
+                const uint64_t* wp = reinterpret_cast<const uint64_t*>(wq + (tok0 + tk) * H_I + 2 * fc);
 #pragma unroll
-              for (int i = 0; i < 32; i += 4) {
-                const float4 ww = w4[i >> 2];
-                float a[4];
+                for (int m = 0; m < 8; ++m) ww[m] = wp[4 * m];
 #pragma unroll
-                for (int u = 0; u < 4; ++u) {
-                  const float x = __uint_as_float(v[c % RD][i + u]);
-                  a[u] = (u & 1) ? x + fabsf(x) : fmaxf(x, 0.f);
+                for (int ks = 0; ks < 4; ++ks) acc2[ks] = 0ull;
+              }
+#pragma unroll
+              for (int m = 0; m < 8; ++m) {
+#pragma unroll
+                for (int r = 0; r < 2; ++r) {
+                  const float x0 = __uint_as_float(v[c % RD][4 * m + 2 * r]);
+                  const float x1 = __uint_as_float(v[c % RD][4 * m + 2 * r + 1]);
+                  acc2[2 * hl + r] = fma_f32x2(ww[m], pack_f32x2(fmaxf(x0, 0.f), x1 + fabsf(x1)), acc2[2 * hl + r]);
                 }
-                acc2[tk][0] = fma_f32x2(pack_f32x2(ww.x, ww.y), pack_f32x2(a[0], a[1]), acc2[tk][0]);
-                acc2[tk][1] = fma_f32x2(pack_f32x2(ww.z, ww.w), pack_f32x2(a[2], a[3]), acc2[tk][1]);
               }
-              if (c + RD - 1 < NCH) {
-                tmem_wait_ld();
-                tmem_regs_after_wait(v[(c + RD - 1) % RD]);
-              }
-            }
+              if (hl == 1) {
+                // the four partial sums of a key: lane ^ 1 trades lane halves, then lane ^ 2 trades rows g / g + 8
+                float sm[4];
 #pragma unroll
-            for (int tk = 0; tk < TOKS; ++tk) {
-              unpack_f32x2(acc2[tk][0], acc[tk][0], acc[tk][1]);
-              unpack_f32x2(acc2[tk][1], acc[tk][2], acc[tk][3]);
+                for (int ks = 0; ks < 4; ++ks) {
+                  float lo, hi;
+                  unpack_f32x2(acc2[ks], lo, hi);
+                  sm[ks] = lo + hi;
+                }
+                float t1[2];
+#pragma unroll
+                for (int r = 0; r < 2; ++r) {
+                  const float keep = odd1 ? sm[2 + r] : sm[r];
+                  const float send = odd1 ? sm[r] : sm[2 + r];
+                  t1[r] = keep + __shfl_xor_sync(0xffffffffu, send, 1);
+                }
+                const float keep = odd2 ? t1[1] : t1[0];
+                const float send = odd2 ? t1[0] : t1[1];
+                acc[tk][0] = keep + __shfl_xor_sync(0xffffffffu, send, 2);
+              }
+              if (c % SPAN == SPAN - 1 && c + 1 - SPAN + LEAD < NCH) {   // loads issued since the last wait
+                tmem_wait_ld_after(acc2[2 * hl], acc2[2 * hl + 1], acc[tk][0]);
+#pragma unroll
+                for (int b = 0; b < SPAN; ++b)
+                  if (c + 1 - SPAN + LEAD + b < NCH) tmem_regs_after_wait(v[(c + 1 - SPAN + LEAD + b) % RD]);
+              }
             }
           } else {
 #pragma unroll

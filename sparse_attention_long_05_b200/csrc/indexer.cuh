@@ -457,14 +457,16 @@ indexer_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
       float* wq = w_s + (qi % QBUF) * C::W_FLOATS;
       named_bar_sync(1, ethreads);
       for (int i = etid; i < C::W_FLOATS; i += ethreads) {
-        const int r = i / H_I;
+        const int r = i / H_I, j = i % H_I;
         float v = 0.f;
         if (r < it.n_tok) {
-          v = p.w[static_cast<long long>(it.q_row0 + r) * H_I + (i % H_I)];
+          v = p.w[static_cast<long long>(it.q_row0 + r) * H_I + j];
           if (p.q_scale) v *= p.q_scale[it.q_row0 + r];
-          if (kPacked && (i & 1)) v *= 0.5f;
+          if (kPacked && (j & 1)) v *= 0.5f;
         }
-        wq[i] = v;
+        // kPacked: head j = 8m + 2c + e goes to 16c + 2m + e, so that the sixteen weights of fragment column
+        // pair c lie together (four 16-byte loads per token)
+        wq[kPacked ? r * H_I + 16 * ((j >> 1) & 3) + 2 * (j >> 3) + (j & 1) : i] = v;
       }
       named_bar_sync(1, ethreads);
       // key scales are loaded one tile ahead: a load issued at the start of its own tile would expose the
@@ -535,11 +537,13 @@ indexer_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
               if (c + LEAD < NCH) tmem_ld16x256_x8(chunk_addr(c + LEAD), v[(c + LEAD) % RD]);
               const int tk = c >> 1, hl = c & 1;
               if (hl == 0) {
-                const uint64_t* wp = reinterpret_cast<const uint64_t*>(wq + (tok0 + tk) * H_I + 2 * fc);
+                const ulonglong2* wp = reinterpret_cast<const ulonglong2*>(wq + (tok0 + tk) * H_I + 16 * fc);
 #pragma unroll
-                for (int m = 0; m < 8; ++m) ww[m] = wp[4 * m];
-#pragma unroll
-                for (int ks = 0; ks < 4; ++ks) acc2[ks] = 0ull;
+                for (int m = 0; m < 8; m += 2) {
+                  const ulonglong2 q2 = wp[m >> 1];
+                  ww[m] = q2.x;
+                  ww[m + 1] = q2.y;
+                }
               }
 #pragma unroll
               for (int m = 0; m < 8; ++m) {
@@ -547,7 +551,8 @@ indexer_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                 for (int r = 0; r < 2; ++r) {
                   const float x0 = __uint_as_float(v[c % RD][4 * m + 2 * r]);
                   const float x1 = __uint_as_float(v[c % RD][4 * m + 2 * r + 1]);
-                  acc2[2 * hl + r] = fma_f32x2(ww[m], pack_f32x2(fmaxf(x0, 0.f), x1 + fabsf(x1)), acc2[2 * hl + r]);
+                  const uint64_t a2 = pack_f32x2(fmaxf(x0, 0.f), x1 + fabsf(x1));
+                  acc2[2 * hl + r] = (m == 0) ? mul_f32x2(ww[m], a2) : fma_f32x2(ww[m], a2, acc2[2 * hl + r]);
                 }
               }
               if (hl == 1) {

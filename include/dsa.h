@@ -50,7 +50,9 @@ typedef enum {
   DSA_ERR_CUDA = 4,               /* a CUDA runtime / driver call failed */
   DSA_ERR_TIMEOUT = 5,            /* device: a pipeline wait ran out of its clock budget */
   DSA_ERR_BAD_INDEX = 6,          /* device: a selected index was outside [-1, S) (treated as -1) */
-  DSA_ERR_WORKSPACE = 7           /* workspace missing or smaller than *_workspace_size() */
+  DSA_ERR_WORKSPACE = 7,          /* workspace missing or smaller than *_workspace_size() */
+  DSA_ERR_CHECK = 8               /* device, DSA_CHECKS builds only: pipeline bookkeeping or a result invariant
+                                     failed (see dsa_checks_enabled) */
 } dsa_status_t;
 
 /* Human-readable name of a status code (static storage). */
@@ -73,6 +75,30 @@ DSA_API dsa_status_t dsa_check_bounded_wait(int32_t* result, void* stream);
 
 /* Number of SMs the launches of the current device are sized for (148 on a B200). */
 DSA_API int dsa_num_sms(void);
+
+/* 1 in a library built with -DDSA_CHECKS (libdsa_checks.so), 0 otherwise.  That debug build runs the same
+ * kernels with checks that record DSA_ERR_CHECK or DSA_ERR_BAD_INDEX in the device status word (read it with
+ * dsa_get_device_status), and otherwise leave every result as the normal build computes it:
+ *   - indexer: the TMA producer, the MMA issuer and the epilogue count the key tiles and accumulator stages they
+ *     pass through, and the counts must agree when the kernel ends; every key tile and query group it loads
+ *     starts inside its tensor;
+ *   - top-k: a check kernel after each top-k launch verifies every output row: min(k, n) entries, strictly
+ *     ascending, each in [0, n) for the row's n keys, then -1 (the selection rule of the velog.io DSA page,
+ *     §1.2, leaves exactly that many);
+ *   - attention: wherever a token's key count is known (the prefill and decode paths, not dsa_sparse_mla_attn),
+ *     a selected entry must lie below it (causality), else DSA_ERR_BAD_INDEX; every warp that walks the
+ *     tokens' key tiles counts them, and the counts of a CTA's warps must agree.
+ * The checks cost time; the normal build compiles none of them. */
+DSA_API int dsa_checks_enabled(void);
+
+/* Self-test of the DSA_CHECKS build: plants one violation the checks must catch, on `stream`.
+ *   which = 0: a top-k output row that is not ascending -> the device status becomes DSA_ERR_CHECK;
+ *   which = 1: a selected entry beyond its token's key count (inside the latent) -> DSA_ERR_BAD_INDEX.
+ * scratch: caller-owned device buffer of dsa_checks_selftest_bytes() bytes (16-byte aligned), overwritten.
+ * Read the outcome with dsa_get_device_status.  Returns DSA_ERR_UNSUPPORTED_SHAPE in the normal build (nothing
+ * launched), DSA_ERR_INVALID_ARG for a null scratch or another `which`.  No counterpart in the paper. */
+DSA_API size_t dsa_checks_selftest_bytes(void);
+DSA_API dsa_status_t dsa_checks_selftest(int which, void* scratch, void* stream);
 
 /*
  * Lightning-indexer scores, materialised for T query rows (velog.io section 1.1).

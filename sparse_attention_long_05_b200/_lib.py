@@ -14,9 +14,11 @@ import torch
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libdsa.so")
+CHECKS_LIB_PATH = os.path.join(_HERE, "libdsa_checks.so")   # the -DDSA_CHECKS build (debugging)
 
 _STATUS = {0: "DSA_OK", 1: "DSA_ERR_INVALID_ARG", 2: "DSA_ERR_UNSUPPORTED_SHAPE", 3: "DSA_ERR_ALIGNMENT",
-           4: "DSA_ERR_CUDA", 5: "DSA_ERR_TIMEOUT", 6: "DSA_ERR_BAD_INDEX", 7: "DSA_ERR_WORKSPACE"}
+           4: "DSA_ERR_CUDA", 5: "DSA_ERR_TIMEOUT", 6: "DSA_ERR_BAD_INDEX", 7: "DSA_ERR_WORKSPACE",
+           8: "DSA_ERR_CHECK"}
 
 # exported symbols and their C signatures
 _P, _I, _I64, _F, _SZ = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_float, ctypes.c_size_t
@@ -25,6 +27,9 @@ SIGNATURES = {
     "dsa_get_device_status": (_I, [_P, ctypes.POINTER(ctypes.c_int)]),
     "dsa_check_bounded_wait": (_I, [_P, _P]),
     "dsa_num_sms": (_I, []),
+    "dsa_checks_enabled": (_I, []),
+    "dsa_checks_selftest_bytes": (_SZ, []),
+    "dsa_checks_selftest": (_I, [_I, _P, _P]),
     "dsa_indexer_scores": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P, _P]),
     "dsa_topk": (_I, [_P, _I, _I64, _P, _I, _I, _P, _P]),
     "dsa_sparse_mla_attn": (_I, [_P, _P, _I, _P, _I, _I, _I, _F, _P, _P, _P]),
@@ -76,6 +81,27 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
 
 
 _lib = load()
+
+
+def use_library(path: str = LIB_PATH) -> str:
+    """Route every binding below to the library at `path` (e.g. CHECKS_LIB_PATH, the -DDSA_CHECKS build, which
+    exports the same entry points); returns the path in use before."""
+    global _lib
+    prev = _lib._name
+    _lib = load(path)
+    return prev
+
+
+def dsa_checks_enabled() -> bool:
+    return bool(_lib.dsa_checks_enabled())
+
+
+def dsa_checks_selftest(which: int, stream=None) -> int:
+    """Plant violation `which` (0: a malformed top-k row, 1: a non-causal selected entry) in the checking build
+    and return the device status it leaves."""
+    scratch = torch.empty((int(_lib.dsa_checks_selftest_bytes()),), dtype=torch.uint8, device="cuda")
+    _check("dsa_checks_selftest", _lib.dsa_checks_selftest(which, _ptr(scratch), _stream(stream)))
+    return dsa_get_device_status(stream)
 
 
 def _ptr(t):

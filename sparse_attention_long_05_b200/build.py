@@ -16,6 +16,7 @@ ROOT = os.path.dirname(HERE)
 SRC = os.path.join(HERE, "csrc", "dsa_api.cu")
 OUT = os.path.join(HERE, "libdsa.so")
 OUT_TRACE = os.path.join(HERE, "libdsa_trace.so")   # -DDSA_TRACE: pipeline event stamps, profiling only
+OUT_CHECKS = os.path.join(HERE, "libdsa_checks.so")  # -DDSA_CHECKS: bookkeeping and invariant checks, debugging
 DEPS = [os.path.join(HERE, "csrc", f) for f in os.listdir(os.path.join(HERE, "csrc"))] + \
        [os.path.join(ROOT, "include", "dsa.h")]
 
@@ -70,9 +71,24 @@ def build_traced(verbose: bool = False) -> str:
     return OUT_TRACE
 
 
+def build_checks(verbose: bool = False) -> str:
+    """The same library with the kernels' debug checks compiled in (a separate .so; see dsa_checks_enabled in
+    include/dsa.h)."""
+    cmd = command(out=OUT_CHECKS, extra=("-DDSA_CHECKS",))
+    if verbose:
+        print(" ".join(cmd), flush=True)
+    res = subprocess.run(cmd, capture_output=True, text=True)
+    if res.returncode != 0:
+        sys.stderr.write(res.stdout + res.stderr)
+        raise RuntimeError("nvcc failed building libdsa_checks.so")
+    return OUT_CHECKS
+
+
 if __name__ == "__main__":
     if "--trace" in sys.argv:
         print(build_traced(verbose=True))
+    elif "--checks" in sys.argv:
+        print(build_checks(verbose=True))
     else:
         build(force="--force" in sys.argv, verbose=True,
               extra=("-Xptxas", "-v") if "--ptxas-v" in sys.argv else ())

@@ -24,6 +24,19 @@ __device__ long long g_wait_limit = (1ll << 31);
 
 __device__ __forceinline__ void raise_status(int code) { atomicCAS(&g_dev_status, 0, code); }
 
+// ------------------------------------------------------------------------------------------ debug checks
+// Built with -DDSA_CHECKS (the checking library, libdsa_checks.so), kernels verify their pipeline bookkeeping and
+// result invariants and record DSA_ERR_CHECK (DSA_ERR_BAD_INDEX for a selection outside a token's keys) in the
+// status word.  In the normal build kChecks is false and the checks compile to nothing.
+#ifdef DSA_CHECKS
+constexpr bool kChecks = true;
+#else
+constexpr bool kChecks = false;
+#endif
+__device__ __forceinline__ void check_that(bool cond, int code = DSA_ERR_CHECK) {
+  if (kChecks && !cond) raise_status(code);
+}
+
 // ------------------------------------------------------------------------------------------ tracing
 // Built with -DDSA_TRACE (the traced library, libdsa_trace.so), kernels record %globaltimer stamps of their
 // pipeline events for the first cluster / CTA into g_trace[event][tile]; read back with dsa_trace_read().

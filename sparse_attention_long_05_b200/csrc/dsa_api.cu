@@ -274,9 +274,12 @@ dsa_status_t launch_indexer(const uint8_t* q_idx, int q_rows, const uint8_t* k_i
   if (!make_map(&tq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, q_idx, qd, qs, qb, sw)) return DSA_ERR_CUDA;
   if (!make_map(&tk, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, k_idx, kd, qs, kb, sw)) return DSA_ERR_CUDA;
   auto kern = indexer_kernel<H_I, D_I, NT, NG, QBUF, KST, EPI, MODE>;
+  IndexerParams pk = p;
+  pk.k_rows = k_rows;
+  pk.q_rows = q_rows;
   const int smem = (C::TMEM_COLS == 512 && C::SMEM < kMinIndexerSmem) ? kMinIndexerSmem : C::SMEM;
   if (set_smem(kern, smem) != cudaSuccess) return DSA_ERR_CUDA;
-  if (launch_pdl(kern, dim3(grid), dim3(C::NUM_THREADS), smem, st, tq, tk, p) != cudaSuccess) return DSA_ERR_CUDA;
+  if (launch_pdl(kern, dim3(grid), dim3(C::NUM_THREADS), smem, st, tq, tk, pk) != cudaSuccess) return DSA_ERR_CUDA;
   return last_launch_status();
 }
 
@@ -367,6 +370,25 @@ dsa_status_t run_indexer_segments(const uint8_t* q_idx, long long q_rows, const 
                                                              st);
 }
 
+#ifdef DSA_CHECKS
+// DSA_CHECKS builds: every output row of a top-k launch holds min(k, n) entries, strictly ascending and in [0, n)
+// for the row's n keys, then -1 padding.  One CTA per row; launched without the dependent-launch attribute, so
+// it starts once the top-k has finished.
+__global__ void __launch_bounds__(256) topk_check_kernel(const TopkParams p) {
+  const int r = blockIdx.x;
+  const long long n = p.row_len ? p.row_len[r] : (p.ld < p.pos0 + r + 1 ? p.ld : p.pos0 + r + 1);
+  const int m = static_cast<int>(n < p.k ? (n > 0 ? n : 0) : p.k);
+  const int* row = p.idx + static_cast<long long>(r) * p.idx_ld;
+  bool good = true;
+  for (int i = threadIdx.x; i < p.k; i += blockDim.x) {
+    const int v = row[i];
+    if (i < m) good &= v >= 0 && v < n && (i == 0 || v > row[i - 1]);
+    else good &= v == -1;
+  }
+  if (!good) raise_status(DSA_ERR_CHECK);
+}
+#endif
+
 dsa_status_t run_topk(const float* scores, long long ld, const long long* row_off, const int* row_len, int pos0,
                       int rows, int k, int* idx, long long idx_ld, cudaStream_t st, float* sel_scores = nullptr) {
   if (rows <= 0) return DSA_OK;
@@ -384,6 +406,13 @@ dsa_status_t run_topk(const float* scores, long long ld, const long long* row_of
                    p) != cudaSuccess)
       return DSA_ERR_CUDA;
   }
+#ifdef DSA_CHECKS
+  {
+    const dsa_status_t e = last_launch_status();
+    if (e != DSA_OK) return e;
+    topk_check_kernel<<<rows, 256, 0, st>>>(p);
+  }
+#endif
   return last_launch_status();
 }
 
@@ -614,6 +643,7 @@ const char* dsa_status_string(dsa_status_t s) {
     case DSA_ERR_TIMEOUT: return "DSA_ERR_TIMEOUT";
     case DSA_ERR_BAD_INDEX: return "DSA_ERR_BAD_INDEX";
     case DSA_ERR_WORKSPACE: return "DSA_ERR_WORKSPACE";
+    case DSA_ERR_CHECK: return "DSA_ERR_CHECK";
   }
   return "DSA_UNKNOWN_STATUS";
 }
@@ -630,6 +660,8 @@ dsa_status_t dsa_get_device_status(void* stream, int* device_status) {
 }
 
 int dsa_num_sms(void) { return num_sms(); }
+
+int dsa_checks_enabled(void) { return kChecks ? 1 : 0; }
 
 dsa_status_t dsa_indexer_scores(const uint8_t* q_idx, const float* q_scale, const uint8_t* k_idx,
                                 const float* k_scale, const float* w, int T, int S, int H_I, int d_I, int pos0,
@@ -1057,6 +1089,50 @@ dsa_status_t dsa_check_bounded_wait(int32_t* result, void* stream) {
   if (!aligned16(result)) return DSA_ERR_ALIGNMENT;
   wait_selfcheck_kernel<<<1, 64, 0, static_cast<cudaStream_t>(stream)>>>(result);
   return last_launch_status();
+}
+
+size_t dsa_checks_selftest_bytes(void) { return size_t(1) << 20; }
+
+dsa_status_t dsa_checks_selftest(int which, void* scratch, void* stream) {
+  if (!scratch || (which != 0 && which != 1)) return DSA_ERR_INVALID_ARG;
+  if (!aligned16(scratch)) return DSA_ERR_ALIGNMENT;
+#ifndef DSA_CHECKS
+  return DSA_ERR_UNSUPPORTED_SHAPE;
+#else
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  char* b = static_cast<char*>(scratch);
+  if (cudaMemsetAsync(b, 0, dsa_checks_selftest_bytes(), st) != cudaSuccess) return DSA_ERR_CUDA;
+  if (which == 0) {
+    // a top-k output row of k = 4 over n = 10 keys, not ascending: [5, 3, 7, -1]
+    static const int32_t row[4] = {5, 3, 7, -1};
+    static const int32_t n = 10;
+    int32_t* idx = reinterpret_cast<int32_t*>(b);
+    int32_t* len = reinterpret_cast<int32_t*>(b + 256);
+    if (cudaMemcpyAsync(idx, row, sizeof(row), cudaMemcpyHostToDevice, st) != cudaSuccess ||
+        cudaMemcpyAsync(len, &n, sizeof(n), cudaMemcpyHostToDevice, st) != cudaSuccess)
+      return DSA_ERR_CUDA;
+    if (cudaStreamSynchronize(st) != cudaSuccess) return DSA_ERR_CUDA;   // the host arrays are read now
+    TopkParams p{nullptr, 10, nullptr, len, 0, 1, 4, idx, 4, nullptr};
+    topk_check_kernel<<<1, 256, 0, st>>>(p);
+    return last_launch_status();
+  }
+  // one decode-style token with n = 200 keys of a 256-row zero latent, k = 128, 8 heads; its first selected
+  // entry (250) lies inside the latent but beyond the token's keys
+  constexpr int S = 256, H = 8, k = 128;
+  uint16_t* c = reinterpret_cast<uint16_t*>(b);                           // [S, 576] bf16 zeros
+  uint16_t* q = reinterpret_cast<uint16_t*>(b + S * 1152);                 // [1, H, 576] bf16 zeros
+  int32_t* idx = reinterpret_cast<int32_t*>(b + S * 1152 + 16384);         // [1, k]
+  int32_t* nk = idx + k;                                                   // [1]
+  uint16_t* out = reinterpret_cast<uint16_t*>(b + S * 1152 + 32768);       // [1, H, 512] bf16
+  float* lse = reinterpret_cast<float*>(b + S * 1152 + 49152);             // [1, H]
+  static int32_t host[k + 1];
+  for (int j = 0; j < k; ++j) host[j] = j;
+  host[0] = 250;
+  host[k] = 200;
+  if (cudaMemcpyAsync(idx, host, sizeof(host), cudaMemcpyHostToDevice, st) != cudaSuccess) return DSA_ERR_CUDA;
+  if (cudaStreamSynchronize(st) != cudaSuccess) return DSA_ERR_CUDA;
+  return run_mla(q, c, S, idx, nullptr, 1, H, k, 0.0416666679f, out, lse, st, kMlaCounts, nk);
+#endif
 }
 
 #ifdef DSA_TRACE

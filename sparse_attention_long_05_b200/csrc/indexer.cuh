@@ -69,6 +69,7 @@ struct IndexerParams {
   int n_segs;
   const int* page_table;       // kModeDecode, paged caches: [B, max_pages] page of each 'page_rows' positions
   int max_pages, page_rows;    // (page_rows a multiple of 128, so that a key tile lies in one page)
+  long long k_rows, q_rows;    // rows of the key and query tensor maps (DSA_CHECKS builds check the loads)
 };
 
 struct IndexerItem {
@@ -146,6 +147,9 @@ struct IndexerBars {
   static constexpr int OFF_TMEM = 8 * COUNT;         // u32: TMEM base address
   static constexpr int OFF_ABORT = OFF_TMEM + 4;     // int: abort flag
   static constexpr int OFF_NITEMS = OFF_TMEM + 8;    // int: key tiles of all sequences (decode)
+  // DSA_CHECKS: ints [key tiles loaded, key tiles consumed by MMAs, accumulator stages committed, stage reads]
+  static constexpr int OFF_CHECK = OFF_NITEMS + 4;
+  static_assert(OFF_CHECK + 16 <= 2048, "barrier area");
 };
 
 // decode: the key-tile range [lo, hi) of this CTA over the tiles of all sequences laid end to end
@@ -255,6 +259,9 @@ indexer_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
       mbar_init(bar(Bars::ACC_EMPTY + i), C::ACC_READERS);
     }
     *abort_flag = 0;
+    if constexpr (kChecks) {
+      for (int i = 0; i < 4; ++i) reinterpret_cast<int*>(smem + Bars::OFF_CHECK)[i] = 0;
+    }
     fence_mbar_init();
   }
   pdl_allow_next();
@@ -359,21 +366,25 @@ indexer_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
           const uint32_t qph = (qi / QBUF) & 1;
           if (!mbar_wait(bar(Bars::Q_EMPTY + qb), qph ^ 1, abort_flag)) { ok = false; break; }
           mbar_arrive_expect_tx(bar(Bars::Q_FULL + qb), NG * C::GBYTES);
-          for (int g = 0; g < NG; ++g)
+          for (int g = 0; g < NG; ++g) {
+            check_that(it.q_row0 + g * NT < p.q_rows || g * NT >= it.n_tok);
             tma_load_2d(q_s + (qb * NG + g) * C::GBYTES, &tm_q, bar(Bars::Q_FULL + qb), 0,
                         (it.q_row0 + g * NT) * H_I);
+          }
           q_issued[qb] += 1;
           q_par[qb] = qph;
           for (int tile = it.tile0; tile < it.tile1; ++tile) {
             if (!tile_active(it, tile)) continue;
             if (!mbar_wait(bar(Bars::K_EMPTY + kp.stage), kp.phase ^ 1, abort_flag)) { ok = false; break; }
             mbar_arrive_expect_tx(bar(Bars::K_FULL + kp.stage), C::KBYTES);
+            check_that(key_row(it, tile, 0) >= 0 && key_row(it, tile, 0) < p.k_rows);
             tma_load_2d(k_s + kp.stage * C::KBYTES, &tm_k, bar(Bars::K_FULL + kp.stage), 0,
                         static_cast<int>(key_row(it, tile, 0)));
             kp.advance();
             ++k_issued;
           }
         }
+        if constexpr (kChecks) reinterpret_cast<int*>(smem + Bars::OFF_CHECK)[0] = k_issued;
         if (*abort_flag) {
           // leave no TMA write in flight into this CTA's shared memory: wait (bounded) for the last load
           // issued on every k stage and q buffer
@@ -391,6 +402,7 @@ indexer_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         constexpr uint32_t idesc = idesc_e4m3(128, C::N);
         int qi = 0;
         bool ok = true;
+        [[maybe_unused]] int chk_tiles = 0, chk_stages = 0;
         for (int item = first_item(); has_item(item) && ok; item = next_item(item), ++qi) {
           const IndexerItem it = indexer_item<MODE, C::TOK>(p, item, prefix, tr);
           const int qb = qi % QBUF;
@@ -407,16 +419,22 @@ indexer_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
               tc_fence_after();
               const uint64_t bdesc = smem_desc(q_s + (qb * NG + g) * C::GBYTES, 16, C::SBO, C::SW_LAYOUT);
               const uint32_t d = tmem_base + ap.stage * C::N;
-  #pragma unroll
+#pragma unroll
               for (int kk = 0; kk < D_I / 32; ++kk)   // K = 32 e4m3 (32 bytes) per instruction
                 mma_f8_ss(d, adesc + 2 * kk, bdesc + 2 * kk, idesc, kk > 0 ? 1u : 0u);
               mma_commit(bar(Bars::ACC_FULL + ap.stage));
               ap.advance();
+              if constexpr (kChecks) ++chk_stages;
             }
             mma_commit(bar(Bars::K_EMPTY + kp.stage));
             kp.advance();
+            if constexpr (kChecks) ++chk_tiles;
           }
           mma_commit(bar(Bars::Q_EMPTY + qb));
+        }
+        if constexpr (kChecks) {
+          reinterpret_cast<int*>(smem + Bars::OFF_CHECK)[1] = chk_tiles;
+          reinterpret_cast<int*>(smem + Bars::OFF_CHECK)[2] = chk_stages;
         }
       }
     }
@@ -452,6 +470,7 @@ indexer_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     Pipe<C::NACC> ap;
     int qi = 0;
     bool ok = true;
+    [[maybe_unused]] int chk_reads = 0;    // accumulator stages this warp read (DSA_CHECKS)
     for (int item = first_item(); has_item(item) && ok; item = next_item(item), ++qi) {
       const IndexerItem it = indexer_item<MODE, C::TOK>(p, item, prefix, tr);
       float* wq = w_s + (qi % QBUF) * C::W_FLOATS;
@@ -603,6 +622,7 @@ indexer_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
           __syncwarp();
           if (lane == 0) mbar_arrive(bar(Bars::ACC_EMPTY + ap.stage));
           ap.advance();
+          if constexpr (kChecks) ++chk_reads;
           if (key_ok) {
 #pragma unroll
             for (int tk = 0; tk < TOKS; ++tk) {
@@ -623,11 +643,20 @@ indexer_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         if (!ok) break;
       }
     }
+    if constexpr (kChecks) {
+      if (lane == 0) atomicAdd(reinterpret_cast<int*>(smem + Bars::OFF_CHECK) + 3, chk_reads);
+    }
   }
 
   // ------------------------------------------------------------------ teardown
   tc_fence_before();
   __syncthreads();
+  if constexpr (kChecks) {
+    // every key tile loaded went through the MMAs, and every accumulator stage committed was read by the
+    // ACC_READERS epilogue warps that take it (a wait that ran out has already recorded DSA_ERR_TIMEOUT)
+    const int* chk = reinterpret_cast<const int*>(smem + Bars::OFF_CHECK);
+    if (threadIdx.x == 0 && !*abort_flag) check_that(chk[0] == chk[1] && chk[3] == chk[2] * C::ACC_READERS);
+  }
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem_base, C::TMEM_COLS);

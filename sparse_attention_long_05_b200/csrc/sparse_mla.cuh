@@ -131,6 +131,7 @@ constexpr int B_COUNT = B_RED_FREE + 2;
 // shared memory map (from a 1024-byte aligned base; both CTAs use the same barrier offsets)
 constexpr int OFF_TMEM = 8 * B_COUNT;
 constexpr int OFF_ABORT = OFF_TMEM + 4;
+constexpr int OFF_CHECK = 576;                                  // DSA_CHECKS: per warp, key tiles walked (16 ints)
 constexpr int OFF_IDX = 1024;                                   // both: 2 x 8 KB index rows
 constexpr int OFF_QST = OFF_IDX + 2 * KMAX * 4;                 // score CTA: Q staging
 constexpr int OFF_ROPE = OFF_QST + QS * QCHUNK_BYTES;           // score CTA: Q chunk 8 of the current token
@@ -141,7 +142,7 @@ constexpr int OFF_RING_V = OFF_PB + NPB * XFER;                 // value CTA: ga
 constexpr int SMEM_S = OFF_RING_S + NS_S * S_STAGE;
 constexpr int SMEM_V = OFF_RING_V + NS_V * V_STAGE;
 constexpr int SMEM = (SMEM_S > SMEM_V ? SMEM_S : SMEM_V) + 1024;
-static_assert(OFF_ABORT + 4 <= OFF_IDX, "barrier area");
+static_assert(OFF_ABORT + 4 <= OFF_CHECK && OFF_CHECK + 64 <= OFF_IDX, "barrier area");
 static_assert(OFF_QST % 1024 == 0 && OFF_ROPE % 1024 == 0 && OFF_RING_S % 1024 == 0, "1 KB aligned tiles");
 static_assert(2 * 4 * NK * 4 <= S_STAGE, "KL mode: head sums in the ring's last stage");
 static_assert(OFF_PB % 1024 == 0 && XFER % 1024 == 0 && OFF_RING_V % 1024 == 0, "1 KB aligned tiles");
@@ -186,6 +187,13 @@ template <bool PAGED>
 __device__ __forceinline__ long long mla_row(const MlaParams& p, int t, int e, long long base, int slot) {
   const bool valid = mla_valid<PAGED>(p, t, e, base);
   if (!valid && e != -1) raise_status(DSA_ERR_BAD_INDEX);
+  if constexpr (kChecks) {
+    // DSA_CHECKS: where the token's key count n is known, a selected entry lies below it (causality)
+    if (valid && p.dense != kMlaSparse) {
+      const long long n = (p.dense == kMlaCausal) ? static_cast<long long>(p.pos0) + t - base + 1 : p.n_keys[t];
+      check_that(e < n, DSA_ERR_BAD_INDEX);
+    }
+  }
   return valid ? mla_pos_row<PAGED>(p, t, base, e) : (slot < p.S ? slot : 0);
 }
 
@@ -292,6 +300,9 @@ sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
       mbar_init(bar(B_O_FREE), 4);
     }
     *abort_flag = 0;
+    if constexpr (kChecks) {
+      for (int i = 0; i < 16; ++i) reinterpret_cast<int*>(smem + OFF_CHECK)[i] = -1;
+    }
     fence_mbar_init();
   }
   if (warp == 0 && lane == 0) {
@@ -308,6 +319,9 @@ sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
   cluster_sync();        // both CTAs' barriers are initialised before any remote arrive
   tc_fence_after();
   const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(smem + OFF_TMEM);
+  // DSA_CHECKS: key tiles this thread's role walked over its tokens (every role of a CTA walks the same tokens)
+  [[maybe_unused]] int chk_tiles = 0;
+  [[maybe_unused]] bool chk_ran = false;
   // the set-up above touches no global memory; from here on the predecessor's results are read
   pdl_allow_next();
   pdl_wait();
@@ -387,6 +401,7 @@ sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
       const long long base = p.row_off ? p.row_off[t] : 0;
       const int nd = mla_dense_keys<DENSE>(p, t, base);
       const int ntiles = mla_tiles(p, nd);
+      if constexpr (kChecks) { chk_tiles += ntiles; chk_ran = true; }
       for (int j = 0; j < ntiles && ok; ++j) {
         const bool full_dense = nd >= 0 && (j + 1) * NK <= nd;    // 128 contiguous rows of keys
         const uint32_t tx = full_dense ? (gw == 0 ? sbytes : 0) : per_warp * 512;
@@ -480,6 +495,7 @@ sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
       for (int t = cluster; t < p.T && ok; t += nclusters, ++ti) {
         const bool has_next = t + nclusters < p.T;
         const int ntiles = mla_tiles(p, mla_dense_keys<DENSE>(p, t, p.row_off ? p.row_off[t] : 0));
+        if constexpr (kChecks) { chk_tiles += ntiles; chk_ran = true; }
         for (int j = 0; j < ntiles && ok; ++j, ++g) {
           const int sb = static_cast<int>(g & 1);
           const bool last = (j == ntiles - 1);
@@ -537,6 +553,7 @@ sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
       constexpr uint32_t idesc = idesc_bf16(128, 256, true);
       for (int t = cluster; t < p.T && ok; t += nclusters, ++ti) {
         const int ntiles = mla_tiles(p, mla_dense_keys<DENSE>(p, t, p.row_off ? p.row_off[t] : 0));
+        if constexpr (kChecks) { chk_tiles += ntiles; chk_ran = true; }
         for (int j = 0; j < ntiles && ok; ++j, ++g) {
           const int pb = static_cast<int>(g % NPB);
           if (j == 0 && !(ok = warp_wait(bar(B_O_FREE), (ti & 1) ^ 1, abort_flag))) break;
@@ -593,6 +610,7 @@ sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
       const long long base = p.row_off ? p.row_off[t] : 0;
       const int nd = mla_dense_keys<DENSE>(p, t, base);
       const int ntiles = mla_tiles(p, nd);
+      if constexpr (kChecks) { chk_tiles += ntiles; chk_ran = true; }
       const bool head_on = h < p.H;
       const float lse2 = head_on ? p.kl_lse[static_cast<long long>(t) * p.H + h] * kLog2e : 0.f;
       const float inv_h = 1.f / static_cast<float>(p.H);
@@ -724,6 +742,7 @@ sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
       const long long base = p.row_off ? p.row_off[t] : 0;
       const int nd = mla_dense_keys<DENSE>(p, t, base);
       const int ntiles = mla_tiles(p, nd);
+      if constexpr (kChecks) { chk_tiles += ntiles; chk_ran = true; }
       // l: sum of the bf16-rounded probabilities that enter P . V (normalises O exactly);
       // le: sum of the unrounded probabilities (for the log-sum-exp output)
       float m_ref = -INFINITY, l = 0.f, le = 0.f;
@@ -831,6 +850,7 @@ sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     bool ok = true;
     for (int t = cluster; t < p.T && ok; t += nclusters, ++ti) {
       const int ntiles = mla_tiles(p, mla_dense_keys<DENSE>(p, t, p.row_off ? p.row_off[t] : 0));
+      if constexpr (kChecks) { chk_tiles += ntiles; chk_ran = true; }
       float l = 0.f;
       for (int j = 0; j < ntiles; ++j, ++g) {
         const int pb = static_cast<int>(g % NPB);
@@ -890,8 +910,27 @@ sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
   }
 
   // ===================================================================== teardown
+  if constexpr (kChecks) {
+    // the threads of a warp that walked the key tiles agree on their count (first writer sets it)
+    if (chk_ran && !*abort_flag) {
+      const int old = atomicCAS(reinterpret_cast<int*>(smem + OFF_CHECK) + warp, -1, chk_tiles);
+      check_that(old == -1 || old == chk_tiles);
+    }
+  }
   tc_fence_before();
   __syncthreads();
+  if constexpr (kChecks) {
+    // ... and so do the warps of the CTA
+    if (threadIdx.x == 0 && !*abort_flag) {
+      const int* chk = reinterpret_cast<const int*>(smem + OFF_CHECK);
+      int ref = -1;
+      for (int w = 0; w < THREADS / 32; ++w) {
+        if (chk[w] < 0) continue;
+        if (ref < 0) ref = chk[w];
+        check_that(chk[w] == ref);
+      }
+    }
+  }
   cluster_sync();       // no CTA leaves while its peer may still touch its shared memory
   if (warp == 1) {
     tc_fence_after();

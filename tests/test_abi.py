@@ -37,8 +37,23 @@ def test_every_declared_symbol_is_exported(lib):
 
 def test_status_strings(lib):
     for code, name in [(0, b"DSA_OK"), (2, b"DSA_ERR_UNSUPPORTED_SHAPE"), (5, b"DSA_ERR_TIMEOUT"),
-                       (7, b"DSA_ERR_WORKSPACE"), (99, b"DSA_UNKNOWN_STATUS")]:
+                       (7, b"DSA_ERR_WORKSPACE"), (8, b"DSA_ERR_CHECK"), (99, b"DSA_UNKNOWN_STATUS")]:
         assert lib.dsa_status_string(code) == name
+
+
+def test_checking_build_exports_the_same_entry_points(lib):
+    """The -DDSA_CHECKS build (libdsa_checks.so) is a drop-in for libdsa.so; only it reports checks enabled."""
+    import importlib.util
+    spec = importlib.util.spec_from_file_location(
+        "dsa_build", os.path.join(ROOT, "sparse_attention_long_05_b200", "build.py"))
+    b = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(b)
+    from sparse_attention_long_05_b200 import _lib
+    chk = _lib.load(b.build_checks())
+    for n in _declared():
+        assert hasattr(chk, n), n
+    assert chk.dsa_checks_enabled() == 1 and lib.dsa_checks_enabled() == 0
+    assert chk.dsa_status_string(8) == b"DSA_ERR_CHECK"
 
 
 def test_workspace_sizes(lib):

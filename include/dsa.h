@@ -345,8 +345,8 @@ DSA_API dsa_status_t dsa_forward_decode_paged(int B, const int32_t* page_table, 
  * dsa_forward_decode without a caller-provided workspace, for callers that cannot allocate device memory
  * (for example a serving loop that runs under a memory pool it may not grow, or code that only receives
  * borrowed buffers).  This entry point has no counterpart in the paper: it is the decode step above with its
- * scratch (the packed score rows, per-sequence lengths and offsets and, when idx_out is NULL, the selected
- * indices) held in a fixed device array inside the library, of dsa_decode_noalloc_scratch_bytes() bytes
+ * scratch (the packed score rows, per-sequence lengths, offsets and score histograms and, when idx_out is NULL,
+ * the selected indices) held in a fixed device array inside the library, of dsa_decode_noalloc_scratch_bytes() bytes
  * (32 MiB).  Every GPU that loads the library keeps that array until the process exits.
  *   - Arguments and results are those of dsa_forward_decode; shapes whose dsa_decode_workspace_size()
  *     exceeds the array return DSA_ERR_WORKSPACE and launch nothing.

@@ -69,11 +69,15 @@ struct DecodeLayout {
 __global__ void __launch_bounds__(kAppendThreads)
     decode_append_kernel(int B, DecodeLayout lay, const int* ctx_len, const uint8_t* k_new,
                          const float* k_scale_new, const uint16_t* c_new, uint8_t* k_cache, float* k_scale_cache,
-                         uint16_t* c_cache, int d_I, int* len1, long long* score_off, long long score_cap) {
+                         uint16_t* c_cache, int d_I, int* len1, long long* score_off, long long score_cap,
+                         unsigned* hist) {
   pdl_allow_next();
   pdl_wait();
   const int b = blockIdx.x;
   if (b >= B) return;
+  // the sequence's score histogram, accumulated by the indexer (when the step uses one)
+  if (hist)
+    for (int i = threadIdx.x; i < kTopkBins; i += blockDim.x) hist[static_cast<long long>(b) * kTopkBins + i] = 0;
   // start of this sequence's score row: the padded lengths of the sequences before it that pass the cheap part
   // of their check (paged: the page-table entries of another sequence are not read here; a sequence that fails
   // only on those keeps its reserved row unused)
@@ -390,9 +394,10 @@ __global__ void __launch_bounds__(256) topk_check_kernel(const TopkParams p) {
 #endif
 
 dsa_status_t run_topk(const float* scores, long long ld, const long long* row_off, const int* row_len, int pos0,
-                      int rows, int k, int* idx, long long idx_ld, cudaStream_t st, float* sel_scores = nullptr) {
+                      int rows, int k, int* idx, long long idx_ld, cudaStream_t st, float* sel_scores = nullptr,
+                      const unsigned* hist = nullptr) {
   if (rows <= 0) return DSA_OK;
-  TopkParams p{scores, ld, row_off, row_len, pos0, rows, k, idx, idx_ld, sel_scores};
+  TopkParams p{scores, ld, row_off, row_len, pos0, rows, k, idx, idx_ld, sel_scores, hist};
   if (rows < num_sms()) {
     // fewer rows than SMs (decode): one cluster of kTkcCluster CTAs per row
     if (set_smem(topk_cluster_kernel, static_cast<int>(sizeof(TkcSmem))) != cudaSuccess) return DSA_ERR_CUDA;
@@ -578,12 +583,14 @@ dsa_status_t decode_args_status(int B, const int64_t* cache_off, const int32_t* 
 
 size_t decode_ws_bytes(int B, size_t score_cap, int k) {
   return align_up(score_cap * 4, 256) + align_up(size_t(B) * 4, 256) + align_up(size_t(B) * 8, 256) +
-         align_up(size_t(B) * k * 4, 256);
+         align_up(size_t(B) * k * 4, 256) + align_up(size_t(B) * kTopkBins * 4, 256);
 }
 
 // One decode step once the arguments are checked: append -> indexer over each sequence's keys -> top-k -> sparse
 // MLA.  Workspace: score rows (packed, 16-byte aligned, score_cap floats), len1 [B], score_off [B], selected
-// indices [B, k] (when idx_out is null).
+// indices [B, k] (when idx_out is null), each sequence's score histogram [B, 2048] (top 11 order-key bits).
+// With fewer sequences than SMs the indexer counts the histogram as it writes the scores, and the cluster top-k
+// reads it instead of counting the row again and merging its CTAs' counts.
 dsa_status_t run_decode(int B, const DecodeLayout& lay, const int32_t* ctx_len, const uint8_t* q_idx,
                         const float* q_scale, const float* w, const uint16_t* q, const uint8_t* k_new,
                         const float* k_scale_new, const uint16_t* c_new, uint8_t* k_cache, float* k_scale_cache,
@@ -598,8 +605,10 @@ dsa_status_t run_decode(int B, const DecodeLayout& lay, const int32_t* ctx_len, 
   long long* soff = reinterpret_cast<long long*>(wsb + at);
   at += align_up(size_t(B) * 8, 256);
   int32_t* idx = idx_out ? idx_out : reinterpret_cast<int32_t*>(wsb + at);
+  at += align_up(size_t(B) * k * 4, 256);
+  unsigned* hist = (B < num_sms()) ? reinterpret_cast<unsigned*>(wsb + at) : nullptr;
   if (launch_pdl(decode_append_kernel, dim3(B), dim3(kAppendThreads), 0, st, B, lay, ctx_len, k_new, k_scale_new,
-                 c_new, k_cache, k_scale_cache, c_cache, d_I, len1, soff, static_cast<long long>(score_cap)) !=
+                 c_new, k_cache, k_scale_cache, c_cache, d_I, len1, soff, static_cast<long long>(score_cap), hist) !=
       cudaSuccess)
     return DSA_ERR_CUDA;
   dsa_status_t e = last_launch_status();
@@ -616,11 +625,12 @@ dsa_status_t run_decode(int B, const DecodeLayout& lay, const int32_t* ctx_len, 
   p.page_table = lay.page_table;
   p.max_pages = lay.max_pages;
   p.page_rows = lay.page_rows;
+  p.hist = hist;
   using DecCfg = IndexerCfg<H_I, d_I, 1, 1, 2, 4, 1, kModeDecode>;
   e = launch_indexer<H_I, d_I, 1, 1, 2, 4, 1, kModeDecode>(q_idx, B, k_cache, lay.cache_rows, p,
                                                          DecCfg::CTAS_PER_SM * num_sms(), st);
   if (e != DSA_OK) return e;
-  e = run_topk(dscores, 0, soff, len1, 0, B, k, idx, k, st);
+  e = run_topk(dscores, 0, soff, len1, 0, B, k, idx, k, st, nullptr, hist);
   if (e != DSA_OK) return e;
   return run_mla(q, c_cache, lay.cache_rows, idx, lay.cache_off, B, H, k, scale, out, lse, st, kMlaCounts, len1,
                  lay.page_table, lay.max_pages, lay.page_rows);

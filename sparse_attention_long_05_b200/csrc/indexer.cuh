@@ -70,6 +70,8 @@ struct IndexerParams {
   const int* page_table;       // kModeDecode, paged caches: [B, max_pages] page of each 'page_rows' positions
   int max_pages, page_rows;    // (page_rows a multiple of 128, so that a key tile lies in one page)
   long long k_rows, q_rows;    // rows of the key and query tensor maps (DSA_CHECKS builds check the loads)
+  unsigned* hist;              // kModeDecode: [B, 2048] counts of the top 11 order-key bits of each sequence's
+                               // scores, accumulated (zeroed by the caller), or null
 };
 
 struct IndexerItem {
@@ -110,7 +112,10 @@ struct IndexerCfg {
   static constexpr int DEC_BYTES = 4 * (kMaxDecodeSeqs + 1) + 4 * kMaxDecodeSeqs + 8 * kMaxDecodeSeqs + 8;
   static constexpr int OFF_W = ((OFF_PREFIX + (MODE != kModeScores ? DEC_BYTES : 0) + 15) / 16) * 16;
   static constexpr int W_FLOATS = TOK * H_I;
-  static constexpr int OFF_Q = ((OFF_W + QBUF * W_FLOATS * 4 + ALIGN - 1) / ALIGN) * ALIGN;
+  // decode: the CTA's histogram of its current item's scores (top 11 order-key bits), flushed to IndexerParams::hist
+  static constexpr int OFF_HIST = OFF_W + QBUF * W_FLOATS * 4;
+  static constexpr int HIST_BYTES = (MODE == kModeDecode) ? 2048 * 4 : 0;
+  static constexpr int OFF_Q = ((OFF_HIST + HIST_BYTES + ALIGN - 1) / ALIGN) * ALIGN;
   static constexpr int OFF_K = OFF_Q + QBUF * NG * GBYTES;
   static constexpr int SMEM = OFF_K + KSTAGES * KBYTES + ALIGN;  // + alignment slack
   // accumulator ring: as many N-column accumulators as tensor memory holds (2 at N = 256), so that the MMAs
@@ -350,6 +355,9 @@ indexer_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     }
   };
 
+  // decode with a histogram: the sequence whose counts sit in the CTA's shared histogram, flushed when the next
+  // item starts and at the end of the kernel (epilogue threads)
+  [[maybe_unused]] int hist_b = -1;
   if (warp < C::EPI_WARP0) {
     if (warp == 0) {
       // ------------------------------------------------------------------ TMA producer
@@ -486,6 +494,18 @@ indexer_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         // kPacked: head j = 8m + 2c + e goes to 16c + 2m + e, so that the sixteen weights of fragment column
         // pair c lie together (four 16-byte loads per token)
         wq[kPacked ? r * H_I + 16 * ((j >> 1) & 3) + 2 * (j >> 3) + (j & 1) : i] = v;
+      }
+      if constexpr (MODE == kModeDecode) {
+        if (p.hist) {
+          // each thread owns the same bins in every item: it flushes the previous item's counts and clears them
+          unsigned* hs = reinterpret_cast<unsigned*>(smem + C::OFF_HIST);
+          for (int i = etid; i < 2048; i += ethreads) {
+            const unsigned v = hs[i];
+            if (hist_b >= 0 && v) atomicAdd(p.hist + static_cast<long long>(hist_b) * 2048 + i, v);
+            hs[i] = 0;
+          }
+          hist_b = it.q_row0;
+        }
       }
       named_bar_sync(1, ethreads);
       // key scales are loaded one tile ahead: a load issued at the start of its own tile would expose the
@@ -636,6 +656,7 @@ indexer_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                 p.scores[it.out_base + static_cast<long long>(r) * it.ld + s] = (s <= it.pos0 + r) ? sc : -INFINITY;
               } else {
                 p.scores[it.out_base + s] = sc;
+                if (p.hist) atomicAdd(reinterpret_cast<unsigned*>(smem + C::OFF_HIST) + (order_key(sc) >> 21), 1u);
               }
             }
           }
@@ -651,6 +672,15 @@ indexer_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
   // ------------------------------------------------------------------ teardown
   tc_fence_before();
   __syncthreads();
+  if constexpr (MODE == kModeDecode) {
+    if (p.hist && hist_b >= 0 && !*abort_flag) {      // the last item's counts (hist_b is set in epilogue threads)
+      const unsigned* hs = reinterpret_cast<const unsigned*>(smem + C::OFF_HIST);
+      for (int i = threadIdx.x - 32 * C::EPI_WARP0; i < 2048; i += 32 * C::NUM_EPI_WARPS) {
+        const unsigned v = hs[i];
+        if (v) atomicAdd(p.hist + static_cast<long long>(hist_b) * 2048 + i, v);
+      }
+    }
+  }
   if constexpr (kChecks) {
     // every key tile loaded went through the MMAs, and every accumulator stage committed was read by the
     // ACC_READERS epilogue warps that take it (a wait that ran out has already recorded DSA_ERR_TIMEOUT)

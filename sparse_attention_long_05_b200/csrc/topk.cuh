@@ -32,6 +32,8 @@ struct TopkParams {
   int* idx;                     // [rows, k]
   long long idx_ld;
   float* sel_scores;            // [rows, k] score of each selected column (-inf for padding), or null
+  const unsigned* hist;         // [rows, 2048] each row's counts of the top 11 order-key bits, or null (the
+                                // cluster kernel then reads them instead of counting; the rows kernel ignores it)
 };
 
 // Inverse of order_key on the keys it produces (+0.0 for a folded -0.0; NaN stays NaN)

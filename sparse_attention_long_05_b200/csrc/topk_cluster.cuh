@@ -163,49 +163,55 @@ __global__ void __cluster_dims__(kTkcCluster, 1, 1) __launch_bounds__(kTkcThread
   const int w0 = min(c1, c0 + warp * wseg), w1 = min(c1, w0 + wseg);
 
   // ---------------------------------------------------------------- 1. histograms, the cluster's bin b*
-  for (int i = tid; i < kTopkBins; i += kTkcThreads) sm.bins[i] = 0;
   if (tid == 0) sm.s_bin = 0xFFFFFFFFu;
-  __syncthreads();
-  if (vec) {
-    for (int i0 = c0 + 4 * tid; i0 < c1; i0 += 16 * kTkcThreads) {
-      float4 v[4];
+  if (p.hist) {
+    // the row's histogram came with the scores (the decode indexer counts them as it writes them)
+    const unsigned* h = p.hist + static_cast<long long>(r) * kTopkBins;
+    for (int i = tid; i < kTopkBins; i += kTkcThreads) sm.merged[i] = h[i];
+  } else {
+    for (int i = tid; i < kTopkBins; i += kTkcThreads) sm.bins[i] = 0;
+    __syncthreads();
+    if (vec) {
+      for (int i0 = c0 + 4 * tid; i0 < c1; i0 += 16 * kTkcThreads) {
+        float4 v[4];
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const int i = i0 + 4 * u * kTkcThreads;
-        if (i + 3 < c1) {
-          v[u] = *reinterpret_cast<const float4*>(x + i);
-        } else {
-          v[u].x = (i < c1) ? x[i] : NAN;
-          v[u].y = (i + 1 < c1) ? x[i + 1] : NAN;
-          v[u].z = (i + 2 < c1) ? x[i + 2] : NAN;
-          v[u].w = NAN;
+        for (int u = 0; u < 4; ++u) {
+          const int i = i0 + 4 * u * kTkcThreads;
+          if (i + 3 < c1) {
+            v[u] = *reinterpret_cast<const float4*>(x + i);
+          } else {
+            v[u].x = (i < c1) ? x[i] : NAN;
+            v[u].y = (i + 1 < c1) ? x[i + 1] : NAN;
+            v[u].z = (i + 2 < c1) ? x[i + 2] : NAN;
+            v[u].w = NAN;
+          }
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int i = i0 + 4 * u * kTkcThreads;
+          if (i < c1) atomicAdd(&sm.bins[order_key(v[u].x) >> 21], 1u);
+          if (i + 1 < c1) atomicAdd(&sm.bins[order_key(v[u].y) >> 21], 1u);
+          if (i + 2 < c1) atomicAdd(&sm.bins[order_key(v[u].z) >> 21], 1u);
+          if (i + 3 < c1) atomicAdd(&sm.bins[order_key(v[u].w) >> 21], 1u);
         }
       }
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const int i = i0 + 4 * u * kTkcThreads;
-        if (i < c1) atomicAdd(&sm.bins[order_key(v[u].x) >> 21], 1u);
-        if (i + 1 < c1) atomicAdd(&sm.bins[order_key(v[u].y) >> 21], 1u);
-        if (i + 2 < c1) atomicAdd(&sm.bins[order_key(v[u].z) >> 21], 1u);
-        if (i + 3 < c1) atomicAdd(&sm.bins[order_key(v[u].w) >> 21], 1u);
-      }
+    } else {
+      for (int i = c0 + tid; i < c1; i += kTkcThreads) atomicAdd(&sm.bins[order_key(x[i]) >> 21], 1u);
     }
-  } else {
-    for (int i = c0 + tid; i < c1; i += kTkcThreads) atomicAdd(&sm.bins[order_key(x[i]) >> 21], 1u);
-  }
-  cluster_sync();                                // every CTA's histogram is complete
-  {
-    // the eight bins of this thread from every CTA: 64 loads issued before any is summed
-    constexpr int BPT = kTopkBins / kTkcThreads;
-    uint32_t v[BPT][kTkcCluster];
+    cluster_sync();                                // every CTA's histogram is complete
+    {
+      // the eight bins of this thread from every CTA: 64 loads issued before any is summed
+      constexpr int BPT = kTopkBins / kTkcThreads;
+      uint32_t v[BPT][kTkcCluster];
 #pragma unroll
-    for (int j = 0; j < BPT; ++j) cluster_load8(&sm.bins[tid + j * kTkcThreads], v[j]);
+      for (int j = 0; j < BPT; ++j) cluster_load8(&sm.bins[tid + j * kTkcThreads], v[j]);
 #pragma unroll
-    for (int j = 0; j < BPT; ++j) {
-      uint32_t s = 0;
+      for (int j = 0; j < BPT; ++j) {
+        uint32_t s = 0;
 #pragma unroll
-      for (int q = 0; q < kTkcCluster; ++q) s += v[j][q];
-      sm.merged[tid + j * kTkcThreads] = s;
+        for (int q = 0; q < kTkcCluster; ++q) s += v[j][q];
+        sm.merged[tid + j * kTkcThreads] = s;
+      }
     }
   }
   __syncthreads();

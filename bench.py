@@ -651,6 +651,9 @@ def parse_args(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--kernels-small", action="store_true",
                     help="run one launch of each main kernel on small inputs (profiling) and exit")
+    ap.add_argument("--decode-only", action="store_true",
+                    help="run only the decode workload (--warmup, then --decode-steps timed steps), print its "
+                         "measurement and exit (profiling)")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("at least 3 warm-up steps")
@@ -692,6 +695,11 @@ def run_dsa(args, ws_n, rank):
         kernels_small(dsa)
         return
     pk = peaks()
+    if args.decode_only:
+        dec = bench_decode(dsa, DECODE, args.decode_steps, args.warmup, ws_n, rank, pk)
+        if rank == 0:
+            print(json.dumps({"decode": dec}), flush=True)
+        return
     if args.prefill_shard and ws_n > 1:
         sh = bench_prefill_sharded(dsa, PREFILL, args.steps, args.warmup, ws_n, rank)
         if rank == 0:

@@ -1118,10 +1118,10 @@ dsa_status_t dsa_checks_selftest(int which, void* scratch, void* stream) {
     static const int32_t n = 10;
     int32_t* idx = reinterpret_cast<int32_t*>(b);
     int32_t* len = reinterpret_cast<int32_t*>(b + 256);
+    // (copies from pageable memory: the source is read before cudaMemcpyAsync returns)
     if (cudaMemcpyAsync(idx, row, sizeof(row), cudaMemcpyHostToDevice, st) != cudaSuccess ||
         cudaMemcpyAsync(len, &n, sizeof(n), cudaMemcpyHostToDevice, st) != cudaSuccess)
       return DSA_ERR_CUDA;
-    if (cudaStreamSynchronize(st) != cudaSuccess) return DSA_ERR_CUDA;   // the host arrays are read now
     TopkParams p{nullptr, 10, nullptr, len, 0, 1, 4, idx, 4, nullptr};
     topk_check_kernel<<<1, 256, 0, st>>>(p);
     return last_launch_status();
@@ -1135,12 +1135,16 @@ dsa_status_t dsa_checks_selftest(int which, void* scratch, void* stream) {
   int32_t* nk = idx + k;                                                   // [1]
   uint16_t* out = reinterpret_cast<uint16_t*>(b + S * 1152 + 32768);       // [1, H, 512] bf16
   float* lse = reinterpret_cast<float*>(b + S * 1152 + 49152);             // [1, H]
-  static int32_t host[k + 1];
-  for (int j = 0; j < k; ++j) host[j] = j;
-  host[0] = 250;
-  host[k] = 200;
-  if (cudaMemcpyAsync(idx, host, sizeof(host), cudaMemcpyHostToDevice, st) != cudaSuccess) return DSA_ERR_CUDA;
-  if (cudaStreamSynchronize(st) != cudaSuccess) return DSA_ERR_CUDA;
+  struct Planted {
+    int32_t v[k + 1];
+    Planted() {
+      for (int j = 0; j < k; ++j) v[j] = j;
+      v[0] = 250;   // idx row [250, 1, 2, ..., 127]
+      v[k] = 200;   // n_keys
+    }
+  };
+  static const Planted host;
+  if (cudaMemcpyAsync(idx, host.v, sizeof(host.v), cudaMemcpyHostToDevice, st) != cudaSuccess) return DSA_ERR_CUDA;
   return run_mla(q, c, S, idx, nullptr, 1, H, k, 0.0416666679f, out, lse, st, kMlaCounts, nk);
 #endif
 }

@@ -462,9 +462,9 @@ indexer_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     constexpr int P = kPacked ? 1 : ((H_I >= 16) ? 4 : 1);   // partial sums per row (ILP)
     // Fragment reads (kPacked): the accumulator is read in 16-lane x 256-bit fragments, so that a thread holds
     // four keys (lanes g, g + 8, g + 16, g + 24 of its warp's 32, g = lane / 4) and, of every eight columns, the
-    // two columns 2c, 2c + 1 (c = lane % 4).  One 8-byte load of a head-weight pair then serves four keys, where
-    // per-key reads (one key per thread) broadcast every weight to the whole warp, and a warp-uniform 16-byte
-    // shared load takes four wavefronts.  Each thread sums its sixteen heads of a token, and two shuffle rounds
+    // two columns 2c, 2c + 1 (c = lane % 4).  Each head weight a thread loads then serves four keys (the sixteen
+    // weights of its heads lie together: four 16-byte loads per token), where per-key reads (one key per thread)
+    // broadcast every weight to the whole warp.  Each thread sums its sixteen heads of a token, and two shuffle rounds
     // (lane ^ 1, lane ^ 2) add the four partial sums of a key, leaving thread (g, c) with key
     // g + 8 (c >> 1) + 16 (c & 1).
     const int e = warp - C::EPI_WARP0;

@@ -76,7 +76,8 @@ def test_clock_summary_reasons_and_median():
 
 
 @pytest.mark.parametrize("argv", [["--gpus", "1", "--steps", "20", "--warmup", "5"], [],
-                                  ["--steps", "3", "--warmup", "40", "--decode-steps", "300"]])
+                                  ["--steps", "3", "--warmup", "40", "--decode-steps", "300"],
+                                  ["--decode-only", "--decode-steps", "3"]])
 def test_decode_caches_hold_every_step_the_run_appends(argv):
     # The run appends one entry per sequence at every warm-up and timed step; the caches bench.py allocates must
     # hold all of them, whatever the warm-up count, and the timed part is the 256 steps of the decode workload

@@ -73,6 +73,13 @@ def test_full_batch_sampled_sequences(dsa):
     _run_steps(dsa, cfg, 43, 2, [0, 7, 21, 63], exact=False)
 
 
+def test_batch_larger_than_the_sm_count_integer_mode_exact(dsa):
+    # 160 sequences (more than the 148 SMs): the top-k takes one CTA per row (no histogram from the indexer) and
+    # each attention cluster serves several tokens; contexts of 100..5000 keys, so some rows select every key
+    cfg = G.DecodeConfig("many_int", B=160, len_lo=100, len_hi=5000, steps=2, mode="int")
+    _run_steps(dsa, cfg, 49, 2, [0, 1, 57, 111, 148, 159], exact=True)
+
+
 def test_long_rows_integer_mode_exact(dsa):
     # Score rows of 16K-40K keys take the top-k's sampled path; integer mode has many tied scores, which it
     # must still break exactly as the oracle does.  The rows' cache offsets are not multiples of 4.

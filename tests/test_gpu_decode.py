@@ -80,6 +80,15 @@ def test_batch_larger_than_the_sm_count_integer_mode_exact(dsa):
     _run_steps(dsa, cfg, 49, 2, [0, 1, 57, 111, 148, 159], exact=True)
 
 
+def test_contexts_around_k_integer_mode_exact(dsa):
+    # contexts n_b of 2044..2050 keys before the step (k = 2048): over three appended steps the tokens cross from the
+    # dense path (n_b + 1 <= k: every key selected, read as contiguous tiles) to the selected path, one key at a time
+    cfg = G.DecodeConfig("around_k", B=12, len_lo=2044, len_hi=2050, steps=3, mode="int")
+    lens = G.decode_lengths(cfg, 50)
+    assert min(lens) + 1 <= cfg.k < max(lens) + 3
+    _run_steps(dsa, cfg, 50, 3, range(12), exact=True)
+
+
 def test_long_rows_integer_mode_exact(dsa):
     # Score rows of 16K-40K keys take the top-k's sampled path; integer mode has many tied scores, which it
     # must still break exactly as the oracle does.  The rows' cache offsets are not multiples of 4.

@@ -183,6 +183,31 @@ def test_varlen_many_sequences_one_select(dsa):
         assert torch.equal(lse[r0:r1], l1), f"sequence {b}: lse"
 
 
+def test_varlen_sequences_around_k(dsa):
+    # sequences of k - 1, k, k + 1 and 1 tokens (and k + 129, one key tile more): the first take no indexer launch at
+    # all, the longer ones score only their rows t >= k; every row matches its sequence's own prefill bit for bit
+    base = G.PREFILL_CONFIGS["prefill_8k"]
+    k = base.k
+    lens = [k - 1, k, k + 1, 1, k + 129]
+    seeds = [70 + b for b in range(len(lens))]
+    cfgs = [dataclasses.replace(base, name=f"varlen_{n}", L=n) for n in lens]
+    parts = [prefill_device(cfg, sd) for cfg, sd in zip(cfgs, seeds)]
+    cat = {key: torch.cat([x[key] for x in parts]) for key in ("q_idx", "k_idx", "w", "q", "c")}
+    cu = np.concatenate([[0], np.cumsum(lens)]).tolist()
+    idx, out, lse = dsa.dsa_forward_prefill_varlen(cu, cat["q_idx"], None, cat["k_idx"], None, cat["w"], cat["q"],
+                                                   cat["c"], k, base.scale)
+    assert dsa.dsa_get_device_status() == 0
+    for b, (cfg, sd) in enumerate(zip(cfgs, seeds)):
+        i1, o1, l1 = _forward_full(dsa, cfg, sd)
+        r0, r1 = cu[b], cu[b + 1]
+        assert torch.equal(idx[r0:r1], i1), f"sequence {b}: selection"
+        assert torch.equal(out[r0:r1], o1), f"sequence {b}: output"
+        assert torch.equal(lse[r0:r1], l1), f"sequence {b}: lse"
+    cfg, sd = cfgs[4], seeds[4]
+    _check_rows(cfg, sd, sample_rows(cfg.L, k, 8, sd), idx[cu[4]:cu[5]].cpu().numpy(), out[cu[4]:cu[5]],
+                exact_idx=True)
+
+
 @pytest.mark.parametrize("name,L", [("prefill_8k", 8192), ("prefill_32k", 5000), ("tiny_1k", 1024)])
 def test_host_buffer_prefill_identical(dsa, name, L):
     # dsa_forward_prefill_host: inputs in page-locked host memory, results copied back by the call, the transfers

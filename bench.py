@@ -467,6 +467,157 @@ def bench_varlen(dsa, cfg, nseq, steps, warmup, ws_n, rank, pk):
                     "bf16 flops, over the whole call"}
 
 
+def timed_steps(step, steps, warmup, ws_n):
+    """Run `warmup` untimed and `steps` timed calls of step(), CUDA events around the timed ones (barriers and
+    max over ranks as for the headline); returns ms per step."""
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize()
+    barrier(ws_n)
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record()
+    for _ in range(steps):
+        step()
+    t1.record()
+    torch.cuda.synchronize()
+    barrier(ws_n)
+    return max_over_ranks(t0.elapsed_time(t1), ws_n) / steps
+
+
+def bench_kl(dsa, cfg, steps, warmup, ws_n, rank, pk):
+    """The prefill with the indexer objective (dsa_forward_prefill_kl: selection, attention and the per-row
+    KL(p_t || Softmax(I_t))) against the plain forward on the same inputs; the difference is the objective's pass."""
+    dev = "cuda"
+    x = G.prefill_keys(cfg, replica_seed(4000, rank), device=dev)
+    x.update(G.prefill_queries(cfg, replica_seed(4000, rank), None, device=dev))
+    args = (x["q_idx"], x["q_scale"], x["k_idx"], x["k_scale"], x["w"], x["q"], x["c"], cfg.k, cfg.scale)
+    L = cfg.L
+    idx = torch.empty((L, cfg.k), dtype=torch.int32, device=dev)
+    out = torch.empty((L, cfg.H, cfg.D_v), dtype=torch.bfloat16, device=dev)
+    lse = torch.empty((L, cfg.H), dtype=torch.float32, device=dev)
+    kl = torch.empty((L,), dtype=torch.float32, device=dev)
+    ws_kl = torch.empty((dsa.dsa_prefill_kl_workspace_size(L, cfg.H_I, cfg.d_I, cfg.H, cfg.k),), dtype=torch.uint8,
+                        device=dev)
+    ms_kl = timed_steps(lambda: dsa.dsa_forward_prefill_kl(*args, idx_out=idx, out=out, lse=lse, kl=kl, ws=ws_kl),
+                        steps, warmup, ws_n)
+    del ws_kl
+    ws = torch.empty((dsa.dsa_prefill_workspace_size(L, cfg.H_I, cfg.d_I, cfg.H, cfg.k),), dtype=torch.uint8,
+                     device=dev)
+    ms_fw = timed_steps(lambda: dsa.dsa_forward_prefill(*args, idx_out=idx, out=out, lse=lse, ws=ws),
+                        steps, warmup, ws_n)
+    assert dsa.dsa_get_device_status() == 0
+    sel = sum(min(t + 1, cfg.k) for t in range(L))
+    obj_ms = max(ms_kl - ms_fw, 1e-9)
+    flops = 2.0 * cfg.H * cfg.D * sel            # the objective recomputes the selected keys' logits
+    del x, ws
+    return {"metric": f"DSA forward + indexer KL objective tokens/s ({cfg.name}, {L} tokens)",
+            "value": job_rate(L, ws_n, ms_kl), "unit": "tokens/s", "ms_per_step": ms_kl, "forward_ms": ms_fw,
+            "objective_ms": obj_ms, "steps": steps, "warmup": warmup,
+            "roofline": {"kernel": "indexer objective pass (logits of the selected keys again)", "bound": "tensor",
+                         "achieved": flops / (obj_ms * 1e-3) / 1e12, "peak": pk["bf16_sustained"],
+                         "unit": "TFLOP/s", "frac": flops / (obj_ms * 1e-3) / 1e12 / pk["bf16_sustained"],
+                         "note": "its time is the KL call's minus the plain forward's"}}
+
+
+def bench_short_prefill(dsa, cfg, steps, warmup, ws_n, rank, pk):
+    """A prefill no longer than k: every row t attends to all of 0..t (no indexer launch; the attention reads the
+    keys as contiguous tiles)."""
+    dev = "cuda"
+    L = cfg.L
+    x = G.prefill_keys(cfg, replica_seed(5000, rank), device=dev)
+    x.update(G.prefill_queries(cfg, replica_seed(5000, rank), None, device=dev))
+    idx = torch.empty((L, cfg.k), dtype=torch.int32, device=dev)
+    out = torch.empty((L, cfg.H, cfg.D_v), dtype=torch.bfloat16, device=dev)
+    lse = torch.empty((L, cfg.H), dtype=torch.float32, device=dev)
+    ws = torch.empty((max(1, dsa.dsa_prefill_workspace_size(L, cfg.H_I, cfg.d_I, cfg.H, cfg.k)),), dtype=torch.uint8,
+                     device=dev)
+    n0 = dsa.dsa_launch_count()
+    ms = timed_steps(lambda: dsa.dsa_forward_prefill(x["q_idx"], x["q_scale"], x["k_idx"], x["k_scale"], x["w"],
+                                                     x["q"], x["c"], cfg.k, cfg.scale, idx_out=idx, out=out, lse=lse,
+                                                     ws=ws), steps, warmup, ws_n)
+    launches = (dsa.dsa_launch_count() - n0) / (steps + warmup)
+    assert dsa.dsa_get_device_status() == 0
+    flops = prefill_work(cfg)["attention_flops"]
+    del x, ws
+    return {"metric": f"DSA prefill tokens/s, L = {L} <= k (masked-MHA mode: every row attends to 0..t)",
+            "value": job_rate(L, ws_n, ms), "unit": "tokens/s", "ms_per_step": ms, "steps": steps, "warmup": warmup,
+            "launches_per_step": launches,
+            "roofline": {"kernel": "sparse_mla_attn (dense tiles)", "bound": "tensor",
+                         "achieved": flops / (ms * 1e-3) / 1e12, "peak": pk["bf16_sustained"], "unit": "TFLOP/s",
+                         "frac": flops / (ms * 1e-3) / 1e12 / pk["bf16_sustained"],
+                         "note": "whole call (the top-k writes the implied selection, then the attention)"}}
+
+
+def paged_layout(cache, lens, offs, nsteps, page_rows, seed):
+    """The flat decode caches' sequences moved into shuffled pages of page pools: (page table [B, max_pages],
+    k_I pool, scale pool, latent pool).  One gather per pool."""
+    B = len(lens)
+    need = [-(-(n + nsteps) // page_rows) for n in lens]
+    max_pages = max(need)
+    num_pages = sum(need)
+    perm = np.random.default_rng(seed).permutation(num_pages)
+    table = np.full((B, max_pages), -1, dtype=np.int32)
+    src = np.zeros(num_pages * page_rows, dtype=np.int64)
+    at = 0
+    for b in range(B):
+        cap = lens[b] + nsteps
+        for j in range(need[b]):
+            pg = int(perm[at])
+            at += 1
+            table[b, j] = pg
+            rows = np.arange(j * page_rows, (j + 1) * page_rows)
+            src[pg * page_rows:(pg + 1) * page_rows] = offs[b] + np.minimum(rows, cap - 1)
+    src_t = torch.from_numpy(src).cuda()
+    kc = cache["k_cache"].view(torch.uint8)[src_t].view(torch.float8_e4m3fn)
+    ks = cache["k_scale_cache"][src_t]
+    cc = cache["c_cache"][src_t]
+    return torch.from_numpy(table).cuda(), kc, ks, cc
+
+
+def bench_decode_paged(dsa, cfg, steps, warmup, ws_n, rank, pk, page_rows=256):
+    """The decode workload over paged caches (pools of page_rows-row pages in shuffled order, a page table per
+    sequence): the same sequences, inputs and algorithmic bytes as the flat-cache decode line."""
+    dev = "cuda"
+    seed = replica_seed(2000, rank)
+    cfg, nsteps = decode_plan(cfg, warmup, steps)
+    cache = G.decode_fill_cache(cfg, seed, device=dev)
+    lens, offs = cache["lens"], cache["offs"]
+    table, kc, ks, cc = paged_layout(cache, lens, offs, nsteps, page_rows, seed)
+    del cache
+    torch.cuda.empty_cache()
+    ctx = torch.tensor(lens, dtype=torch.int32, device=dev)
+    blocks = [G.decode_step_batch(cfg, seed, min(32, nsteps - s0), device=dev, step0=s0)
+              for s0 in range(0, nsteps, 32)]
+    inp = {key: torch.cat([b[key] for b in blocks]) if blocks[0][key] is not None else None for key in blocks[0]}
+    B, k = cfg.B, cfg.k
+    idx = torch.empty((B, k), dtype=torch.int32, device=dev)
+    out = torch.empty((B, cfg.H, cfg.D_v), dtype=torch.bfloat16, device=dev)
+    lse = torch.empty((B, cfg.H), dtype=torch.float32, device=dev)
+    ws = torch.empty((dsa.dsa_decode_paged_workspace_size(B, table.shape[1], page_rows, cfg.H_I, cfg.d_I, cfg.H, k),),
+                     dtype=torch.uint8, device=dev)
+    it = [0]
+
+    def step():
+        s = it[0]
+        g = lambda key: None if inp[key] is None else inp[key][s]   # noqa: E731
+        dsa.dsa_forward_decode_paged(table, page_rows, ctx, g("q_idx"), g("q_scale"), g("w"), g("q"), g("k_new"),
+                                     g("k_scale_new"), g("c_new"), kc, ks, cc, k, cfg.scale, idx_out=idx, out=out,
+                                     lse=lse, ws=ws)
+        ctx.add_(1)
+        it[0] += 1
+
+    ms = timed_steps(step, steps, warmup, ws_n)
+    assert dsa.dsa_get_device_status() == 0
+    byts = decode_bytes(cfg, lens, nsteps) - decode_bytes(cfg, lens, warmup)
+    gbs = byts / steps / (ms * 1e-3) / 1e9
+    del kc, ks, cc, inp
+    return {"metric": f"DSA decode tokens/s over paged caches ({page_rows}-row pages, shuffled; the decode line's "
+                      "workload)", "value": job_rate(B, ws_n, ms), "unit": "tokens/s", "ms_per_step": ms,
+            "steps": steps, "warmup": warmup,
+            "roofline": {"kernel": "decode step (append, indexer, top-k, sparse MLA)", "bound": "hbm",
+                         "achieved": gbs, "peak": pk["hbm_gbs"], "unit": "GB/s", "frac": gbs / pk["hbm_gbs"]}}
+
+
 def decode_plan(cfg, warmup, steps):
     """The decode workload of a run of `warmup` untimed and `steps` timed steps: the same sequences (lengths and
     cache contents depend only on the seed), with caches that hold every entry the run appends.  Returns the
@@ -649,6 +800,8 @@ def parse_args(argv=None):
                     help="with N > 1: one 128K sequence row-sharded over the N ranks (an all-gather of the key-side "
                          "tensors per step, strong scaling) instead of one independent sequence per rank")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-next-rows", action="store_true",
+                    help="skip the lines of the next rows (indexer objective, short prefill, paged decode)")
     ap.add_argument("--kernels-small", action="store_true",
                     help="run one launch of each main kernel on small inputs (profiling) and exit")
     ap.add_argument("--decode-only", action="store_true",
@@ -728,6 +881,23 @@ def run_dsa(args, ws_n, rank):
             cfg = G.PREFILL_CONFIGS[name]
             side[name] = side_line(bench_prefill(dsa, cfg, args.steps, args.warmup, ws_n, rank, pk), cfg)
             torch.cuda.empty_cache()
+    rows_next = None
+    if not args.no_next_rows:
+        # the next rows built beyond the hot path, each measured: the indexer objective, masked-MHA short prefill,
+        # paged decode (varlen prefill is the "varlen" line)
+        import dataclasses
+        rows_next = {
+            "kl": bench_kl(dsa, G.PREFILL_CONFIGS["prefill_32k"], max(3, args.steps // 2), args.warmup, ws_n, rank,
+                           pk),
+            "short_prefill": bench_short_prefill(dsa, dataclasses.replace(G.PREFILL_CONFIGS["prefill_8k"],
+                                                                          name="prefill_2k", L=2048),
+                                                 args.steps, args.warmup, ws_n, rank, pk),
+        }
+        torch.cuda.empty_cache()
+        if not args.no_decode:
+            rows_next["paged_decode"] = bench_decode_paged(dsa, DECODE, args.decode_steps, args.warmup, ws_n, rank,
+                                                           pk)
+            torch.cuda.empty_cache()
     e2e = None
     if not args.no_e2e:
         e2e = bench_prefill_e2e(dsa, PREFILL, args.e2e_steps, rank)
@@ -751,7 +921,7 @@ def run_dsa(args, ws_n, rank):
                    "l2": "inputs larger than L2 (q alone is 19 GB), no flush"},
         "roofline": pre["roofline"], "kernels": pre["kernels"], "clocks": pre["clocks"],
         "e2e": e2e, "gpu_launches": pre["launches"], "cpu_baseline": cpu, "decode": dec, "varlen": var,
-        "configs": side,
+        "configs": side, "next_rows": rows_next,
     }
     print(json.dumps(line), flush=True)
 

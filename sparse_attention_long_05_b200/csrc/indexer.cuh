@@ -134,6 +134,8 @@ struct IndexerCfg {
   static constexpr uint32_t SW_LAYOUT = (D_I == 128) ? kLayoutSW128 : kLayoutSW64;
   static constexpr uint32_t SBO = (D_I == 128) ? 1024 : 512;
   static_assert(N <= 256 && N % 16 == 0, "MMA N");
+  // the SM's 228 KB of shared memory, less 1 KB reserved per CTA, holds CTAS_PER_SM of them
+  static_assert(CTAS_PER_SM * (SMEM + 1024) <= 228 * 1024, "CTAs per SM");
   static_assert(OFF_W % 16 == 0 && (W_FLOATS * 4) % 16 == 0, "head weights are read as 16-byte quads");
   static_assert(D_I == 128 || D_I == 64, "d_I");
   static_assert((N / EPI_WG) % H_I == 0 || H_I > N / EPI_WG, "epilogue column split");
@@ -383,11 +385,20 @@ indexer_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
           q_par[qb] = qph;
           for (int tile = it.tile0; tile < it.tile1; ++tile) {
             if (!tile_active(it, tile)) continue;
+            // the tile's row (a page-table load with paged caches) is looked up before the wait, so that the
+            // load's latency overlaps it instead of delaying the copy
+            const long long krow = key_row(it, tile, 0);
             if (!mbar_wait(bar(Bars::K_EMPTY + kp.stage), kp.phase ^ 1, abort_flag)) { ok = false; break; }
             mbar_arrive_expect_tx(bar(Bars::K_FULL + kp.stage), C::KBYTES);
-            check_that(key_row(it, tile, 0) >= 0 && key_row(it, tile, 0) < p.k_rows);
-            tma_load_2d(k_s + kp.stage * C::KBYTES, &tm_k, bar(Bars::K_FULL + kp.stage), 0,
-                        static_cast<int>(key_row(it, tile, 0)));
+            check_that(krow >= 0 && krow < p.k_rows);
+            if constexpr (MODE == kModeDecode) {
+              // the key cache streams through once per step: its lines go first, so that the score rows the
+              // top-k reads next stay in L2
+              tma_load_2d_hint(k_s + kp.stage * C::KBYTES, &tm_k, bar(Bars::K_FULL + kp.stage), 0,
+                               static_cast<int>(krow), l2_policy_evict_first());
+            } else {
+              tma_load_2d(k_s + kp.stage * C::KBYTES, &tm_k, bar(Bars::K_FULL + kp.stage), 0, static_cast<int>(krow));
+            }
             kp.advance();
             ++k_issued;
           }
@@ -508,19 +519,26 @@ indexer_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         }
       }
       named_bar_sync(1, ethreads);
-      // key scales are loaded one tile ahead: a load issued at the start of its own tile would expose the
-      // global-memory latency once per tile (the epilogue needs it a few hundred cycles later)
+      // key scales are loaded ahead of their tile: a load issued at the start of its own tile would expose the
+      // global-memory latency once per tile (the epilogue needs it a few hundred cycles later).  One tile ahead
+      // in prefill; two in decode, whose tiles take about half a microsecond and whose paged caches put a
+      // page-table load before the scale's.
+      constexpr int KS_AHEAD = (MODE == kModeDecode) ? 2 : 1;
       auto kscale_of = [&](int tile) -> float {
         const int s = tile * 128 + quad * 32 + key_lane;
         return (p.k_scale && tile < it.tile1 && s < it.n_keys) ? p.k_scale[key_row(it, tile, quad * 32 + key_lane)]
                                                                 : 1.f;
       };
-      float kscale_next = kscale_of(it.tile0);
+      float kscale_ahead[KS_AHEAD];
+#pragma unroll
+      for (int a = 0; a < KS_AHEAD; ++a) kscale_ahead[a] = kscale_of(it.tile0 + a);
       for (int tile = it.tile0; tile < it.tile1; ++tile) {
         const int s = tile * 128 + quad * 32 + key_lane;      // key of this thread
         const bool key_ok = s < it.n_keys;
-        const float kscale = kscale_next;
-        kscale_next = kscale_of(tile + 1);
+        const float kscale = kscale_ahead[0];
+#pragma unroll
+        for (int a = 0; a + 1 < KS_AHEAD; ++a) kscale_ahead[a] = kscale_ahead[a + 1];
+        kscale_ahead[KS_AHEAD - 1] = kscale_of(tile + KS_AHEAD);
         for (int g = 0; g < NG; ++g) {
           if (g * NT >= it.n_tok) break;
           if (!group_active<NT>(it, tile, g)) {

@@ -197,6 +197,32 @@ __device__ __forceinline__ long long mla_row(const MlaParams& p, int t, int e, l
   return valid ? mla_pos_row<PAGED>(p, t, base, e) : (slot < p.S ? slot : 0);
 }
 
+// mla_row of four consecutive entries over a page table: the four page-table loads are issued before any of
+// them is used (checked one entry at a time, each load would wait behind the previous entry's check and possible
+// status write, and a tile would pay four global-memory latencies in sequence).
+__device__ __forceinline__ void mla_rows_paged(const MlaParams& p, int t, int4 e4, long long base, int slot,
+                                               int (&r)[4]) {
+  const int e[4] = {e4.x, e4.y, e4.z, e4.w};
+  const int* pr = p.page_table + static_cast<long long>(t) * p.pt_stride;
+  const long long lim = static_cast<long long>(p.pt_stride) * p.page_rows;
+  int pg[4];
+#pragma unroll
+  for (int u = 0; u < 4; ++u) pg[u] = (e[u] >= 0 && e[u] < lim) ? __ldg(pr + e[u] / p.page_rows) : -1;
+#pragma unroll
+  for (int u = 0; u < 4; ++u) {
+    const long long row = static_cast<long long>(pg[u]) * p.page_rows + e[u] % p.page_rows;
+    const bool valid = pg[u] >= 0 && row < p.S;
+    if (!valid && e[u] != -1) raise_status(DSA_ERR_BAD_INDEX);
+    if constexpr (kChecks) {
+      if (valid && p.dense != kMlaSparse) {
+        const long long n = (p.dense == kMlaCausal) ? static_cast<long long>(p.pos0) + t - base + 1 : p.n_keys[t];
+        check_that(e[u] < n, DSA_ERR_BAD_INDEX);
+      }
+    }
+    r[u] = static_cast<int>(valid ? row : (slot + u < p.S ? slot + u : 0));
+  }
+}
+
 // Number of keys n_t of token t when it takes the dense path (n_t <= k), -1 when its index row is gathered.
 template <bool DENSE>
 __device__ __forceinline__ int mla_dense_keys(const MlaParams& p, int t, long long base) {
@@ -411,10 +437,14 @@ sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
           if (nd < 0) {
             // slots past the token's k entries (a k that is not a multiple of the tile) are padding
             const int4 e = (slot < p.k) ? *reinterpret_cast<const int4*>(ids + slot) : make_int4(-1, -1, -1, -1);
-            r[0] = static_cast<int>(mla_row<PAGED>(p, t, e.x, base, slot));
-            r[1] = static_cast<int>(mla_row<PAGED>(p, t, e.y, base, slot + 1));
-            r[2] = static_cast<int>(mla_row<PAGED>(p, t, e.z, base, slot + 2));
-            r[3] = static_cast<int>(mla_row<PAGED>(p, t, e.w, base, slot + 3));
+            if constexpr (PAGED) {
+              mla_rows_paged(p, t, e, base, slot, r);
+            } else {
+              r[0] = static_cast<int>(mla_row<PAGED>(p, t, e.x, base, slot));
+              r[1] = static_cast<int>(mla_row<PAGED>(p, t, e.y, base, slot + 1));
+              r[2] = static_cast<int>(mla_row<PAGED>(p, t, e.z, base, slot + 2));
+              r[3] = static_cast<int>(mla_row<PAGED>(p, t, e.w, base, slot + 3));
+            }
           } else {
 #pragma unroll
             for (int u = 0; u < 4; ++u) {

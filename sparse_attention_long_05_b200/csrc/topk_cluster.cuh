@@ -163,11 +163,23 @@ __global__ void __cluster_dims__(kTkcCluster, 1, 1) __launch_bounds__(kTkcThread
   const int w0 = min(c1, c0 + warp * wseg), w1 = min(c1, w0 + wseg);
 
   // ---------------------------------------------------------------- 1. histograms, the cluster's bin b*
+  // thread t scans bins 2047 - 8 t .. 2040 - 8 t (descending): c8[j] holds bin 2047 - 8 t - j
+  constexpr int BPT = kTopkBins / kTkcThreads;
+  static_assert(BPT == 8, "eight bins per thread");
+  uint32_t c8[BPT];
   if (tid == 0) sm.s_bin = 0xFFFFFFFFu;
   if (p.hist) {
-    // the row's histogram came with the scores (the decode indexer counts them as it writes them)
-    const unsigned* h = p.hist + static_cast<long long>(r) * kTopkBins;
-    for (int i = tid; i < kTopkBins; i += kTkcThreads) sm.merged[i] = h[i];
+    // the row's histogram came with the scores (the decode indexer counts them as it writes them): each thread
+    // loads its own eight bins, with two 16-byte loads in flight when the histogram is aligned
+    const unsigned* h = p.hist + static_cast<long long>(r) * kTopkBins + (kTopkBins - BPT * (tid + 1));
+    if ((reinterpret_cast<uintptr_t>(h) & 15) == 0) {
+      const uint4 lo = reinterpret_cast<const uint4*>(h)[0], hi = reinterpret_cast<const uint4*>(h)[1];
+      c8[0] = hi.w; c8[1] = hi.z; c8[2] = hi.y; c8[3] = hi.x;
+      c8[4] = lo.w; c8[5] = lo.z; c8[6] = lo.y; c8[7] = lo.x;
+    } else {
+#pragma unroll
+      for (int j = 0; j < BPT; ++j) c8[j] = h[BPT - 1 - j];
+    }
   } else {
     for (int i = tid; i < kTopkBins; i += kTkcThreads) sm.bins[i] = 0;
     __syncthreads();
@@ -201,7 +213,6 @@ __global__ void __cluster_dims__(kTkcCluster, 1, 1) __launch_bounds__(kTkcThread
     cluster_sync();                                // every CTA's histogram is complete
     {
       // the eight bins of this thread from every CTA: 64 loads issued before any is summed
-      constexpr int BPT = kTopkBins / kTkcThreads;
       uint32_t v[BPT][kTkcCluster];
 #pragma unroll
       for (int j = 0; j < BPT; ++j) cluster_load8(&sm.bins[tid + j * kTkcThreads], v[j]);
@@ -213,14 +224,16 @@ __global__ void __cluster_dims__(kTkcCluster, 1, 1) __launch_bounds__(kTkcThread
         sm.merged[tid + j * kTkcThreads] = s;
       }
     }
-  }
-  __syncthreads();
-  {
-    // bin holding the k-th largest key of the row: thread t owns bins 2047 - 8 t .. 2040 - 8 t (descending)
-    constexpr int BPT = kTopkBins / kTkcThreads;
-    uint32_t c8[BPT], tot = 0;
+    __syncthreads();
 #pragma unroll
-    for (int j = 0; j < BPT; ++j) { c8[j] = sm.merged[kTopkBins - 1 - BPT * tid - j]; tot += c8[j]; }
+    for (int j = 0; j < BPT; ++j) c8[j] = sm.merged[kTopkBins - 1 - BPT * tid - j];
+  }
+  {
+    // bin holding the k-th largest key of the row (the scan's barrier orders tid 0's reset of s_bin before the
+    // write of the thread that finds it)
+    uint32_t tot = 0;
+#pragma unroll
+    for (int j = 0; j < BPT; ++j) tot += c8[j];
     uint32_t incl = tot;
 #pragma unroll
     for (int d = 1; d < 32; d <<= 1) {
@@ -251,7 +264,7 @@ __global__ void __cluster_dims__(kTkcCluster, 1, 1) __launch_bounds__(kTkcThread
   // ---------------------------------------------------------------- 2. candidates of bin >= b*, in column order
   // A key is in bin >= b* exactly when the score is >= the float whose order key is b* << 21, so the pass compares
   // raw scores.  Lane l takes 16 consecutive columns of each 512-column step of its warp's sub-segment (four
-  // 16-byte loads in flight when the row is aligned); one warp scan of the lanes' counts places the candidates.
+  // 16-byte loads when the row is aligned); one warp scan of the lanes' counts places the candidates.
   {
     const uint32_t kb = bstar << 21;
     uint32_t tb = (kb & 0x80000000u) ? (kb & 0x7FFFFFFFu) : ~kb;
@@ -259,8 +272,10 @@ __global__ void __cluster_dims__(kTkcCluster, 1, 1) __launch_bounds__(kTkcThread
     const float thr = __uint_as_float(tb);
     const bool low = bstar == 0;               // bin 0 holds NaN too, which compares false: take every key
     int cnt = 0;
-    for (int i00 = w0; i00 < w1; i00 += 512) {
-      const int c0l = i00 + 16 * lane;
+    // two 512-column steps per round: their eight 16-byte loads per lane are in flight together, then each step's
+    // passing columns become a 16-bit mask (the data registers are free again) and the few candidates re-read
+    // their scores (L1 hits) when they are written
+    auto pass_mask = [&](int c0l) -> uint32_t {
       float xv[16];
 #pragma unroll
       for (int u = 0; u < 4; ++u) {
@@ -273,9 +288,13 @@ __global__ void __cluster_dims__(kTkcCluster, 1, 1) __launch_bounds__(kTkcThread
           for (int e = 0; e < 4; ++e) xv[4 * u + e] = (col + e < w1) ? x[col + e] : -INFINITY;
         }
       }
-      int c = 0;
+      uint32_t m = 0;
 #pragma unroll
-      for (int e = 0; e < 16; ++e) c += (c0l + e < w1 && (low || xv[e] >= thr)) ? 1 : 0;
+      for (int e = 0; e < 16; ++e) m |= (c0l + e < w1 && (low || xv[e] >= thr)) ? (1u << e) : 0u;
+      return m;
+    };
+    auto place = [&](int c0l, uint32_t m) {
+      const int c = __popc(m);
       int incl = c;
 #pragma unroll
       for (int d = 1; d < 32; d <<= 1) {
@@ -283,20 +302,23 @@ __global__ void __cluster_dims__(kTkcCluster, 1, 1) __launch_bounds__(kTkcThread
         if (lane >= d) incl += v;
       }
       const int tot = __shfl_sync(0xffffffffu, incl, 31);
-      if (c) {
-        int pos = cnt + incl - c;
-#pragma unroll
-        for (int e = 0; e < 16; ++e) {
-          if (c0l + e < w1 && (low || xv[e] >= thr)) {
-            if (pos < kTkcRegion) {
-              sm.cand_key[warp][pos] = order_key(xv[e]);
-              sm.cand_idx[warp][pos] = c0l + e;
-            }
-            ++pos;
-          }
+      int pos = cnt + incl - c;
+      while (m) {
+        const int e = __ffs(m) - 1;
+        m &= m - 1;
+        if (pos < kTkcRegion) {
+          sm.cand_key[warp][pos] = order_key(x[c0l + e]);
+          sm.cand_idx[warp][pos] = c0l + e;
         }
+        ++pos;
       }
       cnt += tot;
+    };
+    for (int i00 = w0; i00 < w1; i00 += 1024) {
+      const int ca = i00 + 16 * lane, cb = ca + 512;
+      const uint32_t ma = pass_mask(ca), mb = pass_mask(cb);   // columns past w1 load nothing and never pass
+      place(ca, ma);
+      place(cb, mb);
     }
     if (lane == 0) {
       sm.region_n[warp] = min(cnt, kTkcRegion);

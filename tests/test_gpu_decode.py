@@ -73,11 +73,13 @@ def test_full_batch_sampled_sequences(dsa):
     _run_steps(dsa, cfg, 43, 2, [0, 7, 21, 63], exact=False)
 
 
-def test_batch_larger_than_the_sm_count_integer_mode_exact(dsa):
-    # 160 sequences (more than the 148 SMs): the top-k takes one CTA per row (no histogram from the indexer) and
-    # each attention cluster serves several tokens; contexts of 100..5000 keys, so some rows select every key
-    cfg = G.DecodeConfig("many_int", B=160, len_lo=100, len_hi=5000, steps=2, mode="int")
-    _run_steps(dsa, cfg, 49, 2, [0, 1, 57, 111, 148, 159], exact=True)
+@pytest.mark.parametrize("B", [160, 300])
+def test_batch_larger_than_the_sm_count_integer_mode_exact(dsa, B):
+    # More sequences than the 148 SMs: the top-k takes one CTA per row (no histogram from the indexer) and each
+    # attention cluster serves several tokens (300 sequences: more than two per cluster).  Contexts of 100..5000
+    # keys, so some rows select every key.
+    cfg = G.DecodeConfig("many_int", B=B, len_lo=100, len_hi=5000, steps=2, mode="int")
+    _run_steps(dsa, cfg, 49, 2, [0, 1, 57, 111, 148, 159, B - 1], exact=True)
 
 
 def test_contexts_around_k_integer_mode_exact(dsa):

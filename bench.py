@@ -548,9 +548,10 @@ def bench_short_prefill(dsa, cfg, steps, warmup, ws_n, rank, pk):
                          "note": "whole call (the top-k writes the implied selection, then the attention)"}}
 
 
-def paged_layout(cache, lens, offs, nsteps, page_rows, seed):
+def paged_layout(cache, lens, offs, nsteps, page_rows, seed, device="cuda"):
     """The flat decode caches' sequences moved into shuffled pages of page pools: (page table [B, max_pages],
-    k_I pool, scale pool, latent pool).  One gather per pool."""
+    k_I pool, scale pool, latent pool).  One gather per pool; rows of a sequence's last page past its capacity
+    repeat its last row."""
     B = len(lens)
     need = [-(-(n + nsteps) // page_rows) for n in lens]
     max_pages = max(need)
@@ -567,11 +568,11 @@ def paged_layout(cache, lens, offs, nsteps, page_rows, seed):
             table[b, j] = pg
             rows = np.arange(j * page_rows, (j + 1) * page_rows)
             src[pg * page_rows:(pg + 1) * page_rows] = offs[b] + np.minimum(rows, cap - 1)
-    src_t = torch.from_numpy(src).cuda()
+    src_t = torch.from_numpy(src).to(device)
     kc = cache["k_cache"].view(torch.uint8)[src_t].view(torch.float8_e4m3fn)
     ks = cache["k_scale_cache"][src_t]
     cc = cache["c_cache"][src_t]
-    return torch.from_numpy(table).cuda(), kc, ks, cc
+    return torch.from_numpy(table).to(device), kc, ks, cc
 
 
 def bench_decode_paged(dsa, cfg, steps, warmup, ws_n, rank, pk, page_rows=256):

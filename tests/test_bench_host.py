@@ -117,3 +117,24 @@ def test_argument_checks():
         bench.parse_args(["--warmup", "2"])
     with pytest.raises(SystemExit):
         bench.parse_args(["--decode-steps", "0"])
+
+
+@pytest.mark.parametrize("page_rows", [128, 256])
+def test_paged_layout_maps_every_position_to_its_flat_row(page_rows):
+    # The paged-decode bench line's caches: every position a sequence holds or appends (n_b + steps of them) sits in
+    # the pool row its page-table entry names, each page is used once, and unused table entries are -1.
+    cfg = G.DecodeConfig("paged_small", B=5, len_lo=200, len_hi=1500, steps=7)
+    cache = G.decode_fill_cache(cfg, 3)
+    lens, offs = cache["lens"], cache["offs"]
+    table, kc, ks, cc = bench.paged_layout(cache, lens, offs, cfg.steps, page_rows, 3, device="cpu")
+    used = table[table >= 0].tolist()
+    assert sorted(used) == list(range(len(used))) and kc.shape[0] == len(used) * page_rows
+    for b in range(cfg.B):
+        cap = lens[b] + cfg.steps
+        npg = -(-cap // page_rows)
+        assert (table[b, :npg] >= 0).all() and (table[b, npg:] == -1).all()
+        pos = torch.arange(cap)
+        rows = table[b, pos // page_rows].long() * page_rows + pos % page_rows
+        assert torch.equal(kc[rows].view(torch.uint8), cache["k_cache"][offs[b] + pos].view(torch.uint8))
+        assert torch.equal(ks[rows], cache["k_scale_cache"][offs[b] + pos])
+        assert torch.equal(cc[rows], cache["c_cache"][offs[b] + pos])

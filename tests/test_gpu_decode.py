@@ -213,11 +213,12 @@ def _paged_copy(cache, lens, offs, steps, page_rows, seed, spare=5):
     return torch.from_numpy(table).cuda(), kc.view(torch.float8_e4m3fn), ks, cc
 
 
-@pytest.mark.parametrize("page_rows", [128, 256])
-def test_paged_cache_identical_to_flat(dsa, page_rows):
+@pytest.mark.parametrize("B,len_hi,page_rows", [(6, 20000, 128), (6, 20000, 256), (160, 5000, 512)])
+def test_paged_cache_identical_to_flat(dsa, B, len_hi, page_rows):
     # The same sequences in flat caches and in shuffled pages of page pools (spare pages hold NaN): every step's
-    # selection, output and LSE are bit-identical, and the appended entries land in the right pages.
-    cfg = G.DecodeConfig("paged", B=6, len_lo=100, len_hi=20000, steps=3)
+    # selection, output and LSE are bit-identical, and the appended entries land in the right pages.  160
+    # sequences: more than the SMs (one top-k CTA per row, several tokens per attention cluster).
+    cfg = G.DecodeConfig("paged", B=B, len_lo=100, len_hi=len_hi, steps=3)
     seed = 47
     cache = G.decode_fill_cache(cfg, seed, device="cuda")
     lens, offs = cache["lens"], cache["offs"]

@@ -50,9 +50,10 @@ def _oracle_kl(cfg, seed, rows, idx):
 
 
 @pytest.mark.parametrize("name,L,k,seed", [("tiny_1k", 1024, None, 71), ("prefill_8k", 3000, None, 72),
-                                            ("prefill_8k", 1500, 320, 73)])
+                                            ("prefill_8k", 1500, 320, 73), ("prefill_8k", 1800, None, 74)])
 def test_prefill_kl_integer_mode(dsa, name, L, k, seed):
-    # k = 320 ends in half a 128-key tile: the objective's masks skip the padded half
+    # k = 320 ends in half a 128-key tile: the objective's masks skip the padded half.  L = 1800 <= k: every row
+    # selects all of 0..t, and the objective still needs the index scores of those keys.
     cfg = dataclasses.replace(G.PREFILL_CONFIGS[name], L=L)
     if k is not None:
         cfg = dataclasses.replace(cfg, k=k)

@@ -82,6 +82,14 @@ def test_batch_larger_than_the_sm_count_integer_mode_exact(dsa, B):
     _run_steps(dsa, cfg, 49, 2, [0, 1, 57, 111, 148, 159, B - 1], exact=True)
 
 
+@pytest.mark.parametrize("len_lo,len_hi", [(30000, 31000), (100, 1000)])
+def test_single_sequence_integer_mode_exact(dsa, len_lo, len_hi):
+    # One sequence: its key tiles are spread over every indexer CTA (most get one or two tiles, some none), one
+    # cluster selects its row, one attention cluster runs.  The short context takes the dense path (every key).
+    cfg = G.DecodeConfig("single_int", B=1, len_lo=len_lo, len_hi=len_hi, steps=2, mode="int")
+    _run_steps(dsa, cfg, 51, 2, [0], exact=True)
+
+
 def test_contexts_around_k_integer_mode_exact(dsa):
     # contexts n_b of 2044..2050 keys before the step (k = 2048): over three appended steps the tokens cross from the
     # dense path (n_b + 1 <= k: every key selected, read as contiguous tiles) to the selected path, one key at a time

@@ -90,6 +90,14 @@ def test_single_sequence_integer_mode_exact(dsa, len_lo, len_hi):
     _run_steps(dsa, cfg, 51, 2, [0], exact=True)
 
 
+@pytest.mark.parametrize("k", [128, 320, 1024])
+def test_smaller_k_integer_mode_exact(dsa, k):
+    # k below 2048 (320: a selection ending in half a 128-key tile); contexts of 100..9000 keys, so some tokens
+    # take every key and the others select k of them
+    cfg = G.DecodeConfig("small_k_int", B=5, len_lo=100, len_hi=9000, steps=2, k=k, mode="int")
+    _run_steps(dsa, cfg, 52, 2, range(5), exact=True)
+
+
 def test_contexts_around_k_integer_mode_exact(dsa):
     # contexts n_b of 2044..2050 keys before the step (k = 2048): over three appended steps the tokens cross from the
     # dense path (n_b + 1 <= k: every key selected, read as contiguous tiles) to the selected path, one key at a time

@@ -219,6 +219,15 @@ def decode_bytes(cfg, lens, steps):
 
 
 # ------------------------------------------------------------------------------------------ GPU arms
+def decode_traffic(step_bytes):
+    """DRAM bytes of one decode step: the ncu capture's bytes per algorithmic byte (append, indexer, cluster top-k
+    and attention of a 16-sequence step) times this step's algorithmic bytes; None once the kernels' source
+    differs from the captured one."""
+    t = _traffic_entry("decode_step", ("dsa_api.cu", "indexer.cuh", "topk_cluster.cuh", "sparse_mla.cuh",
+                                       "common.cuh"))
+    return None if t is None else t["dram_bytes_per_algorithmic_byte"] * step_bytes
+
+
 def select_split(dsa, x, cfg, ws, idx):
     """Per-kernel time of one step's select: its score blocks re-run one by one through dsa_indexer_scores and
     dsa_topk (the kernels and arguments dsa_prefill_select launches block after block), each launch bracketed by
@@ -677,7 +686,8 @@ def bench_decode(dsa, cfg, steps, warmup, ws_n, rank, pk):
             "warmup": warmup,
             "roofline": {"kernel": "decode step (append, indexer, top-k, sparse MLA)", "bound": "hbm",
                          "achieved": gbs, "peak": pk["hbm_gbs"], "unit": "GB/s", "frac": gbs / pk["hbm_gbs"],
-                         "traffic": None, "peak_source": pk["source"] + " copy bandwidth"},
+                         "traffic": decode_traffic(byts / steps),
+                         "peak_source": pk["source"] + " copy bandwidth"},
             "launches": launches}
 
 
@@ -712,7 +722,8 @@ def kernels_small(dsa):
     torch.cuda.synchronize()
     assert dsa.dsa_get_device_status() == 0
     print(json.dumps({"kernels_small": "ok", "attention_tokens": T, "indexer_rows": 2048, "keys": cfg.L,
-                      "decode_sequences": dcfg.B, "decode_keys": sum(n + 1 for n in cache["lens"])}))
+                      "decode_sequences": dcfg.B, "decode_keys": sum(n + 1 for n in cache["lens"]),
+                      "decode_algorithmic_bytes": decode_bytes(dcfg, cache["lens"], 1)}))
 
 
 # ------------------------------------------------------------------------------------------ oracle arm
